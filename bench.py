@@ -1,0 +1,416 @@
+#!/usr/bin/env python
+"""Benchmark of the MSA layer hot path on B200 through the libmsa C ABI; prints one JSON line.
+
+Headline step (one pass of the prefill hot path over one batch): msa_index_topk (index scoring,
+causal block max-pool, Top-k + local block) then msa_sparse_attn_fwd (exact sparse attention) on the
+N=32768, 64-query / 4-KV-head needle workload. value = query tokens per second over all ranks.
+Secondary measurements in the same line: the decode step (16 x 262144 cached tokens, us per step =
+us per generated token of each sequence) and the training KL alignment (N=65536).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Ranks run independent sequences (weak scaling, no data-path collective); timing is on the device
+with CUDA events, the max over ranks. The L2 cache is flushed (a 256 MiB write) before every
+timed step. --impl reference times the float64 CPU oracle on a bounded sample of the same rows.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from msa_inputs import WORKLOADS, prefill_inputs, decode_inputs  # noqa: E402
+
+METRIC = "MSA prefill query-tokens/s (N=32K, 64q/4kv heads); decode µs/token; % roofline"
+HEADLINE = "prefill_32k_needles"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv",
+                                       "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.p is not None:
+            self.p.terminate()
+            try:
+                self.p.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.p.kill()
+
+    def summary(self) -> dict:
+        self.f.flush()
+        self.f.seek(0)
+        rows = [ln.strip().split(", ") for ln in self.f.read().splitlines()[1:] if ln.strip()]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        num = lambda s: float(s.split()[0]) if s and s.split()[0].replace(".", "").isdigit() else None
+        sm = [num(r[1]) for r in rows if len(r) > 2 and num(r[1])]
+        mx = [num(r[2]) for r in rows if len(r) > 2 and num(r[2])]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows if len(r) >= 9 for k in range(4) if r[5 + k].startswith("Active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def selected_tokens(blocks: torch.Tensor, block_k: int) -> int:
+    """Sum over (b, i, r) of |J|: causal tokens of the selected blocks (the algorithmic work)."""
+    B, N, H_kv, K1 = blocks.shape
+    i = torch.arange(N, device=blocks.device).view(1, N, 1, 1)
+    c = blocks.long()
+    n = torch.clamp(i - c * block_k + 1, max=block_k)
+    return int(torch.where(c >= 0, n, torch.zeros_like(n)).sum().item())
+
+
+def timed_steps(fn, steps: int, flush: torch.Tensor):
+    """Per-step device times (ms) with CUDA events on the current stream; L2 flushed before each."""
+    st = torch.cuda.current_stream()
+    times = []
+    for _ in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        fn()
+        b.record(st)
+        times.append((a, b))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in times]
+
+
+def roofline_entry(bound, achieved, peak, unit, traffic=None):
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": (achieved / peak) if (achieved is not None and peak) else None, "traffic": traffic}
+
+
+def profile_avg(prof: dict) -> dict:
+    return {k: {"avg_ms": v[0] / max(v[1], 1), "launches": v[1], "total_ms": v[0]} for k, v in prof.items()}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                             device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ============================================================================ reference arm
+def run_reference(args, world, rank):
+    """The float64 CPU oracle on a bounded row sample of the headline workload per step."""
+    if rank != 0:
+        return None
+    import numpy as np
+    import oracle
+    w = WORKLOADS[HEADLINE]
+    x = prefill_inputs(w, device="cpu")
+    od = oracle.Dims(w.B, w.N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
+    rows_per_step = args.ref_rows
+    rng = np.random.default_rng(0)
+    full_blocks = np.full((w.B, w.N, w.H_kv, w.topk + 1), -1, dtype=np.int32)
+
+    def step():
+        rows = np.sort(rng.choice(w.N, size=rows_per_step, replace=False))
+        b, _, _ = oracle.index_topk(od, x["q_idx"], x["k_idx"], rows=rows)
+        full_blocks[0, rows] = b
+        oracle.sparse_attn(od, x["q"], x["k"], x["v"], full_blocks, rows=rows)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = rows_per_step * args.steps / dt
+    sample = f"{rows_per_step} uniformly drawn query rows of {HEADLINE} per step (index Top-k + sparse attention)"
+    return {"metric": METRIC, "value": value, "unit": "query-tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps * (w.N / rows_per_step),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": HEADLINE, "N": w.N, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d, "d_idx": w.d_idx,
+                       "block_k": w.block_k, "topk": w.topk},
+            "cpu_baseline": {"value": value, "unit": "query-tokens/s", "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "query-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ============================================================================ our arm
+def cpu_baseline(x, w, rows_n: int):
+    """The oracle as it stands on a bounded row sample of the same workload (rank 0, N=1)."""
+    import numpy as np
+    import oracle
+    od = oracle.Dims(w.B, w.N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
+    xc = {k: x[k].cpu() for k in ("q", "k", "v", "q_idx", "k_idx")}
+    rows = np.sort(np.random.default_rng(1).choice(w.N, size=rows_n, replace=False))
+    full = np.full((w.B, w.N, w.H_kv, w.topk + 1), -1, dtype=np.int32)
+    t0 = time.perf_counter()
+    b, _, _ = oracle.index_topk(od, xc["q_idx"], xc["k_idx"], rows=rows)
+    full[0, rows] = b
+    oracle.sparse_attn(od, xc["q"], xc["k"], xc["v"], full, rows=rows)
+    dt = time.perf_counter() - t0
+    return {"value": rows_n / dt, "unit": "query-tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{rows_n} uniformly drawn query rows of {HEADLINE} (index Top-k + sparse attention), "
+                      f"{dt:.1f} s"}
+
+
+def bench_prefill(args, world, rank, msa, pk):
+    w = WORKLOADS[HEADLINE]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    x = prefill_inputs(w, device=dev, seed=1000 + w.cid + 7919 * rank)
+    dims = msa.MsaDims(w.B, w.N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
+    ws_i = msa.workspace(msa.MSA_OP_INDEX_TOPK, dims, dev)
+    ws_a = msa.workspace(msa.MSA_OP_ATTN_FWD, dims, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        blocks = msa.msa_index_topk(dims, x["q_idx"], x["k_idx"], ws=ws_i)
+        return blocks, msa.msa_sparse_attn_fwd(dims, x["q"], x["k"], x["v"], blocks, ws=ws_a)
+
+    for _ in range(args.warmup):
+        blocks, _ = step()
+    torch.cuda.synchronize()
+    sel_tok = selected_tokens(blocks, w.block_k)  # sum_{i,r} |J|
+    G = w.H_q // w.H_kv
+    attn_flops = 4.0 * w.d * G * sel_tok
+    index_flops = 2.0 * w.d_idx * w.H_kv * w.N * (w.N + 1) / 2
+    msa.msa_profile_read()
+    barrier(world)
+    msa.msa_profile_enable(True)
+    with ClockSampler(dev.index) as cs:
+        t = timed_steps(step, args.steps, flush)
+    msa.msa_profile_enable(False)
+    prof = profile_avg(msa.msa_profile_read())
+    barrier(world)
+    step_ms = max_over_ranks(sum(t) / len(t), world)
+    value = w.N * w.B * world / (step_ms * 1e-3)
+    # roofline of the dominant kernel (live CUDA-event durations of its launches)
+    dom = max(prof, key=lambda k: prof[k]["total_ms"])
+    per_kernel = {}
+    for k, v in prof.items():
+        fl = attn_flops if k == "attn_kv_outer" else index_flops if k == "index_topk" else None
+        tf = fl / (v["avg_ms"] * 1e-3) / 1e12 if fl else None
+        per_kernel[k] = {"avg_ms": round(v["avg_ms"], 4), "launches": v["launches"],
+                         "share": round(v["total_ms"] / sum(u["total_ms"] for u in prof.values()), 4),
+                         **({"tflops": round(tf, 1), "frac_of_measured_bf16": round(tf / pk["bf16_tflops"], 4)}
+                            if tf else {})}
+    dfl = attn_flops if dom == "attn_kv_outer" else index_flops if dom == "index_topk" else None
+    roof = roofline_entry("tensor", dfl / (prof[dom]["avg_ms"] * 1e-3) / 1e12 if dfl else None,
+                          pk["bf16_tflops"], "TFLOP/s", None)
+    roof["kernel"] = dom
+    roof["flops_per_launch"] = dfl
+    roof["peak_source"] = f"{pk['source']} bf16 burst"
+    # e2e through the public API with pinned host buffers (H2D inputs, D2H output inside the region)
+    host = {k: x[k].cpu().pin_memory() for k in ("q", "k", "v", "q_idx", "k_idx")}
+    out_host = torch.empty(x["q"].shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        for k in host:
+            x[k].copy_(host[k], non_blocking=True)
+        _, (out, _) = step()
+        out_host.copy_(out, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 5))
+    for _ in range(2):
+        e2e_step()
+    barrier(world)
+    te = timed_steps(e2e_step, e2e_steps, flush)
+    e2e_ms = max_over_ranks(sum(te) / len(te), world)
+    res = {"value": value, "ms_per_step": step_ms, "roofline": roof, "kernels": per_kernel, "clocks": cs.summary(),
+           "e2e": {"value": w.N * w.B * world / (e2e_ms * 1e-3), "unit": "query-tokens/s",
+                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+           "gpu_launches": 7 * args.steps,
+           "work": {"selected_tokens": sel_tok, "mean_J": sel_tok / (w.N * w.H_kv), "attn_flops": attn_flops,
+                    "index_flops": index_flops}}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(x, w, args.cpu_rows)
+    del ws_a, x
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_decode(args, world, rank, msa, pk):
+    w = WORKLOADS["decode_16x256k"]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    x = decode_inputs(w, device=dev, seed=1000 + w.cid + 7919 * rank)
+    dims = msa.MsaDims(w.B, w.N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
+    ws = msa.workspace(msa.MSA_OP_DECODE, dims, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        return msa.msa_sparse_attn_decode(dims, x["cache_len"], x["q"], x["q_idx"], x["k_cache"], x["v_cache"],
+                                          x["k_idx_cache"], ws=ws)
+
+    for _ in range(max(3, args.warmup)):
+        out, blocks = step()
+    torch.cuda.synchronize()
+    L = w.N
+    nscored = ((L - 1) // w.block_k) * w.block_k
+    scan_bytes = w.B * nscored * w.d_idx * 2
+    sel_blocks = int((blocks >= 0).sum().item())
+    kv_bytes = sel_blocks * w.block_k * w.d * 2 * 2
+    step_bytes = scan_bytes + kv_bytes + w.B * (w.H_q * w.d * 2 * 2 + w.H_kv * w.d_idx * 2)
+    msa.msa_profile_read()
+    msa.msa_profile_enable(True)
+    t = timed_steps(step, args.decode_steps, flush)
+    msa.msa_profile_enable(False)
+    prof = profile_avg(msa.msa_profile_read())
+    us = max_over_ranks(1e3 * sum(t) / len(t), world)
+    scan_ms = prof["dec_scan"]["avg_ms"]
+    res = {"workload": "decode_16x256k", "us_per_step": us, "us_per_token": us, "tokens_per_s": w.B * world / (us * 1e-6),
+           "bytes_per_step": step_bytes,
+           "step_roofline": roofline_entry("hbm", step_bytes / (us * 1e-6) / 1e9, pk["hbm_gbs"], "GB/s"),
+           "roofline": {**roofline_entry("hbm", scan_bytes / (scan_ms * 1e-3) / 1e9, pk["hbm_gbs"], "GB/s"),
+                        "kernel": "dec_scan", "bytes_per_launch": scan_bytes},
+           "kernels": {k: {"avg_ms": round(v["avg_ms"], 4), "launches": v["launches"]} for k, v in prof.items()}}
+    del x, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_train(args, world, rank, msa, pk):
+    w = WORKLOADS["train_64k"]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    x = prefill_inputs(w, device=dev, seed=1000 + w.cid + 7919 * rank)
+    dims = msa.MsaDims(w.B, w.N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
+    ws_i = msa.workspace(msa.MSA_OP_INDEX_TOPK_LSE, dims, dev)
+    ws_a = msa.workspace(msa.MSA_OP_ATTN_FWD, dims, dev)
+    ws_k = msa.workspace(msa.MSA_OP_KL, dims, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        blocks, lse_idx = msa.msa_index_topk(dims, x["q_idx"], x["k_idx"], want_lse=True, ws=ws_i)
+        out, lse = msa.msa_sparse_attn_fwd(dims, x["q"], x["k"], x["v"], blocks, ws=ws_a)
+        loss, dq, dk = msa.msa_kl_fwd_grad(dims, x["q"], x["k"], x["q_idx"], x["k_idx"], blocks, lse, lse_idx,
+                                           ws=ws_k)
+        return blocks, loss
+
+    for _ in range(2):
+        blocks, loss = step()
+    torch.cuda.synchronize()
+    sel_tok = selected_tokens(blocks, w.block_k)
+    G = w.H_q // w.H_kv
+    kl_flops = (2.0 * w.d * G + 6.0 * w.d_idx) * sel_tok
+    msa.msa_profile_read()
+    msa.msa_profile_enable(True)
+    t = timed_steps(step, args.train_steps, flush)
+    msa.msa_profile_enable(False)
+    prof = profile_avg(msa.msa_profile_read())
+    ms = max_over_ranks(sum(t) / len(t), world)
+    kl_ms = prof["kl_kv_outer"]["avg_ms"]
+    res = {"workload": "train_64k", "ms_per_step": ms, "loss": float(loss.item()),
+           "roofline": {**roofline_entry("tensor", kl_flops / (kl_ms * 1e-3) / 1e12, pk["bf16_tflops"], "TFLOP/s"),
+                        "kernel": "kl_kv_outer", "flops_per_launch": kl_flops},
+           "kernels": {k: {"avg_ms": round(v["avg_ms"], 4), "launches": v["launches"]} for k, v in prof.items()}}
+    del x, ws_a, ws_k
+    torch.cuda.empty_cache()
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--decode-steps", type=int, default=30)
+    ap.add_argument("--train-steps", type=int, default=3)
+    ap.add_argument("--cpu-rows", type=int, default=384)
+    ap.add_argument("--ref-rows", type=int, default=48)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        world, rank = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0"))
+        line = run_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    world, rank, local = dist_setup(args.gpus)
+    import block_sparse_attention_idx_b200 as msa
+    pk = peaks()
+    pre = bench_prefill(args, world, rank, msa, pk)
+    w = WORKLOADS[HEADLINE]
+    line = {"metric": METRIC, "value": pre["value"], "unit": "query-tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": pre["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": HEADLINE, "N": w.N, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d, "d_idx": w.d_idx,
+                       "block_k": w.block_k, "topk": w.topk, "batch_per_gpu": w.B, "global_batch": w.B * world,
+                       "parallelism": f"dp{world} (independent sequences)",
+                       "l2": "flushed (256 MiB write) before every timed step",
+                       "step": "msa_index_topk + msa_sparse_attn_fwd"},
+            "roofline": pre["roofline"], "e2e": pre["e2e"], "gpu_launches": pre["gpu_launches"],
+            "clocks": pre["clocks"], "kernels": pre["kernels"], "work": pre["work"],
+            "peaks": pk}
+    if "cpu_baseline" in pre:
+        line["cpu_baseline"] = pre["cpu_baseline"]
+    if not args.no_secondary:
+        line["decode"] = bench_decode(args, world, rank, msa, pk)
+        line["train"] = bench_train(args, world, rank, msa, pk)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,234 @@
+"""Python binding of libmsa, the B200 (sm_100a) MiniMax Sparse Attention hot path.
+
+Thin ctypes marshalling over the C ABI in include/msa.h: every function here only checks shapes,
+allocates outputs / workspace through PyTorch and calls the same-named C entry point on the
+current CUDA stream. All arithmetic runs in the library's CUDA kernels; there is no other path.
+Importing works without a GPU (the library loads without one); calling needs a CUDA device.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmsa.so")
+
+MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_WORKSPACE, MSA_ERR_CUDA, MSA_ERR_TIMEOUT, \
+    MSA_ERR_DEVICE_CHECK = range(7)
+MSA_OP_INDEX_TOPK, MSA_OP_INDEX_TOPK_LSE, MSA_OP_ATTN_FWD, MSA_OP_DECODE, MSA_OP_KL = range(5)
+
+
+class MsaError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {msa_status_string(code)} ({code})")
+        self.code = code
+
+
+class _Dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("N", ctypes.c_int), ("H_q", ctypes.c_int), ("H_kv", ctypes.c_int),
+                ("d", ctypes.c_int), ("d_idx", ctypes.c_int), ("block_k", ctypes.c_int), ("topk", ctypes.c_int),
+                ("scale", ctypes.c_float), ("scale_idx", ctypes.c_float)]
+
+
+@dataclass
+class MsaDims:
+    """msa_dims: B sequences of N tokens (cache capacity for decode), H_q / H_kv heads, head dim d,
+    index dim d_idx, KV block size block_k, topk past blocks per (query, group).
+    scale / scale_idx of 0 mean 1/sqrt(d) and 1/sqrt(d_idx)."""
+    B: int
+    N: int
+    H_q: int
+    H_kv: int
+    d: int
+    d_idx: int
+    block_k: int
+    topk: int
+    scale: float = 0.0
+    scale_idx: float = 0.0
+
+    def c(self) -> _Dims:
+        return _Dims(self.B, self.N, self.H_q, self.H_kv, self.d, self.d_idx, self.block_k, self.topk,
+                     self.scale, self.scale_idx)
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libmsa.so; raises if it has not been built (there is no fallback path)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libmsa.so not found at {LIB_PATH}; build it with "
+                               "`python -m block_sparse_attention_idx_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, D, S = ctypes.c_void_p, ctypes.POINTER(_Dims), ctypes.c_size_t
+        L.msa_workspace_size.argtypes = [ctypes.c_int, D, ctypes.POINTER(ctypes.c_size_t)]
+        L.msa_index_topk.argtypes = [D, P, P, P, P, P, S, P]
+        L.msa_sparse_attn_fwd.argtypes = [D, P, P, P, P, P, P, P, S, P]
+        L.msa_sparse_attn_decode.argtypes = [D, P, P, P, P, P, P, P, P, P, S, P]
+        L.msa_kl_fwd_grad.argtypes = [D, P, P, P, P, P, P, P, ctypes.c_float, P, P, P, P, S, P]
+        L.msa_get_device_status.argtypes = [P, P]
+        L.msa_profile_enable.argtypes = [ctypes.c_int]
+        L.msa_profile_enable.restype = None
+        L.msa_profile_read.argtypes = [ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
+                                       ctypes.POINTER(ctypes.c_int), ctypes.c_int]
+        L.msa_profile_read.restype = ctypes.c_int
+        L.msa_status_string.argtypes = [ctypes.c_int]
+        L.msa_status_string.restype = ctypes.c_char_p
+        L.msa_version.restype = ctypes.c_char_p
+        for fn in ("msa_workspace_size", "msa_index_topk", "msa_sparse_attn_fwd", "msa_sparse_attn_decode",
+                   "msa_kl_fwd_grad", "msa_get_device_status"):
+            getattr(L, fn).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def msa_status_string(code: int) -> str:
+    return lib().msa_status_string(code).decode()
+
+
+def msa_version() -> str:
+    return lib().msa_version().decode()
+
+
+def _check(fn: str, code: int):
+    if code != MSA_OK:
+        raise MsaError(fn, code)
+
+
+def msa_workspace_size(op: int, dims: MsaDims) -> int:
+    n = ctypes.c_size_t(0)
+    _check("msa_workspace_size", lib().msa_workspace_size(op, ctypes.byref(dims.c()), ctypes.byref(n)))
+    return n.value
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, shape, dtype, device):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}")
+
+
+def workspace(op: int, dims: MsaDims, device) -> torch.Tensor:
+    """A device workspace buffer of the size `op` needs (256-byte aligned by the allocator)."""
+    return torch.empty(max(msa_workspace_size(op, dims), 256), dtype=torch.uint8, device=device)
+
+
+def msa_index_topk(dims: MsaDims, q_idx, k_idx, want_lse: bool = False, ws=None, stream=None):
+    """Block selection. Returns blocks int32 [B,N,H_kv,topk+1] (and LSE_idx fp32 [B,N,H_kv])."""
+    dev = q_idx.device
+    _need(q_idx, "q_idx", (dims.B, dims.N, dims.H_kv, dims.d_idx), torch.bfloat16, dev)
+    _need(k_idx, "k_idx", (dims.B, dims.N, dims.d_idx), torch.bfloat16, dev)
+    blocks = torch.empty(dims.B, dims.N, dims.H_kv, dims.topk + 1, dtype=torch.int32, device=dev)
+    lse = torch.empty(dims.B, dims.N, dims.H_kv, dtype=torch.float32, device=dev) if want_lse else None
+    if ws is None:
+        ws = workspace(MSA_OP_INDEX_TOPK_LSE if want_lse else MSA_OP_INDEX_TOPK, dims, dev)
+    _check("msa_index_topk", lib().msa_index_topk(ctypes.byref(dims.c()), _p(q_idx), _p(k_idx), _p(blocks), _p(lse),
+                                                  _p(ws), ws.numel(), _stream(stream)))
+    return (blocks, lse) if want_lse else blocks
+
+
+def msa_sparse_attn_fwd(dims: MsaDims, q, k, v, blocks, want_lse: bool = True, ws=None, stream=None):
+    """Sparse attention forward. Returns out bf16 [B,N,H_q,d] and LSE fp32 [B,N,H_q] (or None)."""
+    dev = q.device
+    _need(q, "q", (dims.B, dims.N, dims.H_q, dims.d), torch.bfloat16, dev)
+    _need(k, "k", (dims.B, dims.N, dims.H_kv, dims.d), torch.bfloat16, dev)
+    _need(v, "v", (dims.B, dims.N, dims.H_kv, dims.d), torch.bfloat16, dev)
+    _need(blocks, "blocks", (dims.B, dims.N, dims.H_kv, dims.topk + 1), torch.int32, dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(dims.B, dims.N, dims.H_q, dtype=torch.float32, device=dev) if want_lse else None
+    if ws is None:
+        ws = workspace(MSA_OP_ATTN_FWD, dims, dev)
+    _check("msa_sparse_attn_fwd", lib().msa_sparse_attn_fwd(ctypes.byref(dims.c()), _p(q), _p(k), _p(v), _p(blocks),
+                                                            _p(out), _p(lse), _p(ws), ws.numel(), _stream(stream)))
+    return out, lse
+
+
+def msa_sparse_attn_decode(dims: MsaDims, cache_len, q, q_idx, k_cache, v_cache, k_idx_cache, want_blocks=True,
+                           ws=None, stream=None):
+    """One decode step. dims.N is the cache capacity. Returns out bf16 [B,H_q,d] and the selected
+    blocks int32 [B,H_kv,topk+1] (or None)."""
+    dev = q.device
+    _need(cache_len, "cache_len", (dims.B,), torch.int32, dev)
+    _need(q, "q", (dims.B, dims.H_q, dims.d), torch.bfloat16, dev)
+    _need(q_idx, "q_idx", (dims.B, dims.H_kv, dims.d_idx), torch.bfloat16, dev)
+    _need(k_cache, "k_cache", (dims.B, dims.N, dims.H_kv, dims.d), torch.bfloat16, dev)
+    _need(v_cache, "v_cache", (dims.B, dims.N, dims.H_kv, dims.d), torch.bfloat16, dev)
+    _need(k_idx_cache, "k_idx_cache", (dims.B, dims.N, dims.d_idx), torch.bfloat16, dev)
+    out = torch.empty_like(q)
+    blocks = torch.empty(dims.B, dims.H_kv, dims.topk + 1, dtype=torch.int32, device=dev) if want_blocks else None
+    if ws is None:
+        ws = workspace(MSA_OP_DECODE, dims, dev)
+    _check("msa_sparse_attn_decode",
+           lib().msa_sparse_attn_decode(ctypes.byref(dims.c()), _p(cache_len), _p(q), _p(q_idx), _p(k_cache),
+                                        _p(v_cache), _p(k_idx_cache), _p(out), _p(blocks), _p(ws), ws.numel(),
+                                        _stream(stream)))
+    return out, blocks
+
+
+def msa_kl_fwd_grad(dims: MsaDims, q, k, q_idx, k_idx, blocks, lse, lse_idx=None, grad_scale: float = 1.0, ws=None,
+                    stream=None):
+    """KL alignment. Returns loss fp32 [1], dq_idx fp32 [B,N,H_kv,d_idx], dk_idx fp32 [B,N,d_idx]."""
+    dev = q.device
+    _need(q, "q", (dims.B, dims.N, dims.H_q, dims.d), torch.bfloat16, dev)
+    _need(k, "k", (dims.B, dims.N, dims.H_kv, dims.d), torch.bfloat16, dev)
+    _need(q_idx, "q_idx", (dims.B, dims.N, dims.H_kv, dims.d_idx), torch.bfloat16, dev)
+    _need(k_idx, "k_idx", (dims.B, dims.N, dims.d_idx), torch.bfloat16, dev)
+    _need(blocks, "blocks", (dims.B, dims.N, dims.H_kv, dims.topk + 1), torch.int32, dev)
+    _need(lse, "lse", (dims.B, dims.N, dims.H_q), torch.float32, dev)
+    if lse_idx is not None:
+        _need(lse_idx, "lse_idx", (dims.B, dims.N, dims.H_kv), torch.float32, dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    dq = torch.empty(dims.B, dims.N, dims.H_kv, dims.d_idx, dtype=torch.float32, device=dev)
+    dk = torch.empty(dims.B, dims.N, dims.d_idx, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = workspace(MSA_OP_KL, dims, dev)
+    _check("msa_kl_fwd_grad",
+           lib().msa_kl_fwd_grad(ctypes.byref(dims.c()), _p(q), _p(k), _p(q_idx), _p(k_idx), _p(blocks), _p(lse),
+                                 _p(lse_idx), ctypes.c_float(grad_scale), _p(loss), _p(dq), _p(dk), _p(ws),
+                                 ws.numel(), _stream(stream)))
+    return loss, dq, dk
+
+
+def msa_profile_enable(on: bool = True) -> None:
+    """Record CUDA events around every kernel the library launches (on the launching stream)."""
+    lib().msa_profile_enable(1 if on else 0)
+
+
+def msa_profile_read() -> dict:
+    """{kernel name: (total ms, launches)} since the last read; synchronises on the events."""
+    cap = 64
+    names = (ctypes.c_char_p * cap)()
+    ms = (ctypes.c_double * cap)()
+    n = (ctypes.c_int * cap)()
+    k = lib().msa_profile_read(names, ms, n, cap)
+    if k < 0:
+        raise MsaError("msa_profile_read", MSA_ERR_CUDA)
+    return {names[x].decode(): (ms[x], n[x]) for x in range(k)}
+
+
+def msa_get_device_status(ws: torch.Tensor, stream=None) -> int:
+    """Synchronise the stream and return the status code recorded by the last call using `ws`."""
+    return lib().msa_get_device_status(_p(ws), _stream(stream))
+
+
+__all__ = ["MsaDims", "MsaError", "msa_workspace_size", "msa_index_topk", "msa_sparse_attn_fwd",
+           "msa_sparse_attn_decode", "msa_kl_fwd_grad", "msa_get_device_status", "msa_status_string",
+           "msa_version", "msa_profile_enable", "msa_profile_read", "workspace", "lib", "LIB_PATH"]

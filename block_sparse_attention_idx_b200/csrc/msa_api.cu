@@ -1,0 +1,287 @@
+// C ABI of libmsa (declared in include/msa.h): argument checks, workspace layout and dispatch.
+// Nothing here allocates, frees or synchronises device memory; every call enqueues on `stream`.
+#include <math.h>
+#include <string.h>
+
+#include "msa.h"
+#include "msa_common.cuh"
+#include "msa_internal.h"
+
+using namespace msa;
+
+namespace {
+
+constexpr size_t kStatusBytes = 256;
+
+size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_sms() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+// Sizes shared by every entry point.
+msa_status check_common(const msa_dims* d) {
+    if (!d) return MSA_ERR_INVALID_ARG;
+    if (d->B < 1 || d->N < 1 || d->H_q < 1 || d->H_kv < 1 || d->topk < 1) return MSA_ERR_INVALID_ARG;
+    if (d->H_q % d->H_kv != 0) return MSA_ERR_INVALID_ARG;
+    if (!(d->scale >= 0.f) || !(d->scale_idx >= 0.f)) return MSA_ERR_INVALID_ARG;
+    const int G = d->H_q / d->H_kv;
+    if (128 % G != 0 || 128 % d->H_kv != 0 || d->H_kv > 8) return MSA_ERR_UNSUPPORTED;
+    if (d->d != 64 && d->d != 128) return MSA_ERR_UNSUPPORTED;
+    if (d->d_idx != 32 && d->d_idx != 64) return MSA_ERR_UNSUPPORTED;
+    if (d->block_k != 32 && d->block_k != 64 && d->block_k != 128) return MSA_ERR_UNSUPPORTED;
+    if (d->topk > 16) return MSA_ERR_UNSUPPORTED;
+    if (d->N >= (1 << 24)) return MSA_ERR_UNSUPPORTED;
+    const double entries = (double)d->B * d->N * d->H_kv * (d->topk + 1);
+    if (entries >= 2147483647.0 / 2) return MSA_ERR_UNSUPPORTED;
+    return MSA_OK;
+}
+
+float eff_scale(float s, int dim) { return s > 0.f ? s : 1.0f / sqrtf((float)dim); }
+
+size_t csr_need(const msa_dims* d) { return csr_bytes(d->B, d->N, d->H_kv, d->block_k, d->topk); }
+
+size_t rows_kv(const msa_dims* d) { return (size_t)d->B * d->N * d->H_kv; }
+
+size_t ws_index_lse(const msa_dims* d) {
+    return kStatusBytes + csr_need(d) + al256(rows_kv(d) * (d->topk + 1) * sizeof(float2));
+}
+size_t ws_attn(const msa_dims* d) {
+    const size_t pr = (size_t)d->B * d->N * d->H_q * (d->topk + 1);
+    return kStatusBytes + csr_need(d) + al256(pr * d->d * sizeof(float)) + al256(pr * sizeof(float));
+}
+size_t ws_decode(const msa_dims* d) {
+    return kStatusBytes + decode_ws_bytes(d->B, d->N, d->H_q, d->H_kv, d->d, d->block_k, d->topk);
+}
+size_t ws_kl(const msa_dims* d) {
+    const size_t nb = (size_t)(d->N + d->block_k - 1) / d->block_k;
+    const size_t nl = (size_t)d->B * d->H_kv * nb;
+    const size_t me = rows_kv(d) * (d->topk + 1);
+    const size_t csr_idx_extra = al256((nl + 1) * 4) + al256(me * 8) + 256;
+    return kStatusBytes + csr_need(d) + csr_idx_extra + al256(me * sizeof(float2)) + al256(rows_kv(d) * 4) +
+           al256(me * d->d_idx * 4) + al256(me * 8) + al256(rows_kv(d) * 8);
+}
+
+msa_status ws_check(const void* ws, size_t have, size_t need) {
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MSA_ERR_WORKSPACE;
+    if (have < need) return MSA_ERR_WORKSPACE;
+    return MSA_OK;
+}
+
+msa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
+
+struct Carver {
+    uint8_t* p;
+    uint8_t* take(size_t bytes) {
+        uint8_t* r = p;
+        p += al256(bytes);
+        return r;
+    }
+};
+
+}  // namespace
+
+extern "C" {
+
+const char* msa_version(void) { return "msa-b200 0.1.0"; }
+
+const char* msa_status_string(msa_status s) {
+    switch (s) {
+        case MSA_OK: return "MSA_OK";
+        case MSA_ERR_INVALID_ARG: return "MSA_ERR_INVALID_ARG";
+        case MSA_ERR_UNSUPPORTED: return "MSA_ERR_UNSUPPORTED";
+        case MSA_ERR_WORKSPACE: return "MSA_ERR_WORKSPACE";
+        case MSA_ERR_CUDA: return "MSA_ERR_CUDA";
+        case MSA_ERR_TIMEOUT: return "MSA_ERR_TIMEOUT";
+        case MSA_ERR_DEVICE_CHECK: return "MSA_ERR_DEVICE_CHECK";
+    }
+    return "MSA_ERR_UNKNOWN";
+}
+
+msa_status msa_workspace_size(int op, const msa_dims* d, size_t* bytes) {
+    if (!bytes) return MSA_ERR_INVALID_ARG;
+    msa_status s = check_common(d);
+    if (s != MSA_OK) return s;
+    switch (op) {
+        case MSA_OP_INDEX_TOPK: *bytes = kStatusBytes; return MSA_OK;
+        case MSA_OP_INDEX_TOPK_LSE: *bytes = ws_index_lse(d); return MSA_OK;
+        case MSA_OP_ATTN_FWD: *bytes = ws_attn(d); return MSA_OK;
+        case MSA_OP_DECODE: *bytes = ws_decode(d); return MSA_OK;
+        case MSA_OP_KL: *bytes = ws_kl(d); return MSA_OK;
+    }
+    return MSA_ERR_INVALID_ARG;
+}
+
+msa_status msa_index_topk(const msa_dims* d, const void* q_idx, const void* k_idx, int32_t* blocks, float* lse_idx,
+                          void* ws, size_t ws_bytes, msa_stream_t stream_) {
+    msa_status s = check_common(d);
+    if (s != MSA_OK) return s;
+    if (!q_idx || !k_idx || !blocks || !aligned16(q_idx) || !aligned16(k_idx) || !aligned16(blocks) ||
+        (lse_idx && !aligned16(lse_idx)))
+        return MSA_ERR_INVALID_ARG;
+    s = ws_check(ws, ws_bytes, lse_idx ? ws_index_lse(d) : kStatusBytes);
+    if (s != MSA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_);
+    DevStatus* status = static_cast<DevStatus*>(ws);
+    cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, st);
+    if (e != cudaSuccess) return MSA_ERR_CUDA;
+    IndexArgs a{d->B, d->N, d->H_kv, d->d_idx, d->block_k, d->topk, blocks, status};
+    e = run_index_topk(a, q_idx, k_idx, st);
+    if (e != cudaSuccess || !lse_idx) return cuda_status(e);
+    // LSE_idx over the selected token sets: per-(query, selected block) sum-exps, merged
+    Carver cv{static_cast<uint8_t*>(ws) + kStatusBytes};
+    KlArgs k{};
+    k.B = d->B; k.N = d->N; k.H_q = d->H_q; k.H_kv = d->H_kv; k.d = d->d; k.d_idx = d->d_idx;
+    k.block_k = d->block_k; k.topk = d->topk;
+    k.scale = eff_scale(d->scale, d->d); k.scale_idx = eff_scale(d->scale_idx, d->d_idx);
+    csr_carve(&k.csr_idx, cv.take(csr_need(d)), d->B, d->N, d->H_kv, d->block_k, d->topk);
+    k.ml_part = reinterpret_cast<float2*>(cv.take(rows_kv(d) * (d->topk + 1) * sizeof(float2)));
+    k.lse_idx = lse_idx;
+    k.blocks = blocks;
+    k.status = status;
+    e = run_csr_build(k.csr_idx, blocks, d->B, d->N, d->H_kv, d->block_k, d->topk, kIdxQpc, status, st);
+    if (e == cudaSuccess) e = run_lse_idx(k, q_idx, k_idx, num_sms(), st);
+    return cuda_status(e);
+}
+
+msa_status msa_sparse_attn_fwd(const msa_dims* d, const void* q, const void* k, const void* v, const int32_t* blocks,
+                               void* out, float* lse, void* ws, size_t ws_bytes, msa_stream_t stream_) {
+    msa_status s = check_common(d);
+    if (s != MSA_OK) return s;
+    if (!q || !k || !v || !blocks || !out || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(blocks) ||
+        !aligned16(out) || (lse && !aligned16(lse)))
+        return MSA_ERR_INVALID_ARG;
+    s = ws_check(ws, ws_bytes, ws_attn(d));
+    if (s != MSA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_);
+    DevStatus* status = static_cast<DevStatus*>(ws);
+    cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, st);
+    if (e != cudaSuccess) return MSA_ERR_CUDA;
+    Carver cv{static_cast<uint8_t*>(ws) + kStatusBytes};
+    AttnArgs a{};
+    a.B = d->B; a.N = d->N; a.H_q = d->H_q; a.H_kv = d->H_kv; a.d = d->d; a.block_k = d->block_k;
+    a.topk = d->topk; a.scale = eff_scale(d->scale, d->d);
+    csr_carve(&a.csr, cv.take(csr_need(d)), d->B, d->N, d->H_kv, d->block_k, d->topk);
+    const size_t pr = (size_t)d->B * d->N * d->H_q * (d->topk + 1);
+    a.o_part = reinterpret_cast<float*>(cv.take(pr * d->d * sizeof(float)));
+    a.lse_part = reinterpret_cast<float*>(cv.take(pr * sizeof(float)));
+    a.status = status;
+    const int G = d->H_q / d->H_kv;
+    e = run_csr_build(a.csr, blocks, d->B, d->N, d->H_kv, d->block_k, d->topk, 128 / G, status, st);
+    if (e == cudaSuccess) e = run_attn_kv_outer(a, q, k, v, num_sms(), st);
+    if (e == cudaSuccess) e = run_attn_merge(a, blocks, out, lse, st);
+    return cuda_status(e);
+}
+
+msa_status msa_sparse_attn_decode(const msa_dims* d, const int32_t* cache_len, const void* q, const void* q_idx,
+                                  const void* k_cache, const void* v_cache, const void* k_idx_cache, void* out,
+                                  int32_t* blocks_out, void* ws, size_t ws_bytes, msa_stream_t stream_) {
+    msa_status s = check_common(d);
+    if (s != MSA_OK) return s;
+    if ((d->N + d->block_k - 1) / d->block_k > 8192) return MSA_ERR_UNSUPPORTED;
+    if (!cache_len || !q || !q_idx || !k_cache || !v_cache || !k_idx_cache || !out || !aligned16(q) ||
+        !aligned16(q_idx) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_idx_cache) ||
+        !aligned16(out) || (blocks_out && !aligned16(blocks_out)))
+        return MSA_ERR_INVALID_ARG;
+    s = ws_check(ws, ws_bytes, ws_decode(d));
+    if (s != MSA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_);
+    DevStatus* status = static_cast<DevStatus*>(ws);
+    cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, st);
+    if (e != cudaSuccess) return MSA_ERR_CUDA;
+    Carver cv{static_cast<uint8_t*>(ws) + kStatusBytes};
+    const size_t nb = (size_t)(d->N + d->block_k - 1) / d->block_k;
+    const size_t G = (size_t)d->H_q / d->H_kv, K1 = (size_t)d->topk + 1;
+    DecodeArgs a{};
+    a.B = d->B; a.L = d->N; a.H_q = d->H_q; a.H_kv = d->H_kv; a.d = d->d; a.d_idx = d->d_idx;
+    a.block_k = d->block_k; a.topk = d->topk;
+    a.scale = eff_scale(d->scale, d->d); a.scale_idx = eff_scale(d->scale_idx, d->d_idx);
+    a.cache_len = cache_len;
+    a.bmax = reinterpret_cast<float*>(cv.take((size_t)d->B * d->H_kv * nb * 4));
+    a.sel = reinterpret_cast<int32_t*>(cv.take((size_t)d->B * d->H_kv * K1 * 4));
+    a.o_part = reinterpret_cast<float*>(cv.take((size_t)d->B * d->H_kv * K1 * G * d->d * 4));
+    a.lse_part = reinterpret_cast<float*>(cv.take((size_t)d->B * d->H_kv * K1 * G * 4));
+    a.blocks_out = blocks_out;
+    a.status = status;
+    e = run_decode(a, q, q_idx, k_cache, v_cache, k_idx_cache, out, st);
+    return cuda_status(e);
+}
+
+msa_status msa_kl_fwd_grad(const msa_dims* d, const void* q, const void* k, const void* q_idx, const void* k_idx,
+                           const int32_t* blocks, const float* lse, const float* lse_idx, float grad_scale,
+                           float* loss, float* dq_idx, float* dk_idx, void* ws, size_t ws_bytes,
+                           msa_stream_t stream_) {
+    msa_status s = check_common(d);
+    if (s != MSA_OK) return s;
+    if (!kl_supported(d->d, d->d_idx, d->H_q / d->H_kv)) return MSA_ERR_UNSUPPORTED;
+    if (!q || !k || !q_idx || !k_idx || !blocks || !lse || !loss || !dq_idx || !dk_idx || !aligned16(q) ||
+        !aligned16(k) || !aligned16(q_idx) || !aligned16(k_idx) || !aligned16(blocks) || !aligned16(dq_idx) ||
+        !aligned16(dk_idx))
+        return MSA_ERR_INVALID_ARG;
+    if (!isfinite(grad_scale)) return MSA_ERR_INVALID_ARG;
+    s = ws_check(ws, ws_bytes, ws_kl(d));
+    if (s != MSA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_);
+    DevStatus* status = static_cast<DevStatus*>(ws);
+    cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, st);
+    if (e != cudaSuccess) return MSA_ERR_CUDA;
+    Carver cv{static_cast<uint8_t*>(ws) + kStatusBytes};
+    const size_t nb = (size_t)(d->N + d->block_k - 1) / d->block_k;
+    const size_t nl = (size_t)d->B * d->H_kv * nb;
+    const size_t me = rows_kv(d) * (d->topk + 1);
+    KlArgs a{};
+    a.B = d->B; a.N = d->N; a.H_q = d->H_q; a.H_kv = d->H_kv; a.d = d->d; a.d_idx = d->d_idx;
+    a.block_k = d->block_k; a.topk = d->topk;
+    a.scale = eff_scale(d->scale, d->d); a.scale_idx = eff_scale(d->scale_idx, d->d_idx);
+    a.grad_scale = grad_scale;
+    csr_carve(&a.csr, cv.take(csr_need(d)), d->B, d->N, d->H_kv, d->block_k, d->topk);
+    a.csr_idx = a.csr;  // same lists, its own chunking
+    a.csr_idx.chunk_off = reinterpret_cast<int32_t*>(cv.take((nl + 1) * 4));
+    a.csr_idx.items = reinterpret_cast<int2*>(cv.take(me * 8));
+    a.csr_idx.n_items = reinterpret_cast<int32_t*>(cv.take(256));
+    a.ml_part = reinterpret_cast<float2*>(cv.take(me * sizeof(float2)));
+    float* lse_idx_ws = reinterpret_cast<float*>(cv.take(rows_kv(d) * 4));
+    a.dq_part = reinterpret_cast<float*>(cv.take(me * d->d_idx * 4));
+    a.kl_part = reinterpret_cast<double*>(cv.take(me * 8));
+    a.kl_rows = reinterpret_cast<double*>(cv.take(rows_kv(d) * 8));
+    a.lse = lse;
+    a.dq_idx = dq_idx;
+    a.dk_idx = dk_idx;
+    a.loss = loss;
+    a.blocks = blocks;
+    a.status = status;
+    const int G = d->H_q / d->H_kv;
+    e = run_csr_build(a.csr, blocks, d->B, d->N, d->H_kv, d->block_k, d->topk, 128 / G, status, st);
+    if (e == cudaSuccess && !lse_idx) {
+        a.lse_idx = lse_idx_ws;
+        e = run_csr_items(a.csr_idx, kIdxQpc, st);
+        if (e == cudaSuccess) e = run_lse_idx(a, q_idx, k_idx, num_sms(), st);
+    } else {
+        a.lse_idx = const_cast<float*>(lse_idx);
+    }
+    if (e == cudaSuccess) e = run_kl(a, q, k, q_idx, k_idx, num_sms(), st);
+    return cuda_status(e);
+}
+
+msa_status msa_get_device_status(const void* ws, msa_stream_t stream_) {
+    if (!ws) return MSA_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return MSA_ERR_CUDA;
+    DevStatus h;
+    if (cudaMemcpy(&h, ws, sizeof(unsigned int) * 2, cudaMemcpyDeviceToHost) != cudaSuccess) return MSA_ERR_CUDA;
+    if (h.flags & MSA_DEV_TIMEOUT) return MSA_ERR_TIMEOUT;
+    if (h.flags & MSA_DEV_BAD_BLOCK) return MSA_ERR_DEVICE_CHECK;
+    return MSA_OK;
+}
+
+}  // extern "C"

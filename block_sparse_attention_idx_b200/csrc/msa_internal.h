@@ -1,0 +1,114 @@
+// Internal declarations shared by the libmsa translation units (not part of the C ABI).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+namespace msa {
+
+struct DevStatus;
+
+// Opt-in kernel timing (msa_prof.cu): events around a launch on its stream; no-op when disabled.
+int prof_begin(const char* name, cudaStream_t st);
+void prof_end(int token, cudaStream_t st);
+struct ProfScope {
+    int tok;
+    cudaStream_t st;
+    ProfScope(const char* name, cudaStream_t s) : tok(prof_begin(name, s)), st(s) {}
+    ~ProfScope() { prof_end(tok, st); }
+};
+
+// ---------------------------------------------------------------- tensor maps (msa_tmap.cu)
+// bf16 tensor maps; `swizzle_bytes` is 128, 64, 32 or 0. Dimensions innermost first, strides in bytes.
+bool make_tmap_2d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t stride1, uint32_t box0,
+                  uint32_t box1, int swizzle_bytes);
+bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1,
+                  uint64_t stride2, uint32_t box0, uint32_t box1, uint32_t box2, int swizzle_bytes);
+bool make_tmap_4d(CUtensorMap* m, const void* base, const uint64_t dims[4], const uint64_t strides[3],
+                  const uint32_t box[4], int swizzle_bytes);
+
+// ---------------------------------------------------------------- index Top-k (msa_index.cu)
+struct IndexArgs {
+    int B, N, H_kv, d_idx, block_k, topk;
+    int32_t* blocks;
+    DevStatus* status;
+};
+cudaError_t run_index_topk(const IndexArgs& a, const void* q_idx, const void* k_idx, cudaStream_t st);
+
+// ---------------------------------------------------------------- inverse selection lists (msa_csr.cu)
+// For every (sequence b, group r, block c) the list of (query i, slot s) pairs whose selection
+// row blocks[b,i,r,:] holds c at position s, cut into work items of at most `qpc` queries.
+struct Csr {
+    int nlists;        // B * H_kv * nb
+    int nb;            // blocks per sequence
+    int max_entries;   // B * N * H_kv * (topk+1)
+    int32_t* counts;   // [nlists]
+    int32_t* offsets;  // [nlists + 1]
+    int32_t* cursor;   // [nlists]
+    int32_t* chunk_off;// [nlists + 1]
+    int32_t* entries;  // [max_entries]  (i << 5) | s
+    int2* items;       // [max_entries]  (list, first entry of the chunk within the list)
+    int32_t* n_items;  // [1]
+};
+size_t csr_bytes(int B, int N, int H_kv, int block_k, int topk);
+void csr_carve(Csr* c, void* base, int B, int N, int H_kv, int block_k, int topk);
+cudaError_t run_csr_build(const Csr& c, const int32_t* blocks, int B, int N, int H_kv, int block_k, int topk,
+                          int qpc, DevStatus* st, cudaStream_t stream);
+cudaError_t run_csr_items(const Csr& c, int qpc, cudaStream_t stream);
+
+// ---------------------------------------------------------------- sparse attention (msa_attn.cu)
+struct AttnArgs {
+    int B, N, H_q, H_kv, d, block_k, topk;
+    float scale;
+    Csr csr;
+    float* o_part;    // [B, N, H_q, topk+1, d]
+    float* lse_part;  // [B, N, H_q, topk+1]
+    DevStatus* status;
+};
+cudaError_t run_attn_kv_outer(const AttnArgs& a, const void* q, const void* k, const void* v, int num_sms,
+                              cudaStream_t st);
+cudaError_t run_attn_merge(const AttnArgs& a, const int32_t* blocks, void* out, float* lse, cudaStream_t st);
+
+// ---------------------------------------------------------------- KL alignment (msa_kl.cu)
+struct KlArgs {
+    int B, N, H_q, H_kv, d, d_idx, block_k, topk;
+    float scale, scale_idx, grad_scale;
+    Csr csr;            // chunks of 128/G queries
+    Csr csr_idx;        // same lists, chunks of kIdxQpc queries for the LSE_idx pass
+    const float* lse;   // [B, N, H_q]
+    float* lse_idx;     // [B, N, H_kv]
+    float2* ml_part;    // [B, N, H_kv, topk+1]  (max, sum-exp) of the index logits per slot
+    float* dq_part;     // [B, N, H_kv, topk+1, d_idx]
+    double* kl_part;    // [B, N, H_kv, topk+1]
+    double* kl_rows;    // [B, N, H_kv]
+    float* dq_idx;      // [B, N, H_kv, d_idx]
+    float* dk_idx;      // [B, N, d_idx]
+    float* loss;        // [1]
+    const int32_t* blocks;
+    DevStatus* status;
+};
+constexpr int kIdxQpc = 32;
+bool kl_supported(int d, int d_idx, int G);
+cudaError_t run_lse_idx(const KlArgs& a, const void* q_idx, const void* k_idx, int num_sms, cudaStream_t st);
+cudaError_t run_kl(const KlArgs& a, const void* q, const void* k, const void* q_idx, const void* k_idx, int num_sms,
+                   cudaStream_t st);
+
+// ---------------------------------------------------------------- decode (msa_decode.cu)
+struct DecodeArgs {
+    int B, L, H_q, H_kv, d, d_idx, block_k, topk;
+    float scale, scale_idx;
+    const int32_t* cache_len;
+    float* bmax;       // [B, H_kv, nb]
+    int32_t* sel;      // [B, H_kv, topk+1]
+    float* o_part;     // [B, H_kv, topk+1, G, d]
+    float* lse_part;   // [B, H_kv, topk+1, G]
+    int32_t* blocks_out;
+    DevStatus* status;
+};
+size_t decode_ws_bytes(int B, int L, int H_q, int H_kv, int d, int block_k, int topk);
+cudaError_t run_decode(const DecodeArgs& a, const void* q, const void* q_idx, const void* k_cache, const void* v_cache,
+                       const void* k_idx_cache, void* out, cudaStream_t st);
+
+}  // namespace msa

@@ -1,0 +1,174 @@
+/*
+ * msa.h: C ABI of libmsa, the B200 (sm_100a) implementation of the MiniMax Sparse Attention (MSA)
+ * layer hot path.
+ *
+ * The pages split a sparse layer into a candidate constructor and a main attention,
+ *   S_t = R_theta(q_t, K_{:t}),   o_t = A_phi(q_t, K_{S_t}, V_{S_t})
+ * ("2.4 · 训练原生稀疏", eq (3)). msa_index_topk is R_theta for MSA, msa_sparse_attn_fwd is A_phi,
+ * msa_kl_fwd_grad is the KL alignment of the index branch to the main branch, and
+ * msa_sparse_attn_decode runs R_theta then A_phi for one new token per sequence.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All tensor arguments are DEVICE pointers to dense, contiguous, row-major arrays, 16-byte
+ *   aligned. "bf16" means IEEE bfloat16 stored as 2 bytes.
+ * - The caller owns every buffer, the workspace and the stream. The library never allocates,
+ *   frees or synchronises (except msa_get_device_status, which synchronises the given stream).
+ *   Every call only enqueues work on `stream` and returns.
+ * - Outputs are fully overwritten.
+ * - The workspace `ws` must be at least msa_workspace_size(op, dims) bytes and 256-byte aligned.
+ *   Its contents between calls are undefined, except the device status word, which holds the
+ *   device-side error flags of the last call that used this workspace. Calls that share a
+ *   workspace must be ordered on one stream.
+ * - Host-side argument errors return a status before anything is enqueued. Device-side problems
+ *   (a wait that ran past its time limit, an out-of-range block id in `blocks`) never trap: the
+ *   kernel skips the offending work, sets a flag in the status word and returns; read it with
+ *   msa_get_device_status.
+ * - Deterministic: the same inputs give bit-identical `blocks`, attention outputs, LSEs and KL
+ *   loss. dK_idx is accumulated with float32 atomics and may differ in the last bits.
+ *
+ * Supported sizes (MSA_ERR_UNSUPPORTED otherwise): d in {64, 128}, d_idx in {32, 64},
+ * block_k in {32, 64, 128}, 1 <= topk <= 16, H_q % H_kv == 0 with G = H_q/H_kv dividing 128,
+ * H_kv dividing 128, N >= 1, B >= 1, block ids fit the workspace (N <= 2^24).
+ */
+#ifndef MSA_H
+#define MSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MSA_API __attribute__((visibility("default")))
+#else
+#define MSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream handle (cudaStream_t / CUstream); NULL is the legacy default stream. */
+typedef struct CUstream_st *msa_stream_t;
+
+typedef enum {
+    MSA_OK = 0,
+    MSA_ERR_INVALID_ARG = 1,  /* null or misaligned pointer, inconsistent sizes */
+    MSA_ERR_UNSUPPORTED = 2,  /* sizes outside the supported set above */
+    MSA_ERR_WORKSPACE = 3,    /* ws too small or not 256-byte aligned */
+    MSA_ERR_CUDA = 4,         /* a CUDA launch or driver call failed */
+    MSA_ERR_TIMEOUT = 5,      /* device status: a bounded wait ran out */
+    MSA_ERR_DEVICE_CHECK = 6  /* device status: invalid data found (e.g. a block id out of range) */
+} msa_status;
+
+/*
+ * Problem sizes. B sequences of N tokens; H_q query heads and H_kv KV heads (G = H_q/H_kv query
+ * heads per GQA group); head dim d; index dim d_idx; KV block size block_k (the pages' B_k);
+ * topk = k, the number of past blocks each (query, group) selects.
+ * scale = 0 means 1/sqrt(d); scale_idx = 0 means 1/sqrt(d_idx).
+ */
+typedef struct {
+    int B, N, H_q, H_kv, d, d_idx, block_k, topk;
+    float scale, scale_idx;
+} msa_dims;
+
+enum { MSA_OP_INDEX_TOPK = 0, MSA_OP_INDEX_TOPK_LSE = 1, MSA_OP_ATTN_FWD = 2, MSA_OP_DECODE = 3, MSA_OP_KL = 4 };
+
+/* Workspace bytes `op` needs for `dims` (for MSA_OP_DECODE, dims->N is the cache capacity). */
+MSA_API msa_status msa_workspace_size(int op, const msa_dims *dims, size_t *bytes);
+
+/*
+ * Index branch: block selection ("MSA Indexer 与 DSA Lightning Indexer 的差别", sections 2.1-2.2;
+ * MSA blog, softmax-free Top-K).
+ *   S^{idx,(r)}_{i,j} = Q^{idx,(r)}_i . K^{idx}_j * scale_idx        (one shared index-key head)
+ *   M_{i,b}           = max_{j in block b, j <= i} S_{i,j}          (causal block max-pool)
+ *   blocks[b,i,r,:]   = Top-k of {M_{i,c} : c < b_i} by (M desc, block id asc), plus the query's
+ *                       local block b_i = i / block_k, sorted ascending, padded with -1.
+ * A row therefore holds min(k, b_i) + 1 block ids. Scores are never materialised.
+ *   q_idx   bf16  [B, N, H_kv, d_idx]
+ *   k_idx   bf16  [B, N, d_idx]
+ *   blocks  int32 [B, N, H_kv, topk+1]                              (output)
+ *   lse_idx fp32  [B, N, H_kv] or NULL: log-sum-exp of S^idx over the selected causal token set J
+ *           ("KL 对齐" page, section 6: the index pass supplies LSE_idx)  (output, op
+ *           MSA_OP_INDEX_TOPK_LSE sizes the workspace when non-NULL)
+ */
+MSA_API msa_status msa_index_topk(const msa_dims *dims, const void *q_idx, const void *k_idx, int32_t *blocks,
+                          float *lse_idx, void *ws, size_t ws_bytes, msa_stream_t stream);
+
+/*
+ * Main branch: exact causal softmax attention over the union of the selected blocks, each query
+ * head using its group's list ("2.4 · 训练原生稀疏", eq (2); "MSA Indexer" page, section 2.3).
+ *   o[b,i,h] = sum_{j in J} softmax_J(q[b,i,h] . k[b,j,r] * scale)_j v[b,j,r],  r = h / G,
+ *   J = { j <= i : j / block_k in blocks[b,i,r,:] }.
+ *   q      bf16  [B, N, H_q, d]
+ *   k, v   bf16  [B, N, H_kv, d]
+ *   blocks int32 [B, N, H_kv, topk+1]: ids in [0, i/block_k], -1 entries ignored; normally the
+ *          output of msa_index_topk. The local block must be present for J to be non-empty.
+ *   out    bf16  [B, N, H_q, d]                                      (output)
+ *   lse    fp32  [B, N, H_q] or NULL: natural-log sum-exp of the scaled logits over J (output)
+ */
+MSA_API msa_status msa_sparse_attn_fwd(const msa_dims *dims, const void *q, const void *k, const void *v,
+                               const int32_t *blocks, void *out, float *lse, void *ws, size_t ws_bytes,
+                               msa_stream_t stream);
+
+/*
+ * One decode step per sequence: index Top-k then sparse attention for the newest token, whose K, V
+ * and K_idx are already in the caches at position cache_len[b]-1 (MSA blog, decode; the pages'
+ * rule that decode and prefill compute the same R_theta and A_phi).
+ *   dims->N    cache capacity L (rows of the caches)
+ *   cache_len  int32 [B] device, 1 <= cache_len[b] <= N
+ *   q          bf16 [B, H_q, d];  q_idx bf16 [B, H_kv, d_idx]
+ *   k_cache, v_cache bf16 [B, N, H_kv, d];  k_idx_cache bf16 [B, N, d_idx]
+ *   out        bf16 [B, H_q, d]                                      (output)
+ *   blocks_out int32 [B, H_kv, topk+1] or NULL                       (output)
+ */
+MSA_API msa_status msa_sparse_attn_decode(const msa_dims *dims, const int32_t *cache_len, const void *q, const void *q_idx,
+                                  const void *k_cache, const void *v_cache, const void *k_idx_cache, void *out,
+                                  int32_t *blocks_out, void *ws, size_t ws_bytes, msa_stream_t stream);
+
+/*
+ * KL alignment of the index branch ("MSA 中的 KL 对齐与局部知识蒸馏", sections 2, 3 and 6).
+ * On the selected causal token set J of each (query i, group r):
+ *   teacher P_j     = (1/G) sum_{h in group r} exp(q_h . k_j * scale - lse[b,i,h])
+ *   student P^idx_j = exp(S^idx_{i,j} - LSE_idx[b,i,r])
+ *   loss            = sum_{b,i,r} KL(P || P^idx) / (B * N * H_kv)
+ *   g_j             = grad_scale * (P^idx_j - P_j) / (B * N * H_kv)
+ *   dq_idx[b,i,r]   = sum_j g_j * k_idx[b,j] * scale_idx
+ *   dk_idx[b,j]     = sum_{i,r : j in J} g_j * q_idx[b,i,r] * scale_idx
+ * The teacher is detached: no gradient reaches q or k.
+ *   q bf16 [B,N,H_q,d]; k bf16 [B,N,H_kv,d]; q_idx bf16 [B,N,H_kv,d_idx]; k_idx bf16 [B,N,d_idx]
+ *   blocks  int32 [B,N,H_kv,topk+1] (the selection the forward used)
+ *   lse     fp32 [B,N,H_q]   the main forward's LSE (msa_sparse_attn_fwd)
+ *   lse_idx fp32 [B,N,H_kv] or NULL (then computed here)
+ *   loss fp32 [1]; dq_idx fp32 [B,N,H_kv,d_idx]; dk_idx fp32 [B,N,d_idx]   (outputs)
+ */
+MSA_API msa_status msa_kl_fwd_grad(const msa_dims *dims, const void *q, const void *k, const void *q_idx,
+                           const void *k_idx, const int32_t *blocks, const float *lse, const float *lse_idx,
+                           float grad_scale, float *loss, float *dq_idx, float *dk_idx, void *ws, size_t ws_bytes,
+                           msa_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads the device status word of the last call that used `ws`:
+ * MSA_OK, MSA_ERR_TIMEOUT or MSA_ERR_DEVICE_CHECK (or MSA_ERR_CUDA if the stream holds an error).
+ */
+MSA_API msa_status msa_get_device_status(const void *ws, msa_stream_t stream);
+
+/*
+ * Kernel timing (off by default). While enabled, every entry point records a pair of CUDA events
+ * on its stream around each kernel it launches. msa_profile_read synchronises on those events,
+ * adds their durations per kernel name and clears the record: on return names[x] / total_ms[x] /
+ * launches[x] hold up to `cap` kernels; the return value is the number of kernels written, or -1
+ * on a CUDA error. At most 4096 launches are recorded between reads; later ones are not timed.
+ */
+MSA_API void msa_profile_enable(int on);
+MSA_API int msa_profile_read(const char **names, double *total_ms, int *launches, int cap);
+
+/* Static, human-readable name of a status code. */
+MSA_API const char *msa_status_string(msa_status status);
+
+/* Library version string ("msa-b200 <semver>"). */
+MSA_API const char *msa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MSA_H */

@@ -1,0 +1,43 @@
+"""Comparison helpers for the GPU-vs-oracle parity tests (tolerances from the method's acceptance
+criteria: selection bit-exact except near-ties with cutoff margin < 1e-4; attention output max abs
+error <= 1e-2 and mean abs error <= 1e-3; L_KL relative error <= 1e-4; gradients max abs error
+<= 1e-3)."""
+import numpy as np
+
+NEAR_TIE = 1e-4
+ATT_MAX, ATT_MEAN = 1e-2, 1e-3
+LSE_MAX = 2e-3
+KL_REL = 1e-4
+GRAD_MAX = 1e-3
+GRAD_REL = 2e-3  # stricter check used alongside: max error relative to the largest gradient entry
+
+
+def compare_blocks(gpu_blocks, ora_blocks, margin):
+    """Bit-exact equality of the selected block ids for every (row, group) whose cutoff margin is
+    >= NEAR_TIE; returns (number of mismatching rows outside near-ties, number of near-tie rows)."""
+    g = np.asarray(gpu_blocks).reshape(-1, gpu_blocks.shape[-1])
+    o = np.asarray(ora_blocks).reshape(-1, ora_blocks.shape[-1])
+    m = np.asarray(margin).reshape(-1)
+    near = m < NEAR_TIE
+    bad = np.any(g != o, axis=1) & ~near
+    return int(bad.sum()), int(near.sum())
+
+
+def check_attention(out_gpu, out_ref, lse_gpu=None, lse_ref=None):
+    e = np.abs(np.asarray(out_gpu, dtype=np.float64) - np.asarray(out_ref, dtype=np.float64))
+    assert e.max() <= ATT_MAX, f"attention max abs error {e.max():.3e}"
+    assert e.mean() <= ATT_MEAN, f"attention mean abs error {e.mean():.3e}"
+    if lse_gpu is not None:
+        le = np.abs(np.asarray(lse_gpu, dtype=np.float64) - np.asarray(lse_ref, dtype=np.float64))
+        assert le.max() <= LSE_MAX, f"lse max abs error {le.max():.3e}"
+    return float(e.max()), float(e.mean())
+
+
+def check_grad(g_gpu, g_ref, name):
+    g = np.asarray(g_gpu, dtype=np.float64)
+    r = np.asarray(g_ref, dtype=np.float64)
+    e = np.abs(g - r).max()
+    scale = max(np.abs(r).max(), 1e-30)
+    assert e <= GRAD_MAX, f"{name} max abs error {e:.3e}"
+    assert e <= GRAD_REL * scale, f"{name} max error {e:.3e} vs largest entry {scale:.3e}"
+    return float(e), float(e / scale)
