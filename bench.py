@@ -20,9 +20,7 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 import torch
@@ -46,45 +44,63 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while the timed region runs."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event (throttle) reasons read through NVML every 10 ms in a background
+    thread while the timed region runs (read-only queries; no setting is changed)."""
+    REASONS = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+               "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+               "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+               "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+               "hw_power_brake": "nvmlClocksEventReasonHwPowerBrakeSlowdown"}
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
-        self.p = None
+    def __init__(self, gpu_index: int, period_s: float = 0.01):
+        self.gpu, self.period = gpu_index, period_s
+        self.samples, self.max_mhz, self.err = [], None, None
+        self._stop = None
+
+    def _run(self):
+        import pynvml as nv
+        try:
+            nv.nvmlInit()
+            uuid = torch.cuda.get_device_properties(self.gpu).uuid
+            h = None
+            for x in range(nv.nvmlDeviceGetCount()):
+                hx = nv.nvmlDeviceGetHandleByIndex(x)
+                u = nv.nvmlDeviceGetUUID(hx)
+                u = u.decode() if isinstance(u, bytes) else u
+                if str(uuid) in u:
+                    h = hx
+            if h is None:
+                h = nv.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            bits = {k: getattr(nv, v) for k, v in self.REASONS.items()}
+            while not self._stop.is_set():
+                mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((mhz, [k for k, b in bits.items() if rs & b]))
+                time.sleep(self.period)
+            nv.nvmlShutdown()
+        except Exception as e:  # sampling must never break the benchmark
+            self.err = f"{type(e).__name__}: {e}"
 
     def __enter__(self):
-        try:
-            self.p = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv",
-                                       "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
-        except OSError:
-            self.p = None
+        import threading
+        self._stop = threading.Event()
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        time.sleep(0.05)
         return self
 
     def __exit__(self, *exc):
-        if self.p is not None:
-            self.p.terminate()
-            try:
-                self.p.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.p.kill()
+        self._stop.set()
+        self._t.join(timeout=5)
 
     def summary(self) -> dict:
-        self.f.flush()
-        self.f.seek(0)
-        rows = [ln.strip().split(", ") for ln in self.f.read().splitlines()[1:] if ln.strip()]
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        num = lambda s: float(s.split()[0]) if s and s.split()[0].replace(".", "").isdigit() else None
-        sm = [num(r[1]) for r in rows if len(r) > 2 and num(r[1])]
-        mx = [num(r[2]) for r in rows if len(r) > 2 and num(r[2])]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[k] for r in rows if len(r) >= 9 for k in range(4) if r[5 + k].startswith("Active")})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"], "samples": 0,
+                    "error": self.err}
+        reasons = sorted({r for _, rs in self.samples for r in rs})
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml, 10 ms"}
 
 
 def selected_tokens(blocks: torch.Tensor, block_k: int) -> int:
@@ -180,7 +196,7 @@ def run_reference(args, world, rank):
             "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps * (w.N / rows_per_step),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": HEADLINE, "N": w.N, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d, "d_idx": w.d_idx,
+            "config": {"workload": args.workload, "N": w.N, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d, "d_idx": w.d_idx,
                        "block_k": w.block_k, "topk": w.topk},
             "cpu_baseline": {"value": value, "unit": "query-tokens/s", "cores": oracle.num_threads(),
                              "kind": "oracle", "sample": sample},
@@ -202,12 +218,12 @@ def cpu_baseline(x, w, rows_n: int):
     oracle.sparse_attn(od, xc["q"], xc["k"], xc["v"], full, rows=rows)
     dt = time.perf_counter() - t0
     return {"value": rows_n / dt, "unit": "query-tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{rows_n} uniformly drawn query rows of {HEADLINE} (index Top-k + sparse attention), "
+            "sample": f"{rows_n} uniformly drawn query rows of {w.name} (index Top-k + sparse attention), "
                       f"{dt:.1f} s"}
 
 
 def bench_prefill(args, world, rank, msa, pk):
-    w = WORKLOADS[HEADLINE]
+    w = WORKLOADS[args.workload]
     dev = torch.device("cuda", torch.cuda.current_device())
     x = prefill_inputs(w, device=dev, seed=1000 + w.cid + 7919 * rank)
     dims = msa.MsaDims(w.B, w.N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
@@ -264,12 +280,14 @@ def bench_prefill(args, world, rank, msa, pk):
         _, (out, _) = step()
         out_host.copy_(out, non_blocking=True)
 
-    e2e_steps = max(1, min(args.steps, 5))
-    for _ in range(2):
-        e2e_step()
-    barrier(world)
-    te = timed_steps(e2e_step, e2e_steps, flush)
-    e2e_ms = max_over_ranks(sum(te) / len(te), world)
+    e2e_ms = float("nan")
+    if not args.no_e2e:
+        e2e_steps = max(1, min(args.steps, 5))
+        for _ in range(2):
+            e2e_step()
+        barrier(world)
+        te = timed_steps(e2e_step, e2e_steps, flush)
+        e2e_ms = max_over_ranks(sum(te) / len(te), world)
     res = {"value": value, "ms_per_step": step_ms, "roofline": roof, "kernels": per_kernel, "clocks": cs.summary(),
            "e2e": {"value": w.N * w.B * world / (e2e_ms * 1e-3), "unit": "query-tokens/s",
                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
@@ -369,10 +387,13 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--decode-steps", type=int, default=30)
     ap.add_argument("--train-steps", type=int, default=3)
-    ap.add_argument("--cpu-rows", type=int, default=384)
-    ap.add_argument("--ref-rows", type=int, default=48)
+    ap.add_argument("--cpu-rows", type=int, default=4096)
+    ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--workload", default=HEADLINE, choices=["prefill_8k", "prefill_32k_needles", "train_64k"],
+                    help="prefill workload of the headline step (smaller ones serve profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -388,12 +409,12 @@ def main():
     import block_sparse_attention_idx_b200 as msa
     pk = peaks()
     pre = bench_prefill(args, world, rank, msa, pk)
-    w = WORKLOADS[HEADLINE]
+    w = WORKLOADS[args.workload]
     line = {"metric": METRIC, "value": pre["value"], "unit": "query-tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": pre["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": HEADLINE, "N": w.N, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d, "d_idx": w.d_idx,
+            "config": {"workload": args.workload, "N": w.N, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d, "d_idx": w.d_idx,
                        "block_k": w.block_k, "topk": w.topk, "batch_per_gpu": w.B, "global_batch": w.B * world,
                        "parallelism": f"dp{world} (independent sequences)",
                        "l2": "flushed (256 MiB write) before every timed step",
