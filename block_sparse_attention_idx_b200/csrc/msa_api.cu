@@ -36,7 +36,7 @@ msa_status check_common(const msa_dims* d) {
     if (d->H_q % d->H_kv != 0) return MSA_ERR_INVALID_ARG;
     if (!(d->scale >= 0.f) || !(d->scale_idx >= 0.f)) return MSA_ERR_INVALID_ARG;
     const int G = d->H_q / d->H_kv;
-    if (128 % G != 0 || 128 % d->H_kv != 0 || d->H_kv > 8) return MSA_ERR_UNSUPPORTED;
+    if (128 % G != 0 || G > 32 || 128 % d->H_kv != 0 || d->H_kv > 8) return MSA_ERR_UNSUPPORTED;
     if (d->d != 64 && d->d != 128) return MSA_ERR_UNSUPPORTED;
     if (d->d_idx != 32 && d->d_idx != 64) return MSA_ERR_UNSUPPORTED;
     if (d->block_k != 32 && d->block_k != 64 && d->block_k != 128) return MSA_ERR_UNSUPPORTED;
@@ -49,7 +49,7 @@ msa_status check_common(const msa_dims* d) {
 
 float eff_scale(float s, int dim) { return s > 0.f ? s : 1.0f / sqrtf((float)dim); }
 
-size_t csr_need(const msa_dims* d) { return csr_bytes(d->B, d->N, d->H_kv, d->block_k, d->topk); }
+size_t csr_need(const msa_dims* d) { return csr_bytes(d->B, d->N, d->H_kv, d->block_k, d->topk, 0); }
 
 size_t rows_kv(const msa_dims* d) { return (size_t)d->B * d->N * d->H_kv; }
 
@@ -57,8 +57,7 @@ size_t ws_index_lse(const msa_dims* d) {
     return kStatusBytes + csr_need(d) + al256(rows_kv(d) * (d->topk + 1) * sizeof(float2));
 }
 size_t ws_attn(const msa_dims* d) {
-    const size_t pr = (size_t)d->B * d->N * d->H_q * (d->topk + 1);
-    return kStatusBytes + csr_need(d) + al256(pr * d->d * sizeof(float)) + al256(pr * sizeof(float));
+    return kStatusBytes + attn_ws_bytes(d->B, d->N, d->H_q, d->H_kv, d->d, d->block_k, d->topk);
 }
 size_t ws_decode(const msa_dims* d) {
     return kStatusBytes + decode_ws_bytes(d->B, d->N, d->H_q, d->H_kv, d->d, d->block_k, d->topk);
@@ -67,7 +66,7 @@ size_t ws_kl(const msa_dims* d) {
     const size_t nb = (size_t)(d->N + d->block_k - 1) / d->block_k;
     const size_t nl = (size_t)d->B * d->H_kv * nb;
     const size_t me = rows_kv(d) * (d->topk + 1);
-    const size_t csr_idx_extra = al256((nl + 1) * 4) + al256(me * 8) + 256;
+    const size_t csr_idx_extra = al256((nl + 1) * 4) + al256(me * 16) + 256;
     return kStatusBytes + csr_need(d) + csr_idx_extra + al256(me * sizeof(float2)) + al256(rows_kv(d) * 4) +
            al256(me * d->d_idx * 4) + al256(me * 8) + al256(rows_kv(d) * 8);
 }
@@ -144,7 +143,7 @@ msa_status msa_index_topk(const msa_dims* d, const void* q_idx, const void* k_id
     k.B = d->B; k.N = d->N; k.H_q = d->H_q; k.H_kv = d->H_kv; k.d = d->d; k.d_idx = d->d_idx;
     k.block_k = d->block_k; k.topk = d->topk;
     k.scale = eff_scale(d->scale, d->d); k.scale_idx = eff_scale(d->scale_idx, d->d_idx);
-    csr_carve(&k.csr_idx, cv.take(csr_need(d)), d->B, d->N, d->H_kv, d->block_k, d->topk);
+    csr_carve(&k.csr_idx, cv.take(csr_need(d)), d->B, d->N, d->H_kv, d->block_k, d->topk, 0);
     k.ml_part = reinterpret_cast<float2*>(cv.take(rows_kv(d) * (d->topk + 1) * sizeof(float2)));
     k.lse_idx = lse_idx;
     k.blocks = blocks;
@@ -167,19 +166,15 @@ msa_status msa_sparse_attn_fwd(const msa_dims* d, const void* q, const void* k, 
     DevStatus* status = static_cast<DevStatus*>(ws);
     cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, st);
     if (e != cudaSuccess) return MSA_ERR_CUDA;
-    Carver cv{static_cast<uint8_t*>(ws) + kStatusBytes};
     AttnArgs a{};
     a.B = d->B; a.N = d->N; a.H_q = d->H_q; a.H_kv = d->H_kv; a.d = d->d; a.block_k = d->block_k;
     a.topk = d->topk; a.scale = eff_scale(d->scale, d->d);
-    csr_carve(&a.csr, cv.take(csr_need(d)), d->B, d->N, d->H_kv, d->block_k, d->topk);
-    const size_t pr = (size_t)d->B * d->N * d->H_q * (d->topk + 1);
-    a.o_part = reinterpret_cast<float*>(cv.take(pr * d->d * sizeof(float)));
-    a.lse_part = reinterpret_cast<float*>(cv.take(pr * sizeof(float)));
+    attn_carve(&a, static_cast<uint8_t*>(ws) + kStatusBytes);
+    a.blocks = blocks;
+    a.out = static_cast<__nv_bfloat16*>(out);
+    a.lse = lse;
     a.status = status;
-    const int G = d->H_q / d->H_kv;
-    e = run_csr_build(a.csr, blocks, d->B, d->N, d->H_kv, d->block_k, d->topk, 128 / G, status, st);
-    if (e == cudaSuccess) e = run_attn_kv_outer(a, q, k, v, num_sms(), st);
-    if (e == cudaSuccess) e = run_attn_merge(a, blocks, out, lse, st);
+    e = run_attn(a, q, k, v, num_sms(), st);
     return cuda_status(e);
 }
 
@@ -244,10 +239,10 @@ msa_status msa_kl_fwd_grad(const msa_dims* d, const void* q, const void* k, cons
     a.block_k = d->block_k; a.topk = d->topk;
     a.scale = eff_scale(d->scale, d->d); a.scale_idx = eff_scale(d->scale_idx, d->d_idx);
     a.grad_scale = grad_scale;
-    csr_carve(&a.csr, cv.take(csr_need(d)), d->B, d->N, d->H_kv, d->block_k, d->topk);
+    csr_carve(&a.csr, cv.take(csr_need(d)), d->B, d->N, d->H_kv, d->block_k, d->topk, 0);
     a.csr_idx = a.csr;  // same lists, its own chunking
     a.csr_idx.chunk_off = reinterpret_cast<int32_t*>(cv.take((nl + 1) * 4));
-    a.csr_idx.items = reinterpret_cast<int2*>(cv.take(me * 8));
+    a.csr_idx.items = reinterpret_cast<int4*>(cv.take(me * 16));
     a.csr_idx.n_items = reinterpret_cast<int32_t*>(cv.take(256));
     a.ml_part = reinterpret_cast<float2*>(cv.take(me * sizeof(float2)));
     float* lse_idx_ws = reinterpret_cast<float*>(cv.take(rows_kv(d) * 4));

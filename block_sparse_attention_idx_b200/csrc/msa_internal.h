@@ -2,6 +2,7 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include <algorithm>
@@ -38,38 +39,51 @@ struct IndexArgs {
 cudaError_t run_index_topk(const IndexArgs& a, const void* q_idx, const void* k_idx, cudaStream_t st);
 
 // ---------------------------------------------------------------- inverse selection lists (msa_csr.cu)
-// For every (sequence b, group r, block c) the list of (query i, slot s) pairs whose selection
-// row blocks[b,i,r,:] holds c at position s, cut into work items of at most `qpc` queries.
+// For every (sequence b, query window w, group r, block c) the list of (query i, slot s) pairs
+// whose selection row blocks[b,i,r,:] holds c at position s, cut into work items of at most `qpc`
+// queries. A window is `wq` consecutive queries (wq = 0: one window per sequence). Items are
+// ordered by (b, w, r, c).
 struct Csr {
-    int nlists;        // B * H_kv * nb
+    int nlists;        // B * nW * H_kv * nb
     int nb;            // blocks per sequence
+    int nW;            // windows per sequence
+    int wq;            // queries per window (N when wq = 0)
     int max_entries;   // B * N * H_kv * (topk+1)
+    int nscan;         // scan blocks: ceil(nlists / 1024)
     int32_t* counts;   // [nlists]
     int32_t* offsets;  // [nlists + 1]
     int32_t* cursor;   // [nlists]
     int32_t* chunk_off;// [nlists + 1]
     int32_t* entries;  // [max_entries]  (i << 5) | s
-    int2* items;       // [max_entries]  (list, first entry of the chunk within the list)
+    int4* items;       // [max_entries]  (list, index of the chunk's first entry, queries, 0)
     int32_t* n_items;  // [1]
+    int32_t* bsum;     // [2 * nscan + 2] scan block sums and totals
+    uint8_t* nsel;     // [B * N * H_kv] number of valid blocks of each selection row
 };
-size_t csr_bytes(int B, int N, int H_kv, int block_k, int topk);
-void csr_carve(Csr* c, void* base, int B, int N, int H_kv, int block_k, int topk);
+size_t csr_bytes(int B, int N, int H_kv, int block_k, int topk, int wq);
+void csr_carve(Csr* c, void* base, int B, int N, int H_kv, int block_k, int topk, int wq);
 cudaError_t run_csr_build(const Csr& c, const int32_t* blocks, int B, int N, int H_kv, int block_k, int topk,
                           int qpc, DevStatus* st, cudaStream_t stream);
 cudaError_t run_csr_items(const Csr& c, int qpc, cudaStream_t stream);
 
 // ---------------------------------------------------------------- sparse attention (msa_attn.cu)
+constexpr int kAttnWindow = 128;  // queries per window of the attention's inverse lists
 struct AttnArgs {
     int B, N, H_q, H_kv, d, block_k, topk;
     float scale;
-    Csr csr;
-    float* o_part;    // [B, N, H_q, topk+1, d]
-    float* lse_part;  // [B, N, H_q, topk+1]
+    Csr csr;             // windowed lists, items of 128/G queries
+    __half* o_part;      // [B, N, H_q, topk+1, d]   normalised partial outputs
+    float* lse_part;     // [B, N, H_q, topk+1]
+    int32_t* counter;    // [B, N, H_kv]  items finished per selection row
+    int32_t* sched;      // [1]           next item to hand out
+    const int32_t* blocks;
+    __nv_bfloat16* out;  // [B, N, H_q, d]
+    float* lse;          // [B, N, H_q] or null
     DevStatus* status;
 };
-cudaError_t run_attn_kv_outer(const AttnArgs& a, const void* q, const void* k, const void* v, int num_sms,
-                              cudaStream_t st);
-cudaError_t run_attn_merge(const AttnArgs& a, const int32_t* blocks, void* out, float* lse, cudaStream_t st);
+size_t attn_ws_bytes(int B, int N, int H_q, int H_kv, int d, int block_k, int topk);
+void attn_carve(AttnArgs* a, void* base);
+cudaError_t run_attn(const AttnArgs& a, const void* q, const void* k, const void* v, int num_sms, cudaStream_t st);
 
 // ---------------------------------------------------------------- KL alignment (msa_kl.cu)
 struct KlArgs {

@@ -57,8 +57,8 @@ __global__ void __launch_bounds__(128) k_lse_idx(KlArgs a, const __nv_bfloat16* 
     float kr[DI];
     int prevL = -1;
     for (int item = blockIdx.x; item < T; item += gridDim.x) {
-        const int2 it = cs.items[item];
-        const int L = it.x, count = min(kIdxQpc, cs.counts[L] - it.y);
+        const int4 it = cs.items[item];
+        const int L = it.x, count = it.z;
         const int c = L % cs.nb, r = (L / cs.nb) % a.H_kv, b = L / (cs.nb * a.H_kv);
         const int tok = c * a.block_k + t;
         const bool tvalid = t < a.block_k && tok < a.N;
@@ -68,7 +68,7 @@ __global__ void __launch_bounds__(128) k_lse_idx(KlArgs a, const __nv_bfloat16* 
             prevL = L;
         }
         if (t < count) {
-            const int e = cs.entries[cs.offsets[L] + it.y + t];
+            const int e = cs.entries[it.y + t];
             s_i[t] = e >> 5;
             s_slot[t] = e & 31;
         }
@@ -195,14 +195,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         int kv_loads = 0, prevL = -1;
         int ok = 1;
         for (int t = t0, n = 0; t < t1 && ok; ++t, ++n) {
-            const int2 itm = cs.items[t];
-            const int L = itm.x, count = min(QPC, cs.counts[L] - itm.y);
+            const int4 itm = cs.items[t];
+            const int L = itm.x, count = itm.z;
             const int c = L % cs.nb, r = (L / cs.nb) % a.H_kv, b = L / (cs.nb * a.H_kv);
             const int buf = n & 1;
             if (lane == 0) ok = mbar_wait(&s.q_empty[buf], ((n >> 1) & 1) ^ 1, a.status, 0x801);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
-            const int* ent = cs.entries + cs.offsets[L] + itm.y;
+            const int* ent = cs.entries + itm.y;
             for (int m = lane; m < QPC; m += 32) {
                 const int e = m < count ? ent[m] : 0;
                 s.qi[buf][m] = m < count ? (e >> 5) : -1;
@@ -295,8 +295,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         int prevL = -1, prev_b = 0, prev_tok = 0;
         bool prev_valid = false;
         for (int t = t0, n = 0; t < t1; ++t, ++n) {
-            const int2 itm = cs.items[t];
-            const int L = itm.x, count = min(QPC, cs.counts[L] - itm.y);
+            const int4 itm = cs.items[t];
+            const int L = itm.x, count = itm.z;
             const int c = L % cs.nb, r = (L / cs.nb) % a.H_kv, b = L / (cs.nb * a.H_kv);
             const int buf = n & 1;
             const int tok = c * BK + tt;

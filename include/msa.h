@@ -28,8 +28,11 @@
  *   loss. dK_idx is accumulated with float32 atomics and may differ in the last bits.
  *
  * Supported sizes (MSA_ERR_UNSUPPORTED otherwise): d in {64, 128}, d_idx in {32, 64},
- * block_k in {32, 64, 128}, 1 <= topk <= 16, H_q % H_kv == 0 with G = H_q/H_kv dividing 128,
- * H_kv dividing 128, N >= 1, B >= 1, block ids fit the workspace (N <= 2^24).
+ * block_k in {32, 64, 128}, 1 <= topk <= 16, H_q % H_kv == 0 with G = H_q/H_kv in {1,2,4,8,16,32},
+ * H_kv in {1,2,4,8}, N >= 1, B >= 1, N < 2^24 and B*N*H_kv*(topk+1) < 2^30. The attention keeps
+ * its per-slot partial outputs in fp16: entries of V must stay below 65504 in magnitude (larger
+ * values are reported as MSA_ERR_DEVICE_CHECK). msa_kl_fwd_grad supports (d, d_idx) in
+ * {(128, 64), (64, 32)} with G in {2, 16}.
  */
 #ifndef MSA_H
 #define MSA_H
