@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
         L.msa_sparse_attn_fwd.argtypes = [D, P, P, P, P, P, P, P, S, P]
         L.msa_sparse_attn_decode.argtypes = [D, P, P, P, P, P, P, P, P, P, S, P]
         L.msa_kl_fwd_grad.argtypes = [D, P, P, P, P, P, P, P, ctypes.c_float, P, P, P, P, S, P]
+        L.msa_sparse_attn_decode_noalloc.argtypes = [D, P, P, P, P, P, P, P, P, P]
+        L.msa_sparse_attn_decode_noalloc.restype = ctypes.c_int
         L.msa_get_device_status.argtypes = [P, P]
         L.msa_profile_enable.argtypes = [ctypes.c_int]
         L.msa_profile_enable.restype = None
@@ -183,6 +185,30 @@ def msa_sparse_attn_decode(dims: MsaDims, cache_len, q, q_idx, k_cache, v_cache,
     return out, blocks
 
 
+def msa_sparse_attn_decode_noalloc(dims: MsaDims, cache_len, q, q_idx, k_cache, v_cache, k_idx_cache, out=None,
+                                   blocks=None, stream=None):
+    """Decode step through the allocation-free entry point (the library's static 16 MiB device scratch
+    instead of a workspace). For callers that cannot allocate device memory while decoding; outputs may
+    be passed in preallocated. Calls on one device share the scratch and must not overlap on the GPU."""
+    dev = q.device
+    _need(cache_len, "cache_len", (dims.B,), torch.int32, dev)
+    _need(q, "q", (dims.B, dims.H_q, dims.d), torch.bfloat16, dev)
+    _need(q_idx, "q_idx", (dims.B, dims.H_kv, dims.d_idx), torch.bfloat16, dev)
+    _need(k_cache, "k_cache", (dims.B, dims.N, dims.H_kv, dims.d), torch.bfloat16, dev)
+    _need(v_cache, "v_cache", (dims.B, dims.N, dims.H_kv, dims.d), torch.bfloat16, dev)
+    _need(k_idx_cache, "k_idx_cache", (dims.B, dims.N, dims.d_idx), torch.bfloat16, dev)
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", (dims.B, dims.H_q, dims.d), torch.bfloat16, dev)
+    if blocks is not None:
+        _need(blocks, "blocks", (dims.B, dims.H_kv, dims.topk + 1), torch.int32, dev)
+    _check("msa_sparse_attn_decode_noalloc",
+           lib().msa_sparse_attn_decode_noalloc(ctypes.byref(dims.c()), _p(cache_len), _p(q), _p(q_idx),
+                                                _p(k_cache), _p(v_cache), _p(k_idx_cache), _p(out), _p(blocks),
+                                                _stream(stream)))
+    return out, blocks
+
+
 def msa_kl_fwd_grad(dims: MsaDims, q, k, q_idx, k_idx, blocks, lse, lse_idx=None, grad_scale: float = 1.0, ws=None,
                     stream=None):
     """KL alignment. Returns loss fp32 [1], dq_idx fp32 [B,N,H_kv,d_idx], dk_idx fp32 [B,N,d_idx]."""
@@ -230,5 +256,5 @@ def msa_get_device_status(ws: torch.Tensor, stream=None) -> int:
 
 
 __all__ = ["MsaDims", "MsaError", "msa_workspace_size", "msa_index_topk", "msa_sparse_attn_fwd",
-           "msa_sparse_attn_decode", "msa_kl_fwd_grad", "msa_get_device_status", "msa_status_string",
+           "msa_sparse_attn_decode", "msa_sparse_attn_decode_noalloc", "msa_kl_fwd_grad", "msa_get_device_status", "msa_status_string",
            "msa_version", "msa_profile_enable", "msa_profile_read", "workspace", "lib", "LIB_PATH"]

@@ -150,6 +150,30 @@ MSA_API msa_status msa_kl_fwd_grad(const msa_dims *dims, const void *q, const vo
                            msa_stream_t stream);
 
 /*
+ * Allocation-free decode step (no counterpart in the pages; a convenience of this library).
+ * For callers that cannot allocate device memory where they decode (a plugin inside a host
+ * application that owns every device allocation, a serving loop with a memory budget fixed at
+ * start-up, a latency-bound path that must not call cudaMalloc, which can synchronise the device).
+ * Same arguments, outputs and results as msa_sparse_attn_decode, minus the workspace: the scratch
+ * is a static device array of MSA_DECODE_STATIC_SCRATCH_BYTES (16 MiB) that every GPU loading this
+ * library holds until the process exits. It allocates and frees nothing.
+ * - Returns MSA_ERR_WORKSPACE when `dims` need more scratch than that maximum
+ *   (msa_workspace_size(MSA_OP_DECODE, dims) > MSA_DECODE_STATIC_SCRATCH_BYTES), e.g. the 16 x 262144
+ *   decode step needs about 9.5 MiB, 32 sequences of 262144 tokens would not fit.
+ * - The first call on a device looks up the array's device address with that device current
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ * - All calls on one device share the array and it keeps the last call's contents; calls that can
+ *   overlap on the GPU (unordered streams) race on it and must be serialised by the caller.
+ * - The device status word of these calls lives in the shared array; it cannot be read with
+ *   msa_get_device_status.
+ */
+#define MSA_DECODE_STATIC_SCRATCH_BYTES (16u << 20)
+MSA_API msa_status msa_sparse_attn_decode_noalloc(const msa_dims *dims, const int32_t *cache_len, const void *q,
+                                                  const void *q_idx, const void *k_cache, const void *v_cache,
+                                                  const void *k_idx_cache, void *out, int32_t *blocks_out,
+                                                  msa_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads the device status word of the last call that used `ws`:
  * MSA_OK, MSA_ERR_TIMEOUT or MSA_ERR_DEVICE_CHECK (or MSA_ERR_CUDA if the stream holds an error).
  */
