@@ -63,7 +63,7 @@ struct AttnSmem {
     int epi_done;
     uint64_t meta_full[kMeta], meta_empty[kMeta];
     uint64_t q_full[2], q_empty[2];
-    uint64_t k_full[2], k_release, v_full[2], v_release;
+    uint64_t k_full[2], k_release[2], v_full[2], v_release[2];  // release[b]: one completion per use of buffer b
     uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
     uint64_t drain;
     uint32_t tmem_base;
@@ -110,9 +110,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&s.p_full[x], kRows);
             mbar_init(&s.o_full[x], 1);
             mbar_init(&s.o_free[x], kRows);
+            mbar_init(&s.k_release[x], 1);
+            mbar_init(&s.v_release[x], 1);
         }
-        mbar_init(&s.k_release, 1);
-        mbar_init(&s.v_release, 1);
         mbar_init(&s.drain, 1);
         s.abort = 0;
         s.mq_tail = 0;
@@ -227,10 +227,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s.q_full[buf]);
             }
-            // K of a new block goes to buffer kgroup % 2 once the S MMAs of block kgroup-2 are done
+            // K of block group g goes to buffer g % 2 once the S MMAs of group g-2 (the buffer's
+            // previous use, release number (g-2)/2 of that buffer) are done
             if (L != prevL) {
                 ++kgroup;
-                if (kgroup >= 2 && !wait_lane0(&s.k_release, (kgroup - 2) & 1, a.status, 0x504)) { ok = false; break; }
+                if (kgroup >= 2 &&
+                    !wait_lane0(&s.k_release[kgroup & 1], ((kgroup - 2) >> 1) & 1, a.status, 0x504)) { ok = false; break; }
                 if (lane == 0) {
                     const int kb = kgroup & 1;
                     mbar_arrive_expect_tx(&s.k_full[kb], (uint32_t)Sm::kKVBytes);
@@ -260,7 +262,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (kv_new) {
                 // V of block group g goes to buffer g % 2 once the PV MMAs of group g-2 are done
                 ++vgroup;
-                if (vgroup >= 2 && !wait_lane0(&s.v_release, (vgroup - 2) & 1, a.status, 0x512)) { ok = false; break; }
+                if (vgroup >= 2 &&
+                    !wait_lane0(&s.v_release[vgroup & 1], ((vgroup - 2) >> 1) & 1, a.status, 0x512)) { ok = false; break; }
                 if (lane == 0) {
                     const int vb = vgroup & 1;
                     mbar_arrive_expect_tx(&s.v_full[vb], (uint32_t)Sm::kKVBytes);
@@ -284,9 +287,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             int ns = 0, np = 0, n_end = -1;
             bool meta_read = false;
-            int cur_kvn = 0;
-            int kgroup = -1, vgroup = -1;
-            int kvn_ring[kMeta] = {0, 0, 0, 0}, grp_ring[kMeta] = {0, 0, 0, 0};
+            int cur_kvn = 0, cur_grp = -1;
+            int groups = -1;          // block groups seen so far (metadata order)
+            int pend_pv = -1;         // PV issued whose item's successor group was not yet known
+            int grp_ring[kMeta] = {0, 0, 0, 0};
             uint64_t t_idle = globaltimer();
             while (true) {
                 bool progressed = false;
@@ -299,46 +303,47 @@ __global__ void __launch_bounds__(kThreads, 1)
                         } else {
                             mbar_arrive(&s.meta_empty[ns % kMeta]);
                             meta_read = true;
+                            if (cur_kvn) {
+                                ++groups;
+                                if (ns > 0) {
+                                    // item ns-1 closed block group groups-1: every S of it has been
+                                    // issued, so its K buffer is free once they complete
+                                    umma_commit(&s.k_release[(groups - 1) & 1]);
+                                }
+                            }
+                            cur_grp = groups;
+                            // a PV waiting to learn whether it closed its group
+                            if (pend_pv >= 0 && pend_pv == ns - 1) {
+                                if (cur_kvn) umma_commit(&s.v_release[grp_ring[pend_pv % kMeta] & 1]);
+                                pend_pv = -1;
+                            }
                         }
                         progressed = true;
                     }
-                    if (meta_read && np >= ns - 1 && mbar_test(&s.q_full[ns & 1], (ns >> 1) & 1)) {
-                        const int g = cur_kvn ? kgroup + 1 : kgroup;
-                        if (mbar_test(&s.k_full[g & 1], (g >> 1) & 1)) {
-                            if (cur_kvn) {
-                                // every S of the previous block has been issued: its K buffer is
-                                // released once they complete
-                                if (kgroup >= 0) umma_commit(&s.k_release);
-                                kgroup = g;
-                            }
-                            tc_fence_after();
-                            const uint32_t qb = smem_u32(s.q[ns & 1]), kb = smem_u32(s.k[g & 1]);
-                            const uint32_t tS = tmem + (ns & 1) * 256;
+                    if (meta_read && np >= ns - 1 && mbar_test(&s.q_full[ns & 1], (ns >> 1) & 1) &&
+                        mbar_test(&s.k_full[cur_grp & 1], (cur_grp >> 1) & 1)) {
+                        tc_fence_after();
+                        const uint32_t qb = smem_u32(s.q[ns & 1]), kb = smem_u32(s.k[cur_grp & 1]);
+                        const uint32_t tS = tmem + (ns & 1) * 256;
 #pragma unroll
-                            for (int ks = 0; ks < D / 16; ++ks) {
-                                const uint32_t sub = (ks * 16) / 64, off = (ks & 3) * 32;
-                                const uint64_t da = umma_sdesc(qb + sub * (kRows * 128) + off, 16, 1024, 2);
-                                const uint64_t db = umma_sdesc(kb + sub * (BK * 128) + off, 16, 1024, 2);
-                                umma_bf16(tS, da, db, kIdescS, ks > 0);
-                            }
-                            umma_commit(&s.s_full[ns & 1]);
-                            umma_commit(&s.q_empty[ns & 1]);
-                            kvn_ring[ns % kMeta] = cur_kvn;
-                            grp_ring[ns % kMeta] = g;
-                            ++ns;
-                            meta_read = false;
-                            progressed = true;
+                        for (int ks = 0; ks < D / 16; ++ks) {
+                            const uint32_t sub = (ks * 16) / 64, off = (ks & 3) * 32;
+                            const uint64_t da = umma_sdesc(qb + sub * (kRows * 128) + off, 16, 1024, 2);
+                            const uint64_t db = umma_sdesc(kb + sub * (BK * 128) + off, 16, 1024, 2);
+                            umma_bf16(tS, da, db, kIdescS, ks > 0);
                         }
+                        umma_commit(&s.s_full[ns & 1]);
+                        umma_commit(&s.q_empty[ns & 1]);
+                        grp_ring[ns % kMeta] = cur_grp;
+                        ++ns;
+                        meta_read = false;
+                        progressed = true;
                     }
                 }
                 if (np < ns && mbar_test(&s.p_full[np & 1], (np >> 1) & 1) &&
                     mbar_test(&s.o_free[np & 1], ((np >> 1) & 1) ^ 1)) {
                     const int g = grp_ring[np % kMeta];
                     if (mbar_test(&s.v_full[g & 1], (g >> 1) & 1)) {
-                        if (kvn_ring[np % kMeta]) {
-                            if (vgroup >= 0) umma_commit(&s.v_release);
-                            vgroup = g;
-                        }
                         tc_fence_after();
                         const uint32_t vb = smem_u32(s.v[g & 1]);
                         const uint32_t tP = tmem + (np & 1) * 256;        // P (bf16 pairs) over S
@@ -349,6 +354,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             umma_bf16_tmem_a(tO, tP + ks * 8, db, kIdescO, ks > 0);
                         }
                         umma_commit(&s.o_full[np & 1]);
+                        // if item np closed its block group, its V buffer is free once this PV is done
+                        if (np + 1 < ns) {
+                            if (grp_ring[(np + 1) % kMeta] != g) umma_commit(&s.v_release[g & 1]);
+                        } else if (np + 1 == ns && meta_read) {
+                            if (cur_grp != g) umma_commit(&s.v_release[g & 1]);
+                        } else {
+                            pend_pv = np;
+                        }
                         ++np;
                         progressed = true;
                     }
