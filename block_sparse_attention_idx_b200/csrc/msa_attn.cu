@@ -390,8 +390,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const uint32_t tS = lane_addr + wg * 256, tO = lane_addr + wg * 256 + 128;
         const float sl2 = a.scale * 1.4426950408889634f;
-        bool pend = false;
-        int pend_old = 0, pend_nsel = 0, pend_b = 0, pend_i = 0, pend_r = 0;
+        // Row counting runs two items behind the stores it publishes: the increment for item n is
+        // issued during item n+1 (its release then finds item n's partial stores long performed) and
+        // its returned count is looked at during item n+2.
+        bool inc = false, chk = false;
+        int inc_nsel = 0, inc_b = 0, inc_i = 0, inc_r = 0;
+        int chk_old = 0, chk_nsel = 0, chk_b = 0, chk_i = 0, chk_r = 0;
+        auto push_task = [&](int tb, int ti, int tr, unsigned where) {
+            const int k = atomicAdd(&s.mq_tail, 1);
+            MergeTask& task = s.mq[k % kMQ];
+            const int gen = k / kMQ;
+            const uint64_t t0 = globaltimer();
+            while (task.done != gen) {  // the slot's previous task must have been taken
+                if (globaltimer() - t0 > MSA_WAIT_NS) {
+                    raise_flag(a.status, MSA_DEV_TIMEOUT, where);
+                    break;
+                }
+                __nanosleep(64);
+            }
+            task.b = tb;
+            task.i = ti;
+            task.r = tr;
+            __threadfence_block();
+            task.full = gen + 1;
+        };
         for (int n = wg;; n += 2) {
             const int slot = n % kMeta;
             if (!__all_sync(0xffffffffu, mbar_wait(&s.meta_full[slot], (n / kMeta) & 1, a.status, 0x701))) {
@@ -470,28 +492,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&s.p_full[wg]);
-            // the row-counter increment of this warpgroup's previous item has had a whole item of
-            // time to return: hand finished rows to the merge warps now
-            if (pend) {
-                if (pend_old + 1 == pend_nsel) {
-                    const int k = atomicAdd(&s.mq_tail, 1);
-                    MergeTask& task = s.mq[k % kMQ];
-                    const int gen = k / kMQ;
-                    const uint64_t t0 = globaltimer();
-                    while (task.done != gen) {  // the slot's previous task must have been taken
-                        if (globaltimer() - t0 > MSA_WAIT_NS) {
-                            raise_flag(a.status, MSA_DEV_TIMEOUT, 0x706);
-                            break;
-                        }
-                        __nanosleep(64);
-                    }
-                    task.b = pend_b;
-                    task.i = pend_i;
-                    task.r = pend_r;
-                    __threadfence_block();
-                    task.full = gen + 1;
-                }
-                pend = false;
+            // rows whose count came back complete go to the merge warps; then count the previous item
+            if (chk) {
+                if (chk_old + 1 == chk_nsel) push_task(chk_b, chk_i, chk_r, 0x706);
+                chk = false;
+            }
+            if (inc) {
+                chk_old = atom_add_acq_rel_gpu(&a.counter[((size_t)inc_b * a.N + inc_i) * a.H_kv + inc_r], 1);
+                chk_nsel = inc_nsel;
+                chk_b = inc_b;
+                chk_i = inc_i;
+                chk_r = inc_r;
+                chk = true;
+                inc = false;
             }
             if (!__all_sync(0xffffffffu, mbar_wait(&s.o_full[wg], kk & 1, a.status, 0x704))) {
                 s.abort = 1;
@@ -525,38 +538,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             mbar_arrive(&s.o_free[wg]);
             if (valid) a.lse_part[prow] = mx * a.scale + logf(l);
-            // ---- count this item for its (query, group) rows. The warp barrier orders the G lanes'
-            // partial stores before their leader's acquire-release increment; the returned count is
-            // looked at one item later, so its round trip overlaps the next item.
+            // ---- this item counts for its (query, group) rows. The warp barrier orders the G lanes'
+            // partial stores before their leader's later acquire-release increment.
             __syncwarp();
             if (valid && h == 0) {
-                const size_t krow = ((size_t)b * a.N + i) * a.H_kv + r;
-                pend_old = atom_add_acq_rel_gpu(&a.counter[krow], 1);
-                pend_nsel = my_nsel;
-                pend_b = b;
-                pend_i = i;
-                pend_r = r;
-                pend = true;
+                inc_nsel = my_nsel;
+                inc_b = b;
+                inc_i = i;
+                inc_r = r;
+                inc = true;
             }
         }
-        // flush the last pending row of this warpgroup
-        if (pend && pend_old + 1 == pend_nsel) {
-            const int k = atomicAdd(&s.mq_tail, 1);
-            MergeTask& task = s.mq[k % kMQ];
-            const int gen = k / kMQ;
-            const uint64_t t0 = globaltimer();
-            while (task.done != gen) {
-                if (globaltimer() - t0 > MSA_WAIT_NS) {
-                    raise_flag(a.status, MSA_DEV_TIMEOUT, 0x707);
-                    break;
-                }
-                __nanosleep(64);
-            }
-            task.b = pend_b;
-            task.i = pend_i;
-            task.r = pend_r;
-            __threadfence_block();
-            task.full = gen + 1;
+        // flush the rows still being counted
+        if (chk && chk_old + 1 == chk_nsel) push_task(chk_b, chk_i, chk_r, 0x707);
+        if (inc) {
+            const int old = atom_add_acq_rel_gpu(&a.counter[((size_t)inc_b * a.N + inc_i) * a.H_kv + inc_r], 1);
+            if (old + 1 == inc_nsel) push_task(inc_b, inc_i, inc_r, 0x707);
         }
         __syncwarp();
         if (lane == 0) {
@@ -594,17 +591,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) task.done = gen + 1;
             // valid slots of the row (same rule as the list builder)
             const int32_t* sel = a.blocks + (((size_t)b * a.N + i) * a.H_kv + r) * K1;
-            uint32_t vmask = 0;
-            if (lane == 0) {
-                int prev = -1;
-                for (int x = 0; x < K1; ++x) {
-                    const int cb = __ldg(sel + x);
-                    if (cb < 0 || cb > i / BK || cb <= prev) continue;
-                    prev = cb;
-                    vmask |= 1u << x;
-                }
+            // slot x is kept when its block is causal and above every kept block before it; the
+            // largest kept block so far equals the largest in-range block so far (prefix max)
+            const int cb = lane < K1 ? __ldg(sel + lane) : -1;
+            const bool inr = cb >= 0 && cb <= i / BK;
+            int pm = inr ? cb : -1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, pm, o);
+                if (lane >= o) pm = max(pm, t);
             }
-            vmask = __shfl_sync(0xffffffffu, vmask, 0);
+            int prev = __shfl_up_sync(0xffffffffu, pm, 1);
+            if (lane == 0) prev = -1;
+            const uint32_t vmask = __ballot_sync(0xffffffffu, inr && cb > prev);
             constexpr int kK1Max = 17;
             bool overflow = false;
             for (int u = lane; u < units; u += 32) {
