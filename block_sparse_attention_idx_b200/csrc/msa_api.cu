@@ -56,6 +56,10 @@ size_t rows_kv(const msa_dims* d) { return (size_t)d->B * d->N * d->H_kv; }
 size_t ws_index_lse(const msa_dims* d) {
     return kStatusBytes + csr_need(d) + al256(rows_kv(d) * (d->topk + 1) * sizeof(float2));
 }
+// The prefill attention indexes its (query, head, slot) partial rows with 31 bits.
+bool attn_rows_fit(const msa_dims* d) {
+    return (double)d->B * d->N * d->H_q * (d->topk + 1) < 2147483647.0;
+}
 size_t ws_attn(const msa_dims* d) {
     return kStatusBytes + attn_ws_bytes(d->B, d->N, d->H_q, d->H_kv, d->d, d->block_k, d->topk);
 }
@@ -114,7 +118,10 @@ msa_status msa_workspace_size(int op, const msa_dims* d, size_t* bytes) {
     switch (op) {
         case MSA_OP_INDEX_TOPK: *bytes = kStatusBytes; return MSA_OK;
         case MSA_OP_INDEX_TOPK_LSE: *bytes = ws_index_lse(d); return MSA_OK;
-        case MSA_OP_ATTN_FWD: *bytes = ws_attn(d); return MSA_OK;
+        case MSA_OP_ATTN_FWD:
+            if (!attn_rows_fit(d)) return MSA_ERR_UNSUPPORTED;
+            *bytes = ws_attn(d);
+            return MSA_OK;
         case MSA_OP_DECODE: *bytes = ws_decode(d); return MSA_OK;
         case MSA_OP_KL: *bytes = ws_kl(d); return MSA_OK;
     }
@@ -157,6 +164,7 @@ msa_status msa_sparse_attn_fwd(const msa_dims* d, const void* q, const void* k, 
                                void* out, float* lse, void* ws, size_t ws_bytes, msa_stream_t stream_) {
     msa_status s = check_common(d);
     if (s != MSA_OK) return s;
+    if (!attn_rows_fit(d)) return MSA_ERR_UNSUPPORTED;
     if (!q || !k || !v || !blocks || !out || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(blocks) ||
         !aligned16(out) || (lse && !aligned16(lse)))
         return MSA_ERR_INVALID_ARG;

@@ -67,14 +67,13 @@ cudaError_t run_csr_build(const Csr& c, const int32_t* blocks, int B, int N, int
 cudaError_t run_csr_items(const Csr& c, int qpc, cudaStream_t stream);
 
 // ---------------------------------------------------------------- sparse attention (msa_attn.cu)
-constexpr int kAttnWindow = 128;  // queries per window of the attention's inverse lists
+constexpr int kAttnWindow = 1024;  // queries per window of the attention's inverse lists
 struct AttnArgs {
     int B, N, H_q, H_kv, d, block_k, topk;
     float scale;
     Csr csr;             // windowed lists, items of 128/G queries
     __half* o_part;      // [B, N, H_q, topk+1, d]   normalised partial outputs
     float* lse_part;     // [B, N, H_q, topk+1]
-    int32_t* counter;    // [B, N, H_kv]  items finished per selection row
     int32_t* sched;      // [1]           next item to hand out
     const int32_t* blocks;
     __nv_bfloat16* out;  // [B, N, H_q, d]

@@ -29,8 +29,8 @@
  *
  * Supported sizes (MSA_ERR_UNSUPPORTED otherwise): d in {64, 128}, d_idx in {32, 64},
  * block_k in {32, 64, 128}, 1 <= topk <= 16, H_q % H_kv == 0 with G = H_q/H_kv in {1,2,4,8,16,32},
- * H_kv in {1,2,4,8}, N >= 1, B >= 1, N < 2^24 and B*N*H_kv*(topk+1) < 2^30. The attention keeps
- * its per-slot partial outputs in fp16: entries of V must stay below 65504 in magnitude (larger
+ * H_kv in {1,2,4,8}, N >= 1, B >= 1, N < 2^24 and B*N*H_kv*(topk+1) < 2^30; msa_sparse_attn_fwd
+ * also needs B*N*H_q*(topk+1) < 2^31. The attention keeps its per-slot partial outputs in fp16: entries of V must stay below 65504 in magnitude (larger
  * values are reported as MSA_ERR_DEVICE_CHECK). msa_kl_fwd_grad supports (d, d_idx) in
  * {(128, 64), (64, 32)} with G in {2, 16}.
  */
