@@ -115,251 +115,251 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = s.tmem_base;
 
     if (warp == kProdWarp) {
-    // ------------------------------------------------------------ items, metadata, Q and K
-    // The record and query list of the next item are loaded one item ahead, so their global
-    // latency overlaps the waits of the current item.
-    int prevL = -1, kgroup = -1;
-    bool ok = true;
-    int batch = 0;
-    if (lane == 0) batch = atomicAdd(a.sched, kGrab);
-    batch = __shfl_sync(0xffffffffu, batch, 0);
-    int t_nx = batch;
-    int4 rec_nx = t_nx < T ? a.csr.items[t_nx] : make_int4(-1, 0, 0, 0);
-    int e_nx[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const int m = lane + 32 * j;
-        e_nx[j] = (t_nx < T && m < rec_nx.z) ? a.csr.entries[rec_nx.y + m] : 0;
-    }
-    for (int n = 0;; ++n) {
-        const int t = t_nx;
-        const int4 rec = rec_nx;
-        int e[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) e[j] = e_nx[j];
-        // prefetch item n+1
-        if ((n + 1) % kGrab == 0) {
-            int b2 = 0;
-            if (lane == 0) b2 = atomicAdd(a.sched, kGrab);
-            batch = __shfl_sync(0xffffffffu, b2, 0);
-            t_nx = batch;
-        } else {
-            t_nx = batch + (n + 1) % kGrab;
-        }
-        if (t_nx < T) {
-            rec_nx = a.csr.items[t_nx];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int m = lane + 32 * j;
-                e_nx[j] = m < rec_nx.z ? a.csr.entries[rec_nx.y + m] : 0;
-            }
-        }
-        const int slot = n % kMeta;
-        if (!wait_lane0(&s.meta_empty[slot], ((n / kMeta) & 1) ^ 1, a.status, 0x501)) { ok = false; break; }
-        ItemMeta& mt = s.meta[slot];
-        if (t >= T || s.abort) {  // end marker
-            if (lane == 0) { mt.t = -1; mbar_arrive(&s.meta_full[slot]); }
-            break;
-        }
-        const int L = rec.x, count = rec.z;
-        const int c = L % a.csr.nb;
-        const int r = (L / a.csr.nb) % a.H_kv;
-        const int b = L / (a.csr.nb * a.H_kv * a.csr.nW);
+        // ------------------------------------------------------------ items, metadata, Q and K
+        // The record and query list of the next item are loaded one item ahead, so their global
+        // latency overlaps the waits of the current item.
+        int prevL = -1, kgroup = -1;
+        bool ok = true;
+        int batch = 0;
+        if (lane == 0) batch = atomicAdd(a.sched, kGrab);
+        batch = __shfl_sync(0xffffffffu, batch, 0);
+        int t_nx = batch;
+        int4 rec_nx = t_nx < T ? a.csr.items[t_nx] : make_int4(-1, 0, 0, 0);
+        int e_nx[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int m = lane + 32 * j;
-            if (m < count) {
-                mt.qi[m] = e[j] >> 5;
-                mt.qs[m] = (int8_t)(e[j] & 31);
-            }
+            e_nx[j] = (t_nx < T && m < rec_nx.z) ? a.csr.entries[rec_nx.y + m] : 0;
         }
-        if (lane == 0) {
-            mt.t = t; mt.b = b; mt.r = r; mt.c = c; mt.count = count; mt.kv_new = (L != prevL);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s.meta_full[slot]);
-        // Q: the G head rows of each query of the item
-        const int buf = n & 1;
-        if (!wait_lane0(&s.q_empty[buf], ((n >> 1) & 1) ^ 1, a.status, 0x503)) { ok = false; break; }
-        if (G >= 8) {
-            if (lane == 0) mbar_arrive_expect_tx(&s.q_full[buf], (uint32_t)(count * G * D * 2));
-            __syncwarp();
-            for (int m = lane; m < count; m += 32) {
+        for (int n = 0;; ++n) {
+            const int t = t_nx;
+            const int4 rec = rec_nx;
+            int e[4];
 #pragma unroll
-                for (int sub = 0; sub < D / 64; ++sub)
-                    tma_load_4d(s.q[buf] + sub * (kRows * 128) + m * G * 128, &tm_q, &s.q_full[buf], sub * 64,
-                                r * G, mt.qi[m], b);
-            }
-        } else {
-            const uint32_t qsm = smem_u32(s.q[buf]);
-            constexpr int kChunksPerRow = D * 2 / 16;
-            for (int x = lane; x < count * G * kChunksPerRow; x += 32) {
-                const int row = x / kChunksPerRow, ch = x % kChunksPerRow;
-                const int m = row / G, h = row % G;
-                const __nv_bfloat16* src =
-                    q + ((((size_t)b * a.N + mt.qi[m]) * a.H_q + (size_t)r * G + h) * D + ch * 8);
-                cp_async_16(qsm + ((ch * 16) / 128) * (kRows * 128) + swz(row, (ch * 16) % 128, 128), src);
-            }
-            cp_async_wait_all();
-            fence_proxy_async();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s.q_full[buf]);
-        }
-        // K of block group g goes to buffer g % 2 once the S MMAs of group g-2 (the buffer's
-        // previous use, release number (g-2)/2 of that buffer) are done
-        if (L != prevL) {
-            ++kgroup;
-            if (kgroup >= 2 &&
-                !wait_lane0(&s.k_release[kgroup & 1], ((kgroup - 2) >> 1) & 1, a.status, 0x504)) { ok = false; break; }
-            if (lane == 0) {
-                const int kb = kgroup & 1;
-                mbar_arrive_expect_tx(&s.k_full[kb], (uint32_t)Sm::kKVBytes);
-#pragma unroll
-                for (int sub = 0; sub < D / 64; ++sub)
-                    tma_load_4d(s.k[kb] + sub * BK * 128, &tm_k, &s.k_full[kb], sub * 64, r, c * BK, b);
-            }
-            prevL = L;
-        }
-    }
-    if (!ok) s.abort = 1;
-    if (lane == 0) {  // no copy of ours may still be landing when the CTA leaves
-        for (int g = max(0, kgroup - 1); g <= kgroup; ++g) mbar_wait(&s.k_full[g & 1], (g >> 1) & 1, a.status, 0x505);
-    }
-    } else if (warp == kVWarp) {
-    // ------------------------------------------------------------ V loader
-    int vgroup = -1;
-    bool ok = true;
-    for (int n = 0;; ++n) {
-        const int slot = n % kMeta;
-        if (!wait_lane0(&s.meta_full[slot], (n / kMeta) & 1, a.status, 0x511)) { ok = false; break; }
-        const ItemMeta& mt = s.meta[slot];
-        const int t = mt.t, b = mt.b, r = mt.r, c = mt.c, kv_new = mt.kv_new;
-        __syncwarp();
-        if (lane == 0 && t >= 0) mbar_arrive(&s.meta_empty[slot]);
-        if (t < 0) break;
-        if (kv_new) {
-            // V of block group g goes to buffer g % 2 once the PV MMAs of group g-2 are done
-            ++vgroup;
-            if (vgroup >= 2 &&
-                !wait_lane0(&s.v_release[vgroup & 1], ((vgroup - 2) >> 1) & 1, a.status, 0x512)) { ok = false; break; }
-            if (lane == 0) {
-                const int vb = vgroup & 1;
-                mbar_arrive_expect_tx(&s.v_full[vb], (uint32_t)Sm::kKVBytes);
-#pragma unroll
-                for (int sub = 0; sub < D / 64; ++sub)
-                    tma_load_4d(s.v[vb] + sub * BK * 128, &tm_v, &s.v_full[vb], sub * 64, r, c * BK, b);
-            }
-        }
-    }
-    if (!ok) s.abort = 1;
-    if (lane == 0) {
-        for (int g = max(0, vgroup - 1); g <= vgroup; ++g) mbar_wait(&s.v_full[g & 1], (g >> 1) & 1, a.status, 0x513);
-    }
-    } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
-    // S(ns) needs its metadata, Q, its K buffer, and PV(ns-2) issued (P(ns-2) lives in the TMEM
-    // columns S(ns) overwrites; MMAs of one thread execute in issue order). PV(np) needs P(np),
-    // its V buffer and the O accumulator freed by the epilogue. Both are polled; whichever is
-    // ready goes first.
-    if (lane == 0) {
-        bool ok = true;
-        int ns = 0, np = 0, n_end = -1;
-        bool meta_read = false;
-        int cur_kvn = 0, cur_grp = -1;
-        int groups = -1;          // block groups seen so far (metadata order)
-        int pend_pv = -1;         // PV issued whose item's successor group was not yet known
-        int grp_ring[kMeta] = {0, 0, 0, 0};
-        uint64_t t_idle = globaltimer();
-        while (true) {
-            bool progressed = false;
-            if (n_end < 0) {
-                if (!meta_read && mbar_test(&s.meta_full[ns % kMeta], (ns / kMeta) & 1)) {
-                    const int t = s.meta[ns % kMeta].t;
-                    cur_kvn = s.meta[ns % kMeta].kv_new;
-                    if (t < 0) {
-                        n_end = ns;
-                    } else {
-                        mbar_arrive(&s.meta_empty[ns % kMeta]);
-                        meta_read = true;
-                        if (cur_kvn) {
-                            ++groups;
-                            if (ns > 0) {
-                                // item ns-1 closed block group groups-1: every S of it has been
-                                // issued, so its K buffer is free once they complete
-                                umma_commit(&s.k_release[(groups - 1) & 1]);
-                            }
-                        }
-                        cur_grp = groups;
-                        // a PV waiting to learn whether it closed its group
-                        if (pend_pv >= 0 && pend_pv == ns - 1) {
-                            if (cur_kvn) umma_commit(&s.v_release[grp_ring[pend_pv % kMeta] & 1]);
-                            pend_pv = -1;
-                        }
-                    }
-                    progressed = true;
-                }
-                if (meta_read && np >= ns - 1 && mbar_test(&s.q_full[ns & 1], (ns >> 1) & 1) &&
-                    mbar_test(&s.k_full[cur_grp & 1], (cur_grp >> 1) & 1)) {
-                    tc_fence_after();
-                    const uint32_t qb = smem_u32(s.q[ns & 1]), kb = smem_u32(s.k[cur_grp & 1]);
-                    const uint32_t tS = tmem + (ns & 1) * 256;
-#pragma unroll
-                    for (int ks = 0; ks < D / 16; ++ks) {
-                        const uint32_t sub = (ks * 16) / 64, off = (ks & 3) * 32;
-                        const uint64_t da = umma_sdesc(qb + sub * (kRows * 128) + off, 16, 1024, 2);
-                        const uint64_t db = umma_sdesc(kb + sub * (BK * 128) + off, 16, 1024, 2);
-                        umma_bf16(tS, da, db, kIdescS, ks > 0);
-                    }
-                    umma_commit(&s.s_full[ns & 1]);
-                    umma_commit(&s.q_empty[ns & 1]);
-                    grp_ring[ns % kMeta] = cur_grp;
-                    ++ns;
-                    meta_read = false;
-                    progressed = true;
-                }
-            }
-            if (np < ns && mbar_test(&s.p_full[np & 1], (np >> 1) & 1) &&
-                mbar_test(&s.o_free[np & 1], ((np >> 1) & 1) ^ 1)) {
-                const int g = grp_ring[np % kMeta];
-                if (mbar_test(&s.v_full[g & 1], (g >> 1) & 1)) {
-                    tc_fence_after();
-                    const uint32_t vb = smem_u32(s.v[g & 1]);
-                    const uint32_t tP = tmem + (np & 1) * 256;        // P (bf16 pairs) over S
-                    const uint32_t tO = tmem + (np & 1) * 256 + 128;
-#pragma unroll
-                    for (int ks = 0; ks < BK / 16; ++ks) {
-                        const uint64_t db = umma_sdesc(vb + ks * 16 * 128, BK * 128, 1024, 2);
-                        umma_bf16_tmem_a(tO, tP + ks * 8, db, kIdescO, ks > 0);
-                    }
-                    umma_commit(&s.o_full[np & 1]);
-                    // if item np closed its block group, its V buffer is free once this PV is done
-                    if (np + 1 < ns) {
-                        if (grp_ring[(np + 1) % kMeta] != g) umma_commit(&s.v_release[g & 1]);
-                    } else if (np + 1 == ns && meta_read) {
-                        if (cur_grp != g) umma_commit(&s.v_release[g & 1]);
-                    } else {
-                        pend_pv = np;
-                    }
-                    ++np;
-                    progressed = true;
-                }
-            }
-            if (n_end >= 0 && np == n_end) break;
-            if (progressed) {
-                t_idle = globaltimer();
+            for (int j = 0; j < 4; ++j) e[j] = e_nx[j];
+            // prefetch item n+1
+            if ((n + 1) % kGrab == 0) {
+                int b2 = 0;
+                if (lane == 0) b2 = atomicAdd(a.sched, kGrab);
+                batch = __shfl_sync(0xffffffffu, b2, 0);
+                t_nx = batch;
             } else {
-                __nanosleep(20);
+                t_nx = batch + (n + 1) % kGrab;
             }
-            if (!progressed && globaltimer() - t_idle > MSA_WAIT_NS) {
-                raise_flag(a.status, MSA_DEV_TIMEOUT, 0x601);
-                ok = false;
+            if (t_nx < T) {
+                rec_nx = a.csr.items[t_nx];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int m = lane + 32 * j;
+                    e_nx[j] = m < rec_nx.z ? a.csr.entries[rec_nx.y + m] : 0;
+                }
+            }
+            const int slot = n % kMeta;
+            if (!wait_lane0(&s.meta_empty[slot], ((n / kMeta) & 1) ^ 1, a.status, 0x501)) { ok = false; break; }
+            ItemMeta& mt = s.meta[slot];
+            if (t >= T || s.abort) {  // end marker
+                if (lane == 0) { mt.t = -1; mbar_arrive(&s.meta_full[slot]); }
                 break;
+            }
+            const int L = rec.x, count = rec.z;
+            const int c = L % a.csr.nb;
+            const int r = (L / a.csr.nb) % a.H_kv;
+            const int b = L / (a.csr.nb * a.H_kv * a.csr.nW);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int m = lane + 32 * j;
+                if (m < count) {
+                    mt.qi[m] = e[j] >> 5;
+                    mt.qs[m] = (int8_t)(e[j] & 31);
+                }
+            }
+            if (lane == 0) {
+                mt.t = t; mt.b = b; mt.r = r; mt.c = c; mt.count = count; mt.kv_new = (L != prevL);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.meta_full[slot]);
+            // Q: the G head rows of each query of the item
+            const int buf = n & 1;
+            if (!wait_lane0(&s.q_empty[buf], ((n >> 1) & 1) ^ 1, a.status, 0x503)) { ok = false; break; }
+            if (G >= 8) {
+                if (lane == 0) mbar_arrive_expect_tx(&s.q_full[buf], (uint32_t)(count * G * D * 2));
+                __syncwarp();
+                for (int m = lane; m < count; m += 32) {
+#pragma unroll
+                    for (int sub = 0; sub < D / 64; ++sub)
+                        tma_load_4d(s.q[buf] + sub * (kRows * 128) + m * G * 128, &tm_q, &s.q_full[buf], sub * 64,
+                                    r * G, mt.qi[m], b);
+                }
+            } else {
+                const uint32_t qsm = smem_u32(s.q[buf]);
+                constexpr int kChunksPerRow = D * 2 / 16;
+                for (int x = lane; x < count * G * kChunksPerRow; x += 32) {
+                    const int row = x / kChunksPerRow, ch = x % kChunksPerRow;
+                    const int m = row / G, h = row % G;
+                    const __nv_bfloat16* src =
+                        q + ((((size_t)b * a.N + mt.qi[m]) * a.H_q + (size_t)r * G + h) * D + ch * 8);
+                    cp_async_16(qsm + ((ch * 16) / 128) * (kRows * 128) + swz(row, (ch * 16) % 128, 128), src);
+                }
+                cp_async_wait_all();
+                fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s.q_full[buf]);
+            }
+            // K of block group g goes to buffer g % 2 once the S MMAs of group g-2 (the buffer's
+            // previous use, release number (g-2)/2 of that buffer) are done
+            if (L != prevL) {
+                ++kgroup;
+                if (kgroup >= 2 &&
+                    !wait_lane0(&s.k_release[kgroup & 1], ((kgroup - 2) >> 1) & 1, a.status, 0x504)) { ok = false; break; }
+                if (lane == 0) {
+                    const int kb = kgroup & 1;
+                    mbar_arrive_expect_tx(&s.k_full[kb], (uint32_t)Sm::kKVBytes);
+#pragma unroll
+                    for (int sub = 0; sub < D / 64; ++sub)
+                        tma_load_4d(s.k[kb] + sub * BK * 128, &tm_k, &s.k_full[kb], sub * 64, r, c * BK, b);
+                }
+                prevL = L;
             }
         }
         if (!ok) s.abort = 1;
-        umma_commit(&s.drain);
-        mbar_wait(&s.drain, 0, a.status, 0x608);
-    }
+        if (lane == 0) {  // no copy of ours may still be landing when the CTA leaves
+            for (int g = max(0, kgroup - 1); g <= kgroup; ++g) mbar_wait(&s.k_full[g & 1], (g >> 1) & 1, a.status, 0x505);
+        }
+    } else if (warp == kVWarp) {
+        // ------------------------------------------------------------ V loader
+        int vgroup = -1;
+        bool ok = true;
+        for (int n = 0;; ++n) {
+            const int slot = n % kMeta;
+            if (!wait_lane0(&s.meta_full[slot], (n / kMeta) & 1, a.status, 0x511)) { ok = false; break; }
+            const ItemMeta& mt = s.meta[slot];
+            const int t = mt.t, b = mt.b, r = mt.r, c = mt.c, kv_new = mt.kv_new;
+            __syncwarp();
+            if (lane == 0 && t >= 0) mbar_arrive(&s.meta_empty[slot]);
+            if (t < 0) break;
+            if (kv_new) {
+                // V of block group g goes to buffer g % 2 once the PV MMAs of group g-2 are done
+                ++vgroup;
+                if (vgroup >= 2 &&
+                    !wait_lane0(&s.v_release[vgroup & 1], ((vgroup - 2) >> 1) & 1, a.status, 0x512)) { ok = false; break; }
+                if (lane == 0) {
+                    const int vb = vgroup & 1;
+                    mbar_arrive_expect_tx(&s.v_full[vb], (uint32_t)Sm::kKVBytes);
+#pragma unroll
+                    for (int sub = 0; sub < D / 64; ++sub)
+                        tma_load_4d(s.v[vb] + sub * BK * 128, &tm_v, &s.v_full[vb], sub * 64, r, c * BK, b);
+                }
+            }
+        }
+        if (!ok) s.abort = 1;
+        if (lane == 0) {
+            for (int g = max(0, vgroup - 1); g <= vgroup; ++g) mbar_wait(&s.v_full[g & 1], (g >> 1) & 1, a.status, 0x513);
+        }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        // S(ns) needs its metadata, Q, its K buffer, and PV(ns-2) issued (P(ns-2) lives in the TMEM
+        // columns S(ns) overwrites; MMAs of one thread execute in issue order). PV(np) needs P(np),
+        // its V buffer and the O accumulator freed by the epilogue. Both are polled; whichever is
+        // ready goes first.
+        if (lane == 0) {
+            bool ok = true;
+            int ns = 0, np = 0, n_end = -1;
+            bool meta_read = false;
+            int cur_kvn = 0, cur_grp = -1;
+            int groups = -1;          // block groups seen so far (metadata order)
+            int pend_pv = -1;         // PV issued whose item's successor group was not yet known
+            int grp_ring[kMeta] = {0, 0, 0, 0};
+            uint64_t t_idle = globaltimer();
+            while (true) {
+                bool progressed = false;
+                if (n_end < 0) {
+                    if (!meta_read && mbar_test(&s.meta_full[ns % kMeta], (ns / kMeta) & 1)) {
+                        const int t = s.meta[ns % kMeta].t;
+                        cur_kvn = s.meta[ns % kMeta].kv_new;
+                        if (t < 0) {
+                            n_end = ns;
+                        } else {
+                            mbar_arrive(&s.meta_empty[ns % kMeta]);
+                            meta_read = true;
+                            if (cur_kvn) {
+                                ++groups;
+                                if (ns > 0) {
+                                    // item ns-1 closed block group groups-1: every S of it has been
+                                    // issued, so its K buffer is free once they complete
+                                    umma_commit(&s.k_release[(groups - 1) & 1]);
+                                }
+                            }
+                            cur_grp = groups;
+                            // a PV waiting to learn whether it closed its group
+                            if (pend_pv >= 0 && pend_pv == ns - 1) {
+                                if (cur_kvn) umma_commit(&s.v_release[grp_ring[pend_pv % kMeta] & 1]);
+                                pend_pv = -1;
+                            }
+                        }
+                        progressed = true;
+                    }
+                    if (meta_read && np >= ns - 1 && mbar_test(&s.q_full[ns & 1], (ns >> 1) & 1) &&
+                        mbar_test(&s.k_full[cur_grp & 1], (cur_grp >> 1) & 1)) {
+                        tc_fence_after();
+                        const uint32_t qb = smem_u32(s.q[ns & 1]), kb = smem_u32(s.k[cur_grp & 1]);
+                        const uint32_t tS = tmem + (ns & 1) * 256;
+#pragma unroll
+                        for (int ks = 0; ks < D / 16; ++ks) {
+                            const uint32_t sub = (ks * 16) / 64, off = (ks & 3) * 32;
+                            const uint64_t da = umma_sdesc(qb + sub * (kRows * 128) + off, 16, 1024, 2);
+                            const uint64_t db = umma_sdesc(kb + sub * (BK * 128) + off, 16, 1024, 2);
+                            umma_bf16(tS, da, db, kIdescS, ks > 0);
+                        }
+                        umma_commit(&s.s_full[ns & 1]);
+                        umma_commit(&s.q_empty[ns & 1]);
+                        grp_ring[ns % kMeta] = cur_grp;
+                        ++ns;
+                        meta_read = false;
+                        progressed = true;
+                    }
+                }
+                if (np < ns && mbar_test(&s.p_full[np & 1], (np >> 1) & 1) &&
+                    mbar_test(&s.o_free[np & 1], ((np >> 1) & 1) ^ 1)) {
+                    const int g = grp_ring[np % kMeta];
+                    if (mbar_test(&s.v_full[g & 1], (g >> 1) & 1)) {
+                        tc_fence_after();
+                        const uint32_t vb = smem_u32(s.v[g & 1]);
+                        const uint32_t tP = tmem + (np & 1) * 256;        // P (bf16 pairs) over S
+                        const uint32_t tO = tmem + (np & 1) * 256 + 128;
+#pragma unroll
+                        for (int ks = 0; ks < BK / 16; ++ks) {
+                            const uint64_t db = umma_sdesc(vb + ks * 16 * 128, BK * 128, 1024, 2);
+                            umma_bf16_tmem_a(tO, tP + ks * 8, db, kIdescO, ks > 0);
+                        }
+                        umma_commit(&s.o_full[np & 1]);
+                        // if item np closed its block group, its V buffer is free once this PV is done
+                        if (np + 1 < ns) {
+                            if (grp_ring[(np + 1) % kMeta] != g) umma_commit(&s.v_release[g & 1]);
+                        } else if (np + 1 == ns && meta_read) {
+                            if (cur_grp != g) umma_commit(&s.v_release[g & 1]);
+                        } else {
+                            pend_pv = np;
+                        }
+                        ++np;
+                        progressed = true;
+                    }
+                }
+                if (n_end >= 0 && np == n_end) break;
+                if (progressed) {
+                    t_idle = globaltimer();
+                } else {
+                    __nanosleep(20);
+                }
+                if (!progressed && globaltimer() - t_idle > MSA_WAIT_NS) {
+                    raise_flag(a.status, MSA_DEV_TIMEOUT, 0x601);
+                    ok = false;
+                    break;
+                }
+            }
+            if (!ok) s.abort = 1;
+            umma_commit(&s.drain);
+            mbar_wait(&s.drain, 0, a.status, 0x608);
+        }
     } else if (warp < kEpiWarps) {
         // ------------------------------------------------------------ softmax / epilogue
         // All 16 epilogue warps work on every item: warp w reads TMEM lane quarter w % 4 (tile rows
@@ -375,8 +375,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_addr = tmem + ((uint32_t)(qtr * 32) << 16);
         const uint32_t bar_id = 1 + qtr;
         const float sl2 = a.scale * 1.4426950408889634f;
-        // the item whose O is read out next: the row's partial index (b, i, head, slot) or -1 and
-        // its max (partial indices fit 31 bits, checked by the host)
+        // the item whose O is read out next: the row's partial index ((b, i, r, slot), head) or -1
+        // and its max (partial indices fit 31 bits, checked by the host)
         bool have_prev = false;
         int pv_prow = -1;
         float pv_mx = 0.f;
@@ -398,9 +398,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __half2 hh2 = __floats2half2_rn(__uint_as_float(ov[x]) * inv, __uint_as_float(ov[x + 1]) * inv);
                     hv[x / 2] = *reinterpret_cast<const uint32_t*>(&hh2);
                 }
-                uint4* dst = reinterpret_cast<uint4*>(a.o_part + (size_t)pv_prow * D + e * OC);
+                // chunk x of 8 values goes to [(b, i, r, slot)][x][head]: the G heads of a query
+                // are adjacent, so a warp's store covers whole 128-byte lines
+                uint4* dst = reinterpret_cast<uint4*>(a.o_part) + (size_t)(pv_prow - h) * (D / 8) + h;
 #pragma unroll
-                for (int x = 0; x < OC / 8; ++x) dst[x] = make_uint4(hv[4 * x], hv[4 * x + 1], hv[4 * x + 2], hv[4 * x + 3]);
+                for (int x = 0; x < OC / 8; ++x)
+                    dst[(size_t)(e * (OC / 8) + x) * G] = make_uint4(hv[4 * x], hv[4 * x + 1], hv[4 * x + 2], hv[4 * x + 3]);
                 if (e == 0) {
                     const float l = (s.red_l[pb][0][row] + s.red_l[pb][1][row]) + (s.red_l[pb][2][row] + s.red_l[pb][3][row]);
                     a.lse_part[pv_prow] = pv_mx * a.scale + logf(l);
@@ -500,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(&s.p_full[n & 1]);
             if (have_prev && !store_prev(n - 1)) fail = true;
             have_prev = true;
-            pv_prow = valid ? ((b * a.N + i) * a.H_q + r * G + h) * K1 + qslot : -1;
+            pv_prow = valid ? (((b * a.N + i) * a.H_kv + r) * K1 + qslot) * G + h : -1;
             pv_mx = mx;
         }
     }
@@ -512,7 +515,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Combines each (query, group) row's partials: out = sum_s exp(lse_s - LSE) o_s with
 // LSE = log sum_s exp(lse_s) (the partition merge), over the row's valid slots. One warp per row;
-// lanes take units of 8 output values of one head and keep every slot's load in flight at once.
+// lanes take units of 8 output values of one head (head fastest, matching the partial layout
+// [(b, i, r, slot)][d/8][head][8]) and keep every slot's load in flight at once.
 template <int D, int BK>
 __global__ void __launch_bounds__(256) k_attn_merge(AttnArgs a) {
     const int G = a.H_q / a.H_kv;
@@ -539,16 +543,16 @@ __global__ void __launch_bounds__(256) k_attn_merge(AttnArgs a) {
         if (lane == 0) prev = -1;
         const uint32_t vmask = __ballot_sync(0xffffffffu, inr && cb > prev);
         for (int u = lane; u < units; u += 32) {
-            const int hh = u / (D / 8), d0 = (u % (D / 8)) * 8;
+            const int hh = u % G, ch = u / G, d0 = ch * 8;
             const int hq = r * G + hh;
-            const size_t rb = (((size_t)b * a.N + i) * a.H_q + hq) * K1;
+            const size_t rb = (size_t)row * K1;  // first slot of the row
             float lv[kK1Max];
             uint4 ov[kK1Max];
 #pragma unroll
             for (int x = 0; x < kK1Max; ++x) {
                 if (vmask & (1u << x)) {
-                    lv[x] = __ldcs(a.lse_part + rb + x);
-                    ov[x] = __ldcs(reinterpret_cast<const uint4*>(a.o_part + (rb + x) * D + d0));
+                    lv[x] = __ldcs(a.lse_part + (rb + x) * G + hh);
+                    ov[x] = __ldcs(reinterpret_cast<const uint4*>(a.o_part) + ((rb + x) * (D / 8) + ch) * G + hh);
                 } else {
                     lv[x] = -INFINITY;
                     ov[x] = make_uint4(0, 0, 0, 0);

@@ -72,8 +72,8 @@ struct AttnArgs {
     int B, N, H_q, H_kv, d, block_k, topk;
     float scale;
     Csr csr;             // windowed lists, items of 128/G queries
-    __half* o_part;      // [B, N, H_q, topk+1, d]   normalised partial outputs
-    float* lse_part;     // [B, N, H_q, topk+1]
+    __half* o_part;      // [B, N, H_kv, topk+1, d/8, G, 8]   normalised partial outputs
+    float* lse_part;     // [B, N, H_kv, topk+1, G]
     int32_t* sched;      // [1]           next item to hand out
     const int32_t* blocks;
     __nv_bfloat16* out;  // [B, N, H_q, d]
