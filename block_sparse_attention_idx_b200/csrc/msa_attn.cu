@@ -57,6 +57,7 @@ struct AttnSmem {
     uint64_t q_full[2], q_empty[2];
     uint64_t k_full[2], k_release[2], v_full[2], v_release[2];  // release[b]: one completion per use of buffer b
     uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
+    uint64_t max_bar[2], sum_bar[2];  // every epilogue warp's row max / row sums of item n are in
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -98,6 +99,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&s.p_full[x], kEpiWarps);
             mbar_init(&s.o_full[x], 1);
             mbar_init(&s.o_free[x], kEpiWarps);
+            mbar_init(&s.max_bar[x], kEpiWarps);
+            mbar_init(&s.sum_bar[x], kEpiWarps);
             mbar_init(&s.k_release[x], 1);
             mbar_init(&s.v_release[x], 1);
         }
@@ -364,16 +367,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ softmax / epilogue
         // All 16 epilogue warps work on every item: warp w reads TMEM lane quarter w % 4 (tile rows
         // 32(w%4) .. +31) and column quarter e = w / 4 of S (BK/4 tokens) and of O (D/4 values). Row
-        // max and row sums are combined across the column quarters through shared memory under one
-        // named barrier per lane quarter and item; that barrier also carries the stop decision, so the
-        // four warps of a lane quarter always leave together. The O of item n-1 is read out after the
-        // softmax of item n, while the PV product of item n runs.
+        // max and row sums are combined across the column quarters through shared memory, published
+        // by the max_bar / sum_bar mbarriers. The O of item n-1 is read out while item n is in its
+        // softmax, and the PV product of item n runs after it.
         constexpr int SC = BK / 4, OC = D / 4;
         const int qtr = warp & 3, e = warp >> 2;
         const int row = qtr * 32 + lane;
         const int m = row / G, h = row % G;
         const uint32_t lane_addr = tmem + ((uint32_t)(qtr * 32) << 16);
-        const uint32_t bar_id = 1 + qtr;
         const float sl2 = a.scale * 1.4426950408889634f;
         // the item whose O is read out next: the row's partial index ((b, i, r, slot), head) or -1
         // and its max (partial indices fit 31 bits, checked by the host)
@@ -384,6 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // LSE, free the accumulator
         auto store_prev = [&](int np) -> bool {
             if (!__all_sync(0xffffffffu, mbar_wait(&s.o_full[np & 1], (np >> 1) & 1, a.status, 0x704))) return false;
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.sum_bar[np & 1], (np >> 1) & 1, a.status, 0x705))) return false;
             tc_fence_after();
             uint32_t ov[OC];
             tmem_ld<OC>(lane_addr + (np & 1) * 256 + 128 + e * OC, ov);
@@ -414,62 +416,56 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(&s.o_free[np & 1]);
             return true;
         };
+        // Each warp: row max of its S quarter -> max_bar; softmax of this item -> sum_bar and
+        // p_full (so the PV product can start); then the O of the previous item. Every wait is
+        // bounded; a warp whose wait fails leaves, and the others run into their own bounded waits.
         bool fail = false;
-        for (int n = 0;; ++n) {
+        int n = 0;
+        for (;; ++n) {
             const int slot = n % kMeta;
-            bool ok = __all_sync(0xffffffffu, mbar_wait(&s.meta_full[slot], (n / kMeta) & 1, a.status, 0x701));
-            bool live = false, valid = false;
-            int b = 0, r = 0, c = 0, i = 0, qslot = 0;
-            if (ok) {
-                const ItemMeta& mt = s.meta[slot];
-                live = mt.t >= 0;
-                if (live) {
-                    b = mt.b;
-                    r = mt.r;
-                    c = mt.c;
-                    valid = m < mt.count;
-                    i = valid ? mt.qi[m] : 0;
-                    qslot = valid ? (int)mt.qs[m] : 0;
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&s.meta_empty[slot]);
-                }
-            }
-            const uint32_t tS = lane_addr + (n & 1) * 256;
-            const int lim = valid ? i - c * BK - e * SC : -1;  // this warp's columns x <= lim are causal
-            uint32_t sv[SC];
-            bool full = false;
-            if (live && ok) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&s.s_full[n & 1], (n >> 1) & 1, a.status, 0x702));
-                if (ok) {
-                    tc_fence_after();
-                    tmem_ld<SC>(tS + e * SC, sv);
-                    tmem_ld_wait();
-                    full = __all_sync(0xffffffffu, lim >= SC - 1);
-                    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-                    if (full) {
-#pragma unroll
-                        for (int x = 0; x < SC; ++x) m4[x & 3] = fmaxf(m4[x & 3], __uint_as_float(sv[x]));
-                    } else {
-#pragma unroll
-                        for (int x = 0; x < SC; ++x) m4[x & 3] = x <= lim ? fmaxf(m4[x & 3], __uint_as_float(sv[x])) : m4[x & 3];
-                    }
-                    s.red_max[n & 1][e][row] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-                }
-            }
-            const bool mine_failed = !ok || fail;
-            if (bar_red_or(bar_id, 128, mine_failed || !live)) {
-                // end of the item stream, or a failed wait somewhere in this lane quarter
-                if (bar_red_or(bar_id, 128, mine_failed)) {
-                    s.abort = 1;
-                } else if (have_prev) {
-                    store_prev(n - 1);
-                }
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.meta_full[slot], (n / kMeta) & 1, a.status, 0x701))) {
+                fail = true;
                 break;
             }
-            // P = exp(S - max) rounded to bf16, packed two per TMEM column over S (every S column of
-            // the tile has been read once all four quarters passed the barrier). l: exact sum for the
-            // LSE; lr: sum of the rounded weights the MMA uses, so that O / lr stays a convex
-            // combination of the V rows.
+            const ItemMeta& mt = s.meta[slot];
+            if (mt.t < 0) break;  // end of the item stream
+            const int b = mt.b, r = mt.r, c = mt.c;
+            const bool valid = m < mt.count;
+            const int i = valid ? mt.qi[m] : 0;
+            const int qslot = valid ? (int)mt.qs[m] : 0;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.meta_empty[slot]);
+            const uint32_t tS = lane_addr + (n & 1) * 256;
+            const int lim = valid ? i - c * BK - e * SC : -1;  // this warp's columns x <= lim are causal
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.s_full[n & 1], (n >> 1) & 1, a.status, 0x702))) {
+                fail = true;
+                break;
+            }
+            tc_fence_after();
+            uint32_t sv[SC];
+            tmem_ld<SC>(tS + e * SC, sv);
+            tmem_ld_wait();
+            const bool full = __all_sync(0xffffffffu, lim >= SC - 1);
+            {
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                if (full) {
+#pragma unroll
+                    for (int x = 0; x < SC; ++x) m4[x & 3] = fmaxf(m4[x & 3], __uint_as_float(sv[x]));
+                } else {
+#pragma unroll
+                    for (int x = 0; x < SC; ++x) m4[x & 3] = x <= lim ? fmaxf(m4[x & 3], __uint_as_float(sv[x])) : m4[x & 3];
+                }
+                s.red_max[n & 1][e][row] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.max_bar[n & 1]);
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.max_bar[n & 1], (n >> 1) & 1, a.status, 0x703))) {
+                fail = true;
+                break;
+            }
+            // P = exp(S - max) rounded to bf16, packed two per TMEM column over this warp's own S
+            // columns (already in registers). l: exact sum for the LSE; lr: sum of the rounded
+            // weights the MMA uses, so that O / lr stays a convex combination of the V rows.
             const float mx = fmaxf(fmaxf(s.red_max[n & 1][0][row], s.red_max[n & 1][1][row]),
                                    fmaxf(s.red_max[n & 1][2][row], s.red_max[n & 1][3][row]));
             const float moff = valid ? mx * sl2 : 0.f;
@@ -500,11 +496,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             s.red_l[n & 1][e][row] = l0 + l1;
             s.red_lr[n & 1][e][row] = lr0 + lr1;
             __syncwarp();
-            if (lane == 0) mbar_arrive(&s.p_full[n & 1]);
-            if (have_prev && !store_prev(n - 1)) fail = true;
+            if (lane == 0) {
+                mbar_arrive(&s.sum_bar[n & 1]);
+                mbar_arrive(&s.p_full[n & 1]);
+            }
+            if (have_prev && !store_prev(n - 1)) {
+                fail = true;
+                break;
+            }
             have_prev = true;
             pv_prow = valid ? (((b * a.N + i) * a.H_kv + r) * K1 + qslot) * G + h : -1;
             pv_mx = mx;
+        }
+        if (fail) {
+            s.abort = 1;
+        } else if (have_prev) {
+            store_prev(n - 1);
         }
     }
     tc_fence_before();
