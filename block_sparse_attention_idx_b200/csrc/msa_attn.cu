@@ -30,7 +30,8 @@ namespace {
 constexpr int kRows = 128;
 constexpr int kMeta = 4;        // depth of the item metadata ring
 constexpr int kGrab = 4;        // items taken per scheduler fetch
-constexpr int kEpiWarps = 16;   // warps 0..15: softmax / epilogue
+constexpr int kEpiWarps = 16;   // warps 0..15: softmax / epilogue, two teams of 8
+constexpr int kTeamWarps = 8;
 constexpr int kProdWarp = 16;   // items, metadata, Q and K
 constexpr int kVWarp = 17;      // V
 constexpr int kMmaWarp = 18;    // MMA issue, TMEM owner
@@ -51,13 +52,15 @@ struct AttnSmem {
     alignas(1024) uint8_t k[2][kKVBytes];
     alignas(1024) uint8_t v[2][kKVBytes];
     ItemMeta meta[kMeta];
-    // per-row partial max / sums of the four column quarters, by item parity
-    float red_max[2][4][kRows], red_l[2][4][kRows], red_lr[2][4][kRows];
+    // per-row partial max / sums of the two column halves: [team][team item parity][half][row]
+    float red_max[2][2][2][kRows], red_l[2][2][2][kRows], red_lr[2][2][2][kRows];
     uint64_t meta_full[kMeta], meta_empty[kMeta];
     uint64_t q_full[2], q_empty[2];
     uint64_t k_full[2], k_release[2], v_full[2], v_release[2];  // release[b]: one completion per use of buffer b
     uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
-    uint64_t max_bar[2], sum_bar[2];  // every epilogue warp's row max / row sums of item n are in
+    // a team's row maxima of its item are in (max_bar[team]); its row sums are in
+    // (sum_bar[team][team item parity]: read one item later, after the warp's own next arrival)
+    uint64_t max_bar[2], sum_bar[2][2];
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -79,6 +82,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     constexpr uint32_t kIdescS = umma_idesc_bf16(kRows, BK, false, false);
     constexpr uint32_t kIdescO = umma_idesc_bf16(kRows, D, false, true);
+    constexpr int kSC = BK / 2;  // S columns per epilogue warp
 
     const int G = a.H_q / a.H_kv;
     const int K1 = a.topk + 1;
@@ -88,7 +92,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int x = 0; x < kMeta; ++x) {
             mbar_init(&s.meta_full[x], 1);
-            mbar_init(&s.meta_empty[x], 2 + kEpiWarps);  // V loader, MMA issuer, each epilogue warp
+            mbar_init(&s.meta_empty[x], 2 + kTeamWarps);  // V loader, MMA issuer, the item's team
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(&s.q_full[x], 1);
@@ -96,11 +100,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&s.k_full[x], 1);
             mbar_init(&s.v_full[x], 1);
             mbar_init(&s.s_full[x], 1);
-            mbar_init(&s.p_full[x], kEpiWarps);
+            mbar_init(&s.p_full[x], kTeamWarps);
             mbar_init(&s.o_full[x], 1);
-            mbar_init(&s.o_free[x], kEpiWarps);
-            mbar_init(&s.max_bar[x], kEpiWarps);
-            mbar_init(&s.sum_bar[x], kEpiWarps);
+            mbar_init(&s.o_free[x], kTeamWarps);
+            mbar_init(&s.max_bar[x], kTeamWarps);
+            mbar_init(&s.sum_bar[x][0], kTeamWarps);
+            mbar_init(&s.sum_bar[x][1], kTeamWarps);
             mbar_init(&s.k_release[x], 1);
             mbar_init(&s.v_release[x], 1);
         }
@@ -160,8 +165,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int slot = n % kMeta;
             if (!wait_lane0(&s.meta_empty[slot], ((n / kMeta) & 1) ^ 1, a.status, 0x501)) { ok = false; break; }
             ItemMeta& mt = s.meta[slot];
-            if (t >= T || s.abort) {  // end marker
+            if (t >= T || s.abort) {
+                // two end markers: one for each epilogue team
                 if (lane == 0) { mt.t = -1; mbar_arrive(&s.meta_full[slot]); }
+                const int slot2 = (n + 1) % kMeta;
+                if (!wait_lane0(&s.meta_empty[slot2], (((n + 1) / kMeta) & 1) ^ 1, a.status, 0x502)) { ok = false; break; }
+                if (lane == 0) { s.meta[slot2].t = -1; mbar_arrive(&s.meta_full[slot2]); }
                 break;
             }
             const int L = rec.x, count = rec.z;
@@ -332,7 +341,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int ks = 0; ks < BK / 16; ++ks) {
                             const uint64_t db = umma_sdesc(vb + ks * 16 * 128, BK * 128, 1024, 2);
-                            umma_bf16_tmem_a(tO, tP + ks * 8, db, kIdescO, ks > 0);
+                            // P of S columns [16ks, 16ks+16) sits packed in the columns of the
+                            // epilogue warp that owns them (warp half e = 16ks / (BK/2))
+                            umma_bf16_tmem_a(tO, tP + (ks * 16 / kSC) * kSC + (ks * 16 % kSC) / 2, db, kIdescO, ks > 0);
                         }
                         umma_commit(&s.o_full[np & 1]);
                         // if item np closed its block group, its V buffer is free once this PV is done
@@ -365,63 +376,81 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp < kEpiWarps) {
         // ------------------------------------------------------------ softmax / epilogue
-        // All 16 epilogue warps work on every item: warp w reads TMEM lane quarter w % 4 (tile rows
-        // 32(w%4) .. +31) and column quarter e = w / 4 of S (BK/4 tokens) and of O (D/4 values). Row
-        // max and row sums are combined across the column quarters through shared memory, published
-        // by the max_bar / sum_bar mbarriers. The O of item n-1 is read out while item n is in its
-        // softmax, and the PV product of item n runs after it.
-        constexpr int SC = BK / 4, OC = D / 4;
-        const int qtr = warp & 3, e = warp >> 2;
+        // Two teams of 8 warps take alternate items (team t: items n with n % 2 == t, always in TMEM
+        // buffer t), so one team's exponentials overlap the other team's O read-out and waits.
+        // Within a team, warp w reads TMEM lane quarter w % 4 (tile rows 32(w%4) .. +31) and column
+        // half e of S (BK/2 tokens) and of O (D/2 values). Each team item starts by reading out the
+        // O of the team's previous item, which frees the team's single O accumulator for the PV
+        // product of the item that follows. The row max and row sums of the two halves
+        // meet in shared memory, published by the team's max_bar / sum_bar mbarriers. S is read
+        // twice (for the max, then for the exponentials), and each warp writes its P packed over its
+        // own S columns. Every wait is bounded; a warp whose wait fails leaves, and the others run
+        // into their own bounded waits.
+        constexpr int SC = BK / 2, OC = D / 2;
+        constexpr int CH = SC < 32 ? SC : 32;  // columns per TMEM load
+        const int t = warp >> 3, qtr = warp & 3, e = (warp >> 2) & 1;
         const int row = qtr * 32 + lane;
         const int m = row / G, h = row % G;
         const uint32_t lane_addr = tmem + ((uint32_t)(qtr * 32) << 16);
+        const uint32_t tS = lane_addr + t * 256 + e * SC, tO = lane_addr + t * 256 + 128 + e * OC;
         const float sl2 = a.scale * 1.4426950408889634f;
-        // the item whose O is read out next: the row's partial index ((b, i, r, slot), head) or -1
-        // and its max (partial indices fit 31 bits, checked by the host)
+        // the team's item whose O is read out next: the row's partial index ((b, i, r, slot), head)
+        // or -1 and its max (partial indices fit 31 bits, checked by the host)
         bool have_prev = false;
         int pv_prow = -1;
         float pv_mx = 0.f;
-        // O of item np: normalise by the row's rounded weight sum, store the fp16 partial and its
-        // LSE, free the accumulator
-        auto store_prev = [&](int np) -> bool {
-            if (!__all_sync(0xffffffffu, mbar_wait(&s.o_full[np & 1], (np >> 1) & 1, a.status, 0x704))) return false;
-            if (!__all_sync(0xffffffffu, mbar_wait(&s.sum_bar[np & 1], (np >> 1) & 1, a.status, 0x705))) return false;
+        // O of the team's item number kp: normalise by the row's rounded weight sum, store the fp16
+        // partial and its LSE, free the accumulator
+        auto store_prev = [&](int kp) -> bool {
+            const int pb = kp & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.o_full[t], pb, a.status, 0x704))) return false;
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.sum_bar[t][pb], (kp >> 1) & 1, a.status, 0x705))) return false;
             tc_fence_after();
-            uint32_t ov[OC];
-            tmem_ld<OC>(lane_addr + (np & 1) * 256 + 128 + e * OC, ov);
-            tmem_ld_wait();
-            const int pb = np & 1;
-            if (pv_prow >= 0) {
-                const float lr = (s.red_lr[pb][0][row] + s.red_lr[pb][1][row]) + (s.red_lr[pb][2][row] + s.red_lr[pb][3][row]);
-                const float inv = 1.f / lr;
-                uint32_t hv[OC / 2];
+            float inv = 0.f;
+            if (pv_prow >= 0) inv = 1.f / (s.red_lr[t][pb][0][row] + s.red_lr[t][pb][1][row]);
+            const uint64_t invx2 = f2_packf(inv, inv);
+            // chunk x of 8 values goes to [(b, i, r, slot)][x][head]: the G heads of a query are
+            // adjacent, so a warp's store covers whole 128-byte lines
+            uint4* dst = reinterpret_cast<uint4*>(a.o_part) + (pv_prow >= 0 ? (size_t)(pv_prow - h) * (D / 8) + h : 0);
 #pragma unroll
-                for (int x = 0; x < OC; x += 2) {
-                    const __half2 hh2 = __floats2half2_rn(__uint_as_float(ov[x]) * inv, __uint_as_float(ov[x + 1]) * inv);
-                    hv[x / 2] = *reinterpret_cast<const uint32_t*>(&hh2);
-                }
-                // chunk x of 8 values goes to [(b, i, r, slot)][x][head]: the G heads of a query
-                // are adjacent, so a warp's store covers whole 128-byte lines
-                uint4* dst = reinterpret_cast<uint4*>(a.o_part) + (size_t)(pv_prow - h) * (D / 8) + h;
+            for (int c0 = 0; c0 < OC; c0 += 32) {
+                uint32_t ov[32];
+                tmem_ld32(tO + c0, ov);
+                tmem_ld_wait();
+                if (pv_prow >= 0) {
+                    uint32_t hv[16];
 #pragma unroll
-                for (int x = 0; x < OC / 8; ++x)
-                    dst[(size_t)(e * (OC / 8) + x) * G] = make_uint4(hv[4 * x], hv[4 * x + 1], hv[4 * x + 2], hv[4 * x + 3]);
-                if (e == 0) {
-                    const float l = (s.red_l[pb][0][row] + s.red_l[pb][1][row]) + (s.red_l[pb][2][row] + s.red_l[pb][3][row]);
-                    a.lse_part[pv_prow] = pv_mx * a.scale + logf(l);
+                    for (int x = 0; x < 32; x += 2) {
+                        float o0, o1;
+                        f2_unpack(f2_mul(f2_pack(ov[x], ov[x + 1]), invx2), o0, o1);
+                        const __half2 hh2 = __floats2half2_rn(o0, o1);
+                        hv[x / 2] = *reinterpret_cast<const uint32_t*>(&hh2);
+                    }
+#pragma unroll
+                    for (int x = 0; x < 4; ++x)
+                        dst[(size_t)((e * OC + c0) / 8 + x) * G] = make_uint4(hv[4 * x], hv[4 * x + 1], hv[4 * x + 2], hv[4 * x + 3]);
                 }
             }
+            if (e == 0 && pv_prow >= 0)
+                a.lse_part[pv_prow] = pv_mx * a.scale + logf(s.red_l[t][pb][0][row] + s.red_l[t][pb][1][row]);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&s.o_free[np & 1]);
+            if (lane == 0) mbar_arrive(&s.o_free[t]);
             return true;
         };
-        // Each warp: row max of its S quarter -> max_bar; softmax of this item -> sum_bar and
-        // p_full (so the PV product can start); then the O of the previous item. Every wait is
-        // bounded; a warp whose wait fails leaves, and the others run into their own bounded waits.
         bool fail = false;
-        int n = 0;
-        for (;; ++n) {
+        int k = 0;
+        for (;; ++k) {
+            const int n = 2 * k + t, kb = k & 1;
+            // the O buffer of the team is single: free it (item k-1) before this item's softmax, so
+            // that the PV product of item k can start as soon as its P is in
+            if (have_prev) {
+                if (!store_prev(k - 1)) {
+                    fail = true;
+                    break;
+                }
+                have_prev = false;
+            }
             const int slot = n % kMeta;
             if (!__all_sync(0xffffffffu, mbar_wait(&s.meta_full[slot], (n / kMeta) & 1, a.status, 0x701))) {
                 fail = true;
@@ -435,74 +464,82 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int qslot = valid ? (int)mt.qs[m] : 0;
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.meta_empty[slot]);
-            const uint32_t tS = lane_addr + (n & 1) * 256;
             const int lim = valid ? i - c * BK - e * SC : -1;  // this warp's columns x <= lim are causal
-            if (!__all_sync(0xffffffffu, mbar_wait(&s.s_full[n & 1], (n >> 1) & 1, a.status, 0x702))) {
+            const bool full = __all_sync(0xffffffffu, lim >= SC - 1);
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.s_full[t], kb, a.status, 0x702))) {
                 fail = true;
                 break;
             }
             tc_fence_after();
-            uint32_t sv[SC];
-            tmem_ld<SC>(tS + e * SC, sv);
-            tmem_ld_wait();
-            const bool full = __all_sync(0xffffffffu, lim >= SC - 1);
+            // pass 1: max over this warp's causal columns
             {
                 float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-                if (full) {
 #pragma unroll
-                    for (int x = 0; x < SC; ++x) m4[x & 3] = fmaxf(m4[x & 3], __uint_as_float(sv[x]));
-                } else {
+                for (int c0 = 0; c0 < SC; c0 += CH) {
+                    uint32_t sv[CH];
+                    tmem_ld<CH>(tS + c0, sv);
+                    tmem_ld_wait();
+                    if (full) {
 #pragma unroll
-                    for (int x = 0; x < SC; ++x) m4[x & 3] = x <= lim ? fmaxf(m4[x & 3], __uint_as_float(sv[x])) : m4[x & 3];
+                        for (int x = 0; x < CH; x += 2)
+                            m4[(x >> 1) & 3] = max3f(m4[(x >> 1) & 3], __uint_as_float(sv[x]), __uint_as_float(sv[x + 1]));
+                    } else {
+#pragma unroll
+                        for (int x = 0; x < CH; ++x)
+                            m4[x & 3] = c0 + x <= lim ? fmaxf(m4[x & 3], __uint_as_float(sv[x])) : m4[x & 3];
+                    }
                 }
-                s.red_max[n & 1][e][row] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+                s.red_max[t][kb][e][row] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&s.max_bar[n & 1]);
-            if (!__all_sync(0xffffffffu, mbar_wait(&s.max_bar[n & 1], (n >> 1) & 1, a.status, 0x703))) {
+            if (lane == 0) mbar_arrive(&s.max_bar[t]);
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.max_bar[t], kb, a.status, 0x703))) {
                 fail = true;
                 break;
             }
-            // P = exp(S - max) rounded to bf16, packed two per TMEM column over this warp's own S
-            // columns (already in registers). l: exact sum for the LSE; lr: sum of the rounded
-            // weights the MMA uses, so that O / lr stays a convex combination of the V rows.
-            const float mx = fmaxf(fmaxf(s.red_max[n & 1][0][row], s.red_max[n & 1][1][row]),
-                                   fmaxf(s.red_max[n & 1][2][row], s.red_max[n & 1][3][row]));
+            // pass 2: P = exp(S - max) rounded to bf16, packed two per TMEM column over the warp's
+            // own S columns already read. l: exact sum for the LSE; lr: sum of the rounded weights
+            // the MMA uses, so that O / lr stays a convex combination of the V rows.
+            const float mx = fmaxf(s.red_max[t][kb][0][row], s.red_max[t][kb][1][row]);
             const float moff = valid ? mx * sl2 : 0.f;
-            float l0 = 0.f, l1 = 0.f, lr0 = 0.f, lr1 = 0.f;
-            uint32_t pk[SC / 2];
+            const uint64_t sl2x2 = f2_packf(sl2, sl2), moffx2 = f2_packf(-moff, -moff);
+            uint64_t lx2 = f2_packf(0.f, 0.f), lrx2 = f2_packf(0.f, 0.f);
 #pragma unroll
-            for (int y = 0; y < SC; y += 2) {
-                float p0 = fast_exp2(fmaf(__uint_as_float(sv[y]), sl2, -moff));
-                float p1 = fast_exp2(fmaf(__uint_as_float(sv[y + 1]), sl2, -moff));
-                if (!full) {
-                    p0 = y <= lim ? p0 : 0.f;
-                    p1 = y + 1 <= lim ? p1 : 0.f;
+            for (int c0 = 0; c0 < SC; c0 += CH) {
+                uint32_t sv[CH];
+                tmem_ld<CH>(tS + c0, sv);
+                tmem_ld_wait();
+                uint32_t pk[CH / 2];
+#pragma unroll
+                for (int y = 0; y < CH; y += 2) {
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(sv[y], sv[y + 1]), sl2x2, moffx2), x0, x1);
+                    float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+                    if (!full) {
+                        p0 = c0 + y <= lim ? p0 : 0.f;
+                        p1 = c0 + y + 1 <= lim ? p1 : 0.f;
+                    }
+                    const __nv_bfloat162 pb2 = __floats2bfloat162_rn(p0, p1);
+                    const uint32_t u = *reinterpret_cast<const uint32_t*>(&pb2);
+                    lx2 = f2_add(lx2, f2_packf(p0, p1));
+                    lrx2 = f2_add(lrx2, f2_pack(u << 16, u & 0xffff0000u));
+                    pk[y / 2] = u;
                 }
-                const __nv_bfloat162 pb2 = __floats2bfloat162_rn(p0, p1);
-                const uint32_t u = *reinterpret_cast<const uint32_t*>(&pb2);
-                if (y & 2) {
-                    l1 += p0 + p1;
-                    lr1 += __uint_as_float(u << 16) + __uint_as_float(u & 0xffff0000u);
-                } else {
-                    l0 += p0 + p1;
-                    lr0 += __uint_as_float(u << 16) + __uint_as_float(u & 0xffff0000u);
-                }
-                pk[y / 2] = u;
+                tmem_st<CH / 2>(tS + c0 / 2, pk);
             }
-            tmem_st<SC / 2>(tS + e * (SC / 2), pk);
             tmem_st_wait();
             tc_fence_before();
-            s.red_l[n & 1][e][row] = l0 + l1;
-            s.red_lr[n & 1][e][row] = lr0 + lr1;
+            {
+                float l0, l1, lr0, lr1;
+                f2_unpack(lx2, l0, l1);
+                f2_unpack(lrx2, lr0, lr1);
+                s.red_l[t][kb][e][row] = l0 + l1;
+                s.red_lr[t][kb][e][row] = lr0 + lr1;
+            }
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&s.sum_bar[n & 1]);
-                mbar_arrive(&s.p_full[n & 1]);
-            }
-            if (have_prev && !store_prev(n - 1)) {
-                fail = true;
-                break;
+                mbar_arrive(&s.sum_bar[t][kb]);
+                mbar_arrive(&s.p_full[t]);
             }
             have_prev = true;
             pv_prow = valid ? (((b * a.N + i) * a.H_kv + r) * K1 + qslot) * G + h : -1;
@@ -511,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (fail) {
             s.abort = 1;
         } else if (have_prev) {
-            store_prev(n - 1);
+            store_prev(k - 1);
         }
     }
     tc_fence_before();
