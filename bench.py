@@ -112,6 +112,34 @@ def selected_tokens(blocks: torch.Tensor, block_k: int) -> int:
     return int(torch.where(c >= 0, n, torch.zeros_like(n)).sum().item())
 
 
+def valid_slots(blocks: torch.Tensor, block_k: int) -> int:
+    """Number of (b, i, r, slot) selections that name a causal block (each yields one partial)."""
+    B, N, H_kv, K1 = blocks.shape
+    i = torch.arange(N, device=blocks.device).view(1, N, 1, 1)
+    c = blocks.long()
+    return int(((c >= 0) & (c <= i // block_k)).sum().item())
+
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch, per unit of work, from an
+# ncu capture of the kernel; it holds only for the kernel source it was measured on (sha256 of the
+# file), and reads null once that file changes.
+MEASURED_TRAFFIC = {
+    "attn_kv_outer": {"file": "block_sparse_attention_idx_b200/csrc/msa_attn.cu", "sha256": None,
+                      "bytes_per_unit": None, "unit": "selected token", "capture": None},
+}
+
+
+def measured_traffic(kernel: str, units: float):
+    m = MEASURED_TRAFFIC.get(kernel)
+    if not m or not m["sha256"]:
+        return None
+    import hashlib
+    with open(os.path.join(ROOT, m["file"]), "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != m["sha256"]:
+            return None
+    return m["bytes_per_unit"] * units
+
+
 def timed_steps(fn, steps: int, flush: torch.Tensor):
     """Per-step device times (ms) with CUDA events on the current stream; L2 flushed before each."""
     st = torch.cuda.current_stream()
@@ -156,12 +184,23 @@ def barrier(world):
     torch.cuda.synchronize()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """The largest of the ranks' values (every rank takes part and gets the answer)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(w, rank: int) -> int:
+    """Seed of a rank's synthetic inputs: every rank runs its own independent sequences."""
+    return 1000 + w.cid + 7919 * rank
+
+
+def job_throughput(units_per_rank: float, world: int, slowest_ms: float) -> float:
+    """Whole-job units per second: all ranks' units over the slowest rank's step time."""
+    return units_per_rank * world / (slowest_ms * 1e-3)
 
 
 # ============================================================================ reference arm
@@ -225,7 +264,7 @@ def cpu_baseline(x, w, rows_n: int):
 def bench_prefill(args, world, rank, msa, pk):
     w = WORKLOADS[args.workload]
     dev = torch.device("cuda", torch.cuda.current_device())
-    x = prefill_inputs(w, device=dev, seed=1000 + w.cid + 7919 * rank)
+    x = prefill_inputs(w, device=dev, seed=rank_seed(w, rank))
     dims = msa.MsaDims(w.B, w.N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
     ws_i = msa.workspace(msa.MSA_OP_INDEX_TOPK, dims, dev)
     ws_a = msa.workspace(msa.MSA_OP_ATTN_FWD, dims, dev)
@@ -240,6 +279,9 @@ def bench_prefill(args, world, rank, msa, pk):
     torch.cuda.synchronize()
     sel_tok = selected_tokens(blocks, w.block_k)  # sum_{i,r} |J|
     G = w.H_q // w.H_kv
+    # merge: read every valid partial (fp16 o + fp32 lse) and the selection, write bf16 out + lse
+    merge_bytes = (valid_slots(blocks, w.block_k) * G * (2 * w.d + 4) + w.B * w.N * w.H_q * (2 * w.d + 4)
+                   + blocks.numel() * 4)
     attn_flops = 4.0 * w.d * G * sel_tok
     index_flops = 2.0 * w.d_idx * w.H_kv * w.N * (w.N + 1) / 2
     msa.msa_profile_read()
@@ -251,7 +293,7 @@ def bench_prefill(args, world, rank, msa, pk):
     prof = profile_avg(msa.msa_profile_read())
     barrier(world)
     step_ms = max_over_ranks(sum(t) / len(t), world)
-    value = w.N * w.B * world / (step_ms * 1e-3)
+    value = job_throughput(w.N * w.B, world, step_ms)
     # roofline of the dominant kernel (live CUDA-event durations of its launches)
     dom = max(prof, key=lambda k: prof[k]["total_ms"])
     per_kernel = {}
@@ -262,15 +304,19 @@ def bench_prefill(args, world, rank, msa, pk):
                          "share": round(v["total_ms"] / sum(u["total_ms"] for u in prof.values()), 4),
                          **({"tflops": round(tf, 1), "frac_of_measured_bf16": round(tf / pk["bf16_tflops"], 4)}
                             if tf else {})}
+        if k == "attn_merge":
+            gbs = merge_bytes / (v["avg_ms"] * 1e-3) / 1e9
+            per_kernel[k].update({"bytes": merge_bytes, "gbs": round(gbs, 1),
+                                  "frac_of_measured_hbm": round(gbs / pk["hbm_gbs"], 4)})
     dfl = attn_flops if dom == "attn_kv_outer" else index_flops if dom == "index_topk" else None
     roof = roofline_entry("tensor", dfl / (prof[dom]["avg_ms"] * 1e-3) / 1e12 if dfl else None,
-                          pk["bf16_tflops"], "TFLOP/s", None)
+                          pk["bf16_tflops"], "TFLOP/s", measured_traffic(dom, sel_tok))
     roof["kernel"] = dom
     roof["flops_per_launch"] = dfl
     roof["peak_source"] = f"{pk['source']} bf16 burst"
     # e2e through the public API with pinned host buffers (H2D inputs, D2H output inside the region)
     host = {k: x[k].cpu().pin_memory() for k in ("q", "k", "v", "q_idx", "k_idx")}
-    out_host = torch.empty(x["q"].shape, dtype=torch.bfloat16).pin_memory()
+    out_host = torch.empty(x["q"].shape, dtype=torch.float32).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = out_host.numel() * out_host.element_size()
 
@@ -289,9 +335,10 @@ def bench_prefill(args, world, rank, msa, pk):
         te = timed_steps(e2e_step, e2e_steps, flush)
         e2e_ms = max_over_ranks(sum(te) / len(te), world)
     res = {"value": value, "ms_per_step": step_ms, "roofline": roof, "kernels": per_kernel, "clocks": cs.summary(),
-           "e2e": {"value": w.N * w.B * world / (e2e_ms * 1e-3), "unit": "query-tokens/s",
+           "e2e": {"value": job_throughput(w.N * w.B, world, e2e_ms), "unit": "query-tokens/s",
                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-           "gpu_launches": 7 * args.steps,
+           # index Top-k, the six inverse-list kernels, attention and merge (memsets are not counted)
+           "gpu_launches": 9 * args.steps,
            "work": {"selected_tokens": sel_tok, "mean_J": sel_tok / (w.N * w.H_kv), "attn_flops": attn_flops,
                     "index_flops": index_flops}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -304,7 +351,7 @@ def bench_prefill(args, world, rank, msa, pk):
 def bench_decode(args, world, rank, msa, pk):
     w = WORKLOADS["decode_16x256k"]
     dev = torch.device("cuda", torch.cuda.current_device())
-    x = decode_inputs(w, device=dev, seed=1000 + w.cid + 7919 * rank)
+    x = decode_inputs(w, device=dev, seed=rank_seed(w, rank))
     dims = msa.MsaDims(w.B, w.N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
     ws = msa.workspace(msa.MSA_OP_DECODE, dims, dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -343,7 +390,7 @@ def bench_decode(args, world, rank, msa, pk):
 def bench_train(args, world, rank, msa, pk):
     w = WORKLOADS["train_64k"]
     dev = torch.device("cuda", torch.cuda.current_device())
-    x = prefill_inputs(w, device=dev, seed=1000 + w.cid + 7919 * rank)
+    x = prefill_inputs(w, device=dev, seed=rank_seed(w, rank))
     dims = msa.MsaDims(w.B, w.N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
     ws_i = msa.workspace(msa.MSA_OP_INDEX_TOPK_LSE, dims, dev)
     ws_a = msa.workspace(msa.MSA_OP_ATTN_FWD, dims, dev)

@@ -148,13 +148,13 @@ def msa_index_topk(dims: MsaDims, q_idx, k_idx, want_lse: bool = False, ws=None,
 
 
 def msa_sparse_attn_fwd(dims: MsaDims, q, k, v, blocks, want_lse: bool = True, ws=None, stream=None):
-    """Sparse attention forward. Returns out bf16 [B,N,H_q,d] and LSE fp32 [B,N,H_q] (or None)."""
+    """Sparse attention forward. Returns out fp32 [B,N,H_q,d] and LSE fp32 [B,N,H_q] (or None)."""
     dev = q.device
     _need(q, "q", (dims.B, dims.N, dims.H_q, dims.d), torch.bfloat16, dev)
     _need(k, "k", (dims.B, dims.N, dims.H_kv, dims.d), torch.bfloat16, dev)
     _need(v, "v", (dims.B, dims.N, dims.H_kv, dims.d), torch.bfloat16, dev)
     _need(blocks, "blocks", (dims.B, dims.N, dims.H_kv, dims.topk + 1), torch.int32, dev)
-    out = torch.empty_like(q)
+    out = torch.empty(q.shape, dtype=torch.float32, device=dev)
     lse = torch.empty(dims.B, dims.N, dims.H_q, dtype=torch.float32, device=dev) if want_lse else None
     if ws is None:
         ws = workspace(MSA_OP_ATTN_FWD, dims, dev)
@@ -165,7 +165,7 @@ def msa_sparse_attn_fwd(dims: MsaDims, q, k, v, blocks, want_lse: bool = True, w
 
 def msa_sparse_attn_decode(dims: MsaDims, cache_len, q, q_idx, k_cache, v_cache, k_idx_cache, want_blocks=True,
                            ws=None, stream=None):
-    """One decode step. dims.N is the cache capacity. Returns out bf16 [B,H_q,d] and the selected
+    """One decode step. dims.N is the cache capacity. Returns out fp32 [B,H_q,d] and the selected
     blocks int32 [B,H_kv,topk+1] (or None)."""
     dev = q.device
     _need(cache_len, "cache_len", (dims.B,), torch.int32, dev)
@@ -174,7 +174,7 @@ def msa_sparse_attn_decode(dims: MsaDims, cache_len, q, q_idx, k_cache, v_cache,
     _need(k_cache, "k_cache", (dims.B, dims.N, dims.H_kv, dims.d), torch.bfloat16, dev)
     _need(v_cache, "v_cache", (dims.B, dims.N, dims.H_kv, dims.d), torch.bfloat16, dev)
     _need(k_idx_cache, "k_idx_cache", (dims.B, dims.N, dims.d_idx), torch.bfloat16, dev)
-    out = torch.empty_like(q)
+    out = torch.empty(q.shape, dtype=torch.float32, device=dev)
     blocks = torch.empty(dims.B, dims.H_kv, dims.topk + 1, dtype=torch.int32, device=dev) if want_blocks else None
     if ws is None:
         ws = workspace(MSA_OP_DECODE, dims, dev)
@@ -198,8 +198,8 @@ def msa_sparse_attn_decode_noalloc(dims: MsaDims, cache_len, q, q_idx, k_cache, 
     _need(v_cache, "v_cache", (dims.B, dims.N, dims.H_kv, dims.d), torch.bfloat16, dev)
     _need(k_idx_cache, "k_idx_cache", (dims.B, dims.N, dims.d_idx), torch.bfloat16, dev)
     if out is None:
-        out = torch.empty_like(q)
-    _need(out, "out", (dims.B, dims.H_q, dims.d), torch.bfloat16, dev)
+        out = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    _need(out, "out", (dims.B, dims.H_q, dims.d), torch.float32, dev)
     if blocks is not None:
         _need(blocks, "blocks", (dims.B, dims.H_kv, dims.topk + 1), torch.int32, dev)
     _check("msa_sparse_attn_decode_noalloc",

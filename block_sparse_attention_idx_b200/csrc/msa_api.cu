@@ -161,7 +161,7 @@ msa_status msa_index_topk(const msa_dims* d, const void* q_idx, const void* k_id
 }
 
 msa_status msa_sparse_attn_fwd(const msa_dims* d, const void* q, const void* k, const void* v, const int32_t* blocks,
-                               void* out, float* lse, void* ws, size_t ws_bytes, msa_stream_t stream_) {
+                               float* out, float* lse, void* ws, size_t ws_bytes, msa_stream_t stream_) {
     msa_status s = check_common(d);
     if (s != MSA_OK) return s;
     if (!attn_rows_fit(d)) return MSA_ERR_UNSUPPORTED;
@@ -179,7 +179,7 @@ msa_status msa_sparse_attn_fwd(const msa_dims* d, const void* q, const void* k, 
     a.topk = d->topk; a.scale = eff_scale(d->scale, d->d);
     attn_carve(&a, static_cast<uint8_t*>(ws) + kStatusBytes);
     a.blocks = blocks;
-    a.out = static_cast<__nv_bfloat16*>(out);
+    a.out = static_cast<float*>(out);
     a.lse = lse;
     a.status = status;
     e = run_attn(a, q, k, v, num_sms(), st);
@@ -187,7 +187,7 @@ msa_status msa_sparse_attn_fwd(const msa_dims* d, const void* q, const void* k, 
 }
 
 msa_status msa_sparse_attn_decode(const msa_dims* d, const int32_t* cache_len, const void* q, const void* q_idx,
-                                  const void* k_cache, const void* v_cache, const void* k_idx_cache, void* out,
+                                  const void* k_cache, const void* v_cache, const void* k_idx_cache, float* out,
                                   int32_t* blocks_out, void* ws, size_t ws_bytes, msa_stream_t stream_) {
     msa_status s = check_common(d);
     if (s != MSA_OK) return s;

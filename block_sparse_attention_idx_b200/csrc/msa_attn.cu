@@ -621,14 +621,14 @@ __global__ void __launch_bounds__(256) k_attn_merge(AttnArgs a) {
                 }
             }
             const float zi = 1.f / z;
-            uint32_t pk[4];
 #pragma unroll
-            for (int y = 0; y < 4; ++y) {
-                overflow |= !isfinite(acc[2 * y]) || !isfinite(acc[2 * y + 1]);
-                pk[y] = pack_bf16x2(acc[2 * y] * zi, acc[2 * y + 1] * zi);
+            for (int y = 0; y < 8; ++y) {
+                overflow |= !isfinite(acc[y]);
+                acc[y] *= zi;
             }
-            *reinterpret_cast<uint4*>(a.out + (((size_t)b * a.N + i) * a.H_q + hq) * D + d0) =
-                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            float4* o4 = reinterpret_cast<float4*>(a.out + (((size_t)b * a.N + i) * a.H_q + hq) * D + d0);
+            o4[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            o4[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
             if (a.lse && d0 == 0) a.lse[((size_t)b * a.N + i) * a.H_q + hq] = lmax + logf(z);
         }
     }

@@ -243,7 +243,7 @@ __global__ void __launch_bounds__(128) k_dec_attn(DecodeArgs a, const __nv_bfloa
 
 // One warp per (sequence, head): merge the slot partials.
 template <int D>
-__global__ void k_dec_combine(DecodeArgs a, __nv_bfloat16* __restrict__ out) {
+__global__ void k_dec_combine(DecodeArgs a, float* __restrict__ out) {
     const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (w >= a.B * a.H_q) return;
@@ -268,9 +268,9 @@ __global__ void k_dec_combine(DecodeArgs a, __nv_bfloat16* __restrict__ out) {
         for (int x = 0; x < kPer; ++x) acc[x] = fmaf(wg, op[x], acc[x]);
     }
     const float inv = 1.f / z;
-    __nv_bfloat16* o = out + ((size_t)b * a.H_q + h) * D + lane * kPer;
+    float* o = out + ((size_t)b * a.H_q + h) * D + lane * kPer;
 #pragma unroll
-    for (int x = 0; x < kPer; ++x) o[x] = __float2bfloat16_rn(acc[x] * inv);
+    for (int x = 0; x < kPer; ++x) o[x] = acc[x] * inv;
 }
 
 }  // namespace
@@ -312,12 +312,12 @@ cudaError_t run_decode(const DecodeArgs& a, const void* q, const void* q_idx, co
         e = cudaFuncSetAttribute(k_dec_attn<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         k_dec_attn<128><<<agrid, 128, smem, st>>>(a, qb, kb, vb);
-        k_dec_combine<128><<<(a.B * a.H_q * 32 + 255) / 256, 256, 0, st>>>(a, static_cast<__nv_bfloat16*>(out));
+        k_dec_combine<128><<<(a.B * a.H_q * 32 + 255) / 256, 256, 0, st>>>(a, static_cast<float*>(out));
     } else {
         e = cudaFuncSetAttribute(k_dec_attn<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         k_dec_attn<64><<<agrid, 128, smem, st>>>(a, qb, kb, vb);
-        k_dec_combine<64><<<(a.B * a.H_q * 32 + 255) / 256, 256, 0, st>>>(a, static_cast<__nv_bfloat16*>(out));
+        k_dec_combine<64><<<(a.B * a.H_q * 32 + 255) / 256, 256, 0, st>>>(a, static_cast<float*>(out));
     }
     return cudaGetLastError();
 }

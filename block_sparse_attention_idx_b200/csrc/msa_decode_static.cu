@@ -46,7 +46,7 @@ msa_status scratch_address(void** out) {
 
 extern "C" msa_status msa_sparse_attn_decode_noalloc(const msa_dims* dims, const int32_t* cache_len, const void* q,
                                                       const void* q_idx, const void* k_cache, const void* v_cache,
-                                                      const void* k_idx_cache, void* out, int32_t* blocks_out,
+                                                      const void* k_idx_cache, float* out, int32_t* blocks_out,
                                                       msa_stream_t stream) {
     size_t need = 0;
     msa_status s = msa_workspace_size(MSA_OP_DECODE, dims, &need);

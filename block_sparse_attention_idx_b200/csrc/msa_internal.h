@@ -76,7 +76,7 @@ struct AttnArgs {
     float* lse_part;     // [B, N, H_kv, topk+1, G]
     int32_t* sched;      // [1]           next item to hand out
     const int32_t* blocks;
-    __nv_bfloat16* out;  // [B, N, H_q, d]
+    float* out;          // [B, N, H_q, d]  fp32 (the fp32-accumulated result)
     float* lse;          // [B, N, H_q] or null
     DevStatus* status;
 };

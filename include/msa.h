@@ -106,11 +106,11 @@ MSA_API msa_status msa_index_topk(const msa_dims *dims, const void *q_idx, const
  *   k, v   bf16  [B, N, H_kv, d]
  *   blocks int32 [B, N, H_kv, topk+1]: ids in [0, i/block_k], -1 entries ignored; normally the
  *          output of msa_index_topk. The local block must be present for J to be non-empty.
- *   out    bf16  [B, N, H_q, d]                                      (output)
+ *   out    fp32  [B, N, H_q, d]: the fp32-accumulated result, not rounded to bf16 (output)
  *   lse    fp32  [B, N, H_q] or NULL: natural-log sum-exp of the scaled logits over J (output)
  */
 MSA_API msa_status msa_sparse_attn_fwd(const msa_dims *dims, const void *q, const void *k, const void *v,
-                               const int32_t *blocks, void *out, float *lse, void *ws, size_t ws_bytes,
+                               const int32_t *blocks, float *out, float *lse, void *ws, size_t ws_bytes,
                                msa_stream_t stream);
 
 /*
@@ -121,11 +121,11 @@ MSA_API msa_status msa_sparse_attn_fwd(const msa_dims *dims, const void *q, cons
  *   cache_len  int32 [B] device, 1 <= cache_len[b] <= N
  *   q          bf16 [B, H_q, d];  q_idx bf16 [B, H_kv, d_idx]
  *   k_cache, v_cache bf16 [B, N, H_kv, d];  k_idx_cache bf16 [B, N, d_idx]
- *   out        bf16 [B, H_q, d]                                      (output)
+ *   out        fp32 [B, H_q, d]: the fp32-accumulated result        (output)
  *   blocks_out int32 [B, H_kv, topk+1] or NULL                       (output)
  */
 MSA_API msa_status msa_sparse_attn_decode(const msa_dims *dims, const int32_t *cache_len, const void *q, const void *q_idx,
-                                  const void *k_cache, const void *v_cache, const void *k_idx_cache, void *out,
+                                  const void *k_cache, const void *v_cache, const void *k_idx_cache, float *out,
                                   int32_t *blocks_out, void *ws, size_t ws_bytes, msa_stream_t stream);
 
 /*
@@ -170,7 +170,7 @@ MSA_API msa_status msa_kl_fwd_grad(const msa_dims *dims, const void *q, const vo
 #define MSA_DECODE_STATIC_SCRATCH_BYTES (16u << 20)
 MSA_API msa_status msa_sparse_attn_decode_noalloc(const msa_dims *dims, const int32_t *cache_len, const void *q,
                                                   const void *q_idx, const void *k_cache, const void *v_cache,
-                                                  const void *k_idx_cache, void *out, int32_t *blocks_out,
+                                                  const void *k_idx_cache, float *out, int32_t *blocks_out,
                                                   msa_stream_t stream);
 
 /*

@@ -1,0 +1,113 @@
+"""Full-size workloads in the launch configuration the benchmark times (same entry points, same
+workspaces, whole grids), checked against the float64 oracle on sampled rows and, where a value is
+a reduction over the whole layer, through properties that hold at any size.
+
+Workloads: the 8K and 32K (needle) prefills, the 64K training step (index Top-k with LSE_idx,
+attention, KL alignment) and one decode step of 16 sequences over 256K-token caches."""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_idx_b200 as msa
+import oracle
+from msa_inputs import WORKLOADS, prefill_inputs, decode_inputs
+from parity import compare_blocks, check_attention, check_grad
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def sampled_rows(N, n=40, seed=0):
+    """First and last rows, rows at block edges, and uniformly drawn rows."""
+    rng = np.random.default_rng(seed)
+    rows = {0, 1, 127, 128, 129, N // 2, N - 2, N - 1}
+    rows |= set(rng.choice(N, size=n, replace=False).tolist())
+    return np.array(sorted(r for r in rows if 0 <= r < N), dtype=np.int64)
+
+
+def run_prefill(w, want_lse_idx=False):
+    x = prefill_inputs(w, device=DEV)
+    dm = msa.MsaDims(w.B, w.N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
+    ws_i = msa.workspace(msa.MSA_OP_INDEX_TOPK_LSE if want_lse_idx else msa.MSA_OP_INDEX_TOPK, dm, DEV)
+    ws_a = msa.workspace(msa.MSA_OP_ATTN_FWD, dm, DEV)
+    if want_lse_idx:
+        blocks, lse_idx = msa.msa_index_topk(dm, x["q_idx"], x["k_idx"], want_lse=True, ws=ws_i)
+    else:
+        blocks, lse_idx = msa.msa_index_topk(dm, x["q_idx"], x["k_idx"], ws=ws_i), None
+    out, lse = msa.msa_sparse_attn_fwd(dm, x["q"], x["k"], x["v"], blocks, ws=ws_a)
+    torch.cuda.synchronize()
+    assert msa.msa_get_device_status(ws_a) == msa.MSA_OK
+    return dm, x, blocks, lse_idx, out, lse
+
+
+def check_sampled_prefill(w, x, blocks, out, lse, rows):
+    od = oracle.Dims(w.B, w.N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
+    xc = {k: v.cpu() for k, v in x.items()}
+    ob, om, _ = oracle.index_topk(od, xc["q_idx"], xc["k_idx"], rows=rows)
+    gb = blocks.cpu().numpy().reshape(w.B * w.N, w.H_kv, w.topk + 1)
+    bad, near = compare_blocks(gb[rows], ob, om)
+    assert bad == 0, f"{bad} sampled selection rows differ (near-ties excluded: {near})"
+    # attention over the blocks the GPU selected, on the sampled rows
+    oo, ol = oracle.sparse_attn(od, xc["q"], xc["k"], xc["v"], blocks.cpu().numpy(), rows=rows)
+    og = out.float().cpu().numpy().reshape(w.B * w.N, w.H_q, w.d)[rows]
+    lg = lse.cpu().numpy().reshape(w.B * w.N, w.H_q)[rows]
+    check_attention(og, oo, lg, ol)
+    return xc, od
+
+
+@pytest.mark.parametrize("wname", ["prefill_8k", "prefill_32k_needles"])
+def test_full_prefill_sampled_rows_match_oracle(wname):
+    w = WORKLOADS[wname]
+    dm, x, blocks, _, out, lse = run_prefill(w)
+    check_sampled_prefill(w, x, blocks, out, lse, sampled_rows(w.N, seed=w.cid))
+
+
+def test_full_training_step_sampled_rows_and_invariants():
+    w = WORKLOADS["train_64k"]
+    dm, x, blocks, lse_idx, out, lse = run_prefill(w, want_lse_idx=True)
+    rows = sampled_rows(w.N, n=24, seed=w.cid)
+    xc, od = check_sampled_prefill(w, x, blocks, out, lse, rows)
+    gs = 1.0 / (w.N * w.H_kv)
+    ws_k = msa.workspace(msa.MSA_OP_KL, dm, DEV)
+    loss, dq, dk = msa.msa_kl_fwd_grad(dm, x["q"], x["k"], x["q_idx"], x["k_idx"], blocks, lse, lse_idx,
+                                       grad_scale=gs, ws=ws_k)
+    torch.cuda.synchronize()
+    assert msa.msa_get_device_status(ws_k) == msa.MSA_OK
+    # a KL divergence is never negative
+    assert float(loss.item()) >= 0.0
+    # dq_idx of the sampled rows against the oracle's gradient for those rows (GPU selection)
+    _, _, odq, _ = oracle.kl(od, xc["q"], xc["k"], xc["q_idx"], xc["k_idx"], blocks.cpu().numpy(),
+                             grad_scale=gs, rows=rows)
+    gdq = dq.cpu().numpy().reshape(w.B * w.N, w.H_kv, w.d_idx)[rows]
+    check_grad(gdq, odq, "dq_idx")
+    # P and P_idx both sum to one over each row's token set, so the rows' contributions to dK_idx
+    # cancel when summed over the tokens: sum_j dK_idx[b, j, :] = 0 up to rounding
+    tot = dk.double().sum(dim=1).abs().max().item()
+    scale = dk.double().abs().sum(dim=1).max().item()
+    assert tot <= 1e-3 * max(scale, 1e-30), f"sum over tokens of dK_idx is {tot:.3e} (|dK_idx| sum {scale:.3e})"
+
+
+def test_full_decode_sampled_sequences_match_oracle():
+    w = WORKLOADS["decode_16x256k"]
+    x = decode_inputs(w, device=DEV)
+    dm = msa.MsaDims(w.B, w.N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
+    ws = msa.workspace(msa.MSA_OP_DECODE, dm, DEV)
+    out, blocks = msa.msa_sparse_attn_decode(dm, x["cache_len"], x["q"], x["q_idx"], x["k_cache"], x["v_cache"],
+                                             x["k_idx_cache"], ws=ws)
+    torch.cuda.synchronize()
+    assert msa.msa_get_device_status(ws) == msa.MSA_OK
+    G = w.H_q // w.H_kv
+    od = oracle.Dims(1, w.N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
+    for b in (0, w.B - 1):
+        sl = slice(b, b + 1)
+        ob, om, oo, olse = oracle.decode(od, x["cache_len"][sl].cpu(), x["q"][sl].cpu(), x["q_idx"][sl].cpu(),
+                                         x["k_cache"][sl].cpu(), x["v_cache"][sl].cpu(), x["k_idx_cache"][sl].cpu())
+        gb = blocks[sl].cpu().numpy()
+        bad, near = compare_blocks(gb, ob, om)
+        assert bad == 0, f"sequence {b}: selection differs (near-ties excluded: {near})"
+        same = np.all(gb == ob, axis=-1)[0]
+        og = out[sl].float().cpu().numpy()[0]
+        for r in range(w.H_kv):
+            if same[r]:
+                check_attention(og[r * G:(r + 1) * G], oo[0, r * G:(r + 1) * G])
