@@ -124,8 +124,12 @@ def valid_slots(blocks: torch.Tensor, block_k: int) -> int:
 # ncu capture of the kernel; it holds only for the kernel source it was measured on (sha256 of the
 # file), and reads null once that file changes.
 MEASURED_TRAFFIC = {
-    "attn_kv_outer": {"file": "block_sparse_attention_idx_b200/csrc/msa_attn.cu", "sha256": None,
-                      "bytes_per_unit": None, "unit": "selected token", "capture": None},
+    # prefill_8k capture (dram read 213,596,416 B + write 1,974,181,632 B per launch over 60,309,504
+    # selected tokens), scaled by the selected tokens of the timed launch
+    "attn_kv_outer": {"file": "block_sparse_attention_idx_b200/csrc/msa_attn.cu",
+                      "sha256": "703ca7f5d95ead89b2d8050621f55f8205311920ade863251340ffc79dc52422",
+                      "bytes_per_unit": (213596416 + 1974181632) / 60309504, "unit": "selected token",
+                      "capture": "profiles/attn_kv_outer_prefill_8k.md"},
 }
 
 
@@ -279,8 +283,8 @@ def bench_prefill(args, world, rank, msa, pk):
     torch.cuda.synchronize()
     sel_tok = selected_tokens(blocks, w.block_k)  # sum_{i,r} |J|
     G = w.H_q // w.H_kv
-    # merge: read every valid partial (fp16 o + fp32 lse) and the selection, write bf16 out + lse
-    merge_bytes = (valid_slots(blocks, w.block_k) * G * (2 * w.d + 4) + w.B * w.N * w.H_q * (2 * w.d + 4)
+    # merge: read every valid partial (fp16 o + fp32 lse) and the selection, write fp32 out + lse
+    merge_bytes = (valid_slots(blocks, w.block_k) * G * (2 * w.d + 4) + w.B * w.N * w.H_q * (4 * w.d + 4)
                    + blocks.numel() * 4)
     attn_flops = 4.0 * w.d * G * sel_tok
     index_flops = 2.0 * w.d_idx * w.H_kv * w.N * (w.N + 1) / 2

@@ -41,6 +41,13 @@ def run_prefill(w, want_lse_idx=False):
     return dm, x, blocks, lse_idx, out, lse
 
 
+def oracle_selection(w, rows, ob):
+    """A full selection array holding the oracle's rows at `rows` (-1 elsewhere, never read)."""
+    full = np.full((w.B * w.N, w.H_kv, w.topk + 1), -1, dtype=np.int32)
+    full[rows] = ob
+    return full.reshape(w.B, w.N, w.H_kv, w.topk + 1)
+
+
 def check_sampled_prefill(w, x, blocks, out, lse, rows):
     od = oracle.Dims(w.B, w.N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
     xc = {k: v.cpu() for k, v in x.items()}
@@ -48,12 +55,16 @@ def check_sampled_prefill(w, x, blocks, out, lse, rows):
     gb = blocks.cpu().numpy().reshape(w.B * w.N, w.H_kv, w.topk + 1)
     bad, near = compare_blocks(gb[rows], ob, om)
     assert bad == 0, f"{bad} sampled selection rows differ (near-ties excluded: {near})"
-    # attention over the blocks the GPU selected, on the sampled rows
-    oo, ol = oracle.sparse_attn(od, xc["q"], xc["k"], xc["v"], blocks.cpu().numpy(), rows=rows)
-    og = out.float().cpu().numpy().reshape(w.B * w.N, w.H_q, w.d)[rows]
+    # attention on the oracle's own selection; compared where the GPU selected exactly the same
+    # blocks (every (query, group) row of the sample, unless a near-tie went the other way)
+    full = oracle_selection(w, rows, ob)
+    same = np.all(gb[rows] == ob, axis=(1, 2))
+    assert same.sum() >= len(rows) - near
+    oo, ol = oracle.sparse_attn(od, xc["q"], xc["k"], xc["v"], full, rows=rows)
+    og = out.cpu().numpy().reshape(w.B * w.N, w.H_q, w.d)[rows]
     lg = lse.cpu().numpy().reshape(w.B * w.N, w.H_q)[rows]
-    check_attention(og, oo, lg, ol)
-    return xc, od
+    check_attention(og[same], oo[same], lg[same], ol[same])
+    return xc, od, full, same
 
 
 @pytest.mark.parametrize("wname", ["prefill_8k", "prefill_32k_needles"])
@@ -67,7 +78,7 @@ def test_full_training_step_sampled_rows_and_invariants():
     w = WORKLOADS["train_64k"]
     dm, x, blocks, lse_idx, out, lse = run_prefill(w, want_lse_idx=True)
     rows = sampled_rows(w.N, n=24, seed=w.cid)
-    xc, od = check_sampled_prefill(w, x, blocks, out, lse, rows)
+    xc, od, full, same = check_sampled_prefill(w, x, blocks, out, lse, rows)
     gs = 1.0 / (w.N * w.H_kv)
     ws_k = msa.workspace(msa.MSA_OP_KL, dm, DEV)
     loss, dq, dk = msa.msa_kl_fwd_grad(dm, x["q"], x["k"], x["q_idx"], x["k_idx"], blocks, lse, lse_idx,
@@ -76,11 +87,11 @@ def test_full_training_step_sampled_rows_and_invariants():
     assert msa.msa_get_device_status(ws_k) == msa.MSA_OK
     # a KL divergence is never negative
     assert float(loss.item()) >= 0.0
-    # dq_idx of the sampled rows against the oracle's gradient for those rows (GPU selection)
-    _, _, odq, _ = oracle.kl(od, xc["q"], xc["k"], xc["q_idx"], xc["k_idx"], blocks.cpu().numpy(),
-                             grad_scale=gs, rows=rows)
+    # dq_idx of the sampled rows against the oracle's gradient for those rows (oracle selection,
+    # rows where the GPU selected the same blocks)
+    _, _, odq, _ = oracle.kl(od, xc["q"], xc["k"], xc["q_idx"], xc["k_idx"], full, grad_scale=gs, rows=rows)
     gdq = dq.cpu().numpy().reshape(w.B * w.N, w.H_kv, w.d_idx)[rows]
-    check_grad(gdq, odq, "dq_idx")
+    check_grad(gdq[same], odq[same], "dq_idx")
     # P and P_idx both sum to one over each row's token set, so the rows' contributions to dK_idx
     # cancel when summed over the tokens: sum_j dK_idx[b, j, :] = 0 up to rounding
     tot = dk.double().sum(dim=1).abs().max().item()
@@ -107,7 +118,7 @@ def test_full_decode_sampled_sequences_match_oracle():
         bad, near = compare_blocks(gb, ob, om)
         assert bad == 0, f"sequence {b}: selection differs (near-ties excluded: {near})"
         same = np.all(gb == ob, axis=-1)[0]
-        og = out[sl].float().cpu().numpy()[0]
+        og = out[sl].cpu().numpy()[0]
         for r in range(w.H_kv):
             if same[r]:
                 check_attention(og[r * G:(r + 1) * G], oo[0, r * G:(r + 1) * G])
