@@ -216,7 +216,7 @@ msa_status msa_sparse_attn_decode(const msa_dims* d, const int32_t* cache_len, c
     a.lse_part = reinterpret_cast<float*>(cv.take((size_t)d->B * d->H_kv * K1 * G * 4));
     a.blocks_out = blocks_out;
     a.status = status;
-    e = run_decode(a, q, q_idx, k_cache, v_cache, k_idx_cache, out, st);
+    e = run_decode(a, q, q_idx, k_cache, v_cache, k_idx_cache, out, num_sms(), st);
     return cuda_status(e);
 }
 

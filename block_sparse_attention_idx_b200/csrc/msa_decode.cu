@@ -16,131 +16,205 @@ namespace msa {
 
 namespace {
 
-constexpr int kScanThreads = 256;
-constexpr int kHkvMax = 8;
 
-// One warp per complete past block of one sequence: the block's index scores for every group and
-// their maximum. A token's d_idx row is split over DI/8 lanes (one 16-byte load each), so one warp
-// load instruction covers whole 128-byte lines; eight rounds of loads are in flight before the
-// first use. Partial dot products are summed over the token's lanes by shuffles.
-template <int DI, int HKV>
-__global__ void __launch_bounds__(kScanThreads, 2) k_dec_scan(DecodeArgs a, const __nv_bfloat16* __restrict__ q_idx,
-                                                           const __nv_bfloat16* __restrict__ k_idx) {
-    constexpr int LPT = DI / 8;    // lanes per token
-    constexpr int TPR = 32 / LPT;  // tokens per warp round
-    constexpr int U = HKV >= 8 ? 4 : 8;  // rounds in flight (fewer when q takes more registers)
-    const int b = blockIdx.y;
-    const int len = a.cache_len[b];
-    const int nfull = (len - 1) / a.block_k;  // complete past blocks (the local block is not scored)
-    const int nb = (a.L + a.block_k - 1) / a.block_k;
+// Index scan: every complete past block of every sequence, its index scores for all groups and
+// their maximum. Persistent CTAs (one per SM): warp 4 streams the blocks' K_idx tiles into an
+// 8-stage shared-memory ring by TMA (128- or 64-byte swizzled rows); warps 0-3 take the ring's
+// tiles in turn and compute S^T = K_idx_tile . Q_idx^T with warp-level mma.sync (16 tokens x 8
+// group columns x 16 dims per instruction, A fragments by ldmatrix from the swizzled tile, the
+// groups' Q_idx as B fragments held in registers); each block's maxima come straight from the
+// accumulators. The kernel is HBM-bound: it reads every K_idx byte once.
+constexpr int kScanStages = 8;
+constexpr int kScanWarps = 4;
+
+template <int DI, int BK>
+struct ScanSmem {
+    alignas(1024) __nv_bfloat16 tile[kScanStages][BK * DI];
+    uint64_t full[kScanStages], empty[kScanStages];
+};
+
+template <int DI, int BK>
+__global__ void __launch_bounds__((kScanWarps + 1) * 32, 1)
+    k_dec_scan(const __grid_constant__ CUtensorMap tm_kidx, DecodeArgs a, const __nv_bfloat16* __restrict__ q_idx) {
+    using Sm = ScanSmem<DI, BK>;
+    extern __shared__ uint8_t scan_raw[];
+    Sm& s = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(scan_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int part = lane % LPT, tsub = lane / LPT;
-    float qv[HKV][8];
-#pragma unroll
-    for (int r = 0; r < HKV; ++r) {
-        const __nv_bfloat162* q2 =
-            reinterpret_cast<const __nv_bfloat162*>(q_idx + ((size_t)b * HKV + r) * DI + part * 8);
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            const float2 f = __bfloat1622float2(q2[x]);
-            qv[r][2 * x] = f.x;
-            qv[r][2 * x + 1] = f.y;
+    const int nb = (a.L + BK - 1) / BK;
+    const int total = a.B * nb;
+    if (threadIdx.x == 0) {
+        for (int x = 0; x < kScanStages; ++x) {
+            mbar_init(&s.full[x], 1);
+            mbar_init(&s.empty[x], 1);
         }
+        fence_mbar_init();
     }
-    for (int blk = blockIdx.x * (kScanThreads / 32) + warp; blk < nfull; blk += gridDim.x * (kScanThreads / 32)) {
-        const __nv_bfloat16* base = k_idx + ((size_t)b * a.L + (size_t)blk * a.block_k) * DI + part * 8;
-        float mx[HKV];
-#pragma unroll
-        for (int r = 0; r < HKV; ++r) mx[r] = -INFINITY;
-        for (int t0 = 0; t0 < a.block_k; t0 += TPR * U) {
-            uint4 u0[U];
-#pragma unroll
-            for (int j = 0; j < U; ++j) {
-                const int tok = t0 + j * TPR + tsub;
-                u0[j] = tok < a.block_k ? __ldcs(reinterpret_cast<const uint4*>(base + (size_t)tok * DI))
-                                        : make_uint4(0, 0, 0, 0);
+    __syncthreads();
+    // the n-th block this CTA processes: global ids blockIdx.x + gridDim.x * j that name a complete
+    // past block of their sequence; producer and consumers walk the same list
+    auto next_valid = [&](int gb) -> int {
+        for (; gb < total; gb += gridDim.x) {
+            const int b = gb / nb, blk = gb % nb;
+            if (blk < (a.cache_len[b] - 1) / BK) return gb;
+        }
+        return total;
+    };
+    if (warp == kScanWarps) {
+        if (lane == 0) {
+            int n = 0;
+            for (int gb = next_valid(blockIdx.x); gb < total; gb = next_valid(gb + gridDim.x), ++n) {
+                const int st = n % kScanStages;
+                if (n >= kScanStages && !mbar_wait(&s.empty[st], ((n / kScanStages) - 1) & 1, a.status, 0x901)) break;
+                mbar_arrive_expect_tx(&s.full[st], (uint32_t)(BK * DI * 2));
+                tma_load_3d(s.tile[st], &tm_kidx, &s.full[st], 0, (gb % nb) * BK, gb / nb);
             }
+            // no copy of ours may still be landing when the CTA leaves
+            for (int m = max(0, n - kScanStages); m < n; ++m)
+                mbar_wait(&s.full[m % kScanStages], (m / kScanStages) & 1, a.status, 0x902);
+        }
+        return;
+    }
+    // consumers: B fragments of Q_idx^T (k = dim, n = group; groups beyond H_kv are zero)
+    const int g = lane >> 2, t4 = lane & 3;
+    int cur_b = -1;
+    uint32_t qb[DI / 16][2];
+    int n = 0;
+    for (int gb = next_valid(blockIdx.x); gb < total; gb = next_valid(gb + gridDim.x), ++n) {
+        if (n % kScanWarps != warp) continue;
+        const int b = gb / nb, blk = gb % nb;
+        if (b != cur_b) {
+            cur_b = b;
+            const uint32_t* qrow = reinterpret_cast<const uint32_t*>(q_idx + ((size_t)b * a.H_kv + min(g, a.H_kv - 1)) * DI);
 #pragma unroll
-            for (int j = 0; j < U; ++j) {
-                float kv[8];
-                const __nv_bfloat162* h0 = reinterpret_cast<const __nv_bfloat162*>(&u0[j]);
-#pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    const float2 f0 = __bfloat1622float2(h0[x]);
-                    kv[2 * x] = f0.x;
-                    kv[2 * x + 1] = f0.y;
-                }
-                const bool valid = t0 + j * TPR + tsub < a.block_k;
-#pragma unroll
-                for (int r = 0; r < HKV; ++r) {
-                    float p = 0.f;
-#pragma unroll
-                    for (int x = 0; x < 8; ++x) p = fmaf(qv[r][x], kv[x], p);
-#pragma unroll
-                    for (int o = 1; o < LPT; o <<= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
-                    if (valid) mx[r] = fmaxf(mx[r], p);
-                }
+            for (int ks = 0; ks < DI / 16; ++ks) {
+                qb[ks][0] = g < a.H_kv ? qrow[8 * ks + t4] : 0u;
+                qb[ks][1] = g < a.H_kv ? qrow[8 * ks + 4 + t4] : 0u;
             }
         }
+        const int st = n % kScanStages;
+        if (!__all_sync(0xffffffffu, mbar_wait(&s.full[st], (n / kScanStages) & 1, a.status, 0x903))) break;
+        const uint32_t base = smem_u32(s.tile[st]);
+        float m0 = -INFINITY, m1 = -INFINITY;  // groups 2*t4, 2*t4+1
 #pragma unroll
-        for (int r = 0; r < HKV; ++r) {
+        for (int mt = 0; mt < BK / 16; ++mt) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            const int row = mt * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
 #pragma unroll
-            for (int o = LPT; o < 32; o <<= 1) mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], o));
+            for (int ks = 0; ks < DI / 16; ++ks) {
+                uint32_t a4[4];
+                const uint32_t addr = base + swz(row, (2 * ks + (lane >> 4)) * 16, DI * 2);
+                asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                             : "=r"(a4[0]), "=r"(a4[1]), "=r"(a4[2]), "=r"(a4[3])
+                             : "r"(addr));
+                mma_16816_bf16(acc, a4, qb[ks][0], qb[ks][1]);
+            }
+            m0 = fmaxf(m0, fmaxf(acc[0], acc[2]));
+            m1 = fmaxf(m1, fmaxf(acc[1], acc[3]));
         }
-        if (lane < HKV) {
-            float v = mx[0];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.empty[st]);
 #pragma unroll
-            for (int r = 1; r < HKV; ++r) v = lane == r ? mx[r] : v;
-            a.bmax[((size_t)b * HKV + lane) * nb + blk] = v;
+        for (int o = 4; o < 32; o <<= 1) {
+            m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
+            m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+        }
+        if (lane < 4) {
+            if (2 * t4 < a.H_kv) a.bmax[((size_t)b * a.H_kv + 2 * t4) * nb + blk] = m0;
+            if (2 * t4 + 1 < a.H_kv) a.bmax[((size_t)b * a.H_kv + 2 * t4 + 1) * nb + blk] = m1;
         }
     }
 }
 
-// One CTA per (sequence, group): Top-k of the block maxima of the complete past blocks by
-// (max desc, id asc), plus the local block; written ascending, -1 padded.
+// One CTA (8 warps) per (sequence, group): Top-k of the block maxima of the complete past blocks by
+// (max desc, id asc), plus the local block; written ascending, -1 padded. Stage 1: warp w takes the
+// candidates [w*chunk, (w+1)*chunk) (lane l: ids w*chunk + l + 32j, at most 32 per lane since the
+// host caps the blocks at 8192; staged in shared memory) and picks its own Top-k by k rounds of warp
+// argmax, each lane rescanning its candidates only when its best was taken. Stage 2: warp 0
+// picks the Top-k of the 8k finalists the same way. Any block of the overall Top-k is in its warp's
+// Top-k, so the two stages select the same set as one pass.
+__device__ __forceinline__ void warp_argmax(float& v, int& id) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, v, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, id, o);
+        if (ov > v || (ov == v && oi < id)) { v = ov; id = oi; }
+    }
+}
+
 __global__ void __launch_bounds__(256) k_dec_topk(DecodeArgs a) {
-    __shared__ unsigned char taken[8192];
-    __shared__ float s_v[8];
-    __shared__ int s_i[8];
-    __shared__ int chosen[17];
+    constexpr int kMaxK = 16;
+    __shared__ float fv[8 * kMaxK];
+    __shared__ int fi[8 * kMaxK];
+    __shared__ int chosen[kMaxK + 1];
+    __shared__ float s_vals[8192];
     const int b = blockIdx.x / a.H_kv, r = blockIdx.x % a.H_kv;
     const int len = a.cache_len[b];
-    const int bi = (len - 1) / a.block_k;
+    const int bi = (len - 1) / a.block_k;  // local block; candidates are 0 .. bi-1
     const int nb = (a.L + a.block_k - 1) / a.block_k;
     const float* vals = a.bmax + ((size_t)b * a.H_kv + r) * nb;
     const int K1 = a.topk + 1;
-    for (int c = threadIdx.x; c < bi; c += blockDim.x) taken[c] = 0;
-    __syncthreads();
     const int take = min(a.topk, bi);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int chunk = (bi + 7) / 8;
+    const int lo = warp * chunk, hi = min(bi, lo + chunk);
+    for (int c = threadIdx.x; c < bi; c += blockDim.x) s_vals[c] = vals[c];
+    __syncthreads();
+    uint32_t taken = 0;
+    float lv = -INFINITY;  // this lane's best remaining candidate
+    int lid = 0x7fffffff;
+    auto rescan = [&]() {
+        lv = -INFINITY;
+        lid = 0x7fffffff;
+        int j = 0;
+        for (int c = lo + lane; c < hi; c += 32, ++j) {
+            if ((taken >> j) & 1u) continue;
+            const float v = s_vals[c];
+            if (v > lv || (v == lv && c < lid)) { lv = v; lid = c; }
+        }
+    };
+    rescan();
+    for (int round = 0; round < take; ++round) {
+        float bv = lv;
+        int bid = lid;
+        warp_argmax(bv, bid);
+        if (bid != 0x7fffffff && lid == bid) {
+            taken |= 1u << ((bid - lo) / 32);
+            rescan();
+        }
+        if (lane == 0) {
+            fv[warp * kMaxK + round] = bv;
+            fi[warp * kMaxK + round] = bid;
+        }
+    }
+    __syncthreads();
+    if (warp != 0) return;
+    uint32_t taken2 = 0;
     for (int round = 0; round < take; ++round) {
         float bv = -INFINITY;
-        int bidx = 0x7fffffff;
-        for (int c = threadIdx.x; c < bi; c += blockDim.x) {
-            if (taken[c]) continue;
-            const float v = vals[c];
-            if (v > bv || (v == bv && c < bidx)) { bv = v; bidx = c; }
+        int bid = 0x7fffffff;
+        for (int m = 0; m < 4; ++m) {
+            const int f = lane + 32 * m;  // finalist f: warp f / take, rank f % take
+            if (f >= 8 * take || ((taken2 >> m) & 1u)) continue;
+            const float v = fv[(f / take) * kMaxK + f % take];
+            const int c = fi[(f / take) * kMaxK + f % take];
+            if (v > bv || (v == bv && c < bid)) { bv = v; bid = c; }
         }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
-            if (ov > bv || (ov == bv && oi < bidx)) { bv = ov; bidx = oi; }
+        float wv = bv;
+        int wid = bid;
+        warp_argmax(wv, wid);
+        if (bid == wid && wid != 0x7fffffff) {  // the lane holding the winner marks it
+            for (int m = 0; m < 4; ++m) {
+                const int f = lane + 32 * m;
+                if (f < 8 * take && !((taken2 >> m) & 1u) && fi[(f / take) * kMaxK + f % take] == wid) {
+                    taken2 |= 1u << m;
+                    break;
+                }
+            }
         }
-        if (lane == 0) { s_v[warp] = bv; s_i[warp] = bidx; }
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            float v = s_v[0];
-            int id = s_i[0];
-            for (int w = 1; w < (int)(blockDim.x / 32); ++w)
-                if (s_v[w] > v || (s_v[w] == v && s_i[w] < id)) { v = s_v[w]; id = s_i[w]; }
-            if (id == 0x7fffffff) id = 0;  // every candidate was -inf; pick the lowest untaken id
-            chosen[round] = id;
-            taken[id] = 1;
-        }
-        __syncthreads();
+        if (lane == 0) chosen[round] = wid == 0x7fffffff ? 0 : wid;
     }
-    if (threadIdx.x == 0) {
+    __syncwarp();
+    if (lane == 0) {
         int n = take;
         chosen[n++] = bi;
         for (int x = 1; x < n; ++x) {  // insertion sort, ascending
@@ -159,27 +233,30 @@ __global__ void __launch_bounds__(256) k_dec_topk(DecodeArgs a) {
 }
 
 // One CTA (4 warps) per (sequence, group, selected slot): attention of the group's G heads over one
-// block. K and V of the block are staged in shared memory as bf16 (rows padded by 16 bytes so the
-// fragment loads are conflict-free) with cp.async, all in flight at once. The G heads are the M=16
-// rows of warp-level mma.sync.m16n8k16 tiles (G=32 takes two row tiles, fewer heads are padded
-// with zero rows); each warp owns 16-token units of the block. S = Q.K^T stays in registers, the
-// row max and sum are combined across the warps in shared memory, P is reused from the S
-// accumulators as the A operand of P.V (V fragments via ldmatrix.trans), and the warps' O tiles
-// are summed in shared memory. Writes the slot's normalised fp32 partial and its LSE.
+// block. K and V are staged in shared memory as bf16 (rows padded by 16 bytes: conflict-free
+// fragment loads) with cp.async, V in a second copy group that lands while S is computed. The G
+// heads are the M=16 rows of warp-level mma.sync.m16n8k16 tiles (G=32 takes two row tiles; fewer
+// heads are padded with zero rows). Warp w computes S = Q.K^T for its 16-token units and the
+// softmax statistics (combined across warps in shared memory), then writes P as bf16 to shared
+// memory; after one barrier each warp computes P.V for a quarter of the output columns over all
+// tokens (P by ldmatrix, V by ldmatrix.trans) and writes them: no atomics, no cross-warp O sum.
+// Output: the slot's partial normalised by the sum of the bf16-rounded P the MMA multiplies (as in
+// the prefill attention), and its LSE from the exact sum.
 template <int D, int BK>
 __global__ void __launch_bounds__(128) k_dec_attn(DecodeArgs a, const __nv_bfloat16* __restrict__ q,
                                                   const __nv_bfloat16* __restrict__ kc,
                                                   const __nv_bfloat16* __restrict__ vc) {
-    constexpr int KP = D + 8;          // padded row (bf16)
+    constexpr int KP = D + 8;          // padded K/V row (bf16)
+    constexpr int PP = BK + 8;         // padded P row (bf16)
     constexpr int NU = BK / 16;        // 16-token units
     constexpr int UPW = (NU + 3) / 4;  // units per warp
+    constexpr int DW = D / 4;          // output columns per warp
     extern __shared__ __align__(16) uint8_t dec_smem[];
     __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(dec_smem);  // [BK][KP]
     __nv_bfloat16* sV = sK + BK * KP;                                 // [BK][KP]
-    float* sO = reinterpret_cast<float*>(sV + BK * KP);               // [16][D]
-    float* sRed = sO + 16 * D;                                        // [4][16] per-warp max, then exact sums
+    __nv_bfloat16* sP = sV + BK * KP;                                 // [16][PP]
+    float* sRed = reinterpret_cast<float*>(sP + 16 * PP);             // [4][16] per-warp max, then exact sums
     float* sRedR = sRed + 64;                                         // [4][16] per-warp rounded sums
-    float* sRow = sRedR + 64;                                         // [3][16]: max (log2), exact sum, rounded sum
     const int G = a.H_q / a.H_kv;
     const int K1 = a.topk + 1;
     const int bs = blockIdx.x;  // b * H_kv + r
@@ -197,15 +274,21 @@ __global__ void __launch_bounds__(128) k_dec_attn(DecodeArgs a, const __nv_bfloa
         const bool ok = (size_t)c * BK + t < (size_t)a.L;
         const size_t go = (((size_t)b * a.L + (ok ? (size_t)c * BK + t : 0)) * a.H_kv + r) * D + c8 * 8;
         cp_async_16_zfill(smem_u32(sK + t * KP + c8 * 8), kc + go, ok);
+    }
+    cp_async_commit();
+    for (int x = threadIdx.x; x < BK * D / 8; x += blockDim.x) {
+        const int t = x / (D / 8), c8 = x % (D / 8);
+        const bool ok = (size_t)c * BK + t < (size_t)a.L;
+        const size_t go = (((size_t)b * a.L + (ok ? (size_t)c * BK + t : 0)) * a.H_kv + r) * D + c8 * 8;
         cp_async_16_zfill(smem_u32(sV + t * KP + c8 * 8), vc + go, ok);
     }
-    cp_async_wait_all();
+    cp_async_commit();
+    cp_async_wait_group<1>();
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
     const float sl2 = a.scale * 1.4426950408889634f;
     float* o_out = a.o_part + ((size_t)bs * K1 + slot) * G * D;
     for (int mt = 0; mt * 16 < G; ++mt) {
-        for (int x = threadIdx.x; x < 16 * D; x += blockDim.x) sO[x] = 0.f;
         // Q fragments: rows h0 = 16mt + g and h1 = h0 + 8 (zero beyond G)
         const int h0 = mt * 16 + g, h1 = h0 + 8;
         const int h0c = min(h0, G - 1), h1c = min(h1, G - 1);  // padded rows read nothing
@@ -229,8 +312,7 @@ __global__ void __launch_bounds__(128) k_dec_attn(DecodeArgs a, const __nv_bfloa
             for (int tl = 0; tl < 2; ++tl) {
                 sc[j][tl][0] = sc[j][tl][1] = sc[j][tl][2] = sc[j][tl][3] = 0.f;
                 if (u < NU) {
-                    const int n0 = 16 * u + 8 * tl;
-                    const uint32_t* krow = reinterpret_cast<const uint32_t*>(sK + (n0 + g) * KP);
+                    const uint32_t* krow = reinterpret_cast<const uint32_t*>(sK + (16 * u + 8 * tl + g) * KP);
 #pragma unroll
                     for (int ks = 0; ks < D / 16; ++ks) mma_16816_bf16(sc[j][tl], qa[ks], krow[8 * ks + t4], krow[8 * ks + 4 + t4]);
                 }
@@ -256,25 +338,26 @@ __global__ void __launch_bounds__(128) k_dec_attn(DecodeArgs a, const __nv_bfloa
         const float m0 = fmaxf(fmaxf(sRed[g], sRed[16 + g]), fmaxf(sRed[32 + g], sRed[48 + g]));
         const float m1 = fmaxf(fmaxf(sRed[8 + g], sRed[24 + g]), fmaxf(sRed[40 + g], sRed[56 + g]));
         __syncthreads();
-        // P; l: exact sums (for the LSE); lr: sums of the bf16-rounded P the MMA multiplies (for the
-        // normalisation, as in the prefill attention)
+        // P (bf16 into shared memory); l: exact sums, lr: sums of the rounded P
         float l0 = 0.f, l1 = 0.f, lr0 = 0.f, lr1 = 0.f;
-        uint32_t pk[UPW][4];
 #pragma unroll
         for (int j = 0; j < UPW; ++j) {
+            const int u = warp + 4 * j;
+            if (u >= NU) continue;
 #pragma unroll
             for (int tl = 0; tl < 2; ++tl) {
+                float p[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float m = e < 2 ? m0 : m1;
-                    const float p = sc[j][tl][e] == -INFINITY ? 0.f : exp2f(sc[j][tl][e] - m);
-                    sc[j][tl][e] = p;
-                    if (e < 2) l0 += p; else l1 += p;
+                    p[e] = sc[j][tl][e] == -INFINITY ? 0.f : exp2f(sc[j][tl][e] - (e < 2 ? m0 : m1));
+                    if (e < 2) l0 += p[e]; else l1 += p[e];
                 }
-                pk[j][2 * tl] = pack_bf16x2(sc[j][tl][0], sc[j][tl][1]);
-                pk[j][2 * tl + 1] = pack_bf16x2(sc[j][tl][2], sc[j][tl][3]);
-                lr0 += __uint_as_float(pk[j][2 * tl] << 16) + __uint_as_float(pk[j][2 * tl] & 0xffff0000u);
-                lr1 += __uint_as_float(pk[j][2 * tl + 1] << 16) + __uint_as_float(pk[j][2 * tl + 1] & 0xffff0000u);
+                const uint32_t w0 = pack_bf16x2(p[0], p[1]), w1 = pack_bf16x2(p[2], p[3]);
+                lr0 += __uint_as_float(w0 << 16) + __uint_as_float(w0 & 0xffff0000u);
+                lr1 += __uint_as_float(w1 << 16) + __uint_as_float(w1 & 0xffff0000u);
+                const int col = 16 * u + 8 * tl + 2 * t4;
+                *reinterpret_cast<uint32_t*>(sP + g * PP + col) = w0;
+                *reinterpret_cast<uint32_t*>(sP + (g + 8) * PP + col) = w1;
             }
         }
 #pragma unroll
@@ -290,50 +373,47 @@ __global__ void __launch_bounds__(128) k_dec_attn(DecodeArgs a, const __nv_bfloa
             sRedR[warp * 16 + g] = lr0;
             sRedR[warp * 16 + g + 8] = lr1;
         }
-        // O = P.V over the warp's units
-        float ov[D / 8][4];
+        if (mt == 0) cp_async_wait_group<0>();
+        __syncthreads();
+        // O[:, warp's columns] = P.V over all tokens
+        float ov[DW / 8][4];
 #pragma unroll
-        for (int nd = 0; nd < D / 8; ++nd) ov[nd][0] = ov[nd][1] = ov[nd][2] = ov[nd][3] = 0.f;
+        for (int nd = 0; nd < DW / 8; ++nd) ov[nd][0] = ov[nd][1] = ov[nd][2] = ov[nd][3] = 0.f;
 #pragma unroll
-        for (int j = 0; j < UPW; ++j) {
-            const int u = warp + 4 * j;
-            if (u >= NU) continue;
-            // A fragment of P: rows g / g+8, tokens 2t4.. of the unit's first and second 8-token tile
-            const uint32_t pa[4] = {pk[j][0], pk[j][1], pk[j][2], pk[j][3]};
-            // lane L addresses row (16u + 8*((L/8)%2) + L%8) of V at column 8*(nd + L/16)
+        for (int u = 0; u < NU; ++u) {
+            uint32_t pa[4];
+            {
+                // A = P rows (heads) x 16 tokens: matrices rows 0-7 / 8-15 at token columns +0 / +8
+                const int prow = ((lane >> 3) & 1) * 8 + (lane & 7), pcol = 16 * u + 8 * (lane >> 4);
+                asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                             : "=r"(pa[0]), "=r"(pa[1]), "=r"(pa[2]), "=r"(pa[3])
+                             : "r"(smem_u32(sP + prow * PP + pcol)));
+            }
             const int vrow = 16 * u + 8 * ((lane >> 3) & 1) + (lane & 7);
 #pragma unroll
-            for (int nd = 0; nd < D / 8; nd += 2) {
+            for (int nd = 0; nd < DW / 8; nd += 2) {
                 uint32_t b00, b01, b10, b11;
-                ldsm_x4_trans(smem_u32(sV + vrow * KP + 8 * (nd + (lane >> 4))), b00, b01, b10, b11);
+                ldsm_x4_trans(smem_u32(sV + vrow * KP + warp * DW + 8 * (nd + (lane >> 4))), b00, b01, b10, b11);
                 mma_16816_bf16(ov[nd], pa, b00, b01);
                 mma_16816_bf16(ov[nd + 1], pa, b10, b11);
             }
         }
-        __syncthreads();
-        if (t4 == 0 && warp == 0) {
-            sRow[g] = m0;
-            sRow[g + 8] = m1;
-            sRow[16 + g] = sRed[g] + sRed[16 + g] + sRed[32 + g] + sRed[48 + g];
-            sRow[16 + g + 8] = sRed[8 + g] + sRed[24 + g] + sRed[40 + g] + sRed[56 + g];
-            sRow[32 + g] = sRedR[g] + sRedR[16 + g] + sRedR[32 + g] + sRedR[48 + g];
-            sRow[32 + g + 8] = sRedR[8 + g] + sRedR[24 + g] + sRedR[40 + g] + sRedR[56 + g];
-        }
+        const float Lr0 = sRedR[g] + sRedR[16 + g] + sRedR[32 + g] + sRedR[48 + g];
+        const float Lr1 = sRedR[8 + g] + sRedR[24 + g] + sRedR[40 + g] + sRedR[56 + g];
+        const float i0 = 1.f / Lr0, i1 = 1.f / Lr1;
 #pragma unroll
-        for (int nd = 0; nd < D / 8; ++nd) {
-            atomicAdd(&sO[g * D + nd * 8 + 2 * t4], ov[nd][0]);
-            atomicAdd(&sO[g * D + nd * 8 + 2 * t4 + 1], ov[nd][1]);
-            atomicAdd(&sO[(g + 8) * D + nd * 8 + 2 * t4], ov[nd][2]);
-            atomicAdd(&sO[(g + 8) * D + nd * 8 + 2 * t4 + 1], ov[nd][3]);
+        for (int nd = 0; nd < DW / 8; ++nd) {
+            const int col = warp * DW + 8 * nd + 2 * t4;
+            if (h0 < G) *reinterpret_cast<float2*>(o_out + (size_t)h0 * D + col) = make_float2(ov[nd][0] * i0, ov[nd][1] * i0);
+            if (h1 < G) *reinterpret_cast<float2*>(o_out + (size_t)h1 * D + col) = make_float2(ov[nd][2] * i1, ov[nd][3] * i1);
         }
-        __syncthreads();
-        for (int x = threadIdx.x; x < 16 * D; x += blockDim.x) {
-            const int hh = x / D, h = mt * 16 + hh;
-            if (h < G) o_out[(size_t)h * D + x % D] = sO[x] / sRow[32 + hh];
+        if (warp == 0 && t4 == 0) {
+            const float L0 = sRed[g] + sRed[16 + g] + sRed[32 + g] + sRed[48 + g];
+            const float L1 = sRed[8 + g] + sRed[24 + g] + sRed[40 + g] + sRed[56 + g];
+            if (h0 < G) lse_out[h0] = m0 * 0.6931471805599453f + logf(L0);
+            if (h1 < G) lse_out[h1] = m1 * 0.6931471805599453f + logf(L1);
         }
-        if (threadIdx.x < 16 && mt * 16 + threadIdx.x < G)
-            lse_out[mt * 16 + threadIdx.x] = sRow[threadIdx.x] * 0.6931471805599453f + logf(sRow[16 + threadIdx.x]);
-        __syncthreads();
+        __syncthreads();  // sP and sRed are rewritten by the next row tile
     }
 }
 
@@ -380,24 +460,32 @@ size_t decode_ws_bytes(int B, int L, int H_q, int H_kv, int d, int block_k, int 
 }
 
 cudaError_t run_decode(const DecodeArgs& a, const void* q, const void* q_idx, const void* k_cache,
-                       const void* v_cache, const void* k_idx_cache, void* out, cudaStream_t st) {
+                       const void* v_cache, const void* k_idx_cache, void* out, int num_sms, cudaStream_t st) {
     const auto* qi = static_cast<const __nv_bfloat16*>(q_idx);
     const auto* ki = static_cast<const __nv_bfloat16*>(k_idx_cache);
-    const int nb = (a.L + a.block_k - 1) / a.block_k;
-    const dim3 sgrid((nb + kScanThreads / 32 - 1) / (kScanThreads / 32), a.B);
     {
         ProfScope ps("dec_scan", st);
-        const bool d64 = a.d_idx == 64;
-        switch (a.H_kv) {
-            case 1: d64 ? k_dec_scan<64, 1><<<sgrid, kScanThreads, 0, st>>>(a, qi, ki)
-                        : k_dec_scan<32, 1><<<sgrid, kScanThreads, 0, st>>>(a, qi, ki); break;
-            case 2: d64 ? k_dec_scan<64, 2><<<sgrid, kScanThreads, 0, st>>>(a, qi, ki)
-                        : k_dec_scan<32, 2><<<sgrid, kScanThreads, 0, st>>>(a, qi, ki); break;
-            case 4: d64 ? k_dec_scan<64, 4><<<sgrid, kScanThreads, 0, st>>>(a, qi, ki)
-                        : k_dec_scan<32, 4><<<sgrid, kScanThreads, 0, st>>>(a, qi, ki); break;
-            default: d64 ? k_dec_scan<64, 8><<<sgrid, kScanThreads, 0, st>>>(a, qi, ki)
-                         : k_dec_scan<32, 8><<<sgrid, kScanThreads, 0, st>>>(a, qi, ki); break;
-        }
+        CUtensorMap tm;
+        if (!make_tmap_3d(&tm, k_idx_cache, (uint64_t)a.d_idx, (uint64_t)a.L, (uint64_t)a.B, (uint64_t)a.d_idx * 2,
+                          (uint64_t)a.L * a.d_idx * 2, (uint32_t)a.d_idx, (uint32_t)a.block_k, 1, a.d_idx * 2))
+            return cudaErrorInvalidValue;
+        auto launch = [&](auto kern, size_t bytes) -> cudaError_t {
+            const size_t smem = bytes + 1024;
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            kern<<<num_sms, (kScanWarps + 1) * 32, smem, st>>>(tm, a, qi);
+            return cudaGetLastError();
+        };
+        cudaError_t e;
+        if (a.d_idx == 64)
+            e = a.block_k == 128 ? launch(k_dec_scan<64, 128>, sizeof(ScanSmem<64, 128>))
+                : a.block_k == 64 ? launch(k_dec_scan<64, 64>, sizeof(ScanSmem<64, 64>))
+                                  : launch(k_dec_scan<64, 32>, sizeof(ScanSmem<64, 32>));
+        else
+            e = a.block_k == 128 ? launch(k_dec_scan<32, 128>, sizeof(ScanSmem<32, 128>))
+                : a.block_k == 64 ? launch(k_dec_scan<32, 64>, sizeof(ScanSmem<32, 64>))
+                                  : launch(k_dec_scan<32, 32>, sizeof(ScanSmem<32, 32>));
+        if (e != cudaSuccess) return e;
     }
     {
         ProfScope ps("dec_topk", st);
@@ -408,7 +496,7 @@ cudaError_t run_decode(const DecodeArgs& a, const void* q, const void* q_idx, co
     const auto* qb = static_cast<const __nv_bfloat16*>(q);
     const auto* kb = static_cast<const __nv_bfloat16*>(k_cache);
     const auto* vb = static_cast<const __nv_bfloat16*>(v_cache);
-    const size_t smem = (size_t)2 * a.block_k * (a.d + 8) * 2 + (size_t)16 * a.d * 4 + (64 + 64 + 48) * 4;
+    const size_t smem = (size_t)2 * a.block_k * (a.d + 8) * 2 + (size_t)16 * (a.block_k + 8) * 2 + 128 * 4;
     auto launch = [&](auto kern) -> cudaError_t {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;

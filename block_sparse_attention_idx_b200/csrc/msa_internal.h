@@ -122,6 +122,6 @@ struct DecodeArgs {
 };
 size_t decode_ws_bytes(int B, int L, int H_q, int H_kv, int d, int block_k, int topk);
 cudaError_t run_decode(const DecodeArgs& a, const void* q, const void* q_idx, const void* k_cache, const void* v_cache,
-                       const void* k_idx_cache, void* out, cudaStream_t st);
+                       const void* k_idx_cache, void* out, int num_sms, cudaStream_t st);
 
 }  // namespace msa

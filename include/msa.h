@@ -123,6 +123,7 @@ MSA_API msa_status msa_sparse_attn_fwd(const msa_dims *dims, const void *q, cons
  *   k_cache, v_cache bf16 [B, N, H_kv, d];  k_idx_cache bf16 [B, N, d_idx]
  *   out        fp32 [B, H_q, d]: the fp32-accumulated result        (output)
  *   blocks_out int32 [B, H_kv, topk+1] or NULL                       (output)
+ * Needs ceil(N / block_k) <= 8192 cache blocks (MSA_ERR_UNSUPPORTED otherwise).
  */
 MSA_API msa_status msa_sparse_attn_decode(const msa_dims *dims, const int32_t *cache_len, const void *q, const void *q_idx,
                                   const void *k_cache, const void *v_cache, const void *k_idx_cache, float *out,
