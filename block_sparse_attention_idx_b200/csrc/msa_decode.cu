@@ -125,28 +125,21 @@ __global__ void __launch_bounds__((kScanWarps + 1) * 32, 1)
     }
 }
 
-// One CTA (8 warps) per (sequence, group): Top-k of the block maxima of the complete past blocks by
-// (max desc, id asc), plus the local block; written ascending, -1 padded. Stage 1: warp w takes the
-// candidates [w*chunk, (w+1)*chunk) (lane l: ids w*chunk + l + 32j, at most 32 per lane since the
-// host caps the blocks at 8192; staged in shared memory) and picks its own Top-k by k rounds of warp
-// argmax, each lane rescanning its candidates only when its best was taken. Stage 2: warp 0
-// picks the Top-k of the 8k finalists the same way. Any block of the overall Top-k is in its warp's
-// Top-k, so the two stages select the same set as one pass.
-__device__ __forceinline__ void warp_argmax(float& v, int& id) {
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, v, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, id, o);
-        if (ov > v || (ov == v && oi < id)) { v = ov; id = oi; }
-    }
-}
-
+// One CTA per (sequence, group): Top-k of the block maxima of the complete past blocks by
+// (max desc, id asc), plus the local block; written ascending, -1 padded. Radix select: candidate c
+// gets the 64-bit key (order-preserving bits of its max) << 32 | (0xffffffff - c), unique and
+// larger for the block that ranks first; 8-bit histogram passes over the keys find the key T of the
+// k-th largest, and exactly the k keys >= T are taken. The leading bytes every key shares (block
+// maxima of one sequence have one sign and nearly one exponent) are read off the smallest and the
+// largest key instead of counted, which would pile every key onto one histogram bin.
 __global__ void __launch_bounds__(256) k_dec_topk(DecodeArgs a) {
     constexpr int kMaxK = 16;
-    __shared__ float fv[8 * kMaxK];
-    __shared__ int fi[8 * kMaxK];
-    __shared__ int chosen[kMaxK + 1];
-    __shared__ float s_vals[8192];
+    extern __shared__ unsigned long long s_key[];  // [blocks per sequence] (at most 8192)
+    __shared__ int hist[256];
+    __shared__ unsigned long long s_prefix;
+    __shared__ int s_want, s_cnt, s_p0;
+    __shared__ unsigned long long s_kmin[8], s_kmax[8];
+    __shared__ int chosen[kMaxK];
     const int b = blockIdx.x / a.H_kv, r = blockIdx.x % a.H_kv;
     const int len = a.cache_len[b];
     const int bi = (len - 1) / a.block_k;  // local block; candidates are 0 .. bi-1
@@ -154,81 +147,98 @@ __global__ void __launch_bounds__(256) k_dec_topk(DecodeArgs a) {
     const float* vals = a.bmax + ((size_t)b * a.H_kv + r) * nb;
     const int K1 = a.topk + 1;
     const int take = min(a.topk, bi);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int chunk = (bi + 7) / 8;
-    const int lo = warp * chunk, hi = min(bi, lo + chunk);
-    for (int c = threadIdx.x; c < bi; c += blockDim.x) s_vals[c] = vals[c];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    unsigned long long kmin = ~0ull, kmax = 0ull;
+    for (int c = tid; c < bi; c += blockDim.x) {
+        const uint32_t u = __float_as_uint(vals[c]);
+        const uint32_t ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+        const unsigned long long k = ((unsigned long long)ord << 32) | (0xffffffffu - (uint32_t)c);
+        s_key[c] = k;
+        kmin = min(kmin, k);
+        kmax = max(kmax, k);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        kmin = min(kmin, (unsigned long long)__shfl_xor_sync(0xffffffffu, kmin, o));
+        kmax = max(kmax, (unsigned long long)__shfl_xor_sync(0xffffffffu, kmax, o));
+    }
+    if (lane == 0) {
+        s_kmin[warp] = kmin;
+        s_kmax[warp] = kmax;
+    }
     __syncthreads();
-    uint32_t taken = 0;
-    float lv = -INFINITY;  // this lane's best remaining candidate
-    int lid = 0x7fffffff;
-    auto rescan = [&]() {
-        lv = -INFINITY;
-        lid = 0x7fffffff;
-        int j = 0;
-        for (int c = lo + lane; c < hi; c += 32, ++j) {
-            if ((taken >> j) & 1u) continue;
-            const float v = s_vals[c];
-            if (v > lv || (v == lv && c < lid)) { lv = v; lid = c; }
+    if (tid == 0) {
+        for (int w = 1; w < 8; ++w) {
+            kmin = min(kmin, s_kmin[w]);
+            kmax = max(kmax, s_kmax[w]);
         }
-    };
-    rescan();
-    for (int round = 0; round < take; ++round) {
-        float bv = lv;
-        int bid = lid;
-        warp_argmax(bv, bid);
-        if (bid != 0x7fffffff && lid == bid) {
-            taken |= 1u << ((bid - lo) / 32);
-            rescan();
+        // bytes above the highest one where the smallest and largest key differ are common to all
+        int p0 = 7;
+        while (p0 > 0 && ((kmin ^ kmax) >> (8 * p0)) == 0) --p0;
+        s_p0 = p0;
+        s_prefix = p0 == 7 ? 0ull : (kmax >> (8 * (p0 + 1)));
+        s_want = take;
+        s_cnt = 0;
+    }
+    __syncthreads();
+    for (int p = s_p0; p >= 0 && take > 0; --p) {
+        hist[tid] = 0;
+        __syncthreads();
+        const unsigned long long prefix = s_prefix;
+        const int shift = 8 * p;
+        for (int c = tid; c < bi; c += blockDim.x) {
+            const unsigned long long k = s_key[c];
+            if (p == 7 || (k >> (shift + 8)) == prefix) atomicAdd(&hist[(int)((k >> shift) & 255u)], 1);
         }
-        if (lane == 0) {
-            fv[warp * kMaxK + round] = bv;
-            fi[warp * kMaxK + round] = bid;
+        __syncthreads();
+        if (warp == 0) {
+            // lane l owns digits 255-8l .. 248-8l, visited from the top
+            int cnt[8], sum = 0;
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+                cnt[x] = hist[255 - 8 * lane - x];
+                sum += cnt[x];
+            }
+            int above = sum;  // inclusive prefix over lanes, then made exclusive
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, above, o);
+                if (lane >= o) above += t;
+            }
+            above -= sum;
+            const int want = s_want;
+            int run = above;
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+                if (run < want && want <= run + cnt[x]) {
+                    s_prefix = (prefix << 8) | (unsigned long long)(255 - 8 * lane - x);
+                    s_want = want - run;
+                }
+                run += cnt[x];
+            }
         }
+        __syncthreads();
+    }
+    const unsigned long long T = s_prefix;
+    if (take > 0) {
+        for (int c = tid; c < bi; c += blockDim.x)
+            if (s_key[c] >= T) chosen[atomicAdd(&s_cnt, 1)] = c;
     }
     __syncthreads();
     if (warp != 0) return;
-    uint32_t taken2 = 0;
-    for (int round = 0; round < take; ++round) {
-        float bv = -INFINITY;
-        int bid = 0x7fffffff;
-        for (int m = 0; m < 4; ++m) {
-            const int f = lane + 32 * m;  // finalist f: warp f / take, rank f % take
-            if (f >= 8 * take || ((taken2 >> m) & 1u)) continue;
-            const float v = fv[(f / take) * kMaxK + f % take];
-            const int c = fi[(f / take) * kMaxK + f % take];
-            if (v > bv || (v == bv && c < bid)) { bv = v; bid = c; }
-        }
-        float wv = bv;
-        int wid = bid;
-        warp_argmax(wv, wid);
-        if (bid == wid && wid != 0x7fffffff) {  // the lane holding the winner marks it
-            for (int m = 0; m < 4; ++m) {
-                const int f = lane + 32 * m;
-                if (f < 8 * take && !((taken2 >> m) & 1u) && fi[(f / take) * kMaxK + f % take] == wid) {
-                    taken2 |= 1u << m;
-                    break;
-                }
-            }
-        }
-        if (lane == 0) chosen[round] = wid == 0x7fffffff ? 0 : wid;
-    }
-    __syncwarp();
-    if (lane == 0) {
-        int n = take;
-        chosen[n++] = bi;
-        for (int x = 1; x < n; ++x) {  // insertion sort, ascending
-            const int v = chosen[x];
-            int y = x - 1;
-            while (y >= 0 && chosen[y] > v) { chosen[y + 1] = chosen[y]; --y; }
-            chosen[y + 1] = v;
-        }
-        int32_t* out = a.sel + ((size_t)b * a.H_kv + r) * K1;
-        for (int x = 0; x < K1; ++x) out[x] = x < n ? chosen[x] : -1;
-        if (a.blocks_out) {
-            int32_t* bo = a.blocks_out + ((size_t)b * a.H_kv + r) * K1;
-            for (int x = 0; x < K1; ++x) bo[x] = x < n ? chosen[x] : -1;
-        }
+    // the chosen ids plus the local block, ascending: each lane places its id by its rank
+    const int n = take + 1;
+    const int mine = lane < take ? chosen[lane] : (lane == take ? bi : 0x7fffffff);
+    int rank = 0;
+    for (int x = 0; x < n; ++x) rank += (__shfl_sync(0xffffffffu, mine, x) < mine);
+    int32_t* out = a.sel + ((size_t)b * a.H_kv + r) * K1;
+    int32_t* bo = a.blocks_out ? a.blocks_out + ((size_t)b * a.H_kv + r) * K1 : nullptr;
+    if (lane < n) {
+        out[rank] = mine;
+        if (bo) bo[rank] = mine;
+    } else if (lane < K1) {
+        out[lane] = -1;
+        if (bo) bo[lane] = -1;
     }
 }
 
@@ -283,18 +293,17 @@ __global__ void __launch_bounds__(128) k_dec_attn(DecodeArgs a, const __nv_bfloa
         cp_async_16_zfill(smem_u32(sV + t * KP + c8 * 8), vc + go, ok);
     }
     cp_async_commit();
-    cp_async_wait_group<1>();
-    __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
     const float sl2 = a.scale * 1.4426950408889634f;
     float* o_out = a.o_part + ((size_t)bs * K1 + slot) * G * D;
-    for (int mt = 0; mt * 16 < G; ++mt) {
-        // Q fragments: rows h0 = 16mt + g and h1 = h0 + 8 (zero beyond G)
+    // Q fragments of a row tile: rows h0 = 16mt + g and h1 = h0 + 8 (zero beyond G); the first
+    // tile's are loaded while K and V are still in flight
+    uint32_t qa[D / 16][4];
+    auto load_q = [&](int mt) {
         const int h0 = mt * 16 + g, h1 = h0 + 8;
         const int h0c = min(h0, G - 1), h1c = min(h1, G - 1);  // padded rows read nothing
         const uint32_t* q0 = reinterpret_cast<const uint32_t*>(q + ((size_t)b * a.H_q + (size_t)r * G + h0c) * D);
         const uint32_t* q1 = reinterpret_cast<const uint32_t*>(q + ((size_t)b * a.H_q + (size_t)r * G + h1c) * D);
-        uint32_t qa[D / 16][4];
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
             qa[ks][0] = h0 < G ? q0[8 * ks + t4] : 0u;
@@ -302,6 +311,13 @@ __global__ void __launch_bounds__(128) k_dec_attn(DecodeArgs a, const __nv_bfloa
             qa[ks][2] = h0 < G ? q0[8 * ks + 4 + t4] : 0u;
             qa[ks][3] = h1 < G ? q1[8 * ks + 4 + t4] : 0u;
         }
+    };
+    load_q(0);
+    cp_async_wait_group<1>();
+    __syncthreads();
+    for (int mt = 0; mt * 16 < G; ++mt) {
+        const int h0 = mt * 16 + g, h1 = h0 + 8;
+        if (mt > 0) load_q(mt);
         // S (log2 units) of the warp's units; tokens past the query are -inf
         float sc[UPW][2][4];
         float mx0 = -INFINITY, mx1 = -INFINITY;
@@ -417,9 +433,12 @@ __global__ void __launch_bounds__(128) k_dec_attn(DecodeArgs a, const __nv_bfloa
     }
 }
 
-// One warp per (sequence, head): merge the slot partials.
+// One warp per (sequence, head): merge the slot partials ("2.4" page eq (18)). Lane s holds slot s's
+// LSE (at most 32 slots); the max and the weights come from warp shuffles, and every slot's partial
+// load is issued before the first is used.
 template <int D>
 __global__ void k_dec_combine(DecodeArgs a, float* __restrict__ out) {
+    constexpr int kMaxK1 = 17;
     const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (w >= a.B * a.H_q) return;
@@ -427,21 +446,31 @@ __global__ void k_dec_combine(DecodeArgs a, float* __restrict__ out) {
     const int K1 = a.topk + 1;
     const int b = w / a.H_q, h = w % a.H_q, r = h / G, hg = h % G;
     const size_t bs = (size_t)b * a.H_kv + r;
-    float mx = -INFINITY;
-    for (int s = 0; s < K1; ++s) mx = fmaxf(mx, a.lse_part[(bs * K1 + s) * G + hg]);
+    const float my_l = lane < K1 ? a.lse_part[(bs * K1 + lane) * G + hg] : -INFINITY;
+    float mx = my_l;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float my_w = my_l == -INFINITY ? 0.f : __expf(my_l - mx);
+    float z = my_w;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
     constexpr int kPer = D / 32;
+    float ov[kMaxK1][kPer];
+#pragma unroll
+    for (int s = 0; s < kMaxK1; ++s) {
+        const float* op = a.o_part + ((bs * K1 + s) * G + hg) * D + lane * kPer;
+        const bool live = s < K1 && __shfl_sync(0xffffffffu, my_w, s) > 0.f;
+#pragma unroll
+        for (int x = 0; x < kPer; ++x) ov[s][x] = live ? op[x] : 0.f;
+    }
     float acc[kPer];
 #pragma unroll
     for (int x = 0; x < kPer; ++x) acc[x] = 0.f;
-    float z = 0.f;
-    for (int s = 0; s < K1; ++s) {
-        const float l = a.lse_part[(bs * K1 + s) * G + hg];
-        if (l == -INFINITY) continue;
-        const float wg = __expf(l - mx);
-        z += wg;
-        const float* op = a.o_part + ((bs * K1 + s) * G + hg) * D + lane * kPer;
 #pragma unroll
-        for (int x = 0; x < kPer; ++x) acc[x] = fmaf(wg, op[x], acc[x]);
+    for (int s = 0; s < kMaxK1; ++s) {
+        const float ws = __shfl_sync(0xffffffffu, my_w, s);
+#pragma unroll
+        for (int x = 0; x < kPer; ++x) acc[x] = fmaf(ws, ov[s][x], acc[x]);
     }
     const float inv = 1.f / z;
     float* o = out + ((size_t)b * a.H_q + h) * D + lane * kPer;
@@ -462,7 +491,6 @@ size_t decode_ws_bytes(int B, int L, int H_q, int H_kv, int d, int block_k, int 
 cudaError_t run_decode(const DecodeArgs& a, const void* q, const void* q_idx, const void* k_cache,
                        const void* v_cache, const void* k_idx_cache, void* out, int num_sms, cudaStream_t st) {
     const auto* qi = static_cast<const __nv_bfloat16*>(q_idx);
-    const auto* ki = static_cast<const __nv_bfloat16*>(k_idx_cache);
     {
         ProfScope ps("dec_scan", st);
         CUtensorMap tm;
@@ -489,7 +517,10 @@ cudaError_t run_decode(const DecodeArgs& a, const void* q, const void* q_idx, co
     }
     {
         ProfScope ps("dec_topk", st);
-        k_dec_topk<<<a.B * a.H_kv, 256, 0, st>>>(a);
+        const size_t ksmem = (size_t)((a.L + a.block_k - 1) / a.block_k) * sizeof(unsigned long long);
+        cudaError_t e = cudaFuncSetAttribute(k_dec_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ksmem);
+        if (e != cudaSuccess) return e;
+        k_dec_topk<<<a.B * a.H_kv, 256, ksmem, st>>>(a);
     }
     ProfScope ps("dec_attn_combine", st);
     const dim3 agrid(a.B * a.H_kv, a.topk + 1);
