@@ -130,6 +130,14 @@ __device__ __forceinline__ void cp_async_16_zfill(uint32_t dst, const void* src,
                  : "memory");
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// A kernel launched with programmatic stream serialisation may start while its predecessor in the
+// stream finishes; it must call pdl_wait() before touching anything the predecessor writes. A
+// predecessor calls pdl_trigger() when a CTA's work is done, so the successor launches only once
+// every CTA of the predecessor has reached that point (none of them can still be waiting for a slot).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ warp-level mma (small M)
 // Four 8x8 b16 matrices from shared memory, transposed: with row addresses of a row-major [k][n]
 // tile, each thread receives the (k = 2(lane%4), 2(lane%4)+1; n = lane/4) pairs a B operand needs.

@@ -16,6 +16,22 @@ namespace msa {
 
 namespace {
 
+// Launch after the previous kernel of the stream with programmatic serialisation (see pdl_wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 
 // Index scan: every complete past block of every sequence, its index scores for all groups and
 // their maximum. Persistent CTAs (one per SM): warp 4 streams the blocks' K_idx tiles into an
@@ -72,6 +88,7 @@ __global__ void __launch_bounds__((kScanWarps + 1) * 32, 1)
             for (int m = max(0, n - kScanStages); m < n; ++m)
                 mbar_wait(&s.full[m % kScanStages], (m / kScanStages) & 1, a.status, 0x902);
         }
+        pdl_trigger();
         return;
     }
     // consumers: B fragments of Q_idx^T (k = dim, n = group; groups beyond H_kv are zero)
@@ -123,23 +140,27 @@ __global__ void __launch_bounds__((kScanWarps + 1) * 32, 1)
             if (2 * t4 + 1 < a.H_kv) a.bmax[((size_t)b * a.H_kv + 2 * t4 + 1) * nb + blk] = m1;
         }
     }
+    pdl_trigger();
 }
 
 // One CTA per (sequence, group): Top-k of the block maxima of the complete past blocks by
 // (max desc, id asc), plus the local block; written ascending, -1 padded. Radix select: candidate c
 // gets the 64-bit key (order-preserving bits of its max) << 32 | (0xffffffff - c), unique and
-// larger for the block that ranks first; 8-bit histogram passes over the keys find the key T of the
-// k-th largest, and exactly the k keys >= T are taken. The leading bytes every key shares (block
-// maxima of one sequence have one sign and nearly one exponent) are read off the smallest and the
-// largest key instead of counted, which would pile every key onto one histogram bin.
+// larger for the block that ranks first. Byte by byte from the first byte where the smallest and
+// largest keys differ (the bytes above it are common to all), a histogram finds the bin that holds
+// the k-th largest key; once that boundary bin holds at most 256 keys, the keys of higher bins are
+// taken and the boundary keys are ranked against each other directly.
 __global__ void __launch_bounds__(256) k_dec_topk(DecodeArgs a) {
     constexpr int kMaxK = 16;
+    constexpr int kList = 256;
     extern __shared__ unsigned long long s_key[];  // [blocks per sequence] (at most 8192)
     __shared__ int hist[256];
+    __shared__ unsigned long long s_list[kList];
     __shared__ unsigned long long s_prefix;
-    __shared__ int s_want, s_cnt, s_p0;
+    __shared__ int s_want, s_bin, s_cnt, s_nlist, s_p0;
     __shared__ unsigned long long s_kmin[8], s_kmax[8];
     __shared__ int chosen[kMaxK];
+    pdl_wait();  // the block maxima come from the scan
     const int b = blockIdx.x / a.H_kv, r = blockIdx.x % a.H_kv;
     const int len = a.cache_len[b];
     const int bi = (len - 1) / a.block_k;  // local block; candidates are 0 .. bi-1
@@ -172,16 +193,17 @@ __global__ void __launch_bounds__(256) k_dec_topk(DecodeArgs a) {
             kmin = min(kmin, s_kmin[w]);
             kmax = max(kmax, s_kmax[w]);
         }
-        // bytes above the highest one where the smallest and largest key differ are common to all
         int p0 = 7;
         while (p0 > 0 && ((kmin ^ kmax) >> (8 * p0)) == 0) --p0;
         s_p0 = p0;
         s_prefix = p0 == 7 ? 0ull : (kmax >> (8 * (p0 + 1)));
         s_want = take;
         s_cnt = 0;
+        s_nlist = 0;
     }
     __syncthreads();
-    for (int p = s_p0; p >= 0 && take > 0; --p) {
+    int p = s_p0;
+    for (; take > 0; --p) {
         hist[tid] = 0;
         __syncthreads();
         const unsigned long long prefix = s_prefix;
@@ -199,7 +221,7 @@ __global__ void __launch_bounds__(256) k_dec_topk(DecodeArgs a) {
                 cnt[x] = hist[255 - 8 * lane - x];
                 sum += cnt[x];
             }
-            int above = sum;  // inclusive prefix over lanes, then made exclusive
+            int above = sum;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int t = __shfl_up_sync(0xffffffffu, above, o);
@@ -213,18 +235,34 @@ __global__ void __launch_bounds__(256) k_dec_topk(DecodeArgs a) {
                 if (run < want && want <= run + cnt[x]) {
                     s_prefix = (prefix << 8) | (unsigned long long)(255 - 8 * lane - x);
                     s_want = want - run;
+                    s_bin = cnt[x];
                 }
                 run += cnt[x];
             }
         }
         __syncthreads();
+        if (s_bin <= kList || p == 0) break;
     }
-    const unsigned long long T = s_prefix;
     if (take > 0) {
-        for (int c = tid; c < bi; c += blockDim.x)
-            if (s_key[c] >= T) chosen[atomicAdd(&s_cnt, 1)] = c;
+        // keys above the boundary bin are taken; the boundary bin's keys are listed and ranked
+        const unsigned long long P = s_prefix;
+        const int shift = 8 * p;
+        for (int c = tid; c < bi; c += blockDim.x) {
+            const unsigned long long top = s_key[c] >> shift;
+            if (top > P) chosen[atomicAdd(&s_cnt, 1)] = c;
+            else if (top == P) s_list[atomicAdd(&s_nlist, 1)] = s_key[c];
+        }
+        __syncthreads();
+        const int nlist = s_nlist, want = s_want;
+        if (tid < nlist) {
+            const unsigned long long mk = s_list[tid];
+            int rank = 0;
+            for (int j = 0; j < nlist; ++j) rank += s_list[j] > mk;
+            if (rank < want) chosen[atomicAdd(&s_cnt, 1)] = (int)(0xffffffffu - (uint32_t)(mk & 0xffffffffu));
+        }
     }
     __syncthreads();
+    pdl_trigger();
     if (warp != 0) return;
     // the chosen ids plus the local block, ascending: each lane places its id by its rank
     const int n = take + 1;
@@ -272,10 +310,12 @@ __global__ void __launch_bounds__(128) k_dec_attn(DecodeArgs a, const __nv_bfloa
     const int bs = blockIdx.x;  // b * H_kv + r
     const int slot = blockIdx.y;
     const int b = bs / a.H_kv, r = bs % a.H_kv;
+    pdl_wait();  // the selection comes from the Top-k
     const int c = a.sel[(size_t)bs * K1 + slot];
     float* lse_out = a.lse_part + ((size_t)bs * K1 + slot) * G;
     if (c < 0) {
         for (int h = threadIdx.x; h < G; h += blockDim.x) lse_out[h] = -INFINITY;
+        pdl_trigger();
         return;
     }
     const int len = a.cache_len[b];
@@ -431,6 +471,7 @@ __global__ void __launch_bounds__(128) k_dec_attn(DecodeArgs a, const __nv_bfloa
         }
         __syncthreads();  // sP and sRed are rewritten by the next row tile
     }
+    pdl_trigger();
 }
 
 // One warp per (sequence, head): merge the slot partials ("2.4" page eq (18)). Lane s holds slot s's
@@ -446,6 +487,7 @@ __global__ void k_dec_combine(DecodeArgs a, float* __restrict__ out) {
     const int K1 = a.topk + 1;
     const int b = w / a.H_q, h = w % a.H_q, r = h / G, hg = h % G;
     const size_t bs = (size_t)b * a.H_kv + r;
+    pdl_wait();  // the partials come from the attention
     const float my_l = lane < K1 ? a.lse_part[(bs * K1 + lane) * G + hg] : -INFINITY;
     float mx = my_l;
 #pragma unroll
@@ -520,7 +562,8 @@ cudaError_t run_decode(const DecodeArgs& a, const void* q, const void* q_idx, co
         const size_t ksmem = (size_t)((a.L + a.block_k - 1) / a.block_k) * sizeof(unsigned long long);
         cudaError_t e = cudaFuncSetAttribute(k_dec_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ksmem);
         if (e != cudaSuccess) return e;
-        k_dec_topk<<<a.B * a.H_kv, 256, ksmem, st>>>(a);
+        e = launch_pdl(k_dec_topk, dim3(a.B * a.H_kv), dim3(256), ksmem, st, a);
+        if (e != cudaSuccess) return e;
     }
     ProfScope ps("dec_attn_combine", st);
     const dim3 agrid(a.B * a.H_kv, a.topk + 1);
@@ -531,20 +574,23 @@ cudaError_t run_decode(const DecodeArgs& a, const void* q, const void* q_idx, co
     auto launch = [&](auto kern) -> cudaError_t {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kern<<<agrid, 128, smem, st>>>(a, qb, kb, vb);
-        return cudaGetLastError();
+        return launch_pdl(kern, agrid, dim3(128), smem, st, a, qb, kb, vb);
     };
     cudaError_t e;
     if (a.d == 128) {
         e = a.block_k == 128 ? launch(k_dec_attn<128, 128>) : a.block_k == 64 ? launch(k_dec_attn<128, 64>)
                                                                                : launch(k_dec_attn<128, 32>);
         if (e != cudaSuccess) return e;
-        k_dec_combine<128><<<(a.B * a.H_q * 32 + 255) / 256, 256, 0, st>>>(a, static_cast<float*>(out));
+        e = launch_pdl(k_dec_combine<128>, dim3((a.B * a.H_q * 32 + 255) / 256), dim3(256), 0, st, a,
+                       static_cast<float*>(out));
+        if (e != cudaSuccess) return e;
     } else {
         e = a.block_k == 128 ? launch(k_dec_attn<64, 128>) : a.block_k == 64 ? launch(k_dec_attn<64, 64>)
                                                                               : launch(k_dec_attn<64, 32>);
         if (e != cudaSuccess) return e;
-        k_dec_combine<64><<<(a.B * a.H_q * 32 + 255) / 256, 256, 0, st>>>(a, static_cast<float*>(out));
+        e = launch_pdl(k_dec_combine<64>, dim3((a.B * a.H_q * 32 + 255) / 256), dim3(256), 0, st, a,
+                       static_cast<float*>(out));
+        if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
 }
