@@ -130,34 +130,83 @@ __global__ void k_lse_idx_merge(KlArgs a) {
 }
 
 // ============================================================================ KL kernel
-constexpr int kQpcMax = 64;  // queries per item when G >= 2
+// tf32 operand (round to nearest) of a float; bf16 values are exact in tf32.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ uint32_t bf16_as_tf32(__nv_bfloat16 x) {
+    return (uint32_t)(*reinterpret_cast<const uint16_t*>(&x)) << 16;
+}
+// D += A(16x8, tf32, row) * B(8x8, tf32, col), fp32 accumulate.
+__device__ __forceinline__ void mma_1688_tf32(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 
-template <int D, int DI>
+// Four (or two) 8x8 b16 matrices from shared memory, not transposed.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+// 4-, 8- or 16-byte asynchronous copy global -> shared.
+template <int BYTES>
+__device__ __forceinline__ void cp_async_ca(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(dst), "l"(src), "n"(BYTES) : "memory");
+}
+// One arrival on `bar` once every cp.async this thread issued so far has landed (counted in the
+// barrier's expected arrivals).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// x ~= hi + lo with both parts tf32: products with a tf32-exact operand keep ~fp32 accuracy.
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+    hi = to_tf32(x);
+    lo = to_tf32(x - __uint_as_float(hi));
+}
+
+// Row pitches keep the mma fragment loads of a warp on distinct banks (or at most two-way).
+template <int D, int DI, int QPC>
 struct KlSmem {
+    static constexpr int KBP = DI + 8;   // K_idx / Q_idx bf16 rows
+    static constexpr int GSP = QPC + 4;  // gradient rows [token][query]
+    static constexpr int SIP = QPC + 1;  // index log-probability / KL rows [token][query]
     alignas(1024) uint8_t q[2][kRows * D * 2];
-    alignas(1024) uint8_t k[kRows * D * 2];  // 128 token rows (rows >= block_k unused)
-    float kf[kRows][DI + 1];                 // K_idx rows of the current block (float, padded)
-    float gs[kRows][kQpcMax + 1];            // [token][query] scaled gradient g * scale_idx
-    float klw[4][kQpcMax];                   // per-warp KL sums
-    float lse[2][kRows];                     // LSE_main of the item rows
-    float qf[2][kQpcMax][DI];                // Q_idx of the item queries (float)
-    float lidx[2][kQpcMax];                  // LSE_idx of the item queries
-    int qi[2][kQpcMax], qslot[2][kQpcMax];
-    uint64_t q_full[2], q_empty[2], kv_full, kv_empty, s_full, s_free, drain;
+    alignas(1024) uint8_t k[kRows * D * 2];      // 128 token rows (rows >= block_k unused)
+    alignas(16) __nv_bfloat16 kb[kRows * KBP];   // K_idx rows of the current block (zero past the end)
+    alignas(16) __nv_bfloat16 qb[2][QPC * KBP];  // Q_idx rows of the item queries
+    alignas(16) float lse[2][kRows];             // LSE_main of the item rows (query-major, head-minor)
+    float gs[kRows * GSP];                       // g * scale_idx per (token, query)
+    float sidx[kRows * SIP];                     // log P_idx per (token, query), then the KL terms
+    float lidx[2][QPC];                          // LSE_idx of the item queries
+    int qi[2][QPC], qslot[2][QPC];
+    int4 rec[2];                                 // item: L, count, new K tile, last item of its tile
+    uint64_t q_full[2], q_empty[2], kv_full, kv_empty, s_full[2], s_free[2], drain;
     uint32_t tmem_base;
     int abort;
 };
 
 template <int D, int DI, int G>
 __global__ void __launch_bounds__(kThreads, 1)
-    k_kl_kv_outer(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restrict__ q,
-                  const __nv_bfloat16* __restrict__ q_idx, const __nv_bfloat16* __restrict__ k_idx, KlArgs a) {
-    using Sm = KlSmem<D, DI>;
+    k_kl_kv_outer(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ q_idx,
+                  const __nv_bfloat16* __restrict__ k_idx, KlArgs a) {
+    constexpr int QPC = kRows / G;
+    using Sm = KlSmem<D, DI, QPC>;
+    constexpr int KBP = Sm::KBP, GSP = Sm::GSP, SIP = Sm::SIP;
     extern __shared__ uint8_t smem_raw[];
     Sm& s = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr uint32_t kIdesc = umma_idesc_bf16(kRows, kRows, false, false);
-    constexpr int QPC = kRows / G;
-    static_assert(QPC <= kQpcMax, "KL items hold at most 64 queries");
+    static_assert(QPC % 8 == 0 && QPC <= 64, "KL items hold 8 to 64 queries");
+    static_assert(DI % 16 == 0, "index head dim must be a multiple of 16");
 
     const int K1 = a.topk + 1;
     const int BK = a.block_k;
@@ -170,19 +219,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int x = 0; x < 2; ++x) {
-            mbar_init(&s.q_full[x], 1);
+            mbar_init(&s.q_full[x], 1 + 32);
             mbar_init(&s.q_empty[x], 1 + kRows);
+            mbar_init(&s.s_full[x], 1);
+            mbar_init(&s.s_free[x], kRows);
         }
         mbar_init(&s.kv_full, 1);
         mbar_init(&s.kv_empty, 1);
-        mbar_init(&s.s_full, 1);
-        mbar_init(&s.s_free, kRows);
         mbar_init(&s.drain, 1);
         s.abort = 0;
         fence_mbar_init();
     }
+    if (warp < 4) {
+        // Q_idx rows past an item's count are read by the gradient mma (times a zero gradient), so
+        // they must hold finite values: start from zeros.
+        uint32_t* z = reinterpret_cast<uint32_t*>(s.qb);
+        for (int x = threadIdx.x; x < 2 * QPC * KBP / 2; x += kRows) z[x] = 0u;
+    }
     if (warp == 5) {
-        tmem_alloc(&s.tmem_base, 128);
+        tmem_alloc(&s.tmem_base, 256);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -191,92 +246,137 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = s.tmem_base;
 
     if (warp == 4) {
-        // ---------------------------------------------------------------- loads + item metadata
-        int kv_loads = 0, prevL = -1;
-        int ok = 1;
-        for (int t = t0, n = 0; t < t1 && ok; ++t, ++n) {
-            const int4 itm = cs.items[t];
+        // ---------------------------------------------------------------- loads + item records
+        // The record and entries of the next item are fetched while the current one is issued, and
+        // every copy is asynchronous: this warp never waits on a global load of the current item.
+        constexpr int EPL = (QPC + 31) / 32;
+        int kv_loads = 0, prevL = -1, issued = 0;
+        bool ok = true;
+        int4 itm = make_int4(0, 0, 0, 0);
+        int e[EPL];
+        if (t0 < t1) itm = cs.items[t0];
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) e[j] = (t0 < t1 && lane + 32 * j < itm.z) ? cs.entries[itm.y + lane + 32 * j] : 0;
+        for (int t = t0, n = 0; t < t1; ++t, ++n) {
+            int4 nitm = make_int4(-1, 0, 0, 0);
+            int ne[EPL];
+            if (t + 1 < t1) nitm = cs.items[t + 1];
+#pragma unroll
+            for (int j = 0; j < EPL; ++j)
+                ne[j] = (t + 1 < t1 && lane + 32 * j < nitm.z) ? cs.entries[nitm.y + lane + 32 * j] : 0;
             const int L = itm.x, count = itm.z;
             const int c = L % cs.nb, r = (L / cs.nb) % a.H_kv, b = L / (cs.nb * a.H_kv);
             const int buf = n & 1;
-            if (lane == 0) ok = mbar_wait(&s.q_empty[buf], ((n >> 1) & 1) ^ 1, a.status, 0x801);
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
-            const int* ent = cs.entries + itm.y;
-            for (int m = lane; m < QPC; m += 32) {
-                const int e = m < count ? ent[m] : 0;
-                s.qi[buf][m] = m < count ? (e >> 5) : -1;
-                s.qslot[buf][m] = e & 31;
-                s.lidx[buf][m] = m < count ? a.lse_idx[((size_t)b * a.N + (e >> 5)) * a.H_kv + r] : 0.f;
+            int okl = 1;
+            if (lane == 0) okl = mbar_wait(&s.q_empty[buf], ((n >> 1) & 1) ^ 1, a.status, 0x801);
+            if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) {
+                const int m = lane + 32 * j;
+                if (m < QPC) {
+                    s.qi[buf][m] = m < count ? (e[j] >> 5) : -1;
+                    s.qslot[buf][m] = e[j] & 31;
+                }
             }
+            if (lane == 0) s.rec[buf] = make_int4(L, count, L != prevL, nitm.x != L);
             __syncwarp();
-            for (int x = lane; x < count * G; x += 32) {
-                const int m = x / G, h = x % G;
-                s.lse[buf][x] = a.lse[((size_t)b * a.N + s.qi[buf][m]) * a.H_q + (size_t)r * G + h];
+            // LSE_idx of each query, LSE_main of its G heads, its Q_idx row
+            for (int m = lane; m < count; m += 32)
+                cp_async_ca<4>(smem_u32(&s.lidx[buf][m]), a.lse_idx + ((size_t)b * a.N + s.qi[buf][m]) * a.H_kv + r);
+            constexpr int LB = G * 4 >= 16 ? 16 : G * 4;  // bytes per copy of one query's LSE_main
+            constexpr int LPQ = G * 4 / LB;
+            for (int x = lane; x < count * LPQ; x += 32) {
+                const int m = x / LPQ, part = x % LPQ;
+                const float* src = a.lse + ((size_t)b * a.N + s.qi[buf][m]) * a.H_q + (size_t)r * G + part * (LB / 4);
+                cp_async_ca<LB>(smem_u32(&s.lse[buf][m * G + part * (LB / 4)]), src);
             }
-            for (int x = lane; x < count * DI; x += 32) {
-                const int m = x / DI, dd = x % DI;
-                s.qf[buf][m][dd] = __bfloat162float(q_idx[(((size_t)b * a.N + s.qi[buf][m]) * a.H_kv + r) * DI + dd]);
+            constexpr int QIC = DI / 8;  // 16-byte chunks per Q_idx row
+            for (int x = lane; x < count * QIC; x += 32) {
+                const int m = x / QIC, part = x % QIC;
+                const __nv_bfloat16* src = q_idx + (((size_t)b * a.N + s.qi[buf][m]) * a.H_kv + r) * DI + part * 8;
+                cp_async_ca<16>(smem_u32(&s.qb[buf][m * KBP + part * 8]), src);
             }
-            const uint32_t qs = smem_u32(s.q[buf]);
-            constexpr int kChunksPerRow = D * 2 / 16;
-            const int nchunks = count * G * kChunksPerRow;
-            for (int x = lane; x < nchunks; x += 32) {
-                const int row = x / kChunksPerRow, ch = x % kChunksPerRow;
-                const int m = row / G, h = row % G;
-                const __nv_bfloat16* src =
-                    q + ((((size_t)b * a.N + s.qi[buf][m]) * a.H_q + (size_t)r * G + h) * D + ch * 8);
-                cp_async_16(qs + ((ch * 16) / 128) * (kRows * 128) + swz(row, (ch * 16) % 128, 128), src);
+            // Q: the G head rows of each query, in the 128B-swizzled K-major tile the MMA reads
+            if constexpr (G >= 8) {
+                if (lane == 0) mbar_arrive_expect_tx(&s.q_full[buf], (uint32_t)(count * G * D * 2));
+                __syncwarp();
+                for (int m = lane; m < count; m += 32) {
+#pragma unroll
+                    for (int sub = 0; sub < D / 64; ++sub)
+                        tma_load_4d(s.q[buf] + sub * (kRows * 128) + m * G * 128, &tm_q, &s.q_full[buf], sub * 64,
+                                    r * G, s.qi[buf][m], b);
+                }
+            } else {
+                const uint32_t qs = smem_u32(s.q[buf]);
+                constexpr int kChunksPerRow = D * 2 / 16;
+                for (int x = lane; x < count * G * kChunksPerRow; x += 32) {
+                    const int row = x / kChunksPerRow, ch = x % kChunksPerRow;
+                    const int m = row / G, h = row % G;
+                    const __nv_bfloat16* src =
+                        q + ((((size_t)b * a.N + s.qi[buf][m]) * a.H_q + (size_t)r * G + h) * D + ch * 8);
+                    cp_async_16(qs + ((ch * 16) / 128) * (kRows * 128) + swz(row, (ch * 16) % 128, 128), src);
+                }
+                cp_async_wait_all();
+                fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s.q_full[buf]);
             }
-            cp_async_wait_all();
-            fence_proxy_async();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s.q_full[buf]);
+            cp_async_arrive_noinc(&s.q_full[buf]);
+            ++issued;
             if (L != prevL) {
                 if (lane == 0) {
-                    if (kv_loads > 0) ok = mbar_wait(&s.kv_empty, (kv_loads - 1) & 1, a.status, 0x802);
-                    if (ok) {
+                    if (kv_loads > 0) okl = mbar_wait(&s.kv_empty, (kv_loads - 1) & 1, a.status, 0x802);
+                    if (okl) {
                         mbar_arrive_expect_tx(&s.kv_full, (D / 64) * BK * 128);
 #pragma unroll
                         for (int sub = 0; sub < D / 64; ++sub)
                             tma_load_4d(s.k + sub * kRows * 128, &tm_k, &s.kv_full, sub * 64, r, c * BK, b);
                     }
                 }
-                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
                 ++kv_loads;
                 prevL = L;
             }
+            itm = nitm;
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) e[j] = ne[j];
         }
         if (!ok) s.abort = 1;
-        if (lane == 0 && kv_loads > 0) mbar_wait(&s.kv_full, (kv_loads - 1) & 1, a.status, 0x803);
+        // nothing may still be landing in shared memory when the CTA exits
+        cp_async_wait_all();
+        if (lane == 0) {
+            for (int x = 0; x < 2 && x < issued; ++x) {
+                const int nl = issued - 1 - x;  // last use of buffer nl & 1
+                mbar_wait(&s.q_full[nl & 1], (nl >> 1) & 1, a.status, 0x803);
+            }
+            if (kv_loads > 0) mbar_wait(&s.kv_full, (kv_loads - 1) & 1, a.status, 0x804);
+        }
     } else if (warp == 5) {
-        // ---------------------------------------------------------------- MMA issuer
+        // ---------------------------------------------------------------- MMA issuer: S^T = K Q^T
         if (lane == 0) {
             bool ok = true;
-            int kv_group = -1, prevL = -1;
+            int kv_group = -1;
             for (int t = t0, n = 0; t < t1; ++t, ++n) {
-                const int L = cs.items[t].x;
-                const int buf = n & 1;
+                const int buf = n & 1, sb = n & 1;
                 if (!mbar_wait(&s.q_full[buf], (n >> 1) & 1, a.status, 0x901)) { ok = false; break; }
-                if (L != prevL) {
+                const int4 rec = s.rec[buf];
+                if (rec.z) {
                     ++kv_group;
-                    prevL = L;
                     if (!mbar_wait(&s.kv_full, kv_group & 1, a.status, 0x902)) { ok = false; break; }
                 }
-                if (!mbar_wait(&s.s_free, (n & 1) ^ 1, a.status, 0x903)) { ok = false; break; }
+                if (!mbar_wait(&s.s_free[sb], ((n >> 1) & 1) ^ 1, a.status, 0x903)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t qb = smem_u32(s.q[buf]), kb = smem_u32(s.k);
+                const uint32_t qa = smem_u32(s.q[buf]), ka = smem_u32(s.k);
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
                     const uint32_t sub = (ks * 16) / 64, off = (ks & 3) * 32;
-                    const uint64_t da = umma_sdesc(kb + sub * (kRows * 128) + off, 16, 1024, 2);
-                    const uint64_t db = umma_sdesc(qb + sub * (kRows * 128) + off, 16, 1024, 2);
-                    umma_bf16(tmem, da, db, kIdesc, ks > 0);
+                    const uint64_t da = umma_sdesc(ka + sub * (kRows * 128) + off, 16, 1024, 2);
+                    const uint64_t db = umma_sdesc(qa + sub * (kRows * 128) + off, 16, 1024, 2);
+                    umma_bf16(tmem + sb * kRows, da, db, kIdesc, ks > 0);
                 }
-                umma_commit(&s.s_full);
+                umma_commit(&s.s_full[sb]);
                 umma_commit(&s.q_empty[buf]);
-                const bool last_of_group = (t + 1 >= t1) || (cs.items[t + 1].x != L);
-                if (last_of_group) umma_commit(&s.kv_empty);
+                if (rec.w) umma_commit(&s.kv_empty);
             }
             if (!ok) s.abort = 1;
             umma_commit(&s.drain);
@@ -284,125 +384,224 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ---------------------------------------------------------------- epilogue: thread = token
-        // Control flow stays uniform across the 128 threads (named barriers below): a failed wait
-        // sets the CTA abort flag, and every thread then skips the work but not the barriers.
+        // Warp w owns tokens 32w..32w+31 of the block (its TMEM lane quarter). Control flow stays
+        // uniform across the 128 threads (named barriers): a failed wait sets the CTA abort flag and
+        // every thread then skips the work but not the barriers.
         const int tt = threadIdx.x;
+        const int g8 = lane >> 2, t4 = lane & 3;
         const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
         const float sl2 = a.scale * kLog2e;
-        float dk[DI];
+        constexpr int NDT = DI / 8;  // dK n-tiles
+        float dk[2][NDT][4];
 #pragma unroll
-        for (int x = 0; x < DI; ++x) dk[x] = 0.f;
-        int prevL = -1, prev_b = 0, prev_tok = 0;
-        bool prev_valid = false;
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < NDT; ++nt)
+#pragma unroll
+                for (int x = 0; x < 4; ++x) dk[mt][nt][x] = 0.f;
+        int prev_b = 0, prev_c = 0;
+        bool have_dk = false;
+        const uint32_t kb_u32 = smem_u32(s.kb);
+
+        auto flush_dk = [&]() {
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int hx = 0; hx < 2; ++hx) {
+                    const int row = warp * 32 + mt * 16 + g8 + hx * 8;
+                    const int tok = prev_c * BK + row;
+                    if (row < BK && tok < a.N) {
+                        float* dst = a.dk_idx + ((size_t)prev_b * a.N + tok) * DI + 2 * t4;
+#pragma unroll
+                        for (int nt = 0; nt < NDT; ++nt)
+                            atomicAdd(reinterpret_cast<float2*>(dst + nt * 8),
+                                      make_float2(dk[mt][nt][2 * hx], dk[mt][nt][2 * hx + 1]));
+                    }
+                }
+        };
+
         for (int t = t0, n = 0; t < t1; ++t, ++n) {
-            const int4 itm = cs.items[t];
-            const int L = itm.x, count = itm.z;
+            const int buf = n & 1, sb = n & 1;
+            epi_bar();  // (A) the previous item's readers of gs / sidx / kb are done
+            bool ok = s.abort == 0;
+            if (ok) ok = mbar_wait(&s.q_full[buf], (n >> 1) & 1, a.status, 0xa01);
+            ok = __all_sync(0xffffffffu, ok);
+            const int4 rec = s.rec[buf];
+            const int L = rec.x, count = rec.y;
             const int c = L % cs.nb, r = (L / cs.nb) % a.H_kv, b = L / (cs.nb * a.H_kv);
-            const int buf = n & 1;
             const int tok = c * BK + tt;
             const bool tvalid = tt < BK && tok < a.N;
-            epi_bar();
-            const bool alive = s.abort == 0;
-            if (L != prevL) {
-                if (prev_valid && alive) {
-                    float* dst = a.dk_idx + ((size_t)prev_b * a.N + prev_tok) * DI;
+            if (ok && rec.z) {
+                // new K block: flush this token's dK_idx, load its K_idx row (zeros past the end)
+                if (have_dk) flush_dk();
 #pragma unroll
-                    for (int x = 0; x < DI; ++x) atomicAdd(dst + x, dk[x]);
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < NDT; ++nt)
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) dk[mt][nt][x] = 0.f;
+#pragma unroll
+                for (int x = 0; x < DI / 8; ++x) {
+                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                    if (tvalid) v = *reinterpret_cast<const uint4*>(k_idx + ((size_t)b * a.N + tok) * DI + x * 8);
+                    *reinterpret_cast<uint4*>(&s.kb[tt * KBP + x * 8]) = v;
                 }
-#pragma unroll
-                for (int x = 0; x < DI; ++x) dk[x] = 0.f;
-                {
-                    float kr[DI];
-#pragma unroll
-                    for (int x = 0; x < DI; ++x) kr[x] = 0.f;
-                    if (tvalid) load_bf16_row(k_idx + ((size_t)b * a.N + tok) * DI, kr, DI);
-#pragma unroll
-                    for (int x = 0; x < DI; ++x) s.kf[tt][x] = kr[x];
-                }
-                prevL = L;
                 prev_b = b;
-                prev_tok = tok;
-                prev_valid = tvalid;
+                prev_c = c;
+                have_dk = true;
+                __syncwarp();
             }
-            bool ok = alive;
-            if (ok) ok = mbar_wait(&s.q_full[buf], (n >> 1) & 1, a.status, 0xa01);
-            if (ok) ok = mbar_wait(&s.s_full, n & 1, a.status, 0xa02);
+            if (ok) {
+                // index log-probabilities log P_idx = S_idx scale_idx - LSE_idx for the warp's 32 tokens
+                const uint32_t qb_u32 = smem_u32(s.qb[buf]);
+                float acc[2][QPC / 8][4];
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < QPC / 8; ++nt)
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) acc[mt][nt][x] = 0.f;
+#pragma unroll
+                for (int ks = 0; ks < DI / 16; ++ks) {
+                    uint32_t af[2][4];
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt)
+                        ldsm_x4(kb_u32 + ((warp * 32 + mt * 16 + (lane & 15)) * KBP + ks * 16 + (lane >> 4) * 8) * 2,
+                                af[mt]);
+#pragma unroll
+                    for (int nt = 0; nt < QPC / 8; ++nt) {
+                        uint32_t b0, b1;
+                        ldsm_x2(qb_u32 + ((nt * 8 + (lane & 7)) * KBP + ks * 16 + ((lane >> 3) & 1) * 8) * 2, b0, b1);
+#pragma unroll
+                        for (int mt = 0; mt < 2; ++mt) mma_16816_bf16(acc[mt][nt], af[mt], b0, b1);
+                    }
+                }
+#pragma unroll
+                for (int nt = 0; nt < QPC / 8; ++nt) {
+                    const int m0 = nt * 8 + 2 * t4;
+                    const float l0 = s.lidx[buf][m0], l1 = s.lidx[buf][m0 + 1];
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                        for (int hx = 0; hx < 2; ++hx) {
+                            const int row = warp * 32 + mt * 16 + g8 + hx * 8;
+                            s.sidx[row * SIP + m0] = fmaf(acc[mt][nt][2 * hx], a.scale_idx, -l0);
+                            s.sidx[row * SIP + m0 + 1] = fmaf(acc[mt][nt][2 * hx + 1], a.scale_idx, -l1);
+                        }
+                }
+                __syncwarp();
+            }
+            if (ok) ok = mbar_wait(&s.s_full[sb], (n >> 1) & 1, a.status, 0xa02);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) s.abort = 1;
-            float sv[kRows];
             if (ok) {
+                // teacher P = mean over the G heads of exp(S scale - LSE_main); gradient and KL terms
                 tc_fence_after();
+                constexpr int QC = 64 / G;  // queries per 64-column TMEM chunk
 #pragma unroll
-                for (int c0 = 0; c0 < kRows; c0 += 32) {
-                    uint32_t r32[32];
-                    tmem_ld32(lane_addr + c0, r32);
+                for (int ch = 0; ch < QPC / QC; ++ch) {
+                    uint32_t sv[64];
+                    tmem_ld32(lane_addr + sb * kRows + ch * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+                    tmem_ld32(lane_addr + sb * kRows + ch * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
                     tmem_ld_wait();
-#pragma unroll
-                    for (int x = 0; x < 32; ++x) sv[c0 + x] = __uint_as_float(r32[x]);
-                }
-                tc_fence_before();
-                mbar_arrive(&s.s_free);
-            }
-#pragma unroll
-            for (int m = 0; m < QPC; ++m) {
-                float gval = 0.f, klv = 0.f;
-                if (ok && m < count && tvalid && tok <= s.qi[buf][m]) {
-                    float P = 0.f;
-#pragma unroll
-                    for (int h = 0; h < G; ++h)
-                        P += fast_exp2(fmaf(sv[m * G + h], sl2, -s.lse[buf][m * G + h] * kLog2e));
-                    P *= 1.f / (float)G;
-                    float si = 0.f;
-#pragma unroll
-                    for (int x = 0; x < DI; ++x) si = fmaf(s.qf[buf][m][x], s.kf[tt][x], si);
-                    const float lp_idx = si * a.scale_idx - s.lidx[buf][m];
-                    const float g = coef * (__expf(lp_idx) - P);
-                    klv = P > 0.f ? P * (__logf(P) - lp_idx) : 0.f;
-                    gval = g * a.scale_idx;
-#pragma unroll
-                    for (int x = 0; x < DI; ++x) dk[x] = fmaf(gval, s.qf[buf][m][x], dk[x]);
-                }
-                s.gs[tt][m] = gval;
-#pragma unroll
-                for (int o = 16; o; o >>= 1) klv += __shfl_xor_sync(0xffffffffu, klv, o);
-                if (lane == 0) s.klw[warp][m] = klv;
-            }
-            epi_bar();
-            // per-(query, slot) reductions over the 128 tokens, fixed order
-            if (ok) {
-                for (int x = tt; x < count * (DI / 4); x += kRows) {
-                    const int m = x / (DI / 4), dg = (x % (DI / 4)) * 4;
-                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                    for (int u = 0; u < kRows; ++u) {
-                        const float g = s.gs[u][m];
-                        acc.x = fmaf(g, s.kf[u][dg], acc.x);
-                        acc.y = fmaf(g, s.kf[u][dg + 1], acc.y);
-                        acc.z = fmaf(g, s.kf[u][dg + 2], acc.z);
-                        acc.w = fmaf(g, s.kf[u][dg + 3], acc.w);
+                    if (ch == QPC / QC - 1) {
+                        tc_fence_before();
+                        mbar_arrive(&s.s_free[sb]);
                     }
-                    const size_t pr = (((size_t)b * a.N + s.qi[buf][m]) * a.H_kv + r) * K1 + s.qslot[buf][m];
-                    *reinterpret_cast<float4*>(a.dq_part + pr * DI + dg) = acc;
+#pragma unroll
+                    for (int qq = 0; qq < QC; ++qq) {
+                        const int m = ch * QC + qq;
+                        float P = 0.f;
+#pragma unroll
+                        for (int h = 0; h < G; ++h)
+                            P += fast_exp2(fmaf(__uint_as_float(sv[qq * G + h]), sl2, -s.lse[buf][m * G + h] * kLog2e));
+                        P *= 1.f / (float)G;
+                        const bool valid = m < count && tvalid && tok <= s.qi[buf][m];
+                        const float lp = s.sidx[tt * SIP + m];
+                        const float gval = coef * (__expf(lp) - P) * a.scale_idx;
+                        const float klv = P > 0.f ? P * (__logf(P) - lp) : 0.f;
+                        s.gs[tt * GSP + m] = valid ? gval : 0.f;
+                        s.sidx[tt * SIP + m] = valid ? klv : 0.f;
+                    }
                 }
-                if (tt < count) {
-                    const double kl = ((double)s.klw[0][tt] + (double)s.klw[1][tt]) +
-                                      ((double)s.klw[2][tt] + (double)s.klw[3][tt]);
-                    const size_t pr = (((size_t)b * a.N + s.qi[buf][tt]) * a.H_kv + r) * K1 + s.qslot[buf][tt];
-                    a.kl_part[pr] = kl;
+                __syncwarp();
+                // dK_idx[token] += sum_q g(token, q) scale_idx Q_idx[q]   (tf32 mma, gradient split in two)
+#pragma unroll
+                for (int kq = 0; kq < QPC / 8; ++kq) {
+                    uint32_t ah[2][4], al[2][4];
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt) {
+                        const int row = warp * 32 + mt * 16 + g8;
+                        split_tf32(s.gs[row * GSP + kq * 8 + t4], ah[mt][0], al[mt][0]);
+                        split_tf32(s.gs[(row + 8) * GSP + kq * 8 + t4], ah[mt][1], al[mt][1]);
+                        split_tf32(s.gs[row * GSP + kq * 8 + t4 + 4], ah[mt][2], al[mt][2]);
+                        split_tf32(s.gs[(row + 8) * GSP + kq * 8 + t4 + 4], ah[mt][3], al[mt][3]);
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < NDT; ++nt) {
+                        const uint32_t b0 = bf16_as_tf32(s.qb[buf][(kq * 8 + t4) * KBP + nt * 8 + g8]);
+                        const uint32_t b1 = bf16_as_tf32(s.qb[buf][(kq * 8 + t4 + 4) * KBP + nt * 8 + g8]);
+#pragma unroll
+                        for (int mt = 0; mt < 2; ++mt) {
+                            mma_1688_tf32(dk[mt][nt], ah[mt][0], ah[mt][1], ah[mt][2], ah[mt][3], b0, b1);
+                            mma_1688_tf32(dk[mt][nt], al[mt][0], al[mt][1], al[mt][2], al[mt][3], b0, b1);
+                        }
+                    }
+                }
+            }
+            epi_bar();  // (B) gradients and KL terms of all 128 tokens are in shared memory
+            if (ok) {
+                // dQ_idx^T[d][q] = sum_token K_idx[token][d] g(token, q) scale_idx: (d, q) tiles over warps
+                constexpr int MT = DI / 16, NT = QPC / 8;
+                for (int x = warp; x < MT * NT; x += 4) {
+                    const int mt = x % MT, nt = x / MT;
+                    float cq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+                    for (int ks = 0; ks < kRows / 8; ++ks) {
+                        const __nv_bfloat16* k0 = &s.kb[(ks * 8 + t4) * KBP + mt * 16 + g8];
+                        const __nv_bfloat16* k1 = k0 + 4 * KBP;
+                        uint32_t bh0, bl0, bh1, bl1;
+                        split_tf32(s.gs[(ks * 8 + t4) * GSP + nt * 8 + g8], bh0, bl0);
+                        split_tf32(s.gs[(ks * 8 + t4 + 4) * GSP + nt * 8 + g8], bh1, bl1);
+                        const uint32_t a0 = bf16_as_tf32(k0[0]), a1 = bf16_as_tf32(k0[8]);
+                        const uint32_t a2 = bf16_as_tf32(k1[0]), a3 = bf16_as_tf32(k1[8]);
+                        mma_1688_tf32(cq, a0, a1, a2, a3, bh0, bh1);
+                        mma_1688_tf32(cq, a0, a1, a2, a3, bl0, bl1);
+                    }
+                    const int d0 = mt * 16 + g8;
+#pragma unroll
+                    for (int cx = 0; cx < 2; ++cx) {
+                        const int m = nt * 8 + 2 * t4 + cx;
+                        if (m < count) {
+                            const size_t pr =
+                                (((size_t)b * a.N + s.qi[buf][m]) * a.H_kv + r) * K1 + s.qslot[buf][m];
+                            a.dq_part[pr * DI + d0] = cq[cx];
+                            a.dq_part[pr * DI + d0 + 8] = cq[2 + cx];
+                        }
+                    }
+                }
+                // KL of each (query, slot): sum of its token terms, fixed order
+                constexpr int TPQ = kRows / QPC;  // threads per query
+                const int m = tt / TPQ, part = tt % TPQ;
+                float kl = 0.f;
+#pragma unroll 8
+                for (int j = 0; j < QPC; ++j) kl += s.sidx[(part + TPQ * j) * SIP + m];
+#pragma unroll
+                for (int o = TPQ / 2; o; o >>= 1) kl += __shfl_xor_sync(0xffffffffu, kl, o);
+                if (part == 0 && m < count) {
+                    const size_t pr = (((size_t)b * a.N + s.qi[buf][m]) * a.H_kv + r) * K1 + s.qslot[buf][m];
+                    a.kl_part[pr] = (double)kl;
                 }
                 mbar_arrive(&s.q_empty[buf]);
             }
         }
         epi_bar();
-        if (prev_valid && s.abort == 0) {
-            float* dst = a.dk_idx + ((size_t)prev_b * a.N + prev_tok) * DI;
-#pragma unroll
-            for (int x = 0; x < DI; ++x) atomicAdd(dst + x, dk[x]);
-        }
+        if (have_dk && s.abort == 0) flush_dk();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 5) tmem_dealloc(tmem, 128);
+    if (warp == 5) tmem_dealloc(tmem, 256);
 }
 
 // One thread per (b, i, r): dQ_idx = sum of the slot partials; KL row = sum of the slot partials.
@@ -448,14 +647,14 @@ __global__ void k_kl_loss(KlArgs a) {
 }
 
 template <int D, int DI, int G>
-cudaError_t launch_kl(const KlArgs& a, const CUtensorMap& tk, const void* q, const void* q_idx, const void* k_idx,
-                      int num_sms, cudaStream_t st) {
-    const size_t smem = std::max<size_t>(sizeof(KlSmem<D, DI>) + 1024, 116 * 1024);  // one CTA per SM
+cudaError_t launch_kl(const KlArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const void* q,
+                      const void* q_idx, const void* k_idx, int num_sms, cudaStream_t st) {
+    const size_t smem = std::max<size_t>(sizeof(KlSmem<D, DI, kRows / G>) + 1024, 116 * 1024);  // one CTA per SM
     cudaError_t e = cudaFuncSetAttribute(k_kl_kv_outer<D, DI, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     ProfScope ps("kl_kv_outer", st);
-    k_kl_kv_outer<D, DI, G><<<num_sms, kThreads, smem, st>>>(tk, static_cast<const __nv_bfloat16*>(q),
+    k_kl_kv_outer<D, DI, G><<<num_sms, kThreads, smem, st>>>(tq, tk, static_cast<const __nv_bfloat16*>(q),
                                                               static_cast<const __nv_bfloat16*>(q_idx),
                                                               static_cast<const __nv_bfloat16*>(k_idx), a);
     return cudaGetLastError();
@@ -482,18 +681,22 @@ cudaError_t run_lse_idx(const KlArgs& a, const void* q_idx, const void* k_idx, i
 
 cudaError_t run_kl(const KlArgs& a, const void* q, const void* k, const void* q_idx, const void* k_idx, int num_sms,
                    cudaStream_t st) {
-    CUtensorMap tk;
+    const int G = a.H_q / a.H_kv;
+    CUtensorMap tq, tk;
+    const uint64_t dq[4] = {(uint64_t)a.d, (uint64_t)a.H_q, (uint64_t)a.N, (uint64_t)a.B};
+    const uint64_t sq[3] = {(uint64_t)a.d * 2, (uint64_t)a.H_q * a.d * 2, (uint64_t)a.N * a.H_q * a.d * 2};
+    const uint32_t bq[4] = {64, (uint32_t)std::min(G, 256), 1, 1};
     const uint64_t dims[4] = {(uint64_t)a.d, (uint64_t)a.H_kv, (uint64_t)a.N, (uint64_t)a.B};
     const uint64_t strides[3] = {(uint64_t)a.d * 2, (uint64_t)a.H_kv * a.d * 2, (uint64_t)a.N * a.H_kv * a.d * 2};
     const uint32_t box[4] = {64, 1, (uint32_t)a.block_k, 1};
-    if (!make_tmap_4d(&tk, k, dims, strides, box, 128)) return cudaErrorInvalidValue;
+    if (!make_tmap_4d(&tq, q, dq, sq, bq, 128) || !make_tmap_4d(&tk, k, dims, strides, box, 128))
+        return cudaErrorInvalidValue;
     cudaError_t e = cudaMemsetAsync(a.dk_idx, 0, (size_t)a.B * a.N * a.d_idx * 4, st);
     if (e != cudaSuccess) return e;
-    const int G = a.H_q / a.H_kv;
-    if (a.d == 128 && G == 16) e = launch_kl<128, 64, 16>(a, tk, q, q_idx, k_idx, num_sms, st);
-    else if (a.d == 128 && G == 2) e = launch_kl<128, 64, 2>(a, tk, q, q_idx, k_idx, num_sms, st);
-    else if (a.d == 64 && G == 16) e = launch_kl<64, 32, 16>(a, tk, q, q_idx, k_idx, num_sms, st);
-    else if (a.d == 64 && G == 2) e = launch_kl<64, 32, 2>(a, tk, q, q_idx, k_idx, num_sms, st);
+    if (a.d == 128 && G == 16) e = launch_kl<128, 64, 16>(a, tq, tk, q, q_idx, k_idx, num_sms, st);
+    else if (a.d == 128 && G == 2) e = launch_kl<128, 64, 2>(a, tq, tk, q, q_idx, k_idx, num_sms, st);
+    else if (a.d == 64 && G == 16) e = launch_kl<64, 32, 16>(a, tq, tk, q, q_idx, k_idx, num_sms, st);
+    else if (a.d == 64 && G == 2) e = launch_kl<64, 32, 2>(a, tq, tk, q, q_idx, k_idx, num_sms, st);
     else return cudaErrorInvalidValue;
     if (e != cudaSuccess) return e;
     const long long rows = (long long)a.B * a.N * a.H_kv;
