@@ -22,11 +22,8 @@ namespace msa {
 
 namespace {
 
-constexpr int kThreads = 192;
 constexpr int kRows = 128;
 constexpr float kLog2e = 1.4426950408889634f;
-
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 __device__ __forceinline__ void load_bf16_row(const __nv_bfloat16* src, float* dst, int n) {
 #pragma unroll
@@ -173,40 +170,64 @@ __device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) 
     lo = to_tf32(x - __uint_as_float(hi));
 }
 
-// Row pitches keep the mma fragment loads of a warp on distinct banks (or at most two-way).
-template <int D, int DI, int QPC>
+// Epilogue teams: with G >= 8 (8 or 16 queries per item) two teams of four warps take alternate
+// items, so that one team's mma and reduction work overlaps the other's exponentials.
+template <int G>
+__host__ __device__ constexpr int kl_teams() { return G >= 8 ? 2 : 1; }
+// Producer warps: with G >= 8 one warp issues the Q and K tiles and another the item metadata, so
+// that the two sets of copies are issued side by side.
+template <int G>
+__host__ __device__ constexpr int kl_prods() { return G >= 8 ? 2 : 1; }
+template <int G>
+__host__ __device__ constexpr int kl_threads() { return (4 * kl_teams<G>() + kl_prods<G>() + 1) * 32; }
+// Item metadata stages (Q_idx rows, LSE values, query ids): the Q tile itself has two stages that
+// the MMA releases, the metadata more, released by the epilogue, so loads run ahead of it.
+template <int G>
+__host__ __device__ constexpr int kl_meta_stages() { return G >= 8 ? 4 : 2; }
+
+// Row pitches keep the mma fragment loads of a warp on distinct banks (or at most two-way) and the
+// per-token row writes conflict-free.
+template <int D, int DI, int QPC, int TEAMS, int NMETA, int PRODS>
 struct KlSmem {
     static constexpr int KBP = DI + 8;   // K_idx / Q_idx bf16 rows
-    static constexpr int GSP = QPC + 4;  // gradient rows [token][query]
+    static constexpr int GSP = QPC + 1;  // gradient rows [token][query]
     static constexpr int SIP = QPC + 1;  // index log-probability / KL rows [token][query]
     alignas(1024) uint8_t q[2][kRows * D * 2];
-    alignas(1024) uint8_t k[kRows * D * 2];      // 128 token rows (rows >= block_k unused)
-    alignas(16) __nv_bfloat16 kb[kRows * KBP];   // K_idx rows of the current block (zero past the end)
-    alignas(16) __nv_bfloat16 qb[2][QPC * KBP];  // Q_idx rows of the item queries
-    alignas(16) float lse[2][kRows];             // LSE_main of the item rows (query-major, head-minor)
-    float gs[kRows * GSP];                       // g * scale_idx per (token, query)
-    float sidx[kRows * SIP];                     // log P_idx per (token, query), then the KL terms
-    float lidx[2][QPC];                          // LSE_idx of the item queries
-    int qi[2][QPC], qslot[2][QPC];
-    int4 rec[2];                                 // item: L, count, new K tile, last item of its tile
-    uint64_t q_full[2], q_empty[2], kv_full, kv_empty, s_full[2], s_free[2], drain;
+    alignas(1024) uint8_t k[kRows * D * 2];             // 128 token rows (rows >= block_k unused)
+    alignas(16) __nv_bfloat16 kb[TEAMS][kRows * KBP];   // K_idx rows of each team's block (zero past the end)
+    alignas(16) __nv_bfloat16 qb[NMETA][QPC * KBP];     // Q_idx rows of the item queries
+    alignas(16) float lse[NMETA][kRows];                // LSE_main of the item rows (query-major, head-minor)
+    float gs[TEAMS][kRows * GSP];                       // g * scale_idx per (token, query)
+    float sidx[TEAMS][kRows * SIP];                     // log P_idx per (token, query), then the KL terms
+    float lidx[NMETA][QPC];                             // LSE_idx of the item queries
+    int ent[NMETA][QPC];                                // query entries (i << 5 | slot) of the item
+    int4 rec[NMETA];                                    // item record (L, first entry, count, -)
+    int4 crec[PRODS][2][32];                            // per producer warp: item records of the current /
+    int cent[PRODS][2][32][QPC];                        // next chunk of 32 items and their query entries
+    uint64_t q_full[2], q_empty[2], meta_full[NMETA], meta_empty[NMETA];
+    uint64_t kv_full, kv_empty, s_full[2], s_free[2], drain;
     uint32_t tmem_base;
     int abort;
 };
 
 template <int D, int DI, int G>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kl_threads<G>(), 1)
     k_kl_kv_outer(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ q_idx,
                   const __nv_bfloat16* __restrict__ k_idx, KlArgs a) {
     constexpr int QPC = kRows / G;
-    using Sm = KlSmem<D, DI, QPC>;
+    constexpr int TEAMS = kl_teams<G>();
+    constexpr int NMETA = kl_meta_stages<G>();
+    constexpr int PRODS = kl_prods<G>();
+    constexpr int kProdWarp = 4 * TEAMS, kMmaWarp = 4 * TEAMS + PRODS;
+    using Sm = KlSmem<D, DI, QPC, TEAMS, NMETA, PRODS>;
     constexpr int KBP = Sm::KBP, GSP = Sm::GSP, SIP = Sm::SIP;
     extern __shared__ uint8_t smem_raw[];
     Sm& s = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr uint32_t kIdesc = umma_idesc_bf16(kRows, kRows, false, false);
     static_assert(QPC % 8 == 0 && QPC <= 64, "KL items hold 8 to 64 queries");
     static_assert(DI % 16 == 0, "index head dim must be a multiple of 16");
+    static_assert(G % 2 == 0, "heads are processed in pairs");
 
     const int K1 = a.topk + 1;
     const int BK = a.block_k;
@@ -219,10 +240,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int x = 0; x < 2; ++x) {
-            mbar_init(&s.q_full[x], 1 + 32);
-            mbar_init(&s.q_empty[x], 1 + kRows);
+            mbar_init(&s.q_full[x], 1);
+            mbar_init(&s.q_empty[x], 1);
             mbar_init(&s.s_full[x], 1);
             mbar_init(&s.s_free[x], kRows);
+        }
+        for (int x = 0; x < NMETA; ++x) {
+            mbar_init(&s.meta_full[x], 32);
+            mbar_init(&s.meta_empty[x], kRows);
         }
         mbar_init(&s.kv_full, 1);
         mbar_init(&s.kv_empty, 1);
@@ -234,9 +259,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Q_idx rows past an item's count are read by the gradient mma (times a zero gradient), so
         // they must hold finite values: start from zeros.
         uint32_t* z = reinterpret_cast<uint32_t*>(s.qb);
-        for (int x = threadIdx.x; x < 2 * QPC * KBP / 2; x += kRows) z[x] = 0u;
+        for (int x = threadIdx.x; x < NMETA * QPC * KBP / 2; x += kRows) z[x] = 0u;
     }
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         tmem_alloc(&s.tmem_base, 256);
         tmem_relinquish();
     }
@@ -245,123 +270,156 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = s.tmem_base;
 
-    if (warp == 4) {
+    if (warp >= kProdWarp && warp < kProdWarp + PRODS) {
         // ---------------------------------------------------------------- loads + item records
-        // The record and entries of the next item are fetched while the current one is issued, and
-        // every copy is asynchronous: this warp never waits on a global load of the current item.
-        constexpr int EPL = (QPC + 31) / 32;
+        // Item records and query entries come in chunks of 32 items, one per lane: the next chunk's
+        // records are loaded at item 0 of a chunk, their entries at item 8, and both are stored to
+        // the warp's shared ring at item 16, so no global load latency sits on the per-item path.
+        // Everything an item's consumers read arrives by cp.async (metadata, counted by one arrival
+        // per lane once its copies land) or by TMA (Q and K tiles, relaxed arrives): no release arrive
+        // here, which would wait for this warp's copies still in flight.
+        const int pw = warp - kProdWarp;
+        const bool do_meta = PRODS == 1 || pw == 1, do_q = PRODS == 1 || pw == 0;
+        constexpr int CH = 32;
+        int4 (*crec)[32] = s.crec[pw];
+        int (*cent)[32][QPC] = s.cent[pw];
         int kv_loads = 0, prevL = -1, issued = 0;
         bool ok = true;
-        int4 itm = make_int4(0, 0, 0, 0);
-        int e[EPL];
-        if (t0 < t1) itm = cs.items[t0];
+        int4 r_next = make_int4(-1, 0, 0, 0);
+        int e_next[QPC];
+        {
+            const int4 rr = t0 + lane < t1 ? cs.items[t0 + lane] : make_int4(-1, 0, 0, 0);
+            crec[0][lane] = rr;
 #pragma unroll
-        for (int j = 0; j < EPL; ++j) e[j] = (t0 < t1 && lane + 32 * j < itm.z) ? cs.entries[itm.y + lane + 32 * j] : 0;
+            for (int x = 0; x < QPC; ++x) cent[0][lane][x] = x < rr.z ? cs.entries[rr.y + x] : 0;
+            __syncwarp();
+        }
         for (int t = t0, n = 0; t < t1; ++t, ++n) {
-            int4 nitm = make_int4(-1, 0, 0, 0);
-            int ne[EPL];
-            if (t + 1 < t1) nitm = cs.items[t + 1];
-#pragma unroll
-            for (int j = 0; j < EPL; ++j)
-                ne[j] = (t + 1 < t1 && lane + 32 * j < nitm.z) ? cs.entries[nitm.y + lane + 32 * j] : 0;
+            const int j = n % CH, cb = (n / CH) & 1;
+            const int4 itm = crec[cb][j];
             const int L = itm.x, count = itm.z;
             const int c = L % cs.nb, r = (L / cs.nb) % a.H_kv, b = L / (cs.nb * a.H_kv);
-            const int buf = n & 1;
+            const int* qe = cent[cb][j];
+            const int ms = n % NMETA, buf = n & 1;
             int okl = 1;
-            if (lane == 0) okl = mbar_wait(&s.q_empty[buf], ((n >> 1) & 1) ^ 1, a.status, 0x801);
-            if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
-#pragma unroll
-            for (int j = 0; j < EPL; ++j) {
-                const int m = lane + 32 * j;
-                if (m < QPC) {
-                    s.qi[buf][m] = m < count ? (e[j] >> 5) : -1;
-                    s.qslot[buf][m] = e[j] & 31;
-                }
-            }
-            if (lane == 0) s.rec[buf] = make_int4(L, count, L != prevL, nitm.x != L);
-            __syncwarp();
-            // LSE_idx of each query, LSE_main of its G heads, its Q_idx row
-            for (int m = lane; m < count; m += 32)
-                cp_async_ca<4>(smem_u32(&s.lidx[buf][m]), a.lse_idx + ((size_t)b * a.N + s.qi[buf][m]) * a.H_kv + r);
-            constexpr int LB = G * 4 >= 16 ? 16 : G * 4;  // bytes per copy of one query's LSE_main
-            constexpr int LPQ = G * 4 / LB;
-            for (int x = lane; x < count * LPQ; x += 32) {
-                const int m = x / LPQ, part = x % LPQ;
-                const float* src = a.lse + ((size_t)b * a.N + s.qi[buf][m]) * a.H_q + (size_t)r * G + part * (LB / 4);
-                cp_async_ca<LB>(smem_u32(&s.lse[buf][m * G + part * (LB / 4)]), src);
-            }
-            constexpr int QIC = DI / 8;  // 16-byte chunks per Q_idx row
-            for (int x = lane; x < count * QIC; x += 32) {
-                const int m = x / QIC, part = x % QIC;
-                const __nv_bfloat16* src = q_idx + (((size_t)b * a.N + s.qi[buf][m]) * a.H_kv + r) * DI + part * 8;
-                cp_async_ca<16>(smem_u32(&s.qb[buf][m * KBP + part * 8]), src);
-            }
-            // Q: the G head rows of each query, in the 128B-swizzled K-major tile the MMA reads
-            if constexpr (G >= 8) {
-                if (lane == 0) mbar_arrive_expect_tx(&s.q_full[buf], (uint32_t)(count * G * D * 2));
-                __syncwarp();
+            if (do_meta) {
+                if (lane == 0) okl = mbar_wait(&s.meta_empty[ms], ((n / NMETA) & 1) ^ 1, a.status, 0x801);
+                if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
+                // item record, query entries, LSE_idx of each query, LSE_main of its G heads, its Q_idx row
+                if (lane == 0) cp_async_ca<16>(smem_u32(&s.rec[ms]), cs.items + t);
                 for (int m = lane; m < count; m += 32) {
-#pragma unroll
-                    for (int sub = 0; sub < D / 64; ++sub)
-                        tma_load_4d(s.q[buf] + sub * (kRows * 128) + m * G * 128, &tm_q, &s.q_full[buf], sub * 64,
-                                    r * G, s.qi[buf][m], b);
+                    cp_async_ca<4>(smem_u32(&s.ent[ms][m]), cs.entries + itm.y + m);
+                    cp_async_ca<4>(smem_u32(&s.lidx[ms][m]),
+                                   a.lse_idx + ((size_t)b * a.N + (qe[m] >> 5)) * a.H_kv + r);
                 }
-            } else {
-                const uint32_t qs = smem_u32(s.q[buf]);
-                constexpr int kChunksPerRow = D * 2 / 16;
-                for (int x = lane; x < count * G * kChunksPerRow; x += 32) {
-                    const int row = x / kChunksPerRow, ch = x % kChunksPerRow;
-                    const int m = row / G, h = row % G;
+                constexpr int LB = G * 4 >= 16 ? 16 : G * 4;  // bytes per copy of one query's LSE_main
+                constexpr int LPQ = G * 4 / LB;
+                for (int x = lane; x < count * LPQ; x += 32) {
+                    const int m = x / LPQ, part = x % LPQ;
+                    const float* src =
+                        a.lse + ((size_t)b * a.N + (qe[m] >> 5)) * a.H_q + (size_t)r * G + part * (LB / 4);
+                    cp_async_ca<LB>(smem_u32(&s.lse[ms][m * G + part * (LB / 4)]), src);
+                }
+                constexpr int QIC = DI / 8;  // 16-byte chunks per Q_idx row
+                for (int x = lane; x < count * QIC; x += 32) {
+                    const int m = x / QIC, part = x % QIC;
                     const __nv_bfloat16* src =
-                        q + ((((size_t)b * a.N + s.qi[buf][m]) * a.H_q + (size_t)r * G + h) * D + ch * 8);
-                    cp_async_16(qs + ((ch * 16) / 128) * (kRows * 128) + swz(row, (ch * 16) % 128, 128), src);
+                        q_idx + (((size_t)b * a.N + (qe[m] >> 5)) * a.H_kv + r) * DI + part * 8;
+                    cp_async_ca<16>(smem_u32(&s.qb[ms][m * KBP + part * 8]), src);
                 }
-                cp_async_wait_all();
-                fence_proxy_async();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s.q_full[buf]);
+                cp_async_arrive_noinc(&s.meta_full[ms]);
             }
-            cp_async_arrive_noinc(&s.q_full[buf]);
-            ++issued;
-            if (L != prevL) {
-                if (lane == 0) {
-                    if (kv_loads > 0) okl = mbar_wait(&s.kv_empty, (kv_loads - 1) & 1, a.status, 0x802);
-                    if (okl) {
-                        mbar_arrive_expect_tx(&s.kv_full, (D / 64) * BK * 128);
+            if (do_q) {
+                // Q: the G head rows of each query, in the 128B-swizzled K-major tile the MMA reads
+                if (lane == 0) okl = mbar_wait(&s.q_empty[buf], ((n >> 1) & 1) ^ 1, a.status, 0x805);
+                if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
+                if constexpr (G >= 8) {
+                    if (lane == 0) mbar_arrive_expect_tx_relaxed(&s.q_full[buf], (uint32_t)(count * G * D * 2));
+                    __syncwarp();
+                    for (int m = lane; m < count; m += 32) {
 #pragma unroll
                         for (int sub = 0; sub < D / 64; ++sub)
-                            tma_load_4d(s.k + sub * kRows * 128, &tm_k, &s.kv_full, sub * 64, r, c * BK, b);
+                            tma_load_4d(s.q[buf] + sub * (kRows * 128) + m * G * 128, &tm_q, &s.q_full[buf],
+                                        sub * 64, r * G, qe[m] >> 5, b);
                     }
+                } else {
+                    const uint32_t qs = smem_u32(s.q[buf]);
+                    constexpr int kChunksPerRow = D * 2 / 16;
+                    for (int x = lane; x < count * G * kChunksPerRow; x += 32) {
+                        const int row = x / kChunksPerRow, ch = x % kChunksPerRow;
+                        const int m = row / G, h = row % G;
+                        const __nv_bfloat16* src =
+                            q + ((((size_t)b * a.N + (qe[m] >> 5)) * a.H_q + (size_t)r * G + h) * D + ch * 8);
+                        cp_async_16(qs + ((ch * 16) / 128) * (kRows * 128) + swz(row, (ch * 16) % 128, 128), src);
+                    }
+                    cp_async_wait_all();
+                    fence_proxy_async();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s.q_full[buf]);
                 }
-                if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
-                ++kv_loads;
-                prevL = L;
-            }
-            itm = nitm;
+                // K tile of a new (block, group); the MMA releases the previous one when it reaches
+                // the first item of this one
+                if (L != prevL) {
+                    if (lane == 0) {
+                        if (kv_loads > 0) okl = mbar_wait(&s.kv_empty, (kv_loads - 1) & 1, a.status, 0x802);
+                        if (okl) {
+                            mbar_arrive_expect_tx_relaxed(&s.kv_full, (D / 64) * BK * 128);
 #pragma unroll
-            for (int j = 0; j < EPL; ++j) e[j] = ne[j];
+                            for (int sub = 0; sub < D / 64; ++sub)
+                                tma_load_4d(s.k + sub * kRows * 128, &tm_k, &s.kv_full, sub * 64, r, c * BK, b);
+                        }
+                    }
+                    if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
+                    ++kv_loads;
+                    prevL = L;
+                }
+            }
+            ++issued;
+            // next chunk of item records and entries
+            if (j == 0) r_next = t + CH + lane < t1 ? cs.items[t + CH + lane] : make_int4(-1, 0, 0, 0);
+            if (j == 8) {
+#pragma unroll
+                for (int x = 0; x < QPC; ++x) e_next[x] = x < r_next.z ? cs.entries[r_next.y + x] : 0;
+            }
+            if (j == 16) {
+                crec[cb ^ 1][lane] = r_next;
+#pragma unroll
+                for (int x = 0; x < QPC; ++x) cent[cb ^ 1][lane][x] = e_next[x];
+                __syncwarp();
+            }
         }
         if (!ok) s.abort = 1;
         // nothing may still be landing in shared memory when the CTA exits
         cp_async_wait_all();
         if (lane == 0) {
-            for (int x = 0; x < 2 && x < issued; ++x) {
-                const int nl = issued - 1 - x;  // last use of buffer nl & 1
-                mbar_wait(&s.q_full[nl & 1], (nl >> 1) & 1, a.status, 0x803);
+            if (do_q) {
+                for (int x = 0; x < 2 && x < issued; ++x) {
+                    const int nl = issued - 1 - x;  // last use of buffer nl & 1
+                    mbar_wait(&s.q_full[nl & 1], (nl >> 1) & 1, a.status, 0x803);
+                }
+                if (kv_loads > 0) mbar_wait(&s.kv_full, (kv_loads - 1) & 1, a.status, 0x804);
             }
-            if (kv_loads > 0) mbar_wait(&s.kv_full, (kv_loads - 1) & 1, a.status, 0x804);
+            if (do_meta) {
+                for (int x = 0; x < NMETA && x < issued; ++x) {
+                    const int nl = issued - 1 - x;  // last use of metadata stage nl % NMETA
+                    mbar_wait(&s.meta_full[nl % NMETA], (nl / NMETA) & 1, a.status, 0x806);
+                }
+            }
         }
-    } else if (warp == 5) {
+    } else if (warp == kMmaWarp) {
         // ---------------------------------------------------------------- MMA issuer: S^T = K Q^T
         if (lane == 0) {
             bool ok = true;
-            int kv_group = -1;
+            int kv_group = -1, prevL = -1;
             for (int t = t0, n = 0; t < t1; ++t, ++n) {
-                const int buf = n & 1, sb = n & 1;
+                const int buf = n & 1, sb = n & 1, ms = n % NMETA;
+                if (!mbar_wait(&s.meta_full[ms], (n / NMETA) & 1, a.status, 0x905)) { ok = false; break; }
+                const int L = s.rec[ms].x;
                 if (!mbar_wait(&s.q_full[buf], (n >> 1) & 1, a.status, 0x901)) { ok = false; break; }
-                const int4 rec = s.rec[buf];
-                if (rec.z) {
+                if (L != prevL) {
+                    if (kv_group >= 0) umma_commit(&s.kv_empty);  // previous K tile no longer read
                     ++kv_group;
+                    prevL = L;
                     if (!mbar_wait(&s.kv_full, kv_group & 1, a.status, 0x902)) { ok = false; break; }
                 }
                 if (!mbar_wait(&s.s_free[sb], ((n >> 1) & 1) ^ 1, a.status, 0x903)) { ok = false; break; }
@@ -376,7 +434,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 umma_commit(&s.s_full[sb]);
                 umma_commit(&s.q_empty[buf]);
-                if (rec.w) umma_commit(&s.kv_empty);
             }
             if (!ok) s.abort = 1;
             umma_commit(&s.drain);
@@ -384,13 +441,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ---------------------------------------------------------------- epilogue: thread = token
-        // Warp w owns tokens 32w..32w+31 of the block (its TMEM lane quarter). Control flow stays
-        // uniform across the 128 threads (named barriers): a failed wait sets the CTA abort flag and
+        // Team `team` takes the CTA's items team, team + TEAMS, ...; its warp wq owns tokens
+        // 32wq..32wq+31 of the block (TMEM lane quarter wq). Control flow stays uniform across the
+        // team's 128 threads (named barrier per team): a failed wait sets the CTA abort flag and
         // every thread then skips the work but not the barriers.
-        const int tt = threadIdx.x;
+        const int team = warp / 4, wq = warp % 4;
+        const int tt = wq * 32 + lane;
         const int g8 = lane >> 2, t4 = lane & 3;
-        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-        const float sl2 = a.scale * kLog2e;
+        const uint32_t lane_addr = tmem + ((uint32_t)(wq * 32) << 16);
+        const uint64_t sl2x2 = f2_packf(a.scale * kLog2e, a.scale * kLog2e);
+        const uint64_t nlog2e = f2_packf(-kLog2e, -kLog2e);
+        __nv_bfloat16* kbt = s.kb[team];
+        float* gst = s.gs[team];
+        float* sit = s.sidx[team];
+        const uint32_t kb_u32 = smem_u32(kbt);
         constexpr int NDT = DI / 8;  // dK n-tiles
         float dk[2][NDT][4];
 #pragma unroll
@@ -399,16 +463,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int nt = 0; nt < NDT; ++nt)
 #pragma unroll
                 for (int x = 0; x < 4; ++x) dk[mt][nt][x] = 0.f;
-        int prev_b = 0, prev_c = 0;
-        bool have_dk = false;
-        const uint32_t kb_u32 = smem_u32(s.kb);
+        int myL = -1, prev_b = 0, prev_c = 0;
+        auto team_bar = [&]() { asm volatile("bar.sync %0, 128;" ::"r"(1 + team) : "memory"); };
 
         auto flush_dk = [&]() {
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
                 for (int hx = 0; hx < 2; ++hx) {
-                    const int row = warp * 32 + mt * 16 + g8 + hx * 8;
+                    const int row = wq * 32 + mt * 16 + g8 + hx * 8;
                     const int tok = prev_c * BK + row;
                     if (row < BK && tok < a.N) {
                         float* dst = a.dk_idx + ((size_t)prev_b * a.N + tok) * DI + 2 * t4;
@@ -420,20 +483,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
         };
 
-        for (int t = t0, n = 0; t < t1; ++t, ++n) {
-            const int buf = n & 1, sb = n & 1;
-            epi_bar();  // (A) the previous item's readers of gs / sidx / kb are done
+        for (int t = t0 + team, n = team; t < t1; t += TEAMS, n += TEAMS) {
+            const int buf = n % NMETA, sb = n & 1;
+            team_bar();  // (A) the team's previous item is done with gs / sidx / kb
             bool ok = s.abort == 0;
-            if (ok) ok = mbar_wait(&s.q_full[buf], (n >> 1) & 1, a.status, 0xa01);
+            if (ok) ok = mbar_wait(&s.meta_full[buf], (n / NMETA) & 1, a.status, 0xa01);
             ok = __all_sync(0xffffffffu, ok);
             const int4 rec = s.rec[buf];
-            const int L = rec.x, count = rec.y;
+            const int L = rec.x, count = rec.z;
             const int c = L % cs.nb, r = (L / cs.nb) % a.H_kv, b = L / (cs.nb * a.H_kv);
             const int tok = c * BK + tt;
             const bool tvalid = tt < BK && tok < a.N;
-            if (ok && rec.z) {
-                // new K block: flush this token's dK_idx, load its K_idx row (zeros past the end)
-                if (have_dk) flush_dk();
+            if (ok && L != myL) {
+                // new K block for this team: flush dK_idx, load this token's K_idx row (zeros past the end)
+                if (myL >= 0) flush_dk();
 #pragma unroll
                 for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
@@ -444,11 +507,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int x = 0; x < DI / 8; ++x) {
                     uint4 v = make_uint4(0u, 0u, 0u, 0u);
                     if (tvalid) v = *reinterpret_cast<const uint4*>(k_idx + ((size_t)b * a.N + tok) * DI + x * 8);
-                    *reinterpret_cast<uint4*>(&s.kb[tt * KBP + x * 8]) = v;
+                    *reinterpret_cast<uint4*>(&kbt[tt * KBP + x * 8]) = v;
                 }
+                myL = L;
                 prev_b = b;
                 prev_c = c;
-                have_dk = true;
                 __syncwarp();
             }
             if (ok) {
@@ -466,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint32_t af[2][4];
 #pragma unroll
                     for (int mt = 0; mt < 2; ++mt)
-                        ldsm_x4(kb_u32 + ((warp * 32 + mt * 16 + (lane & 15)) * KBP + ks * 16 + (lane >> 4) * 8) * 2,
+                        ldsm_x4(kb_u32 + ((wq * 32 + mt * 16 + (lane & 15)) * KBP + ks * 16 + (lane >> 4) * 8) * 2,
                                 af[mt]);
 #pragma unroll
                     for (int nt = 0; nt < QPC / 8; ++nt) {
@@ -484,9 +547,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
                         for (int hx = 0; hx < 2; ++hx) {
-                            const int row = warp * 32 + mt * 16 + g8 + hx * 8;
-                            s.sidx[row * SIP + m0] = fmaf(acc[mt][nt][2 * hx], a.scale_idx, -l0);
-                            s.sidx[row * SIP + m0 + 1] = fmaf(acc[mt][nt][2 * hx + 1], a.scale_idx, -l1);
+                            const int row = wq * 32 + mt * 16 + g8 + hx * 8;
+                            sit[row * SIP + m0] = fmaf(acc[mt][nt][2 * hx], a.scale_idx, -l0);
+                            sit[row * SIP + m0 + 1] = fmaf(acc[mt][nt][2 * hx + 1], a.scale_idx, -l1);
                         }
                 }
                 __syncwarp();
@@ -497,12 +560,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok) {
                 // teacher P = mean over the G heads of exp(S scale - LSE_main); gradient and KL terms
                 tc_fence_after();
-                constexpr int QC = 64 / G;  // queries per 64-column TMEM chunk
+                constexpr int QC = 32 / G > 0 ? 32 / G : 1;  // queries per 32-column TMEM chunk
+                constexpr int CW = QC * G;                    // columns per chunk
 #pragma unroll
                 for (int ch = 0; ch < QPC / QC; ++ch) {
-                    uint32_t sv[64];
-                    tmem_ld32(lane_addr + sb * kRows + ch * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-                    tmem_ld32(lane_addr + sb * kRows + ch * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+                    uint32_t sv[CW];
+                    tmem_ld<CW>(lane_addr + sb * kRows + ch * CW, sv);
                     tmem_ld_wait();
                     if (ch == QPC / QC - 1) {
                         tc_fence_before();
@@ -511,17 +574,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int qq = 0; qq < QC; ++qq) {
                         const int m = ch * QC + qq;
-                        float P = 0.f;
+                        const float2* l2 = reinterpret_cast<const float2*>(&s.lse[buf][m * G]);
+                        uint64_t pacc = f2_packf(0.f, 0.f);
 #pragma unroll
-                        for (int h = 0; h < G; ++h)
-                            P += fast_exp2(fmaf(__uint_as_float(sv[qq * G + h]), sl2, -s.lse[buf][m * G + h] * kLog2e));
-                        P *= 1.f / (float)G;
-                        const bool valid = m < count && tvalid && tok <= s.qi[buf][m];
-                        const float lp = s.sidx[tt * SIP + m];
+                        for (int hp = 0; hp < G / 2; ++hp) {
+                            const float2 lv = l2[hp];
+                            const uint64_t nl = f2_mul(f2_packf(lv.x, lv.y), nlog2e);
+                            const uint64_t x2 = f2_fma(f2_pack(sv[qq * G + 2 * hp], sv[qq * G + 2 * hp + 1]), sl2x2, nl);
+                            float x0, x1;
+                            f2_unpack(x2, x0, x1);
+                            pacc = f2_add(pacc, f2_packf(fast_exp2(x0), fast_exp2(x1)));
+                        }
+                        float p0, p1;
+                        f2_unpack(pacc, p0, p1);
+                        const float P = (p0 + p1) * (1.f / (float)G);
+                        const bool valid = m < count && tvalid && tok <= (s.ent[buf][m] >> 5);
+                        const float lp = sit[tt * SIP + m];
                         const float gval = coef * (__expf(lp) - P) * a.scale_idx;
                         const float klv = P > 0.f ? P * (__logf(P) - lp) : 0.f;
-                        s.gs[tt * GSP + m] = valid ? gval : 0.f;
-                        s.sidx[tt * SIP + m] = valid ? klv : 0.f;
+                        gst[tt * GSP + m] = valid ? gval : 0.f;
+                        sit[tt * SIP + m] = valid ? klv : 0.f;
                     }
                 }
                 __syncwarp();
@@ -531,11 +603,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint32_t ah[2][4], al[2][4];
 #pragma unroll
                     for (int mt = 0; mt < 2; ++mt) {
-                        const int row = warp * 32 + mt * 16 + g8;
-                        split_tf32(s.gs[row * GSP + kq * 8 + t4], ah[mt][0], al[mt][0]);
-                        split_tf32(s.gs[(row + 8) * GSP + kq * 8 + t4], ah[mt][1], al[mt][1]);
-                        split_tf32(s.gs[row * GSP + kq * 8 + t4 + 4], ah[mt][2], al[mt][2]);
-                        split_tf32(s.gs[(row + 8) * GSP + kq * 8 + t4 + 4], ah[mt][3], al[mt][3]);
+                        const int row = wq * 32 + mt * 16 + g8;
+                        split_tf32(gst[row * GSP + kq * 8 + t4], ah[mt][0], al[mt][0]);
+                        split_tf32(gst[(row + 8) * GSP + kq * 8 + t4], ah[mt][1], al[mt][1]);
+                        split_tf32(gst[row * GSP + kq * 8 + t4 + 4], ah[mt][2], al[mt][2]);
+                        split_tf32(gst[(row + 8) * GSP + kq * 8 + t4 + 4], ah[mt][3], al[mt][3]);
                     }
 #pragma unroll
                     for (int nt = 0; nt < NDT; ++nt) {
@@ -549,34 +621,40 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            epi_bar();  // (B) gradients and KL terms of all 128 tokens are in shared memory
+            team_bar();  // (B) gradients and KL terms of all 128 tokens are in shared memory
             if (ok) {
-                // dQ_idx^T[d][q] = sum_token K_idx[token][d] g(token, q) scale_idx: (d, q) tiles over warps
+                // dQ_idx^T[d][q] = sum_token K_idx[token][d] g(token, q) scale_idx: (d, q) tiles over
+                // the team's warps, four independent accumulator chains summed at the end
                 constexpr int MT = DI / 16, NT = QPC / 8;
-                for (int x = warp; x < MT * NT; x += 4) {
+                for (int x = wq; x < MT * NT; x += 4) {
                     const int mt = x % MT, nt = x / MT;
-                    float cq[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
+                    float cq[4][4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) cq[u][v] = 0.f;
+#pragma unroll
                     for (int ks = 0; ks < kRows / 8; ++ks) {
-                        const __nv_bfloat16* k0 = &s.kb[(ks * 8 + t4) * KBP + mt * 16 + g8];
+                        const __nv_bfloat16* k0 = &kbt[(ks * 8 + t4) * KBP + mt * 16 + g8];
                         const __nv_bfloat16* k1 = k0 + 4 * KBP;
                         uint32_t bh0, bl0, bh1, bl1;
-                        split_tf32(s.gs[(ks * 8 + t4) * GSP + nt * 8 + g8], bh0, bl0);
-                        split_tf32(s.gs[(ks * 8 + t4 + 4) * GSP + nt * 8 + g8], bh1, bl1);
+                        split_tf32(gst[(ks * 8 + t4) * GSP + nt * 8 + g8], bh0, bl0);
+                        split_tf32(gst[(ks * 8 + t4 + 4) * GSP + nt * 8 + g8], bh1, bl1);
                         const uint32_t a0 = bf16_as_tf32(k0[0]), a1 = bf16_as_tf32(k0[8]);
                         const uint32_t a2 = bf16_as_tf32(k1[0]), a3 = bf16_as_tf32(k1[8]);
-                        mma_1688_tf32(cq, a0, a1, a2, a3, bh0, bh1);
-                        mma_1688_tf32(cq, a0, a1, a2, a3, bl0, bl1);
+                        mma_1688_tf32(cq[(ks & 1) * 2], a0, a1, a2, a3, bh0, bh1);
+                        mma_1688_tf32(cq[(ks & 1) * 2 + 1], a0, a1, a2, a3, bl0, bl1);
                     }
                     const int d0 = mt * 16 + g8;
 #pragma unroll
                     for (int cx = 0; cx < 2; ++cx) {
                         const int m = nt * 8 + 2 * t4 + cx;
                         if (m < count) {
-                            const size_t pr =
-                                (((size_t)b * a.N + s.qi[buf][m]) * a.H_kv + r) * K1 + s.qslot[buf][m];
-                            a.dq_part[pr * DI + d0] = cq[cx];
-                            a.dq_part[pr * DI + d0 + 8] = cq[2 + cx];
+                            const int qe = s.ent[buf][m];
+                            const size_t pr = (((size_t)b * a.N + (qe >> 5)) * a.H_kv + r) * K1 + (qe & 31);
+                            a.dq_part[pr * DI + d0] = (cq[0][cx] + cq[1][cx]) + (cq[2][cx] + cq[3][cx]);
+                            a.dq_part[pr * DI + d0 + 8] =
+                                (cq[0][2 + cx] + cq[1][2 + cx]) + (cq[2][2 + cx] + cq[3][2 + cx]);
                         }
                     }
                 }
@@ -585,23 +663,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int m = tt / TPQ, part = tt % TPQ;
                 float kl = 0.f;
 #pragma unroll 8
-                for (int j = 0; j < QPC; ++j) kl += s.sidx[(part + TPQ * j) * SIP + m];
+                for (int j = 0; j < QPC; ++j) kl += sit[(part + TPQ * j) * SIP + m];
 #pragma unroll
                 for (int o = TPQ / 2; o; o >>= 1) kl += __shfl_xor_sync(0xffffffffu, kl, o);
                 if (part == 0 && m < count) {
-                    const size_t pr = (((size_t)b * a.N + s.qi[buf][m]) * a.H_kv + r) * K1 + s.qslot[buf][m];
+                    const int qe = s.ent[buf][m];
+                    const size_t pr = (((size_t)b * a.N + (qe >> 5)) * a.H_kv + r) * K1 + (qe & 31);
                     a.kl_part[pr] = (double)kl;
                 }
-                mbar_arrive(&s.q_empty[buf]);
+                mbar_arrive(&s.meta_empty[buf]);
             }
         }
-        epi_bar();
-        if (have_dk && s.abort == 0) flush_dk();
+        team_bar();
+        if (myL >= 0 && s.abort == 0) flush_dk();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 5) tmem_dealloc(tmem, 256);
+    if (warp == kMmaWarp) tmem_dealloc(tmem, 256);
 }
 
 // One thread per (b, i, r): dQ_idx = sum of the slot partials; KL row = sum of the slot partials.
@@ -649,12 +728,12 @@ __global__ void k_kl_loss(KlArgs a) {
 template <int D, int DI, int G>
 cudaError_t launch_kl(const KlArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const void* q,
                       const void* q_idx, const void* k_idx, int num_sms, cudaStream_t st) {
-    const size_t smem = std::max<size_t>(sizeof(KlSmem<D, DI, kRows / G>) + 1024, 116 * 1024);  // one CTA per SM
+    const size_t smem = std::max<size_t>(sizeof(KlSmem<D, DI, kRows / G, kl_teams<G>(), kl_meta_stages<G>(), kl_prods<G>()>) + 1024, 116 * 1024);  // one CTA per SM
     cudaError_t e = cudaFuncSetAttribute(k_kl_kv_outer<D, DI, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     ProfScope ps("kl_kv_outer", st);
-    k_kl_kv_outer<D, DI, G><<<num_sms, kThreads, smem, st>>>(tq, tk, static_cast<const __nv_bfloat16*>(q),
+    k_kl_kv_outer<D, DI, G><<<num_sms, kl_threads<G>(), smem, st>>>(tq, tk, static_cast<const __nv_bfloat16*>(q),
                                                               static_cast<const __nv_bfloat16*>(q_idx),
                                                               static_cast<const __nv_bfloat16*>(k_idx), a);
     return cudaGetLastError();
