@@ -236,6 +236,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "memory");
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Registers written by an asynchronous tcgen05.ld hold their values only after tcgen05.wait::ld: this
+// empty asm, placed after the wait, makes every later use depend on it, so the compiler cannot move
+// a use of the loaded registers above the wait.
+template <int N>
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[N]) {
+    static_assert(N % 8 == 0, "fence in groups of 8 registers");
+#pragma unroll
+    for (int i = 0; i < N; i += 8)
+        asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]), "+r"(r[i + 5]),
+                     "+r"(r[i + 6]), "+r"(r[i + 7])::"memory");
+}
 // 32 lanes x 16 consecutive 32-bit columns from registers.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
     asm volatile(

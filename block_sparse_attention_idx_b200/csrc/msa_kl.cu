@@ -205,7 +205,7 @@ struct KlSmem {
     int4 crec[PRODS][2][32];                            // per producer warp: item records of the current /
     int cent[PRODS][2][32][QPC];                        // next chunk of 32 items and their query entries
     uint64_t q_full[2], q_empty[2], meta_full[NMETA], meta_empty[NMETA];
-    uint64_t kv_full, kv_empty, s_full[2], s_free[2], drain;
+    uint64_t kv_full, kv_empty, s_full[4], s_free[4], drain;
     uint32_t tmem_base;
     int abort;
 };
@@ -228,6 +228,8 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
     static_assert(QPC % 8 == 0 && QPC <= 64, "KL items hold 8 to 64 queries");
     static_assert(DI % 16 == 0, "index head dim must be a multiple of 16");
     static_assert(G % 2 == 0, "heads are processed in pairs");
+    // S^T buffers in TMEM, 128 columns each: one per epilogue team with two teams.
+    constexpr int kSBuf = 2;
 
     const int K1 = a.topk + 1;
     const int BK = a.block_k;
@@ -242,6 +244,8 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
         for (int x = 0; x < 2; ++x) {
             mbar_init(&s.q_full[x], 1);
             mbar_init(&s.q_empty[x], 1);
+        }
+        for (int x = 0; x < kSBuf; ++x) {
             mbar_init(&s.s_full[x], 1);
             mbar_init(&s.s_free[x], kRows);
         }
@@ -262,7 +266,7 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
         for (int x = threadIdx.x; x < NMETA * QPC * KBP / 2; x += kRows) z[x] = 0u;
     }
     if (warp == kMmaWarp) {
-        tmem_alloc(&s.tmem_base, 256);
+        tmem_alloc(&s.tmem_base, 128 * kSBuf);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -412,7 +416,7 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
             bool ok = true;
             int kv_group = -1, prevL = -1;
             for (int t = t0, n = 0; t < t1; ++t, ++n) {
-                const int buf = n & 1, sb = n & 1, ms = n % NMETA;
+                const int buf = n & 1, sb = n % kSBuf, ms = n % NMETA;
                 if (!mbar_wait(&s.meta_full[ms], (n / NMETA) & 1, a.status, 0x905)) { ok = false; break; }
                 const int L = s.rec[ms].x;
                 if (!mbar_wait(&s.q_full[buf], (n >> 1) & 1, a.status, 0x901)) { ok = false; break; }
@@ -422,7 +426,7 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
                     prevL = L;
                     if (!mbar_wait(&s.kv_full, kv_group & 1, a.status, 0x902)) { ok = false; break; }
                 }
-                if (!mbar_wait(&s.s_free[sb], ((n >> 1) & 1) ^ 1, a.status, 0x903)) { ok = false; break; }
+                if (!mbar_wait(&s.s_free[sb], ((n / kSBuf) & 1) ^ 1, a.status, 0x903)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t qa = smem_u32(s.q[buf]), ka = smem_u32(s.k);
 #pragma unroll
@@ -484,7 +488,7 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
         };
 
         for (int t = t0 + team, n = team; t < t1; t += TEAMS, n += TEAMS) {
-            const int buf = n % NMETA, sb = n & 1;
+            const int buf = n % NMETA, sb = n % kSBuf;
             team_bar();  // (A) the team's previous item is done with gs / sidx / kb
             bool ok = s.abort == 0;
             if (ok) ok = mbar_wait(&s.meta_full[buf], (n / NMETA) & 1, a.status, 0xa01);
@@ -554,7 +558,7 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
                 }
                 __syncwarp();
             }
-            if (ok) ok = mbar_wait(&s.s_full[sb], (n >> 1) & 1, a.status, 0xa02);
+            if (ok) ok = mbar_wait(&s.s_full[sb], (n / kSBuf) & 1, a.status, 0xa02);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) s.abort = 1;
             if (ok) {
@@ -562,28 +566,49 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
                 tc_fence_after();
                 constexpr int QC = 32 / G > 0 ? 32 / G : 1;  // queries per 32-column TMEM chunk
                 constexpr int CW = QC * G;                    // columns per chunk
+                constexpr int NCH = QPC / QC;
+                static_assert(G % 4 == 0 || G == 2, "LSE_main rows are read four or two at a time");
+                // the next chunk's TMEM load is in flight while the current one is processed
+                uint32_t sv[2][CW];
+                tmem_ld<CW>(lane_addr + sb * kRows, sv[0]);
 #pragma unroll
-                for (int ch = 0; ch < QPC / QC; ++ch) {
-                    uint32_t sv[CW];
-                    tmem_ld<CW>(lane_addr + sb * kRows + ch * CW, sv);
+                for (int ch = 0; ch < NCH; ++ch) {
                     tmem_ld_wait();
-                    if (ch == QPC / QC - 1) {
+                    reg_fence(sv[ch & 1]);
+                    if (ch + 1 < NCH) {
+                        tmem_ld<CW>(lane_addr + sb * kRows + (ch + 1) * CW, sv[(ch + 1) & 1]);
+                    } else {
                         tc_fence_before();
                         mbar_arrive(&s.s_free[sb]);
                     }
+                    const uint32_t* cv = sv[ch & 1];
 #pragma unroll
                     for (int qq = 0; qq < QC; ++qq) {
                         const int m = ch * QC + qq;
-                        const float2* l2 = reinterpret_cast<const float2*>(&s.lse[buf][m * G]);
                         uint64_t pacc = f2_packf(0.f, 0.f);
+                        if constexpr (G % 4 == 0) {
+                            const float4* l4 = reinterpret_cast<const float4*>(&s.lse[buf][m * G]);
 #pragma unroll
-                        for (int hp = 0; hp < G / 2; ++hp) {
-                            const float2 lv = l2[hp];
-                            const uint64_t nl = f2_mul(f2_packf(lv.x, lv.y), nlog2e);
-                            const uint64_t x2 = f2_fma(f2_pack(sv[qq * G + 2 * hp], sv[qq * G + 2 * hp + 1]), sl2x2, nl);
-                            float x0, x1;
-                            f2_unpack(x2, x0, x1);
-                            pacc = f2_add(pacc, f2_packf(fast_exp2(x0), fast_exp2(x1)));
+                            for (int hq = 0; hq < G / 4; ++hq) {
+                                const float4 lv = l4[hq];
+                                const uint64_t nl0 = f2_mul(f2_packf(lv.x, lv.y), nlog2e);
+                                const uint64_t nl1 = f2_mul(f2_packf(lv.z, lv.w), nlog2e);
+                                const uint64_t x0 = f2_fma(f2_pack(cv[qq * G + 4 * hq], cv[qq * G + 4 * hq + 1]), sl2x2, nl0);
+                                const uint64_t x1 =
+                                    f2_fma(f2_pack(cv[qq * G + 4 * hq + 2], cv[qq * G + 4 * hq + 3]), sl2x2, nl1);
+                                float e0, e1, e2, e3;
+                                f2_unpack(x0, e0, e1);
+                                f2_unpack(x1, e2, e3);
+                                pacc = f2_add(pacc, f2_packf(fast_exp2(e0), fast_exp2(e1)));
+                                pacc = f2_add(pacc, f2_packf(fast_exp2(e2), fast_exp2(e3)));
+                            }
+                        } else {
+                            const float2 lv = *reinterpret_cast<const float2*>(&s.lse[buf][m * G]);
+                            const uint64_t x0 =
+                                f2_fma(f2_pack(cv[qq * G], cv[qq * G + 1]), sl2x2, f2_mul(f2_packf(lv.x, lv.y), nlog2e));
+                            float e0, e1;
+                            f2_unpack(x0, e0, e1);
+                            pacc = f2_packf(fast_exp2(e0), fast_exp2(e1));
                         }
                         float p0, p1;
                         f2_unpack(pacc, p0, p1);
@@ -680,7 +705,7 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == kMmaWarp) tmem_dealloc(tmem, 256);
+    if (warp == kMmaWarp) tmem_dealloc(tmem, 128 * kSBuf);
 }
 
 // One thread per (b, i, r): dQ_idx = sum of the slot partials; KL row = sum of the slot partials.
