@@ -25,76 +25,136 @@ namespace {
 constexpr int kRows = 128;
 constexpr float kLog2e = 1.4426950408889634f;
 
-__device__ __forceinline__ void load_bf16_row(const __nv_bfloat16* src, float* dst, int n) {
-#pragma unroll
-    for (int c = 0; c < n; c += 8) {
-        const uint4 u = *reinterpret_cast<const uint4*>(src + c);
-        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            const float2 f = __bfloat1622float2(h[x]);
-            dst[c + 2 * x] = f.x;
-            dst[c + 2 * x + 1] = f.y;
-        }
-    }
-}
-
 // ============================================================================ LSE_idx pass
-// Item = one selected block c of group r and up to kIdxQpc queries. Thread t owns token c*BK+t.
-// Writes (max, sum-exp) of the scaled index logits of every (query, slot) over its causal tokens.
+// Item = one selected block c of group r and up to kIdxQpc queries; each CTA takes a contiguous
+// range of items, so the block's K_idx rows stay in shared memory across the items of one list.
+// The index logits of the item (128 tokens x 32 queries) come from bf16 mma.sync, warp w holding
+// tokens 32w..32w+31; each warp reduces its tokens to a (max, sum-exp) pair per query and the four
+// pairs are merged in a fixed order into the (query, slot) partial.
 template <int DI>
 __global__ void __launch_bounds__(128) k_lse_idx(KlArgs a, const __nv_bfloat16* __restrict__ q_idx,
                                                   const __nv_bfloat16* __restrict__ k_idx) {
-    __shared__ float s_q[kIdxQpc][DI];
-    __shared__ float s_s[kIdxQpc][129];
-    __shared__ int s_i[kIdxQpc], s_slot[kIdxQpc];
+    constexpr int QP = kIdxQpc;
+    constexpr int KBP = DI + 8;  // bf16 row pitch: ldmatrix rows on distinct banks
+    static_assert(QP == 32, "four query n-tiles per item");
+    __shared__ alignas(16) __nv_bfloat16 kb[kRows * KBP];
+    __shared__ alignas(16) __nv_bfloat16 qb[QP * KBP];
+    __shared__ float red_m[4][QP], red_s[4][QP];
+    __shared__ int s_i[QP], s_slot[QP];
     const Csr& cs = a.csr_idx;
     const int T = *cs.n_items;
-    const int t = threadIdx.x;
-    float kr[DI];
-    int prevL = -1;
-    for (int item = blockIdx.x; item < T; item += gridDim.x) {
-        const int4 it = cs.items[item];
+    const int per = (T + gridDim.x - 1) / gridDim.x;
+    const int t0 = blockIdx.x * per, t1 = min(T, t0 + per);
+    const int tt = threadIdx.x, warp = tt >> 5, lane = tt & 31;
+    const int g8 = lane >> 2, t4 = lane & 3;
+    const int K1 = a.topk + 1;
+    const uint32_t kb_u32 = smem_u32(kb), qb_u32 = smem_u32(qb);
+    int curL = -1;
+    for (int t = t0; t < t1; ++t) {
+        const int4 it = cs.items[t];
         const int L = it.x, count = it.z;
         const int c = L % cs.nb, r = (L / cs.nb) % a.H_kv, b = L / (cs.nb * a.H_kv);
-        const int tok = c * a.block_k + t;
-        const bool tvalid = t < a.block_k && tok < a.N;
-        __syncthreads();  // previous item done with s_q / s_s / s_i
-        if (L != prevL) {
-            if (tvalid) load_bf16_row(k_idx + ((size_t)b * a.N + tok) * DI, kr, DI);
-            prevL = L;
+        __syncthreads();  // the previous item is done with kb / qb / s_i / red
+        if (L != curL) {
+            const int tok = c * a.block_k + tt;
+            const bool tvalid = tt < a.block_k && tok < a.N;
+#pragma unroll
+            for (int x = 0; x < DI / 8; ++x) {
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (tvalid) v = *reinterpret_cast<const uint4*>(k_idx + ((size_t)b * a.N + tok) * DI + x * 8);
+                *reinterpret_cast<uint4*>(&kb[tt * KBP + x * 8]) = v;
+            }
+            curL = L;
         }
-        if (t < count) {
-            const int e = cs.entries[it.y + t];
-            s_i[t] = e >> 5;
-            s_slot[t] = e & 31;
+        if (tt < QP) {
+            const int e = tt < count ? cs.entries[it.y + tt] : 0;
+            s_i[tt] = tt < count ? (e >> 5) : -1;
+            s_slot[tt] = e & 31;
+        }
+        for (int x = tt; x < QP * (DI / 8); x += 128) {
+            const int m = x / (DI / 8), part = x % (DI / 8);
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (m < count) {
+                const int qi = cs.entries[it.y + m] >> 5;
+                v = *reinterpret_cast<const uint4*>(q_idx + (((size_t)b * a.N + qi) * a.H_kv + r) * DI + part * 8);
+            }
+            *reinterpret_cast<uint4*>(&qb[m * KBP + part * 8]) = v;
         }
         __syncthreads();
-        for (int x = t; x < count * DI; x += 128) {
-            const int m = x / DI, dd = x % DI;
-            s_q[m][dd] = __bfloat162float(q_idx[(((size_t)b * a.N + s_i[m]) * a.H_kv + r) * DI + dd]);
+        float acc[2][4][4];
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int x = 0; x < 4; ++x) acc[mt][nt][x] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < DI / 16; ++ks) {
+            uint32_t af[2][4];
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+                const uint32_t ad = kb_u32 + ((warp * 32 + mt * 16 + (lane & 15)) * KBP + ks * 16 + (lane >> 4) * 8) * 2;
+                asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                             : "=r"(af[mt][0]), "=r"(af[mt][1]), "=r"(af[mt][2]), "=r"(af[mt][3])
+                             : "r"(ad));
+            }
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+                uint32_t bf[4];
+                const uint32_t ad =
+                    qb_u32 + ((np * 16 + (lane & 7) + ((lane >> 4) << 3)) * KBP + ks * 16 + ((lane >> 3) & 1) * 8) * 2;
+                asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                             : "=r"(bf[0]), "=r"(bf[1]), "=r"(bf[2]), "=r"(bf[3])
+                             : "r"(ad));
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt) {
+                    mma_16816_bf16(acc[mt][2 * np], af[mt], bf[0], bf[1]);
+                    mma_16816_bf16(acc[mt][2 * np + 1], af[mt], bf[2], bf[3]);
+                }
+            }
         }
+        // per query: the warp's (max, sum-exp) over its 32 tokens
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int cx = 0; cx < 2; ++cx) {
+                const int m = nt * 8 + 2 * t4 + cx;
+                const int qi = s_i[m];
+                float v[4];
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int hx = 0; hx < 2; ++hx) {
+                        const int row = warp * 32 + mt * 16 + g8 + 8 * hx;
+                        const int tok = c * a.block_k + row;
+                        const bool ok = m < count && row < a.block_k && tok < a.N && tok <= qi;
+                        v[mt * 2 + hx] = ok ? acc[mt][nt][2 * hx + cx] * a.scale_idx : -INFINITY;
+                    }
+                float mx = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                float z = 0.f;
+                if (mx != -INFINITY) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) z += v[u] == -INFINITY ? 0.f : __expf(v[u] - mx);
+                }
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+                if (g8 == 0) {
+                    red_m[warp][m] = mx;
+                    red_s[warp][m] = z;
+                }
+            }
         __syncthreads();
-        for (int m = 0; m < count; ++m) {
-            float acc = 0.f;
+        if (tt < count) {
+            float M = -INFINITY;
 #pragma unroll
-            for (int dd = 0; dd < DI; ++dd) acc = fmaf(s_q[m][dd], kr[dd], acc);
-            s_s[m][t] = (tvalid && tok <= s_i[m]) ? acc * a.scale_idx : -INFINITY;
-        }
-        __syncthreads();
-        // one warp per query: max and sum-exp over the 128 token lanes
-        const int w = t >> 5, ln = t & 31;
-        for (int m = w; m < count; m += 4) {
-            float mx = -INFINITY;
-            for (int x = ln; x < 128; x += 32) mx = fmaxf(mx, s_s[m][x]);
+            for (int w = 0; w < 4; ++w) M = fmaxf(M, red_m[w][tt]);
+            float Z = 0.f;
 #pragma unroll
-            for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            float z = 0.f;
-            for (int x = ln; x < 128; x += 32) z += s_s[m][x] == -INFINITY ? 0.f : __expf(s_s[m][x] - mx);
-#pragma unroll
-            for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-            if (ln == 0)
-                a.ml_part[(((size_t)b * a.N + s_i[m]) * a.H_kv + r) * (a.topk + 1) + s_slot[m]] = make_float2(mx, z);
+            for (int w = 0; w < 4; ++w)
+                if (red_m[w][tt] != -INFINITY) Z += red_s[w][tt] * __expf(red_m[w][tt] - M);
+            a.ml_part[(((size_t)b * a.N + s_i[tt]) * a.H_kv + r) * K1 + s_slot[tt]] = make_float2(M, Z);
         }
     }
 }
@@ -708,31 +768,51 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
     if (warp == kMmaWarp) tmem_dealloc(tmem, 128 * kSBuf);
 }
 
-// One thread per (b, i, r): dQ_idx = sum of the slot partials; KL row = sum of the slot partials.
+// One warp per (b, i, r): dQ_idx = sum of the slot partials, KL row = sum of the slot partials, both
+// in ascending slot order (each slot's dQ_idx row read as one coalesced 4 * d_idx byte segment).
 template <int DI>
 __global__ void k_kl_rows(KlArgs a) {
-    const long long row = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
     if (row >= (long long)a.B * a.N * a.H_kv) return;
     const int K1 = a.topk + 1;
     const int i = (int)((row / a.H_kv) % a.N);
     const int32_t* sel = a.blocks + row * K1;
-    float acc[DI];
-#pragma unroll
-    for (int x = 0; x < DI; ++x) acc[x] = 0.f;
-    double kl = 0.0;
-    int prev = -1;
-    for (int s = 0; s < K1; ++s) {
-        const int c = sel[s];
-        if (c < 0 || c > i / a.block_k || c <= prev) continue;
-        prev = c;
-        const float* dp = a.dq_part + (row * K1 + s) * DI;
-#pragma unroll
-        for (int x = 0; x < DI; ++x) acc[x] += dp[x];
-        kl += a.kl_part[row * K1 + s];
+    // slots holding a distinct causal block (the same rule as the list build)
+    uint32_t mask = 0;
+    if (lane == 0) {
+        int prev = -1;
+        for (int s = 0; s < K1; ++s) {
+            const int c = sel[s];
+            if (c < 0 || c > i / a.block_k || c <= prev) continue;
+            prev = c;
+            mask |= 1u << s;
+        }
     }
+    mask = __shfl_sync(0xffffffffu, mask, 0);
+    constexpr int VPL = DI / 32;  // dQ_idx values per lane
+    float acc[VPL];
 #pragma unroll
-    for (int x = 0; x < DI; ++x) a.dq_idx[row * DI + x] = acc[x];
-    a.kl_rows[row] = kl;
+    for (int x = 0; x < VPL; ++x) acc[x] = 0.f;
+    for (uint32_t m = mask; m; m &= m - 1) {
+        const int s = __ffs(m) - 1;
+        const float* dp = a.dq_part + (row * K1 + s) * DI + lane * VPL;
+        if constexpr (VPL == 2) {
+            const float2 v = *reinterpret_cast<const float2*>(dp);
+            acc[0] += v.x;
+            acc[1] += v.y;
+        } else {
+            acc[0] += dp[0];
+        }
+    }
+    if constexpr (VPL == 2)
+        *reinterpret_cast<float2*>(a.dq_idx + row * DI + lane * 2) = make_float2(acc[0], acc[1]);
+    else
+        a.dq_idx[row * DI + lane] = acc[0];
+    const double kv = (lane < K1 && ((mask >> lane) & 1u)) ? a.kl_part[row * K1 + lane] : 0.0;
+    double kl = 0.0;
+    for (int s = 0; s < K1; ++s) kl += __shfl_sync(0xffffffffu, kv, s);
+    if (lane == 0) a.kl_rows[row] = kl;
 }
 
 // Single CTA: loss = sum of the KL rows / (B N H_kv), in a fixed order (float64).
@@ -775,9 +855,9 @@ cudaError_t run_lse_idx(const KlArgs& a, const void* q_idx, const void* k_idx, i
     const auto* ki = static_cast<const __nv_bfloat16*>(k_idx);
     ProfScope ps("lse_idx", st);
     if (a.d_idx == 64)
-        k_lse_idx<64><<<num_sms * 8, 128, 0, st>>>(a, qi, ki);
+        k_lse_idx<64><<<num_sms * 6, 128, 0, st>>>(a, qi, ki);
     else
-        k_lse_idx<32><<<num_sms * 8, 128, 0, st>>>(a, qi, ki);
+        k_lse_idx<32><<<num_sms * 6, 128, 0, st>>>(a, qi, ki);
     const long long rows = (long long)a.B * a.N * a.H_kv;
     k_lse_idx_merge<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(a);
     return cudaGetLastError();
@@ -805,10 +885,11 @@ cudaError_t run_kl(const KlArgs& a, const void* q, const void* k, const void* q_
     if (e != cudaSuccess) return e;
     const long long rows = (long long)a.B * a.N * a.H_kv;
     ProfScope ps("kl_finalize", st);
+    const unsigned grid_rows = (unsigned)((rows * 32 + 255) / 256);
     if (a.d_idx == 64)
-        k_kl_rows<64><<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(a);
+        k_kl_rows<64><<<grid_rows, 256, 0, st>>>(a);
     else
-        k_kl_rows<32><<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(a);
+        k_kl_rows<32><<<grid_rows, 256, 0, st>>>(a);
     k_kl_loss<<<1, 1024, 0, st>>>(a);
     return cudaGetLastError();
 }
