@@ -11,15 +11,15 @@
 // The normalised partial (o = O / sum P, lse) of every row goes to its (query, head, slot) place
 // in the workspace (fp16 o, fp32 lse). A second kernel combines each (query, group) row's <= topk+1
 // partials with the log-sum-exp rule and writes the bf16 output and the LSE. Items are handed out
-// in (window, group, block) order by an atomic counter, four at a time, so consecutive items of a
-// CTA often share their K/V block; a wide window fills items with more queries.
+// in (window, group, block) order by an atomic counter, up to 16 at a time, so consecutive items of
+// a CTA often share their K/V block; a wide window fills items with more queries.
 //
-// Warp roles (608 threads): warps 0-15 run the softmax and the epilogue of every item (warp w: TMEM
-// lane quarter w % 4, column quarter w / 4), warp 16 hands out items (prefetching the next item's
-// record and query list), stages their metadata and loads Q (TMA gather of each query's G head rows)
-// and K, warp 17 loads V, warp 18 issues the MMAs and owns TMEM. Q, K, V and the two accumulators
-// (S/P and O) are double-buffered; the MMA issuer polls and issues whichever of the next S or the
-// next PV is ready.
+// Warp roles (640 threads): warps 0-15 run the softmax and the epilogue of every item (warp w: TMEM
+// lane quarter w % 4, column quarter w / 4), warp 16 hands out items and stages their metadata,
+// warps 17 and 18 each gather half of an item's Q rows (TMA, each query's G head rows) and load K
+// and V respectively, warp 19 issues the MMAs and owns TMEM. Q, K, V and the two accumulators (S/P
+// and O) are double-buffered; the MMA issuer polls and issues whichever of the next S or the next
+// PV is ready.
 #include "msa_common.cuh"
 #include "msa_internal.h"
 
@@ -29,13 +29,14 @@ namespace {
 
 constexpr int kRows = 128;
 constexpr int kMeta = 4;        // depth of the item metadata ring
-constexpr int kGrab = 4;        // items taken per scheduler fetch
 constexpr int kEpiWarps = 16;   // warps 0..15: softmax / epilogue, two teams of 8
 constexpr int kTeamWarps = 8;
-constexpr int kProdWarp = 16;   // items, metadata, Q and K
-constexpr int kVWarp = 17;      // V
-constexpr int kMmaWarp = 18;    // MMA issue, TMEM owner
-constexpr int kThreads = 19 * 32;
+constexpr int kSchedWarp = 16;  // hands out items, stages their metadata
+constexpr int kQKWarp = 17;     // first half of each item's Q rows, K
+constexpr int kQVWarp = 18;     // second half of each item's Q rows, V
+constexpr int kMmaWarp = 19;    // MMA issue, TMEM owner
+constexpr int kThreads = 20 * 32;
+constexpr int kStage = 512;     // query entries staged per scheduler fetch
 
 struct ItemMeta {
     int t;  // item index; -1: no more items
@@ -52,6 +53,7 @@ struct AttnSmem {
     alignas(1024) uint8_t k[2][kKVBytes];
     alignas(1024) uint8_t v[2][kKVBytes];
     ItemMeta meta[kMeta];
+    int stage[kStage];  // query entries of the items of the current scheduler fetch
     // per-row partial max / sums of the two column halves: [team][team item parity][half][row]
     float red_max[2][2][2][kRows], red_l[2][2][2][kRows], red_lr[2][2][2][kRows];
     uint64_t meta_full[kMeta], meta_empty[kMeta];
@@ -92,10 +94,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int x = 0; x < kMeta; ++x) {
             mbar_init(&s.meta_full[x], 1);
-            mbar_init(&s.meta_empty[x], 2 + kTeamWarps);  // V loader, MMA issuer, the item's team
+            mbar_init(&s.meta_empty[x], 3 + kTeamWarps);  // both Q loaders, the MMA issuer, the item's team
         }
         for (int x = 0; x < 2; ++x) {
-            mbar_init(&s.q_full[x], 1);
+            mbar_init(&s.q_full[x], 2);  // one arrival per Q loader
             mbar_init(&s.q_empty[x], 1);
             mbar_init(&s.k_full[x], 1);
             mbar_init(&s.v_full[x], 1);
@@ -122,87 +124,92 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = s.tmem_base;
 
-    if (warp == kProdWarp) {
-        // ------------------------------------------------------------ items, metadata, Q and K
-        // The record and query list of the next item are loaded one item ahead, so their global
-        // latency overlaps the waits of the current item.
-        int prevL = -1, kgroup = -1;
+    if (warp == kSchedWarp) {
+        // ------------------------------------------------------------ item scheduler
+        // Takes CH consecutive items per atomic fetch (their records, one per lane, and their query
+        // entries, one contiguous range of the list arrays), then stages the items' metadata one by
+        // one. No global load is in flight when a metadata slot is released to its consumers.
+        const int QPC = max(1, kRows / G);
+        const int CH = min(16, kStage / QPC);
+        int n = 0, prevL = -1;
         bool ok = true;
-        int batch = 0;
-        if (lane == 0) batch = atomicAdd(a.sched, kGrab);
-        batch = __shfl_sync(0xffffffffu, batch, 0);
-        int t_nx = batch;
-        int4 rec_nx = t_nx < T ? a.csr.items[t_nx] : make_int4(-1, 0, 0, 0);
-        int e_nx[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int m = lane + 32 * j;
-            e_nx[j] = (t_nx < T && m < rec_nx.z) ? a.csr.entries[rec_nx.y + m] : 0;
-        }
-        for (int n = 0;; ++n) {
-            const int t = t_nx;
-            const int4 rec = rec_nx;
-            int e[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) e[j] = e_nx[j];
-            // prefetch item n+1
-            if ((n + 1) % kGrab == 0) {
-                int b2 = 0;
-                if (lane == 0) b2 = atomicAdd(a.sched, kGrab);
-                batch = __shfl_sync(0xffffffffu, b2, 0);
-                t_nx = batch;
-            } else {
-                t_nx = batch + (n + 1) % kGrab;
-            }
-            if (t_nx < T) {
-                rec_nx = a.csr.items[t_nx];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int m = lane + 32 * j;
-                    e_nx[j] = m < rec_nx.z ? a.csr.entries[rec_nx.y + m] : 0;
-                }
-            }
-            const int slot = n % kMeta;
-            if (!wait_lane0(&s.meta_empty[slot], ((n / kMeta) & 1) ^ 1, a.status, 0x501)) { ok = false; break; }
-            ItemMeta& mt = s.meta[slot];
-            if (t >= T || s.abort) {
+        while (ok) {
+            int base = 0;
+            if (lane == 0) base = s.abort ? T : atomicAdd(a.sched, CH);
+            base = __shfl_sync(0xffffffffu, base, 0);
+            if (base >= T) {
                 // two end markers: one for each epilogue team
-                if (lane == 0) { mt.t = -1; mbar_arrive(&s.meta_full[slot]); }
-                const int slot2 = (n + 1) % kMeta;
-                if (!wait_lane0(&s.meta_empty[slot2], (((n + 1) / kMeta) & 1) ^ 1, a.status, 0x502)) { ok = false; break; }
-                if (lane == 0) { s.meta[slot2].t = -1; mbar_arrive(&s.meta_full[slot2]); }
+                for (int x = 0; x < 2 && ok; ++x, ++n) {
+                    const int slot = n % kMeta;
+                    if (!wait_lane0(&s.meta_empty[slot], ((n / kMeta) & 1) ^ 1, a.status, 0x501)) { ok = false; break; }
+                    if (lane == 0) { s.meta[slot].t = -1; mbar_arrive(&s.meta_full[slot]); }
+                }
                 break;
             }
-            const int L = rec.x, count = rec.z;
-            const int c = L % a.csr.nb;
-            const int r = (L / a.csr.nb) % a.H_kv;
-            const int b = L / (a.csr.nb * a.H_kv * a.csr.nW);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int m = lane + 32 * j;
-                if (m < count) {
-                    mt.qi[m] = e[j] >> 5;
-                    mt.qs[m] = (int8_t)(e[j] & 31);
-                }
-            }
-            if (lane == 0) {
-                mt.t = t; mt.b = b; mt.r = r; mt.c = c; mt.count = count; mt.kv_new = (L != prevL);
-            }
+            const int cnt = min(CH, T - base);
+            const int4 rec = lane < cnt ? a.csr.items[base + lane] : make_int4(-1, 0, 0, 0);
+            // the entries of consecutive items are contiguous in the list arrays
+            const int y0 = __shfl_sync(0xffffffffu, rec.y, 0);
+            const int y1 = __shfl_sync(0xffffffffu, rec.y + rec.z, cnt - 1);
+            for (int x = lane; x < y1 - y0; x += 32) s.stage[x] = a.csr.entries[y0 + x];
             __syncwarp();
-            if (lane == 0) mbar_arrive(&s.meta_full[slot]);
-            // Q: the G head rows of each query of the item
-            const int buf = n & 1;
-            if (!wait_lane0(&s.q_empty[buf], ((n >> 1) & 1) ^ 1, a.status, 0x503)) { ok = false; break; }
-            if (G >= 8) {
-                if (lane == 0) mbar_arrive_expect_tx(&s.q_full[buf], (uint32_t)(count * G * D * 2));
-                __syncwarp();
+            for (int j = 0; j < cnt; ++j, ++n) {
+                const int L = __shfl_sync(0xffffffffu, rec.x, j);
+                const int off = __shfl_sync(0xffffffffu, rec.y, j) - y0;
+                const int count = __shfl_sync(0xffffffffu, rec.z, j);
+                const int slot = n % kMeta;
+                if (!wait_lane0(&s.meta_empty[slot], ((n / kMeta) & 1) ^ 1, a.status, 0x502)) { ok = false; break; }
+                ItemMeta& mt = s.meta[slot];
                 for (int m = lane; m < count; m += 32) {
+                    const int e = s.stage[off + m];
+                    mt.qi[m] = e >> 5;
+                    mt.qs[m] = (int8_t)(e & 31);
+                }
+                if (lane == 0) {
+                    mt.t = base + j;
+                    mt.c = L % a.csr.nb;
+                    mt.r = (L / a.csr.nb) % a.H_kv;
+                    mt.b = L / (a.csr.nb * a.H_kv * a.csr.nW);
+                    mt.count = count;
+                    mt.kv_new = (L != prevL);
+                }
+                prevL = L;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s.meta_full[slot]);
+            }
+            __syncwarp();  // the staged entries are read before the next fetch overwrites them
+        }
+        if (!ok) s.abort = 1;
+    } else if (warp == kQKWarp || warp == kQVWarp) {
+        // ------------------------------------------------------------ Q (half each), K / V
+        // Both warps gather Q rows (the TMA issue rate of one warp is the limit otherwise): the
+        // first loads the first half of the item's queries and the K blocks, the second the other
+        // half and the V blocks. All their barriers carry TMA data only: relaxed arrives.
+        const bool is_k = warp == kQKWarp;
+        int group = -1, n_issued = 0;
+        bool ok = true;
+        for (int n = 0;; ++n) {
+            const int slot = n % kMeta;
+            if (!wait_lane0(&s.meta_full[slot], (n / kMeta) & 1, a.status, 0x511)) { ok = false; break; }
+            const ItemMeta& mt = s.meta[slot];
+            const int t = mt.t;
+            if (t < 0) break;
+            const int b = mt.b, r = mt.r, c = mt.c, count = mt.count, kv_new = mt.kv_new;
+            const int half = (count + 1) >> 1;
+            const int m0 = is_k ? 0 : half, m1 = is_k ? half : count;
+            const int buf = n & 1;
+            if (!wait_lane0(&s.q_empty[buf], ((n >> 1) & 1) ^ 1, a.status, 0x512)) { ok = false; break; }
+            if (G >= 8) {
+                if (lane == 0) mbar_arrive_expect_tx_relaxed(&s.q_full[buf], (uint32_t)((m1 - m0) * G * D * 2));
+                __syncwarp();
+                for (int m = m0 + lane; m < m1; m += 32) {
 #pragma unroll
                     for (int sub = 0; sub < D / 64; ++sub)
                         tma_load_4d(s.q[buf] + sub * (kRows * 128) + m * G * 128, &tm_q, &s.q_full[buf], sub * 64,
                                     r * G, mt.qi[m], b);
                 }
-            } else {
+            } else if (is_k) {
+                // few heads per group: one warp copies every row, then makes them visible to the MMA
                 const uint32_t qsm = smem_u32(s.q[buf]);
                 constexpr int kChunksPerRow = D * 2 / 16;
                 for (int x = lane; x < count * G * kChunksPerRow; x += 32) {
@@ -216,56 +223,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                 fence_proxy_async();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s.q_full[buf]);
+            } else {
+                if (lane == 0) mbar_arrive_relaxed(&s.q_full[buf]);
             }
-            // K of block group g goes to buffer g % 2 once the S MMAs of group g-2 (the buffer's
-            // previous use, release number (g-2)/2 of that buffer) are done
-            if (L != prevL) {
-                ++kgroup;
-                if (kgroup >= 2 &&
-                    !wait_lane0(&s.k_release[kgroup & 1], ((kgroup - 2) >> 1) & 1, a.status, 0x504)) { ok = false; break; }
+            ++n_issued;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.meta_empty[slot]);
+            // K (or V) of block group g goes to buffer g % 2 once the MMAs of group g-2 that read it
+            // (the buffer's previous use, release number (g-2)/2) are done
+            if (kv_new) {
+                ++group;
+                uint64_t* rel = is_k ? s.k_release : s.v_release;
+                if (group >= 2 &&
+                    !wait_lane0(&rel[group & 1], ((group - 2) >> 1) & 1, a.status, 0x513)) { ok = false; break; }
                 if (lane == 0) {
-                    const int kb = kgroup & 1;
-                    mbar_arrive_expect_tx(&s.k_full[kb], (uint32_t)Sm::kKVBytes);
+                    const int kb = group & 1;
+                    uint64_t* full = is_k ? &s.k_full[kb] : &s.v_full[kb];
+                    uint8_t* dst = is_k ? s.k[kb] : s.v[kb];
+                    const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
+                    mbar_arrive_expect_tx_relaxed(full, (uint32_t)Sm::kKVBytes);
 #pragma unroll
                     for (int sub = 0; sub < D / 64; ++sub)
-                        tma_load_4d(s.k[kb] + sub * BK * 128, &tm_k, &s.k_full[kb], sub * 64, r, c * BK, b);
+                        tma_load_4d(dst + sub * BK * 128, tm, full, sub * 64, r, c * BK, b);
                 }
-                prevL = L;
             }
         }
         if (!ok) s.abort = 1;
         if (lane == 0) {  // no copy of ours may still be landing when the CTA leaves
-            for (int g = max(0, kgroup - 1); g <= kgroup; ++g) mbar_wait(&s.k_full[g & 1], (g >> 1) & 1, a.status, 0x505);
-        }
-    } else if (warp == kVWarp) {
-        // ------------------------------------------------------------ V loader
-        int vgroup = -1;
-        bool ok = true;
-        for (int n = 0;; ++n) {
-            const int slot = n % kMeta;
-            if (!wait_lane0(&s.meta_full[slot], (n / kMeta) & 1, a.status, 0x511)) { ok = false; break; }
-            const ItemMeta& mt = s.meta[slot];
-            const int t = mt.t, b = mt.b, r = mt.r, c = mt.c, kv_new = mt.kv_new;
-            __syncwarp();
-            if (lane == 0 && t >= 0) mbar_arrive(&s.meta_empty[slot]);
-            if (t < 0) break;
-            if (kv_new) {
-                // V of block group g goes to buffer g % 2 once the PV MMAs of group g-2 are done
-                ++vgroup;
-                if (vgroup >= 2 &&
-                    !wait_lane0(&s.v_release[vgroup & 1], ((vgroup - 2) >> 1) & 1, a.status, 0x512)) { ok = false; break; }
-                if (lane == 0) {
-                    const int vb = vgroup & 1;
-                    mbar_arrive_expect_tx(&s.v_full[vb], (uint32_t)Sm::kKVBytes);
-#pragma unroll
-                    for (int sub = 0; sub < D / 64; ++sub)
-                        tma_load_4d(s.v[vb] + sub * BK * 128, &tm_v, &s.v_full[vb], sub * 64, r, c * BK, b);
-                }
+            uint64_t* full = is_k ? s.k_full : s.v_full;
+            for (int g = max(0, group - 1); g <= group; ++g) mbar_wait(&full[g & 1], (g >> 1) & 1, a.status, 0x514);
+            for (int x = 0; x < 2 && x < n_issued; ++x) {
+                const int nl = n_issued - 1 - x;
+                mbar_wait(&s.q_full[nl & 1], (nl >> 1) & 1, a.status, 0x515);
             }
-        }
-        if (!ok) s.abort = 1;
-        if (lane == 0) {
-            for (int g = max(0, vgroup - 1); g <= vgroup; ++g) mbar_wait(&s.v_full[g & 1], (g >> 1) & 1, a.status, 0x513);
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
