@@ -199,15 +199,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int m0 = is_k ? 0 : half, m1 = is_k ? half : count;
             const int buf = n & 1;
             if (!wait_lane0(&s.q_empty[buf], ((n >> 1) & 1) ^ 1, a.status, 0x512)) { ok = false; break; }
-            if (G >= 8) {
+            if (G % 8 == 0) {
                 if (lane == 0) mbar_arrive_expect_tx_relaxed(&s.q_full[buf], (uint32_t)((m1 - m0) * G * D * 2));
                 __syncwarp();
-                for (int m = m0 + lane; m < m1; m += 32) {
-#pragma unroll
-                    for (int sub = 0; sub < D / 64; ++sub)
-                        tma_load_4d(s.q[buf] + sub * (kRows * 128) + m * G * 128, &tm_q, &s.q_full[buf], sub * 64,
-                                    r * G, mt.qi[m], b);
-                }
+                for (int m = m0 + lane; m < m1; m += 32)
+                    tma_load_5d(s.q[buf] + m * G * D * 2, &tm_q, &s.q_full[buf], 0, 0, 0, r * G / 8,
+                                b * a.N + mt.qi[m]);
             } else if (is_k) {
                 // few heads per group: one warp copies every row, then makes them visible to the MMA
                 const uint32_t qsm = smem_u32(s.q[buf]);
@@ -217,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int m = row / G, h = row % G;
                     const __nv_bfloat16* src =
                         q + ((((size_t)b * a.N + mt.qi[m]) * a.H_q + (size_t)r * G + h) * D + ch * 8);
-                    cp_async_16(qsm + ((ch * 16) / 128) * (kRows * 128) + swz(row, (ch * 16) % 128, 128), src);
+                    cp_async_16(qsm + qtile_off<D>(row, ch * 16), src);
                 }
                 cp_async_wait_all();
                 fence_proxy_async();
@@ -308,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int ks = 0; ks < D / 16; ++ks) {
                             const uint32_t sub = (ks * 16) / 64, off = (ks & 3) * 32;
-                            const uint64_t da = umma_sdesc(qb + sub * (kRows * 128) + off, 16, 1024, 2);
+                            const uint64_t da = umma_sdesc(qb + sub * 1024 + off, 16, (D / 64) * 1024, 2);
                             const uint64_t db = umma_sdesc(kb + sub * (BK * 128) + off, 16, 1024, 2);
                             umma_bf16(tS, da, db, kIdescS, ks > 0);
                         }
@@ -673,15 +670,16 @@ cudaError_t run_attn(const AttnArgs& a, const void* q, const void* k, const void
     e = cudaMemsetAsync(a.sched, 0, 4, st);
     if (e != cudaSuccess) return e;
     CUtensorMap tq, tk, tv;
-    const uint64_t dq[4] = {(uint64_t)a.d, (uint64_t)a.H_q, (uint64_t)a.N, (uint64_t)a.B};
-    const uint64_t sq[3] = {(uint64_t)a.d * 2, (uint64_t)a.H_q * a.d * 2, (uint64_t)a.N * a.H_q * a.d * 2};
-    const uint32_t bq[4] = {64, (uint32_t)std::min(G, 256), 1, 1};
     const uint64_t dkv[4] = {(uint64_t)a.d, (uint64_t)a.H_kv, (uint64_t)a.N, (uint64_t)a.B};
     const uint64_t skv[3] = {(uint64_t)a.d * 2, (uint64_t)a.H_kv * a.d * 2, (uint64_t)a.N * a.H_kv * a.d * 2};
     const uint32_t bkv[4] = {64, 1, (uint32_t)a.block_k, 1};
-    if (!make_tmap_4d(&tq, q, dq, sq, bq, 128) || !make_tmap_4d(&tk, k, dkv, skv, bkv, 128) ||
-        !make_tmap_4d(&tv, v, dkv, skv, bkv, 128))
+    if (!make_tmap_4d(&tk, k, dkv, skv, bkv, 128) || !make_tmap_4d(&tv, v, dkv, skv, bkv, 128))
         return cudaErrorInvalidValue;
+    if (G % 8 == 0) {
+        if (!make_tmap_qrows(&tq, q, a.B, a.N, a.H_q, a.d, G)) return cudaErrorInvalidValue;
+    } else {
+        tq = tk;  // not read: the query rows are copied without TMA
+    }
     if (a.d == 128) {
         if (a.block_k == 128) return launch_attn<128, 128>(a, tq, tk, tv, q, num_sms, st);
         if (a.block_k == 64) return launch_attn<128, 64>(a, tq, tk, tv, q, num_sms, st);

@@ -122,6 +122,14 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
         "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
         : "memory");
 }
+__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z,
+                                            int w, int v) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, "
+        "%6, %7}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(v)
+        : "memory");
+}
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
@@ -333,6 +341,14 @@ __device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t byte_in_row, uint
     uint32_t off = row * pitch + byte_in_row;
     uint32_t mask = pitch == 128 ? 7u : (pitch == 64 ? 3u : 1u);
     return off ^ (((off >> 7) & mask) << 4);
+}
+// Query-row tiles (128 rows x D bf16) are stored as 1024-byte 128B-swizzled atoms of 8 rows x 64
+// columns, ordered [row / 8][column / 64]: the G head rows of one query (G a multiple of 8) are one
+// contiguous block that a single 5-D TMA box fills, and the MMA reads the tile as a K-major operand
+// whose 8-row atoms are D / 64 KB apart. Byte offset of (row, byte of the row) in such a tile:
+template <int D>
+__device__ __forceinline__ uint32_t qtile_off(uint32_t row, uint32_t byte_in_row) {
+    return (row >> 3) * (D / 64) * 1024 + (byte_in_row >> 7) * 1024 + swz(row & 7, byte_in_row & 127, 128);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

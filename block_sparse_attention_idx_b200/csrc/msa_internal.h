@@ -29,6 +29,9 @@ bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, ui
                   uint64_t stride2, uint32_t box0, uint32_t box1, uint32_t box2, int swizzle_bytes);
 bool make_tmap_4d(CUtensorMap* m, const void* base, const uint64_t dims[4], const uint64_t strides[3],
                   const uint32_t box[4], int swizzle_bytes);
+// Query rows [B, N, H_q, d] as 5-D boxes of one query's G heads (G % 8 == 0, H_q % 8 == 0, d % 64 == 0)
+// laid out in 8-row x 64-column 128B-swizzled atoms.
+bool make_tmap_qrows(CUtensorMap* m, const void* q, int B, int N, int H_q, int d, int G);
 
 // ---------------------------------------------------------------- index Top-k (msa_index.cu)
 struct IndexArgs {

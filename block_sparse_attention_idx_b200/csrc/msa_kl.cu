@@ -397,15 +397,12 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
                 // Q: the G head rows of each query, in the 128B-swizzled K-major tile the MMA reads
                 if (lane == 0) okl = mbar_wait(&s.q_empty[buf], ((n >> 1) & 1) ^ 1, a.status, 0x805);
                 if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
-                if constexpr (G >= 8) {
+                if constexpr (G % 8 == 0) {
                     if (lane == 0) mbar_arrive_expect_tx_relaxed(&s.q_full[buf], (uint32_t)(count * G * D * 2));
                     __syncwarp();
-                    for (int m = lane; m < count; m += 32) {
-#pragma unroll
-                        for (int sub = 0; sub < D / 64; ++sub)
-                            tma_load_4d(s.q[buf] + sub * (kRows * 128) + m * G * 128, &tm_q, &s.q_full[buf],
-                                        sub * 64, r * G, qe[m] >> 5, b);
-                    }
+                    for (int m = lane; m < count; m += 32)
+                        tma_load_5d(s.q[buf] + m * G * D * 2, &tm_q, &s.q_full[buf], 0, 0, 0, r * G / 8,
+                                    b * a.N + (qe[m] >> 5));
                 } else {
                     const uint32_t qs = smem_u32(s.q[buf]);
                     constexpr int kChunksPerRow = D * 2 / 16;
@@ -414,7 +411,7 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
                         const int m = row / G, h = row % G;
                         const __nv_bfloat16* src =
                             q + ((((size_t)b * a.N + (qe[m] >> 5)) * a.H_q + (size_t)r * G + h) * D + ch * 8);
-                        cp_async_16(qs + ((ch * 16) / 128) * (kRows * 128) + swz(row, (ch * 16) % 128, 128), src);
+                        cp_async_16(qs + qtile_off<D>(row, ch * 16), src);
                     }
                     cp_async_wait_all();
                     fence_proxy_async();
@@ -493,7 +490,7 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
                 for (int ks = 0; ks < D / 16; ++ks) {
                     const uint32_t sub = (ks * 16) / 64, off = (ks & 3) * 32;
                     const uint64_t da = umma_sdesc(ka + sub * (kRows * 128) + off, 16, 1024, 2);
-                    const uint64_t db = umma_sdesc(qa + sub * (kRows * 128) + off, 16, 1024, 2);
+                    const uint64_t db = umma_sdesc(qa + sub * 1024 + off, 16, (D / 64) * 1024, 2);
                     umma_bf16(tmem + sb * kRows, da, db, kIdesc, ks > 0);
                 }
                 umma_commit(&s.s_full[sb]);
@@ -867,14 +864,15 @@ cudaError_t run_kl(const KlArgs& a, const void* q, const void* k, const void* q_
                    cudaStream_t st) {
     const int G = a.H_q / a.H_kv;
     CUtensorMap tq, tk;
-    const uint64_t dq[4] = {(uint64_t)a.d, (uint64_t)a.H_q, (uint64_t)a.N, (uint64_t)a.B};
-    const uint64_t sq[3] = {(uint64_t)a.d * 2, (uint64_t)a.H_q * a.d * 2, (uint64_t)a.N * a.H_q * a.d * 2};
-    const uint32_t bq[4] = {64, (uint32_t)std::min(G, 256), 1, 1};
     const uint64_t dims[4] = {(uint64_t)a.d, (uint64_t)a.H_kv, (uint64_t)a.N, (uint64_t)a.B};
     const uint64_t strides[3] = {(uint64_t)a.d * 2, (uint64_t)a.H_kv * a.d * 2, (uint64_t)a.N * a.H_kv * a.d * 2};
     const uint32_t box[4] = {64, 1, (uint32_t)a.block_k, 1};
-    if (!make_tmap_4d(&tq, q, dq, sq, bq, 128) || !make_tmap_4d(&tk, k, dims, strides, box, 128))
-        return cudaErrorInvalidValue;
+    if (!make_tmap_4d(&tk, k, dims, strides, box, 128)) return cudaErrorInvalidValue;
+    if (G % 8 == 0) {
+        if (!make_tmap_qrows(&tq, q, a.B, a.N, a.H_q, a.d, G)) return cudaErrorInvalidValue;
+    } else {
+        tq = tk;  // not read: the query rows are copied without TMA
+    }
     cudaError_t e = cudaMemsetAsync(a.dk_idx, 0, (size_t)a.B * a.N * a.d_idx * 4, st);
     if (e != cudaSuccess) return e;
     if (a.d == 128 && G == 16) e = launch_kl<128, 64, 16>(a, tq, tk, q, q_idx, k_idx, num_sms, st);

@@ -60,4 +60,13 @@ bool make_tmap_4d(CUtensorMap* m, const void* base, const uint64_t dims[4], cons
     return encode(m, base, 4, dims, strides, box, swizzle_bytes);
 }
 
+bool make_tmap_qrows(CUtensorMap* m, const void* q, int B, int N, int H_q, int d, int G) {
+    // dims: column within a 64-column half, head within a group of 8, column half, group of 8 heads,
+    // query (batch-major); one box = the G heads x d columns of one query in 8-row x 64-column atoms
+    const uint64_t dims[5] = {64, 8, (uint64_t)d / 64, (uint64_t)H_q / 8, (uint64_t)B * N};
+    const uint64_t strides[4] = {(uint64_t)d * 2, 128, (uint64_t)8 * d * 2, (uint64_t)H_q * d * 2};
+    const uint32_t box[5] = {64, 8, (uint32_t)d / 64, (uint32_t)G / 8, 1};
+    return encode(m, q, 5, dims, strides, box, 128);
+}
+
 }  // namespace msa
