@@ -124,12 +124,18 @@ def valid_slots(blocks: torch.Tensor, block_k: int) -> int:
 # ncu capture of the kernel; it holds only for the kernel source it was measured on (sha256 of the
 # file), and reads null once that file changes.
 MEASURED_TRAFFIC = {
-    # prefill_8k capture (dram read 213,596,416 B + write 1,974,181,632 B per launch over 60,309,504
+    # prefill_8k capture (dram read 233,849,344 B + write 1,971,176,448 B per launch over 60,309,504
     # selected tokens), scaled by the selected tokens of the timed launch
     "attn_kv_outer": {"file": "block_sparse_attention_idx_b200/csrc/msa_attn.cu",
-                      "sha256": "703ca7f5d95ead89b2d8050621f55f8205311920ade863251340ffc79dc52422",
-                      "bytes_per_unit": (213596416 + 1974181632) / 60309504, "unit": "selected token",
+                      "sha256": "bc28a00638a31a27274af096224e7045b44ea20be2cc75208377eb36eaaa5ccb",
+                      "bytes_per_unit": (233849344 + 1971176448) / 60309504, "unit": "selected token",
                       "capture": "profiles/attn_kv_outer_prefill_8k.md"},
+    # training capture at N=8192 (dram read 976,273,152 B + write 136,482,560 B per launch over
+    # 60,309,504 selected tokens), scaled by the selected tokens of the timed launch
+    "kl_kv_outer": {"file": "block_sparse_attention_idx_b200/csrc/msa_kl.cu",
+                    "sha256": "18b2cd05ba8bd860913a08262712d229a3e533033a53a5e00349e2684a6e5c7e",
+                    "bytes_per_unit": (976273152 + 136482560) / 60309504, "unit": "selected token",
+                    "capture": "profiles/kl_kv_outer_train_8k.md"},
 }
 
 
@@ -355,8 +361,9 @@ def bench_prefill(args, world, rank, msa, pk):
 def bench_decode(args, world, rank, msa, pk):
     w = WORKLOADS["decode_16x256k"]
     dev = torch.device("cuda", torch.cuda.current_device())
-    x = decode_inputs(w, device=dev, seed=rank_seed(w, rank))
-    dims = msa.MsaDims(w.B, w.N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
+    L = args.decode_len or w.N
+    x = decode_inputs(w, device=dev, seed=rank_seed(w, rank), L=L)
+    dims = msa.MsaDims(w.B, L, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
     ws = msa.workspace(msa.MSA_OP_DECODE, dims, dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
@@ -367,7 +374,6 @@ def bench_decode(args, world, rank, msa, pk):
     for _ in range(max(3, args.warmup)):
         out, blocks = step()
     torch.cuda.synchronize()
-    L = w.N
     nscored = ((L - 1) // w.block_k) * w.block_k
     scan_bytes = w.B * nscored * w.d_idx * 2
     sel_blocks = int((blocks >= 0).sum().item())
@@ -404,7 +410,7 @@ def bench_decode(args, world, rank, msa, pk):
     msa.msa_profile_enable(False)
     prof = profile_avg(msa.msa_profile_read())
     scan_ms = prof["dec_scan"]["avg_ms"]
-    res = {"workload": "decode_16x256k", "us_per_step": us, "us_per_token": us, "tokens_per_s": w.B * world / (us * 1e-6),
+    res = {"workload": "decode_16x256k" if L == w.N else f"decode_16x{L}", "us_per_step": us, "us_per_token": us, "tokens_per_s": w.B * world / (us * 1e-6),
            "us_per_step_graph": us_graph, "bytes_per_step": step_bytes,
            "step_roofline": roofline_entry("hbm", step_bytes / (us * 1e-6) / 1e9, pk["hbm_gbs"], "GB/s"),
            "step_roofline_graph": roofline_entry("hbm", step_bytes / (us_graph * 1e-6) / 1e9, pk["hbm_gbs"], "GB/s")
@@ -422,8 +428,9 @@ def bench_decode(args, world, rank, msa, pk):
 def bench_train(args, world, rank, msa, pk):
     w = WORKLOADS["train_64k"]
     dev = torch.device("cuda", torch.cuda.current_device())
-    x = prefill_inputs(w, device=dev, seed=rank_seed(w, rank))
-    dims = msa.MsaDims(w.B, w.N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
+    N = args.train_n or w.N
+    x = prefill_inputs(w, device=dev, seed=rank_seed(w, rank), N=N)
+    dims = msa.MsaDims(w.B, N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
     ws_i = msa.workspace(msa.MSA_OP_INDEX_TOPK_LSE, dims, dev)
     ws_a = msa.workspace(msa.MSA_OP_ATTN_FWD, dims, dev)
     ws_k = msa.workspace(msa.MSA_OP_KL, dims, dev)
@@ -449,9 +456,11 @@ def bench_train(args, world, rank, msa, pk):
     prof = profile_avg(msa.msa_profile_read())
     ms = max_over_ranks(sum(t) / len(t), world)
     kl_ms = prof["kl_kv_outer"]["avg_ms"]
-    res = {"workload": "train_64k", "ms_per_step": ms, "loss": float(loss.item()),
-           "roofline": {**roofline_entry("tensor", kl_flops / (kl_ms * 1e-3) / 1e12, pk["bf16_tflops"], "TFLOP/s"),
+    res = {"workload": "train_64k" if N == w.N else f"train_{N}", "ms_per_step": ms, "loss": float(loss.item()),
+           "roofline": {**roofline_entry("tensor", kl_flops / (kl_ms * 1e-3) / 1e12, pk["bf16_tflops"], "TFLOP/s",
+                                         measured_traffic("kl_kv_outer", sel_tok)),
                         "kernel": "kl_kv_outer", "flops_per_launch": kl_flops},
+           "work": {"selected_tokens": sel_tok, "kl_flops": kl_flops},
            "kernels": {k: {"avg_ms": round(v["avg_ms"], 4), "launches": v["launches"]} for k, v in prof.items()}}
     del x, ws_a, ws_k
     torch.cuda.empty_cache()
@@ -473,6 +482,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--workload", default=HEADLINE, choices=["prefill_8k", "prefill_32k_needles", "train_64k"],
                     help="prefill workload of the headline step (smaller ones serve profiler captures)")
+    ap.add_argument("--only", choices=["decode", "train"], default=None,
+                    help="profiler captures: run only this secondary measurement and print its object")
+    ap.add_argument("--decode-len", type=int, default=0, help="profiler captures: decode cache length")
+    ap.add_argument("--train-n", type=int, default=0, help="profiler captures: training sequence length")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -487,6 +500,13 @@ def main():
     world, rank, local = dist_setup(args.gpus)
     import block_sparse_attention_idx_b200 as msa
     pk = peaks()
+    if args.only:
+        res = (bench_decode if args.only == "decode" else bench_train)(args, world, rank, msa, pk)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"only": args.only, args.only: res}), flush=True)
+        return
     pre = bench_prefill(args, world, rank, msa, pk)
     w = WORKLOADS[args.workload]
     line = {"metric": METRIC, "value": pre["value"], "unit": "query-tokens/s", "n_gpus": world,
