@@ -44,15 +44,16 @@ def peaks():
 
 
 class ClockSampler:
-    """SM clock and clock-event (throttle) reasons read through NVML every 10 ms in a background
-    thread while the timed region runs (read-only queries; no setting is changed)."""
+    """SM clock and clock-event (throttle) reasons read through NVML every 2 ms in a background
+    thread while the timed region runs (read-only queries; no setting is changed). Entering waits
+    until the first sample is in, so sampling covers the whole timed region."""
     REASONS = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
                "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
                "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
                "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
                "hw_power_brake": "nvmlClocksEventReasonHwPowerBrakeSlowdown"}
 
-    def __init__(self, gpu_index: int, period_s: float = 0.01):
+    def __init__(self, gpu_index: int, period_s: float = 0.002):
         self.gpu, self.period = gpu_index, period_s
         self.samples, self.max_mhz, self.err = [], None, None
         self._stop = None
@@ -87,7 +88,9 @@ class ClockSampler:
         self._stop = threading.Event()
         self._t = threading.Thread(target=self._run, daemon=True)
         self._t.start()
-        time.sleep(0.05)
+        t0 = time.time()
+        while not self.samples and self.err is None and time.time() - t0 < 5.0:
+            time.sleep(0.005)
         return self
 
     def __exit__(self, *exc):
@@ -95,12 +98,14 @@ class ClockSampler:
         self._t.join(timeout=5)
 
     def summary(self) -> dict:
+        if len(self.samples) > 2:
+            self.samples = self.samples[1:]  # the first one is taken before the timed region starts
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"], "samples": 0,
                     "error": self.err}
         reasons = sorted({r for _, rs in self.samples for r in rs})
         return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": reasons, "samples": len(self.samples), "source": "nvml, 10 ms"}
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml, 2 ms"}
 
 
 def selected_tokens(blocks: torch.Tensor, block_k: int) -> int:
