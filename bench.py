@@ -414,15 +414,18 @@ def bench_decode(args, world, rank, msa, pk):
     timed_steps(step, args.decode_steps, flush)
     msa.msa_profile_enable(False)
     prof = profile_avg(msa.msa_profile_read())
-    scan_ms = prof["dec_scan"]["avg_ms"]
+    # the batch may be cut into parts (one scan launch each): time per step = total / steps
+    scan_ms = prof["dec_scan"]["total_ms"] / args.decode_steps
     res = {"workload": "decode_16x256k" if L == w.N else f"decode_16x{L}", "us_per_step": us, "us_per_token": us, "tokens_per_s": w.B * world / (us * 1e-6),
            "us_per_step_graph": us_graph, "bytes_per_step": step_bytes,
            "step_roofline": roofline_entry("hbm", step_bytes / (us * 1e-6) / 1e9, pk["hbm_gbs"], "GB/s"),
            "step_roofline_graph": roofline_entry("hbm", step_bytes / (us_graph * 1e-6) / 1e9, pk["hbm_gbs"], "GB/s")
            if us_graph == us_graph else None,
            "roofline": {**roofline_entry("hbm", scan_bytes / (scan_ms * 1e-3) / 1e9, pk["hbm_gbs"], "GB/s"),
-                        "kernel": "dec_scan", "bytes_per_launch": scan_bytes},
-           "kernels": {k: {"avg_ms": round(v["avg_ms"], 4), "launches": v["launches"]} for k, v in prof.items()}}
+                        "kernel": "dec_scan", "bytes_per_step": scan_bytes,
+                        "launches_per_step": prof["dec_scan"]["launches"] // args.decode_steps},
+           "kernels": {k: {"ms_per_step": round(v["total_ms"] / args.decode_steps, 4),
+                           "launches_per_step": v["launches"] // args.decode_steps} for k, v in prof.items()}}
     if graph_note:
         res["graph_note"] = graph_note
     del x, ws

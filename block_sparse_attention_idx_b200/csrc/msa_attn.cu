@@ -186,6 +186,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // first loads the first half of the item's queries and the K blocks, the second the other
         // half and the V blocks. All their barriers carry TMA data only: relaxed arrives.
         const bool is_k = warp == kQKWarp;
+        // a query's rows are read again by the items of its other selected blocks: keep them in L2
+        const uint64_t q_policy = l2_policy_evict_last();
         int group = -1, n_issued = 0;
         bool ok = true;
         for (int n = 0;; ++n) {
@@ -203,8 +205,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) mbar_arrive_expect_tx_relaxed(&s.q_full[buf], (uint32_t)((m1 - m0) * G * D * 2));
                 __syncwarp();
                 for (int m = m0 + lane; m < m1; m += 32)
-                    tma_load_5d(s.q[buf] + m * G * D * 2, &tm_q, &s.q_full[buf], 0, 0, 0, r * G / 8,
-                                b * a.N + mt.qi[m]);
+                    tma_load_5d_hint(s.q[buf] + m * G * D * 2, &tm_q, &s.q_full[buf], 0, 0, 0, r * G / 8,
+                                     b * a.N + mt.qi[m], q_policy);
             } else if (is_k) {
                 // few heads per group: one warp copies every row, then makes them visible to the MMA
                 const uint32_t qsm = smem_u32(s.q[buf]);
@@ -388,6 +390,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         float pv_mx = 0.f;
         // O of the team's item number kp: normalise by the row's rounded weight sum, store the fp16
         // partial and its LSE, free the accumulator
+        // the partials are written once here and read once by the merge: they must not push the
+        // query rows out of L2
+        const uint64_t part_policy = l2_policy_evict_first();
         auto store_prev = [&](int kp) -> bool {
             const int pb = kp & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(&s.o_full[t], pb, a.status, 0x704))) return false;
@@ -415,7 +420,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
 #pragma unroll
                     for (int x = 0; x < 4; ++x)
-                        dst[(size_t)((e * OC + c0) / 8 + x) * G] = make_uint4(hv[4 * x], hv[4 * x + 1], hv[4 * x + 2], hv[4 * x + 3]);
+                        st_global_v4_hint(&dst[(size_t)((e * OC + c0) / 8 + x) * G],
+                                          make_uint4(hv[4 * x], hv[4 * x + 1], hv[4 * x + 2], hv[4 * x + 3]),
+                                          part_policy);
                 }
             }
             if (e == 0 && pv_prow >= 0)
