@@ -224,6 +224,12 @@ __device__ __forceinline__ void cp_async_ca(uint32_t dst, const void* src) {
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
+// D += A(16x8, bf16, row) * B(8x8, bf16, col), fp32 accumulate.
+__device__ __forceinline__ void mma_1688_bf16(float (&c)[4], const uint32_t (&a)[2], uint32_t b) {
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(b));
+}
 // x ~= hi + lo with both parts tf32: products with a tf32-exact operand keep ~fp32 accuracy.
 __device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
     hi = to_tf32(x);
@@ -257,7 +263,13 @@ struct KlSmem {
     alignas(16) __nv_bfloat16 kb[TEAMS][kRows * KBP];   // K_idx rows of each team's block (zero past the end)
     alignas(16) __nv_bfloat16 qb[NMETA][QPC * KBP];     // Q_idx rows of the item queries
     alignas(16) float lse[NMETA][kRows];                // LSE_main of the item rows (query-major, head-minor)
-    float gs[TEAMS][kRows * GSP];                       // g * scale_idx per (token, query)
+    // g * scale_idx per (token, query): fp32 for the tf32 gradient products (items of more than 16
+    // queries), or split as bf16 hi + lo in [token][query] and [query][token] order for the bf16 ones
+    static constexpr bool kBf = QPC <= 16;
+    static constexpr int GBP = kRows + 8;
+    float gs[TEAMS][kBf ? 1 : kRows * GSP];
+    alignas(16) __nv_bfloat16 ga[TEAMS][2][kBf ? kRows * QPC : 8];
+    alignas(16) __nv_bfloat16 gb[TEAMS][2][kBf ? QPC * GBP : 8];
     float sidx[TEAMS][kRows * SIP];                     // log P_idx per (token, query), then the KL terms
     float lidx[NMETA][QPC];                             // LSE_idx of the item queries
     int ent[NMETA][QPC];                                // query entries (i << 5 | slot) of the item
@@ -511,7 +523,6 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
         const int g8 = lane >> 2, t4 = lane & 3;
         const uint32_t lane_addr = tmem + ((uint32_t)(wq * 32) << 16);
         const uint64_t sl2x2 = f2_packf(a.scale * kLog2e, a.scale * kLog2e);
-        const uint64_t nlog2e = f2_packf(-kLog2e, -kLog2e);
         __nv_bfloat16* kbt = s.kb[team];
         float* gst = s.gs[team];
         float* sit = s.sidx[team];
@@ -615,6 +626,11 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
                 }
                 __syncwarp();
             }
+            if (ok) {
+                // LSE_main of the item's rows, pre-scaled once: exp(S scale - LSE) = 2^(S sl2 + lse')
+                s.lse[buf][tt] *= -kLog2e;
+            }
+            team_bar();  // the scaled LSE_main values of the whole item are in place
             if (ok) ok = mbar_wait(&s.s_full[sb], (n / kSBuf) & 1, a.status, 0xa02);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) s.abort = 1;
@@ -627,6 +643,7 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
                 static_assert(G % 4 == 0 || G == 2, "LSE_main rows are read four or two at a time");
                 // the next chunk's TMEM load is in flight while the current one is processed
                 uint32_t sv[2][CW];
+                alignas(16) __nv_bfloat16 gha[Sm::kBf ? QPC : 8], gla[Sm::kBf ? QPC : 8];
                 tmem_ld<CW>(lane_addr + sb * kRows, sv[0]);
 #pragma unroll
                 for (int ch = 0; ch < NCH; ++ch) {
@@ -648,11 +665,10 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
 #pragma unroll
                             for (int hq = 0; hq < G / 4; ++hq) {
                                 const float4 lv = l4[hq];
-                                const uint64_t nl0 = f2_mul(f2_packf(lv.x, lv.y), nlog2e);
-                                const uint64_t nl1 = f2_mul(f2_packf(lv.z, lv.w), nlog2e);
-                                const uint64_t x0 = f2_fma(f2_pack(cv[qq * G + 4 * hq], cv[qq * G + 4 * hq + 1]), sl2x2, nl0);
-                                const uint64_t x1 =
-                                    f2_fma(f2_pack(cv[qq * G + 4 * hq + 2], cv[qq * G + 4 * hq + 3]), sl2x2, nl1);
+                                const uint64_t x0 =
+                                    f2_fma(f2_pack(cv[qq * G + 4 * hq], cv[qq * G + 4 * hq + 1]), sl2x2, f2_packf(lv.x, lv.y));
+                                const uint64_t x1 = f2_fma(f2_pack(cv[qq * G + 4 * hq + 2], cv[qq * G + 4 * hq + 3]), sl2x2,
+                                                           f2_packf(lv.z, lv.w));
                                 float e0, e1, e2, e3;
                                 f2_unpack(x0, e0, e1);
                                 f2_unpack(x1, e2, e3);
@@ -661,8 +677,7 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
                             }
                         } else {
                             const float2 lv = *reinterpret_cast<const float2*>(&s.lse[buf][m * G]);
-                            const uint64_t x0 =
-                                f2_fma(f2_pack(cv[qq * G], cv[qq * G + 1]), sl2x2, f2_mul(f2_packf(lv.x, lv.y), nlog2e));
+                            const uint64_t x0 = f2_fma(f2_pack(cv[qq * G], cv[qq * G + 1]), sl2x2, f2_packf(lv.x, lv.y));
                             float e0, e1;
                             f2_unpack(x0, e0, e1);
                             pacc = f2_packf(fast_exp2(e0), fast_exp2(e1));
@@ -674,12 +689,56 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
                         const float lp = sit[tt * SIP + m];
                         const float gval = coef * (__expf(lp) - P) * a.scale_idx;
                         const float klv = P > 0.f ? P * (__logf(P) - lp) : 0.f;
-                        gst[tt * GSP + m] = valid ? gval : 0.f;
+                        const float gv = valid ? gval : 0.f;
+                        if constexpr (Sm::kBf) {
+                            const __nv_bfloat16 hi = __float2bfloat16_rn(gv);
+                            const __nv_bfloat16 lo = __float2bfloat16_rn(gv - __bfloat162float(hi));
+                            gha[m] = hi;
+                            gla[m] = lo;
+                            s.gb[team][0][m * Sm::GBP + tt] = hi;
+                            s.gb[team][1][m * Sm::GBP + tt] = lo;
+                        } else {
+                            gst[tt * GSP + m] = gv;
+                        }
                         sit[tt * SIP + m] = valid ? klv : 0.f;
                     }
                 }
+                if constexpr (Sm::kBf) {
+#pragma unroll
+                    for (int x = 0; x < QPC; x += 8) {
+                        *reinterpret_cast<uint4*>(&s.ga[team][0][tt * QPC + x]) = *reinterpret_cast<const uint4*>(&gha[x]);
+                        *reinterpret_cast<uint4*>(&s.ga[team][1][tt * QPC + x]) = *reinterpret_cast<const uint4*>(&gla[x]);
+                    }
+                }
                 __syncwarp();
-                // dK_idx[token] += sum_q g(token, q) scale_idx Q_idx[q]   (tf32 mma, gradient split in two)
+                // dK_idx[token] += sum_q g(token, q) scale_idx Q_idx[q]: bf16 mma, gradient split in hi + lo
+                if constexpr (Sm::kBf) {
+                    const uint32_t ga_hi = smem_u32(s.ga[team][0]), ga_lo = smem_u32(s.ga[team][1]);
+                    const uint32_t qbu = smem_u32(s.qb[buf]);
+#pragma unroll
+                    for (int kq = 0; kq < QPC / 8; ++kq) {
+                        uint32_t ah[2][2], al[2][2];
+#pragma unroll
+                        for (int mt = 0; mt < 2; ++mt) {
+                            const uint32_t off = ((wq * 32 + mt * 16 + (lane & 15)) * QPC + kq * 8) * 2;
+                            ldsm_x2(ga_hi + off, ah[mt][0], ah[mt][1]);
+                            ldsm_x2(ga_lo + off, al[mt][0], al[mt][1]);
+                        }
+#pragma unroll
+                        for (int j = 0; j < NDT / 4; ++j) {
+                            uint32_t bq[4];
+                            ldsm_x4_trans(qbu + ((kq * 8 + (lane & 7)) * KBP + (j * 4 + (lane >> 3)) * 8) * 2, bq[0], bq[1],
+                                          bq[2], bq[3]);
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                                for (int mt = 0; mt < 2; ++mt) {
+                                    mma_1688_bf16(dk[mt][j * 4 + u], ah[mt], bq[u]);
+                                    mma_1688_bf16(dk[mt][j * 4 + u], al[mt], bq[u]);
+                                }
+                        }
+                    }
+                } else
 #pragma unroll
                 for (int kq = 0; kq < QPC / 8; ++kq) {
                     uint32_t ah[2][4], al[2][4];
@@ -708,6 +767,37 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
                 // dQ_idx^T[d][q] = sum_token K_idx[token][d] g(token, q) scale_idx: (d, q) tiles over
                 // the team's warps, four independent accumulator chains summed at the end
                 constexpr int MT = DI / 16, NT = QPC / 8;
+                if constexpr (Sm::kBf) {
+                    // K_idx^T fragments by transposed ldmatrix of the token-major tile, the gradient's
+                    // (query, token) hi and lo rows by ldmatrix; hi and lo in separate accumulators
+                    const uint32_t kbu = smem_u32(kbt);
+                    for (int x = wq; x < MT * NT; x += 4) {
+                        const int mt = x % MT, nt = x / MT;
+                        float ch[4] = {0.f, 0.f, 0.f, 0.f}, cl[4] = {0.f, 0.f, 0.f, 0.f};
+                        const uint32_t gsrc = smem_u32(s.gb[team][lane >> 4]);
+#pragma unroll
+                        for (int ks = 0; ks < kRows / 16; ++ks) {
+                            uint32_t af[4], bg[4];
+                            ldsm_x4_trans(kbu + ((ks * 16 + (lane & 7) + ((lane >> 4) << 3)) * KBP + mt * 16 +
+                                                 ((lane >> 3) & 1) * 8) * 2,
+                                          af[0], af[1], af[2], af[3]);
+                            ldsm_x4(gsrc + ((nt * 8 + (lane & 7)) * Sm::GBP + ks * 16 + ((lane >> 3) & 1) * 8) * 2, bg);
+                            mma_16816_bf16(ch, af, bg[0], bg[1]);
+                            mma_16816_bf16(cl, af, bg[2], bg[3]);
+                        }
+                        const int d0 = mt * 16 + g8;
+#pragma unroll
+                        for (int cx = 0; cx < 2; ++cx) {
+                            const int m = nt * 8 + 2 * t4 + cx;
+                            if (m < count) {
+                                const int qe = s.ent[buf][m];
+                                const size_t pr = (((size_t)b * a.N + (qe >> 5)) * a.H_kv + r) * K1 + (qe & 31);
+                                a.dq_part[pr * DI + d0] = ch[cx] + cl[cx];
+                                a.dq_part[pr * DI + d0 + 8] = ch[2 + cx] + cl[2 + cx];
+                            }
+                        }
+                    }
+                } else
                 for (int x = wq; x < MT * NT; x += 4) {
                     const int mt = x % MT, nt = x / MT;
                     float cq[4][4];
