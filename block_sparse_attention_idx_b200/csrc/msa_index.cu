@@ -148,21 +148,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool got = mbar_wait(&s.acc_full[acc], (kt >> 1) & 1, a.status, 0x301);
             if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             tc_fence_after();
+            // the tile's 128 scores of this row: four loads in flight, one wait, then the maxima of
+            // its 32-column chunks (three-input max)
             float cmax[4];
+            {
+                uint32_t v[4][32];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t v0[32], v1[32];
-                tmem_ld32(lane_addr + acc * kCols + half * 64, v0);
-                tmem_ld32(lane_addr + acc * kCols + half * 64 + 32, v1);
+                for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(lane_addr + acc * kCols + q4 * 32, v[q4]);
                 tmem_ld_wait();
-                float m0 = __uint_as_float(v0[0]), m1 = __uint_as_float(v1[0]);
 #pragma unroll
-                for (int c = 1; c < 32; ++c) {
-                    m0 = fmaxf(m0, __uint_as_float(v0[c]));
-                    m1 = fmaxf(m1, __uint_as_float(v1[c]));
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    reg_fence(v[q4]);
+                    const float* f = reinterpret_cast<const float*>(v[q4]);
+                    float m0 = max3f(f[0], f[1], f[2]), m1 = max3f(f[3], f[4], f[5]);
+#pragma unroll
+                    for (int c = 6; c < 30; c += 4) {  // columns 6 .. 29
+                        m0 = max3f(m0, f[c], f[c + 1]);
+                        m1 = max3f(m1, f[c + 2], f[c + 3]);
+                    }
+                    cmax[q4] = max3f(m0, m1, fmaxf(f[30], f[31]));
                 }
-                cmax[half * 2] = m0;
-                cmax[half * 2 + 1] = m1;
             }
             tc_fence_before();
             mbar_arrive(&s.acc_empty[acc]);
