@@ -129,17 +129,17 @@ def valid_slots(blocks: torch.Tensor, block_k: int) -> int:
 # ncu capture of the kernel; it holds only for the kernel source it was measured on (sha256 of the
 # file), and reads null once that file changes.
 MEASURED_TRAFFIC = {
-    # prefill_8k capture (dram read 233,849,344 B + write 1,971,176,448 B per launch over 60,309,504
+    # prefill_8k capture (dram read 206,054,656 B + write 1,970,213,120 B per launch over 60,309,504
     # selected tokens), scaled by the selected tokens of the timed launch
     "attn_kv_outer": {"file": "block_sparse_attention_idx_b200/csrc/msa_attn.cu",
-                      "sha256": "bc28a00638a31a27274af096224e7045b44ea20be2cc75208377eb36eaaa5ccb",
-                      "bytes_per_unit": (233849344 + 1971176448) / 60309504, "unit": "selected token",
+                      "sha256": "55bbdf3d16d2cb6f83b7bcb203d7af9aa655fe16e19d10c2c80fd62fe8a7188e",
+                      "bytes_per_unit": (206054656 + 1970213120) / 60309504, "unit": "selected token",
                       "capture": "profiles/attn_kv_outer_prefill_8k.md"},
-    # training capture at N=8192 (dram read 976,273,152 B + write 136,482,560 B per launch over
+    # training capture at N=8192 (dram read 991,507,200 B + write 136,743,680 B per launch over
     # 60,309,504 selected tokens), scaled by the selected tokens of the timed launch
     "kl_kv_outer": {"file": "block_sparse_attention_idx_b200/csrc/msa_kl.cu",
-                    "sha256": "18b2cd05ba8bd860913a08262712d229a3e533033a53a5e00349e2684a6e5c7e",
-                    "bytes_per_unit": (976273152 + 136482560) / 60309504, "unit": "selected token",
+                    "sha256": "14cb19baa5ea1a26ed617e36066629b07b8a9f99a90d086cb3700db4150cafa5",
+                    "bytes_per_unit": (991507200 + 136743680) / 60309504, "unit": "selected token",
                     "capture": "profiles/kl_kv_outer_train_8k.md"},
 }
 
