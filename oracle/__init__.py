@@ -86,12 +86,51 @@ def lib():
         _lib.orc_attend_tokens.argtypes = [ctypes.c_int, ctypes.c_double, P, P, P, P, ctypes.c_int, P, P]
         _lib.orc_kl.argtypes = [D, P, P, P, P, ctypes.c_int, P, ctypes.c_double, P, i64, P, P, P, P]
         _lib.orc_decode.argtypes = [D, P, P, P, P, P, P, ctypes.c_int, P, P, P, P]
+        _lib.orc_e4m3_values.argtypes = [P, i64, P]
+        _lib.orc_e4m3_round_many.argtypes = [P, i64, P]
+        _lib.orc_quantize_e4m3_rows.argtypes = [P, i64, ctypes.c_int, P, P]
         _lib.orc_num_threads.restype = ctypes.c_int
     return _lib
 
 
 def num_threads() -> int:
     return lib().orc_num_threads()
+
+
+def e4m3_values(codes) -> np.ndarray:
+    """float64 values of e4m3 codes (uint8 bit patterns), from the format's definition."""
+    c = np.ascontiguousarray(np.asarray(codes, dtype=np.uint8))
+    out = np.empty(c.shape, dtype=np.float64)
+    lib().orc_e4m3_values(c.ctypes.data, c.size, out.ctypes.data)
+    return out
+
+
+def e4m3_round(y) -> np.ndarray:
+    """e4m3 codes of float32 values: nearest value, ties to even, saturated to +-448."""
+    f = np.ascontiguousarray(np.asarray(y, dtype=np.float32))
+    out = np.empty(f.shape, dtype=np.uint8)
+    lib().orc_e4m3_round_many(f.ctypes.data, f.size, out.ctypes.data)
+    return out
+
+
+def quantize_e4m3_rows(x):
+    """Row-wise e4m3 quantisation of a bf16 tensor [..., n]: (codes uint8 [..., n], scale float32
+    [...]) with scale = max|row| / 448 and codes = e4m3(x / scale), quotients in float32."""
+    t = torch.as_tensor(x).detach().to("cpu").contiguous()
+    if t.dtype != torch.bfloat16:
+        raise TypeError("quantize_e4m3_rows takes bfloat16")
+    n = t.shape[-1]
+    rows = t.numel() // n
+    codes = np.empty(tuple(t.shape), dtype=np.uint8)
+    scale = np.empty(tuple(t.shape[:-1]), dtype=np.float32)
+    lib().orc_quantize_e4m3_rows(_ptr(t.view(torch.int16)), rows, n, codes.ctypes.data, scale.ctypes.data)
+    return codes, scale
+
+
+def dequantize_e4m3_rows(codes, scale) -> torch.Tensor:
+    """float64 values scale[r] * e4m3(codes[r, c])."""
+    v = e4m3_values(codes) * np.asarray(scale, dtype=np.float64)[..., None]
+    return torch.from_numpy(v)
 
 
 def _inp(*ts):
@@ -228,3 +267,15 @@ def decode(dims: Dims, cache_len, q, q_idx, k_cache, v_cache, k_idx_cache):
     lib().orc_decode(ctypes.byref(dims.c()), _ptr(cl), _ptr(qt), _ptr(qit), _ptr(kc), _ptr(vc), _ptr(kic), ty,
                      blocks.ctypes.data, margin.ctypes.data, out.ctypes.data, lse.ctypes.data)
     return blocks, margin, out, lse
+
+
+def decode_fp8idx(dims: Dims, cache_len, q, q_idx, k_cache, v_cache, k_idx_codes, k_idx_scale):
+    """One decode step with FP8 index scoring: the K_idx cache given as e4m3 codes [B,N,d_idx] and
+    per-token scales [B,N]; Q_idx (bf16) rounded to e4m3 per (sequence, group) row by the same rule.
+    The step is ``decode`` on the dequantised index vectors scale * e4m3(code) (exact in float64),
+    so the index score is scale_idx * sq * sk * sum_c q8[c] k8[c]. Same returns as ``decode``."""
+    qc, qs = quantize_e4m3_rows(q_idx)
+    qd = dequantize_e4m3_rows(qc, qs)
+    kd = dequantize_e4m3_rows(k_idx_codes, k_idx_scale)
+    f64 = lambda t: torch.as_tensor(t).detach().to("cpu").to(torch.float64)
+    return decode(dims, cache_len, f64(q), qd, f64(k_cache), f64(v_cache), kd)

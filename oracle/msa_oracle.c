@@ -21,6 +21,11 @@
  *   - loss          L_KL = 1/(N H_kv) sum_i sum_r KL(stopgrad(P_i^{(r)}) || P_i^{idx,(r)})
  *       ("KL alignment in MSA", section 3)
  *   - logit grad    dKL/dz_j = P^idx_j - P_j ("KL alignment in MSA", section 3, key gradient)
+ *   - FP8 keys      selector keys kept in bf16 for training, quantised to FP8 for serving
+ *       ("4.1.1 supervision and joint training", section 2; "MSA Indexer vs DSA Lightning
+ *        Indexer", section 3.1: the indexer can run in FP8). Reading: e4m3 with one fp32 scale
+ *        per row, scale = max|x| / 448, codes rounded to nearest (ties to even), saturated.
+ *   - cutoff margin Delta_i = r_(k) - r_(k+1) ("4.1.1 supervision and joint training", eq (9))
  *
  * Readings of points the pages leave open (each is listed in the design notes):
  *   - local_mode 0 (the reading the GPU library implements): Top-k runs over the query's
@@ -37,7 +42,9 @@
  * two-position example), the deletion and partition-merge identities, dense causal attention when
  * k covers every block (against torch SDPA in float64), brute force of the selection, LSE_idx,
  * sparse attention and KL on tiny inputs, finite differences of the KL gradient, KL = 0 when the
- * student equals the teacher, decode = last prefill row. Which of the three local-block readings
+ * student equals the teacher, decode = last prefill row, the e4m3 code values against the format's
+ * table in torch, nearest-even rounding, and FP8 decode = bf16 decode on inputs that are already
+ * e4m3 values with power-of-two row scales. Which of the three local-block readings
  * the method uses is not fixed by any page: that choice is parity unpinned (the code of each
  * reading is pinned, the choice between them is not).
  *
@@ -427,6 +434,82 @@ int orc_decode(const orc_dims *D, const int32_t *cache_len, const void *q, const
         free(z);
     }
     return 0;
+}
+
+/* ---------------------------------------------------------------------------------------------
+ * e4m3: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits. Exponent field 0 holds the
+ * subnormals m * 2^-9; field e > 0 holds (1 + m/8) * 2^(e-7); code 0x7f (and 0xff) is NaN, so the
+ * largest finite value is 0x7e = 1.75 * 2^8 = 448. There are no infinities.
+ * -------------------------------------------------------------------------------------------- */
+double orc_e4m3_value(int code) {
+    const int e = (code >> 3) & 15, m = code & 7;
+    const double sign = (code & 0x80) ? -1.0 : 1.0;
+    if ((code & 0x7f) == 0x7f) return NAN;
+    if (e == 0) return sign * ldexp((double)m, -9);
+    return sign * ldexp(1.0 + m / 8.0, e - 7);
+}
+
+/* tab[c] = value of the non-negative finite code c, c = 0..126 */
+static void e4m3_table(double *tab) {
+    for (int c = 0; c < 0x7f; ++c) tab[c] = orc_e4m3_value(c);
+}
+
+/* The code of the e4m3 value nearest to y, ties to the even code (even mantissa), values beyond
+ * 448 in magnitude saturated to +-448. Brute force over the 127 finite magnitudes. */
+static int e4m3_round_tab(float y, const double *tab) {
+    const double a = fabs((double)y);
+    const int sign = signbit(y) ? 0x80 : 0;
+    if (a >= 448.0) return sign | 0x7e;
+    int best = 0;
+    double best_err = a;
+    for (int c = 1; c < 0x7f; ++c) {
+        const double err = fabs(a - tab[c]);
+        if (err < best_err || (err == best_err && (c & 1) == 0)) {
+            best = c;
+            best_err = err;
+        }
+    }
+    return sign | best;
+}
+
+int orc_e4m3_round(float y) {
+    double tab[0x7f];
+    e4m3_table(tab);
+    return e4m3_round_tab(y, tab);
+}
+
+void orc_e4m3_values(const uint8_t *codes, int64_t n, double *out) {
+    for (int64_t x = 0; x < n; ++x) out[x] = orc_e4m3_value(codes[x]);
+}
+
+void orc_e4m3_round_many(const float *y, int64_t n, uint8_t *out) {
+    double tab[0x7f];
+    e4m3_table(tab);
+#pragma omp parallel for schedule(static)
+    for (int64_t x = 0; x < n; ++x) out[x] = (uint8_t)e4m3_round_tab(y[x], tab);
+}
+
+/* Row quantisation: scale[r] = max_c |x[r,c]| / 448 and codes[r,c] = e4m3(x[r,c] / scale[r]),
+ * both quotients in float32 (the precision the serving path rounds in); scale 1 for a zero row.
+ * x is bf16 bits [rows, n]. */
+void orc_quantize_e4m3_rows(const uint16_t *x, int64_t rows, int n, uint8_t *codes, float *scale) {
+    double tab[0x7f];
+    e4m3_table(tab);
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        float amax = 0.0f;
+        for (int c = 0; c < n; ++c) {
+            const float v = (float)ld(x, ORC_BF16, (size_t)r * n + c);
+            if (fabsf(v) > amax) amax = fabsf(v);
+        }
+        const float sc = amax > 0.0f ? amax / 448.0f : 1.0f;
+        scale[r] = sc;
+        for (int c = 0; c < n; ++c) {
+            const float v = (float)ld(x, ORC_BF16, (size_t)r * n + c);
+            const float y = v / sc;
+            codes[(size_t)r * n + c] = (uint8_t)e4m3_round_tab(y, tab);
+        }
+    }
 }
 
 int orc_num_threads(void) {

@@ -355,3 +355,99 @@ def test_decode_equals_prefill_last_row():
     np.testing.assert_array_equal(db[0], blocks[L - 1])
     np.testing.assert_allclose(do[0], out[0], atol=1e-13)
     np.testing.assert_allclose(dl[0], lse[0], atol=1e-13)
+
+
+# ----------------------------------------------------------------------------- FP8 index keys
+def test_e4m3_code_values_match_the_format_table():
+    """Every e4m3 code decodes as the format defines it (1 sign, 4 exponent bits with bias 7,
+    3 mantissa bits, subnormals, 0x7f/0xff NaN): checked against torch's float8_e4m3fn table and
+    a few values written out."""
+    codes = np.arange(256, dtype=np.uint8)
+    v = oracle.e4m3_values(codes)
+    t = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert list(np.where(np.isnan(v))[0]) == [0x7F, 0xFF]
+    fin = ~np.isnan(v)
+    np.testing.assert_array_equal(v[fin], t[fin])
+    assert v[0x7E] == 448.0 and v[0xFE] == -448.0  # largest finite
+    assert v[0x38] == 1.0 and v[0x08] == 2.0 ** -6 and v[0x01] == 2.0 ** -9 and v[0x07] == 7 * 2.0 ** -9
+    assert v[0x3F] == 1.875
+
+
+def test_e4m3_rounding_nearest_even_and_saturation():
+    """Rounding to the nearest e4m3 value with ties to the even mantissa, as torch's float8 cast
+    does for |y| <= 448; beyond 448 the serving conversion saturates to +-448."""
+    rng = np.random.default_rng(7)
+    y = (rng.choice([-1.0, 1.0], 200000) * np.exp2(rng.uniform(-12, 9, 200000))).astype(np.float32)
+    y = y[np.abs(y) <= 448]
+    c = oracle.e4m3_round(y)
+    tc = torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(c, tc)
+    v = lambda x: float(oracle.e4m3_values(oracle.e4m3_round([x]))[0])
+    assert v(1.0 + 1 / 16) == 1.0          # tie between 1 and 1.125 -> even mantissa 0
+    assert v(1.0 + 3 / 16) == 1.25         # tie between 1.125 and 1.25 -> even mantissa 2
+    assert v(2.0 ** -10) == 0.0            # half the smallest subnormal -> 0
+    assert v(3 * 2.0 ** -10) == 2.0 ** -8  # tie between 1 and 2 subnormal quanta -> 2
+    assert v(-0.3) == -0.3125
+    assert v(460.0) == 448.0 and v(1e6) == 448.0 and v(-1e6) == -448.0
+
+
+def test_e4m3_row_quantisation_properties():
+    """Row scale max|x| / 448: each row's largest magnitude becomes exactly +-448, every value is
+    reproduced within half an e4m3 step (relative 2^-4 for normal codes), and a zero row keeps
+    scale 1 with zero codes."""
+    g = torch.Generator().manual_seed(11)
+    x = (torch.randn(64, 32, generator=g) * torch.exp2(torch.randint(-8, 8, (64, 1), generator=g).float()))
+    x[5] = 0.0
+    x = x.to(torch.bfloat16)
+    codes, scale = oracle.quantize_e4m3_rows(x)
+    xf = x.double().numpy()
+    amax = np.abs(xf).max(1)
+    np.testing.assert_array_equal(scale[amax > 0], (amax[amax > 0].astype(np.float32) / np.float32(448.0)))
+    assert scale[5] == 1.0 and not codes[5].any()
+    vals = oracle.e4m3_values(codes)
+    arg = np.abs(xf).argmax(1)
+    for r in range(64):
+        if amax[r] > 0:
+            assert abs(vals[r, arg[r]]) == 448.0
+    deq = oracle.dequantize_e4m3_rows(codes, scale).numpy()
+    y = np.abs(xf) / scale[:, None]
+    normal = y >= 2.0 ** -6
+    err = np.abs(deq - xf) / scale[:, None]
+    assert np.all(err[normal] <= y[normal] * 2.0 ** -4 * (1 + 1e-6))
+    assert np.all(err[~normal] <= 2.0 ** -10 * (1 + 1e-6))
+
+
+def test_decode_fp8_equals_bf16_decode_on_e4m3_grid():
+    """When every index vector is already an e4m3 value times a power of two and each row holds
+    +-448 times that power, quantisation is exact (scale 2^p, codes reproduce the values), so FP8
+    decode must equal the bf16 decode: same blocks, margins and outputs. The powers differ per row,
+    so a scale applied to the wrong row or a dropped scale fails."""
+    L, Bk, G, Hkv, di = 150, 16, 2, 2, 16
+    B = 2
+    dims = oracle.Dims(B=B, N=L, H_q=G * Hkv, H_kv=Hkv, d=16, d_idx=di, block_k=Bk, topk=3)
+    g = torch.Generator().manual_seed(31)
+    fin = oracle.e4m3_values(np.arange(0x7F, dtype=np.uint8))  # finite non-negative values
+
+    def grid_rows(*shape):
+        idx = torch.randint(0, 0x7F, shape, generator=g).numpy()
+        sign = np.where(torch.rand(shape, generator=g).numpy() < 0.5, -1.0, 1.0)
+        v = fin[idx] * sign
+        v[..., 0] = 448.0 * np.where(torch.rand(shape[:-1], generator=g).numpy() < 0.5, -1.0, 1.0)
+        p = torch.randint(-9, 1, shape[:-1] + (1,), generator=g).numpy()
+        return torch.from_numpy(v * np.exp2(p)).to(torch.bfloat16)
+
+    q_idx = grid_rows(B, Hkv, di)
+    k_idx = grid_rows(B, L, di)
+    assert torch.equal(q_idx.double().to(torch.bfloat16), q_idx)
+    mk = lambda *s: torch.randn(*s, generator=g).to(torch.bfloat16)
+    q, kc, vc = mk(B, G * Hkv, 16), mk(B, L, Hkv, 16), mk(B, L, Hkv, 16)
+    lens = [L, 97]
+    kcodes, kscale = oracle.quantize_e4m3_rows(k_idx)
+    assert np.all(np.log2(kscale) == np.round(np.log2(kscale)))
+    np.testing.assert_array_equal(oracle.dequantize_e4m3_rows(kcodes, kscale).numpy(), k_idx.double().numpy())
+    b8, m8, o8, l8 = oracle.decode_fp8idx(dims, lens, q, q_idx, kc, vc, kcodes, kscale)
+    b16, m16, o16, l16 = oracle.decode(dims, lens, q, q_idx, kc, vc, k_idx)
+    np.testing.assert_array_equal(b8, b16)
+    np.testing.assert_allclose(m8, m16, rtol=1e-14, atol=0)
+    np.testing.assert_allclose(o8, o16, atol=1e-13)
+    np.testing.assert_allclose(l8, l16, atol=1e-13)
