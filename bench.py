@@ -363,27 +363,10 @@ def bench_prefill(args, world, rank, msa, pk):
     return res
 
 
-def bench_decode(args, world, rank, msa, pk):
-    w = WORKLOADS["decode_16x256k"]
+def measure_decode(args, world, step, scan_kernel, scan_bytes, step_bytes, pk, msa):
+    """Eager and graph-replayed µs per decode step, and a profiled pass for the kernel split."""
     dev = torch.device("cuda", torch.cuda.current_device())
-    L = args.decode_len or w.N
-    x = decode_inputs(w, device=dev, seed=rank_seed(w, rank), L=L)
-    dims = msa.MsaDims(w.B, L, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
-    ws = msa.workspace(msa.MSA_OP_DECODE, dims, dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-
-    def step():
-        return msa.msa_sparse_attn_decode(dims, x["cache_len"], x["q"], x["q_idx"], x["k_cache"], x["v_cache"],
-                                          x["k_idx_cache"], ws=ws)
-
-    for _ in range(max(3, args.warmup)):
-        out, blocks = step()
-    torch.cuda.synchronize()
-    nscored = ((L - 1) // w.block_k) * w.block_k
-    scan_bytes = w.B * nscored * w.d_idx * 2
-    sel_blocks = int((blocks >= 0).sum().item())
-    kv_bytes = sel_blocks * w.block_k * w.d * 2 * 2
-    step_bytes = scan_bytes + kv_bytes + w.B * (w.H_q * w.d * 2 * 2 + w.H_kv * w.d_idx * 2)
     # (1) eager API calls, no profiler events in the stream
     barrier(world)
     t = timed_steps(step, args.decode_steps, flush)
@@ -415,20 +398,87 @@ def bench_decode(args, world, rank, msa, pk):
     msa.msa_profile_enable(False)
     prof = profile_avg(msa.msa_profile_read())
     # the batch may be cut into parts (one scan launch each): time per step = total / steps
-    scan_ms = prof["dec_scan"]["total_ms"] / args.decode_steps
-    res = {"workload": "decode_16x256k" if L == w.N else f"decode_16x{L}", "us_per_step": us, "us_per_token": us, "tokens_per_s": w.B * world / (us * 1e-6),
-           "us_per_step_graph": us_graph, "bytes_per_step": step_bytes,
+    scan_ms = prof[scan_kernel]["total_ms"] / args.decode_steps
+    res = {"us_per_step": us, "us_per_step_graph": us_graph, "bytes_per_step": step_bytes,
            "step_roofline": roofline_entry("hbm", step_bytes / (us * 1e-6) / 1e9, pk["hbm_gbs"], "GB/s"),
            "step_roofline_graph": roofline_entry("hbm", step_bytes / (us_graph * 1e-6) / 1e9, pk["hbm_gbs"], "GB/s")
            if us_graph == us_graph else None,
            "roofline": {**roofline_entry("hbm", scan_bytes / (scan_ms * 1e-3) / 1e9, pk["hbm_gbs"], "GB/s"),
-                        "kernel": "dec_scan", "bytes_per_step": scan_bytes,
-                        "launches_per_step": prof["dec_scan"]["launches"] // args.decode_steps},
+                        "kernel": scan_kernel, "bytes_per_step": scan_bytes,
+                        "launches_per_step": prof[scan_kernel]["launches"] // args.decode_steps},
            "kernels": {k: {"ms_per_step": round(v["total_ms"] / args.decode_steps, 4),
                            "launches_per_step": v["launches"] // args.decode_steps} for k, v in prof.items()}}
     if graph_note:
         res["graph_note"] = graph_note
-    del x, ws
+    return res
+
+
+def bench_decode(args, world, rank, msa, pk):
+    """The bf16 decode step, and the same step with FP8 (e4m3) index keys plus the report of the
+    rows whose selection differs between the two scorings (with their bf16 cutoff margins)."""
+    w = WORKLOADS["decode_16x256k"]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    L = args.decode_len or w.N
+    x = decode_inputs(w, device=dev, seed=rank_seed(w, rank), L=L)
+    dims = msa.MsaDims(w.B, L, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
+    ws = msa.workspace(msa.MSA_OP_DECODE, dims, dev)
+
+    def step():
+        return msa.msa_sparse_attn_decode(dims, x["cache_len"], x["q"], x["q_idx"], x["k_cache"], x["v_cache"],
+                                          x["k_idx_cache"], ws=ws)
+
+    for _ in range(max(3, args.warmup)):
+        out, blocks = step()
+    torch.cuda.synchronize()
+    nscored = ((L - 1) // w.block_k) * w.block_k
+    scan_bytes = w.B * nscored * w.d_idx * 2
+    sel_blocks = int((blocks >= 0).sum().item())
+    kv_bytes = sel_blocks * w.block_k * w.d * 2 * 2
+    small_bytes = w.B * (w.H_q * w.d * 2 * 2 + w.H_kv * w.d_idx * 2)
+    m = measure_decode(args, world, step, "dec_scan", scan_bytes, scan_bytes + kv_bytes + small_bytes, pk, msa)
+    res = {"workload": "decode_16x256k" if L == w.N else f"decode_16x{L}", "us_per_token": m["us_per_step"],
+           "tokens_per_s": w.B * world / (m["us_per_step"] * 1e-6), **m}
+
+    # FP8 index keys: the cache's K_idx quantised once (as a serving cache stores it), then the
+    # same step scoring from e4m3 codes + per-token scales
+    codes, kscale = msa.msa_quantize_e4m3_rows(x["k_idx_cache"])
+
+    def step8():
+        return msa.msa_sparse_attn_decode_fp8idx(dims, x["cache_len"], x["q"], x["q_idx"], x["k_cache"],
+                                                 x["v_cache"], codes, kscale, ws=ws)
+
+    for _ in range(max(3, args.warmup)):
+        out8, blocks8 = step8()
+    torch.cuda.synchronize()
+    scan8 = w.B * nscored * (w.d_idx + 4)
+    sel8 = int((blocks8 >= 0).sum().item())
+    m8 = measure_decode(args, world, step8, "dec_scan_e4m3", scan8,
+                        scan8 + sel8 * w.block_k * w.d * 2 * 2 + small_bytes, pk, msa)
+    # flip report: bf16 vs FP8 selection, bf16 margins of the rows that flip, planted-block recall
+    _, b16, mg16 = msa.msa_sparse_attn_decode(dims, x["cache_len"], x["q"], x["q_idx"], x["k_cache"],
+                                              x["v_cache"], x["k_idx_cache"], ws=ws, want_margin=True)
+    _, b8, mg8 = msa.msa_sparse_attn_decode_fp8idx(dims, x["cache_len"], x["q"], x["q_idx"], x["k_cache"],
+                                                   x["v_cache"], codes, kscale, ws=ws, want_margin=True)
+    torch.cuda.synchronize()
+    flipped = (b16 != b8).any(dim=-1)
+    planted = x["planted_blocks"]
+
+    def planted_recall(sel):
+        hit = (sel[:, :, :, None] == planted[:, None, None, :]).any(dim=2)  # [B, H_kv, n_planted]
+        return float(hit.float().mean().item())
+
+    fin16 = mg16[torch.isfinite(mg16)]
+    m8["flip_report"] = {
+        "rows": int(flipped.numel()), "rows_flipped": int(flipped.sum().item()),
+        "slots_changed": int(sum(len(set(b16[i, r].tolist()) ^ set(b8[i, r].tolist())) // 2
+                                 for i in range(w.B) for r in range(w.H_kv))),
+        "bf16_margin_median": float(fin16.median().item()) if fin16.numel() else None,
+        "bf16_margin_max_of_flipped": float(mg16[flipped].max().item()) if flipped.any() else None,
+        "fp8_margin_median": float(mg8[torch.isfinite(mg8)].median().item()) if torch.isfinite(mg8).any() else None,
+        "planted_recall_bf16": planted_recall(b16), "planted_recall_fp8": planted_recall(b8)}
+    m8["cache_bytes"] = {"k_idx_bf16": w.B * L * w.d_idx * 2, "k_idx_e4m3_codes_and_scales": w.B * L * (w.d_idx + 4)}
+    res["fp8_index"] = m8
+    del x, ws, codes, kscale
     torch.cuda.empty_cache()
     return res
 

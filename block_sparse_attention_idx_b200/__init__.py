@@ -69,7 +69,9 @@ def lib() -> ctypes.CDLL:
         L.msa_workspace_size.argtypes = [ctypes.c_int, D, ctypes.POINTER(ctypes.c_size_t)]
         L.msa_index_topk.argtypes = [D, P, P, P, P, P, S, P]
         L.msa_sparse_attn_fwd.argtypes = [D, P, P, P, P, P, P, P, S, P]
-        L.msa_sparse_attn_decode.argtypes = [D, P, P, P, P, P, P, P, P, P, S, P]
+        L.msa_sparse_attn_decode.argtypes = [D, P, P, P, P, P, P, P, P, P, P, S, P]
+        L.msa_sparse_attn_decode_fp8idx.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, S, P]
+        L.msa_quantize_e4m3_rows.argtypes = [P, ctypes.c_int64, ctypes.c_int, P, P, P]
         L.msa_kl_fwd_grad.argtypes = [D, P, P, P, P, P, P, P, ctypes.c_float, P, P, P, P, S, P]
         L.msa_sparse_attn_decode_noalloc.argtypes = [D, P, P, P, P, P, P, P, P, P]
         L.msa_sparse_attn_decode_noalloc.restype = ctypes.c_int
@@ -83,7 +85,8 @@ def lib() -> ctypes.CDLL:
         L.msa_status_string.restype = ctypes.c_char_p
         L.msa_version.restype = ctypes.c_char_p
         for fn in ("msa_workspace_size", "msa_index_topk", "msa_sparse_attn_fwd", "msa_sparse_attn_decode",
-                   "msa_kl_fwd_grad", "msa_get_device_status"):
+                   "msa_sparse_attn_decode_fp8idx", "msa_quantize_e4m3_rows", "msa_kl_fwd_grad",
+                   "msa_get_device_status"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -163,26 +166,67 @@ def msa_sparse_attn_fwd(dims: MsaDims, q, k, v, blocks, want_lse: bool = True, w
     return out, lse
 
 
-def msa_sparse_attn_decode(dims: MsaDims, cache_len, q, q_idx, k_cache, v_cache, k_idx_cache, want_blocks=True,
-                           ws=None, stream=None):
-    """One decode step. dims.N is the cache capacity. Returns out fp32 [B,H_q,d] and the selected
-    blocks int32 [B,H_kv,topk+1] (or None)."""
+def _decode_io(dims: MsaDims, cache_len, q, q_idx, k_cache, v_cache, want_blocks, want_margin):
     dev = q.device
     _need(cache_len, "cache_len", (dims.B,), torch.int32, dev)
     _need(q, "q", (dims.B, dims.H_q, dims.d), torch.bfloat16, dev)
     _need(q_idx, "q_idx", (dims.B, dims.H_kv, dims.d_idx), torch.bfloat16, dev)
     _need(k_cache, "k_cache", (dims.B, dims.N, dims.H_kv, dims.d), torch.bfloat16, dev)
     _need(v_cache, "v_cache", (dims.B, dims.N, dims.H_kv, dims.d), torch.bfloat16, dev)
-    _need(k_idx_cache, "k_idx_cache", (dims.B, dims.N, dims.d_idx), torch.bfloat16, dev)
     out = torch.empty(q.shape, dtype=torch.float32, device=dev)
     blocks = torch.empty(dims.B, dims.H_kv, dims.topk + 1, dtype=torch.int32, device=dev) if want_blocks else None
+    margin = torch.empty(dims.B, dims.H_kv, dtype=torch.float32, device=dev) if want_margin else None
+    return out, blocks, margin
+
+
+def msa_sparse_attn_decode(dims: MsaDims, cache_len, q, q_idx, k_cache, v_cache, k_idx_cache, want_blocks=True,
+                           ws=None, stream=None, want_margin=False):
+    """One decode step. dims.N is the cache capacity. Returns out fp32 [B,H_q,d] and the selected
+    blocks int32 [B,H_kv,topk+1] (or None); with want_margin, also the cutoff margins fp32 [B,H_kv]."""
+    out, blocks, margin = _decode_io(dims, cache_len, q, q_idx, k_cache, v_cache, want_blocks, want_margin)
+    _need(k_idx_cache, "k_idx_cache", (dims.B, dims.N, dims.d_idx), torch.bfloat16, q.device)
     if ws is None:
-        ws = workspace(MSA_OP_DECODE, dims, dev)
+        ws = workspace(MSA_OP_DECODE, dims, q.device)
     _check("msa_sparse_attn_decode",
            lib().msa_sparse_attn_decode(ctypes.byref(dims.c()), _p(cache_len), _p(q), _p(q_idx), _p(k_cache),
-                                        _p(v_cache), _p(k_idx_cache), _p(out), _p(blocks), _p(ws), ws.numel(),
-                                        _stream(stream)))
-    return out, blocks
+                                        _p(v_cache), _p(k_idx_cache), _p(out), _p(blocks), _p(margin), _p(ws),
+                                        ws.numel(), _stream(stream)))
+    return (out, blocks, margin) if want_margin else (out, blocks)
+
+
+def msa_quantize_e4m3_rows(x, codes=None, scale=None, stream=None):
+    """Row-wise e4m3 quantisation of a bf16 tensor [..., n]: codes uint8 [..., n] (e4m3 bit
+    patterns) and scales fp32 [...], scale = max|row| / 448."""
+    if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous bf16 CUDA tensor")
+    n = x.shape[-1]
+    rows = x.numel() // n if n else 0
+    if codes is None:
+        codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if scale is None:
+        scale = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    _need(codes, "codes", tuple(x.shape), torch.uint8, x.device)
+    _need(scale, "scale", tuple(x.shape[:-1]), torch.float32, x.device)
+    _check("msa_quantize_e4m3_rows",
+           lib().msa_quantize_e4m3_rows(_p(x), rows, n, _p(codes), _p(scale), _stream(stream)))
+    return codes, scale
+
+
+def msa_sparse_attn_decode_fp8idx(dims: MsaDims, cache_len, q, q_idx, k_cache, v_cache, k_idx_codes, k_idx_scale,
+                                  want_blocks=True, ws=None, stream=None, want_margin=False):
+    """Decode step with FP8 index scoring: the K_idx cache as e4m3 codes uint8 [B,N,d_idx] plus
+    per-token scales fp32 [B,N] (msa_quantize_e4m3_rows). Returns as msa_sparse_attn_decode."""
+    out, blocks, margin = _decode_io(dims, cache_len, q, q_idx, k_cache, v_cache, want_blocks, want_margin)
+    _need(k_idx_codes, "k_idx_codes", (dims.B, dims.N, dims.d_idx), torch.uint8, q.device)
+    _need(k_idx_scale, "k_idx_scale", (dims.B, dims.N), torch.float32, q.device)
+    if ws is None:
+        ws = workspace(MSA_OP_DECODE, dims, q.device)
+    _check("msa_sparse_attn_decode_fp8idx",
+           lib().msa_sparse_attn_decode_fp8idx(ctypes.byref(dims.c()), _p(cache_len), _p(q), _p(q_idx),
+                                               _p(k_cache), _p(v_cache), _p(k_idx_codes), _p(k_idx_scale),
+                                               _p(out), _p(blocks), _p(margin), _p(ws), ws.numel(),
+                                               _stream(stream)))
+    return (out, blocks, margin) if want_margin else (out, blocks)
 
 
 def msa_sparse_attn_decode_noalloc(dims: MsaDims, cache_len, q, q_idx, k_cache, v_cache, k_idx_cache, out=None,
@@ -256,5 +300,6 @@ def msa_get_device_status(ws: torch.Tensor, stream=None) -> int:
 
 
 __all__ = ["MsaDims", "MsaError", "msa_workspace_size", "msa_index_topk", "msa_sparse_attn_fwd",
-           "msa_sparse_attn_decode", "msa_sparse_attn_decode_noalloc", "msa_kl_fwd_grad", "msa_get_device_status", "msa_status_string",
+           "msa_sparse_attn_decode", "msa_sparse_attn_decode_noalloc", "msa_sparse_attn_decode_fp8idx",
+           "msa_quantize_e4m3_rows", "msa_kl_fwd_grad", "msa_get_device_status", "msa_status_string",
            "msa_version", "msa_profile_enable", "msa_profile_read", "workspace", "lib", "LIB_PATH"]

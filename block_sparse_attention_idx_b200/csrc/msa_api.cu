@@ -186,15 +186,18 @@ msa_status msa_sparse_attn_fwd(const msa_dims* d, const void* q, const void* k, 
     return cuda_status(e);
 }
 
-msa_status msa_sparse_attn_decode(const msa_dims* d, const int32_t* cache_len, const void* q, const void* q_idx,
-                                  const void* k_cache, const void* v_cache, const void* k_idx_cache, float* out,
-                                  int32_t* blocks_out, void* ws, size_t ws_bytes, msa_stream_t stream_) {
+// The decode step with a bf16 K_idx cache (k_idx_scale null) or an e4m3 one (codes + scales).
+static msa_status decode_step(const msa_dims* d, const int32_t* cache_len, const void* q, const void* q_idx,
+                              const void* k_cache, const void* v_cache, const void* k_idx, const float* k_idx_scale,
+                              float* out, int32_t* blocks_out, float* margin_out, void* ws, size_t ws_bytes,
+                              msa_stream_t stream_) {
     msa_status s = check_common(d);
     if (s != MSA_OK) return s;
     if ((d->N + d->block_k - 1) / d->block_k > 8192) return MSA_ERR_UNSUPPORTED;
-    if (!cache_len || !q || !q_idx || !k_cache || !v_cache || !k_idx_cache || !out || !aligned16(q) ||
-        !aligned16(q_idx) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_idx_cache) ||
-        !aligned16(out) || (blocks_out && !aligned16(blocks_out)))
+    if (!cache_len || !q || !q_idx || !k_cache || !v_cache || !k_idx || !out || !aligned16(q) ||
+        !aligned16(q_idx) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_idx) ||
+        !aligned16(out) || (blocks_out && !aligned16(blocks_out)) || (margin_out && !aligned16(margin_out)) ||
+        (k_idx_scale && !aligned16(k_idx_scale)))
         return MSA_ERR_INVALID_ARG;
     s = ws_check(ws, ws_bytes, ws_decode(d));
     if (s != MSA_OK) return s;
@@ -215,9 +218,39 @@ msa_status msa_sparse_attn_decode(const msa_dims* d, const int32_t* cache_len, c
     a.o_part = reinterpret_cast<float*>(cv.take((size_t)d->B * d->H_kv * K1 * G * d->d * 4));
     a.lse_part = reinterpret_cast<float*>(cv.take((size_t)d->B * d->H_kv * K1 * G * 4));
     a.blocks_out = blocks_out;
+    a.margin_out = margin_out;
+    a.k_idx_scale = k_idx_scale;
     a.status = status;
-    e = run_decode(a, q, q_idx, k_cache, v_cache, k_idx_cache, out, num_sms(), st);
+    e = run_decode(a, q, q_idx, k_cache, v_cache, k_idx, out, num_sms(), st);
     return cuda_status(e);
+}
+
+msa_status msa_sparse_attn_decode(const msa_dims* d, const int32_t* cache_len, const void* q, const void* q_idx,
+                                  const void* k_cache, const void* v_cache, const void* k_idx_cache, float* out,
+                                  int32_t* blocks_out, float* margin_out, void* ws, size_t ws_bytes,
+                                  msa_stream_t stream) {
+    return decode_step(d, cache_len, q, q_idx, k_cache, v_cache, k_idx_cache, nullptr, out, blocks_out, margin_out,
+                       ws, ws_bytes, stream);
+}
+
+msa_status msa_sparse_attn_decode_fp8idx(const msa_dims* d, const int32_t* cache_len, const void* q,
+                                         const void* q_idx, const void* k_cache, const void* v_cache,
+                                         const uint8_t* k_idx_codes, const float* k_idx_scale, float* out,
+                                         int32_t* blocks_out, float* margin_out, void* ws, size_t ws_bytes,
+                                         msa_stream_t stream) {
+    if (!k_idx_scale) return MSA_ERR_INVALID_ARG;
+    return decode_step(d, cache_len, q, q_idx, k_cache, v_cache, k_idx_codes, k_idx_scale, out, blocks_out,
+                       margin_out, ws, ws_bytes, stream);
+}
+
+msa_status msa_quantize_e4m3_rows(const void* x, int64_t rows, int n, uint8_t* codes, float* scale,
+                                  msa_stream_t stream) {
+    if (rows < 0 || (rows > 0 && (!x || !codes || !scale || !aligned16(x) || !aligned16(codes) || !aligned16(scale))))
+        return MSA_ERR_INVALID_ARG;
+    if (n != 16 && n != 32 && n != 64 && n != 128 && n != 256) return MSA_ERR_UNSUPPORTED;
+    if (rows > ((int64_t)1 << 40) / n) return MSA_ERR_UNSUPPORTED;
+    return cuda_status(run_quantize_e4m3_rows(x, rows, n, codes, scale, num_sms(),
+                                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
 msa_status msa_kl_fwd_grad(const msa_dims* d, const void* q, const void* k, const void* q_idx, const void* k_idx,

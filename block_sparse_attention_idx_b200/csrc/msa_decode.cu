@@ -9,6 +9,11 @@
 //   k_dec_topk     per (sequence, group): Top-k over the complete past blocks + local block
 //   k_dec_attn     split-KV over (sequence, group, selected slot): one block of K/V for the G heads
 //   k_dec_combine  per (sequence, head): log-sum-exp merge of the slot partials
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
+#include <algorithm>
+
 #include "msa_common.cuh"
 #include "msa_internal.h"
 
@@ -40,6 +45,59 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 // group columns x 16 dims per instruction, A fragments by ldmatrix from the swizzled tile, the
 // groups' Q_idx as B fragments held in registers); each block's maxima come straight from the
 // accumulators. The kernel is HBM-bound: it reads every K_idx byte once.
+// The scan's work list: the complete past blocks of all sequences in (sequence, block) order, T
+// items in all. CTA c takes the contiguous range [c*T/grid, (c+1)*T/grid): a CTA streams one
+// contiguous stretch of the cache and meets at most a few sequences, so it reloads a sequence's
+// length and its Q_idx rarely. A cursor walks the range.
+struct ScanCursor {
+    int b, blk, nbv;  // current item: block blk of sequence b, which has nbv complete past blocks
+};
+__device__ __forceinline__ int complete_blocks(const DecodeArgs& a, int b, int BK) {
+    return max(a.cache_len[b] - 1, 0) / BK;
+}
+// Called by all lanes of a warp: sets c to the CTA's first item, returns its number of items.
+__device__ int scan_range(const DecodeArgs& a, int BK, ScanCursor& c) {
+    const int lane = threadIdx.x & 31;
+    long long T = 0;
+    for (int b0 = 0; b0 < a.B; b0 += 32) {
+        int v = b0 + lane < a.B ? complete_blocks(a, b0 + lane, BK) : 0;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        T += v;
+    }
+    const long long lo = T * blockIdx.x / gridDim.x, hi = T * (blockIdx.x + 1) / gridDim.x;
+    long long cum = 0;  // items before sequence b0
+    for (int b0 = 0; b0 < a.B && lo < hi; b0 += 32) {
+        const int v = b0 + lane < a.B ? complete_blocks(a, b0 + lane, BK) : 0;
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        const unsigned hit = __ballot_sync(0xffffffffu, cum + incl > lo);
+        if (hit) {
+            const int l = __ffs(hit) - 1;
+            c.b = b0 + l;
+            c.nbv = __shfl_sync(0xffffffffu, v, l);
+            c.blk = (int)(lo - (cum + __shfl_sync(0xffffffffu, incl, l) - c.nbv));
+            return (int)(hi - lo);
+        }
+        cum += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    c.b = a.B;
+    c.blk = c.nbv = 0;
+    return 0;
+}
+// Moves c forward by k items (sequences without complete past blocks are skipped).
+__device__ __forceinline__ void scan_advance(const DecodeArgs& a, int BK, ScanCursor& c, int k) {
+    c.blk += k;
+    while (c.b < a.B && c.blk >= c.nbv) {
+        c.blk -= c.nbv;
+        if (++c.b < a.B) c.nbv = complete_blocks(a, c.b, BK);
+    }
+}
+
 constexpr int kScanStages = 8;
 constexpr int kScanWarps = 4;
 
@@ -57,7 +115,6 @@ __global__ void __launch_bounds__((kScanWarps + 1) * 32, 1)
     Sm& s = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(scan_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nb = (a.L + BK - 1) / BK;
-    const int total = a.B * nb;
     if (threadIdx.x == 0) {
         for (int x = 0; x < kScanStages; ++x) {
             mbar_init(&s.full[x], 1);
@@ -66,23 +123,16 @@ __global__ void __launch_bounds__((kScanWarps + 1) * 32, 1)
         fence_mbar_init();
     }
     __syncthreads();
-    // the n-th block this CTA processes: global ids blockIdx.x + gridDim.x * j that name a complete
-    // past block of their sequence; producer and consumers walk the same list
-    auto next_valid = [&](int gb) -> int {
-        for (; gb < total; gb += gridDim.x) {
-            const int b = gb / nb, blk = gb % nb;
-            if (blk < (a.cache_len[b] - 1) / BK) return gb;
-        }
-        return total;
-    };
+    ScanCursor cur;
+    const int count = scan_range(a, BK, cur);
     if (warp == kScanWarps) {
         if (lane == 0) {
             int n = 0;
-            for (int gb = next_valid(blockIdx.x); gb < total; gb = next_valid(gb + gridDim.x), ++n) {
+            for (; n < count; ++n, scan_advance(a, BK, cur, 1)) {
                 const int st = n % kScanStages;
                 if (n >= kScanStages && !mbar_wait(&s.empty[st], ((n / kScanStages) - 1) & 1, a.status, 0x901)) break;
                 mbar_arrive_expect_tx(&s.full[st], (uint32_t)(BK * DI * 2));
-                tma_load_3d(s.tile[st], &tm_kidx, &s.full[st], 0, (gb % nb) * BK, gb / nb);
+                tma_load_3d(s.tile[st], &tm_kidx, &s.full[st], 0, cur.blk * BK, cur.b);
             }
             // no copy of ours may still be landing when the CTA leaves
             for (int m = max(0, n - kScanStages); m < n; ++m)
@@ -95,10 +145,9 @@ __global__ void __launch_bounds__((kScanWarps + 1) * 32, 1)
     const int g = lane >> 2, t4 = lane & 3;
     int cur_b = -1;
     uint32_t qb[DI / 16][2];
-    int n = 0;
-    for (int gb = next_valid(blockIdx.x); gb < total; gb = next_valid(gb + gridDim.x), ++n) {
-        if (n % kScanWarps != warp) continue;
-        const int b = gb / nb, blk = gb % nb;
+    scan_advance(a, BK, cur, warp);
+    for (int n = warp; n < count; n += kScanWarps, scan_advance(a, BK, cur, kScanWarps)) {
+        const int b = cur.b, blk = cur.blk;
         if (b != cur_b) {
             cur_b = b;
             const uint32_t* qrow = reinterpret_cast<const uint32_t*>(q_idx + ((size_t)b * a.H_kv + min(g, a.H_kv - 1)) * DI);
@@ -138,6 +187,230 @@ __global__ void __launch_bounds__((kScanWarps + 1) * 32, 1)
         if (lane < 4) {
             if (2 * t4 < a.H_kv) a.bmax[((size_t)b * a.H_kv + 2 * t4) * nb + blk] = m0;
             if (2 * t4 + 1 < a.H_kv) a.bmax[((size_t)b * a.H_kv + 2 * t4 + 1) * nb + blk] = m1;
+        }
+    }
+    pdl_trigger();
+}
+
+// ------------------------------------------------------------------------------ FP8 index keys
+// e4m3 helpers. Conversions go through cuda_fp8.h: float -> e4m3 rounds to nearest even and, with
+// __NV_SATFINITE, clamps to +-448; e4m3 -> f16 is exact (every e4m3 value is an f16 value).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+__device__ __forceinline__ uint32_t e4m3_code(float x, float scale) {
+    return (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(x, scale), __NV_SATFINITE, __NV_E4M3);
+}
+// Row scale max|x| / 448 (1 for an all-zero row), correctly rounded in fp32.
+__device__ __forceinline__ float e4m3_row_scale(float amax) { return amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f; }
+
+__device__ __forceinline__ void mma_16816_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+// Arrives on `bar` once this thread's earlier cp.async copies have landed (counted in its init).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Row-wise e4m3 quantisation (the serving copy of the index keys: keys kept in bf16 for training
+// are quantised to FP8 for inference). Each row gets the scale max|x| / 448 and codes
+// e4m3(x / scale). Threads own 8 consecutive elements; the NL = n / 8 threads of a row are
+// consecutive lanes of one warp and combine their maxima by shuffles. HBM-bound.
+template <int NL>
+__global__ void __launch_bounds__(256) k_quant_e4m3_rows(const __nv_bfloat16* __restrict__ x, int64_t rows,
+                                                         uint8_t* __restrict__ codes, float* __restrict__ scale) {
+    const int64_t per_pass = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < rows * NL; t += per_pass) {
+        const int64_t row = t / NL;
+        const uint4 raw = *reinterpret_cast<const uint4*>(x + t * 8);
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(h[e]);
+            v[2 * e] = f.x;
+            v[2 * e + 1] = f.y;
+        }
+        float amax = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
+        // the NL lanes of a row are aligned within the warp (NL divides 32 and every pass moves by
+        // whole rows), so they are active together; the last pass may leave other rows' lanes idle
+        const int lane = threadIdx.x & 31;
+        const uint32_t row_mask = (NL == 32 ? 0xffffffffu : ((1u << NL) - 1u)) << (lane & ~(NL - 1));
+#pragma unroll
+        for (int o = 1; o < NL; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(row_mask, amax, o));
+        const float sc = e4m3_row_scale(amax);
+        uint32_t w[2] = {0u, 0u};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e >> 2] |= e4m3_code(v[e], sc) << (8 * (e & 3));
+        *reinterpret_cast<uint2*>(codes + t * 8) = make_uint2(w[0], w[1]);
+        if (t % NL == 0) scale[row] = sc;
+    }
+}
+
+// FP8 index scan: the pass of k_dec_scan over every complete past block, reading K_idx as e4m3
+// codes (DI bytes per token, half the bf16 bytes) plus one fp32 scale per token. Q_idx is rounded
+// to e4m3 here with the row scale of k_quant_e4m3_rows, per (sequence, group). The score of token
+// j for group r is scale_q[r] * scale_k[j] * (q8[r] . k8[j]).
+// Each 16-byte chunk of a token's codes (16 dims) is one k=16 step of f16 mma.sync: e4m3 values
+// are exact in f16, so every product is exact and only the fp32 accumulation rounds, as in the
+// bf16 scan. ldmatrix gives each lane 4 consecutive dims (4*t4 .. 4*t4+3) of a chunk for its
+// rows; they are widened into the A fragment's k slots (2*t4, 2*t4+1) and (8+2*t4, 9+2*t4), and
+// Q's B fragment places the same dims in the same slots (a dot product only needs A and B to agree
+// on which dim each k slot holds). The producer (one thread) streams the code tiles by TMA; each
+// consumer warp loads the token scales of its next block itself (plain coalesced loads, one block
+// ahead) and parks them in its own shared-memory row while it computes.
+// Eight consumer warps and a 16-stage ring (128 KB of code tiles for 128-token blocks of 64 dims):
+// at this tile size a CTA must keep more tiles in flight than the bf16 scan to reach the same HBM
+// rate, and its per-tile compute (widening plus 32 MMAs) needs more warps to keep up.
+constexpr int kScan8Warps = 8;
+constexpr int kScan8Stages = 16;
+
+template <int DI, int BK>
+struct ScanSmem8 {
+    alignas(1024) uint8_t tile[kScan8Stages][BK * DI];
+    float scale[kScan8Warps][BK];
+    uint64_t full[kScan8Stages], empty[kScan8Stages];
+};
+
+template <int DI, int BK>
+__global__ void __launch_bounds__((kScan8Warps + 1) * 32, 1)
+    k_dec_scan_e4m3(const __grid_constant__ CUtensorMap tm_codes, DecodeArgs a,
+                    const __nv_bfloat16* __restrict__ q_idx) {
+    static_assert(DI % 32 == 0 && BK % 32 == 0, "chunk pairs and 32-row scale loads");
+    // item n uses stage n % stages and warp n % warps: the next item on a stage then belongs to the
+    // same warp, so no warp can wait on a stage's full barrier a phase early
+    static_assert(kScan8Stages % kScan8Warps == 0, "stages must be a multiple of the consumer warps");
+    using Sm = ScanSmem8<DI, BK>;
+    extern __shared__ uint8_t scan8_raw[];
+    Sm& s = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(scan8_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nb = (a.L + BK - 1) / BK;
+    if (threadIdx.x == 0) {
+        for (int x = 0; x < kScan8Stages; ++x) {
+            mbar_init(&s.full[x], 1);
+            mbar_init(&s.empty[x], 1);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    ScanCursor cur;
+    const int count = scan_range(a, BK, cur);
+    if (warp == kScan8Warps) {
+        if (lane == 0) {
+            int n = 0;
+            for (; n < count; ++n, scan_advance(a, BK, cur, 1)) {
+                const int st = n % kScan8Stages;
+                if (n >= kScan8Stages && !mbar_wait(&s.empty[st], ((n / kScan8Stages) - 1) & 1, a.status, 0x911))
+                    break;
+                mbar_arrive_expect_tx(&s.full[st], (uint32_t)(BK * DI));
+                tma_load_3d(s.tile[st], &tm_codes, &s.full[st], 0, cur.blk * BK, cur.b);
+            }
+            // no copy of ours may still be landing when the CTA leaves
+            for (int m = max(0, n - kScan8Stages); m < n; ++m)
+                mbar_wait(&s.full[m % kScan8Stages], (m / kScan8Stages) & 1, a.status, 0x912);
+        }
+        pdl_trigger();
+        return;
+    }
+    const int g = lane >> 2, t4 = lane & 3;
+    int cur_b = -1;
+    uint32_t qb[DI / 16][2];
+    float sq0 = 0.f, sq1 = 0.f;  // Q scales of groups 2*t4 and 2*t4+1
+    float scn[BK / 32];          // token scales of this warp's next block, rows lane + 32*x
+    auto load_scales = [&](const ScanCursor& c) {
+        const float* src = a.k_idx_scale + (size_t)c.b * a.L + (size_t)c.blk * BK;
+#pragma unroll
+        for (int x = 0; x < BK / 32; ++x) scn[x] = __ldg(src + lane + 32 * x);
+    };
+    scan_advance(a, BK, cur, warp);
+    if (warp < count) load_scales(cur);
+    for (int n = warp; n < count; n += kScan8Warps) {
+        const int b = cur.b, blk = cur.blk;
+        // park this block's scales, then start loading the next block's
+#pragma unroll
+        for (int x = 0; x < BK / 32; ++x) s.scale[warp][lane + 32 * x] = scn[x];
+        __syncwarp();
+        scan_advance(a, BK, cur, kScan8Warps);
+        if (n + kScan8Warps < count) load_scales(cur);
+        if (b != cur_b) {
+            // Q_idx row of group g (zero for g >= H_kv): this lane's dims 16c + 4*t4 + {0..3}
+            cur_b = b;
+            const bool gv = g < a.H_kv;
+            const __nv_bfloat16* qrow = q_idx + ((size_t)b * a.H_kv + min(g, a.H_kv - 1)) * DI;
+            float qv[DI / 16][4];
+            float amax = 0.f;
+#pragma unroll
+            for (int c = 0; c < DI / 16; ++c) {
+                const uint2 raw = *reinterpret_cast<const uint2*>(qrow + 16 * c + 4 * t4);
+                const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+                const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+                qv[c][0] = lo.x;
+                qv[c][1] = lo.y;
+                qv[c][2] = hi.x;
+                qv[c][3] = hi.y;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(qv[c][e]));
+            }
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+            const float sq = e4m3_row_scale(amax);
+#pragma unroll
+            for (int c = 0; c < DI / 16; ++c) {
+                const uint32_t c01 = e4m3_code(qv[c][0], sq) | (e4m3_code(qv[c][1], sq) << 8);
+                const uint32_t c23 = e4m3_code(qv[c][2], sq) | (e4m3_code(qv[c][3], sq) << 8);
+                qb[c][0] = gv ? e4m3x2_to_f16x2(c01) : 0u;
+                qb[c][1] = gv ? e4m3x2_to_f16x2(c23) : 0u;
+            }
+            sq0 = __shfl_sync(0xffffffffu, sq, 8 * t4);      // lane of (group 2*t4, t4 = 0)
+            sq1 = __shfl_sync(0xffffffffu, sq, 8 * t4 + 4);  // lane of (group 2*t4+1, t4 = 0)
+        }
+        const int st = n % kScan8Stages;
+        if (!__all_sync(0xffffffffu, mbar_wait(&s.full[st], (n / kScan8Stages) & 1, a.status, 0x913))) break;
+        const uint32_t base = smem_u32(s.tile[st]);
+        float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+        for (int mt = 0; mt < BK / 16; ++mt) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            const int row = mt * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+#pragma unroll
+            for (int cc = 0; cc < DI / 32; ++cc) {
+                uint32_t r[4];
+                const uint32_t addr = base + swz(row, (2 * cc + (lane >> 4)) * 16, DI);
+                asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                             : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                             : "r"(addr));
+                // r[0] / r[1]: rows g / g+8 of chunk 2*cc; r[2] / r[3]: the same rows of chunk 2*cc+1
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t a4[4] = {e4m3x2_to_f16x2(r[2 * h]), e4m3x2_to_f16x2(r[2 * h + 1]),
+                                            e4m3x2_to_f16x2(r[2 * h] >> 16), e4m3x2_to_f16x2(r[2 * h + 1] >> 16)};
+                    mma_16816_f16(acc, a4, qb[2 * cc + h][0], qb[2 * cc + h][1]);
+                }
+            }
+            const float sk0 = s.scale[warp][mt * 16 + g], sk1 = s.scale[warp][mt * 16 + g + 8];
+            m0 = fmaxf(m0, fmaxf(acc[0] * sk0, acc[2] * sk1));
+            m1 = fmaxf(m1, fmaxf(acc[1] * sk0, acc[3] * sk1));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.empty[st]);
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+            m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
+            m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+        }
+        if (lane < 4) {
+            if (2 * t4 < a.H_kv) a.bmax[((size_t)b * a.H_kv + 2 * t4) * nb + blk] = m0 * sq0;
+            if (2 * t4 + 1 < a.H_kv) a.bmax[((size_t)b * a.H_kv + 2 * t4 + 1) * nb + blk] = m1 * sq1;
         }
     }
     pdl_trigger();
@@ -262,6 +535,38 @@ __global__ void __launch_bounds__(256) k_dec_topk(DecodeArgs a) {
         }
     }
     __syncthreads();
+    if (a.margin_out) {
+        // cutoff margin r_(k) - r_(k+1) of the ranking (+inf when every candidate is taken): the
+        // k-th key is the smallest chosen key, the (k+1)-th the largest key below it
+        __shared__ unsigned long long s_kth, s_next[8];
+        float* mo = a.margin_out + (size_t)b * a.H_kv + r;
+        if (bi > a.topk) {
+            if (tid == 0) {
+                unsigned long long m = ~0ull;
+                for (int x = 0; x < take; ++x) m = min(m, s_key[chosen[x]]);
+                s_kth = m;
+            }
+            __syncthreads();
+            const unsigned long long kth = s_kth;
+            unsigned long long nx = 0ull;
+            for (int c = tid; c < bi; c += blockDim.x) {
+                const unsigned long long k = s_key[c];
+                if (k < kth) nx = max(nx, k);
+            }
+#pragma unroll
+            for (int o = 16; o; o >>= 1) nx = max(nx, (unsigned long long)__shfl_xor_sync(0xffffffffu, nx, o));
+            if (lane == 0) s_next[warp] = nx;
+            __syncthreads();
+            if (tid == 0) {
+                for (int w = 1; w < 8; ++w) nx = max(nx, s_next[w]);
+                const int id_k = (int)(0xffffffffu - (uint32_t)(kth & 0xffffffffu));
+                const int id_k1 = (int)(0xffffffffu - (uint32_t)(nx & 0xffffffffu));
+                *mo = (vals[id_k] - vals[id_k1]) * a.scale_idx;
+            }
+        } else if (tid == 0) {
+            *mo = INFINITY;
+        }
+    }
     pdl_trigger();
     if (warp != 0) return;
     // the chosen ids plus the local block, ascending: each lane places its id by its rank
@@ -522,6 +827,24 @@ __global__ void k_dec_combine(DecodeArgs a, float* __restrict__ out) {
 
 }  // namespace
 
+cudaError_t run_quantize_e4m3_rows(const void* x, int64_t rows, int n, uint8_t* codes, float* scale, int num_sms,
+                                   cudaStream_t st) {
+    if (rows <= 0) return cudaSuccess;
+    ProfScope ps("quant_e4m3_rows", st);
+    const auto* xb = static_cast<const __nv_bfloat16*>(x);
+    const int64_t threads = rows * (n / 8);
+    const int grid = (int)std::min<int64_t>((threads + 255) / 256, (int64_t)num_sms * 8);
+    switch (n) {
+        case 16: k_quant_e4m3_rows<2><<<grid, 256, 0, st>>>(xb, rows, codes, scale); break;
+        case 32: k_quant_e4m3_rows<4><<<grid, 256, 0, st>>>(xb, rows, codes, scale); break;
+        case 64: k_quant_e4m3_rows<8><<<grid, 256, 0, st>>>(xb, rows, codes, scale); break;
+        case 128: k_quant_e4m3_rows<16><<<grid, 256, 0, st>>>(xb, rows, codes, scale); break;
+        case 256: k_quant_e4m3_rows<32><<<grid, 256, 0, st>>>(xb, rows, codes, scale); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
 size_t decode_ws_bytes(int B, int L, int H_q, int H_kv, int d, int block_k, int topk) {
     const size_t nb = (size_t)(L + block_k - 1) / block_k;
     const size_t G = (size_t)H_q / H_kv, K1 = (size_t)topk + 1;
@@ -533,7 +856,30 @@ size_t decode_ws_bytes(int B, int L, int H_q, int H_kv, int d, int block_k, int 
 cudaError_t run_decode(const DecodeArgs& a, const void* q, const void* q_idx, const void* k_cache,
                        const void* v_cache, const void* k_idx_cache, void* out, int num_sms, cudaStream_t st) {
     const auto* qi = static_cast<const __nv_bfloat16*>(q_idx);
-    {
+    if (a.k_idx_scale) {
+        ProfScope ps("dec_scan_e4m3", st);
+        CUtensorMap tm;
+        if (!make_tmap_3d_u8(&tm, k_idx_cache, (uint64_t)a.d_idx, (uint64_t)a.L, (uint64_t)a.B, (uint64_t)a.d_idx,
+                             (uint64_t)a.L * a.d_idx, (uint32_t)a.d_idx, (uint32_t)a.block_k, a.d_idx))
+            return cudaErrorInvalidValue;
+        auto launch = [&](auto kern, size_t bytes) -> cudaError_t {
+            const size_t smem = bytes + 1024;
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            kern<<<num_sms, (kScan8Warps + 1) * 32, smem, st>>>(tm, a, qi);
+            return cudaGetLastError();
+        };
+        cudaError_t e;
+        if (a.d_idx == 64)
+            e = a.block_k == 128 ? launch(k_dec_scan_e4m3<64, 128>, sizeof(ScanSmem8<64, 128>))
+                : a.block_k == 64 ? launch(k_dec_scan_e4m3<64, 64>, sizeof(ScanSmem8<64, 64>))
+                                  : launch(k_dec_scan_e4m3<64, 32>, sizeof(ScanSmem8<64, 32>));
+        else
+            e = a.block_k == 128 ? launch(k_dec_scan_e4m3<32, 128>, sizeof(ScanSmem8<32, 128>))
+                : a.block_k == 64 ? launch(k_dec_scan_e4m3<32, 64>, sizeof(ScanSmem8<32, 64>))
+                                  : launch(k_dec_scan_e4m3<32, 32>, sizeof(ScanSmem8<32, 32>));
+        if (e != cudaSuccess) return e;
+    } else {
         ProfScope ps("dec_scan", st);
         CUtensorMap tm;
         if (!make_tmap_3d(&tm, k_idx_cache, (uint64_t)a.d_idx, (uint64_t)a.L, (uint64_t)a.B, (uint64_t)a.d_idx * 2,

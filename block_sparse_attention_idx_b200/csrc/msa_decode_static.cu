@@ -55,6 +55,6 @@ extern "C" msa_status msa_sparse_attn_decode_noalloc(const msa_dims* dims, const
     void* scratch = nullptr;
     s = scratch_address(&scratch);
     if (s != MSA_OK) return s;
-    return msa_sparse_attn_decode(dims, cache_len, q, q_idx, k_cache, v_cache, k_idx_cache, out, blocks_out, scratch,
+    return msa_sparse_attn_decode(dims, cache_len, q, q_idx, k_cache, v_cache, k_idx_cache, out, blocks_out, nullptr, scratch,
                                   (size_t)MSA_DECODE_STATIC_SCRATCH_BYTES, stream);
 }

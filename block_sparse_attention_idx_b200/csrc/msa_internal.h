@@ -31,6 +31,9 @@ bool make_tmap_4d(CUtensorMap* m, const void* base, const uint64_t dims[4], cons
                   const uint32_t box[4], int swizzle_bytes);
 // Query rows [B, N, H_q, d] as 5-D boxes of one query's G heads (G % 8 == 0, H_q % 8 == 0, d % 64 == 0)
 // laid out in 8-row x 64-column 128B-swizzled atoms.
+// Byte tensor [d2][d1][d0] (8-bit elements, e.g. e4m3), box {box0, box1, 1}.
+bool make_tmap_3d_u8(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1,
+                     uint64_t stride2, uint32_t box0, uint32_t box1, int swizzle_bytes);
 bool make_tmap_qrows(CUtensorMap* m, const void* q, int B, int N, int H_q, int d, int G);
 
 // ---------------------------------------------------------------- index Top-k (msa_index.cu)
@@ -121,9 +124,15 @@ struct DecodeArgs {
     float* o_part;     // [B, H_kv, topk+1, G, d]
     float* lse_part;   // [B, H_kv, topk+1, G]
     int32_t* blocks_out;
+    float* margin_out;         // [B, H_kv] cutoff margins, or null
+    const float* k_idx_scale;  // [B, L] per-token scales when the K_idx cache holds e4m3 codes, else null
     DevStatus* status;
 };
 size_t decode_ws_bytes(int B, int L, int H_q, int H_kv, int d, int block_k, int topk);
+// Row-wise e4m3 quantisation of a bf16 [rows, n] array (n in {16, 32, 64, 128, 256}).
+cudaError_t run_quantize_e4m3_rows(const void* x, int64_t rows, int n, uint8_t* codes, float* scale, int num_sms,
+                                   cudaStream_t st);
+// k_idx_cache is bf16 [B, L, d_idx], or e4m3 codes [B, L, d_idx] when a.k_idx_scale is set.
 cudaError_t run_decode(const DecodeArgs& a, const void* q, const void* q_idx, const void* k_cache, const void* v_cache,
                        const void* k_idx_cache, void* out, int num_sms, cudaStream_t st);
 

@@ -28,11 +28,12 @@ static CUtensorMapSwizzle swizzle_of(int bytes) {
 }
 
 static bool encode(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
-                   const uint32_t* box, int swizzle_bytes) {
+                   const uint32_t* box, int swizzle_bytes,
+                   CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base),
+    CUresult r = fn(m, dtype, rank, const_cast<void*>(base),
                     reinterpret_cast<const cuuint64_t*>(dims), reinterpret_cast<const cuuint64_t*>(strides),
                     reinterpret_cast<const cuuint32_t*>(box), estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     swizzle_of(swizzle_bytes), CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -58,6 +59,14 @@ bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, ui
 bool make_tmap_4d(CUtensorMap* m, const void* base, const uint64_t dims[4], const uint64_t strides[3],
                   const uint32_t box[4], int swizzle_bytes) {
     return encode(m, base, 4, dims, strides, box, swizzle_bytes);
+}
+
+bool make_tmap_3d_u8(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1,
+                     uint64_t stride2, uint32_t box0, uint32_t box1, int swizzle_bytes) {
+    const uint64_t dims[3] = {d0, d1, d2};
+    const uint64_t strides[2] = {stride1, stride2};
+    const uint32_t box[3] = {box0, box1, 1};
+    return encode(m, base, 3, dims, strides, box, swizzle_bytes, CU_TENSOR_MAP_DATA_TYPE_UINT8);
 }
 
 bool make_tmap_qrows(CUtensorMap* m, const void* q, int B, int N, int H_q, int d, int G) {

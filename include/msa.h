@@ -6,7 +6,8 @@
  *   S_t = R_theta(q_t, K_{:t}),   o_t = A_phi(q_t, K_{S_t}, V_{S_t})
  * ("2.4 · 训练原生稀疏", eq (3)). msa_index_topk is R_theta for MSA, msa_sparse_attn_fwd is A_phi,
  * msa_kl_fwd_grad is the KL alignment of the index branch to the main branch, and
- * msa_sparse_attn_decode runs R_theta then A_phi for one new token per sequence.
+ * msa_sparse_attn_decode runs R_theta then A_phi for one new token per sequence, and
+ * msa_sparse_attn_decode_fp8idx does the same from an e4m3 copy of the index keys.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -123,11 +124,52 @@ MSA_API msa_status msa_sparse_attn_fwd(const msa_dims *dims, const void *q, cons
  *   k_cache, v_cache bf16 [B, N, H_kv, d];  k_idx_cache bf16 [B, N, d_idx]
  *   out        fp32 [B, H_q, d]: the fp32-accumulated result        (output)
  *   blocks_out int32 [B, H_kv, topk+1] or NULL                       (output)
+ *   margin_out fp32 [B, H_kv] or NULL: the cutoff margin r_(k) - r_(k+1) of each (sequence, group)
+ *              ranking of block maxima (scaled by scale_idx), +inf when every complete past block
+ *              is taken ("4.1.1 · 监督与联合训练", section 1.1, eq (9): a small margin marks
+ *              the rows whose selection FP8 rounding or reduction order can flip)   (output)
  * Needs ceil(N / block_k) <= 8192 cache blocks (MSA_ERR_UNSUPPORTED otherwise).
  */
 MSA_API msa_status msa_sparse_attn_decode(const msa_dims *dims, const int32_t *cache_len, const void *q, const void *q_idx,
                                   const void *k_cache, const void *v_cache, const void *k_idx_cache, float *out,
-                                  int32_t *blocks_out, void *ws, size_t ws_bytes, msa_stream_t stream);
+                                  int32_t *blocks_out, float *margin_out, void *ws, size_t ws_bytes,
+                                  msa_stream_t stream);
+
+/*
+ * Row-wise e4m3 quantisation: the serving copy of the index keys. The selector keys are kept in
+ * bf16 for training and quantised to FP8 for inference ("4.1.1 · 监督与联合训练", section 2;
+ * "MSA Indexer 与 DSA Lightning Indexer 的差别", section 3.1: the indexer can run in FP8).
+ * For each row r of x:
+ *   scale[r]   = max_c |x[r,c]| / 448 in fp32 (1 for an all-zero row)
+ *   codes[r,c] = e4m3(x[r,c] / scale[r]): the fp32 quotient rounded to the nearest e4m3 value
+ *                (ties to even mantissa), saturated to +-448; e4m3 = 1 sign, 4 exponent (bias 7)
+ *                and 3 mantissa bits, finite range +-448, no infinities
+ *   x     bf16  [rows, n]
+ *   codes uint8 [rows, n] (e4m3 bit patterns)                          (output)
+ *   scale fp32  [rows]                                                 (output)
+ * n in {16, 32, 64, 128, 256}; rows >= 0 (0 enqueues nothing). Used on a K_idx cache, rows = B*N
+ * and n = d_idx give the layout msa_sparse_attn_decode_fp8idx reads.
+ */
+MSA_API msa_status msa_quantize_e4m3_rows(const void *x, int64_t rows, int n, uint8_t *codes, float *scale,
+                                          msa_stream_t stream);
+
+/*
+ * msa_sparse_attn_decode with FP8 index scoring: the K_idx cache is held as e4m3 codes with one
+ * fp32 scale per token (msa_quantize_e4m3_rows of the bf16 keys), half the bytes of the index
+ * scan that dominates a decode step. Q_idx stays bf16 in memory; the step rounds each (sequence,
+ * group) row to e4m3 with the same row-scale rule. The index score of token j for group r is
+ *   S_j = scale_idx * sq_r * sk_j * sum_c q8_r[c] * k8_j[c]
+ * with every product exact and the sum accumulated in fp32; pooling, Top-k, the local block and
+ * the attention are those of msa_sparse_attn_decode. Rows whose bf16 margin is small may select
+ * other blocks than the bf16 step: margin_out (the FP8 ranking's margin) reports them.
+ *   k_idx_codes uint8 [B, N, d_idx];  k_idx_scale fp32 [B, N]
+ * Other arguments, sizes and errors as msa_sparse_attn_decode; same workspace.
+ */
+MSA_API msa_status msa_sparse_attn_decode_fp8idx(const msa_dims *dims, const int32_t *cache_len, const void *q,
+                                                 const void *q_idx, const void *k_cache, const void *v_cache,
+                                                 const uint8_t *k_idx_codes, const float *k_idx_scale, float *out,
+                                                 int32_t *blocks_out, float *margin_out, void *ws, size_t ws_bytes,
+                                                 msa_stream_t stream);
 
 /*
  * KL alignment of the index branch ("MSA 中的 KL 对齐与局部知识蒸馏", sections 2, 3 and 6).
@@ -155,7 +197,8 @@ MSA_API msa_status msa_kl_fwd_grad(const msa_dims *dims, const void *q, const vo
  * For callers that cannot allocate device memory where they decode (a plugin inside a host
  * application that owns every device allocation, a serving loop with a memory budget fixed at
  * start-up, a latency-bound path that must not call cudaMalloc, which can synchronise the device).
- * Same arguments, outputs and results as msa_sparse_attn_decode, minus the workspace: the scratch
+ * Same arguments, outputs and results as msa_sparse_attn_decode, minus the workspace and the
+ * margin output: the scratch
  * is a static device array of MSA_DECODE_STATIC_SCRATCH_BYTES (16 MiB) that every GPU loading this
  * library holds until the process exits. It allocates and frees nothing.
  * - Returns MSA_ERR_WORKSPACE when `dims` need more scratch than that maximum

@@ -122,3 +122,51 @@ def test_full_decode_sampled_sequences_match_oracle():
         for r in range(w.H_kv):
             if same[r]:
                 check_attention(og[r * G:(r + 1) * G], oo[0, r * G:(r + 1) * G])
+
+
+def test_full_decode_fp8idx_sampled_sequences_match_oracle():
+    """The FP8-scored decode step over the full 16 x 256K caches: the GPU quantiser's codes and
+    scales bit-exact for the sampled sequences' whole caches, selection, margins and attention
+    against the oracle, and every planted block selected by every group in both scorings."""
+    w = WORKLOADS["decode_16x256k"]
+    x = decode_inputs(w, device=DEV)
+    dm = msa.MsaDims(w.B, w.N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
+    ws = msa.workspace(msa.MSA_OP_DECODE, dm, DEV)
+    kcodes, kscale = msa.msa_quantize_e4m3_rows(x["k_idx_cache"])
+    out, blocks, margin = msa.msa_sparse_attn_decode_fp8idx(dm, x["cache_len"], x["q"], x["q_idx"], x["k_cache"],
+                                                            x["v_cache"], kcodes, kscale, ws=ws, want_margin=True)
+    _, b16 = msa.msa_sparse_attn_decode(dm, x["cache_len"], x["q"], x["q_idx"], x["k_cache"], x["v_cache"],
+                                        x["k_idx_cache"], ws=ws)
+    torch.cuda.synchronize()
+    assert msa.msa_get_device_status(ws) == msa.MSA_OK
+    planted = x["planted_blocks"].cpu().numpy()
+    for sel in (blocks.cpu().numpy(), b16.cpu().numpy()):
+        for b in range(w.B):
+            for r in range(w.H_kv):
+                assert set(planted[b].tolist()) <= set(sel[b, r].tolist()), f"sequence {b} group {r}"
+    G = w.H_q // w.H_kv
+    od = oracle.Dims(1, w.N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
+    for b in (0, w.B - 1):
+        sl = slice(b, b + 1)
+        kic = x["k_idx_cache"][sl].cpu()
+        okc, oks = oracle.quantize_e4m3_rows(kic)
+        gc = kcodes[sl].cpu().numpy()
+        gc[gc == 0x80] = 0
+        okc0 = okc.copy()
+        okc0[okc0 == 0x80] = 0
+        np.testing.assert_array_equal(gc, okc0)
+        np.testing.assert_array_equal(kscale[sl].cpu().numpy(), oks)
+        ob, om, oo, _ = oracle.decode_fp8idx(od, x["cache_len"][sl].cpu(), x["q"][sl].cpu(), x["q_idx"][sl].cpu(),
+                                             x["k_cache"][sl].cpu(), x["v_cache"][sl].cpu(), okc, oks)
+        gb = blocks[sl].cpu().numpy()
+        bad, near = compare_blocks(gb, ob, om)
+        assert bad == 0, f"sequence {b}: selection differs (near-ties excluded: {near})"
+        gm = margin[sl].cpu().numpy()
+        assert np.array_equal(np.isinf(gm), np.isinf(om))
+        fin = np.isfinite(om)
+        assert np.abs(gm[fin] - om[fin]).max(initial=0.0) <= 1e-4
+        same = np.all(gb == ob, axis=-1)[0]
+        og = out[sl].cpu().numpy()[0]
+        for r in range(w.H_kv):
+            if same[r]:
+                check_attention(og[r * G:(r + 1) * G], oo[0, r * G:(r + 1) * G])

@@ -7,7 +7,7 @@ import torch
 import block_sparse_attention_idx_b200 as msa
 import oracle
 from msa_inputs import small_prefill, WORKLOADS, prefill_inputs
-from parity import compare_blocks, check_attention, check_grad, KL_REL
+from parity import compare_blocks, check_attention, check_grad, KL_REL, NEAR_TIE
 
 pytestmark = pytest.mark.gpu
 
@@ -132,12 +132,15 @@ def test_decode_matches_oracle(shape):
     lens = torch.tensor([L, L // 2 + 17, 130][:B], dtype=torch.int32)
     dm = msa.MsaDims(B, L, H_q, H_kv, d, d_idx, bk, k)
     od = oracle.Dims(B, L, H_q, H_kv, d, d_idx, bk, k)
-    out, blocks = msa.msa_sparse_attn_decode(dm, lens.to(DEV), q.to(DEV), qi.to(DEV), kc.to(DEV), vc.to(DEV),
-                                             kic.to(DEV))
+    out, blocks, margin = msa.msa_sparse_attn_decode(dm, lens.to(DEV), q.to(DEV), qi.to(DEV), kc.to(DEV),
+                                                     vc.to(DEV), kic.to(DEV), want_margin=True)
     torch.cuda.synchronize()
     ob, om, oo, olse = oracle.decode(od, lens, q, qi, kc, vc, kic)
     bad, near = compare_blocks(blocks.cpu().numpy(), ob, om)
     assert bad == 0
+    gm = margin.cpu().numpy()
+    assert np.array_equal(np.isinf(gm), np.isinf(om))
+    assert np.abs(gm[np.isfinite(om)] - om[np.isfinite(om)]).max(initial=0.0) <= NEAR_TIE
     same = np.all(blocks.cpu().numpy() == ob, axis=-1)  # [B, H_kv]
     G = H_q // H_kv
     og = out.float().cpu().numpy()
