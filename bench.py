@@ -10,7 +10,7 @@ us per generated token of each sequence) and the training KL alignment (N=65536)
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
 Ranks run independent sequences (weak scaling, no data-path collective); timing is on the device
-with CUDA events, the max over ranks. The L2 cache is flushed (a 256 MiB write) before every
+with CUDA events, the max over ranks. The L2 cache is flushed (a 256 MiB read) before every
 timed step. --impl reference times the float64 CPU oracle on a bounded sample of the same rows.
 """
 from __future__ import annotations
@@ -155,12 +155,19 @@ def measured_traffic(kernel: str, units: float):
     return m["bytes_per_unit"] * units
 
 
+def flush_l2(flush: torch.Tensor) -> None:
+    """Evicts the previous step's lines from the 126 MB L2 by READING a 256 MiB buffer. A write
+    would also evict them, but would leave the L2 full of dirty lines whose write-back then lands
+    inside the timed step and competes with its reads."""
+    torch.amax(flush.view(torch.int32))
+
+
 def timed_steps(fn, steps: int, flush: torch.Tensor):
     """Per-step device times (ms) with CUDA events on the current stream; L2 flushed before each."""
     st = torch.cuda.current_stream()
     times = []
     for _ in range(steps):
-        flush.zero_()
+        flush_l2(flush)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(st)
         fn()
@@ -283,7 +290,7 @@ def bench_prefill(args, world, rank, msa, pk):
     dims = msa.MsaDims(w.B, w.N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
     ws_i = msa.workspace(msa.MSA_OP_INDEX_TOPK, dims, dev)
     ws_a = msa.workspace(msa.MSA_OP_ATTN_FWD, dims, dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = torch.zeros(256 << 20, dtype=torch.uint8, device=dev)
 
     def step():
         blocks = msa.msa_index_topk(dims, x["q_idx"], x["k_idx"], ws=ws_i)
@@ -366,7 +373,7 @@ def bench_prefill(args, world, rank, msa, pk):
 def measure_decode(args, world, step, scan_kernel, scan_bytes, step_bytes, pk, msa):
     """Eager and graph-replayed µs per decode step, and a profiled pass for the kernel split."""
     dev = torch.device("cuda", torch.cuda.current_device())
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = torch.zeros(256 << 20, dtype=torch.uint8, device=dev)
     # (1) eager API calls, no profiler events in the stream
     barrier(world)
     t = timed_steps(step, args.decode_steps, flush)
@@ -492,7 +499,7 @@ def bench_train(args, world, rank, msa, pk):
     ws_i = msa.workspace(msa.MSA_OP_INDEX_TOPK_LSE, dims, dev)
     ws_a = msa.workspace(msa.MSA_OP_ATTN_FWD, dims, dev)
     ws_k = msa.workspace(msa.MSA_OP_KL, dims, dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = torch.zeros(256 << 20, dtype=torch.uint8, device=dev)
 
     def step():
         blocks, lse_idx = msa.msa_index_topk(dims, x["q_idx"], x["k_idx"], want_lse=True, ws=ws_i)
@@ -574,7 +581,7 @@ def main():
             "config": {"workload": args.workload, "N": w.N, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d, "d_idx": w.d_idx,
                        "block_k": w.block_k, "topk": w.topk, "batch_per_gpu": w.B, "global_batch": w.B * world,
                        "parallelism": f"dp{world} (independent sequences)",
-                       "l2": "flushed (256 MiB write) before every timed step",
+                       "l2": "flushed (256 MiB read) before every timed step; inputs also larger than L2",
                        "step": "msa_index_topk + msa_sparse_attn_fwd"},
             "roofline": pre["roofline"], "e2e": pre["e2e"], "gpu_launches": pre["gpu_launches"],
             "clocks": pre["clocks"], "kernels": pre["kernels"], "work": pre["work"],
