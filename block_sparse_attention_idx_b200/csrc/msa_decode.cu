@@ -212,14 +212,6 @@ __device__ __forceinline__ void mma_16816_f16(float (&c)[4], const uint32_t (&a)
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
-// Arrives on `bar` once this thread's earlier cp.async copies have landed (counted in its init).
-__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
 // Row-wise e4m3 quantisation (the serving copy of the index keys: keys kept in bf16 for training
 // are quantised to FP8 for inference). Each row gets the scale max|x| / 448 and codes
 // e4m3(x / scale). Threads own 8 consecutive elements; the NL = n / 8 threads of a row are
@@ -585,196 +577,258 @@ __global__ void __launch_bounds__(256) k_dec_topk(DecodeArgs a) {
     }
 }
 
-// One CTA (4 warps) per (sequence, group, selected slot): attention of the group's G heads over one
-// block. K and V are staged in shared memory as bf16 (rows padded by 16 bytes: conflict-free
-// fragment loads) with cp.async, V in a second copy group that lands while S is computed. The G
-// heads are the M=16 rows of warp-level mma.sync.m16n8k16 tiles (G=32 takes two row tiles; fewer
-// heads are padded with zero rows). Warp w computes S = Q.K^T for its 16-token units and the
-// softmax statistics (combined across warps in shared memory), then writes P as bf16 to shared
-// memory; after one barrier each warp computes P.V for a quarter of the output columns over all
-// tokens (P by ldmatrix, V by ldmatrix.trans) and writes them: no atomics, no cross-warp O sum.
-// Output: the slot's partial normalised by the sum of the bf16-rounded P the MMA multiplies (as in
-// the prefill attention), and its LSE from the exact sum.
+// Decode attention, persistent: one CTA per SM takes the (sequence, group, slot) items c, c + grid,
+// ... of the selection. Warp 8 streams each item's K and V block and the group's Q rows by TMA
+// (64-column boxes, 128B-swizzled) through a 3-stage ring; warps 0-7 compute the item: S = Q.K^T
+// for the G heads (mma.sync with Q by ldmatrix, 16-token units spread over the warps), the softmax
+// statistics (combined across warps in shared memory), P as bf16 in shared memory, then P.V split
+// by output columns. The slot's partial is normalised by the sum of the bf16-rounded P that the MMA
+// multiplies, as in the prefill attention, with its LSE from the exact sum; k_dec_combine merges
+// the slots.
+constexpr int kAttnStages = 3;
+constexpr int kAttnWarps = 8;
+
 template <int D, int BK>
-__global__ void __launch_bounds__(128) k_dec_attn(DecodeArgs a, const __nv_bfloat16* __restrict__ q,
-                                                  const __nv_bfloat16* __restrict__ kc,
-                                                  const __nv_bfloat16* __restrict__ vc) {
-    constexpr int KP = D + 8;          // padded K/V row (bf16)
-    constexpr int PP = BK + 8;         // padded P row (bf16)
-    constexpr int NU = BK / 16;        // 16-token units
-    constexpr int UPW = (NU + 3) / 4;  // units per warp
-    constexpr int DW = D / 4;          // output columns per warp
-    extern __shared__ __align__(16) uint8_t dec_smem[];
-    __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(dec_smem);  // [BK][KP]
-    __nv_bfloat16* sV = sK + BK * KP;                                 // [BK][KP]
-    __nv_bfloat16* sP = sV + BK * KP;                                 // [16][PP]
-    float* sRed = reinterpret_cast<float*>(sP + 16 * PP);             // [4][16] per-warp max, then exact sums
-    float* sRedR = sRed + 64;                                         // [4][16] per-warp rounded sums
+struct AttnSmem {
+    alignas(1024) __nv_bfloat16 kv[kAttnStages][2][BK * D];  // [stage][K, V][D/64 halves of BK x 64]
+    __nv_bfloat16 qt[kAttnStages][2][16 * D];                // [stage][row tile][D/64 halves of 16 x 64]
+    __nv_bfloat16 p[16][BK + 8];                             // P rows (heads) of one 16-row tile
+    float red[3][kAttnWarps][16];                            // per-warp maxima, exact sums, rounded sums
+    uint64_t full[kAttnStages], empty[kAttnStages];
+};
+
+// byte offset of (row, column col) in a tile of D/64 swizzled halves of `rows` x 64 bf16
+template <int ROWS>
+__device__ __forceinline__ uint32_t tile_off(int row, int col) {
+    return (uint32_t)(col >> 6) * (ROWS * 128) + swz(row, (col & 63) * 2, 128);
+}
+
+__device__ __forceinline__ void ldsm_x2_trans(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+
+template <int D, int BK>
+__global__ void __launch_bounds__((kAttnWarps + 1) * 32, 1)
+    k_dec_attn_tma(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const __grid_constant__ CUtensorMap tm_q, DecodeArgs a) {
+    using Sm = AttnSmem<D, BK>;
+    constexpr int NU = BK / 16;                              // 16-token units
+    constexpr int UPW = (NU + kAttnWarps - 1) / kAttnWarps;  // units per warp
+    constexpr int DW = D / kAttnWarps;                       // output columns per warp (8 or 16)
+    constexpr uint32_t kTileBytes = BK * D * 2;
+    extern __shared__ uint8_t attn_raw[];
+    Sm& s = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(attn_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
     const int G = a.H_q / a.H_kv;
+    const int n_mt = (G + 15) / 16;
     const int K1 = a.topk + 1;
-    const int bs = blockIdx.x;  // b * H_kv + r
-    const int slot = blockIdx.y;
-    const int b = bs / a.H_kv, r = bs % a.H_kv;
+    const int n_items = a.B * a.H_kv * K1;
+    if (threadIdx.x == 0) {
+        for (int x = 0; x < kAttnStages; ++x) {
+            mbar_init(&s.full[x], 1);
+            mbar_init(&s.empty[x], kAttnWarps);  // each consumer warp releases the stage after its reads
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
     pdl_wait();  // the selection comes from the Top-k
-    const int c = a.sel[(size_t)bs * K1 + slot];
-    float* lse_out = a.lse_part + ((size_t)bs * K1 + slot) * G;
-    if (c < 0) {
-        for (int h = threadIdx.x; h < G; h += blockDim.x) lse_out[h] = -INFINITY;
+    if (warp == kAttnWarps) {
+        if (lane == 0) {
+            int n = 0;
+            for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+                const int c = a.sel[it];  // items are numbered like the selection [B, H_kv, K1]
+                if (c < 0) continue;
+                const int st = n % kAttnStages;
+                if (n >= kAttnStages && !mbar_wait(&s.empty[st], ((n / kAttnStages) - 1) & 1, a.status, 0x921)) break;
+                mbar_arrive_expect_tx(&s.full[st], 2 * kTileBytes + (uint32_t)n_mt * 16 * D * 2);
+                const int bs = it / K1, b = bs / a.H_kv, r = bs % a.H_kv;
+#pragma unroll
+                for (int h = 0; h < D / 64; ++h) {
+                    tma_load_4d(&s.kv[st][0][h * BK * 64], &tm_k, &s.full[st], 64 * h, r, c * BK, b);
+                    tma_load_4d(&s.kv[st][1][h * BK * 64], &tm_v, &s.full[st], 64 * h, r, c * BK, b);
+                    for (int mt = 0; mt < n_mt; ++mt)
+                        tma_load_2d(&s.qt[st][mt][h * 16 * 64], &tm_q, &s.full[st], 64 * h,
+                                    b * a.H_q + r * G + 16 * mt);
+                }
+                ++n;
+            }
+            for (int m = max(0, n - kAttnStages); m < n; ++m)
+                mbar_wait(&s.full[m % kAttnStages], (m / kAttnStages) & 1, a.status, 0x922);
+        }
         pdl_trigger();
         return;
     }
-    const int len = a.cache_len[b];
-    for (int x = threadIdx.x; x < BK * D / 8; x += blockDim.x) {
-        const int t = x / (D / 8), c8 = x % (D / 8);
-        const bool ok = (size_t)c * BK + t < (size_t)a.L;
-        const size_t go = (((size_t)b * a.L + (ok ? (size_t)c * BK + t : 0)) * a.H_kv + r) * D + c8 * 8;
-        cp_async_16_zfill(smem_u32(sK + t * KP + c8 * 8), kc + go, ok);
-    }
-    cp_async_commit();
-    for (int x = threadIdx.x; x < BK * D / 8; x += blockDim.x) {
-        const int t = x / (D / 8), c8 = x % (D / 8);
-        const bool ok = (size_t)c * BK + t < (size_t)a.L;
-        const size_t go = (((size_t)b * a.L + (ok ? (size_t)c * BK + t : 0)) * a.H_kv + r) * D + c8 * 8;
-        cp_async_16_zfill(smem_u32(sV + t * KP + c8 * 8), vc + go, ok);
-    }
-    cp_async_commit();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
     const float sl2 = a.scale * 1.4426950408889634f;
-    float* o_out = a.o_part + ((size_t)bs * K1 + slot) * G * D;
-    // Q fragments of a row tile: rows h0 = 16mt + g and h1 = h0 + 8 (zero beyond G); the first
-    // tile's are loaded while K and V are still in flight
-    uint32_t qa[D / 16][4];
-    auto load_q = [&](int mt) {
-        const int h0 = mt * 16 + g, h1 = h0 + 8;
-        const int h0c = min(h0, G - 1), h1c = min(h1, G - 1);  // padded rows read nothing
-        const uint32_t* q0 = reinterpret_cast<const uint32_t*>(q + ((size_t)b * a.H_q + (size_t)r * G + h0c) * D);
-        const uint32_t* q1 = reinterpret_cast<const uint32_t*>(q + ((size_t)b * a.H_q + (size_t)r * G + h1c) * D);
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-            qa[ks][0] = h0 < G ? q0[8 * ks + t4] : 0u;
-            qa[ks][1] = h1 < G ? q1[8 * ks + t4] : 0u;
-            qa[ks][2] = h0 < G ? q0[8 * ks + 4 + t4] : 0u;
-            qa[ks][3] = h1 < G ? q1[8 * ks + 4 + t4] : 0u;
+    int n = 0;
+    int c_next = blockIdx.x < n_items ? a.sel[blockIdx.x] : -1;
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+        const int c = c_next;
+        if (it + (int)gridDim.x < n_items) c_next = a.sel[it + gridDim.x];  // in flight during this item
+        float* lse_out = a.lse_part + (size_t)it * G;
+        if (c < 0) {
+            for (int h = threadIdx.x; h < G; h += kAttnWarps * 32) lse_out[h] = -INFINITY;
+            continue;
         }
-    };
-    load_q(0);
-    cp_async_wait_group<1>();
-    __syncthreads();
-    for (int mt = 0; mt * 16 < G; ++mt) {
-        const int h0 = mt * 16 + g, h1 = h0 + 8;
-        if (mt > 0) load_q(mt);
-        // S (log2 units) of the warp's units; tokens past the query are -inf
-        float sc[UPW][2][4];
-        float mx0 = -INFINITY, mx1 = -INFINITY;
+        const int b = (it / K1) / a.H_kv;
+        const int len = a.cache_len[b];
+        const int st = n % kAttnStages;
+        const uint32_t kbase = smem_u32(&s.kv[st][0][0]), vbase = smem_u32(&s.kv[st][1][0]);
+        float* o_out = a.o_part + (size_t)it * G * D;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&s.full[st], (n / kAttnStages) & 1, a.status, 0x923));
+        // every warp learns whether any warp timed out
+        if (bar_red_or(1, kAttnWarps * 32, !ok)) break;
+        for (int mt = 0; mt < n_mt; ++mt) {
+            const int h0 = mt * 16 + g, h1 = h0 + 8;
+            const uint32_t qbase = smem_u32(&s.qt[st][mt][0]);
+            // S (log2 units) of the warp's units; tokens past the query are -inf
+            float sc[UPW][2][4];
+            float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < UPW; ++j) {
-            const int u = warp + 4 * j;
+            for (int j = 0; j < UPW; ++j) {
+                const int u = warp + kAttnWarps * j;
 #pragma unroll
-            for (int tl = 0; tl < 2; ++tl) {
-                sc[j][tl][0] = sc[j][tl][1] = sc[j][tl][2] = sc[j][tl][3] = 0.f;
+                for (int tl = 0; tl < 2; ++tl) sc[j][tl][0] = sc[j][tl][1] = sc[j][tl][2] = sc[j][tl][3] = 0.f;
                 if (u < NU) {
-                    const uint32_t* krow = reinterpret_cast<const uint32_t*>(sK + (16 * u + 8 * tl + g) * KP);
 #pragma unroll
-                    for (int ks = 0; ks < D / 16; ++ks) mma_16816_bf16(sc[j][tl], qa[ks], krow[8 * ks + t4], krow[8 * ks + 4 + t4]);
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        uint32_t qa[4];
+                        asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                                     : "=r"(qa[0]), "=r"(qa[1]), "=r"(qa[2]), "=r"(qa[3])
+                                     : "r"(qbase + tile_off<16>((lane & 7) + 8 * ((lane >> 3) & 1),
+                                                                16 * ks + 8 * (lane >> 4))));
+#pragma unroll
+                        for (int tl = 0; tl < 2; ++tl) {
+                            const int t = 16 * u + 8 * tl + g;
+                            uint32_t b0, b1;
+                            asm volatile("ld.shared.b32 %0, [%1];" : "=r"(b0) : "r"(kbase + tile_off<BK>(t, 16 * ks + 2 * t4)));
+                            asm volatile("ld.shared.b32 %0, [%1];" : "=r"(b1) : "r"(kbase + tile_off<BK>(t, 16 * ks + 8 + 2 * t4)));
+                            mma_16816_bf16(sc[j][tl], qa, b0, b1);
+                        }
+                    }
                 }
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int tok = c * BK + 16 * u + 8 * tl + 2 * t4 + (e & 1);
-                    sc[j][tl][e] = (u < NU && tok <= len - 1) ? sc[j][tl][e] * sl2 : -INFINITY;
+                for (int tl = 0; tl < 2; ++tl) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int tok = c * BK + 16 * u + 8 * tl + 2 * t4 + (e & 1);
+                        sc[j][tl][e] = (u < NU && tok <= len - 1) ? sc[j][tl][e] * sl2 : -INFINITY;
+                    }
+                    mx0 = fmaxf(mx0, fmaxf(sc[j][tl][0], sc[j][tl][1]));
+                    mx1 = fmaxf(mx1, fmaxf(sc[j][tl][2], sc[j][tl][3]));
                 }
-                mx0 = fmaxf(mx0, fmaxf(sc[j][tl][0], sc[j][tl][1]));
-                mx1 = fmaxf(mx1, fmaxf(sc[j][tl][2], sc[j][tl][3]));
             }
-        }
 #pragma unroll
-        for (int o = 1; o < 4; o <<= 1) {
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-        }
-        if (t4 == 0) {
-            sRed[warp * 16 + g] = mx0;
-            sRed[warp * 16 + g + 8] = mx1;
-        }
-        __syncthreads();
-        const float m0 = fmaxf(fmaxf(sRed[g], sRed[16 + g]), fmaxf(sRed[32 + g], sRed[48 + g]));
-        const float m1 = fmaxf(fmaxf(sRed[8 + g], sRed[24 + g]), fmaxf(sRed[40 + g], sRed[56 + g]));
-        __syncthreads();
-        // P (bf16 into shared memory); l: exact sums, lr: sums of the rounded P
-        float l0 = 0.f, l1 = 0.f, lr0 = 0.f, lr1 = 0.f;
+            for (int o = 1; o < 4; o <<= 1) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+            }
+            if (t4 == 0) {
+                s.red[0][warp][g] = mx0;
+                s.red[0][warp][g + 8] = mx1;
+            }
+            bar_sync_named(1, kAttnWarps * 32);
+            float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < UPW; ++j) {
-            const int u = warp + 4 * j;
-            if (u >= NU) continue;
+            for (int w = 0; w < kAttnWarps; ++w) {
+                m0 = fmaxf(m0, s.red[0][w][g]);
+                m1 = fmaxf(m1, s.red[0][w][g + 8]);
+            }
+            // P (bf16 into shared memory); l: exact sums, lr: sums of the rounded P
+            float l0 = 0.f, l1 = 0.f, lr0 = 0.f, lr1 = 0.f;
 #pragma unroll
-            for (int tl = 0; tl < 2; ++tl) {
-                float p[4];
+            for (int j = 0; j < UPW; ++j) {
+                const int u = warp + kAttnWarps * j;
+                if (u >= NU) continue;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    p[e] = sc[j][tl][e] == -INFINITY ? 0.f : exp2f(sc[j][tl][e] - (e < 2 ? m0 : m1));
-                    if (e < 2) l0 += p[e]; else l1 += p[e];
+                for (int tl = 0; tl < 2; ++tl) {
+                    float p[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        p[e] = sc[j][tl][e] == -INFINITY ? 0.f : exp2f(sc[j][tl][e] - (e < 2 ? m0 : m1));
+                        if (e < 2) l0 += p[e]; else l1 += p[e];
+                    }
+                    const uint32_t w0 = pack_bf16x2(p[0], p[1]), w1 = pack_bf16x2(p[2], p[3]);
+                    lr0 += __uint_as_float(w0 << 16) + __uint_as_float(w0 & 0xffff0000u);
+                    lr1 += __uint_as_float(w1 << 16) + __uint_as_float(w1 & 0xffff0000u);
+                    const int col = 16 * u + 8 * tl + 2 * t4;
+                    *reinterpret_cast<uint32_t*>(&s.p[g][col]) = w0;
+                    *reinterpret_cast<uint32_t*>(&s.p[g + 8][col]) = w1;
                 }
-                const uint32_t w0 = pack_bf16x2(p[0], p[1]), w1 = pack_bf16x2(p[2], p[3]);
-                lr0 += __uint_as_float(w0 << 16) + __uint_as_float(w0 & 0xffff0000u);
-                lr1 += __uint_as_float(w1 << 16) + __uint_as_float(w1 & 0xffff0000u);
-                const int col = 16 * u + 8 * tl + 2 * t4;
-                *reinterpret_cast<uint32_t*>(sP + g * PP + col) = w0;
-                *reinterpret_cast<uint32_t*>(sP + (g + 8) * PP + col) = w1;
             }
-        }
 #pragma unroll
-        for (int o = 1; o < 4; o <<= 1) {
-            l0 += __shfl_xor_sync(0xffffffffu, l0, o);
-            l1 += __shfl_xor_sync(0xffffffffu, l1, o);
-            lr0 += __shfl_xor_sync(0xffffffffu, lr0, o);
-            lr1 += __shfl_xor_sync(0xffffffffu, lr1, o);
-        }
-        if (t4 == 0) {
-            sRed[warp * 16 + g] = l0;
-            sRed[warp * 16 + g + 8] = l1;
-            sRedR[warp * 16 + g] = lr0;
-            sRedR[warp * 16 + g + 8] = lr1;
-        }
-        if (mt == 0) cp_async_wait_group<0>();
-        __syncthreads();
-        // O[:, warp's columns] = P.V over all tokens
-        float ov[DW / 8][4];
-#pragma unroll
-        for (int nd = 0; nd < DW / 8; ++nd) ov[nd][0] = ov[nd][1] = ov[nd][2] = ov[nd][3] = 0.f;
-#pragma unroll
-        for (int u = 0; u < NU; ++u) {
-            uint32_t pa[4];
-            {
-                // A = P rows (heads) x 16 tokens: matrices rows 0-7 / 8-15 at token columns +0 / +8
-                const int prow = ((lane >> 3) & 1) * 8 + (lane & 7), pcol = 16 * u + 8 * (lane >> 4);
-                asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                             : "=r"(pa[0]), "=r"(pa[1]), "=r"(pa[2]), "=r"(pa[3])
-                             : "r"(smem_u32(sP + prow * PP + pcol)));
+            for (int o = 1; o < 4; o <<= 1) {
+                l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+                l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+                lr0 += __shfl_xor_sync(0xffffffffu, lr0, o);
+                lr1 += __shfl_xor_sync(0xffffffffu, lr1, o);
             }
-            const int vrow = 16 * u + 8 * ((lane >> 3) & 1) + (lane & 7);
-#pragma unroll
-            for (int nd = 0; nd < DW / 8; nd += 2) {
-                uint32_t b00, b01, b10, b11;
-                ldsm_x4_trans(smem_u32(sV + vrow * KP + warp * DW + 8 * (nd + (lane >> 4))), b00, b01, b10, b11);
-                mma_16816_bf16(ov[nd], pa, b00, b01);
-                mma_16816_bf16(ov[nd + 1], pa, b10, b11);
+            if (t4 == 0) {
+                s.red[1][warp][g] = l0;
+                s.red[1][warp][g + 8] = l1;
+                s.red[2][warp][g] = lr0;
+                s.red[2][warp][g + 8] = lr1;
             }
-        }
-        const float Lr0 = sRedR[g] + sRedR[16 + g] + sRedR[32 + g] + sRedR[48 + g];
-        const float Lr1 = sRedR[8 + g] + sRedR[24 + g] + sRedR[40 + g] + sRedR[56 + g];
-        const float i0 = 1.f / Lr0, i1 = 1.f / Lr1;
+            bar_sync_named(1, kAttnWarps * 32);
+            // O[:, this warp's DW columns] = P.V over all tokens, even and odd units in two
+            // accumulator sets (two independent MMA chains)
+            float ov[DW / 8][4], ow[DW / 8][4];
 #pragma unroll
-        for (int nd = 0; nd < DW / 8; ++nd) {
-            const int col = warp * DW + 8 * nd + 2 * t4;
-            if (h0 < G) *reinterpret_cast<float2*>(o_out + (size_t)h0 * D + col) = make_float2(ov[nd][0] * i0, ov[nd][1] * i0);
-            if (h1 < G) *reinterpret_cast<float2*>(o_out + (size_t)h1 * D + col) = make_float2(ov[nd][2] * i1, ov[nd][3] * i1);
+            for (int nd = 0; nd < DW / 8; ++nd)
+                ov[nd][0] = ov[nd][1] = ov[nd][2] = ov[nd][3] = ow[nd][0] = ow[nd][1] = ow[nd][2] = ow[nd][3] = 0.f;
+#pragma unroll
+            for (int u = 0; u < NU; ++u) {
+                float (&acc)[DW / 8][4] = (u & 1) ? ow : ov;
+                uint32_t pa[4];
+                {
+                    const int prow = ((lane >> 3) & 1) * 8 + (lane & 7), pcol = 16 * u + 8 * (lane >> 4);
+                    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                                 : "=r"(pa[0]), "=r"(pa[1]), "=r"(pa[2]), "=r"(pa[3])
+                                 : "r"(smem_u32(&s.p[prow][pcol])));
+                }
+                const int vrow = 16 * u + 8 * ((lane >> 3) & 1) + (lane & 7);
+                if constexpr (DW == 16) {
+                    uint32_t b00, b01, b10, b11;
+                    ldsm_x4_trans(vbase + tile_off<BK>(vrow, warp * DW + 8 * (lane >> 4)), b00, b01, b10, b11);
+                    mma_16816_bf16(acc[0], pa, b00, b01);
+                    mma_16816_bf16(acc[1], pa, b10, b11);
+                } else {
+                    uint32_t b00, b01;
+                    ldsm_x2_trans(vbase + tile_off<BK>(vrow, warp * DW), b00, b01);
+                    mma_16816_bf16(acc[0], pa, b00, b01);
+                }
+            }
+            // this warp's last read of the stage is done: release it after the last row tile
+            if (mt == n_mt - 1) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive_relaxed(&s.empty[st]);
+            }
+#pragma unroll
+            for (int nd = 0; nd < DW / 8; ++nd)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) ov[nd][e] += ow[nd][e];
+            float L0 = 0.f, L1 = 0.f, Lr0 = 0.f, Lr1 = 0.f;
+#pragma unroll
+            for (int w = 0; w < kAttnWarps; ++w) {
+                L0 += s.red[1][w][g];
+                L1 += s.red[1][w][g + 8];
+                Lr0 += s.red[2][w][g];
+                Lr1 += s.red[2][w][g + 8];
+            }
+            const float i0 = 1.f / Lr0, i1 = 1.f / Lr1;
+#pragma unroll
+            for (int nd = 0; nd < DW / 8; ++nd) {
+                const int col = warp * DW + 8 * nd + 2 * t4;
+                if (h0 < G) *reinterpret_cast<float2*>(o_out + (size_t)h0 * D + col) = make_float2(ov[nd][0] * i0, ov[nd][1] * i0);
+                if (h1 < G) *reinterpret_cast<float2*>(o_out + (size_t)h1 * D + col) = make_float2(ov[nd][2] * i1, ov[nd][3] * i1);
+            }
+            if (warp == 0 && t4 == 0) {
+                if (h0 < G) lse_out[h0] = m0 * 0.6931471805599453f + logf(L0);
+                if (h1 < G) lse_out[h1] = m1 * 0.6931471805599453f + logf(L1);
+            }
+            // the P tile and the reduction rows are rewritten only after the next row tile's (or
+            // item's) first barrier, which every warp reaches after its reads here
         }
-        if (warp == 0 && t4 == 0) {
-            const float L0 = sRed[g] + sRed[16 + g] + sRed[32 + g] + sRed[48 + g];
-            const float L1 = sRed[8 + g] + sRed[24 + g] + sRed[40 + g] + sRed[56 + g];
-            if (h0 < G) lse_out[h0] = m0 * 0.6931471805599453f + logf(L0);
-            if (h1 < G) lse_out[h1] = m1 * 0.6931471805599453f + logf(L1);
-        }
-        __syncthreads();  // sP and sRed are rewritten by the next row tile
+        ++n;
     }
     pdl_trigger();
 }
@@ -912,32 +966,33 @@ cudaError_t run_decode(const DecodeArgs& a, const void* q, const void* q_idx, co
         if (e != cudaSuccess) return e;
     }
     ProfScope ps("dec_attn_combine", st);
-    const dim3 agrid(a.B * a.H_kv, a.topk + 1);
-    const auto* qb = static_cast<const __nv_bfloat16*>(q);
-    const auto* kb = static_cast<const __nv_bfloat16*>(k_cache);
-    const auto* vb = static_cast<const __nv_bfloat16*>(v_cache);
-    const size_t smem = (size_t)2 * a.block_k * (a.d + 8) * 2 + (size_t)16 * (a.block_k + 8) * 2 + 128 * 4;
-    auto launch = [&](auto kern) -> cudaError_t {
+    CUtensorMap tk, tv, tq;
+    const uint64_t dims[4] = {(uint64_t)a.d, (uint64_t)a.H_kv, (uint64_t)a.L, (uint64_t)a.B};
+    const uint64_t strides[3] = {(uint64_t)a.d * 2, (uint64_t)a.H_kv * a.d * 2, (uint64_t)a.L * a.H_kv * a.d * 2};
+    const uint32_t box[4] = {64, 1, (uint32_t)a.block_k, 1};
+    if (!make_tmap_4d(&tk, k_cache, dims, strides, box, 128) || !make_tmap_4d(&tv, v_cache, dims, strides, box, 128) ||
+        !make_tmap_2d(&tq, q, (uint64_t)a.d, (uint64_t)a.B * a.H_q, (uint64_t)a.d * 2, 64, 16, 128))
+        return cudaErrorInvalidValue;
+    auto launch = [&](auto kern, size_t bytes) -> cudaError_t {
+        const size_t smem = bytes + 1024;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        return launch_pdl(kern, agrid, dim3(128), smem, st, a, qb, kb, vb);
+        return launch_pdl(kern, dim3(num_sms), dim3((kAttnWarps + 1) * 32), smem, st, tk, tv, tq, a);
     };
     cudaError_t e;
-    if (a.d == 128) {
-        e = a.block_k == 128 ? launch(k_dec_attn<128, 128>) : a.block_k == 64 ? launch(k_dec_attn<128, 64>)
-                                                                               : launch(k_dec_attn<128, 32>);
-        if (e != cudaSuccess) return e;
-        e = launch_pdl(k_dec_combine<128>, dim3((a.B * a.H_q * 32 + 255) / 256), dim3(256), 0, st, a,
-                       static_cast<float*>(out));
-        if (e != cudaSuccess) return e;
-    } else {
-        e = a.block_k == 128 ? launch(k_dec_attn<64, 128>) : a.block_k == 64 ? launch(k_dec_attn<64, 64>)
-                                                                              : launch(k_dec_attn<64, 32>);
-        if (e != cudaSuccess) return e;
-        e = launch_pdl(k_dec_combine<64>, dim3((a.B * a.H_q * 32 + 255) / 256), dim3(256), 0, st, a,
-                       static_cast<float*>(out));
-        if (e != cudaSuccess) return e;
-    }
+    if (a.d == 128)
+        e = a.block_k == 128 ? launch(k_dec_attn_tma<128, 128>, sizeof(AttnSmem<128, 128>))
+            : a.block_k == 64 ? launch(k_dec_attn_tma<128, 64>, sizeof(AttnSmem<128, 64>))
+                              : launch(k_dec_attn_tma<128, 32>, sizeof(AttnSmem<128, 32>));
+    else
+        e = a.block_k == 128 ? launch(k_dec_attn_tma<64, 128>, sizeof(AttnSmem<64, 128>))
+            : a.block_k == 64 ? launch(k_dec_attn_tma<64, 64>, sizeof(AttnSmem<64, 64>))
+                              : launch(k_dec_attn_tma<64, 32>, sizeof(AttnSmem<64, 32>));
+    if (e != cudaSuccess) return e;
+    const dim3 cgrid((a.B * a.H_q * 32 + 255) / 256);
+    e = a.d == 128 ? launch_pdl(k_dec_combine<128>, cgrid, dim3(256), 0, st, a, static_cast<float*>(out))
+                   : launch_pdl(k_dec_combine<64>, cgrid, dim3(256), 0, st, a, static_cast<float*>(out));
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
