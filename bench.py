@@ -141,6 +141,16 @@ MEASURED_TRAFFIC = {
                     "sha256": "14cb19baa5ea1a26ed617e36066629b07b8a9f99a90d086cb3700db4150cafa5",
                     "bytes_per_unit": (991507200 + 136743680) / 60309504, "unit": "selected token",
                     "capture": "profiles/kl_kv_outer_train_8k.md"},
+    # decode scans at 16 x 131,072 (read + write per launch over 16 x 130,944 scanned tokens), scaled
+    # by the scanned tokens of the timed launch
+    "dec_scan": {"file": "block_sparse_attention_idx_b200/csrc/msa_decode.cu",
+                 "sha256": "5420651959775c3eda231b8e78682d94e3e90e5128be9c7164f520c3120e3f31",
+                 "bytes_per_unit": (268226784 + 696704) / (16 * 130944), "unit": "scanned token",
+                 "capture": "profiles/decode_16x256k.md"},
+    "dec_scan_e4m3": {"file": "block_sparse_attention_idx_b200/csrc/msa_decode.cu",
+                      "sha256": "5420651959775c3eda231b8e78682d94e3e90e5128be9c7164f520c3120e3f31",
+                      "bytes_per_unit": (142527168 + 238272) / (16 * 130944), "unit": "scanned token",
+                      "capture": "profiles/decode_16x256k.md"},
 }
 
 
@@ -370,7 +380,7 @@ def bench_prefill(args, world, rank, msa, pk):
     return res
 
 
-def measure_decode(args, world, step, scan_kernel, scan_bytes, step_bytes, pk, msa):
+def measure_decode(args, world, step, scan_kernel, scan_bytes, step_bytes, pk, msa, scanned_tokens=None):
     """Eager and graph-replayed µs per decode step, and a profiled pass for the kernel split."""
     dev = torch.device("cuda", torch.cuda.current_device())
     flush = torch.zeros(256 << 20, dtype=torch.uint8, device=dev)
@@ -410,7 +420,8 @@ def measure_decode(args, world, step, scan_kernel, scan_bytes, step_bytes, pk, m
            "step_roofline": roofline_entry("hbm", step_bytes / (us * 1e-6) / 1e9, pk["hbm_gbs"], "GB/s"),
            "step_roofline_graph": roofline_entry("hbm", step_bytes / (us_graph * 1e-6) / 1e9, pk["hbm_gbs"], "GB/s")
            if us_graph == us_graph else None,
-           "roofline": {**roofline_entry("hbm", scan_bytes / (scan_ms * 1e-3) / 1e9, pk["hbm_gbs"], "GB/s"),
+           "roofline": {**roofline_entry("hbm", scan_bytes / (scan_ms * 1e-3) / 1e9, pk["hbm_gbs"], "GB/s",
+                                         measured_traffic(scan_kernel, scanned_tokens or 0) if scanned_tokens else None),
                         "kernel": scan_kernel, "bytes_per_step": scan_bytes,
                         "launches_per_step": prof[scan_kernel]["launches"] // args.decode_steps},
            "kernels": {k: {"ms_per_step": round(v["total_ms"] / args.decode_steps, 4),
@@ -442,7 +453,8 @@ def bench_decode(args, world, rank, msa, pk):
     sel_blocks = int((blocks >= 0).sum().item())
     kv_bytes = sel_blocks * w.block_k * w.d * 2 * 2
     small_bytes = w.B * (w.H_q * w.d * 2 * 2 + w.H_kv * w.d_idx * 2)
-    m = measure_decode(args, world, step, "dec_scan", scan_bytes, scan_bytes + kv_bytes + small_bytes, pk, msa)
+    m = measure_decode(args, world, step, "dec_scan", scan_bytes, scan_bytes + kv_bytes + small_bytes, pk, msa,
+                       scanned_tokens=w.B * nscored)
     res = {"workload": "decode_16x256k" if L == w.N else f"decode_16x{L}", "us_per_token": m["us_per_step"],
            "tokens_per_s": w.B * world / (m["us_per_step"] * 1e-6), **m}
 
@@ -460,7 +472,7 @@ def bench_decode(args, world, rank, msa, pk):
     scan8 = w.B * nscored * (w.d_idx + 4)
     sel8 = int((blocks8 >= 0).sum().item())
     m8 = measure_decode(args, world, step8, "dec_scan_e4m3", scan8,
-                        scan8 + sel8 * w.block_k * w.d * 2 * 2 + small_bytes, pk, msa)
+                        scan8 + sel8 * w.block_k * w.d * 2 * 2 + small_bytes, pk, msa, scanned_tokens=w.B * nscored)
     # flip report: bf16 vs FP8 selection, bf16 margins of the rows that flip, planted-block recall
     _, b16, mg16 = msa.msa_sparse_attn_decode(dims, x["cache_len"], x["q"], x["q_idx"], x["k_cache"],
                                               x["v_cache"], x["k_idx_cache"], ws=ws, want_margin=True)
