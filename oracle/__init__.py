@@ -86,6 +86,7 @@ def lib():
         _lib.orc_attend_tokens.argtypes = [ctypes.c_int, ctypes.c_double, P, P, P, P, ctypes.c_int, P, P]
         _lib.orc_kl.argtypes = [D, P, P, P, P, ctypes.c_int, P, ctypes.c_double, P, i64, P, P, P, P]
         _lib.orc_decode.argtypes = [D, P, P, P, P, P, P, ctypes.c_int, P, P, P, P]
+        _lib.orc_sparse_attn_bwd.argtypes = [D, P, P, P, P, ctypes.c_int, P, P, P, P]
         _lib.orc_e4m3_values.argtypes = [P, i64, P]
         _lib.orc_e4m3_round_many.argtypes = [P, i64, P]
         _lib.orc_quantize_e4m3_rows.argtypes = [P, i64, ctypes.c_int, P, P]
@@ -221,6 +222,19 @@ def sparse_attn(dims: Dims, q, k, v, blocks, rows=None):
     lib().orc_sparse_attn(ctypes.byref(dims.c()), _ptr(qt), _ptr(kt), _ptr(vt), ty, _ptr(bt),
                           _ptr(rt) if rt is not None else None, nrows, out.ctypes.data, lse.ctypes.data)
     return out, lse
+
+
+def sparse_attn_bwd(dims: Dims, q, k, v, blocks, dout):
+    """Gradients of sum(dout * o) of the sparse attention with the selection fixed: (dq [B,N,H_q,d],
+    dk [B,N,H_kv,d], dv [B,N,H_kv,d]) in float64."""
+    (qt, kt, vt, gt), ty = _inp(q, k, v, dout)
+    bl = _full_blocks(dims, blocks)
+    dq = np.zeros((dims.B, dims.N, dims.H_q, dims.d), dtype=np.float64)
+    dk = np.zeros((dims.B, dims.N, dims.H_kv, dims.d), dtype=np.float64)
+    dv = np.zeros((dims.B, dims.N, dims.H_kv, dims.d), dtype=np.float64)
+    lib().orc_sparse_attn_bwd(ctypes.byref(dims.c()), _ptr(qt), _ptr(kt), _ptr(vt), _ptr(gt), ty, _ptr(bl),
+                              dq.ctypes.data, dk.ctypes.data, dv.ctypes.data)
+    return dq, dk, dv
 
 
 def attend_tokens(q: np.ndarray, k: np.ndarray, v: np.ndarray, J, scale: float):

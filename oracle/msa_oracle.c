@@ -21,6 +21,8 @@
  *   - loss          L_KL = 1/(N H_kv) sum_i sum_r KL(stopgrad(P_i^{(r)}) || P_i^{idx,(r)})
  *       ("KL alignment in MSA", section 3)
  *   - logit grad    dKL/dz_j = P^idx_j - P_j ("KL alignment in MSA", section 3, key gradient)
+ *   - attention bwd dL/dz_j = alpha_j g.(v_j - o) on the fixed selected set, zero elsewhere
+ *       ("2.4 training-native sparse", section 2.2, eq (11))
  *   - FP8 keys      selector keys kept in bf16 for training, quantised to FP8 for serving
  *       ("4.1.1 supervision and joint training", section 2; "MSA Indexer vs DSA Lightning
  *        Indexer", section 3.1: the indexer can run in FP8). Reading: e4m3 with one fp32 scale
@@ -283,6 +285,65 @@ int orc_sparse_attn(const orc_dims *D, const void *q, const void *k, const void 
         }
         free(J);
         free(z);
+    }
+    return 0;
+}
+
+/*
+ * Backward of the sparse attention with the selection held fixed ("2.4" page, section 2.2, eq (11):
+ * with the set fixed, selected attention is ordinary attention on it, and positions outside the set
+ * get no gradient). For each (b, i, h) with token set J, alpha = softmax_J(z), z_j = scale q.k_j,
+ * o = sum_j alpha_j v_j and upstream gradient g = dout[b,i,h]:
+ *   dL/dz_j = alpha_j g.(v_j - o)
+ *   dq     = scale sum_j dL/dz_j k_j
+ *   dk_j  += scale dL/dz_j q          (over every (i, h) of the group whose set holds j)
+ *   dv_j  += alpha_j g
+ * dq [B,N,H_q,d]; dk, dv [B,N,H_kv,d]; all float64, overwritten. Parallel over (b, group): each
+ * owns its KV head's dk/dv rows and its heads' dq rows.
+ */
+int orc_sparse_attn_bwd(const orc_dims *D, const void *q, const void *k, const void *v, const void *dout, int ty,
+                        const int32_t *blocks, double *dq, double *dk, double *dv) {
+    const int K1 = D->topk + 1, G = D->H_q / D->H_kv;
+    const double sc = eff_scale(D);
+    memset(dq, 0, sizeof(double) * (size_t)D->B * D->N * D->H_q * D->d);
+    memset(dk, 0, sizeof(double) * (size_t)D->B * D->N * D->H_kv * D->d);
+    memset(dv, 0, sizeof(double) * (size_t)D->B * D->N * D->H_kv * D->d);
+#pragma omp parallel
+    {
+        int32_t *J = (int32_t *)malloc(sizeof(int32_t) * (size_t)D->N);
+        double *z = (double *)malloc(sizeof(double) * (size_t)D->N);
+        double *o = (double *)malloc(sizeof(double) * (size_t)D->d);
+#pragma omp for schedule(dynamic, 1)
+        for (int x = 0; x < D->B * D->H_kv; ++x) {
+            const int b = x / D->H_kv, r = x % D->H_kv;
+            const size_t kv_base = ((size_t)b * D->N * D->H_kv + r) * D->d, kv_stride = (size_t)D->H_kv * D->d;
+            for (int i = 0; i < D->N; ++i) {
+                const int32_t *sel = blocks + (((size_t)b * D->N + i) * D->H_kv + r) * K1;
+                const int nJ = token_set(D, sel, K1, i, J);
+                for (int h = r * G; h < (r + 1) * G; ++h) {
+                    const size_t q_off = (((size_t)b * D->N + i) * D->H_q + h) * D->d;
+                    double lse;
+                    attend_tokens(D->d, sc, q, k, v, ty, q_off, kv_base, kv_stride, J, nJ, z, o, &lse);
+                    double go = 0.0;
+                    for (int c = 0; c < D->d; ++c) go += ld(dout, ty, q_off + c) * o[c];
+                    for (int t = 0; t < nJ; ++t) {
+                        const size_t kvo = kv_base + (size_t)J[t] * kv_stride;
+                        const double alpha = exp(z[t] - lse);
+                        double gv = 0.0;
+                        for (int c = 0; c < D->d; ++c) gv += ld(dout, ty, q_off + c) * ld(v, ty, kvo + c);
+                        const double dz = alpha * (gv - go);
+                        for (int c = 0; c < D->d; ++c) {
+                            dq[q_off + c] += sc * dz * ld(k, ty, kvo + c);
+                            dk[kvo + c] += sc * dz * ld(q, ty, q_off + c);
+                            dv[kvo + c] += alpha * ld(dout, ty, q_off + c);
+                        }
+                    }
+                }
+            }
+        }
+        free(J);
+        free(z);
+        free(o);
     }
     return 0;
 }

@@ -451,3 +451,94 @@ def test_decode_fp8_equals_bf16_decode_on_e4m3_grid():
     np.testing.assert_allclose(m8, m16, rtol=1e-14, atol=0)
     np.testing.assert_allclose(o8, o16, atol=1e-13)
     np.testing.assert_allclose(l8, l16, atol=1e-13)
+
+
+# ----------------------------------------------------------------------------- attention backward
+def test_bwd_eq11_two_position_example():
+    """2.4 · 训练原生稀疏 eq (11) through the backward: weights (0.75, 0.25) from a logit gap of ln 3,
+    v = (2,0), (0,2), upstream g = (1,-1) at the second query. The logit gradients 0.75 / -0.75 of
+    the page appear as dk (q = e_0), dv = alpha g, and dq = scale sum dz k."""
+    gld = GOLDEN["eq11_two_position"]
+    dims = oracle.Dims(B=1, N=2, H_q=1, H_kv=1, d=2, d_idx=2, block_k=1, topk=1, scale=1.0)
+    q = torch.tensor([[[[0.0, 0.0]], [[1.0, 0.0]]]], dtype=torch.float64)        # [1,2,1,2]
+    k = torch.tensor([[[[math.log(3.0), 0.0]], [[0.0, 0.0]]]], dtype=torch.float64)
+    v = torch.tensor(gld["values"], dtype=torch.float64).reshape(1, 2, 1, 2)
+    dout = torch.zeros(1, 2, 1, 2, dtype=torch.float64)
+    dout[0, 1, 0] = torch.tensor(gld["upstream_grad"], dtype=torch.float64)
+    blocks = np.array([[[[0, -1]], [[0, 1]]]], dtype=np.int32)  # row 1: past block 0 + local block 1
+    o, _ = oracle.sparse_attn(dims, q, k, v, blocks)
+    np.testing.assert_allclose(o[1, 0], gld["output"], atol=1e-14)
+    dq, dk, dv = oracle.sparse_attn_bwd(dims, q, k, v, blocks, dout)
+    dz = np.array(gld["logit_grads"])
+    np.testing.assert_allclose(dk[0, :, 0, 0], dz, atol=1e-14)      # dk_j = dz_j q, q = e_0
+    np.testing.assert_allclose(dk[0, :, 0, 1], 0.0, atol=1e-14)
+    np.testing.assert_allclose(dv[0, 0, 0], 0.75 * np.array(gld["upstream_grad"]), atol=1e-14)
+    np.testing.assert_allclose(dv[0, 1, 0], 0.25 * np.array(gld["upstream_grad"]), atol=1e-14)
+    np.testing.assert_allclose(dq[0, 1, 0], [0.75 * math.log(3.0), 0.0], atol=1e-14)
+    np.testing.assert_allclose(dq[0, 0, 0], 0.0, atol=1e-14)         # row 0 has a zero upstream gradient
+
+
+def _bwd_case(N=45, Bk=8, k=2, G=2, Hkv=2, d=8, seed=41):
+    dims = oracle.Dims(B=1, N=N, H_q=G * Hkv, H_kv=Hkv, d=d, d_idx=4, block_k=Bk, topk=k)
+    x = small_prefill(N, G * Hkv, Hkv, d, 4, Bk, k, seed=seed, dtype=torch.float64)
+    blocks, _, _ = oracle.index_topk(dims, x["q_idx"], x["k_idx"])
+    g = torch.Generator().manual_seed(seed + 1)
+    dout = torch.randn(1, N, G * Hkv, d, generator=g, dtype=torch.float64)
+    return dims, x, blocks, dout
+
+
+def test_bwd_matches_central_differences():
+    """The backward against central differences of the oracle's forward, L = sum(dout * o), on
+    sampled entries of q, k and v (selection held fixed, ragged last block)."""
+    dims, x, blocks, dout = _bwd_case()
+    dq, dk, dv = oracle.sparse_attn_bwd(dims, x["q"], x["k"], x["v"], blocks, dout)
+    grads = {"q": dq, "k": dk, "v": dv}
+    L = lambda xx: float((torch.from_numpy(oracle.sparse_attn(dims, xx["q"], xx["k"], xx["v"], blocks)[0])
+                          * dout.reshape(-1, dims.H_q, dims.d)).sum())
+    rng = np.random.default_rng(3)
+    h = 1e-6
+    for name in ("q", "k", "v"):
+        t = x[name]
+        for _ in range(12):
+            idx = tuple(int(rng.integers(0, s)) for s in t.shape)
+            xp = dict(x); xm = dict(x)
+            xp[name] = t.clone(); xm[name] = t.clone()
+            xp[name][idx] += h
+            xm[name][idx] -= h
+            fd = (L(xp) - L(xm)) / (2 * h)
+            assert grads[name][idx] == pytest.approx(fd, abs=1e-7, rel=1e-6), (name, idx)
+
+
+def test_bwd_sums_over_tokens():
+    """Closed forms from softmax normalisation: per (sequence, group), sum_j dv_j equals the sum of
+    the group's upstream gradients (the weights of each row sum to one), and sum_j dk_j = 0 (the
+    logit gradients of each row sum to zero)."""
+    dims, x, blocks, dout = _bwd_case(N=70, Bk=16, k=2, G=4, Hkv=2, d=8, seed=9)
+    dq, dk, dv = oracle.sparse_attn_bwd(dims, x["q"], x["k"], x["v"], blocks, dout)
+    G = dims.H_q // dims.H_kv
+    for r in range(dims.H_kv):
+        want = dout[0, :, r * G:(r + 1) * G].sum(dim=(0, 1)).numpy()
+        np.testing.assert_allclose(dv[0, :, r].sum(0), want, atol=1e-12)
+        np.testing.assert_allclose(dk[0, :, r].sum(0), 0.0, atol=1e-12)
+
+
+def test_bwd_dense_limit_matches_autograd():
+    """k >= every block: the backward is that of dense causal attention, checked against torch
+    autograd of scaled_dot_product_attention in float64 (GQA heads expanded)."""
+    N, Bk, G, Hkv, d = 37, 8, 2, 2, 8
+    dims = oracle.Dims(B=1, N=N, H_q=G * Hkv, H_kv=Hkv, d=d, d_idx=4, block_k=Bk, topk=8)
+    x = small_prefill(N, G * Hkv, Hkv, d, 4, Bk, 8, seed=5, dtype=torch.float64)
+    blocks, _, _ = oracle.index_topk(dims, x["q_idx"], x["k_idx"])
+    g = torch.Generator().manual_seed(6)
+    dout = torch.randn(1, N, G * Hkv, d, generator=g, dtype=torch.float64)
+    dq, dk, dv = oracle.sparse_attn_bwd(dims, x["q"], x["k"], x["v"], blocks, dout)
+    q = x["q"].clone().requires_grad_(True)
+    k = x["k"].clone().requires_grad_(True)
+    v = x["v"].clone().requires_grad_(True)
+    o = torch.nn.functional.scaled_dot_product_attention(
+        q.transpose(1, 2), k.repeat_interleave(G, dim=2).transpose(1, 2), v.repeat_interleave(G, dim=2).transpose(1, 2),
+        is_causal=True)
+    (o.transpose(1, 2) * dout).sum().backward()
+    np.testing.assert_allclose(dq, q.grad.numpy(), atol=1e-12)
+    np.testing.assert_allclose(dk, k.grad.numpy(), atol=1e-12)
+    np.testing.assert_allclose(dv, v.grad.numpy(), atol=1e-12)
