@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libmsa.so")
 
 MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_WORKSPACE, MSA_ERR_CUDA, MSA_ERR_TIMEOUT, \
     MSA_ERR_DEVICE_CHECK = range(7)
-MSA_OP_INDEX_TOPK, MSA_OP_INDEX_TOPK_LSE, MSA_OP_ATTN_FWD, MSA_OP_DECODE, MSA_OP_KL = range(5)
+MSA_OP_INDEX_TOPK, MSA_OP_INDEX_TOPK_LSE, MSA_OP_ATTN_FWD, MSA_OP_DECODE, MSA_OP_KL, MSA_OP_ATTN_BWD = range(6)
 
 
 class MsaError(RuntimeError):
@@ -73,6 +73,7 @@ def lib() -> ctypes.CDLL:
         L.msa_sparse_attn_decode_fp8idx.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, S, P]
         L.msa_quantize_e4m3_rows.argtypes = [P, ctypes.c_int64, ctypes.c_int, P, P, P]
         L.msa_kl_fwd_grad.argtypes = [D, P, P, P, P, P, P, P, ctypes.c_float, P, P, P, P, S, P]
+        L.msa_sparse_attn_bwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, S, P]
         L.msa_sparse_attn_decode_noalloc.argtypes = [D, P, P, P, P, P, P, P, P, P]
         L.msa_sparse_attn_decode_noalloc.restype = ctypes.c_int
         L.msa_get_device_status.argtypes = [P, P]
@@ -86,7 +87,7 @@ def lib() -> ctypes.CDLL:
         L.msa_version.restype = ctypes.c_char_p
         for fn in ("msa_workspace_size", "msa_index_topk", "msa_sparse_attn_fwd", "msa_sparse_attn_decode",
                    "msa_sparse_attn_decode_fp8idx", "msa_quantize_e4m3_rows", "msa_kl_fwd_grad",
-                   "msa_get_device_status"):
+                   "msa_sparse_attn_bwd", "msa_get_device_status"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -253,6 +254,28 @@ def msa_sparse_attn_decode_noalloc(dims: MsaDims, cache_len, q, q_idx, k_cache, 
     return out, blocks
 
 
+def msa_sparse_attn_bwd(dims: MsaDims, q, k, v, blocks, out, lse, dout, ws=None, stream=None):
+    """Backward of the sparse attention with the selection fixed. out / lse are the forward's
+    (fp32), dout bf16 [B,N,H_q,d]. Returns dq fp32 [B,N,H_q,d], dk and dv fp32 [B,N,H_kv,d]."""
+    dev = q.device
+    _need(q, "q", (dims.B, dims.N, dims.H_q, dims.d), torch.bfloat16, dev)
+    _need(k, "k", (dims.B, dims.N, dims.H_kv, dims.d), torch.bfloat16, dev)
+    _need(v, "v", (dims.B, dims.N, dims.H_kv, dims.d), torch.bfloat16, dev)
+    _need(blocks, "blocks", (dims.B, dims.N, dims.H_kv, dims.topk + 1), torch.int32, dev)
+    _need(out, "out", (dims.B, dims.N, dims.H_q, dims.d), torch.float32, dev)
+    _need(lse, "lse", (dims.B, dims.N, dims.H_q), torch.float32, dev)
+    _need(dout, "dout", (dims.B, dims.N, dims.H_q, dims.d), torch.bfloat16, dev)
+    dq = torch.empty(dims.B, dims.N, dims.H_q, dims.d, dtype=torch.float32, device=dev)
+    dk = torch.empty(dims.B, dims.N, dims.H_kv, dims.d, dtype=torch.float32, device=dev)
+    dv = torch.empty(dims.B, dims.N, dims.H_kv, dims.d, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = workspace(MSA_OP_ATTN_BWD, dims, dev)
+    _check("msa_sparse_attn_bwd",
+           lib().msa_sparse_attn_bwd(ctypes.byref(dims.c()), _p(q), _p(k), _p(v), _p(blocks), _p(out), _p(lse),
+                                     _p(dout), _p(dq), _p(dk), _p(dv), _p(ws), ws.numel(), _stream(stream)))
+    return dq, dk, dv
+
+
 def msa_kl_fwd_grad(dims: MsaDims, q, k, q_idx, k_idx, blocks, lse, lse_idx=None, grad_scale: float = 1.0, ws=None,
                     stream=None):
     """KL alignment. Returns loss fp32 [1], dq_idx fp32 [B,N,H_kv,d_idx], dk_idx fp32 [B,N,d_idx]."""
@@ -301,5 +324,5 @@ def msa_get_device_status(ws: torch.Tensor, stream=None) -> int:
 
 __all__ = ["MsaDims", "MsaError", "msa_workspace_size", "msa_index_topk", "msa_sparse_attn_fwd",
            "msa_sparse_attn_decode", "msa_sparse_attn_decode_noalloc", "msa_sparse_attn_decode_fp8idx",
-           "msa_quantize_e4m3_rows", "msa_kl_fwd_grad", "msa_get_device_status", "msa_status_string",
+           "msa_quantize_e4m3_rows", "msa_kl_fwd_grad", "msa_sparse_attn_bwd", "msa_get_device_status", "msa_status_string",
            "msa_version", "msa_profile_enable", "msa_profile_read", "workspace", "lib", "LIB_PATH"]

@@ -66,6 +66,9 @@ size_t ws_attn(const msa_dims* d) {
 size_t ws_decode(const msa_dims* d) {
     return kStatusBytes + decode_ws_bytes(d->B, d->N, d->H_q, d->H_kv, d->d, d->block_k, d->topk);
 }
+size_t ws_bwd(const msa_dims* d) {
+    return kStatusBytes + csr_need(d) + al256((size_t)d->B * d->N * d->H_q * 4);
+}
 size_t ws_kl(const msa_dims* d) {
     const size_t nb = (size_t)(d->N + d->block_k - 1) / d->block_k;
     const size_t nl = (size_t)d->B * d->H_kv * nb;
@@ -124,6 +127,10 @@ msa_status msa_workspace_size(int op, const msa_dims* d, size_t* bytes) {
             return MSA_OK;
         case MSA_OP_DECODE: *bytes = ws_decode(d); return MSA_OK;
         case MSA_OP_KL: *bytes = ws_kl(d); return MSA_OK;
+        case MSA_OP_ATTN_BWD:
+            if (!bwd_supported(d->d, d->H_q / d->H_kv)) return MSA_ERR_UNSUPPORTED;
+            *bytes = ws_bwd(d);
+            return MSA_OK;
     }
     return MSA_ERR_INVALID_ARG;
 }
@@ -251,6 +258,39 @@ msa_status msa_quantize_e4m3_rows(const void* x, int64_t rows, int n, uint8_t* c
     if (rows > ((int64_t)1 << 40) / n) return MSA_ERR_UNSUPPORTED;
     return cuda_status(run_quantize_e4m3_rows(x, rows, n, codes, scale, num_sms(),
                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+msa_status msa_sparse_attn_bwd(const msa_dims* d, const void* q, const void* k, const void* v, const int32_t* blocks,
+                               const float* out, const float* lse, const void* dout, float* dq, float* dk, float* dv,
+                               void* ws, size_t ws_bytes, msa_stream_t stream_) {
+    msa_status s = check_common(d);
+    if (s != MSA_OK) return s;
+    if (!bwd_supported(d->d, d->H_q / d->H_kv)) return MSA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !blocks || !out || !lse || !dout || !dq || !dk || !dv || !aligned16(q) || !aligned16(k) ||
+        !aligned16(v) || !aligned16(blocks) || !aligned16(out) || !aligned16(lse) || !aligned16(dout) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return MSA_ERR_INVALID_ARG;
+    s = ws_check(ws, ws_bytes, ws_bwd(d));
+    if (s != MSA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_);
+    DevStatus* status = static_cast<DevStatus*>(ws);
+    cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, st);
+    if (e != cudaSuccess) return MSA_ERR_CUDA;
+    Carver cv{static_cast<uint8_t*>(ws) + kStatusBytes};
+    BwdArgs a{};
+    a.B = d->B; a.N = d->N; a.H_q = d->H_q; a.H_kv = d->H_kv; a.d = d->d; a.block_k = d->block_k;
+    a.topk = d->topk; a.scale = eff_scale(d->scale, d->d);
+    csr_carve(&a.csr, cv.take(csr_need(d)), d->B, d->N, d->H_kv, d->block_k, d->topk, 0);
+    a.delta = reinterpret_cast<float*>(cv.take((size_t)d->B * d->N * d->H_q * 4));
+    a.lse = lse;
+    a.dq = dq;
+    a.dk = dk;
+    a.dv = dv;
+    a.status = status;
+    const int G = d->H_q / d->H_kv;
+    e = run_csr_build(a.csr, blocks, d->B, d->N, d->H_kv, d->block_k, d->topk, 128 / G, status, st);
+    if (e == cudaSuccess) e = run_attn_bwd(a, q, k, v, dout, out, num_sms(), st);
+    return cuda_status(e);
 }
 
 msa_status msa_kl_fwd_grad(const msa_dims* d, const void* q, const void* k, const void* q_idx, const void* k_idx,

@@ -1,0 +1,470 @@
+// Backward of the main-branch sparse attention with the selection held fixed ("2.4 · 训练原生稀疏",
+// section 2.2, eq (11): on the fixed set, selected attention is ordinary attention, and positions
+// outside the set get no gradient; the backward must stay on the sparse edges, section 3.2).
+// For each (query i, head h) with token set J, upstream gradient g = dO and output o:
+//   P_j  = exp(scale q.k_j - LSE)           (recomputed from the forward's LSE)
+//   dS_j = P_j (g.v_j - g.o)                (the gradient of the logit, eq (11))
+//   dV_j += P_j g,  dK_j += scale dS_j q,  dQ += scale sum_j dS_j k_j
+//
+// KV-outer over the inverse lists of the forward: one item = one selected block c of group r plus
+// up to 128/G queries that chose it (their G heads are the 128 rows). Per item, in TMEM:
+//   S^T  = K_c . Q^T          tcgen05.mma M=128 tokens, N=128 rows, K=d       cols [0,128)
+//   dP^T = V_c . dO^T         tcgen05.mma                                      cols [128,256)
+//   thread = token: P^T, dS^T = P^T (dP^T - delta) as bf16 back into TMEM over S^T / dP^T, and dS^T
+//   as bf16 into shared memory
+//   dV_c += P^T . dO          tcgen05.mma A = P^T from TMEM, B = dO (MN-major)  cols [256,256+d)
+//   dK_c += dS^T . Q          tcgen05.mma A = dS^T from TMEM, B = Q (MN-major)  cols [384,384+d)
+//   dQ    = dS . K_c          tcgen05.mma A = dS (MN-major smem), B = K_c, in 64-column halves
+//                             placed in the free upper halves of the S^T and dP^T columns
+// dQ rows are added to the fp32 output with vector reductions after every item; dK_c and dV_c stay
+// in TMEM across the consecutive items of one block and are added to the outputs when the block
+// changes (a block's items can be split between two CTAs, hence reductions rather than stores).
+// P and dS enter the tensor cores as bf16, as in the forward's P.
+//
+// Warp roles (192 threads): warps 0-3 epilogue (thread = token lane, or item row for dQ), warp 4
+// loads (item metadata, the Q and dO rows by one 5-D TMA box per query, K and V tiles), warp 5
+// issues the MMAs and owns TMEM.
+#include "msa_common.cuh"
+#include "msa_internal.h"
+
+namespace msa {
+
+namespace {
+
+constexpr int kRows = 128;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kProdWarp = 4, kMmaWarp = 5;
+constexpr int kThreads = 6 * 32;
+
+__device__ __forceinline__ void red_add_v4(float* p, float x, float y, float z, float w) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(x), "f"(y), "f"(z), "f"(w)
+                 : "memory");
+}
+
+template <int QPC>
+struct BwdMeta {
+    int L, count, flush, pad;  // list id (b, r, c), item queries, 1 when the next item is another block or none
+    int qi[QPC];               // query index of each item query
+    float lse2[kRows];         // LSE * log2(e) per item row (query-major, head-minor)
+    float delta[kRows];        // dO . O per item row
+};
+
+template <int D, int QPC>
+struct BwdSmem {
+    alignas(1024) uint8_t q[kRows * D * 2];     // Q rows: 8-row x 64-column 128B-swizzled atoms [row/8][D/64]
+    alignas(1024) uint8_t dout[kRows * D * 2];  // dO rows, same layout
+    alignas(1024) uint8_t k[kRows * D * 2];     // K tile: D/64 sub-tiles of [128 token rows x 128 B], rows >= BK zero
+    alignas(1024) uint8_t v[kRows * D * 2];     // V tile, same
+    alignas(1024) uint8_t ds[kRows * kRows * 2];  // dS^T: 2 sub-tiles of [128 token rows x 64 item rows]
+    BwdMeta<QPC> meta[2];
+    uint64_t meta_full[2], meta_empty[2], q_full, q_empty, kv_full, kv_empty, s_full, p_full, d_full, t_free, drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+template <int D, int BK, int G>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_attn_bwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+               const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, BwdArgs a) {
+    constexpr int QPC = kRows / G;
+    using Sm = BwdSmem<D, QPC>;
+    static_assert(G % 8 == 0 && G <= 32, "one 5-D box of G/8 head groups per query");
+    extern __shared__ uint8_t smem_raw[];
+    Sm& s = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    constexpr uint32_t kIdescS = umma_idesc_bf16(kRows, kRows, false, false);  // S^T, dP^T
+    constexpr uint32_t kIdescKV = umma_idesc_bf16(kRows, D, false, true);      // dV, dK (A from TMEM)
+    constexpr uint32_t kIdescQ = umma_idesc_bf16(kRows, 64, true, true);       // dQ halves
+    constexpr uint32_t kColS = 0, kColP = 128, kColDV = 256, kColDK = 384;
+
+    const Csr& cs = a.csr;
+    const int T = *cs.n_items;
+    const int per = (T + gridDim.x - 1) / gridDim.x;
+    const int t0 = blockIdx.x * per, t1 = min(T, t0 + per);
+    const int warp = warp_id(), lane = lane_id();
+
+    if (threadIdx.x == 0) {
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&s.meta_full[x], 32);
+            mbar_init(&s.meta_empty[x], kRows + 1);  // the epilogue threads and the MMA issuer
+        }
+        mbar_init(&s.q_full, 1);
+        mbar_init(&s.q_empty, 1);
+        mbar_init(&s.kv_full, 1);
+        mbar_init(&s.kv_empty, 1);
+        mbar_init(&s.s_full, 1);
+        mbar_init(&s.p_full, kRows);
+        mbar_init(&s.d_full, 1);
+        mbar_init(&s.t_free, kRows);
+        mbar_init(&s.drain, 1);
+        s.abort = 0;
+        fence_mbar_init();
+    }
+    // every tile row an MMA may read must hold finite values: Q / dO rows past an item's count and
+    // K / V rows past block_k are multiplied by zeros, and start as zeros
+    {
+        uint4* z = reinterpret_cast<uint4*>(s.q);
+        for (int x = threadIdx.x; x < 4 * kRows * D * 2 / 16; x += kThreads) z[x] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async();
+    if (warp == kMmaWarp) {
+        tmem_alloc(&s.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s.tmem_base;
+
+    if (warp == kProdWarp) {
+        // ------------------------------------------------------------------------ loads
+        // Item n's metadata goes to meta[n % 2] (plain loads into registers, stored once they have
+        // arrived, then one arrival per lane: no load is in flight at these release arrives), its Q
+        // and dO rows into the single Q / dO buffers once the MMA has released them, and K / V on
+        // a new block once the MMA has released the previous block.
+        bool ok = true;
+        int kv_loads = 0, prevL = -1, issued = 0;
+        int4 rec = t0 < t1 ? cs.items[t0] : make_int4(-1, 0, 0, 0);
+        for (int t = t0, n = 0; t < t1; ++t, ++n) {
+            const int L = rec.x, count = rec.z;
+            const int c = L % cs.nb, r = (L / cs.nb) % a.H_kv, b = L / (cs.nb * a.H_kv);
+            const int4 nrec = t + 1 < t1 ? cs.items[t + 1] : make_int4(-1, 0, 0, 0);
+            const int e = lane < count ? cs.entries[rec.y + lane] : 0;
+            const int qi = e >> 5;
+            float l2[4], dl[4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const int row = lane + 32 * x;
+                const int m = row / G, h = row % G;
+                const int qm = __shfl_sync(0xffffffffu, qi, m < QPC ? m : 0);
+                const size_t o = ((size_t)b * a.N + qm) * a.H_q + (size_t)r * G + h;
+                l2[x] = m < count ? a.lse[o] * kLog2e : 0.f;
+                dl[x] = m < count ? a.delta[o] : 0.f;
+            }
+            const int ms = n & 1;
+            int okl = 1;
+            if (lane == 0) okl = mbar_wait(&s.meta_empty[ms], ((n >> 1) & 1) ^ 1, a.status, 0xa01);
+            if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
+            BwdMeta<QPC>& mt = s.meta[ms];
+            if (lane == 0) {
+                mt.L = L;
+                mt.count = count;
+                mt.flush = nrec.x != L;
+            }
+            if (lane < QPC) mt.qi[lane] = lane < count ? qi : 0;
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                mt.lse2[lane + 32 * x] = l2[x];
+                mt.delta[lane + 32 * x] = dl[x];
+            }
+            mbar_arrive(&s.meta_full[ms]);
+            // Q and dO rows of the item queries
+            if (lane == 0) okl = mbar_wait(&s.q_empty, (n & 1) ^ 1, a.status, 0xa02);
+            if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
+            if (lane == 0) mbar_arrive_expect_tx_relaxed(&s.q_full, (uint32_t)(2 * count * G * D * 2));
+            __syncwarp();
+            if (lane < count) {
+                tma_load_5d(s.q + lane * G * D * 2, &tm_q, &s.q_full, 0, 0, 0, r * G / 8, b * a.N + qi);
+                tma_load_5d(s.dout + lane * G * D * 2, &tm_do, &s.q_full, 0, 0, 0, r * G / 8, b * a.N + qi);
+            }
+            // K and V of a new block
+            if (L != prevL) {
+                if (lane == 0) {
+                    if (kv_loads > 0) okl = mbar_wait(&s.kv_empty, (kv_loads - 1) & 1, a.status, 0xa03);
+                    if (okl) {
+                        mbar_arrive_expect_tx_relaxed(&s.kv_full, 2 * (D / 64) * BK * 128);
+#pragma unroll
+                        for (int sub = 0; sub < D / 64; ++sub) {
+                            tma_load_4d(s.k + sub * kRows * 128, &tm_k, &s.kv_full, sub * 64, r, c * BK, b);
+                            tma_load_4d(s.v + sub * kRows * 128, &tm_v, &s.kv_full, sub * 64, r, c * BK, b);
+                        }
+                    }
+                }
+                if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
+                ++kv_loads;
+                prevL = L;
+            }
+            ++issued;
+            rec = nrec;
+        }
+        if (!ok) s.abort = 1;
+        // nothing may still be landing in shared memory when the CTA exits
+        if (lane == 0) {
+            if (issued > 0) mbar_wait(&s.q_full, (issued - 1) & 1, a.status, 0xa04);
+            if (kv_loads > 0) mbar_wait(&s.kv_full, (kv_loads - 1) & 1, a.status, 0xa05);
+        }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            bool ok = true;
+            int kv_group = -1, prevL = -1;
+            const uint32_t qa = smem_u32(s.q), da = smem_u32(s.dout), ka = smem_u32(s.k), va = smem_u32(s.v),
+                           dsa = smem_u32(s.ds);
+            for (int t = t0, n = 0; t < t1; ++t, ++n) {
+                const int ms = n & 1;
+                if (!mbar_wait(&s.meta_full[ms], (n >> 1) & 1, a.status, 0xa11)) { ok = false; break; }
+                const int L = s.meta[ms].L;
+                mbar_arrive(&s.meta_empty[ms]);
+                bool first = false;
+                if (L != prevL) {
+                    if (kv_group >= 0) umma_commit(&s.kv_empty);  // the previous block's tiles are no longer read
+                    ++kv_group;
+                    prevL = L;
+                    first = true;
+                    if (!mbar_wait(&s.kv_full, kv_group & 1, a.status, 0xa12)) { ok = false; break; }
+                }
+                if (!mbar_wait(&s.q_full, n & 1, a.status, 0xa13)) { ok = false; break; }
+                if (n > 0 && !mbar_wait(&s.t_free, (n - 1) & 1, a.status, 0xa14)) { ok = false; break; }
+                tc_fence_after();
+                // S^T = K . Q^T and dP^T = V . dO^T (both operands K-major)
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint32_t sub = (ks * 16) / 64, off = (ks & 3) * 32;
+                    const uint64_t dk_ = umma_sdesc(ka + sub * (kRows * 128) + off, 16, 1024, 2);
+                    const uint64_t dq_ = umma_sdesc(qa + sub * 1024 + off, 16, (D / 64) * 1024, 2);
+                    umma_bf16(tmem + kColS, dk_, dq_, kIdescS, ks > 0);
+                }
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint32_t sub = (ks * 16) / 64, off = (ks & 3) * 32;
+                    const uint64_t dv_ = umma_sdesc(va + sub * (kRows * 128) + off, 16, 1024, 2);
+                    const uint64_t do_ = umma_sdesc(da + sub * 1024 + off, 16, (D / 64) * 1024, 2);
+                    umma_bf16(tmem + kColP, dv_, do_, kIdescS, ks > 0);
+                }
+                umma_commit(&s.s_full);
+                if (!mbar_wait(&s.p_full, n & 1, a.status, 0xa15)) { ok = false; break; }
+                tc_fence_after();
+                // dV += P^T . dO, dK += dS^T . Q: A from TMEM (bf16 pairs, 8 columns per 16 rows),
+                // B = the row tiles read MN-major (16 rows = two 8-row atom groups per k-step)
+#pragma unroll
+                for (int ks = 0; ks < kRows / 16; ++ks) {
+                    const uint64_t bdo = umma_sdesc(da + 2 * ks * (D / 64) * 1024, 1024, (D / 64) * 1024, 2);
+                    umma_bf16_tmem_a(tmem + kColDV, tmem + kColS + 8 * ks, bdo, kIdescKV, (first && ks == 0) ? 0u : 1u);
+                }
+#pragma unroll
+                for (int ks = 0; ks < kRows / 16; ++ks) {
+                    const uint64_t bq = umma_sdesc(qa + 2 * ks * (D / 64) * 1024, 1024, (D / 64) * 1024, 2);
+                    umma_bf16_tmem_a(tmem + kColDK, tmem + kColP + 8 * ks, bq, kIdescKV, (first && ks == 0) ? 0u : 1u);
+                }
+                // dQ = dS . K in 64-column halves: A = dS^T tile read MN-major, B = K sub-tile MN-major
+#pragma unroll
+                for (int h = 0; h < D / 64; ++h) {
+#pragma unroll
+                    for (int ks = 0; ks < BK / 16; ++ks) {
+                        const uint64_t ads = umma_sdesc(dsa + ks * 16 * 128, kRows * 128, 1024, 2);
+                        const uint64_t bk_ = umma_sdesc(ka + h * (kRows * 128) + ks * 16 * 128, kRows * 128, 1024, 2);
+                        umma_bf16(tmem + (h == 0 ? 64u : 192u), ads, bk_, kIdescQ, ks > 0);
+                    }
+                }
+                umma_commit(&s.d_full);
+                umma_commit(&s.q_empty);
+            }
+            if (!ok) s.abort = 1;
+            umma_commit(&s.drain);
+            mbar_wait(&s.drain, 0, a.status, 0xa16);
+        }
+    } else {
+        // ------------------------------------------------------------------------ epilogue
+        const int tt = warp * 32 + lane;  // token lane for S^T / dP^T / dV / dK, item row for dQ
+        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+        const float sl2 = a.scale * kLog2e;
+        for (int t = t0, n = 0; t < t1; ++t, ++n) {
+            const int ms = n & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.meta_full[ms], (n >> 1) & 1, a.status, 0xa21))) {
+                s.abort = 1;
+                break;
+            }
+            const BwdMeta<QPC>& mt = s.meta[ms];
+            const int L = mt.L, count = mt.count, flush = mt.flush;
+            const int c = L % cs.nb, r = (L / cs.nb) % a.H_kv, b = L / (cs.nb * a.H_kv);
+            const int tok = c * BK + tt;
+            const int nrows = count * G;
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.s_full, n & 1, a.status, 0xa22))) {
+                s.abort = 1;
+                break;
+            }
+            tc_fence_after();
+#pragma unroll 1
+            for (int cc = 0; cc < kRows / 32; ++cc) {
+                uint32_t sv[32], pv[32];
+                tmem_ld32(lane_addr + kColS + 32 * cc, sv);
+                tmem_ld32(lane_addr + kColP + 32 * cc, pv);
+                tmem_ld_wait();
+                reg_fence(sv);
+                reg_fence(pv);
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    float p2[2], d2[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int row = 32 * cc + e + u;
+                        const bool valid = row < nrows && tt < BK && tok <= mt.qi[row / G];
+                        const float p = valid ? exp2f(fmaf(__uint_as_float(sv[e + u]), sl2, -mt.lse2[row])) : 0.f;
+                        p2[u] = p;
+                        d2[u] = valid ? p * (__uint_as_float(pv[e + u]) - mt.delta[row]) : 0.f;
+                    }
+                    pk[e / 2] = pack_bf16x2(p2[0], p2[1]);
+                    dk[e / 2] = pack_bf16x2(d2[0], d2[1]);
+                }
+                tmem_st16(lane_addr + kColS + 16 * cc, pk);
+                tmem_st16(lane_addr + kColP + 16 * cc, dk);
+                // dS^T row of this token: item rows 32cc..32cc+31, four 16-byte chunks of 8 rows
+                uint8_t* dsrow = s.ds + (cc >> 1) * (kRows * 128);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t ch = 4 * (cc & 1) + j;
+                    *reinterpret_cast<uint4*>(dsrow + swz(tt, ch * 16, 128)) =
+                        make_uint4(dk[4 * j], dk[4 * j + 1], dk[4 * j + 2], dk[4 * j + 3]);
+                }
+            }
+            tmem_st_wait();
+            fence_proxy_async();
+            tc_fence_before();
+            mbar_arrive(&s.p_full);
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.d_full, n & 1, a.status, 0xa23))) {
+                s.abort = 1;
+                break;
+            }
+            tc_fence_after();
+            // dQ row tt of the item (TMEM lane = item row)
+            {
+                const bool rv = tt < nrows;
+                const int m = rv ? tt / G : 0, h = tt % G;
+                float* dst = a.dq + (((size_t)b * a.N + mt.qi[m]) * a.H_q + (size_t)r * G + h) * D;
+#pragma unroll
+                for (int hh = 0; hh < D / 64; ++hh) {
+#pragma unroll
+                    for (int q2 = 0; q2 < 2; ++q2) {
+                        uint32_t x[32];
+                        tmem_ld32(lane_addr + (hh == 0 ? 64u : 192u) + 32 * q2, x);
+                        tmem_ld_wait();
+                        reg_fence(x);
+                        if (rv) {
+#pragma unroll
+                            for (int e = 0; e < 32; e += 4)
+                                red_add_v4(dst + 64 * hh + 32 * q2 + e, __uint_as_float(x[e]) * a.scale,
+                                           __uint_as_float(x[e + 1]) * a.scale, __uint_as_float(x[e + 2]) * a.scale,
+                                           __uint_as_float(x[e + 3]) * a.scale);
+                        }
+                    }
+                }
+            }
+            // the block's dV and dK when its last item of this CTA is done (TMEM lane = token)
+            if (flush) {
+                const bool tv = tt < BK && tok < a.N;
+                float* dvp = a.dv + (((size_t)b * a.N + (tv ? tok : 0)) * a.H_kv + r) * D;
+                float* dkp = a.dk + (((size_t)b * a.N + (tv ? tok : 0)) * a.H_kv + r) * D;
+#pragma unroll
+                for (int q2 = 0; q2 < D / 32; ++q2) {
+                    uint32_t xv[32], xk[32];
+                    tmem_ld32(lane_addr + kColDV + 32 * q2, xv);
+                    tmem_ld32(lane_addr + kColDK + 32 * q2, xk);
+                    tmem_ld_wait();
+                    reg_fence(xv);
+                    reg_fence(xk);
+                    if (tv) {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 4) {
+                            red_add_v4(dvp + 32 * q2 + e, __uint_as_float(xv[e]), __uint_as_float(xv[e + 1]),
+                                       __uint_as_float(xv[e + 2]), __uint_as_float(xv[e + 3]));
+                            red_add_v4(dkp + 32 * q2 + e, __uint_as_float(xk[e]) * a.scale,
+                                       __uint_as_float(xk[e + 1]) * a.scale, __uint_as_float(xk[e + 2]) * a.scale,
+                                       __uint_as_float(xk[e + 3]) * a.scale);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&s.t_free);
+            mbar_arrive(&s.meta_empty[ms]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+}
+
+// delta[b,i,h] = dO . O (one warp per row)
+template <int D>
+__global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16* __restrict__ dout, const float* __restrict__ out,
+                                                   float* __restrict__ delta, long long rows) {
+    const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (w >= rows) return;
+    constexpr int kPer = D / 32;
+    float acc = 0.f;
+    const __nv_bfloat16* g = dout + w * D + lane * kPer;
+    const float* o = out + w * D + lane * kPer;
+#pragma unroll
+    for (int x = 0; x < kPer; ++x) acc = fmaf(__bfloat162float(g[x]), o[x], acc);
+#pragma unroll
+    for (int s = 16; s; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+    if (lane == 0) delta[w] = acc;
+}
+
+template <int D, int BK, int G>
+cudaError_t launch_bwd(const BwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+                       const CUtensorMap& tv, int num_sms, cudaStream_t st) {
+    const size_t smem = sizeof(BwdSmem<D, kRows / G>) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(k_attn_bwd<D, BK, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    ProfScope ps("attn_bwd", st);
+    k_attn_bwd<D, BK, G><<<num_sms, kThreads, smem, st>>>(tq, tdo, tk, tv, a);
+    return cudaGetLastError();
+}
+
+template <int D, int G>
+cudaError_t launch_bwd_bk(const BwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+                          const CUtensorMap& tv, int num_sms, cudaStream_t st) {
+    switch (a.block_k) {
+        case 128: return launch_bwd<D, 128, G>(a, tq, tdo, tk, tv, num_sms, st);
+        case 64: return launch_bwd<D, 64, G>(a, tq, tdo, tk, tv, num_sms, st);
+        case 32: return launch_bwd<D, 32, G>(a, tq, tdo, tk, tv, num_sms, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+bool bwd_supported(int d, int G) { return (d == 64 || d == 128) && (G == 8 || G == 16 || G == 32); }
+
+cudaError_t run_attn_bwd(const BwdArgs& a, const void* q, const void* k, const void* v, const void* dout,
+                         const float* out, int num_sms, cudaStream_t st) {
+    const int G = a.H_q / a.H_kv;
+    const size_t nq = (size_t)a.B * a.N * a.H_q * a.d, nkv = (size_t)a.B * a.N * a.H_kv * a.d;
+    cudaError_t e = cudaMemsetAsync(a.dq, 0, nq * 4, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(a.dk, 0, nkv * 4, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(a.dv, 0, nkv * 4, st);
+    if (e != cudaSuccess) return e;
+    const long long rows = (long long)a.B * a.N * a.H_q;
+    {
+        ProfScope ps("bwd_delta", st);
+        const unsigned grid = (unsigned)((rows * 32 + 255) / 256);
+        if (a.d == 128)
+            k_bwd_delta<128><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(dout), out, a.delta, rows);
+        else
+            k_bwd_delta<64><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(dout), out, a.delta, rows);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    CUtensorMap tq, tdo, tk, tv;
+    const uint64_t dims[4] = {(uint64_t)a.d, (uint64_t)a.H_kv, (uint64_t)a.N, (uint64_t)a.B};
+    const uint64_t strides[3] = {(uint64_t)a.d * 2, (uint64_t)a.H_kv * a.d * 2, (uint64_t)a.N * a.H_kv * a.d * 2};
+    const uint32_t box[4] = {64, 1, (uint32_t)a.block_k, 1};
+    if (!make_tmap_4d(&tk, k, dims, strides, box, 128) || !make_tmap_4d(&tv, v, dims, strides, box, 128) ||
+        !make_tmap_qrows(&tq, q, a.B, a.N, a.H_q, a.d, G) || !make_tmap_qrows(&tdo, dout, a.B, a.N, a.H_q, a.d, G))
+        return cudaErrorInvalidValue;
+    if (a.d == 128) {
+        if (G == 16) return launch_bwd_bk<128, 16>(a, tq, tdo, tk, tv, num_sms, st);
+        if (G == 8) return launch_bwd_bk<128, 8>(a, tq, tdo, tk, tv, num_sms, st);
+        if (G == 32) return launch_bwd_bk<128, 32>(a, tq, tdo, tk, tv, num_sms, st);
+    } else {
+        if (G == 16) return launch_bwd_bk<64, 16>(a, tq, tdo, tk, tv, num_sms, st);
+        if (G == 8) return launch_bwd_bk<64, 8>(a, tq, tdo, tk, tv, num_sms, st);
+        if (G == 32) return launch_bwd_bk<64, 32>(a, tq, tdo, tk, tv, num_sms, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace msa

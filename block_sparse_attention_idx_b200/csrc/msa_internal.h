@@ -90,6 +90,22 @@ size_t attn_ws_bytes(int B, int N, int H_q, int H_kv, int d, int block_k, int to
 void attn_carve(AttnArgs* a, void* base);
 cudaError_t run_attn(const AttnArgs& a, const void* q, const void* k, const void* v, int num_sms, cudaStream_t st);
 
+// ---------------------------------------------------------------- attention backward (msa_bwd.cu)
+struct BwdArgs {
+    int B, N, H_q, H_kv, d, block_k, topk;
+    float scale;
+    Csr csr;            // lists of the forward, items of 128/G queries
+    const float* lse;   // [B, N, H_q] natural-log LSE of the forward
+    float* delta;       // [B, N, H_q] dO . O (workspace)
+    float* dq;          // [B, N, H_q, d]
+    float* dk;          // [B, N, H_kv, d]
+    float* dv;          // [B, N, H_kv, d]
+    DevStatus* status;
+};
+bool bwd_supported(int d, int G);
+cudaError_t run_attn_bwd(const BwdArgs& a, const void* q, const void* k, const void* v, const void* dout,
+                         const float* out, int num_sms, cudaStream_t st);
+
 // ---------------------------------------------------------------- KL alignment (msa_kl.cu)
 struct KlArgs {
     int B, N, H_q, H_kv, d, d_idx, block_k, topk;

@@ -6,6 +6,7 @@
  *   S_t = R_theta(q_t, K_{:t}),   o_t = A_phi(q_t, K_{S_t}, V_{S_t})
  * ("2.4 · 训练原生稀疏", eq (3)). msa_index_topk is R_theta for MSA, msa_sparse_attn_fwd is A_phi,
  * msa_kl_fwd_grad is the KL alignment of the index branch to the main branch, and
+ * msa_sparse_attn_bwd is A_phi's backward with the selection held fixed,
  * msa_sparse_attn_decode runs R_theta then A_phi for one new token per sequence, and
  * msa_sparse_attn_decode_fp8idx does the same from an e4m3 copy of the index keys.
  *
@@ -26,7 +27,8 @@
  *   kernel skips the offending work, sets a flag in the status word and returns; read it with
  *   msa_get_device_status.
  * - Deterministic: the same inputs give bit-identical `blocks`, attention outputs, LSEs and KL
- *   loss. dK_idx is accumulated with float32 atomics and may differ in the last bits.
+ *   loss. dK_idx and the attention gradients are accumulated with float32 atomics and may differ
+ *   in the last bits.
  *
  * Supported sizes (MSA_ERR_UNSUPPORTED otherwise): d in {64, 128}, d_idx in {32, 64},
  * block_k in {32, 64, 128}, 1 <= topk <= 16, H_q % H_kv == 0 with G = H_q/H_kv in {1,2,4,8,16,32},
@@ -75,7 +77,14 @@ typedef struct {
     float scale, scale_idx;
 } msa_dims;
 
-enum { MSA_OP_INDEX_TOPK = 0, MSA_OP_INDEX_TOPK_LSE = 1, MSA_OP_ATTN_FWD = 2, MSA_OP_DECODE = 3, MSA_OP_KL = 4 };
+enum {
+    MSA_OP_INDEX_TOPK = 0,
+    MSA_OP_INDEX_TOPK_LSE = 1,
+    MSA_OP_ATTN_FWD = 2,
+    MSA_OP_DECODE = 3,
+    MSA_OP_KL = 4,
+    MSA_OP_ATTN_BWD = 5
+};
 
 /* Workspace bytes `op` needs for `dims` (for MSA_OP_DECODE, dims->N is the cache capacity). */
 MSA_API msa_status msa_workspace_size(int op, const msa_dims *dims, size_t *bytes);
@@ -113,6 +122,29 @@ MSA_API msa_status msa_index_topk(const msa_dims *dims, const void *q_idx, const
 MSA_API msa_status msa_sparse_attn_fwd(const msa_dims *dims, const void *q, const void *k, const void *v,
                                const int32_t *blocks, float *out, float *lse, void *ws, size_t ws_bytes,
                                msa_stream_t stream);
+
+/*
+ * Backward of msa_sparse_attn_fwd with the selection held fixed ("2.4 · 训练原生稀疏", section 2.2,
+ * eq (11): on a fixed set the selected attention is ordinary attention, and positions outside the
+ * set get no gradient). With J, o and LSE as in the forward and g = dout[b,i,h]:
+ *   P_j = exp(q.k_j * scale - LSE),   dS_j = P_j * (g.v_j - g.o)        (j in J)
+ *   dq[b,i,h]   = scale * sum_j dS_j k_j
+ *   dk[b,j,r]   = scale * sum over (i, h in group r) with j in J of dS_j q[b,i,h]
+ *   dv[b,j,r]   = sum over the same (i, h) of P_j g
+ * The computation stays on the selected (query, block) pairs: no dense score matrix.
+ *   q, k, v, blocks  as for msa_sparse_attn_fwd
+ *   out    fp32 [B, N, H_q, d]   the forward's output (used for g.o)
+ *   lse    fp32 [B, N, H_q]      the forward's LSE
+ *   dout   bf16 [B, N, H_q, d]   upstream gradient
+ *   dq fp32 [B, N, H_q, d]; dk, dv fp32 [B, N, H_kv, d]              (outputs)
+ * P and dS enter the tensor cores as bf16 (as the forward's P does); the products accumulate in
+ * fp32. dq, dk and dv are accumulated with fp32 reductions (atomics) and may differ in the last bits
+ * between runs. Supports G = H_q / H_kv in {8, 16, 32} (MSA_ERR_UNSUPPORTED otherwise).
+ */
+MSA_API msa_status msa_sparse_attn_bwd(const msa_dims *dims, const void *q, const void *k, const void *v,
+                                       const int32_t *blocks, const float *out, const float *lse, const void *dout,
+                                       float *dq, float *dk, float *dv, void *ws, size_t ws_bytes,
+                                       msa_stream_t stream);
 
 /*
  * One decode step per sequence: index Top-k then sparse attention for the newest token, whose K, V
