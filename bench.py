@@ -511,11 +511,18 @@ def bench_train(args, world, rank, msa, pk):
     ws_i = msa.workspace(msa.MSA_OP_INDEX_TOPK_LSE, dims, dev)
     ws_a = msa.workspace(msa.MSA_OP_ATTN_FWD, dims, dev)
     ws_k = msa.workspace(msa.MSA_OP_KL, dims, dev)
+    ws_b = msa.workspace(msa.MSA_OP_ATTN_BWD, dims, dev)
     flush = torch.zeros(256 << 20, dtype=torch.uint8, device=dev)
+    # upstream gradient of the layer output: synthetic N(0,1), drawn once
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(rank_seed(w, rank) + 17)
+    dout = torch.randn(w.B, N, w.H_q, w.d, generator=gen, device=dev).to(torch.bfloat16)
 
     def step():
+        # index branch (selection, LSE_idx), main forward, main backward, KL of the index branch
         blocks, lse_idx = msa.msa_index_topk(dims, x["q_idx"], x["k_idx"], want_lse=True, ws=ws_i)
         out, lse = msa.msa_sparse_attn_fwd(dims, x["q"], x["k"], x["v"], blocks, ws=ws_a)
+        gq, gk, gv = msa.msa_sparse_attn_bwd(dims, x["q"], x["k"], x["v"], blocks, out, lse, dout, ws=ws_b)
         loss, dq, dk = msa.msa_kl_fwd_grad(dims, x["q"], x["k"], x["q_idx"], x["k_idx"], blocks, lse, lse_idx,
                                            ws=ws_k)
         return blocks, loss
@@ -526,6 +533,7 @@ def bench_train(args, world, rank, msa, pk):
     sel_tok = selected_tokens(blocks, w.block_k)
     G = w.H_q // w.H_kv
     kl_flops = (2.0 * w.d * G + 6.0 * w.d_idx) * sel_tok
+    bwd_flops = 10.0 * w.d * G * sel_tok  # S, dP, dV, dK, dQ: 2 d FLOPs each per selected (head, token) pair
     msa.msa_profile_read()
     msa.msa_profile_enable(True)
     t = timed_steps(step, args.train_steps, flush)
@@ -533,13 +541,17 @@ def bench_train(args, world, rank, msa, pk):
     prof = profile_avg(msa.msa_profile_read())
     ms = max_over_ranks(sum(t) / len(t), world)
     kl_ms = prof["kl_kv_outer"]["avg_ms"]
+    bwd_ms = prof["attn_bwd"]["avg_ms"]
     res = {"workload": "train_64k" if N == w.N else f"train_{N}", "ms_per_step": ms, "loss": float(loss.item()),
            "roofline": {**roofline_entry("tensor", kl_flops / (kl_ms * 1e-3) / 1e12, pk["bf16_tflops"], "TFLOP/s",
                                          measured_traffic("kl_kv_outer", sel_tok)),
                         "kernel": "kl_kv_outer", "flops_per_launch": kl_flops},
-           "work": {"selected_tokens": sel_tok, "kl_flops": kl_flops},
+           "roofline_attn_bwd": {**roofline_entry("tensor", bwd_flops / (bwd_ms * 1e-3) / 1e12, pk["bf16_tflops"],
+                                                  "TFLOP/s", measured_traffic("attn_bwd", sel_tok)),
+                                 "kernel": "attn_bwd", "flops_per_launch": bwd_flops},
+           "work": {"selected_tokens": sel_tok, "kl_flops": kl_flops, "attn_bwd_flops": bwd_flops},
            "kernels": {k: {"avg_ms": round(v["avg_ms"], 4), "launches": v["launches"]} for k, v in prof.items()}}
-    del x, ws_a, ws_k
+    del x, ws_a, ws_k, ws_b, dout
     torch.cuda.empty_cache()
     return res
 

@@ -21,9 +21,9 @@
 // changes (a block's items can be split between two CTAs, hence reductions rather than stores).
 // P and dS enter the tensor cores as bf16, as in the forward's P.
 //
-// Warp roles (192 threads): warps 0-3 epilogue (thread = token lane, or item row for dQ), warp 4
-// loads (item metadata, the Q and dO rows by one 5-D TMA box per query, K and V tiles), warp 5
-// issues the MMAs and owns TMEM.
+// Warp roles (320 threads): warps 0-7 epilogue (warp w: TMEM lane quarter w % 4, i.e. 32 tokens,
+// or 32 item rows for dQ; column half w / 4), warp 8 loads (item metadata, the Q and dO rows by one
+// 5-D TMA box per query, K and V tiles), warp 9 issues the MMAs and owns TMEM.
 #include "msa_common.cuh"
 #include "msa_internal.h"
 
@@ -33,8 +33,10 @@ namespace {
 
 constexpr int kRows = 128;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kProdWarp = 4, kMmaWarp = 5;
-constexpr int kThreads = 6 * 32;
+constexpr int kEpiWarps = 8;  // two per TMEM lane quarter: item rows (S^T columns) split in halves
+constexpr int kEpi = kEpiWarps * 32;
+constexpr int kProdWarp = 8, kMmaWarp = 9;
+constexpr int kThreads = 10 * 32;
 
 __device__ __forceinline__ void red_add_v4(float* p, float x, float y, float z, float w) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(x), "f"(y), "f"(z), "f"(w)
@@ -57,6 +59,7 @@ struct BwdSmem {
     alignas(1024) uint8_t v[kRows * D * 2];     // V tile, same
     alignas(1024) uint8_t ds[kRows * kRows * 2];  // dS^T: 2 sub-tiles of [128 token rows x 64 item rows]
     BwdMeta<QPC> meta[2];
+    alignas(16) float xbuf[kEpiWarps][32][36];  // per epilogue warp: 32 rows x 32 columns in transit to global
     uint64_t meta_full[2], meta_empty[2], q_full, q_empty, kv_full, kv_empty, s_full, p_full, d_full, t_free, drain;
     uint32_t tmem_base;
     int abort;
@@ -85,16 +88,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int x = 0; x < 2; ++x) {
             mbar_init(&s.meta_full[x], 32);
-            mbar_init(&s.meta_empty[x], kRows + 1);  // the epilogue threads and the MMA issuer
+            mbar_init(&s.meta_empty[x], kEpi + 1);  // the epilogue threads and the MMA issuer
         }
         mbar_init(&s.q_full, 1);
         mbar_init(&s.q_empty, 1);
         mbar_init(&s.kv_full, 1);
         mbar_init(&s.kv_empty, 1);
         mbar_init(&s.s_full, 1);
-        mbar_init(&s.p_full, kRows);
+        mbar_init(&s.p_full, kEpi);
         mbar_init(&s.d_full, 1);
-        mbar_init(&s.t_free, kRows);
+        mbar_init(&s.t_free, kEpi);
         mbar_init(&s.drain, 1);
         s.abort = 0;
         fence_mbar_init();
@@ -264,8 +267,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------------------ epilogue
-        const int tt = warp * 32 + lane;  // token lane for S^T / dP^T / dV / dK, item row for dQ
-        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+        const int wq = warp & 3, hf = warp >> 2;
+        const int tt = wq * 32 + lane;  // token lane for S^T / dP^T / dV / dK, item row for dQ
+        const uint32_t lane_addr = tmem + ((uint32_t)(wq * 32) << 16);
         const float sl2 = a.scale * kLog2e;
         for (int t = t0, n = 0; t < t1; ++t, ++n) {
             const int ms = n & 1;
@@ -283,38 +287,60 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-#pragma unroll 1
-            for (int cc = 0; cc < kRows / 32; ++cc) {
+            // Each warp forms P and dS of its two 32-row chunks in registers first: P / dS are stored
+            // packed over columns that the other warp half of the lane quarter may not have read yet
+            // (chunk cc goes to columns 16cc..16cc+15), so the stores wait for a barrier of the
+            // epilogue warps.
+            uint32_t pk[2][16], dk[2][16];
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+                const int cc = 2 * hf + k2;
                 uint32_t sv[32], pv[32];
                 tmem_ld32(lane_addr + kColS + 32 * cc, sv);
                 tmem_ld32(lane_addr + kColP + 32 * cc, pv);
+                // rows 32cc..32cc+31 hold 32 / G queries (or part of one): is each query's block token
+                // causal for this thread?
+                bool cz[(32 + G - 1) / G];
+#pragma unroll
+                for (int u = 0; u < (32 + G - 1) / G; ++u) {
+                    const int row0 = 32 * cc + u * G;
+                    cz[u] = row0 < nrows && tt < BK && tok <= mt.qi[row0 / G];
+                }
                 tmem_ld_wait();
                 reg_fence(sv);
                 reg_fence(pv);
-                uint32_t pk[16], dk[16];
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float p2[2], d2[2];
+                for (int e = 0; e < 32; e += 4) {
+                    const float4 l4 = *reinterpret_cast<const float4*>(&mt.lse2[32 * cc + e]);
+                    const float4 d4 = *reinterpret_cast<const float4*>(&mt.delta[32 * cc + e]);
+                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+                    float p4[4], g4[4];
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int row = 32 * cc + e + u;
-                        const bool valid = row < nrows && tt < BK && tok <= mt.qi[row / G];
-                        const float p = valid ? exp2f(fmaf(__uint_as_float(sv[e + u]), sl2, -mt.lse2[row])) : 0.f;
-                        p2[u] = p;
-                        d2[u] = valid ? p * (__uint_as_float(pv[e + u]) - mt.delta[row]) : 0.f;
+                    for (int u = 0; u < 4; ++u) {
+                        const bool valid = cz[(e + u) / G];
+                        const float p = fast_exp2(fmaf(__uint_as_float(sv[e + u]), sl2, -lv[u]));
+                        p4[u] = valid ? p : 0.f;
+                        g4[u] = valid ? p * (__uint_as_float(pv[e + u]) - dv[u]) : 0.f;
                     }
-                    pk[e / 2] = pack_bf16x2(p2[0], p2[1]);
-                    dk[e / 2] = pack_bf16x2(d2[0], d2[1]);
+                    pk[k2][e / 2] = pack_bf16x2(p4[0], p4[1]);
+                    pk[k2][e / 2 + 1] = pack_bf16x2(p4[2], p4[3]);
+                    dk[k2][e / 2] = pack_bf16x2(g4[0], g4[1]);
+                    dk[k2][e / 2 + 1] = pack_bf16x2(g4[2], g4[3]);
                 }
-                tmem_st16(lane_addr + kColS + 16 * cc, pk);
-                tmem_st16(lane_addr + kColP + 16 * cc, dk);
+            }
+            bar_sync_named(1, kEpi);  // every epilogue warp has read its S^T / dP^T columns
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+                const int cc = 2 * hf + k2;
+                tmem_st16(lane_addr + kColS + 16 * cc, pk[k2]);
+                tmem_st16(lane_addr + kColP + 16 * cc, dk[k2]);
                 // dS^T row of this token: item rows 32cc..32cc+31, four 16-byte chunks of 8 rows
                 uint8_t* dsrow = s.ds + (cc >> 1) * (kRows * 128);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const uint32_t ch = 4 * (cc & 1) + j;
                     *reinterpret_cast<uint4*>(dsrow + swz(tt, ch * 16, 128)) =
-                        make_uint4(dk[4 * j], dk[4 * j + 1], dk[4 * j + 2], dk[4 * j + 3]);
+                        make_uint4(dk[k2][4 * j], dk[k2][4 * j + 1], dk[k2][4 * j + 2], dk[k2][4 * j + 3]);
                 }
             }
             tmem_st_wait();
@@ -326,52 +352,58 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            // dQ row tt of the item (TMEM lane = item row)
-            {
+            // The reductions leave TMEM a lane (row) per thread; each 32 x 32 chunk goes through the
+            // warp's shared buffer so that one warp instruction adds 8 consecutive float4s to each of
+            // 4 rows (4 cache lines) instead of one float4 to each of 32 rows.
+            float(*xb)[36] = s.xbuf[warp];
+            auto red_chunk = [&](const uint32_t (&x)[32], float* row, float mul) {
+#pragma unroll
+                for (int e = 0; e < 32; e += 4)
+                    *reinterpret_cast<float4*>(&xb[lane][e]) =
+                        make_float4(__uint_as_float(x[e]) * mul, __uint_as_float(x[e + 1]) * mul,
+                                    __uint_as_float(x[e + 2]) * mul, __uint_as_float(x[e + 3]) * mul);
+                __syncwarp();
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int rr = 4 * j + (lane >> 3), c4 = 4 * (lane & 7);
+                    float* p = reinterpret_cast<float*>(
+                        __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(row), rr));
+                    if (p) {
+                        const float4 v4 = *reinterpret_cast<const float4*>(&xb[rr][c4]);
+                        red_add_v4(p + c4, v4.x, v4.y, v4.z, v4.w);
+                    }
+                }
+                __syncwarp();
+            };
+            // dQ row tt of the item (TMEM lane = item row); warp half hf takes dQ columns 64hf..
+            if (hf < D / 64) {
                 const bool rv = tt < nrows;
                 const int m = rv ? tt / G : 0, h = tt % G;
-                float* dst = a.dq + (((size_t)b * a.N + mt.qi[m]) * a.H_q + (size_t)r * G + h) * D;
+                float* dst = rv ? a.dq + (((size_t)b * a.N + mt.qi[m]) * a.H_q + (size_t)r * G + h) * D : nullptr;
 #pragma unroll
-                for (int hh = 0; hh < D / 64; ++hh) {
-#pragma unroll
-                    for (int q2 = 0; q2 < 2; ++q2) {
-                        uint32_t x[32];
-                        tmem_ld32(lane_addr + (hh == 0 ? 64u : 192u) + 32 * q2, x);
-                        tmem_ld_wait();
-                        reg_fence(x);
-                        if (rv) {
-#pragma unroll
-                            for (int e = 0; e < 32; e += 4)
-                                red_add_v4(dst + 64 * hh + 32 * q2 + e, __uint_as_float(x[e]) * a.scale,
-                                           __uint_as_float(x[e + 1]) * a.scale, __uint_as_float(x[e + 2]) * a.scale,
-                                           __uint_as_float(x[e + 3]) * a.scale);
-                        }
-                    }
+                for (int q2 = 0; q2 < 2; ++q2) {
+                    uint32_t x[32];
+                    tmem_ld32(lane_addr + (hf == 0 ? 64u : 192u) + 32 * q2, x);
+                    tmem_ld_wait();
+                    reg_fence(x);
+                    red_chunk(x, dst ? dst + 64 * hf + 32 * q2 : nullptr, a.scale);
                 }
             }
             // the block's dV and dK when its last item of this CTA is done (TMEM lane = token)
             if (flush) {
                 const bool tv = tt < BK && tok < a.N;
-                float* dvp = a.dv + (((size_t)b * a.N + (tv ? tok : 0)) * a.H_kv + r) * D;
-                float* dkp = a.dk + (((size_t)b * a.N + (tv ? tok : 0)) * a.H_kv + r) * D;
+                float* dvp = tv ? a.dv + (((size_t)b * a.N + tok) * a.H_kv + r) * D : nullptr;
+                float* dkp = tv ? a.dk + (((size_t)b * a.N + tok) * a.H_kv + r) * D : nullptr;
 #pragma unroll
-                for (int q2 = 0; q2 < D / 32; ++q2) {
+                for (int q2 = hf * (D / 64); q2 < (hf + 1) * (D / 64); ++q2) {
                     uint32_t xv[32], xk[32];
                     tmem_ld32(lane_addr + kColDV + 32 * q2, xv);
                     tmem_ld32(lane_addr + kColDK + 32 * q2, xk);
                     tmem_ld_wait();
                     reg_fence(xv);
                     reg_fence(xk);
-                    if (tv) {
-#pragma unroll
-                        for (int e = 0; e < 32; e += 4) {
-                            red_add_v4(dvp + 32 * q2 + e, __uint_as_float(xv[e]), __uint_as_float(xv[e + 1]),
-                                       __uint_as_float(xv[e + 2]), __uint_as_float(xv[e + 3]));
-                            red_add_v4(dkp + 32 * q2 + e, __uint_as_float(xk[e]) * a.scale,
-                                       __uint_as_float(xk[e + 1]) * a.scale, __uint_as_float(xk[e + 2]) * a.scale,
-                                       __uint_as_float(xk[e + 3]) * a.scale);
-                        }
-                    }
+                    red_chunk(xv, dvp ? dvp + 32 * q2 : nullptr, 1.f);
+                    red_chunk(xk, dkp ? dkp + 32 * q2 : nullptr, a.scale);
                 }
             }
             tc_fence_before();
