@@ -53,14 +53,13 @@ struct BwdMeta {
 
 template <int D, int QPC>
 struct BwdSmem {
-    alignas(1024) uint8_t q[kRows * D * 2];     // Q rows: 8-row x 64-column 128B-swizzled atoms [row/8][D/64]
-    alignas(1024) uint8_t dout[kRows * D * 2];  // dO rows, same layout
+    alignas(1024) uint8_t q[2][kRows * D * 2];     // Q rows: 8-row x 64-column 128B-swizzled atoms [row/8][D/64]
+    alignas(1024) uint8_t dout[2][kRows * D * 2];  // dO rows, same layout
     alignas(1024) uint8_t k[kRows * D * 2];     // K tile: D/64 sub-tiles of [128 token rows x 128 B], rows >= BK zero
     alignas(1024) uint8_t v[kRows * D * 2];     // V tile, same
     alignas(1024) uint8_t ds[kRows * kRows * 2];  // dS^T: 2 sub-tiles of [128 token rows x 64 item rows]
-    BwdMeta<QPC> meta[2];
-    alignas(16) float xbuf[kEpiWarps][32][36];  // per epilogue warp: 32 rows x 32 columns in transit to global
-    uint64_t meta_full[2], meta_empty[2], q_full, q_empty, kv_full, kv_empty, s_full, p_full, d_full, t_free, drain;
+    BwdMeta<QPC> meta;
+    uint64_t meta_full, meta_empty, q_full[2], q_empty[2], kv_full, kv_empty, s_full, p_full, d_full, t_free, drain;
     uint32_t tmem_base;
     int abort;
 };
@@ -86,12 +85,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = warp_id(), lane = lane_id();
 
     if (threadIdx.x == 0) {
+        mbar_init(&s.meta_full, 32);
+        mbar_init(&s.meta_empty, kEpi + 1);  // the epilogue threads and the MMA issuer
         for (int x = 0; x < 2; ++x) {
-            mbar_init(&s.meta_full[x], 32);
-            mbar_init(&s.meta_empty[x], kEpi + 1);  // the epilogue threads and the MMA issuer
+            mbar_init(&s.q_full[x], 1);
+            mbar_init(&s.q_empty[x], 1);
         }
-        mbar_init(&s.q_full, 1);
-        mbar_init(&s.q_empty, 1);
         mbar_init(&s.kv_full, 1);
         mbar_init(&s.kv_empty, 1);
         mbar_init(&s.s_full, 1);
@@ -106,7 +105,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // K / V rows past block_k are multiplied by zeros, and start as zeros
     {
         uint4* z = reinterpret_cast<uint4*>(s.q);
-        for (int x = threadIdx.x; x < 4 * kRows * D * 2 / 16; x += kThreads) z[x] = make_uint4(0u, 0u, 0u, 0u);
+        for (int x = threadIdx.x; x < 6 * kRows * D * 2 / 16; x += kThreads) z[x] = make_uint4(0u, 0u, 0u, 0u);
     }
     fence_proxy_async();
     if (warp == kMmaWarp) {
@@ -120,10 +119,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == kProdWarp) {
         // ------------------------------------------------------------------------ loads
-        // Item n's metadata goes to meta[n % 2] (plain loads into registers, stored once they have
-        // arrived, then one arrival per lane: no load is in flight at these release arrives), its Q
-        // and dO rows into the single Q / dO buffers once the MMA has released them, and K / V on
-        // a new block once the MMA has released the previous block.
+        // Item n: its Q and dO rows into buffer n % 2 once the MMA has released it (item n-2), then
+        // its metadata (plain loads into registers, stored once the epilogue is done with item n-1,
+        // then one arrival per lane: no load is in flight at these release arrives), then K / V of a
+        // new block once the MMA has released the previous block. Loads thus run one item ahead.
         bool ok = true;
         int kv_loads = 0, prevL = -1, issued = 0;
         int4 rec = t0 < t1 ? cs.items[t0] : make_int4(-1, 0, 0, 0);
@@ -143,11 +142,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 l2[x] = m < count ? a.lse[o] * kLog2e : 0.f;
                 dl[x] = m < count ? a.delta[o] : 0.f;
             }
-            const int ms = n & 1;
+            const int qb = n & 1;
             int okl = 1;
-            if (lane == 0) okl = mbar_wait(&s.meta_empty[ms], ((n >> 1) & 1) ^ 1, a.status, 0xa01);
+            // Q and dO rows of the item queries
+            if (lane == 0) okl = mbar_wait(&s.q_empty[qb], ((n >> 1) & 1) ^ 1, a.status, 0xa02);
             if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
-            BwdMeta<QPC>& mt = s.meta[ms];
+            if (lane == 0) mbar_arrive_expect_tx_relaxed(&s.q_full[qb], (uint32_t)(2 * count * G * D * 2));
+            __syncwarp();
+            if (lane < count) {
+                tma_load_5d(s.q[qb] + lane * G * D * 2, &tm_q, &s.q_full[qb], 0, 0, 0, r * G / 8, b * a.N + qi);
+                tma_load_5d(s.dout[qb] + lane * G * D * 2, &tm_do, &s.q_full[qb], 0, 0, 0, r * G / 8, b * a.N + qi);
+            }
+            if (lane == 0) okl = mbar_wait(&s.meta_empty, (n & 1) ^ 1, a.status, 0xa01);
+            if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
+            BwdMeta<QPC>& mt = s.meta;
             if (lane == 0) {
                 mt.L = L;
                 mt.count = count;
@@ -159,16 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mt.lse2[lane + 32 * x] = l2[x];
                 mt.delta[lane + 32 * x] = dl[x];
             }
-            mbar_arrive(&s.meta_full[ms]);
-            // Q and dO rows of the item queries
-            if (lane == 0) okl = mbar_wait(&s.q_empty, (n & 1) ^ 1, a.status, 0xa02);
-            if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
-            if (lane == 0) mbar_arrive_expect_tx_relaxed(&s.q_full, (uint32_t)(2 * count * G * D * 2));
-            __syncwarp();
-            if (lane < count) {
-                tma_load_5d(s.q + lane * G * D * 2, &tm_q, &s.q_full, 0, 0, 0, r * G / 8, b * a.N + qi);
-                tma_load_5d(s.dout + lane * G * D * 2, &tm_do, &s.q_full, 0, 0, 0, r * G / 8, b * a.N + qi);
-            }
+            mbar_arrive(&s.meta_full);
             // K and V of a new block
             if (L != prevL) {
                 if (lane == 0) {
@@ -192,7 +191,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) s.abort = 1;
         // nothing may still be landing in shared memory when the CTA exits
         if (lane == 0) {
-            if (issued > 0) mbar_wait(&s.q_full, (issued - 1) & 1, a.status, 0xa04);
+            for (int x = 0; x < 2 && x < issued; ++x) {
+                const int nl = issued - 1 - x;  // last use of buffer nl & 1
+                mbar_wait(&s.q_full[nl & 1], (nl >> 1) & 1, a.status, 0xa04);
+            }
             if (kv_loads > 0) mbar_wait(&s.kv_full, (kv_loads - 1) & 1, a.status, 0xa05);
         }
     } else if (warp == kMmaWarp) {
@@ -200,13 +202,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             bool ok = true;
             int kv_group = -1, prevL = -1;
-            const uint32_t qa = smem_u32(s.q), da = smem_u32(s.dout), ka = smem_u32(s.k), va = smem_u32(s.v),
-                           dsa = smem_u32(s.ds);
+            const uint32_t ka = smem_u32(s.k), va = smem_u32(s.v), dsa = smem_u32(s.ds);
             for (int t = t0, n = 0; t < t1; ++t, ++n) {
-                const int ms = n & 1;
-                if (!mbar_wait(&s.meta_full[ms], (n >> 1) & 1, a.status, 0xa11)) { ok = false; break; }
-                const int L = s.meta[ms].L;
-                mbar_arrive(&s.meta_empty[ms]);
+                const int qb = n & 1;
+                const uint32_t qa = smem_u32(s.q[qb]), da = smem_u32(s.dout[qb]);
+                if (!mbar_wait(&s.meta_full, n & 1, a.status, 0xa11)) { ok = false; break; }
+                const int L = s.meta.L;
+                mbar_arrive(&s.meta_empty);
                 bool first = false;
                 if (L != prevL) {
                     if (kv_group >= 0) umma_commit(&s.kv_empty);  // the previous block's tiles are no longer read
@@ -215,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     first = true;
                     if (!mbar_wait(&s.kv_full, kv_group & 1, a.status, 0xa12)) { ok = false; break; }
                 }
-                if (!mbar_wait(&s.q_full, n & 1, a.status, 0xa13)) { ok = false; break; }
+                if (!mbar_wait(&s.q_full[qb], (n >> 1) & 1, a.status, 0xa13)) { ok = false; break; }
                 if (n > 0 && !mbar_wait(&s.t_free, (n - 1) & 1, a.status, 0xa14)) { ok = false; break; }
                 tc_fence_after();
                 // S^T = K . Q^T and dP^T = V . dO^T (both operands K-major)
@@ -259,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 umma_commit(&s.d_full);
-                umma_commit(&s.q_empty);
+                umma_commit(&s.q_empty[qb]);
             }
             if (!ok) s.abort = 1;
             umma_commit(&s.drain);
@@ -272,12 +274,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_addr = tmem + ((uint32_t)(wq * 32) << 16);
         const float sl2 = a.scale * kLog2e;
         for (int t = t0, n = 0; t < t1; ++t, ++n) {
-            const int ms = n & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&s.meta_full[ms], (n >> 1) & 1, a.status, 0xa21))) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.meta_full, n & 1, a.status, 0xa21))) {
                 s.abort = 1;
                 break;
             }
-            const BwdMeta<QPC>& mt = s.meta[ms];
+            const BwdMeta<QPC>& mt = s.meta;
             const int L = mt.L, count = mt.count, flush = mt.flush;
             const int c = L % cs.nb, r = (L / cs.nb) % a.H_kv, b = L / (cs.nb * a.H_kv);
             const int tok = c * BK + tt;
@@ -352,26 +353,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            // The reductions leave TMEM a lane (row) per thread; each 32 x 32 chunk goes through the
-            // warp's shared buffer so that one warp instruction adds 8 consecutive float4s to each of
-            // 4 rows (4 cache lines) instead of one float4 to each of 32 rows.
-            float(*xb)[36] = s.xbuf[warp];
+            // The reductions leave TMEM a lane (row) per thread. Each 32 x 32 chunk goes through a
+            // per-warp 4 KB buffer in the dS^T tile (free here: the dQ MMA that read it is complete,
+            // and the next item's dS^T is written only after this item releases TMEM), so that one
+            // warp instruction adds 8 consecutive float4s to each of 4 rows instead of one float4 to
+            // each of 32 rows. Float4 columns are XOR-swizzled by row against bank conflicts.
+            float4* xb = reinterpret_cast<float4*>(s.ds) + warp * 32 * 8;  // [32 rows][8 float4]
             auto red_chunk = [&](const uint32_t (&x)[32], float* row, float mul) {
 #pragma unroll
-                for (int e = 0; e < 32; e += 4)
-                    *reinterpret_cast<float4*>(&xb[lane][e]) =
-                        make_float4(__uint_as_float(x[e]) * mul, __uint_as_float(x[e + 1]) * mul,
-                                    __uint_as_float(x[e + 2]) * mul, __uint_as_float(x[e + 3]) * mul);
+                for (int e = 0; e < 8; ++e)
+                    xb[lane * 8 + (e ^ (lane & 7))] =
+                        make_float4(__uint_as_float(x[4 * e]) * mul, __uint_as_float(x[4 * e + 1]) * mul,
+                                    __uint_as_float(x[4 * e + 2]) * mul, __uint_as_float(x[4 * e + 3]) * mul);
                 __syncwarp();
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    const int rr = 4 * j + (lane >> 3), c4 = 4 * (lane & 7);
+                    const int rr = 4 * j + (lane >> 3), c4 = lane & 7;
                     float* p = reinterpret_cast<float*>(
                         __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(row), rr));
-                    if (p) {
-                        const float4 v4 = *reinterpret_cast<const float4*>(&xb[rr][c4]);
-                        red_add_v4(p + c4, v4.x, v4.y, v4.z, v4.w);
-                    }
+                    const float4 v4 = xb[rr * 8 + (c4 ^ (rr & 7))];
+                    if (p) red_add_v4(p + 4 * c4, v4.x, v4.y, v4.z, v4.w);
                 }
                 __syncwarp();
             };
@@ -408,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_before();
             mbar_arrive(&s.t_free);
-            mbar_arrive(&s.meta_empty[ms]);
+            mbar_arrive(&s.meta_empty);
         }
     }
     tc_fence_before();
