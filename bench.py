@@ -141,6 +141,12 @@ MEASURED_TRAFFIC = {
                     "sha256": "14cb19baa5ea1a26ed617e36066629b07b8a9f99a90d086cb3700db4150cafa5",
                     "bytes_per_unit": (991507200 + 136743680) / 60309504, "unit": "selected token",
                     "capture": "profiles/kl_kv_outer_train_8k.md"},
+    # attention backward at N=8192 (dram read 6,612,550,485 B + write 3,289,236,480 B per launch over
+    # 60,309,504 selected tokens; most of it is the read-modify-write of dQ by the per-item reductions)
+    "attn_bwd": {"file": "block_sparse_attention_idx_b200/csrc/msa_bwd.cu",
+                 "sha256": "a4643c88591d2bddd8e05910abc956258cb6b52d27530488526b1f18be7f5e2e",
+                 "bytes_per_unit": (6612550485 + 3289236480) / 60309504, "unit": "selected token",
+                 "capture": "profiles/attn_bwd_train_8k.md"},
     # decode scans at 16 x 131,072 (read + write per launch over 16 x 130,944 scanned tokens), scaled
     # by the scanned tokens of the timed launch
     "dec_scan": {"file": "block_sparse_attention_idx_b200/csrc/msa_decode.cu",
