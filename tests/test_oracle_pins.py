@@ -542,3 +542,38 @@ def test_bwd_dense_limit_matches_autograd():
     np.testing.assert_allclose(dq, q.grad.numpy(), atol=1e-12)
     np.testing.assert_allclose(dk, k.grad.numpy(), atol=1e-12)
     np.testing.assert_allclose(dv, v.grad.numpy(), atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- sequence-parallel indexer
+def test_sp_eq16_hand_values():
+    """4.1.1 · 监督与联合训练 eq (16) on written-out values: ranks with (a_p, z_p) = (1, 2) and (3, 1)
+    give a = 3, z = 2 e^-2 + 1; a rank with no tokens (-inf, 0) changes nothing."""
+    from oracle import sp
+    got = sp.combine_lse([[1.0, 2.0], [3.0, 1.0], [-np.inf, 0.0]])
+    assert got == pytest.approx(3.0 + math.log(1.0 + 2.0 * math.exp(-2.0)), abs=1e-15)
+    # it equals the log-sum-exp of the union of the ranks' scores
+    s1, s2 = np.array([1.0, 1.0]), np.array([3.0])
+    assert got == pytest.approx(math.log(np.exp(s1).sum() + np.exp(s2).sum()), abs=1e-14)
+
+
+@pytest.mark.parametrize("bounds", [[0, 4, 8], [0, 3, 6, 8], [0, 1, 2, 5, 8], [0, 8]])
+def test_sp_merge_and_lse_equal_single_device(bounds):
+    """Each rank's local Top-k of its block range, merged by (score desc, id asc), plus the local
+    block, is the single-device selection; eq (16) over the ranks' (a_p, z_p) is the single-device
+    LSE_idx (uneven ranges, a ragged last block, ranks without candidates for early rows)."""
+    from oracle import sp
+    N, Bk, k, Hkv = 61, 8, 3, 2
+    dims = oracle.Dims(B=2, N=N, H_q=2 * Hkv, H_kv=Hkv, d=8, d_idx=8, block_k=Bk, topk=k)
+    x = small_prefill(N, 2 * Hkv, Hkv, 8, 8, Bk, k, seed=71, B=2)
+    blocks, _, lse = oracle.index_topk(dims, x["q_idx"], x["k_idx"], want_lse=True)
+    blocks = blocks.reshape(2, N, Hkv, k + 1)
+    cs, ci, ml = [], [], []
+    for p in range(len(bounds) - 1):
+        s_, i_ = sp.local_topk(dims, x["q_idx"], x["k_idx"], bounds[p], bounds[p + 1])
+        cs.append(s_)
+        ci.append(i_)
+    merged = sp.merge(dims, cs, ci)
+    np.testing.assert_array_equal(merged, blocks)
+    for p in range(len(bounds) - 1):
+        ml.append(sp.local_lse(dims, x["q_idx"], x["k_idx"], blocks, bounds[p], bounds[p + 1]))
+    np.testing.assert_allclose(sp.combine_lse(ml), lse.reshape(2, N, Hkv), atol=1e-12)
