@@ -74,6 +74,11 @@ def lib() -> ctypes.CDLL:
         L.msa_quantize_e4m3_rows.argtypes = [P, ctypes.c_int64, ctypes.c_int, P, P, P]
         L.msa_kl_fwd_grad.argtypes = [D, P, P, P, P, P, P, P, ctypes.c_float, P, P, P, P, S, P]
         L.msa_sparse_attn_bwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, S, P]
+        I = ctypes.c_int
+        L.msa_index_topk_local.argtypes = [D, P, P, I, I, P, P, P, S, P]
+        L.msa_topk_merge.argtypes = [D, I, P, P, P, P]
+        L.msa_lse_idx_local.argtypes = [D, P, P, I, I, P, P, P]
+        L.msa_lse_combine.argtypes = [D, I, P, P, P]
         L.msa_sparse_attn_decode_noalloc.argtypes = [D, P, P, P, P, P, P, P, P, P]
         L.msa_sparse_attn_decode_noalloc.restype = ctypes.c_int
         L.msa_get_device_status.argtypes = [P, P]
@@ -87,7 +92,8 @@ def lib() -> ctypes.CDLL:
         L.msa_version.restype = ctypes.c_char_p
         for fn in ("msa_workspace_size", "msa_index_topk", "msa_sparse_attn_fwd", "msa_sparse_attn_decode",
                    "msa_sparse_attn_decode_fp8idx", "msa_quantize_e4m3_rows", "msa_kl_fwd_grad",
-                   "msa_sparse_attn_bwd", "msa_get_device_status"):
+                   "msa_sparse_attn_bwd", "msa_index_topk_local", "msa_topk_merge", "msa_lse_idx_local",
+                   "msa_lse_combine", "msa_get_device_status"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -276,6 +282,59 @@ def msa_sparse_attn_bwd(dims: MsaDims, q, k, v, blocks, out, lse, dout, ws=None,
     return dq, dk, dv
 
 
+def msa_index_topk_local(dims: MsaDims, q_idx, k_idx_local, tok0: int, ws=None, stream=None):
+    """This rank's candidates for the sequence-parallel selection: k_idx_local bf16 [B, ntok, d_idx]
+    holds tokens [tok0, tok0 + ntok). Returns (raw block maxima fp32, block ids int32), each
+    [B, N, H_kv, topk], best first, -inf / -1 padded."""
+    dev = q_idx.device
+    _need(q_idx, "q_idx", (dims.B, dims.N, dims.H_kv, dims.d_idx), torch.bfloat16, dev)
+    ntok = k_idx_local.shape[1]
+    _need(k_idx_local, "k_idx_local", (dims.B, ntok, dims.d_idx), torch.bfloat16, dev)
+    cs = torch.empty(dims.B, dims.N, dims.H_kv, dims.topk, dtype=torch.float32, device=dev)
+    ci = torch.empty(dims.B, dims.N, dims.H_kv, dims.topk, dtype=torch.int32, device=dev)
+    if ws is None:
+        ws = workspace(MSA_OP_INDEX_TOPK, dims, dev)
+    _check("msa_index_topk_local",
+           lib().msa_index_topk_local(ctypes.byref(dims.c()), _p(q_idx), _p(k_idx_local), tok0, ntok, _p(cs), _p(ci),
+                                      _p(ws), ws.numel(), _stream(stream)))
+    return cs, ci
+
+
+def msa_topk_merge(dims: MsaDims, cand_scores, cand_ids, stream=None):
+    """Merge of P ranks' candidates [P, B, N, H_kv, topk] into blocks int32 [B, N, H_kv, topk+1]."""
+    P = cand_scores.shape[0]
+    dev = cand_scores.device
+    _need(cand_scores, "cand_scores", (P, dims.B, dims.N, dims.H_kv, dims.topk), torch.float32, dev)
+    _need(cand_ids, "cand_ids", (P, dims.B, dims.N, dims.H_kv, dims.topk), torch.int32, dev)
+    blocks = torch.empty(dims.B, dims.N, dims.H_kv, dims.topk + 1, dtype=torch.int32, device=dev)
+    _check("msa_topk_merge", lib().msa_topk_merge(ctypes.byref(dims.c()), P, _p(cand_scores), _p(cand_ids), _p(blocks),
+                                                  _stream(stream)))
+    return blocks
+
+
+def msa_lse_idx_local(dims: MsaDims, q_idx, k_idx_local, tok0: int, blocks, stream=None):
+    """This rank's (max, exp-sum) of the index scores over the selected tokens it holds:
+    fp32 [B, N, H_kv, 2]."""
+    dev = q_idx.device
+    ntok = k_idx_local.shape[1]
+    _need(q_idx, "q_idx", (dims.B, dims.N, dims.H_kv, dims.d_idx), torch.bfloat16, dev)
+    _need(k_idx_local, "k_idx_local", (dims.B, ntok, dims.d_idx), torch.bfloat16, dev)
+    _need(blocks, "blocks", (dims.B, dims.N, dims.H_kv, dims.topk + 1), torch.int32, dev)
+    ml = torch.empty(dims.B, dims.N, dims.H_kv, 2, dtype=torch.float32, device=dev)
+    _check("msa_lse_idx_local", lib().msa_lse_idx_local(ctypes.byref(dims.c()), _p(q_idx), _p(k_idx_local), tok0, ntok,
+                                                        _p(blocks), _p(ml), _stream(stream)))
+    return ml
+
+
+def msa_lse_combine(dims: MsaDims, ml, stream=None):
+    """Eq (16) over the P ranks' pairs ml [P, B, N, H_kv, 2]: LSE_idx fp32 [B, N, H_kv]."""
+    P = ml.shape[0]
+    _need(ml, "ml", (P, dims.B, dims.N, dims.H_kv, 2), torch.float32, ml.device)
+    lse = torch.empty(dims.B, dims.N, dims.H_kv, dtype=torch.float32, device=ml.device)
+    _check("msa_lse_combine", lib().msa_lse_combine(ctypes.byref(dims.c()), P, _p(ml), _p(lse), _stream(stream)))
+    return lse
+
+
 def msa_kl_fwd_grad(dims: MsaDims, q, k, q_idx, k_idx, blocks, lse, lse_idx=None, grad_scale: float = 1.0, ws=None,
                     stream=None):
     """KL alignment. Returns loss fp32 [1], dq_idx fp32 [B,N,H_kv,d_idx], dk_idx fp32 [B,N,d_idx]."""
@@ -324,5 +383,6 @@ def msa_get_device_status(ws: torch.Tensor, stream=None) -> int:
 
 __all__ = ["MsaDims", "MsaError", "msa_workspace_size", "msa_index_topk", "msa_sparse_attn_fwd",
            "msa_sparse_attn_decode", "msa_sparse_attn_decode_noalloc", "msa_sparse_attn_decode_fp8idx",
-           "msa_quantize_e4m3_rows", "msa_kl_fwd_grad", "msa_sparse_attn_bwd", "msa_get_device_status", "msa_status_string",
+           "msa_quantize_e4m3_rows", "msa_kl_fwd_grad", "msa_sparse_attn_bwd", "msa_index_topk_local",
+           "msa_topk_merge", "msa_lse_idx_local", "msa_lse_combine", "msa_get_device_status", "msa_status_string",
            "msa_version", "msa_profile_enable", "msa_profile_read", "workspace", "lib", "LIB_PATH"]

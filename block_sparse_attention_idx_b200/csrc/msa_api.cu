@@ -148,7 +148,7 @@ msa_status msa_index_topk(const msa_dims* d, const void* q_idx, const void* k_id
     DevStatus* status = static_cast<DevStatus*>(ws);
     cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, st);
     if (e != cudaSuccess) return MSA_ERR_CUDA;
-    IndexArgs a{d->B, d->N, d->H_kv, d->d_idx, d->block_k, d->topk, blocks, status};
+    IndexArgs a{d->B, d->N, d->H_kv, d->d_idx, d->block_k, d->topk, blocks, status, 0, d->N, nullptr, nullptr};
     e = run_index_topk(a, q_idx, k_idx, st);
     if (e != cudaSuccess || !lse_idx) return cuda_status(e);
     // LSE_idx over the selected token sets: per-(query, selected block) sum-exps, merged
@@ -258,6 +258,61 @@ msa_status msa_quantize_e4m3_rows(const void* x, int64_t rows, int n, uint8_t* c
     if (rows > ((int64_t)1 << 40) / n) return MSA_ERR_UNSUPPORTED;
     return cuda_status(run_quantize_e4m3_rows(x, rows, n, codes, scale, num_sms(),
                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static bool sp_range_ok(const msa_dims* d, int tok0, int ntok) {
+    return tok0 >= 0 && ntok > 0 && tok0 % d->block_k == 0 && (long long)tok0 + ntok <= d->N &&
+           (ntok % d->block_k == 0 || tok0 + ntok == d->N);
+}
+
+msa_status msa_index_topk_local(const msa_dims* d, const void* q_idx, const void* k_idx_local, int tok0, int ntok,
+                                float* cand_scores, int32_t* cand_ids, void* ws, size_t ws_bytes,
+                                msa_stream_t stream_) {
+    msa_status s = check_common(d);
+    if (s != MSA_OK) return s;
+    if (!q_idx || !k_idx_local || !cand_scores || !cand_ids || !aligned16(q_idx) || !aligned16(k_idx_local) ||
+        !aligned16(cand_scores) || !aligned16(cand_ids) || !sp_range_ok(d, tok0, ntok))
+        return MSA_ERR_INVALID_ARG;
+    s = ws_check(ws, ws_bytes, kStatusBytes);
+    if (s != MSA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_);
+    DevStatus* status = static_cast<DevStatus*>(ws);
+    cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, st);
+    if (e != cudaSuccess) return MSA_ERR_CUDA;
+    IndexArgs a{d->B, d->N, d->H_kv, d->d_idx, d->block_k, d->topk, nullptr, status, tok0, ntok, cand_scores, cand_ids};
+    return cuda_status(run_index_topk(a, q_idx, k_idx_local, st));
+}
+
+msa_status msa_topk_merge(const msa_dims* d, int P, const float* cand_scores, const int32_t* cand_ids,
+                          int32_t* blocks, msa_stream_t stream) {
+    msa_status s = check_common(d);
+    if (s != MSA_OK) return s;
+    if (P < 1 || P * d->topk > 128) return MSA_ERR_UNSUPPORTED;
+    if (!cand_scores || !cand_ids || !blocks || !aligned16(cand_scores) || !aligned16(cand_ids) || !aligned16(blocks))
+        return MSA_ERR_INVALID_ARG;
+    return cuda_status(run_topk_merge(d->B, d->N, d->H_kv, d->block_k, d->topk, P, cand_scores, cand_ids, blocks,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+msa_status msa_lse_idx_local(const msa_dims* d, const void* q_idx, const void* k_idx_local, int tok0, int ntok,
+                             const int32_t* blocks, float* ml, msa_stream_t stream) {
+    msa_status s = check_common(d);
+    if (s != MSA_OK) return s;
+    if (!q_idx || !k_idx_local || !blocks || !ml || !aligned16(q_idx) || !aligned16(k_idx_local) ||
+        !aligned16(blocks) || !aligned16(ml) || !sp_range_ok(d, tok0, ntok))
+        return MSA_ERR_INVALID_ARG;
+    return cuda_status(run_lse_idx_local(d->B, d->N, d->H_kv, d->d_idx, d->block_k, d->topk,
+                                         eff_scale(d->scale_idx, d->d_idx), q_idx, k_idx_local, tok0, ntok, blocks,
+                                         reinterpret_cast<float2*>(ml), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+msa_status msa_lse_combine(const msa_dims* d, int P, const float* ml, float* lse_idx, msa_stream_t stream) {
+    msa_status s = check_common(d);
+    if (s != MSA_OK) return s;
+    if (P < 1) return MSA_ERR_INVALID_ARG;
+    if (!ml || !lse_idx || !aligned16(ml) || !aligned16(lse_idx)) return MSA_ERR_INVALID_ARG;
+    return cuda_status(run_lse_combine(P, (long long)d->B * d->N * d->H_kv, reinterpret_cast<const float2*>(ml),
+                                       lse_idx, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 msa_status msa_sparse_attn_bwd(const msa_dims* d, const void* q, const void* k, const void* v, const int32_t* blocks,

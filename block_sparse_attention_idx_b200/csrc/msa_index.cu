@@ -58,7 +58,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int i_hi = min(a.N - 1, (R0 + kRows - 1) / a.H_kv);
     const int bmax = i_hi / a.block_k;                      // largest local block among the rows
     const int ntok = bmax * a.block_k;                      // tokens of complete past blocks
-    const int nkt = (ntok + kCols - 1) / kCols;
+    // tiles of the held key range [tok0, tok0 + ntok_held) that hold complete past blocks
+    const int span = min(ntok, a.tok0 + a.ntok) - a.tok0;
+    const int nkt = span > 0 ? (span + kCols - 1) / kCols : 0;
+    const int blk_end = (a.tok0 + a.ntok) / a.block_k;      // first block past the held range
 
     const int warp = warp_id(), lane = lane_id();
     if (threadIdx.x == 0) {
@@ -174,10 +177,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             // one candidate per complete past block inside this tile
             const int chunks_per_block = a.block_k / 32;
             for (int c0 = 0; c0 < 4; c0 += chunks_per_block) {
-                const int cb = (kt * kCols + c0 * 32) / a.block_k;
+                const int cb = (a.tok0 + kt * kCols + c0 * 32) / a.block_k;
                 float v = cmax[c0];
                 for (int x = 1; x < chunks_per_block; ++x) v = fmaxf(v, cmax[c0 + x]);
-                if (cb < bi && v > topv[kKMax - 1]) {
+                if (cb < bi && cb < blk_end && v > topv[kKMax - 1]) {
                     // stable insertion: equal maxima keep the earlier (lower) block id first
 #pragma unroll
                     for (int p = kKMax - 1; p > 0; --p) {
@@ -191,7 +194,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         if (!ok) s.abort = 1;
-        if (valid && ok) {
+        if (valid && ok && a.cand_ids) {
+            // the row's Top-k of the held range, best first, unmerged
+            const size_t o = ((size_t)b * rows_per_seq + R) * a.topk;
+#pragma unroll
+            for (int p = 0; p < kKMax; ++p)
+                if (p < a.topk) {
+                    a.cand_scores[o + p] = topi[p] >= 0 ? topv[p] : -INFINITY;
+                    a.cand_ids[o + p] = topi[p];
+                }
+        } else if (valid && ok) {
             // first topk entries plus the local block, ascending, -1 padded
             int sel[kKMax + 1];
 #pragma unroll
@@ -237,8 +249,8 @@ cudaError_t run_index_topk(const IndexArgs& a, const void* q_idx, const void* k_
     const uint64_t rows = (uint64_t)a.B * a.N * a.H_kv;
     const int sw = a.d_idx == 64 ? 128 : 64;
     if (!make_tmap_2d(&tq, q_idx, a.d_idx, rows, (uint64_t)a.d_idx * 2, a.d_idx, kRows, sw)) return cudaErrorInvalidValue;
-    if (!make_tmap_3d(&tk, k_idx, a.d_idx, a.N, a.B, (uint64_t)a.d_idx * 2, (uint64_t)a.N * a.d_idx * 2, a.d_idx,
-                      kCols, 1, sw))
+    if (!make_tmap_3d(&tk, k_idx, a.d_idx, a.ntok, a.B, (uint64_t)a.d_idx * 2, (uint64_t)a.ntok * a.d_idx * 2,
+                      a.d_idx, kCols, 1, sw))
         return cudaErrorInvalidValue;
     return a.d_idx == 64 ? launch_index<64>(a, tq, tk, st) : launch_index<32>(a, tq, tk, st);
 }

@@ -41,8 +41,23 @@ struct IndexArgs {
     int B, N, H_kv, d_idx, block_k, topk;
     int32_t* blocks;
     DevStatus* status;
+    // key range held in k_idx: tokens [tok0, tok0 + ntok) of every sequence, k_idx [B, ntok, d_idx]
+    // (0 and N for the whole sequence). With cand_ids set, the kernel writes each row's Top-k of the
+    // complete past blocks inside that range, unmerged (raw block maxima, -inf / -1 padded), instead
+    // of `blocks`.
+    int tok0, ntok;
+    float* cand_scores;   // [B, N, H_kv, topk]
+    int32_t* cand_ids;    // [B, N, H_kv, topk]
 };
 cudaError_t run_index_topk(const IndexArgs& a, const void* q_idx, const void* k_idx, cudaStream_t st);
+
+// ---------------------------------------------------------------- sequence-parallel indexer (msa_sp.cu)
+cudaError_t run_topk_merge(int B, int N, int H_kv, int block_k, int topk, int P, const float* cand_scores,
+                           const int32_t* cand_ids, int32_t* blocks, cudaStream_t st);
+cudaError_t run_lse_idx_local(int B, int N, int H_kv, int d_idx, int block_k, int topk, float scale_idx,
+                              const void* q_idx, const void* k_idx_local, int tok0, int ntok, const int32_t* blocks,
+                              float2* ml, cudaStream_t st);
+cudaError_t run_lse_combine(int P, long long rows, const float2* ml, float* lse, cudaStream_t st);
 
 // ---------------------------------------------------------------- inverse selection lists (msa_csr.cu)
 // For every (sequence b, query window w, group r, block c) the list of (query i, slot s) pairs

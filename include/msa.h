@@ -124,6 +124,37 @@ MSA_API msa_status msa_sparse_attn_fwd(const msa_dims *dims, const void *q, cons
                                msa_stream_t stream);
 
 /*
+ * Sequence-parallel index branch ("4.1.1 · 监督与联合训练", section 3, eq (16)): P ranks each hold a
+ * contiguous range of every sequence's keys; only (score, block id) candidates and per-row
+ * (max, exp-sum) pairs are exchanged, and the result equals the single-device msa_index_topk.
+ * The key range of a rank is tokens [tok0, tok0 + ntok): tok0 a multiple of block_k, ntok a
+ * multiple of block_k unless the range ends at N; k_idx_local holds those tokens, bf16
+ * [B, ntok, d_idx]. The ranks' ranges tile [0, N) in rank order.
+ *
+ * msa_index_topk_local: for every (b, i, r), the Top-k of the complete past blocks c < b_i that this
+ *   rank holds, by (M desc, block id asc), best first. cand_scores fp32 [B, N, H_kv, topk] are the
+ *   raw block maxima of Q^idx . K^idx (without scale_idx, so that every rank compares the same
+ *   numbers as the single-device kernel), -inf padded; cand_ids int32, -1 padded. Workspace: the
+ *   MSA_OP_INDEX_TOPK size.
+ * msa_topk_merge: cand_scores / cand_ids [P, B, N, H_kv, topk] gathered in rank order -> blocks
+ *   int32 [B, N, H_kv, topk+1]: Top-k of the union by (score desc, id asc) plus the local block,
+ *   ascending, -1 padded (identical to msa_index_topk's output). P * topk <= 128.
+ * msa_lse_idx_local: ml fp32 [B, N, H_kv, 2] = (a_p, z_p): the maximum of the index scores
+ *   (scale_idx included) over the causal tokens of the row's selected blocks held here, and the
+ *   sum of exp(score - a_p) over them; (-inf, 0) if this rank holds none.
+ * msa_lse_combine: eq (16) over ml [P, B, N, H_kv, 2] gathered in rank order: lse_idx fp32
+ *   [B, N, H_kv] = a + log(z), a = max_p a_p, z = sum_p exp(a_p - a) z_p.
+ */
+MSA_API msa_status msa_index_topk_local(const msa_dims *dims, const void *q_idx, const void *k_idx_local, int tok0,
+                                        int ntok, float *cand_scores, int32_t *cand_ids, void *ws, size_t ws_bytes,
+                                        msa_stream_t stream);
+MSA_API msa_status msa_topk_merge(const msa_dims *dims, int P, const float *cand_scores, const int32_t *cand_ids,
+                                  int32_t *blocks, msa_stream_t stream);
+MSA_API msa_status msa_lse_idx_local(const msa_dims *dims, const void *q_idx, const void *k_idx_local, int tok0,
+                                     int ntok, const int32_t *blocks, float *ml, msa_stream_t stream);
+MSA_API msa_status msa_lse_combine(const msa_dims *dims, int P, const float *ml, float *lse_idx, msa_stream_t stream);
+
+/*
  * Backward of msa_sparse_attn_fwd with the selection held fixed ("2.4 · 训练原生稀疏", section 2.2,
  * eq (11): on a fixed set the selected attention is ordinary attention, and positions outside the
  * set get no gradient). With J, o and LSE as in the forward and g = dout[b,i,h]:
