@@ -508,6 +508,61 @@ def bench_decode(args, world, rank, msa, pk):
     return res
 
 
+def bench_sp(args, world, rank, msa, pk):
+    """Sequence-parallel index branch on the headline workload with P ranks emulated on this GPU:
+    each rank's local Top-k and local (max, exp-sum) on its own K_idx slice timed separately (on P
+    GPUs they run side by side, so the step's compute is the slowest rank), plus the merge and the
+    eq (16) combine that every rank runs after the all-gather. The all-gather itself is not timed
+    here (one GPU); its bytes per rank are reported."""
+    from block_sparse_attention_idx_b200 import sp
+    w = WORKLOADS[HEADLINE]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    x = prefill_inputs(w, device=dev, seed=rank_seed(w, rank))
+    dims = msa.MsaDims(w.B, w.N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
+    ref_blocks, ref_lse = msa.msa_index_topk(dims, x["q_idx"], x["k_idx"], want_lse=True)
+    flush = torch.zeros(256 << 20, dtype=torch.uint8, device=dev)
+    res = {"workload": HEADLINE, "note": "ranks emulated on one GPU; the all-gather is not timed"}
+    for P in (2, 8):
+        ranges = [sp.split_range(w.N, w.block_k, P, p) for p in range(P)]
+        slices = [x["k_idx"][:, t0:t0 + n].contiguous() for t0, n in ranges]
+        ws = msa.workspace(msa.MSA_OP_INDEX_TOPK, dims, dev)
+        local_ms = []
+        cands = []
+        for (t0, n), kl in zip(ranges, slices):
+            for _ in range(max(3, args.warmup)):
+                c = msa.msa_index_topk_local(dims, x["q_idx"], kl, t0, ws=ws)
+            t = timed_steps(lambda: msa.msa_index_topk_local(dims, x["q_idx"], kl, t0, ws=ws), 5, flush)
+            local_ms.append(sorted(t)[len(t) // 2])
+            cands.append(c)
+        cs = torch.stack([c[0] for c in cands])
+        ci = torch.stack([c[1] for c in cands])
+        for _ in range(3):
+            blocks = msa.msa_topk_merge(dims, cs, ci)
+        tm = timed_steps(lambda: msa.msa_topk_merge(dims, cs, ci), 5, flush)
+        lse_ms = []
+        mls = []
+        for (t0, n), kl in zip(ranges, slices):
+            ml = msa.msa_lse_idx_local(dims, x["q_idx"], kl, t0, blocks)
+            t = timed_steps(lambda: msa.msa_lse_idx_local(dims, x["q_idx"], kl, t0, blocks), 3, flush)
+            lse_ms.append(sorted(t)[len(t) // 2])
+            mls.append(ml)
+        ml_all = torch.stack(mls)
+        lse = msa.msa_lse_combine(dims, ml_all)
+        tc = timed_steps(lambda: msa.msa_lse_combine(dims, ml_all), 5, flush)
+        torch.cuda.synchronize()
+        rows = w.B * w.N * w.H_kv
+        res[f"P{P}"] = {
+            "local_topk_ms_max_rank": max(local_ms), "local_topk_ms_per_rank": [round(v, 4) for v in local_ms],
+            "merge_ms": sorted(tm)[len(tm) // 2], "local_lse_ms_max_rank": max(lse_ms),
+            "lse_combine_ms": sorted(tc)[len(tc) // 2],
+            "gather_bytes_per_rank": rows * w.topk * 8 + rows * 8,
+            "blocks_equal_single_device": bool(torch.equal(blocks, ref_blocks)),
+            "lse_max_abs_diff": float((lse - ref_lse).abs().max())}
+    del x, flush
+    torch.cuda.empty_cache()
+    return res
+
+
 def bench_train(args, world, rank, msa, pk):
     w = WORKLOADS["train_64k"]
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -577,7 +632,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--workload", default=HEADLINE, choices=["prefill_8k", "prefill_32k_needles", "train_64k"],
                     help="prefill workload of the headline step (smaller ones serve profiler captures)")
-    ap.add_argument("--only", choices=["decode", "train"], default=None,
+    ap.add_argument("--only", choices=["decode", "train", "sp"], default=None,
                     help="profiler captures: run only this secondary measurement and print its object")
     ap.add_argument("--decode-len", type=int, default=0, help="profiler captures: decode cache length")
     ap.add_argument("--train-n", type=int, default=0, help="profiler captures: training sequence length")
@@ -596,7 +651,7 @@ def main():
     import block_sparse_attention_idx_b200 as msa
     pk = peaks()
     if args.only:
-        res = (bench_decode if args.only == "decode" else bench_train)(args, world, rank, msa, pk)
+        res = {"decode": bench_decode, "train": bench_train, "sp": bench_sp}[args.only](args, world, rank, msa, pk)
         if world > 1:
             torch.distributed.destroy_process_group()
         if rank == 0:
@@ -621,6 +676,7 @@ def main():
     if not args.no_secondary:
         line["decode"] = bench_decode(args, world, rank, msa, pk)
         line["train"] = bench_train(args, world, rank, msa, pk)
+        line["sp_index"] = bench_sp(args, world, rank, msa, pk)
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank == 0:
