@@ -541,9 +541,10 @@ def bench_sp(args, world, rank, msa, pk):
         tm = timed_steps(lambda: msa.msa_topk_merge(dims, cs, ci), 5, flush)
         lse_ms = []
         mls = []
+        ws_l = msa.workspace(msa.MSA_OP_LSE_IDX_LOCAL, dims, dev)
         for (t0, n), kl in zip(ranges, slices):
-            ml = msa.msa_lse_idx_local(dims, x["q_idx"], kl, t0, blocks)
-            t = timed_steps(lambda: msa.msa_lse_idx_local(dims, x["q_idx"], kl, t0, blocks), 3, flush)
+            ml = msa.msa_lse_idx_local(dims, x["q_idx"], kl, t0, blocks, ws=ws_l).clone()
+            t = timed_steps(lambda: msa.msa_lse_idx_local(dims, x["q_idx"], kl, t0, blocks, ws=ws_l), 3, flush)
             lse_ms.append(sorted(t)[len(t) // 2])
             mls.append(ml)
         ml_all = torch.stack(mls)

@@ -18,7 +18,8 @@ LIB_PATH = os.path.join(_PKG, "libmsa.so")
 
 MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_WORKSPACE, MSA_ERR_CUDA, MSA_ERR_TIMEOUT, \
     MSA_ERR_DEVICE_CHECK = range(7)
-MSA_OP_INDEX_TOPK, MSA_OP_INDEX_TOPK_LSE, MSA_OP_ATTN_FWD, MSA_OP_DECODE, MSA_OP_KL, MSA_OP_ATTN_BWD = range(6)
+(MSA_OP_INDEX_TOPK, MSA_OP_INDEX_TOPK_LSE, MSA_OP_ATTN_FWD, MSA_OP_DECODE, MSA_OP_KL, MSA_OP_ATTN_BWD,
+ MSA_OP_LSE_IDX_LOCAL) = range(7)
 
 
 class MsaError(RuntimeError):
@@ -77,7 +78,7 @@ def lib() -> ctypes.CDLL:
         I = ctypes.c_int
         L.msa_index_topk_local.argtypes = [D, P, P, I, I, P, P, P, S, P]
         L.msa_topk_merge.argtypes = [D, I, P, P, P, P]
-        L.msa_lse_idx_local.argtypes = [D, P, P, I, I, P, P, P]
+        L.msa_lse_idx_local.argtypes = [D, P, P, I, I, P, P, P, S, P]
         L.msa_lse_combine.argtypes = [D, I, P, P, P]
         L.msa_sparse_attn_decode_noalloc.argtypes = [D, P, P, P, P, P, P, P, P, P]
         L.msa_sparse_attn_decode_noalloc.restype = ctypes.c_int
@@ -312,7 +313,7 @@ def msa_topk_merge(dims: MsaDims, cand_scores, cand_ids, stream=None):
     return blocks
 
 
-def msa_lse_idx_local(dims: MsaDims, q_idx, k_idx_local, tok0: int, blocks, stream=None):
+def msa_lse_idx_local(dims: MsaDims, q_idx, k_idx_local, tok0: int, blocks, ws=None, stream=None):
     """This rank's (max, exp-sum) of the index scores over the selected tokens it holds:
     fp32 [B, N, H_kv, 2]."""
     dev = q_idx.device
@@ -321,8 +322,10 @@ def msa_lse_idx_local(dims: MsaDims, q_idx, k_idx_local, tok0: int, blocks, stre
     _need(k_idx_local, "k_idx_local", (dims.B, ntok, dims.d_idx), torch.bfloat16, dev)
     _need(blocks, "blocks", (dims.B, dims.N, dims.H_kv, dims.topk + 1), torch.int32, dev)
     ml = torch.empty(dims.B, dims.N, dims.H_kv, 2, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = workspace(MSA_OP_LSE_IDX_LOCAL, dims, dev)
     _check("msa_lse_idx_local", lib().msa_lse_idx_local(ctypes.byref(dims.c()), _p(q_idx), _p(k_idx_local), tok0, ntok,
-                                                        _p(blocks), _p(ml), _stream(stream)))
+                                                        _p(blocks), _p(ml), _p(ws), ws.numel(), _stream(stream)))
     return ml
 
 

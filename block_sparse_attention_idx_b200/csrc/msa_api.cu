@@ -66,6 +66,10 @@ size_t ws_attn(const msa_dims* d) {
 size_t ws_decode(const msa_dims* d) {
     return kStatusBytes + decode_ws_bytes(d->B, d->N, d->H_q, d->H_kv, d->d, d->block_k, d->topk);
 }
+size_t ws_lse_local(const msa_dims* d) {
+    return ws_index_lse(d) + al256(rows_kv(d) * (d->topk + 1) * 4);
+}
+
 size_t ws_bwd(const msa_dims* d) {
     return kStatusBytes + csr_need(d) + al256((size_t)d->B * d->N * d->H_q * 4);
 }
@@ -127,6 +131,7 @@ msa_status msa_workspace_size(int op, const msa_dims* d, size_t* bytes) {
             return MSA_OK;
         case MSA_OP_DECODE: *bytes = ws_decode(d); return MSA_OK;
         case MSA_OP_KL: *bytes = ws_kl(d); return MSA_OK;
+        case MSA_OP_LSE_IDX_LOCAL: *bytes = ws_lse_local(d); return MSA_OK;
         case MSA_OP_ATTN_BWD:
             if (!bwd_supported(d->d, d->H_q / d->H_kv)) return MSA_ERR_UNSUPPORTED;
             *bytes = ws_bwd(d);
@@ -159,6 +164,8 @@ msa_status msa_index_topk(const msa_dims* d, const void* q_idx, const void* k_id
     k.scale = eff_scale(d->scale, d->d); k.scale_idx = eff_scale(d->scale_idx, d->d_idx);
     csr_carve(&k.csr_idx, cv.take(csr_need(d)), d->B, d->N, d->H_kv, d->block_k, d->topk, 0);
     k.ml_part = reinterpret_cast<float2*>(cv.take(rows_kv(d) * (d->topk + 1) * sizeof(float2)));
+    k.kv_tok0 = 0;
+    k.kv_ntok = d->N;
     k.lse_idx = lse_idx;
     k.blocks = blocks;
     k.status = status;
@@ -295,15 +302,37 @@ msa_status msa_topk_merge(const msa_dims* d, int P, const float* cand_scores, co
 }
 
 msa_status msa_lse_idx_local(const msa_dims* d, const void* q_idx, const void* k_idx_local, int tok0, int ntok,
-                             const int32_t* blocks, float* ml, msa_stream_t stream) {
+                             const int32_t* blocks, float* ml, void* ws, size_t ws_bytes, msa_stream_t stream_) {
     msa_status s = check_common(d);
     if (s != MSA_OK) return s;
     if (!q_idx || !k_idx_local || !blocks || !ml || !aligned16(q_idx) || !aligned16(k_idx_local) ||
         !aligned16(blocks) || !aligned16(ml) || !sp_range_ok(d, tok0, ntok))
         return MSA_ERR_INVALID_ARG;
-    return cuda_status(run_lse_idx_local(d->B, d->N, d->H_kv, d->d_idx, d->block_k, d->topk,
-                                         eff_scale(d->scale_idx, d->d_idx), q_idx, k_idx_local, tok0, ntok, blocks,
-                                         reinterpret_cast<float2*>(ml), reinterpret_cast<cudaStream_t>(stream)));
+    s = ws_check(ws, ws_bytes, ws_lse_local(d));
+    if (s != MSA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_);
+    DevStatus* status = static_cast<DevStatus*>(ws);
+    cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, st);
+    if (e != cudaSuccess) return MSA_ERR_CUDA;
+    Carver cv{static_cast<uint8_t*>(ws) + kStatusBytes};
+    KlArgs k{};
+    k.B = d->B; k.N = d->N; k.H_q = d->H_q; k.H_kv = d->H_kv; k.d = d->d; k.d_idx = d->d_idx;
+    k.block_k = d->block_k; k.topk = d->topk;
+    k.scale = eff_scale(d->scale, d->d); k.scale_idx = eff_scale(d->scale_idx, d->d_idx);
+    csr_carve(&k.csr_idx, cv.take(csr_need(d)), d->B, d->N, d->H_kv, d->block_k, d->topk, 0);
+    k.ml_part = reinterpret_cast<float2*>(cv.take(rows_kv(d) * (d->topk + 1) * sizeof(float2)));
+    int32_t* held = reinterpret_cast<int32_t*>(cv.take(rows_kv(d) * (d->topk + 1) * 4));
+    k.blocks = held;
+    k.status = status;
+    k.kv_tok0 = tok0;
+    k.kv_ntok = ntok;
+    k.ml_out = reinterpret_cast<float2*>(ml);
+    const int blk0 = tok0 / d->block_k, blk1 = (tok0 + ntok + d->block_k - 1) / d->block_k;
+    e = run_blocks_in_range((long long)rows_kv(d), d->topk + 1, blk0, blk1, blocks, held, st);
+    if (e == cudaSuccess)
+        e = run_csr_build(k.csr_idx, held, d->B, d->N, d->H_kv, d->block_k, d->topk, kIdxQpc, status, st);
+    if (e == cudaSuccess) e = run_lse_idx(k, q_idx, k_idx_local, num_sms(), st);
+    return cuda_status(e);
 }
 
 msa_status msa_lse_combine(const msa_dims* d, int P, const float* ml, float* lse_idx, msa_stream_t stream) {
@@ -375,6 +404,8 @@ msa_status msa_kl_fwd_grad(const msa_dims* d, const void* q, const void* k, cons
     a.block_k = d->block_k; a.topk = d->topk;
     a.scale = eff_scale(d->scale, d->d); a.scale_idx = eff_scale(d->scale_idx, d->d_idx);
     a.grad_scale = grad_scale;
+    a.kv_tok0 = 0;
+    a.kv_ntok = d->N;
     csr_carve(&a.csr, cv.take(csr_need(d)), d->B, d->N, d->H_kv, d->block_k, d->topk, 0);
     a.csr_idx = a.csr;  // same lists, its own chunking
     a.csr_idx.chunk_off = reinterpret_cast<int32_t*>(cv.take((nl + 1) * 4));

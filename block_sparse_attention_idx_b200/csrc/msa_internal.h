@@ -54,9 +54,8 @@ cudaError_t run_index_topk(const IndexArgs& a, const void* q_idx, const void* k_
 // ---------------------------------------------------------------- sequence-parallel indexer (msa_sp.cu)
 cudaError_t run_topk_merge(int B, int N, int H_kv, int block_k, int topk, int P, const float* cand_scores,
                            const int32_t* cand_ids, int32_t* blocks, cudaStream_t st);
-cudaError_t run_lse_idx_local(int B, int N, int H_kv, int d_idx, int block_k, int topk, float scale_idx,
-                              const void* q_idx, const void* k_idx_local, int tok0, int ntok, const int32_t* blocks,
-                              float2* ml, cudaStream_t st);
+cudaError_t run_blocks_in_range(long long rows, int K1, int blk0, int blk1, const int32_t* blocks, int32_t* out,
+                                cudaStream_t st);
 cudaError_t run_lse_combine(int P, long long rows, const float2* ml, float* lse, cudaStream_t st);
 
 // ---------------------------------------------------------------- inverse selection lists (msa_csr.cu)
@@ -138,6 +137,11 @@ struct KlArgs {
     float* loss;        // [1]
     const int32_t* blocks;
     DevStatus* status;
+    // LSE_idx pass only: k_idx holds tokens [kv_tok0, kv_tok0 + kv_ntok) ([B, kv_ntok, d_idx]; 0 and N
+    // for the whole sequence); with ml_out set, each row's (max, exp-sum) is written there instead
+    // of lse_idx
+    int kv_tok0, kv_ntok;
+    float2* ml_out;     // [B, N, H_kv]
 };
 constexpr int kIdxQpc = 32;
 bool kl_supported(int d, int d_idx, int G);

@@ -57,11 +57,12 @@ __global__ void __launch_bounds__(128) k_lse_idx(KlArgs a, const __nv_bfloat16* 
         __syncthreads();  // the previous item is done with kb / qb / s_i / red
         if (L != curL) {
             const int tok = c * a.block_k + tt;
-            const bool tvalid = tt < a.block_k && tok < a.N;
+            const bool tvalid = tt < a.block_k && tok < a.N && tok >= a.kv_tok0 && tok < a.kv_tok0 + a.kv_ntok;
 #pragma unroll
             for (int x = 0; x < DI / 8; ++x) {
                 uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if (tvalid) v = *reinterpret_cast<const uint4*>(k_idx + ((size_t)b * a.N + tok) * DI + x * 8);
+                if (tvalid)
+                    v = *reinterpret_cast<const uint4*>(k_idx + ((size_t)b * a.kv_ntok + (tok - a.kv_tok0)) * DI + x * 8);
                 *reinterpret_cast<uint4*>(&kb[tt * KBP + x * 8]) = v;
             }
             curL = L;
@@ -183,7 +184,8 @@ __global__ void k_lse_idx_merge(KlArgs a) {
         const float2 ml = a.ml_part[row * K1 + s];
         z += ml.y * __expf(ml.x - mx);
     }
-    a.lse_idx[row] = mx + logf(z);
+    if (a.ml_out) a.ml_out[row] = make_float2(mx, z);
+    else a.lse_idx[row] = mx + logf(z);
 }
 
 // ============================================================================ KL kernel

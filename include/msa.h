@@ -83,7 +83,8 @@ enum {
     MSA_OP_ATTN_FWD = 2,
     MSA_OP_DECODE = 3,
     MSA_OP_KL = 4,
-    MSA_OP_ATTN_BWD = 5
+    MSA_OP_ATTN_BWD = 5,
+    MSA_OP_LSE_IDX_LOCAL = 6
 };
 
 /* Workspace bytes `op` needs for `dims` (for MSA_OP_DECODE, dims->N is the cache capacity). */
@@ -141,7 +142,8 @@ MSA_API msa_status msa_sparse_attn_fwd(const msa_dims *dims, const void *q, cons
  *   ascending, -1 padded (identical to msa_index_topk's output). P * topk <= 128.
  * msa_lse_idx_local: ml fp32 [B, N, H_kv, 2] = (a_p, z_p): the maximum of the index scores
  *   (scale_idx included) over the causal tokens of the row's selected blocks held here, and the
- *   sum of exp(score - a_p) over them; (-inf, 0) if this rank holds none.
+ *   sum of exp(score - a_p) over them; (-inf, 0) if this rank holds none. Workspace:
+ *   msa_workspace_size(MSA_OP_LSE_IDX_LOCAL).
  * msa_lse_combine: eq (16) over ml [P, B, N, H_kv, 2] gathered in rank order: lse_idx fp32
  *   [B, N, H_kv] = a + log(z), a = max_p a_p, z = sum_p exp(a_p - a) z_p.
  */
@@ -151,7 +153,8 @@ MSA_API msa_status msa_index_topk_local(const msa_dims *dims, const void *q_idx,
 MSA_API msa_status msa_topk_merge(const msa_dims *dims, int P, const float *cand_scores, const int32_t *cand_ids,
                                   int32_t *blocks, msa_stream_t stream);
 MSA_API msa_status msa_lse_idx_local(const msa_dims *dims, const void *q_idx, const void *k_idx_local, int tok0,
-                                     int ntok, const int32_t *blocks, float *ml, msa_stream_t stream);
+                                     int ntok, const int32_t *blocks, float *ml, void *ws, size_t ws_bytes,
+                                     msa_stream_t stream);
 MSA_API msa_status msa_lse_combine(const msa_dims *dims, int P, const float *ml, float *lse_idx, msa_stream_t stream);
 
 /*
