@@ -87,6 +87,7 @@ def lib():
         _lib.orc_kl.argtypes = [D, P, P, P, P, ctypes.c_int, P, ctypes.c_double, P, i64, P, P, P, P]
         _lib.orc_decode.argtypes = [D, P, P, P, P, P, P, ctypes.c_int, P, P, P, P]
         _lib.orc_sparse_attn_bwd.argtypes = [D, P, P, P, P, ctypes.c_int, P, P, P, P]
+        _lib.orc_sparse_attn_bwd_dq_rows.argtypes = [D, P, P, P, P, ctypes.c_int, P, P, i64, P]
         _lib.orc_e4m3_values.argtypes = [P, i64, P]
         _lib.orc_e4m3_round_many.argtypes = [P, i64, P]
         _lib.orc_quantize_e4m3_rows.argtypes = [P, i64, ctypes.c_int, P, P]
@@ -235,6 +236,17 @@ def sparse_attn_bwd(dims: Dims, q, k, v, blocks, dout):
     lib().orc_sparse_attn_bwd(ctypes.byref(dims.c()), _ptr(qt), _ptr(kt), _ptr(vt), _ptr(gt), ty, _ptr(bl),
                               dq.ctypes.data, dk.ctypes.data, dv.ctypes.data)
     return dq, dk, dv
+
+
+def sparse_attn_bwd_dq_rows(dims: Dims, q, k, v, blocks, dout, rows):
+    """dq [nrows, H_q, d] of the given rows (flat b*N + i) only; same definition as sparse_attn_bwd."""
+    (qt, kt, vt, gt), ty = _inp(q, k, v, dout)
+    bl = _full_blocks(dims, blocks)
+    rt, nrows = _rows(rows)
+    dq = np.zeros((nrows, dims.H_q, dims.d), dtype=np.float64)
+    lib().orc_sparse_attn_bwd_dq_rows(ctypes.byref(dims.c()), _ptr(qt), _ptr(kt), _ptr(vt), _ptr(gt), ty, _ptr(bl),
+                                      _ptr(rt), nrows, dq.ctypes.data)
+    return dq
 
 
 def attend_tokens(q: np.ndarray, k: np.ndarray, v: np.ndarray, J, scale: float):

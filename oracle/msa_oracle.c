@@ -348,6 +348,49 @@ int orc_sparse_attn_bwd(const orc_dims *D, const void *q, const void *k, const v
     return 0;
 }
 
+/* dq rows only (same definition as orc_sparse_attn_bwd): dq of row (b, i) depends on that row's set
+ * alone, so sampled rows of a large problem can be checked. rows: flat b*N + i; dq [nrows, H_q, d]. */
+int orc_sparse_attn_bwd_dq_rows(const orc_dims *D, const void *q, const void *k, const void *v, const void *dout,
+                                int ty, const int32_t *blocks, const int64_t *rows, int64_t nrows, double *dq) {
+    const int K1 = D->topk + 1, G = D->H_q / D->H_kv;
+    const double sc = eff_scale(D);
+#pragma omp parallel
+    {
+        int32_t *J = (int32_t *)malloc(sizeof(int32_t) * (size_t)D->N);
+        double *z = (double *)malloc(sizeof(double) * (size_t)D->N);
+        double *o = (double *)malloc(sizeof(double) * (size_t)D->d);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t x = 0; x < nrows; ++x) {
+            const int b = (int)(rows[x] / D->N), i = (int)(rows[x] % D->N);
+            for (int h = 0; h < D->H_q; ++h) {
+                const int r = h / G;
+                const int32_t *sel = blocks + (((size_t)b * D->N + i) * D->H_kv + r) * K1;
+                const int nJ = token_set(D, sel, K1, i, J);
+                const size_t q_off = (((size_t)b * D->N + i) * D->H_q + h) * D->d;
+                const size_t kv_base = ((size_t)b * D->N * D->H_kv + r) * D->d, kv_stride = (size_t)D->H_kv * D->d;
+                double lse;
+                attend_tokens(D->d, sc, q, k, v, ty, q_off, kv_base, kv_stride, J, nJ, z, o, &lse);
+                double go = 0.0;
+                for (int c = 0; c < D->d; ++c) go += ld(dout, ty, q_off + c) * o[c];
+                double *dqr = dq + ((size_t)x * D->H_q + h) * D->d;
+                for (int c = 0; c < D->d; ++c) dqr[c] = 0.0;
+                for (int t = 0; t < nJ; ++t) {
+                    const size_t kvo = kv_base + (size_t)J[t] * kv_stride;
+                    const double alpha = exp(z[t] - lse);
+                    double gv = 0.0;
+                    for (int c = 0; c < D->d; ++c) gv += ld(dout, ty, q_off + c) * ld(v, ty, kvo + c);
+                    const double dz = alpha * (gv - go);
+                    for (int c = 0; c < D->d; ++c) dqr[c] += sc * dz * ld(k, ty, kvo + c);
+                }
+            }
+        }
+        free(J);
+        free(z);
+        free(o);
+    }
+    return 0;
+}
+
 /* Attention of one query vector over an explicit token list (exposed for the pins). */
 void orc_attend_tokens(int d, double scale, const double *q, const double *k, const double *v, const int32_t *J,
                        int nJ, double *o, double *lse) {

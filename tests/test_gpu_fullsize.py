@@ -11,7 +11,7 @@ import torch
 import block_sparse_attention_idx_b200 as msa
 import oracle
 from msa_inputs import WORKLOADS, prefill_inputs, decode_inputs
-from parity import compare_blocks, check_attention, check_grad
+from parity import compare_blocks, check_attention, check_grad, check_bwd
 
 pytestmark = pytest.mark.gpu
 
@@ -97,6 +97,26 @@ def test_full_training_step_sampled_rows_and_invariants():
     tot = dk.double().sum(dim=1).abs().max().item()
     scale = dk.double().abs().sum(dim=1).max().item()
     assert tot <= 1e-3 * max(scale, 1e-30), f"sum over tokens of dK_idx is {tot:.3e} (|dK_idx| sum {scale:.3e})"
+    del dq, dk, ws_k
+    # main-branch backward in the benchmark's configuration: dq of the sampled rows against the
+    # oracle (its own selection, rows where the GPU chose the same blocks), and the sums over tokens
+    # that hold at any size (sum_j dv_j = the group's upstream gradients, sum_j dk_j = 0)
+    gen = torch.Generator().manual_seed(4242)
+    dout = torch.randn(w.B, w.N, w.H_q, w.d, generator=gen).to(torch.bfloat16)
+    ws_b = msa.workspace(msa.MSA_OP_ATTN_BWD, dm, DEV)
+    gq, gk, gv = msa.msa_sparse_attn_bwd(dm, x["q"], x["k"], x["v"], blocks, out, lse, dout.to(DEV), ws=ws_b)
+    torch.cuda.synchronize()
+    assert msa.msa_get_device_status(ws_b) == msa.MSA_OK
+    odq = oracle.sparse_attn_bwd_dq_rows(od, xc["q"], xc["k"], xc["v"], full, dout, rows)
+    gqr = gq.cpu().numpy().reshape(w.B * w.N, w.H_q, w.d)[rows]
+    check_bwd(gqr[same], odq[same], "dq (sampled rows)")
+    G = w.H_q // w.H_kv
+    for r in range(w.H_kv):
+        want = dout[0, :, r * G:(r + 1) * G].double().sum(dim=(0, 1))
+        got = gv[0, :, r].double().sum(0).cpu()
+        assert (got - want).abs().max().item() <= 1e-3 * max(want.abs().max().item(), 1.0)
+        ks = gk[0, :, r].double()
+        assert ks.sum(0).abs().max().item() <= 1e-3 * ks.abs().sum(0).max().item()
 
 
 def test_full_decode_sampled_sequences_match_oracle():

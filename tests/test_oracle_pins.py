@@ -577,3 +577,13 @@ def test_sp_merge_and_lse_equal_single_device(bounds):
     for p in range(len(bounds) - 1):
         ml.append(sp.local_lse(dims, x["q_idx"], x["k_idx"], blocks, bounds[p], bounds[p + 1]))
     np.testing.assert_allclose(sp.combine_lse(ml), lse.reshape(2, N, Hkv), atol=1e-12)
+
+
+def test_bwd_dq_rows_equal_full_backward():
+    """The row-subset dq of the oracle is the full backward's dq on those rows (so that sampled rows
+    of full-size problems can be checked)."""
+    dims, x, blocks, dout = _bwd_case(N=50, Bk=8, k=2, G=2, Hkv=2, d=8, seed=13)
+    dq, _, _ = oracle.sparse_attn_bwd(dims, x["q"], x["k"], x["v"], blocks, dout)
+    rows = [0, 7, 8, 31, 49]
+    sub = oracle.sparse_attn_bwd_dq_rows(dims, x["q"], x["k"], x["v"], blocks, dout, rows)
+    np.testing.assert_allclose(sub, dq[0, rows], atol=1e-14)
