@@ -135,11 +135,11 @@ MEASURED_TRAFFIC = {
                       "sha256": "55bbdf3d16d2cb6f83b7bcb203d7af9aa655fe16e19d10c2c80fd62fe8a7188e",
                       "bytes_per_unit": (206054656 + 1970213120) / 60309504, "unit": "selected token",
                       "capture": "profiles/attn_kv_outer_prefill_8k.md"},
-    # training capture at N=8192 (dram read 991,507,200 B + write 136,743,680 B per launch over
+    # training capture at N=8192 (dram read 990,195,968 B + write 133,234,176 B per launch over
     # 60,309,504 selected tokens), scaled by the selected tokens of the timed launch
     "kl_kv_outer": {"file": "block_sparse_attention_idx_b200/csrc/msa_kl.cu",
-                    "sha256": "14cb19baa5ea1a26ed617e36066629b07b8a9f99a90d086cb3700db4150cafa5",
-                    "bytes_per_unit": (991507200 + 136743680) / 60309504, "unit": "selected token",
+                    "sha256": "cd1f5a11cf7d642f437922350ed4ec35ece93132b5aabbecb7fd3a8cd1695605",
+                    "bytes_per_unit": (990195968 + 133234176) / 60309504, "unit": "selected token",
                     "capture": "profiles/kl_kv_outer_train_8k.md"},
     # attention backward at N=8192 (dram read 6,612,550,485 B + write 3,289,236,480 B per launch over
     # 60,309,504 selected tokens; most of it is the read-modify-write of dQ by the per-item reductions)
