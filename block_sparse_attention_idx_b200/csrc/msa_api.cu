@@ -294,7 +294,7 @@ msa_status msa_topk_merge(const msa_dims* d, int P, const float* cand_scores, co
                           int32_t* blocks, msa_stream_t stream) {
     msa_status s = check_common(d);
     if (s != MSA_OK) return s;
-    if (P < 1 || P * d->topk > 128) return MSA_ERR_UNSUPPORTED;
+    if (P < 1 || P > 8) return MSA_ERR_UNSUPPORTED;
     if (!cand_scores || !cand_ids || !blocks || !aligned16(cand_scores) || !aligned16(cand_ids) || !aligned16(blocks))
         return MSA_ERR_INVALID_ARG;
     return cuda_status(run_topk_merge(d->B, d->N, d->H_kv, d->block_k, d->topk, P, cand_scores, cand_ids, blocks,

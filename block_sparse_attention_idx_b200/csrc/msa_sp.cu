@@ -12,70 +12,55 @@ namespace msa {
 
 namespace {
 
-constexpr int kMaxCand = 128;  // P * topk candidates per row (at most 8 ranks x 16)
+constexpr int kMaxRanks = 8;
 
-// One warp per (b, i, r) row: Top-k of the P ranks' candidates by (score desc, block id asc), then
-// the local block b_i, written ascending and -1 padded. The scores are raw block maxima computed
-// the same way on every rank, so the order is the single-device order, ties included.
+// One thread per (b, i, r) row: each rank's candidate list is already ordered best first by
+// (score desc, block id asc), so the Top-k of the union is a P-way merge of the list heads. The
+// scores are raw block maxima computed the same way on every rank, so the order is the
+// single-device order, ties included. Then the local block b_i; written ascending, -1 padded.
 __global__ void __launch_bounds__(256) k_topk_merge(int B, int N, int H_kv, int block_k, int topk, int P,
                                                     const float* __restrict__ cs, const int32_t* __restrict__ ci,
                                                     int32_t* __restrict__ blocks) {
-    const long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const long long rows = (long long)B * N * H_kv;
     if (row >= rows) return;
     const int i = (int)((row / H_kv) % N);
-    const int bi = i / block_k;
-    const int nc = P * topk;  // candidate x = p * topk + slot
-    float v[kMaxCand / 32];
-    int id[kMaxCand / 32];
-#pragma unroll
-    for (int u = 0; u < kMaxCand / 32; ++u) {
-        const int x = lane + 32 * u;
-        const int p = x / topk, sl = x % topk;
-        const size_t o = ((size_t)p * rows + row) * topk + sl;
-        id[u] = x < nc ? ci[o] : -1;
-        v[u] = id[u] >= 0 ? cs[o] : -INFINITY;
-    }
-    int mine = 0x7fffffff;  // lane p < topk: the p-th chosen id
-    int take = 0;
-    for (int p = 0; p < topk; ++p) {
-        // this lane's best untaken candidate
+    int head[kMaxRanks];
+    for (int p = 0; p < P; ++p) head[p] = 0;
+    int sel[17];
+    int n = 0;
+    for (; n < topk; ++n) {
+        int best = -1, bid = 0x7fffffff;
         float bv = -INFINITY;
-        int bid = 0x7fffffff, bu = -1;
-#pragma unroll
-        for (int u = 0; u < kMaxCand / 32; ++u)
-            if (id[u] >= 0 && (v[u] > bv || (v[u] == bv && id[u] < bid))) {
-                bv = v[u];
-                bid = id[u];
-                bu = u;
-            }
-        // warp-wide best, ties to the lower block id
-#pragma unroll
-        for (int o = 16; o; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oid = __shfl_xor_sync(0xffffffffu, bid, o);
-            if (ov > bv || (ov == bv && oid < bid)) {
-                bv = ov;
-                bid = oid;
+        for (int p = 0; p < P; ++p) {
+            if (head[p] >= topk) continue;
+            const size_t o = ((size_t)p * rows + row) * topk + head[p];
+            const int id = ci[o];
+            if (id < 0) continue;
+            const float v = cs[o];
+            if (best < 0 || v > bv || (v == bv && id < bid)) {
+                best = p;
+                bv = v;
+                bid = id;
             }
         }
-        if (bid == 0x7fffffff) break;  // no candidates left (warp-uniform)
-        if (lane == p) mine = bid;
-        // a block id appears on at most one rank: retire it wherever it sits
-#pragma unroll
-        for (int u = 0; u < kMaxCand / 32; ++u)
-            if (id[u] == bid) id[u] = -1;
-        (void)bu;
-        ++take;
+        if (best < 0) break;
+        ++head[best];
+        sel[n] = bid;
     }
-    if (lane == take) mine = bi;
-    const int n = take + 1;
-    int rank = 0;
-    for (int x = 0; x < n; ++x) rank += (__shfl_sync(0xffffffffu, mine, x) < mine);
+    sel[n] = i / block_k;  // the local block (larger than every past block)
+    // ascending: insertion sort of at most 17 ids
+    for (int x = 1; x <= n; ++x) {
+        const int v = sel[x];
+        int y = x - 1;
+        while (y >= 0 && sel[y] > v) {
+            sel[y + 1] = sel[y];
+            --y;
+        }
+        sel[y + 1] = v;
+    }
     int32_t* out = blocks + row * (topk + 1);
-    if (lane < n) out[rank] = mine;
-    else if (lane < topk + 1) out[lane] = -1;
+    for (int x = 0; x <= topk; ++x) out[x] = x <= n ? sel[x] : -1;
 }
 
 // The selection restricted to the blocks [blk0, blk1) a rank holds (others -1): the LSE_idx pass
@@ -108,8 +93,8 @@ cudaError_t run_topk_merge(int B, int N, int H_kv, int block_k, int topk, int P,
                            const int32_t* cand_ids, int32_t* blocks, cudaStream_t st) {
     const long long rows = (long long)B * N * H_kv;
     ProfScope ps("sp_topk_merge", st);
-    k_topk_merge<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>(B, N, H_kv, block_k, topk, P, cand_scores,
-                                                                      cand_ids, blocks);
+    k_topk_merge<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(B, N, H_kv, block_k, topk, P, cand_scores, cand_ids,
+                                                                 blocks);
     return cudaGetLastError();
 }
 

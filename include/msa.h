@@ -139,7 +139,7 @@ MSA_API msa_status msa_sparse_attn_fwd(const msa_dims *dims, const void *q, cons
  *   MSA_OP_INDEX_TOPK size.
  * msa_topk_merge: cand_scores / cand_ids [P, B, N, H_kv, topk] gathered in rank order -> blocks
  *   int32 [B, N, H_kv, topk+1]: Top-k of the union by (score desc, id asc) plus the local block,
- *   ascending, -1 padded (identical to msa_index_topk's output). P * topk <= 128.
+ *   ascending, -1 padded (identical to msa_index_topk's output). 1 <= P <= 8.
  * msa_lse_idx_local: ml fp32 [B, N, H_kv, 2] = (a_p, z_p): the maximum of the index scores
  *   (scale_idx included) over the causal tokens of the row's selected blocks held here, and the
  *   sum of exp(score - a_p) over them; (-inf, 0) if this rank holds none. Workspace:
