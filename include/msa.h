@@ -87,7 +87,12 @@ enum {
     MSA_OP_LSE_IDX_LOCAL = 6
 };
 
-/* Workspace bytes `op` needs for `dims` (for MSA_OP_DECODE, dims->N is the cache capacity). */
+/*
+ * Workspace bytes `op` needs for `dims` (for MSA_OP_DECODE, dims->N is the cache capacity).
+ * MSA_OP_DECODE also serves msa_sparse_attn_decode_fp8idx, MSA_OP_INDEX_TOPK also serves
+ * msa_index_topk_local, MSA_OP_ATTN_BWD is msa_sparse_attn_bwd's (MSA_ERR_UNSUPPORTED for its
+ * unsupported G), MSA_OP_LSE_IDX_LOCAL is msa_lse_idx_local's.
+ */
 MSA_API msa_status msa_workspace_size(int op, const msa_dims *dims, size_t *bytes);
 
 /*
