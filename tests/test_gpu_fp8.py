@@ -164,3 +164,33 @@ def test_fp8_flips_only_within_the_quantisation_bound():
     assert np.all(om16[flipped] <= 2 * eps[flipped] + 2 * NEAR_TIE), (om16[flipped], eps[flipped])
     print(f"fp8 vs bf16 selection: {int(flipped.sum())} of {flipped.size} rows differ; "
           f"median bf16 margin {np.median(om16):.3e}, score change bound median {np.median(eps):.3e}")
+
+
+def test_decode_short_caches_both_scorings():
+    """Edge cases of the decode step in both scorings: a cache of one token (no past block, the
+    local block only), exactly one block, one block plus one token, and a cache with exactly topk
+    complete past blocks (every candidate taken: margin +inf)."""
+    B, L, H_q, H_kv, d, d_idx, bk, k = 4, 700, 16, 2, 128, 64, 64, 5
+    gen = torch.Generator().manual_seed(5150)
+    mkr = lambda *s: torch.randn(*s, generator=gen).to(torch.bfloat16)
+    kc, vc, kic = mkr(B, L, H_kv, d), mkr(B, L, H_kv, d), mkr(B, L, d_idx)
+    q, qi = mkr(B, H_q, d), mkr(B, H_kv, d_idx)
+    lens = torch.tensor([1, bk, bk + 1, k * bk + 3], dtype=torch.int32)
+    dm = msa.MsaDims(B, L, H_q, H_kv, d, d_idx, bk, k)
+    od = oracle.Dims(B, L, H_q, H_kv, d, d_idx, bk, k)
+    g = {n: t.to(DEV) for n, t in dict(q=q, qi=qi, kc=kc, vc=vc, kic=kic, lens=lens).items()}
+    codes, kscale = msa.msa_quantize_e4m3_rows(g["kic"])
+    out16, b16, m16 = msa.msa_sparse_attn_decode(dm, g["lens"], g["q"], g["qi"], g["kc"], g["vc"], g["kic"],
+                                                 want_margin=True)
+    out8, b8, m8 = msa.msa_sparse_attn_decode_fp8idx(dm, g["lens"], g["q"], g["qi"], g["kc"], g["vc"], codes, kscale,
+                                                     want_margin=True)
+    torch.cuda.synchronize()
+    ob, om, oo, _ = oracle.decode(od, lens, q, qi, kc, vc, kic)
+    okc, oks = oracle.quantize_e4m3_rows(kic)
+    ob8, om8, oo8, _ = oracle.decode_fp8idx(od, lens, q, qi, kc, vc, okc, oks)
+    for gb, gm, go, rb, rm, ro in ((b16, m16, out16, ob, om, oo), (b8, m8, out8, ob8, om8, oo8)):
+        bad, _ = compare_blocks(gb.cpu().numpy(), rb, rm)
+        assert bad == 0
+        check_margins(gm.cpu().numpy(), rm)
+        assert np.isinf(gm.cpu().numpy()).all()  # at most topk complete past blocks in every row
+        check_attention(go.cpu().numpy(), ro)
