@@ -129,11 +129,11 @@ def valid_slots(blocks: torch.Tensor, block_k: int) -> int:
 # ncu capture of the kernel; it holds only for the kernel source it was measured on (sha256 of the
 # file), and reads null once that file changes.
 MEASURED_TRAFFIC = {
-    # prefill_8k capture (dram read 206,054,656 B + write 1,970,213,120 B per launch over 60,309,504
+    # prefill_8k capture (dram read 206,501,632 B + write 1,970,068,224 B per launch over 60,309,504
     # selected tokens), scaled by the selected tokens of the timed launch
     "attn_kv_outer": {"file": "block_sparse_attention_idx_b200/csrc/msa_attn.cu",
-                      "sha256": "55bbdf3d16d2cb6f83b7bcb203d7af9aa655fe16e19d10c2c80fd62fe8a7188e",
-                      "bytes_per_unit": (206054656 + 1970213120) / 60309504, "unit": "selected token",
+                      "sha256": "269122850540640827a73f8abc33c40ae5a5a5d3d25f6e037bf24701df279270",
+                      "bytes_per_unit": (206501632 + 1970068224) / 60309504, "unit": "selected token",
                       "capture": "profiles/attn_kv_outer_prefill_8k.md"},
     # training capture at N=8192 (dram read 990,195,968 B + write 133,234,176 B per launch over
     # 60,309,504 selected tokens), scaled by the selected tokens of the timed launch

@@ -55,7 +55,7 @@ struct AttnSmem {
     ItemMeta meta[kMeta];
     int stage[kStage];  // query entries of the items of the current scheduler fetch
     // per-row partial max / sums of the two column halves: [team][team item parity][half][row]
-    float red_max[2][2][2][kRows], red_l[2][2][2][kRows], red_lr[2][2][2][kRows];
+    float red_max[2][2][2][kRows], red_l[2][2][2][kRows];
     uint64_t meta_full[kMeta], meta_empty[kMeta];
     uint64_t q_full[2], q_empty[2];
     uint64_t k_full[2], k_release[2], v_full[2], v_release[2];  // release[b]: one completion per use of buffer b
@@ -388,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool have_prev = false;
         int pv_prow = -1;
         float pv_mx = 0.f;
-        // O of the team's item number kp: normalise by the row's rounded weight sum, store the fp16
+        // O of the team's item number kp: normalise by the row's weight sum l, store the fp16
         // partial and its LSE, free the accumulator
         // the partials are written once here and read once by the merge: they must not push the
         // query rows out of L2
@@ -399,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!__all_sync(0xffffffffu, mbar_wait(&s.sum_bar[t][pb], (kp >> 1) & 1, a.status, 0x705))) return false;
             tc_fence_after();
             float inv = 0.f;
-            if (pv_prow >= 0) inv = 1.f / (s.red_lr[t][pb][0][row] + s.red_lr[t][pb][1][row]);
+            if (pv_prow >= 0) inv = 1.f / (s.red_l[t][pb][0][row] + s.red_l[t][pb][1][row]);
             const uint64_t invx2 = f2_packf(inv, inv);
             // chunk x of 8 values goes to [(b, i, r, slot)][x][head]: the G heads of a query are
             // adjacent, so a warp's store covers whole 128-byte lines
@@ -492,12 +492,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             // pass 2: P = exp(S - max) rounded to bf16, packed two per TMEM column over the warp's
-            // own S columns already read. l: exact sum for the LSE; lr: sum of the rounded weights
-            // the MMA uses, so that O / lr stays a convex combination of the V rows.
+            // own S columns already read. l, the fp32 sum of the weights before rounding, gives the LSE
+            // and normalises O (the bf16 rounding of the weights changes their sum by ~1e-4 relative,
+            // well inside the attention tolerance; a second, rounded sum cost four more instructions
+            // per pair of columns and 2-4 % of the kernel's time).
             const float mx = fmaxf(s.red_max[t][kb][0][row], s.red_max[t][kb][1][row]);
             const float moff = valid ? mx * sl2 : 0.f;
             const uint64_t sl2x2 = f2_packf(sl2, sl2), moffx2 = f2_packf(-moff, -moff);
-            uint64_t lx2 = f2_packf(0.f, 0.f), lrx2 = f2_packf(0.f, 0.f);
+            uint64_t lx2 = f2_packf(0.f, 0.f);
 #pragma unroll
             for (int c0 = 0; c0 < SC; c0 += CH) {
                 uint32_t sv[CH];
@@ -516,7 +518,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __nv_bfloat162 pb2 = __floats2bfloat162_rn(p0, p1);
                     const uint32_t u = *reinterpret_cast<const uint32_t*>(&pb2);
                     lx2 = f2_add(lx2, f2_packf(p0, p1));
-                    lrx2 = f2_add(lrx2, f2_pack(u << 16, u & 0xffff0000u));
                     pk[y / 2] = u;
                 }
                 tmem_st<CH / 2>(tS + c0 / 2, pk);
@@ -524,11 +525,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st_wait();
             tc_fence_before();
             {
-                float l0, l1, lr0, lr1;
+                float l0, l1;
                 f2_unpack(lx2, l0, l1);
-                f2_unpack(lrx2, lr0, lr1);
                 s.red_l[t][kb][e][row] = l0 + l1;
-                s.red_lr[t][kb][e][row] = lr0 + lr1;
             }
             __syncwarp();
             if (lane == 0) {
