@@ -337,6 +337,39 @@ def test_kl_row_subset_matches_full():
     np.testing.assert_allclose(dqr, dq[rows], atol=1e-15)
 
 
+
+def test_kl_all_blocks_is_dense_causal_kl():
+    """Dense warm-up limit (k >= the number of blocks; "MSA 中的 KL 对齐与局部知识蒸馏", section 5: the
+    warm-up aligns over the whole causal context): the oracle's L_KL, KL rows
+    and both index gradients equal a whole-matrix computation in torch float64 -- causal masks on
+    the full score matrices, the teacher as the head average of per-head softmaxes, the student as
+    the index log-softmax, and autograd (not the analytic P_idx - P) for the gradients."""
+    N, Bk, G, Hkv, d, di = 48, 8, 3, 2, 8, 4
+    nb = N // Bk
+    dims = oracle.Dims(B=1, N=N, H_q=G * Hkv, H_kv=Hkv, d=d, d_idx=di, block_k=Bk, topk=nb)
+    x = _f64(small_prefill(N, G * Hkv, Hkv, d, di, Bk, nb, seed=23))
+    blocks, _, _ = oracle.index_topk(dims, x["q_idx"], x["k_idx"])
+    loss, kl_rows, dq, dk = oracle.kl(dims, x["q"], x["k"], x["q_idx"], x["k_idx"], blocks)
+    causal = torch.ones(N, N, dtype=torch.bool).tril()
+    qi = x["q_idx"][0].clone().requires_grad_(True)  # [N, H_kv, d_idx]
+    ki = x["k_idx"][0].clone().requires_grad_(True)  # [N, d_idx]
+    rows = []
+    for r in range(Hkv):
+        kr = x["k"][0, :, r]
+        P = torch.stack([torch.softmax((x["q"][0, :, h] @ kr.T / math.sqrt(d)).masked_fill(~causal, -math.inf), -1)
+                         for h in range(r * G, (r + 1) * G)]).mean(0)
+        logq = torch.log_softmax((qi[:, r] @ ki.T / math.sqrt(di)).masked_fill(~causal, -math.inf), -1)
+        terms = torch.where(causal, P * (P.clamp_min(1e-300).log() - logq), torch.zeros((), dtype=P.dtype))
+        rows.append(terms.sum(-1))
+    R = torch.stack(rows, -1)
+    L = R.sum() / (N * Hkv)
+    L.backward()
+    assert (blocks[:, :, 0] == 0).all() and (blocks >= 0).sum() == sum(i // Bk + 1 for i in range(N)) * Hkv
+    np.testing.assert_allclose(kl_rows, R.detach().numpy(), rtol=0, atol=1e-12)
+    assert loss == pytest.approx(float(L.detach()), rel=1e-12)
+    np.testing.assert_allclose(dq.reshape(N, Hkv, di), qi.grad.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dk[0], ki.grad.numpy(), rtol=0, atol=1e-12)
+
 # ----------------------------------------------------------------------------- decode
 def test_decode_equals_prefill_last_row():
     """Replaying one new token over the cache gives the parallel causal path's row L-1
