@@ -123,12 +123,22 @@ def _p(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream):
+def _stream(stream, dev: torch.device):
+    """The stream to launch on. The library launches on the current CUDA device, so the tensors'
+    device must be the current one (and an explicit stream must belong to it)."""
+    cur = torch.cuda.current_device()
+    if dev.type != "cuda" or (dev.index is not None and dev.index != cur):
+        raise ValueError(f"tensors are on {dev}, but the current CUDA device is cuda:{cur}; "
+                         "call under torch.cuda.device(...)")
     s = torch.cuda.current_stream() if stream is None else stream
+    if s.device.index != cur:
+        raise ValueError(f"stream belongs to {s.device}, not to the current device cuda:{cur}")
     return ctypes.c_void_p(s.cuda_stream)
 
 
 def _need(t: torch.Tensor, name: str, shape, dtype, device):
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (the library takes device pointers), got {t.device}")
     if tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
     if t.dtype != dtype:
@@ -144,6 +154,16 @@ def workspace(op: int, dims: MsaDims, device) -> torch.Tensor:
     return torch.empty(max(msa_workspace_size(op, dims), 256), dtype=torch.uint8, device=device)
 
 
+def _ws(ws, op: int, dims: MsaDims, dev) -> torch.Tensor:
+    """The caller's workspace, checked (a contiguous uint8 CUDA tensor on the inputs' device; the
+    library checks its size and alignment), or a new one for `op`."""
+    if ws is None:
+        return workspace(op, dims, dev)
+    if ws.dtype != torch.uint8 or not ws.is_contiguous() or ws.device != dev:
+        raise ValueError(f"ws must be a contiguous uint8 tensor on {dev}")
+    return ws
+
+
 def msa_index_topk(dims: MsaDims, q_idx, k_idx, want_lse: bool = False, ws=None, stream=None):
     """Block selection. Returns blocks int32 [B,N,H_kv,topk+1] (and LSE_idx fp32 [B,N,H_kv])."""
     dev = q_idx.device
@@ -151,10 +171,9 @@ def msa_index_topk(dims: MsaDims, q_idx, k_idx, want_lse: bool = False, ws=None,
     _need(k_idx, "k_idx", (dims.B, dims.N, dims.d_idx), torch.bfloat16, dev)
     blocks = torch.empty(dims.B, dims.N, dims.H_kv, dims.topk + 1, dtype=torch.int32, device=dev)
     lse = torch.empty(dims.B, dims.N, dims.H_kv, dtype=torch.float32, device=dev) if want_lse else None
-    if ws is None:
-        ws = workspace(MSA_OP_INDEX_TOPK_LSE if want_lse else MSA_OP_INDEX_TOPK, dims, dev)
+    ws = _ws(ws, MSA_OP_INDEX_TOPK_LSE if want_lse else MSA_OP_INDEX_TOPK, dims, dev)
     _check("msa_index_topk", lib().msa_index_topk(ctypes.byref(dims.c()), _p(q_idx), _p(k_idx), _p(blocks), _p(lse),
-                                                  _p(ws), ws.numel(), _stream(stream)))
+                                                  _p(ws), ws.numel(), _stream(stream, dev)))
     return (blocks, lse) if want_lse else blocks
 
 
@@ -167,10 +186,9 @@ def msa_sparse_attn_fwd(dims: MsaDims, q, k, v, blocks, want_lse: bool = True, w
     _need(blocks, "blocks", (dims.B, dims.N, dims.H_kv, dims.topk + 1), torch.int32, dev)
     out = torch.empty(q.shape, dtype=torch.float32, device=dev)
     lse = torch.empty(dims.B, dims.N, dims.H_q, dtype=torch.float32, device=dev) if want_lse else None
-    if ws is None:
-        ws = workspace(MSA_OP_ATTN_FWD, dims, dev)
+    ws = _ws(ws, MSA_OP_ATTN_FWD, dims, dev)
     _check("msa_sparse_attn_fwd", lib().msa_sparse_attn_fwd(ctypes.byref(dims.c()), _p(q), _p(k), _p(v), _p(blocks),
-                                                            _p(out), _p(lse), _p(ws), ws.numel(), _stream(stream)))
+                                                            _p(out), _p(lse), _p(ws), ws.numel(), _stream(stream, dev)))
     return out, lse
 
 
@@ -193,12 +211,11 @@ def msa_sparse_attn_decode(dims: MsaDims, cache_len, q, q_idx, k_cache, v_cache,
     blocks int32 [B,H_kv,topk+1] (or None); with want_margin, also the cutoff margins fp32 [B,H_kv]."""
     out, blocks, margin = _decode_io(dims, cache_len, q, q_idx, k_cache, v_cache, want_blocks, want_margin)
     _need(k_idx_cache, "k_idx_cache", (dims.B, dims.N, dims.d_idx), torch.bfloat16, q.device)
-    if ws is None:
-        ws = workspace(MSA_OP_DECODE, dims, q.device)
+    ws = _ws(ws, MSA_OP_DECODE, dims, q.device)
     _check("msa_sparse_attn_decode",
            lib().msa_sparse_attn_decode(ctypes.byref(dims.c()), _p(cache_len), _p(q), _p(q_idx), _p(k_cache),
                                         _p(v_cache), _p(k_idx_cache), _p(out), _p(blocks), _p(margin), _p(ws),
-                                        ws.numel(), _stream(stream)))
+                                        ws.numel(), _stream(stream, q.device)))
     return (out, blocks, margin) if want_margin else (out, blocks)
 
 
@@ -216,7 +233,7 @@ def msa_quantize_e4m3_rows(x, codes=None, scale=None, stream=None):
     _need(codes, "codes", tuple(x.shape), torch.uint8, x.device)
     _need(scale, "scale", tuple(x.shape[:-1]), torch.float32, x.device)
     _check("msa_quantize_e4m3_rows",
-           lib().msa_quantize_e4m3_rows(_p(x), rows, n, _p(codes), _p(scale), _stream(stream)))
+           lib().msa_quantize_e4m3_rows(_p(x), rows, n, _p(codes), _p(scale), _stream(stream, x.device)))
     return codes, scale
 
 
@@ -227,13 +244,12 @@ def msa_sparse_attn_decode_fp8idx(dims: MsaDims, cache_len, q, q_idx, k_cache, v
     out, blocks, margin = _decode_io(dims, cache_len, q, q_idx, k_cache, v_cache, want_blocks, want_margin)
     _need(k_idx_codes, "k_idx_codes", (dims.B, dims.N, dims.d_idx), torch.uint8, q.device)
     _need(k_idx_scale, "k_idx_scale", (dims.B, dims.N), torch.float32, q.device)
-    if ws is None:
-        ws = workspace(MSA_OP_DECODE, dims, q.device)
+    ws = _ws(ws, MSA_OP_DECODE, dims, q.device)
     _check("msa_sparse_attn_decode_fp8idx",
            lib().msa_sparse_attn_decode_fp8idx(ctypes.byref(dims.c()), _p(cache_len), _p(q), _p(q_idx),
                                                _p(k_cache), _p(v_cache), _p(k_idx_codes), _p(k_idx_scale),
                                                _p(out), _p(blocks), _p(margin), _p(ws), ws.numel(),
-                                               _stream(stream)))
+                                               _stream(stream, q.device)))
     return (out, blocks, margin) if want_margin else (out, blocks)
 
 
@@ -257,7 +273,7 @@ def msa_sparse_attn_decode_noalloc(dims: MsaDims, cache_len, q, q_idx, k_cache, 
     _check("msa_sparse_attn_decode_noalloc",
            lib().msa_sparse_attn_decode_noalloc(ctypes.byref(dims.c()), _p(cache_len), _p(q), _p(q_idx),
                                                 _p(k_cache), _p(v_cache), _p(k_idx_cache), _p(out), _p(blocks),
-                                                _stream(stream)))
+                                                _stream(stream, dev)))
     return out, blocks
 
 
@@ -275,11 +291,10 @@ def msa_sparse_attn_bwd(dims: MsaDims, q, k, v, blocks, out, lse, dout, ws=None,
     dq = torch.empty(dims.B, dims.N, dims.H_q, dims.d, dtype=torch.float32, device=dev)
     dk = torch.empty(dims.B, dims.N, dims.H_kv, dims.d, dtype=torch.float32, device=dev)
     dv = torch.empty(dims.B, dims.N, dims.H_kv, dims.d, dtype=torch.float32, device=dev)
-    if ws is None:
-        ws = workspace(MSA_OP_ATTN_BWD, dims, dev)
+    ws = _ws(ws, MSA_OP_ATTN_BWD, dims, dev)
     _check("msa_sparse_attn_bwd",
            lib().msa_sparse_attn_bwd(ctypes.byref(dims.c()), _p(q), _p(k), _p(v), _p(blocks), _p(out), _p(lse),
-                                     _p(dout), _p(dq), _p(dk), _p(dv), _p(ws), ws.numel(), _stream(stream)))
+                                     _p(dout), _p(dq), _p(dk), _p(dv), _p(ws), ws.numel(), _stream(stream, dev)))
     return dq, dk, dv
 
 
@@ -293,11 +308,10 @@ def msa_index_topk_local(dims: MsaDims, q_idx, k_idx_local, tok0: int, ws=None, 
     _need(k_idx_local, "k_idx_local", (dims.B, ntok, dims.d_idx), torch.bfloat16, dev)
     cs = torch.empty(dims.B, dims.N, dims.H_kv, dims.topk, dtype=torch.float32, device=dev)
     ci = torch.empty(dims.B, dims.N, dims.H_kv, dims.topk, dtype=torch.int32, device=dev)
-    if ws is None:
-        ws = workspace(MSA_OP_INDEX_TOPK, dims, dev)
+    ws = _ws(ws, MSA_OP_INDEX_TOPK, dims, dev)
     _check("msa_index_topk_local",
            lib().msa_index_topk_local(ctypes.byref(dims.c()), _p(q_idx), _p(k_idx_local), tok0, ntok, _p(cs), _p(ci),
-                                      _p(ws), ws.numel(), _stream(stream)))
+                                      _p(ws), ws.numel(), _stream(stream, dev)))
     return cs, ci
 
 
@@ -309,7 +323,7 @@ def msa_topk_merge(dims: MsaDims, cand_scores, cand_ids, stream=None):
     _need(cand_ids, "cand_ids", (P, dims.B, dims.N, dims.H_kv, dims.topk), torch.int32, dev)
     blocks = torch.empty(dims.B, dims.N, dims.H_kv, dims.topk + 1, dtype=torch.int32, device=dev)
     _check("msa_topk_merge", lib().msa_topk_merge(ctypes.byref(dims.c()), P, _p(cand_scores), _p(cand_ids), _p(blocks),
-                                                  _stream(stream)))
+                                                  _stream(stream, dev)))
     return blocks
 
 
@@ -322,10 +336,9 @@ def msa_lse_idx_local(dims: MsaDims, q_idx, k_idx_local, tok0: int, blocks, ws=N
     _need(k_idx_local, "k_idx_local", (dims.B, ntok, dims.d_idx), torch.bfloat16, dev)
     _need(blocks, "blocks", (dims.B, dims.N, dims.H_kv, dims.topk + 1), torch.int32, dev)
     ml = torch.empty(dims.B, dims.N, dims.H_kv, 2, dtype=torch.float32, device=dev)
-    if ws is None:
-        ws = workspace(MSA_OP_LSE_IDX_LOCAL, dims, dev)
+    ws = _ws(ws, MSA_OP_LSE_IDX_LOCAL, dims, dev)
     _check("msa_lse_idx_local", lib().msa_lse_idx_local(ctypes.byref(dims.c()), _p(q_idx), _p(k_idx_local), tok0, ntok,
-                                                        _p(blocks), _p(ml), _p(ws), ws.numel(), _stream(stream)))
+                                                        _p(blocks), _p(ml), _p(ws), ws.numel(), _stream(stream, dev)))
     return ml
 
 
@@ -334,7 +347,7 @@ def msa_lse_combine(dims: MsaDims, ml, stream=None):
     P = ml.shape[0]
     _need(ml, "ml", (P, dims.B, dims.N, dims.H_kv, 2), torch.float32, ml.device)
     lse = torch.empty(dims.B, dims.N, dims.H_kv, dtype=torch.float32, device=ml.device)
-    _check("msa_lse_combine", lib().msa_lse_combine(ctypes.byref(dims.c()), P, _p(ml), _p(lse), _stream(stream)))
+    _check("msa_lse_combine", lib().msa_lse_combine(ctypes.byref(dims.c()), P, _p(ml), _p(lse), _stream(stream, ml.device)))
     return lse
 
 
@@ -353,12 +366,11 @@ def msa_kl_fwd_grad(dims: MsaDims, q, k, q_idx, k_idx, blocks, lse, lse_idx=None
     loss = torch.empty(1, dtype=torch.float32, device=dev)
     dq = torch.empty(dims.B, dims.N, dims.H_kv, dims.d_idx, dtype=torch.float32, device=dev)
     dk = torch.empty(dims.B, dims.N, dims.d_idx, dtype=torch.float32, device=dev)
-    if ws is None:
-        ws = workspace(MSA_OP_KL, dims, dev)
+    ws = _ws(ws, MSA_OP_KL, dims, dev)
     _check("msa_kl_fwd_grad",
            lib().msa_kl_fwd_grad(ctypes.byref(dims.c()), _p(q), _p(k), _p(q_idx), _p(k_idx), _p(blocks), _p(lse),
                                  _p(lse_idx), ctypes.c_float(grad_scale), _p(loss), _p(dq), _p(dk), _p(ws),
-                                 ws.numel(), _stream(stream)))
+                                 ws.numel(), _stream(stream, dev)))
     return loss, dq, dk
 
 
@@ -381,7 +393,7 @@ def msa_profile_read() -> dict:
 
 def msa_get_device_status(ws: torch.Tensor, stream=None) -> int:
     """Synchronise the stream and return the status code recorded by the last call using `ws`."""
-    return lib().msa_get_device_status(_p(ws), _stream(stream))
+    return lib().msa_get_device_status(_p(ws), _stream(stream, ws.device))
 
 
 __all__ = ["MsaDims", "MsaError", "msa_workspace_size", "msa_index_topk", "msa_sparse_attn_fwd",

@@ -82,3 +82,54 @@ def test_null_and_misaligned_pointers_are_rejected_on_the_host():
     assert L.msa_kl_fwd_grad(ctypes.byref(d2.c()), *([P(0x1000)] * 7), ctypes.c_float(1.0), P(0x1000), P(0x1000),
                              P(0x1000), P(0x10000), 1 << 30, None) == msa.MSA_ERR_UNSUPPORTED
     assert L.msa_get_device_status(None, None) == msa.MSA_ERR_INVALID_ARG
+
+
+def test_bindings_reject_host_tensors():
+    """The library takes device pointers: every binding refuses host tensors before any call into
+    it (a host pointer handed to a kernel would be an illegal address on the GPU)."""
+    import torch
+    d = dims()
+    bf = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)
+    blocks = torch.zeros(1, 512, 2, 5, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        msa.msa_index_topk(d, bf(1, 512, 2, 32), bf(1, 512, 32))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        msa.msa_sparse_attn_fwd(d, bf(1, 512, 4, 64), bf(1, 512, 2, 64), bf(1, 512, 2, 64), blocks)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        msa.msa_sparse_attn_decode(d, torch.ones(1, dtype=torch.int32), bf(1, 4, 64), bf(1, 2, 32),
+                                   bf(1, 512, 2, 64), bf(1, 512, 2, 64), bf(1, 512, 32))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        msa.msa_quantize_e4m3_rows(bf(8, 64))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        msa.msa_topk_merge(d, torch.zeros(2, 1, 512, 2, 4), torch.zeros(2, 1, 512, 2, 4, dtype=torch.int32))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        msa.msa_lse_combine(d, torch.zeros(2, 1, 512, 2, 2))
+
+
+def test_stream_device_and_workspace_checks(monkeypatch):
+    """Launches go to the current CUDA device: tensors or a stream of another device are refused,
+    and a caller's workspace must be a contiguous uint8 tensor on the inputs' device (host logic,
+    checked with a stand-in for the current device and stream)."""
+    import torch
+
+    class FakeStream:
+        def __init__(self, idx):
+            self.device = torch.device("cuda", idx)
+            self.cuda_stream = 0x1234
+
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda *a: FakeStream(0))
+    assert msa._stream(None, torch.device("cuda", 0)).value == 0x1234
+    assert msa._stream(FakeStream(0), torch.device("cuda", 0)).value == 0x1234
+    with pytest.raises(ValueError, match="current CUDA device"):
+        msa._stream(None, torch.device("cuda", 1))
+    with pytest.raises(ValueError, match="current CUDA device"):
+        msa._stream(None, torch.device("cpu"))
+    with pytest.raises(ValueError, match="stream belongs"):
+        msa._stream(FakeStream(1), torch.device("cuda", 0))
+    with pytest.raises(ValueError, match="ws must be"):
+        msa._ws(torch.zeros(64, dtype=torch.int32), msa.MSA_OP_DECODE, dims(), torch.device("cpu"))
+    with pytest.raises(ValueError, match="ws must be"):
+        msa._ws(torch.zeros(64, 4, dtype=torch.uint8)[:, 0], msa.MSA_OP_DECODE, dims(), torch.device("cpu"))
+    ws = torch.zeros(256, dtype=torch.uint8)
+    assert msa._ws(ws, msa.MSA_OP_DECODE, dims(), torch.device("cpu")) is ws
