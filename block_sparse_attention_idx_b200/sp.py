@@ -34,9 +34,25 @@ def gather(t: torch.Tensor, group=None) -> torch.Tensor:
 def sp_index_topk(dims: MsaDims, q_idx, k_idx_local, tok0: int, want_lse: bool = False, group=None):
     """Selection blocks [B, N, H_kv, topk+1] (and LSE_idx [B, N, H_kv]) of all N tokens from this
     rank's key range; q_idx [B, N, H_kv, d_idx] is replicated on every rank."""
-    cs, ci = msa_index_topk_local(dims, q_idx, k_idx_local, tok0)
+    empty = k_idx_local.shape[1] == 0  # more ranks than blocks: this rank holds no key
+    cs, ci = no_candidates(dims, q_idx.device) if empty else msa_index_topk_local(dims, q_idx, k_idx_local, tok0)
     blocks = msa_topk_merge(dims, gather(cs, group), gather(ci, group))
     if not want_lse:
         return blocks
-    ml = msa_lse_idx_local(dims, q_idx, k_idx_local, tok0, blocks)
+    ml = no_lse_pairs(dims, q_idx.device) if empty else msa_lse_idx_local(dims, q_idx, k_idx_local, tok0, blocks)
     return blocks, msa_lse_combine(dims, gather(ml, group))
+
+
+def no_candidates(dims: MsaDims, device):
+    """The candidates of a rank that holds no key: scores -inf and ids -1 [B, N, H_kv, topk], the
+    padding of a row without candidates."""
+    shape = (dims.B, dims.N, dims.H_kv, dims.topk)
+    return (torch.full(shape, float("-inf"), dtype=torch.float32, device=device),
+            torch.full(shape, -1, dtype=torch.int32, device=device))
+
+
+def no_lse_pairs(dims: MsaDims, device):
+    """The (max, exp-sum) pairs of a rank that holds no key: (-inf, 0), which eq (16) ignores."""
+    ml = torch.zeros(dims.B, dims.N, dims.H_kv, 2, dtype=torch.float32, device=device)
+    ml[..., 0] = float("-inf")
+    return ml

@@ -69,3 +69,28 @@ def test_sp_exchange_on_gloo_ranks(tmp_path, world):
     for r in res:
         assert r["blocks_equal"]
         assert r["lse_err"] <= 1e-12
+
+
+def test_rank_without_keys_contributes_padding_only():
+    """With more ranks than blocks a rank holds no key: its candidates are the padding the oracle
+    gives for an empty range (-inf, -1), its (max, exp-sum) pairs are (-inf, 0), and adding such a
+    rank changes neither the merged selection nor eq (16)."""
+    sys.path.insert(0, ROOT)
+    import oracle
+    from oracle import sp as osp
+    from block_sparse_attention_idx_b200 import sp
+    from msa_inputs import small_prefill
+    N, Bk, k, Hkv = 40, 8, 3, 2
+    dims = oracle.Dims(B=1, N=N, H_q=2 * Hkv, H_kv=Hkv, d=8, d_idx=8, block_k=Bk, topk=k)
+    x = small_prefill(N, 2 * Hkv, Hkv, 8, 8, Bk, k, seed=5)
+    assert sp.split_range(N, Bk, 8, 0)[1] == 0  # 5 blocks over 8 ranks: rank 0 holds none
+    cs, ci = sp.no_candidates(dims, torch.device("cpu"))
+    ocs, oci = osp.local_topk(dims, x["q_idx"], x["k_idx"], 3, 3)
+    np.testing.assert_array_equal(cs.double().numpy(), ocs)
+    np.testing.assert_array_equal(ci.numpy(), oci)
+    full_s, full_i = osp.local_topk(dims, x["q_idx"], x["k_idx"], 0, 5)
+    np.testing.assert_array_equal(osp.merge(dims, [full_s, ocs], [full_i, oci]), osp.merge(dims, [full_s], [full_i]))
+    ml = sp.no_lse_pairs(dims, torch.device("cpu")).double().numpy()
+    blocks = osp.merge(dims, [full_s], [full_i])
+    own = osp.local_lse(dims, x["q_idx"], x["k_idx"], blocks, 0, 5)
+    np.testing.assert_array_equal(osp.combine_lse([own, ml]), osp.combine_lse([own]))
