@@ -12,14 +12,30 @@ GRAD_MAX = 1e-3
 GRAD_REL = 2e-3  # stricter check used alongside: max error relative to the largest gradient entry
 
 
+# Near-tie rows excluded by each selection comparison of the session, as (test id, (row, group)
+# pairs compared, near-tie pairs, near-tie pairs whose selection differs); printed at the end of the
+# run by the terminal summary in conftest.py.
+CURRENT_TEST = ""
+NEAR_TIE_LOG = []
+# Achieved errors that a test chooses to report (printed with the near-tie summary).
+REPORT_LOG = []
+
+
+def report(line: str) -> None:
+    REPORT_LOG.append((CURRENT_TEST, line))
+
+
 def compare_blocks(gpu_blocks, ora_blocks, margin):
     """Bit-exact equality of the selected block ids for every (row, group) whose cutoff margin is
-    >= NEAR_TIE; returns (number of mismatching rows outside near-ties, number of near-tie rows)."""
+    >= NEAR_TIE; returns (number of mismatching rows outside near-ties, number of near-tie rows).
+    The near-tie count of every comparison is logged for the session report."""
     g = np.asarray(gpu_blocks).reshape(-1, gpu_blocks.shape[-1])
     o = np.asarray(ora_blocks).reshape(-1, ora_blocks.shape[-1])
     m = np.asarray(margin).reshape(-1)
     near = m < NEAR_TIE
-    bad = np.any(g != o, axis=1) & ~near
+    differ = np.any(g != o, axis=1)
+    bad = differ & ~near
+    NEAR_TIE_LOG.append((CURRENT_TEST, int(g.shape[0]), int(near.sum()), int((differ & near).sum())))
     return int(bad.sum()), int(near.sum())
 
 

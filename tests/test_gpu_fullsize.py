@@ -18,11 +18,19 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def sampled_rows(N, n=40, seed=0):
-    """First and last rows, rows at block edges, and uniformly drawn rows."""
+def sampled_rows(N, n=40, seed=0, carry=None, n_carry=12):
+    """First and last rows, rows at block edges, and uniformly drawn rows. With `carry` (the needle
+    workload's mask of query rows that carry the needle direction), n_carry of those rows and as
+    many of the others are added: the carrying rows select the hot needle blocks, block 0 among
+    them, so the sample always reaches the hot-block path."""
     rng = np.random.default_rng(seed)
     rows = {0, 1, 127, 128, 129, N // 2, N - 2, N - 1}
     rows |= set(rng.choice(N, size=n, replace=False).tolist())
+    if carry is not None:
+        c = np.asarray(carry).reshape(-1)[:N]
+        for pool in (np.flatnonzero(c), np.flatnonzero(~c)):
+            pool = pool[pool >= 128 * 16]  # rows with more complete past blocks than topk
+            rows |= set(rng.choice(pool, size=min(n_carry, len(pool)), replace=False).tolist())
     return np.array(sorted(r for r in rows if 0 <= r < N), dtype=np.int64)
 
 
@@ -71,7 +79,15 @@ def check_sampled_prefill(w, x, blocks, out, lse, rows):
 def test_full_prefill_sampled_rows_match_oracle(wname):
     w = WORKLOADS[wname]
     dm, x, blocks, _, out, lse = run_prefill(w)
-    check_sampled_prefill(w, x, blocks, out, lse, sampled_rows(w.N, seed=w.cid))
+    carry = x["needle_rows"].cpu().numpy() if w.needles else None
+    rows = sampled_rows(w.N, seed=w.cid, carry=carry)
+    if w.needles:
+        # the sample reaches the hot blocks: some sampled rows select block 0 and other needle blocks
+        gb = blocks.cpu().numpy().reshape(w.B * w.N, w.H_kv, w.topk + 1)[rows]
+        needles = set(x["needle_blocks"].cpu().tolist())
+        assert (gb == 0).any(axis=(1, 2)).sum() >= 8
+        assert np.isin(gb, list(needles - {0})).any(axis=(1, 2)).sum() >= 8
+    check_sampled_prefill(w, x, blocks, out, lse, rows)
 
 
 def test_full_training_step_sampled_rows_and_invariants():
