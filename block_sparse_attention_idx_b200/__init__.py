@@ -83,6 +83,12 @@ def lib() -> ctypes.CDLL:
         L.msa_sparse_attn_decode_noalloc.argtypes = [D, P, P, P, P, P, P, P, P, P]
         L.msa_sparse_attn_decode_noalloc.restype = ctypes.c_int
         L.msa_get_device_status.argtypes = [P, P]
+        L.msa_decode_noalloc_status.argtypes = [P]
+        L.msa_decode_noalloc_status.restype = ctypes.c_int
+        L.msa_debug_set_wait_ns.argtypes = [ctypes.c_ulonglong]
+        L.msa_debug_set_wait_ns.restype = None
+        L.msa_debug_wait_probe.argtypes = [P, S, P]
+        L.msa_debug_wait_probe.restype = ctypes.c_int
         L.msa_profile_enable.argtypes = [ctypes.c_int]
         L.msa_profile_enable.restype = None
         L.msa_profile_read.argtypes = [ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
@@ -396,8 +402,28 @@ def msa_get_device_status(ws: torch.Tensor, stream=None) -> int:
     return lib().msa_get_device_status(_p(ws), _stream(stream, ws.device))
 
 
+def msa_decode_noalloc_status(stream=None) -> int:
+    """Synchronise the stream and return the status code of the last allocation-free decode call on
+    the current device (its status word lives in the library's static scratch array)."""
+    return lib().msa_decode_noalloc_status(_stream(stream, torch.device("cuda", torch.cuda.current_device())))
+
+
+def msa_debug_set_wait_ns(ns: int) -> None:
+    """Test hook: time limit (ns) of every bounded device wait of later calls (0: the 2 s default)."""
+    lib().msa_debug_set_wait_ns(int(ns))
+
+
+def msa_debug_wait_probe(ws: torch.Tensor, stream=None) -> None:
+    """Test hook: enqueue the launch whose bounded wait can only run out (status MSA_ERR_TIMEOUT).
+    ws: a uint8 CUDA tensor of at least 256 + 4096 bytes."""
+    if ws.dtype != torch.uint8 or not ws.is_contiguous() or ws.device.type != "cuda":
+        raise ValueError("ws must be a contiguous uint8 CUDA tensor")
+    _check("msa_debug_wait_probe", lib().msa_debug_wait_probe(_p(ws), ws.numel(), _stream(stream, ws.device)))
+
+
 __all__ = ["MsaDims", "MsaError", "msa_workspace_size", "msa_index_topk", "msa_sparse_attn_fwd",
            "msa_sparse_attn_decode", "msa_sparse_attn_decode_noalloc", "msa_sparse_attn_decode_fp8idx",
            "msa_quantize_e4m3_rows", "msa_kl_fwd_grad", "msa_sparse_attn_bwd", "msa_index_topk_local",
            "msa_topk_merge", "msa_lse_idx_local", "msa_lse_combine", "msa_get_device_status", "msa_status_string",
-           "msa_version", "msa_profile_enable", "msa_profile_read", "workspace", "lib", "LIB_PATH"]
+           "msa_version", "msa_profile_enable", "msa_profile_read", "msa_decode_noalloc_status",
+           "msa_debug_set_wait_ns", "msa_debug_wait_probe", "workspace", "lib", "LIB_PATH"]

@@ -3,6 +3,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "msa.h"
 #include "msa_common.cuh"
 #include "msa_internal.h"
@@ -90,6 +92,18 @@ msa_status ws_check(const void* ws, size_t have, size_t need) {
 
 msa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
 
+// Wait limit that the test hook msa_debug_set_wait_ns put in place (0: the default, nothing to do).
+std::atomic<unsigned long long> g_wait_ns{0};
+
+// Clears a call's status word on its stream; with the test hook set, also writes the shorter limit
+// of the call's bounded waits.
+cudaError_t status_init(DevStatus* status, cudaStream_t st) {
+    cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, st);
+    const unsigned long long w = g_wait_ns.load(std::memory_order_relaxed);
+    if (e == cudaSuccess && w != 0) e = run_set_wait(status, w, st);
+    return e;
+}
+
 struct Carver {
     uint8_t* p;
     uint8_t* take(size_t bytes) {
@@ -151,7 +165,7 @@ msa_status msa_index_topk(const msa_dims* d, const void* q_idx, const void* k_id
     if (s != MSA_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_);
     DevStatus* status = static_cast<DevStatus*>(ws);
-    cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, st);
+    cudaError_t e = status_init(status, st);
     if (e != cudaSuccess) return MSA_ERR_CUDA;
     IndexArgs a{d->B, d->N, d->H_kv, d->d_idx, d->block_k, d->topk, blocks, status, 0, d->N, nullptr, nullptr};
     e = run_index_topk(a, q_idx, k_idx, st);
@@ -186,7 +200,7 @@ msa_status msa_sparse_attn_fwd(const msa_dims* d, const void* q, const void* k, 
     if (s != MSA_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_);
     DevStatus* status = static_cast<DevStatus*>(ws);
-    cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, st);
+    cudaError_t e = status_init(status, st);
     if (e != cudaSuccess) return MSA_ERR_CUDA;
     AttnArgs a{};
     a.B = d->B; a.N = d->N; a.H_q = d->H_q; a.H_kv = d->H_kv; a.d = d->d; a.block_k = d->block_k;
@@ -217,7 +231,7 @@ static msa_status decode_step(const msa_dims* d, const int32_t* cache_len, const
     if (s != MSA_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_);
     DevStatus* status = static_cast<DevStatus*>(ws);
-    cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, st);
+    cudaError_t e = status_init(status, st);
     if (e != cudaSuccess) return MSA_ERR_CUDA;
     Carver cv{static_cast<uint8_t*>(ws) + kStatusBytes};
     const size_t nb = (size_t)(d->N + d->block_k - 1) / d->block_k;
@@ -284,7 +298,7 @@ msa_status msa_index_topk_local(const msa_dims* d, const void* q_idx, const void
     if (s != MSA_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_);
     DevStatus* status = static_cast<DevStatus*>(ws);
-    cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, st);
+    cudaError_t e = status_init(status, st);
     if (e != cudaSuccess) return MSA_ERR_CUDA;
     IndexArgs a{d->B, d->N, d->H_kv, d->d_idx, d->block_k, d->topk, nullptr, status, tok0, ntok, cand_scores, cand_ids};
     return cuda_status(run_index_topk(a, q_idx, k_idx_local, st));
@@ -312,7 +326,7 @@ msa_status msa_lse_idx_local(const msa_dims* d, const void* q_idx, const void* k
     if (s != MSA_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_);
     DevStatus* status = static_cast<DevStatus*>(ws);
-    cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, st);
+    cudaError_t e = status_init(status, st);
     if (e != cudaSuccess) return MSA_ERR_CUDA;
     Carver cv{static_cast<uint8_t*>(ws) + kStatusBytes};
     KlArgs k{};
@@ -358,7 +372,7 @@ msa_status msa_sparse_attn_bwd(const msa_dims* d, const void* q, const void* k, 
     if (s != MSA_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_);
     DevStatus* status = static_cast<DevStatus*>(ws);
-    cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, st);
+    cudaError_t e = status_init(status, st);
     if (e != cudaSuccess) return MSA_ERR_CUDA;
     Carver cv{static_cast<uint8_t*>(ws) + kStatusBytes};
     BwdArgs a{};
@@ -393,7 +407,7 @@ msa_status msa_kl_fwd_grad(const msa_dims* d, const void* q, const void* k, cons
     if (s != MSA_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_);
     DevStatus* status = static_cast<DevStatus*>(ws);
-    cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, st);
+    cudaError_t e = status_init(status, st);
     if (e != cudaSuccess) return MSA_ERR_CUDA;
     Carver cv{static_cast<uint8_t*>(ws) + kStatusBytes};
     const size_t nb = (size_t)(d->N + d->block_k - 1) / d->block_k;
@@ -432,6 +446,18 @@ msa_status msa_kl_fwd_grad(const msa_dims* d, const void* q, const void* k, cons
         a.lse_idx = const_cast<float*>(lse_idx);
     }
     if (e == cudaSuccess) e = run_kl(a, q, k, q_idx, k_idx, num_sms(), st);
+    return cuda_status(e);
+}
+
+void msa_debug_set_wait_ns(unsigned long long ns) { g_wait_ns.store(ns, std::memory_order_relaxed); }
+
+msa_status msa_debug_wait_probe(void* ws, size_t ws_bytes, msa_stream_t stream_) {
+    msa_status s = ws_check(ws, ws_bytes, kStatusBytes + wait_probe_bytes());
+    if (s != MSA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_);
+    DevStatus* status = static_cast<DevStatus*>(ws);
+    cudaError_t e = status_init(status, st);
+    if (e == cudaSuccess) e = run_wait_probe(static_cast<uint8_t*>(ws) + kStatusBytes, status, st);
     return cuda_status(e);
 }
 

@@ -271,6 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int pend_pv = -1;         // PV issued whose item's successor group was not yet known
             int grp_ring[kMeta] = {0, 0, 0, 0};
             uint64_t t_idle = globaltimer();
+            const uint64_t lim = wait_limit(a.status);
             while (true) {
                 bool progressed = false;
                 if (n_end < 0) {
@@ -353,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 } else {
                     __nanosleep(20);
                 }
-                if (!progressed && globaltimer() - t_idle > MSA_WAIT_NS) {
+                if (!progressed && globaltimer() - t_idle > lim) {
                     raise_flag(a.status, MSA_DEV_TIMEOUT, 0x601);
                     ok = false;
                     break;

@@ -52,8 +52,11 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 struct ScanCursor {
     int b, blk, nbv;  // current item: block blk of sequence b, which has nbv complete past blocks
 };
+// cache_len[b] clamped to [1, L]: every kernel reads the length through this, so a value outside
+// the caches' capacity can never index past them (the Top-k kernel reports it).
+__device__ __forceinline__ int dec_len(const DecodeArgs& a, int b) { return min(max(a.cache_len[b], 1), a.L); }
 __device__ __forceinline__ int complete_blocks(const DecodeArgs& a, int b, int BK) {
-    return max(a.cache_len[b] - 1, 0) / BK;
+    return (dec_len(a, b) - 1) / BK;
 }
 // Called by all lanes of a warp: sets c to the CTA's first item, returns its number of items.
 __device__ int scan_range(const DecodeArgs& a, int BK, ScanCursor& c) {
@@ -427,7 +430,8 @@ __global__ void __launch_bounds__(256) k_dec_topk(DecodeArgs a) {
     __shared__ int chosen[kMaxK];
     pdl_wait();  // the block maxima come from the scan
     const int b = blockIdx.x / a.H_kv, r = blockIdx.x % a.H_kv;
-    const int len = a.cache_len[b];
+    const int len = dec_len(a, b);
+    if (threadIdx.x == 0 && r == 0 && len != a.cache_len[b]) raise_flag(a.status, MSA_DEV_BAD_BLOCK, 0x931);
     const int bi = (len - 1) / a.block_k;  // local block; candidates are 0 .. bi-1
     const int nb = (a.L + a.block_k - 1) / a.block_k;
     const float* vals = a.bmax + ((size_t)b * a.H_kv + r) * nb;
@@ -670,7 +674,7 @@ __global__ void __launch_bounds__((kAttnWarps + 1) * 32, 1)
             continue;
         }
         const int b = (it / K1) / a.H_kv;
-        const int len = a.cache_len[b];
+        const int len = dec_len(a, b);
         const int st = n % kAttnStages;
         const uint32_t kbase = smem_u32(&s.kv[st][0][0]), vbase = smem_u32(&s.kv[st][1][0]);
         float* o_out = a.o_part + (size_t)it * G * D;

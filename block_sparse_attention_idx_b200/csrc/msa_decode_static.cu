@@ -44,6 +44,14 @@ msa_status scratch_address(void** out) {
 
 }  // namespace
 
+// Status word of the last call on the current device: the first bytes of the static array.
+extern "C" msa_status msa_decode_noalloc_status(msa_stream_t stream) {
+    void* scratch = nullptr;
+    msa_status s = scratch_address(&scratch);
+    if (s != MSA_OK) return s;
+    return msa_get_device_status(scratch, stream);
+}
+
 extern "C" msa_status msa_sparse_attn_decode_noalloc(const msa_dims* dims, const int32_t* cache_len, const void* q,
                                                       const void* q_idx, const void* k_cache, const void* v_cache,
                                                       const void* k_idx_cache, float* out, int32_t* blocks_out,

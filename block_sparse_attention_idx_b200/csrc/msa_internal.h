@@ -171,4 +171,11 @@ cudaError_t run_quantize_e4m3_rows(const void* x, int64_t rows, int n, uint8_t* 
 cudaError_t run_decode(const DecodeArgs& a, const void* q, const void* q_idx, const void* k_cache, const void* v_cache,
                        const void* k_idx_cache, void* out, int num_sms, cudaStream_t st);
 
+// ---------------------------------------------------------------- test hooks (msa_debug.cu)
+// Writes a wait limit (ns) into a cleared status word; the launch whose bounded wait can only run
+// out (reads wait_probe_bytes() bytes at `src`).
+cudaError_t run_set_wait(DevStatus* st, unsigned long long ns, cudaStream_t s);
+size_t wait_probe_bytes();
+cudaError_t run_wait_probe(const void* src, DevStatus* st, cudaStream_t s);
+
 }  // namespace msa

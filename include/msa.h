@@ -190,7 +190,8 @@ MSA_API msa_status msa_sparse_attn_bwd(const msa_dims *dims, const void *q, cons
  * and K_idx are already in the caches at position cache_len[b]-1 (MSA blog, decode; the pages'
  * rule that decode and prefill compute the same R_theta and A_phi).
  *   dims->N    cache capacity L (rows of the caches)
- *   cache_len  int32 [B] device, 1 <= cache_len[b] <= N
+ *   cache_len  int32 [B] device, 1 <= cache_len[b] <= N. A value outside [1, N] is clamped into it
+ *              on the device and reported as MSA_ERR_DEVICE_CHECK by msa_get_device_status.
  *   q          bf16 [B, H_q, d];  q_idx bf16 [B, H_kv, d_idx]
  *   k_cache, v_cache bf16 [B, N, H_kv, d];  k_idx_cache bf16 [B, N, d_idx]
  *   out        fp32 [B, H_q, d]: the fp32-accumulated result        (output)
@@ -279,20 +280,47 @@ MSA_API msa_status msa_kl_fwd_grad(const msa_dims *dims, const void *q, const vo
  *   (cudaGetSymbolAddress); make that first call before any stream capture.
  * - All calls on one device share the array and it keeps the last call's contents; calls that can
  *   overlap on the GPU (unordered streams) race on it and must be serialised by the caller.
- * - The device status word of these calls lives in the shared array; it cannot be read with
- *   msa_get_device_status.
+ * - The device status word of these calls lives in the shared array: read it with
+ *   msa_decode_noalloc_status, not msa_get_device_status.
+ * - The array's device address is cached per device ordinal for the life of the process: the
+ *   entry point assumes the device's primary context (the one the CUDA runtime uses) throughout,
+ *   with no cudaDeviceReset in between.
  */
 #define MSA_DECODE_STATIC_SCRATCH_BYTES (16u << 20)
 MSA_API msa_status msa_sparse_attn_decode_noalloc(const msa_dims *dims, const int32_t *cache_len, const void *q,
                                                   const void *q_idx, const void *k_cache, const void *v_cache,
                                                   const void *k_idx_cache, float *out, int32_t *blocks_out,
                                                   msa_stream_t stream);
+/*
+ * Device status of the last msa_sparse_attn_decode_noalloc call on the current device: synchronises
+ * `stream`, then reads the status word in the static array. MSA_OK, MSA_ERR_TIMEOUT or
+ * MSA_ERR_DEVICE_CHECK (MSA_ERR_CUDA if the stream holds an error or the lookup fails). It
+ * allocates nothing.
+ */
+MSA_API msa_status msa_decode_noalloc_status(msa_stream_t stream);
 
 /*
  * Synchronises `stream`, then reads the device status word of the last call that used `ws`:
  * MSA_OK, MSA_ERR_TIMEOUT or MSA_ERR_DEVICE_CHECK (or MSA_ERR_CUDA if the stream holds an error).
  */
 MSA_API msa_status msa_get_device_status(const void *ws, msa_stream_t stream);
+
+/*
+ * Test hooks of the failure-detection path (no counterpart in the pages). Every wait inside a
+ * kernel of this library (an mbarrier, a copy or MMA completion, a work-queue poll) is bounded by
+ * a time limit, 2 s by default. A wait that runs out sets MSA_ERR_TIMEOUT in the call's status
+ * word; the kernel drains the copies and MMAs it issued, frees its TMEM and returns, leaving the
+ * context usable.
+ * msa_debug_set_wait_ns: the limit (ns) of every bounded wait of the calls made after it, in all
+ *   threads of the process; 0 restores the default. For tests only: a short limit turns ordinary
+ *   latency into timeouts.
+ * msa_debug_wait_probe: one launch whose consumer waits on an mbarrier that its producer never
+ *   arrives on, while the producer's bulk copy of 4096 bytes (read from ws + 256) is in flight and
+ *   the CTA holds TMEM. The wait can only run out: msa_get_device_status(ws) then returns
+ *   MSA_ERR_TIMEOUT. ws: at least 256 + 4096 bytes, 256-byte aligned (MSA_ERR_WORKSPACE otherwise).
+ */
+MSA_API void msa_debug_set_wait_ns(unsigned long long ns);
+MSA_API msa_status msa_debug_wait_probe(void *ws, size_t ws_bytes, msa_stream_t stream);
 
 /*
  * Kernel timing (off by default). While enabled, every entry point records a pair of CUDA events
