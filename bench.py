@@ -275,6 +275,27 @@ def rank_seed(w, rank: int) -> int:
     return 1000 + w.cid + 7919 * rank
 
 
+def workload_config(w, world: int) -> dict:
+    """The `config` object of the JSON line (the same in both arms)."""
+    return {"workload": w.name, "N": w.N, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d, "d_idx": w.d_idx,
+            "block_k": w.block_k, "topk": w.topk, "batch_per_gpu": w.B, "global_batch": w.B * world,
+            "parallelism": f"dp{world} (independent sequences)",
+            "l2": "flushed (256 MiB read) before every timed step; inputs also larger than L2; the pipelined "
+                  "e2e steps are not flushed (625 MB uploaded per step)",
+            "step": "msa_index_topk + msa_sparse_attn_fwd"}
+
+
+def rnd(x, sig: int = 4):
+    """Floats rounded to `sig` significant digits, recursively (keeps the JSON line short)."""
+    if isinstance(x, float):
+        return float(f"{x:.{sig}g}") if math.isfinite(x) else x
+    if isinstance(x, dict):
+        return {k: rnd(v, sig) for k, v in x.items()}
+    if isinstance(x, (list, tuple)):
+        return [rnd(v, sig) for v in x]
+    return x
+
+
 def job_throughput(units_per_rank: float, world: int, slowest_ms: float) -> float:
     """Whole-job units per second: all ranks' units over the slowest rank's step time."""
     return units_per_rank * world / (slowest_ms * 1e-3)
@@ -307,21 +328,25 @@ def run_reference(args, world, rank):
         step()
     dt = time.perf_counter() - t0
     value = rows_per_step * args.steps / dt
-    sample = f"{rows_per_step} uniformly drawn query rows of {HEADLINE} per step (index Top-k + sparse attention)"
+    sample = (f"{rows_per_step} uniformly drawn query rows of {HEADLINE} per step (index Top-k + sparse "
+              f"attention); a step is one such sample, timed")
     return {"metric": METRIC, "value": value, "unit": "query-tokens/s", "n_gpus": args.gpus, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps * (w.N / rows_per_step),
+            "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+            # not a measurement: the time a whole N-row step would take at the sampled rate
+            "full_step_ms_extrapolated": 1e3 * dt / args.steps * (w.N / rows_per_step),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "impl": "reference",
-            "config": {"workload": args.workload, "N": w.N, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d, "d_idx": w.d_idx,
-                       "block_k": w.block_k, "topk": w.topk},
+            "data": "synthetic", "impl": "reference", "config": workload_config(w, world),
             "cpu_baseline": {"value": value, "unit": "query-tokens/s", "cores": oracle.num_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "query-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
 # ============================================================================ our arm
-def cpu_baseline(x, w, rows_n: int):
-    """The oracle as it stands on a bounded row sample of the same workload (rank 0, N=1)."""
+def cpu_baseline(x, w, rows_n: int, blocks=None, out=None):
+    """The oracle as it stands on a bounded row sample of the same workload (rank 0, N=1). With the
+    GPU's selection and output of the same inputs, also their parity on that sample: selection
+    (bit-exact except near-ties: cutoff margin < 1e-4, counted) and attention error on the rows
+    where both selected the same blocks."""
     import numpy as np
     import oracle
     od = oracle.Dims(w.B, w.N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
@@ -329,13 +354,31 @@ def cpu_baseline(x, w, rows_n: int):
     rows = np.sort(np.random.default_rng(1).choice(w.N, size=rows_n, replace=False))
     full = np.full((w.B, w.N, w.H_kv, w.topk + 1), -1, dtype=np.int32)
     t0 = time.perf_counter()
-    b, _, _ = oracle.index_topk(od, xc["q_idx"], xc["k_idx"], rows=rows)
+    b, margin, _ = oracle.index_topk(od, xc["q_idx"], xc["k_idx"], rows=rows)
     full[0, rows] = b
-    oracle.sparse_attn(od, xc["q"], xc["k"], xc["v"], full, rows=rows)
+    oo, _ = oracle.sparse_attn(od, xc["q"], xc["k"], xc["v"], full, rows=rows)
     dt = time.perf_counter() - t0
-    return {"value": rows_n / dt, "unit": "query-tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{rows_n} uniformly drawn query rows of {w.name} (index Top-k + sparse attention), "
-                      f"{dt:.1f} s"}
+    res = {"value": rows_n / dt, "unit": "query-tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+           "sample": f"{rows_n} uniformly drawn query rows of {w.name} (index Top-k + sparse attention), "
+                     f"{dt:.1f} s"}
+    par = None
+    if blocks is not None and out is not None:
+        rt = torch.from_numpy(rows).to(blocks.device)
+        gb = blocks.reshape(w.B * w.N, w.H_kv, w.topk + 1)[rt].cpu().numpy()
+        og = out.reshape(w.B * w.N, w.H_q, w.d)[rt].double().cpu().numpy()
+        near = margin < 1e-4
+        differ = (gb != b).any(axis=-1)
+        same = ~differ.any(axis=-1)
+        err = np.abs(og[same] - oo[same])
+        par = {"sample": f"the cpu_baseline rows ({rows_n} query rows x {w.H_kv} groups)",
+               "selection_pairs": int(gb.shape[0] * w.H_kv), "near_ties": int(near.sum()),
+               "near_ties_selected_differently": int((differ & near).sum()),
+               "mismatches_outside_near_ties": int((differ & ~near).sum()),
+               "attn_rows_compared": int(same.sum()),
+               "attn_max_abs_err": float(err.max()) if err.size else None,
+               "attn_mean_abs_err": float(err.mean()) if err.size else None,
+               "tolerance": "selection bit-exact outside near-ties; attention max abs 1e-2, mean abs 1e-3"}
+    return res, par
 
 
 def bench_prefill(args, world, rank, msa, pk):
@@ -427,7 +470,9 @@ def bench_prefill(args, world, rank, msa, pk):
            "work": {"selected_tokens": sel_tok, "mean_J": sel_tok / (w.N * w.H_kv), "attn_flops": attn_flops,
                     "index_flops": index_flops}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(x, w, args.cpu_rows)
+        blocks, (out, _) = step()
+        res["cpu_baseline"], res["parity"] = cpu_baseline(x, w, args.cpu_rows, blocks, out)
+        del blocks, out
     del ws_a, x
     torch.cuda.empty_cache()
     return res
@@ -711,20 +756,19 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": pre["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": args.workload, "N": w.N, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d, "d_idx": w.d_idx,
-                       "block_k": w.block_k, "topk": w.topk, "batch_per_gpu": w.B, "global_batch": w.B * world,
-                       "parallelism": f"dp{world} (independent sequences)",
-                       "l2": "flushed (256 MiB read) before every timed step; inputs also larger than L2; the pipelined e2e steps are not flushed (625 MB uploaded per step)",
-                       "step": "msa_index_topk + msa_sparse_attn_fwd"},
+            "config": workload_config(w, world),
             "roofline": pre["roofline"], "e2e": pre["e2e"], "gpu_launches": pre["gpu_launches"],
-            "clocks": pre["clocks"], "kernels": pre["kernels"], "work": pre["work"],
+            "clocks": pre["clocks"], "kernels": rnd(pre["kernels"]), "work": rnd(pre["work"]),
             "peaks": pk}
     if "cpu_baseline" in pre:
         line["cpu_baseline"] = pre["cpu_baseline"]
+        line["parity"] = rnd(pre["parity"])
     if not args.no_secondary:
-        line["decode"] = bench_decode(args, world, rank, msa, pk)
-        line["train"] = bench_train(args, world, rank, msa, pk)
-        line["sp_index"] = bench_sp(args, world, rank, msa, pk)
+        # the decode object goes last: the end of the line is what a truncated log keeps
+        dec = bench_decode(args, world, rank, msa, pk)
+        line["train"] = rnd(bench_train(args, world, rank, msa, pk))
+        line["sp_index"] = rnd(bench_sp(args, world, rank, msa, pk))
+        line["decode"] = rnd(dec)
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank == 0:
