@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libmsa.so")
 MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_WORKSPACE, MSA_ERR_CUDA, MSA_ERR_TIMEOUT, \
     MSA_ERR_DEVICE_CHECK = range(7)
 (MSA_OP_INDEX_TOPK, MSA_OP_INDEX_TOPK_LSE, MSA_OP_ATTN_FWD, MSA_OP_DECODE, MSA_OP_KL, MSA_OP_ATTN_BWD,
- MSA_OP_LSE_IDX_LOCAL) = range(7)
+ MSA_OP_LSE_IDX_LOCAL, MSA_OP_KL_DENSE) = range(8)
 
 
 class MsaError(RuntimeError):
@@ -74,6 +74,7 @@ def lib() -> ctypes.CDLL:
         L.msa_sparse_attn_decode_fp8idx.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, S, P]
         L.msa_quantize_e4m3_rows.argtypes = [P, ctypes.c_int64, ctypes.c_int, P, P, P]
         L.msa_kl_fwd_grad.argtypes = [D, P, P, P, P, P, P, P, ctypes.c_float, P, P, P, P, S, P]
+        L.msa_kl_dense_fwd_grad.argtypes = [D, P, P, P, P, ctypes.c_float, P, P, P, P, P, S, P]
         L.msa_sparse_attn_bwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, S, P]
         I = ctypes.c_int
         L.msa_index_topk_local.argtypes = [D, P, P, I, I, P, P, P, S, P]
@@ -100,7 +101,7 @@ def lib() -> ctypes.CDLL:
         for fn in ("msa_workspace_size", "msa_index_topk", "msa_sparse_attn_fwd", "msa_sparse_attn_decode",
                    "msa_sparse_attn_decode_fp8idx", "msa_quantize_e4m3_rows", "msa_kl_fwd_grad",
                    "msa_sparse_attn_bwd", "msa_index_topk_local", "msa_topk_merge", "msa_lse_idx_local",
-                   "msa_lse_combine", "msa_get_device_status"):
+                   "msa_lse_combine", "msa_get_device_status", "msa_kl_dense_fwd_grad"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -380,6 +381,27 @@ def msa_kl_fwd_grad(dims: MsaDims, q, k, q_idx, k_idx, blocks, lse, lse_idx=None
     return loss, dq, dk
 
 
+def msa_kl_dense_fwd_grad(dims: MsaDims, q, k, q_idx, k_idx, grad_scale: float = 1.0, want_lse: bool = False,
+                          ws=None, stream=None):
+    """Dense warm-up KL (every causal block selected). Returns (loss fp32 [1], dq_idx [B,N,H_kv,d_idx],
+    dk_idx [B,N,d_idx]) and, with want_lse, the teacher LSE fp32 [B,N,H_q]."""
+    dev = q.device
+    _need(q, "q", (dims.B, dims.N, dims.H_q, dims.d), torch.bfloat16, dev)
+    _need(k, "k", (dims.B, dims.N, dims.H_kv, dims.d), torch.bfloat16, dev)
+    _need(q_idx, "q_idx", (dims.B, dims.N, dims.H_kv, dims.d_idx), torch.bfloat16, dev)
+    _need(k_idx, "k_idx", (dims.B, dims.N, dims.d_idx), torch.bfloat16, dev)
+    ws = _ws(ws, MSA_OP_KL_DENSE, dims, dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    dq = torch.empty(dims.B, dims.N, dims.H_kv, dims.d_idx, dtype=torch.float32, device=dev)
+    dk = torch.empty(dims.B, dims.N, dims.d_idx, dtype=torch.float32, device=dev)
+    lse = torch.empty(dims.B, dims.N, dims.H_q, dtype=torch.float32, device=dev) if want_lse else None
+    _check("msa_kl_dense_fwd_grad",
+           lib().msa_kl_dense_fwd_grad(ctypes.byref(dims.c()), _p(q), _p(k), _p(q_idx), _p(k_idx),
+                                       ctypes.c_float(grad_scale), _p(loss), _p(dq), _p(dk), _p(lse), _p(ws),
+                                       ws.numel(), _stream(stream, dev)))
+    return (loss, dq, dk, lse) if want_lse else (loss, dq, dk)
+
+
 def msa_profile_enable(on: bool = True) -> None:
     """Record CUDA events around every kernel the library launches (on the launching stream)."""
     lib().msa_profile_enable(1 if on else 0)
@@ -426,4 +448,5 @@ __all__ = ["MsaDims", "MsaError", "msa_workspace_size", "msa_index_topk", "msa_s
            "msa_quantize_e4m3_rows", "msa_kl_fwd_grad", "msa_sparse_attn_bwd", "msa_index_topk_local",
            "msa_topk_merge", "msa_lse_idx_local", "msa_lse_combine", "msa_get_device_status", "msa_status_string",
            "msa_version", "msa_profile_enable", "msa_profile_read", "msa_decode_noalloc_status",
-           "msa_debug_set_wait_ns", "msa_debug_wait_probe", "workspace", "lib", "LIB_PATH"]
+           "msa_debug_set_wait_ns", "msa_debug_wait_probe", "msa_kl_dense_fwd_grad", "workspace", "lib",
+           "LIB_PATH"]

@@ -84,6 +84,34 @@ size_t ws_kl(const msa_dims* d) {
            al256(me * d->d_idx * 4) + al256(me * 8) + al256(rows_kv(d) * 8);
 }
 
+// Dense warm-up KL: teacher LSE, LSE_idx, the dense lists (shared entries, items of 128/G queries for
+// the KL and of kIdxQpc for LSE_idx), per-(row, block) (max, sum-exp) of the index logits, KL rows.
+struct DenseLayout {
+    long long entries, items_kl, items_idx;
+    size_t nb;
+};
+DenseLayout dense_layout(const msa_dims* d) {
+    DenseLayout L;
+    const int G = d->H_q / d->H_kv;
+    dense_list_sizes(d->B, d->N, d->H_kv, d->block_k, 128 / G, &L.entries, &L.items_kl);
+    long long e2 = 0;
+    dense_list_sizes(d->B, d->N, d->H_kv, d->block_k, kIdxQpc, &e2, &L.items_idx);
+    L.nb = (size_t)(d->N + d->block_k - 1) / d->block_k;
+    return L;
+}
+size_t ws_kl_dense(const msa_dims* d) {
+    const DenseLayout L = dense_layout(d);
+    const size_t nl = (size_t)d->B * d->H_kv * L.nb;
+    return kStatusBytes + al256((size_t)d->B * d->N * d->H_q * 4) + al256(rows_kv(d) * 4) +
+           al256((size_t)L.entries * 4) + al256((size_t)L.items_kl * 16) + al256((size_t)L.items_idx * 16) + 256 +
+           256 + al256(rows_kv(d) * L.nb * sizeof(float2)) + al256(rows_kv(d) * 8) + al256((nl + 1) * 4);
+}
+// The dense lists index entries and items with 31 bits.
+bool dense_fits(const msa_dims* d) {
+    const DenseLayout L = dense_layout(d);
+    return L.entries < 2147483647LL && L.items_kl < 2147483647LL && rows_kv(d) * L.nb < (1ull << 40);
+}
+
 msa_status ws_check(const void* ws, size_t have, size_t need) {
     if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MSA_ERR_WORKSPACE;
     if (have < need) return MSA_ERR_WORKSPACE;
@@ -149,6 +177,12 @@ msa_status msa_workspace_size(int op, const msa_dims* d, size_t* bytes) {
         case MSA_OP_ATTN_BWD:
             if (!bwd_supported(d->d, d->H_q / d->H_kv)) return MSA_ERR_UNSUPPORTED;
             *bytes = ws_bwd(d);
+            return MSA_OK;
+        case MSA_OP_KL_DENSE:
+            if (!kl_supported(d->d, d->d_idx, d->H_q / d->H_kv) ||
+                !dense_lse_supported(d->d, d->block_k, d->H_q / d->H_kv) || !dense_fits(d))
+                return MSA_ERR_UNSUPPORTED;
+            *bytes = ws_kl_dense(d);
             return MSA_OK;
     }
     return MSA_ERR_INVALID_ARG;
@@ -445,6 +479,68 @@ msa_status msa_kl_fwd_grad(const msa_dims* d, const void* q, const void* k, cons
     } else {
         a.lse_idx = const_cast<float*>(lse_idx);
     }
+    if (e == cudaSuccess) e = run_kl(a, q, k, q_idx, k_idx, num_sms(), st);
+    return cuda_status(e);
+}
+
+msa_status msa_kl_dense_fwd_grad(const msa_dims* d, const void* q, const void* k, const void* q_idx,
+                                 const void* k_idx, float grad_scale, float* loss, float* dq_idx, float* dk_idx,
+                                 float* lse_out, void* ws, size_t ws_bytes, msa_stream_t stream_) {
+    msa_status s = check_common(d);
+    if (s != MSA_OK) return s;
+    const int G = d->H_q / d->H_kv;
+    if (!kl_supported(d->d, d->d_idx, G) || !dense_lse_supported(d->d, d->block_k, G) || !dense_fits(d))
+        return MSA_ERR_UNSUPPORTED;
+    if (!q || !k || !q_idx || !k_idx || !loss || !dq_idx || !dk_idx || !aligned16(q) || !aligned16(k) ||
+        !aligned16(q_idx) || !aligned16(k_idx) || !aligned16(dq_idx) || !aligned16(dk_idx) ||
+        (lse_out && !aligned16(lse_out)))
+        return MSA_ERR_INVALID_ARG;
+    if (!isfinite(grad_scale)) return MSA_ERR_INVALID_ARG;
+    s = ws_check(ws, ws_bytes, ws_kl_dense(d));
+    if (s != MSA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_);
+    DevStatus* status = static_cast<DevStatus*>(ws);
+    cudaError_t e = status_init(status, st);
+    if (e != cudaSuccess) return MSA_ERR_CUDA;
+    const DenseLayout L = dense_layout(d);
+    const size_t nl = (size_t)d->B * d->H_kv * L.nb;
+    Carver cv{static_cast<uint8_t*>(ws) + kStatusBytes};
+    float* lse_ws = reinterpret_cast<float*>(cv.take((size_t)d->B * d->N * d->H_q * 4));
+    float* lse_main = lse_out ? lse_out : lse_ws;
+    float* lse_idx = reinterpret_cast<float*>(cv.take(rows_kv(d) * 4));
+    KlArgs a{};
+    a.B = d->B; a.N = d->N; a.H_q = d->H_q; a.H_kv = d->H_kv; a.d = d->d; a.d_idx = d->d_idx;
+    a.block_k = d->block_k; a.topk = d->topk;
+    a.scale = eff_scale(d->scale, d->d); a.scale_idx = eff_scale(d->scale_idx, d->d_idx);
+    a.grad_scale = grad_scale;
+    a.kv_tok0 = 0;
+    a.kv_ntok = d->N;
+    a.dense = 1;
+    // lists: one window per sequence (nW = 1), list (b, r, c) = queries c*block_k .. N-1
+    a.csr.nb = (int)L.nb;
+    a.csr.nW = 1;
+    a.csr.wq = d->N;
+    a.csr.nlists = (int)nl;
+    a.csr.entries = reinterpret_cast<int32_t*>(cv.take((size_t)L.entries * 4));
+    a.csr.items = reinterpret_cast<int4*>(cv.take((size_t)L.items_kl * 16));
+    a.csr_idx = a.csr;
+    a.csr_idx.items = reinterpret_cast<int4*>(cv.take((size_t)L.items_idx * 16));
+    a.csr.n_items = reinterpret_cast<int32_t*>(cv.take(256));
+    a.csr_idx.n_items = reinterpret_cast<int32_t*>(cv.take(256));
+    a.ml_part = reinterpret_cast<float2*>(cv.take(rows_kv(d) * L.nb * sizeof(float2)));
+    a.kl_rows = reinterpret_cast<double*>(cv.take(rows_kv(d) * 8));
+    a.lse = lse_main;
+    a.lse_idx = lse_idx;
+    a.dq_idx = dq_idx;
+    a.dk_idx = dk_idx;
+    a.loss = loss;
+    a.blocks = nullptr;
+    a.status = status;
+    DenseLseArgs dl{d->B, d->N, d->H_q, d->H_kv, G, d->d, d->block_k, a.scale, lse_main, status};
+    e = run_dense_lse(dl, q, k, num_sms(), st);
+    if (e == cudaSuccess) e = run_dense_lists(a.csr, d->B, d->N, d->H_kv, d->block_k, 128 / G, true, st);
+    if (e == cudaSuccess) e = run_dense_lists(a.csr_idx, d->B, d->N, d->H_kv, d->block_k, kIdxQpc, false, st);
+    if (e == cudaSuccess) e = run_lse_idx(a, q_idx, k_idx, num_sms(), st);
     if (e == cudaSuccess) e = run_kl(a, q, k, q_idx, k_idx, num_sms(), st);
     return cuda_status(e);
 }

@@ -142,6 +142,10 @@ struct KlArgs {
     // of lse_idx
     int kv_tok0, kv_ntok;
     float2* ml_out;     // [B, N, H_kv]
+    // dense warm-up: every causal block is selected; the lists come from run_dense_lists, the
+    // LSE_idx partial slot of an entry is its block (ml_part [B, N, H_kv, nb]), and dQ_idx / the
+    // KL rows are accumulated with atomics instead of per-slot partials (blocks is not read)
+    int dense;
 };
 constexpr int kIdxQpc = 32;
 bool kl_supported(int d, int d_idx, int G);
@@ -170,6 +174,21 @@ cudaError_t run_quantize_e4m3_rows(const void* x, int64_t rows, int n, uint8_t* 
 // k_idx_cache is bf16 [B, L, d_idx], or e4m3 codes [B, L, d_idx] when a.k_idx_scale is set.
 cudaError_t run_decode(const DecodeArgs& a, const void* q, const void* q_idx, const void* k_cache, const void* v_cache,
                        const void* k_idx_cache, void* out, int num_sms, cudaStream_t st);
+
+// ---------------------------------------------------------------- dense warm-up (msa_dense.cu)
+struct DenseLseArgs {
+    int B, N, H_q, H_kv, G, d, block_k;
+    float scale;
+    float* lse;          // [B, N, H_q] natural-log LSE over all causal keys
+    DevStatus* status;
+};
+bool dense_lse_supported(int d, int block_k, int G);
+cudaError_t run_dense_lse(const DenseLseArgs& a, const void* q, const void* k, int num_sms, cudaStream_t st);
+// Entry and item counts of the dense inverse lists (every query of block c and after, for every
+// (b, r, c)), and their build into a Csr carved with room for them (nb, nW = 1 set by csr_carve).
+void dense_list_sizes(int B, int N, int H_kv, int block_k, int qpc, long long* entries, long long* items);
+cudaError_t run_dense_lists(const Csr& cs, int B, int N, int H_kv, int block_k, int qpc, bool write_entries,
+                            cudaStream_t st);
 
 // ---------------------------------------------------------------- test hooks (msa_debug.cu)
 // Writes a wait limit (ns) into a cleared status word; the launch whose bounded wait can only run

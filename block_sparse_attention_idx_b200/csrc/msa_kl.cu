@@ -47,7 +47,9 @@ __global__ void __launch_bounds__(128) k_lse_idx(KlArgs a, const __nv_bfloat16* 
     const int t0 = blockIdx.x * per, t1 = min(T, t0 + per);
     const int tt = threadIdx.x, warp = tt >> 5, lane = tt & 31;
     const int g8 = lane >> 2, t4 = lane & 3;
-    const int K1 = a.topk + 1;
+    // partial slots per row: the selection's k+1, or every block of the sequence in dense mode
+    // (the slot of a dense entry is its block)
+    const int K1 = a.dense ? cs.nb : a.topk + 1;
     const uint32_t kb_u32 = smem_u32(kb), qb_u32 = smem_u32(qb);
     int curL = -1;
     for (int t = t0; t < t1; ++t) {
@@ -70,7 +72,7 @@ __global__ void __launch_bounds__(128) k_lse_idx(KlArgs a, const __nv_bfloat16* 
         if (tt < QP) {
             const int e = tt < count ? cs.entries[it.y + tt] : 0;
             s_i[tt] = tt < count ? (e >> 5) : -1;
-            s_slot[tt] = e & 31;
+            s_slot[tt] = a.dense ? c : (e & 31);
         }
         for (int x = tt; x < QP * (DI / 8); x += 128) {
             const int m = x / (DI / 8), part = x % (DI / 8);
@@ -164,8 +166,19 @@ __global__ void __launch_bounds__(128) k_lse_idx(KlArgs a, const __nv_bfloat16* 
 __global__ void k_lse_idx_merge(KlArgs a) {
     const long long row = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (row >= (long long)a.B * a.N * a.H_kv) return;
-    const int K1 = a.topk + 1;
     const int i = (int)((row / a.H_kv) % a.N);
+    if (a.dense) {
+        // every causal block 0 .. i / block_k, slot = block
+        const int nb = a.csr_idx.nb, nc = i / a.block_k + 1;
+        const float2* mp = a.ml_part + row * nb;
+        float mx = -INFINITY;
+        for (int c = 0; c < nc; ++c) mx = fmaxf(mx, mp[c].x);
+        float z = 0.f;
+        for (int c = 0; c < nc; ++c) z += mp[c].y * __expf(mp[c].x - mx);
+        a.lse_idx[row] = mx + logf(z);
+        return;
+    }
+    const int K1 = a.topk + 1;
     const int32_t* sel = a.blocks + row * K1;
     float mx = -INFINITY;
     int prev = -1;
@@ -793,9 +806,15 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
                             const int m = nt * 8 + 2 * t4 + cx;
                             if (m < count) {
                                 const int qe = s.ent[buf][m];
-                                const size_t pr = (((size_t)b * a.N + (qe >> 5)) * a.H_kv + r) * K1 + (qe & 31);
-                                a.dq_part[pr * DI + d0] = ch[cx] + cl[cx];
-                                a.dq_part[pr * DI + d0 + 8] = ch[2 + cx] + cl[2 + cx];
+                                const size_t row = ((size_t)b * a.N + (qe >> 5)) * a.H_kv + r;
+                                if (a.dense) {
+                                    atomicAdd(a.dq_idx + row * DI + d0, ch[cx] + cl[cx]);
+                                    atomicAdd(a.dq_idx + row * DI + d0 + 8, ch[2 + cx] + cl[2 + cx]);
+                                } else {
+                                    const size_t pr = row * K1 + (qe & 31);
+                                    a.dq_part[pr * DI + d0] = ch[cx] + cl[cx];
+                                    a.dq_part[pr * DI + d0 + 8] = ch[2 + cx] + cl[2 + cx];
+                                }
                             }
                         }
                     }
@@ -825,10 +844,17 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
                         const int m = nt * 8 + 2 * t4 + cx;
                         if (m < count) {
                             const int qe = s.ent[buf][m];
-                            const size_t pr = (((size_t)b * a.N + (qe >> 5)) * a.H_kv + r) * K1 + (qe & 31);
-                            a.dq_part[pr * DI + d0] = (cq[0][cx] + cq[1][cx]) + (cq[2][cx] + cq[3][cx]);
-                            a.dq_part[pr * DI + d0 + 8] =
-                                (cq[0][2 + cx] + cq[1][2 + cx]) + (cq[2][2 + cx] + cq[3][2 + cx]);
+                            const size_t row = ((size_t)b * a.N + (qe >> 5)) * a.H_kv + r;
+                            const float v0 = (cq[0][cx] + cq[1][cx]) + (cq[2][cx] + cq[3][cx]);
+                            const float v1 = (cq[0][2 + cx] + cq[1][2 + cx]) + (cq[2][2 + cx] + cq[3][2 + cx]);
+                            if (a.dense) {
+                                atomicAdd(a.dq_idx + row * DI + d0, v0);
+                                atomicAdd(a.dq_idx + row * DI + d0 + 8, v1);
+                            } else {
+                                const size_t pr = row * K1 + (qe & 31);
+                                a.dq_part[pr * DI + d0] = v0;
+                                a.dq_part[pr * DI + d0 + 8] = v1;
+                            }
                         }
                     }
                 }
@@ -842,8 +868,9 @@ __global__ void __launch_bounds__(kl_threads<G>(), 1)
                 for (int o = TPQ / 2; o; o >>= 1) kl += __shfl_xor_sync(0xffffffffu, kl, o);
                 if (part == 0 && m < count) {
                     const int qe = s.ent[buf][m];
-                    const size_t pr = (((size_t)b * a.N + (qe >> 5)) * a.H_kv + r) * K1 + (qe & 31);
-                    a.kl_part[pr] = (double)kl;
+                    const size_t row = ((size_t)b * a.N + (qe >> 5)) * a.H_kv + r;
+                    if (a.dense) atomicAdd(a.kl_rows + row, (double)kl);
+                    else a.kl_part[row * K1 + (qe & 31)] = (double)kl;
                 }
                 mbar_arrive(&s.meta_empty[buf]);
             }
@@ -967,19 +994,28 @@ cudaError_t run_kl(const KlArgs& a, const void* q, const void* k, const void* q_
     }
     cudaError_t e = cudaMemsetAsync(a.dk_idx, 0, (size_t)a.B * a.N * a.d_idx * 4, st);
     if (e != cudaSuccess) return e;
+    const long long rows = (long long)a.B * a.N * a.H_kv;
+    if (a.dense) {
+        // dQ_idx and the KL rows are accumulated by the kernel
+        e = cudaMemsetAsync(a.dq_idx, 0, (size_t)rows * a.d_idx * 4, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(a.kl_rows, 0, (size_t)rows * 8, st);
+        if (e != cudaSuccess) return e;
+    }
     if (a.d == 128 && G == 16) e = launch_kl<128, 64, 16>(a, tq, tk, q, q_idx, k_idx, num_sms, st);
     else if (a.d == 128 && G == 2) e = launch_kl<128, 64, 2>(a, tq, tk, q, q_idx, k_idx, num_sms, st);
     else if (a.d == 64 && G == 16) e = launch_kl<64, 32, 16>(a, tq, tk, q, q_idx, k_idx, num_sms, st);
     else if (a.d == 64 && G == 2) e = launch_kl<64, 32, 2>(a, tq, tk, q, q_idx, k_idx, num_sms, st);
     else return cudaErrorInvalidValue;
     if (e != cudaSuccess) return e;
-    const long long rows = (long long)a.B * a.N * a.H_kv;
     ProfScope ps("kl_finalize", st);
     const unsigned grid_rows = (unsigned)((rows * 32 + 255) / 256);
-    if (a.d_idx == 64)
+    if (a.dense) {
+        // the rows are complete; only the loss remains
+    } else if (a.d_idx == 64) {
         k_kl_rows<64><<<grid_rows, 256, 0, st>>>(a);
-    else
+    } else {
         k_kl_rows<32><<<grid_rows, 256, 0, st>>>(a);
+    }
     k_kl_loss<<<1, 1024, 0, st>>>(a);
     return cudaGetLastError();
 }

@@ -84,14 +84,16 @@ enum {
     MSA_OP_DECODE = 3,
     MSA_OP_KL = 4,
     MSA_OP_ATTN_BWD = 5,
-    MSA_OP_LSE_IDX_LOCAL = 6
+    MSA_OP_LSE_IDX_LOCAL = 6,
+    MSA_OP_KL_DENSE = 7
 };
 
 /*
  * Workspace bytes `op` needs for `dims` (for MSA_OP_DECODE, dims->N is the cache capacity).
  * MSA_OP_DECODE also serves msa_sparse_attn_decode_fp8idx, MSA_OP_INDEX_TOPK also serves
  * msa_index_topk_local, MSA_OP_ATTN_BWD is msa_sparse_attn_bwd's (MSA_ERR_UNSUPPORTED for its
- * unsupported G), MSA_OP_LSE_IDX_LOCAL is msa_lse_idx_local's.
+ * unsupported G), MSA_OP_LSE_IDX_LOCAL is msa_lse_idx_local's, MSA_OP_KL_DENSE is
+ * msa_kl_dense_fwd_grad's (MSA_ERR_UNSUPPORTED for its unsupported sizes).
  */
 MSA_API msa_status msa_workspace_size(int op, const msa_dims *dims, size_t *bytes);
 
@@ -263,6 +265,28 @@ MSA_API msa_status msa_kl_fwd_grad(const msa_dims *dims, const void *q, const vo
                            const void *k_idx, const int32_t *blocks, const float *lse, const float *lse_idx,
                            float grad_scale, float *loss, float *dq_idx, float *dk_idx, void *ws, size_t ws_bytes,
                            msa_stream_t stream);
+
+/*
+ * Dense warm-up of the KL alignment ("MSA 中的 KL 对齐与局部知识蒸馏", section 5: the index branch
+ * is first aligned to a teacher over the whole causal context, before sparse training): the KL of
+ * msa_kl_fwd_grad with every causal block selected, J = { j <= i }. The teacher's per-head LSE is
+ * the dense causal attention LSE, computed here over all keys (or returned through lse_out); LSE_idx
+ * likewise. With the same definitions as msa_kl_fwd_grad:
+ *   loss            = sum_{b,i,r} KL(P || P^idx) / (B * N * H_kv)
+ *   dq_idx, dk_idx  = grad_scale times the gradients of that loss
+ *   q, k, q_idx, k_idx  as for msa_kl_fwd_grad (topk is not used)
+ *   loss fp32 [1]; dq_idx fp32 [B,N,H_kv,d_idx]; dk_idx fp32 [B,N,d_idx]             (outputs)
+ *   lse_out fp32 [B,N,H_q] or NULL: the teacher's LSE (natural log, scaled logits)  (output)
+ * Sizes: those of msa_kl_fwd_grad, block_k in {32, 64, 128}, and B*H_kv*N*N/(2*block_k) < 2^31 list
+ * entries (N = 262144 fits with H_kv = 4). The workspace (MSA_OP_KL_DENSE) holds the dense inverse
+ * lists and one (max, sum-exp) pair per (row, block): about 1.5 GB at N = 65536, H_kv = 4. dQ_idx,
+ * dK_idx and the per-row KL terms are accumulated with float atomics: the results may differ in the
+ * last bits between runs.
+ */
+MSA_API msa_status msa_kl_dense_fwd_grad(const msa_dims *dims, const void *q, const void *k, const void *q_idx,
+                                         const void *k_idx, float grad_scale, float *loss, float *dq_idx,
+                                         float *dk_idx, float *lse_out, void *ws, size_t ws_bytes,
+                                         msa_stream_t stream);
 
 /*
  * Allocation-free decode step (no counterpart in the pages; a convenience of this library).
