@@ -705,9 +705,50 @@ def bench_train(args, world, rank, msa, pk):
                                  "kernel": "attn_bwd", "flops_per_launch": bwd_flops},
            "work": {"selected_tokens": sel_tok, "kl_flops": kl_flops, "attn_bwd_flops": bwd_flops},
            "kernels": {k: {"avg_ms": round(v["avg_ms"], 4), "launches": v["launches"]} for k, v in prof.items()}}
-    del x, ws_a, ws_k, ws_b, dout
+    del ws_a, ws_k, ws_b, dout
+    torch.cuda.empty_cache()
+    res["dense_warmup"] = bench_dense_warmup(args, world, x, w, N, msa, pk, flush)
+    del x
     torch.cuda.empty_cache()
     return res
+
+
+def bench_dense_warmup(args, world, x, w, N, msa, pk, flush):
+    """The dense warm-up KL (every causal block selected: teacher LSE over all keys, LSE_idx, KL and
+    index gradients) on the training workload's inputs, with its tensor roofline."""
+    dims = msa.MsaDims(w.B, N, w.H_q, w.H_kv, w.d, w.d_idx, w.block_k, w.topk)
+    dev = x["q"].device
+    ws = msa.workspace(msa.MSA_OP_KL_DENSE, dims, dev)
+
+    def step():
+        return msa.msa_kl_dense_fwd_grad(dims, x["q"], x["k"], x["q_idx"], x["k_idx"], ws=ws)
+
+    loss, _, _ = step()
+    torch.cuda.synchronize()
+    G = w.H_q // w.H_kv
+    pairs = w.B * w.H_kv * N * (N + 1) / 2  # causal (row, group, token) triples
+    fl = {"teacher_lse": 2.0 * w.d * G * pairs, "lse_idx": 2.0 * w.d_idx * pairs,
+          "kl": (2.0 * w.d * G + 6.0 * w.d_idx) * pairs}
+    msa.msa_profile_read()
+    msa.msa_profile_enable(True)
+    t = timed_steps(step, 2, flush)
+    msa.msa_profile_enable(False)
+    prof = profile_avg(msa.msa_profile_read())
+    ms = max_over_ranks(sum(t) / len(t), world)
+    total = sum(fl.values())
+    tf = total / (ms * 1e-3) / 1e12
+    kern = {k: {"avg_ms": v["avg_ms"], "launches": v["launches"]} for k, v in prof.items()}
+    for k, f in (("dense_lse", fl["teacher_lse"]), ("lse_idx", fl["lse_idx"]), ("kl_kv_outer", fl["kl"])):
+        if k in kern:
+            kern[k]["tflops"] = f / (kern[k]["avg_ms"] * 1e-3) / 1e12
+    del ws
+    torch.cuda.empty_cache()
+    return {"workload": "train_64k" if N == w.N else f"train_{N}", "ms_per_step": ms, "loss": float(loss.item()),
+            "flops": fl,
+            "roofline": {**roofline_entry("tensor", tf, pk["bf16_tflops_sustained"], "TFLOP/s"),
+                         "peak_source": f"{pk['source']} bf16 sustained (a step of this length runs under the "
+                                        f"power cap)", "frac_of_burst": tf / pk["bf16_tflops"]},
+            "kernels": kern}
 
 
 def main():
@@ -769,6 +810,13 @@ def main():
         line["train"] = rnd(bench_train(args, world, rank, msa, pk))
         line["sp_index"] = rnd(bench_sp(args, world, rank, msa, pk))
         line["decode"] = rnd(dec)
+        # the decode step's figures once more, compactly, as the line's last key
+        f8 = dec["fp8_index"]
+        line["decode_summary"] = rnd({
+            "bf16_us_per_step": dec["us_per_step"], "bf16_us_per_step_graph": dec["us_per_step_graph"],
+            "bf16_step_frac_hbm": dec["step_roofline"]["frac"], "bf16_scan_frac_hbm": dec["roofline"]["frac"],
+            "fp8_us_per_step": f8["us_per_step"], "fp8_us_per_step_graph": f8["us_per_step_graph"],
+            "fp8_step_frac_hbm": f8["step_roofline"]["frac"], "fp8_scan_frac_hbm": f8["roofline"]["frac"]})
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank == 0:
