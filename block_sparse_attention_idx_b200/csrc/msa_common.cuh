@@ -309,18 +309,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-// 32 lanes x 32 consecutive 32-bit columns from registers.
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
-        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
-        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
-}
 // 32 lanes x 32 consecutive 32-bit columns into r[0..31] (r may point into a larger register array
 // whose indices are compile-time constants after unrolling).
 __device__ __forceinline__ void tmem_ld32p(uint32_t taddr, uint32_t* r) {
@@ -336,12 +324,6 @@ __device__ __forceinline__ void tmem_ld32p(uint32_t taddr, uint32_t* r) {
         : "memory");
 }
 
-// Register split between warpgroups (all four warps of a warpgroup execute the same one): the
-// launch's registers per thread become N for this warpgroup's threads.
-template <int N>
-__device__ __forceinline__ void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
-template <int N>
-__device__ __forceinline__ void setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
 // 32 lanes x 16 / 8 consecutive 32-bit columns to registers.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
@@ -473,34 +455,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
-}
-
-// 2^x for two values on the FMA and integer pipes instead of the MUFU unit. Cody-Waite range
-// reduction: x = n + f with n = round-to-nearest(x) (by adding and subtracting 1.5 * 2^23) and
-// f in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose coefficients are the minimax fit of 2^f in
-// relative error on [-1/2, 1/2] (Remez exchange algorithm; largest relative error 7.5e-5, below the
-// 2^-9 rounding of the bf16 weights these values become); 2^n enters through the exponent bits.
-// Inputs are clamped below at -126 (so every result is a normal number): the callers use it for
-// softmax weights relative to a row maximum of weight 1, where anything below 2^-126 is far below
-// the float32 resolution of the row's sum.
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
-    constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f, kC2 = 0.2426111251115799f,
-                    kC3 = 0.0551716685295105f;
-    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound keeps round(x) in the low mantissa bits
-    float x0, x1;
-    f2_unpack(x2, x0, x1);
-    const uint64_t xc = f2_packf(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
-    const uint64_t j = f2_add(xc, f2_packf(kRound, kRound));
-    const uint64_t n = f2_add(j, f2_packf(-kRound, -kRound));
-    const uint64_t f = f2_fma(n, f2_packf(-1.f, -1.f), xc);
-    uint64_t p = f2_fma(f2_packf(kC3, kC3), f, f2_packf(kC2, kC2));
-    p = f2_fma(p, f, f2_packf(kC1, kC1));
-    p = f2_fma(p, f, f2_packf(kC0, kC0));
-    uint32_t jl, jh, pl, ph;
-    asm("mov.b64 {%0, %1}, %2;" : "=r"(jl), "=r"(jh) : "l"(j));
-    asm("mov.b64 {%0, %1}, %2;" : "=r"(pl), "=r"(ph) : "l"(p));
-    // the low bits of j's pattern hold n (two's complement); shifted into the exponent field
-    return f2_pack(pl + (jl << 23), ph + (jh << 23));
 }
 
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }

@@ -40,7 +40,7 @@ struct IndexSmem {
 };
 
 template <int DIDX>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     k_index_topk(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, IndexArgs a) {
     extern __shared__ uint8_t smem_raw[];
     IndexSmem<DIDX>& s = *reinterpret_cast<IndexSmem<DIDX>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
