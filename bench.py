@@ -602,10 +602,12 @@ def bench_decode(args, world, rank, msa, pk):
 
 def bench_sp(args, world, rank, msa, pk):
     """Sequence-parallel index branch on the headline workload with P ranks emulated on this GPU:
-    each rank's local Top-k and local (max, exp-sum) on its own K_idx slice timed separately (on P
-    GPUs they run side by side, so the step's compute is the slowest rank), plus the merge and the
-    eq (16) combine that every rank runs after the all-gather. The all-gather itself is not timed
-    here (one GPU); its bytes per rank are reported."""
+    each rank's local Top-k and local (max, exp-sum) on its own K_idx timed separately (on P GPUs
+    they run side by side, so the step's compute is the slowest rank), plus the merge and the
+    eq (16) combine that every rank runs after the all-gather. Both key assignments are measured:
+    contiguous ranges, and the zig-zag one (chunks p and 2P-1-p of 2P) that the library's
+    sp_index_topk callers use. The all-gather itself is not timed here (one GPU); its bytes per
+    rank are reported."""
     from block_sparse_attention_idx_b200 import sp
     w = WORKLOADS[HEADLINE]
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -614,44 +616,47 @@ def bench_sp(args, world, rank, msa, pk):
     ref_blocks, ref_lse = msa.msa_index_topk(dims, x["q_idx"], x["k_idx"], want_lse=True)
     flush = torch.zeros(256 << 20, dtype=torch.uint8, device=dev)
     res = {"workload": HEADLINE, "note": "ranks emulated on one GPU; the all-gather is not timed"}
+    ws = msa.workspace(msa.MSA_OP_INDEX_TOPK, dims, dev)
+    ws_l = msa.workspace(msa.MSA_OP_LSE_IDX_LOCAL, dims, dev)
     for P in (2, 8):
-        ranges = [sp.split_range(w.N, w.block_k, P, p) for p in range(P)]
-        slices = [x["k_idx"][:, t0:t0 + n].contiguous() for t0, n in ranges]
-        ws = msa.workspace(msa.MSA_OP_INDEX_TOPK, dims, dev)
-        local_ms = []
-        cands = []
-        for (t0, n), kl in zip(ranges, slices):
-            for _ in range(max(3, args.warmup)):
-                c = msa.msa_index_topk_local(dims, x["q_idx"], kl, t0, ws=ws)
-            t = timed_steps(lambda: msa.msa_index_topk_local(dims, x["q_idx"], kl, t0, ws=ws), 5, flush)
-            local_ms.append(sorted(t)[len(t) // 2])
-            cands.append(c)
-        cs = torch.stack([c[0] for c in cands])
-        ci = torch.stack([c[1] for c in cands])
-        for _ in range(3):
-            blocks = msa.msa_topk_merge(dims, cs, ci)
-        tm = timed_steps(lambda: msa.msa_topk_merge(dims, cs, ci), 5, flush)
-        lse_ms = []
-        mls = []
-        ws_l = msa.workspace(msa.MSA_OP_LSE_IDX_LOCAL, dims, dev)
-        for (t0, n), kl in zip(ranges, slices):
-            ml = msa.msa_lse_idx_local(dims, x["q_idx"], kl, t0, blocks, ws=ws_l).clone()
-            t = timed_steps(lambda: msa.msa_lse_idx_local(dims, x["q_idx"], kl, t0, blocks, ws=ws_l), 3, flush)
-            lse_ms.append(sorted(t)[len(t) // 2])
-            mls.append(ml)
-        ml_all = torch.stack(mls)
-        lse = msa.msa_lse_combine(dims, ml_all)
-        tc = timed_steps(lambda: msa.msa_lse_combine(dims, ml_all), 5, flush)
-        torch.cuda.synchronize()
-        rows = w.B * w.N * w.H_kv
-        res[f"P{P}"] = {
-            "local_topk_ms_max_rank": max(local_ms), "local_topk_ms_per_rank": [round(v, 4) for v in local_ms],
-            "merge_ms": sorted(tm)[len(tm) // 2], "local_lse_ms_max_rank": max(lse_ms),
-            "lse_combine_ms": sorted(tc)[len(tc) // 2],
-            "gather_bytes_per_rank": rows * w.topk * 8 + rows * 8,
-            "blocks_equal_single_device": bool(torch.equal(blocks, ref_blocks)),
-            "lse_max_abs_diff": float((lse - ref_lse).abs().max())}
-    del x, flush
+        for assign, ranges_of in (("zigzag", sp.zigzag_ranges), ("contiguous", sp.contiguous_ranges)):
+            helds = [ranges_of(w.N, w.block_k, P, p) for p in range(P)]
+            keys = [sp.local_keys(x["k_idx"], h) for h in helds]
+            local_ms, cands = [], []
+            for h, kl in zip(helds, keys):
+                for _ in range(max(3, args.warmup)):
+                    c = msa.msa_index_topk_local(dims, x["q_idx"], kl, h, ws=ws)
+                t = timed_steps(lambda: msa.msa_index_topk_local(dims, x["q_idx"], kl, h, ws=ws), 5, flush)
+                local_ms.append(sorted(t)[len(t) // 2])
+                cands.append(c)
+            cs = torch.stack([c[0] for c in cands])
+            ci = torch.stack([c[1] for c in cands])
+            for _ in range(3):
+                blocks = msa.msa_topk_merge(dims, cs, ci)
+            tm = timed_steps(lambda: msa.msa_topk_merge(dims, cs, ci), 5, flush)
+            lse_ms, mls = [], []
+            for h, kl in zip(helds, keys):
+                ml = msa.msa_lse_idx_local(dims, x["q_idx"], kl, h, blocks, ws=ws_l).clone()
+                t = timed_steps(lambda: msa.msa_lse_idx_local(dims, x["q_idx"], kl, h, blocks, ws=ws_l), 3, flush)
+                lse_ms.append(sorted(t)[len(t) // 2])
+                mls.append(ml)
+            ml_all = torch.stack(mls)
+            lse = msa.msa_lse_combine(dims, ml_all)
+            tc = timed_steps(lambda: msa.msa_lse_combine(dims, ml_all), 5, flush)
+            torch.cuda.synchronize()
+            rows = w.B * w.N * w.H_kv
+            res[f"P{P}_{assign}"] = {
+                "held_tokens": [[list(r) for r in h] for h in helds] if P <= 2 else None,
+                "local_topk_ms_max_rank": max(local_ms), "local_topk_ms_per_rank": [round(v, 4) for v in local_ms],
+                "local_topk_max_over_min": max(local_ms) / min(local_ms),
+                "merge_ms": sorted(tm)[len(tm) // 2], "local_lse_ms_max_rank": max(lse_ms),
+                "local_lse_max_over_min": max(lse_ms) / min(lse_ms),
+                "lse_combine_ms": sorted(tc)[len(tc) // 2],
+                "gather_bytes_per_rank": rows * w.topk * 8 + rows * 8,
+                "blocks_equal_single_device": bool(torch.equal(blocks, ref_blocks)),
+                "lse_max_abs_diff": float((lse - ref_lse).abs().max())}
+            del keys, cands, cs, ci, mls, ml_all
+    del x, flush, ws, ws_l
     torch.cuda.empty_cache()
     return res
 

@@ -34,6 +34,23 @@ class _Dims(ctypes.Structure):
                 ("scale", ctypes.c_float), ("scale_idx", ctypes.c_float)]
 
 
+class _KeyRanges(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_int32), ("tok0", ctypes.c_int32 * 2), ("ntok", ctypes.c_int32 * 2)]
+
+
+def _held(held, k_idx_local) -> _KeyRanges:
+    """msa_key_ranges from a list of one or two (tok0, ntok) ranges, or from a single first token
+    (one range spanning k_idx_local); the tokens must add up to k_idx_local's length."""
+    rng = [(int(held), int(k_idx_local.shape[1]))] if isinstance(held, int) else [(int(a), int(n)) for a, n in held]
+    if not 1 <= len(rng) <= 2 or sum(n for _, n in rng) != k_idx_local.shape[1]:
+        raise ValueError(f"held ranges {rng} do not describe k_idx_local of {k_idx_local.shape[1]} tokens")
+    h = _KeyRanges()
+    h.n = len(rng)
+    for x, (a, n) in enumerate(rng):
+        h.tok0[x], h.ntok[x] = a, n
+    return h
+
+
 @dataclass
 class MsaDims:
     """msa_dims: B sequences of N tokens (cache capacity for decode), H_q / H_kv heads, head dim d,
@@ -77,9 +94,10 @@ def lib() -> ctypes.CDLL:
         L.msa_kl_dense_fwd_grad.argtypes = [D, P, P, P, P, ctypes.c_float, P, P, P, P, P, S, P]
         L.msa_sparse_attn_bwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, S, P]
         I = ctypes.c_int
-        L.msa_index_topk_local.argtypes = [D, P, P, I, I, P, P, P, S, P]
+        H = ctypes.POINTER(_KeyRanges)
+        L.msa_index_topk_local.argtypes = [D, P, P, H, P, P, P, S, P]
         L.msa_topk_merge.argtypes = [D, I, P, P, P, P]
-        L.msa_lse_idx_local.argtypes = [D, P, P, I, I, P, P, P, S, P]
+        L.msa_lse_idx_local.argtypes = [D, P, P, H, P, P, P, S, P]
         L.msa_lse_combine.argtypes = [D, I, P, P, P]
         L.msa_sparse_attn_decode_noalloc.argtypes = [D, P, P, P, P, P, P, P, P, P]
         L.msa_sparse_attn_decode_noalloc.restype = ctypes.c_int
@@ -305,20 +323,22 @@ def msa_sparse_attn_bwd(dims: MsaDims, q, k, v, blocks, out, lse, dout, ws=None,
     return dq, dk, dv
 
 
-def msa_index_topk_local(dims: MsaDims, q_idx, k_idx_local, tok0: int, ws=None, stream=None):
+def msa_index_topk_local(dims: MsaDims, q_idx, k_idx_local, held, ws=None, stream=None):
     """This rank's candidates for the sequence-parallel selection: k_idx_local bf16 [B, ntok, d_idx]
-    holds tokens [tok0, tok0 + ntok). Returns (raw block maxima fp32, block ids int32), each
-    [B, N, H_kv, topk], best first, -inf / -1 padded."""
+    holds the tokens of `held`, one or two (tok0, ntok) ranges in order (or a single tok0: one range
+    of ntok tokens). Returns (raw block maxima fp32, block ids int32), each [B, N, H_kv, topk], best
+    first, -inf / -1 padded."""
     dev = q_idx.device
     _need(q_idx, "q_idx", (dims.B, dims.N, dims.H_kv, dims.d_idx), torch.bfloat16, dev)
     ntok = k_idx_local.shape[1]
     _need(k_idx_local, "k_idx_local", (dims.B, ntok, dims.d_idx), torch.bfloat16, dev)
+    h = _held(held, k_idx_local)
     cs = torch.empty(dims.B, dims.N, dims.H_kv, dims.topk, dtype=torch.float32, device=dev)
     ci = torch.empty(dims.B, dims.N, dims.H_kv, dims.topk, dtype=torch.int32, device=dev)
     ws = _ws(ws, MSA_OP_INDEX_TOPK, dims, dev)
     _check("msa_index_topk_local",
-           lib().msa_index_topk_local(ctypes.byref(dims.c()), _p(q_idx), _p(k_idx_local), tok0, ntok, _p(cs), _p(ci),
-                                      _p(ws), ws.numel(), _stream(stream, dev)))
+           lib().msa_index_topk_local(ctypes.byref(dims.c()), _p(q_idx), _p(k_idx_local), ctypes.byref(h), _p(cs),
+                                      _p(ci), _p(ws), ws.numel(), _stream(stream, dev)))
     return cs, ci
 
 
@@ -334,18 +354,20 @@ def msa_topk_merge(dims: MsaDims, cand_scores, cand_ids, stream=None):
     return blocks
 
 
-def msa_lse_idx_local(dims: MsaDims, q_idx, k_idx_local, tok0: int, blocks, ws=None, stream=None):
-    """This rank's (max, exp-sum) of the index scores over the selected tokens it holds:
-    fp32 [B, N, H_kv, 2]."""
+def msa_lse_idx_local(dims: MsaDims, q_idx, k_idx_local, held, blocks, ws=None, stream=None):
+    """This rank's (max, exp-sum) of the index scores over the selected tokens it holds (`held` as in
+    msa_index_topk_local): fp32 [B, N, H_kv, 2]."""
     dev = q_idx.device
     ntok = k_idx_local.shape[1]
     _need(q_idx, "q_idx", (dims.B, dims.N, dims.H_kv, dims.d_idx), torch.bfloat16, dev)
     _need(k_idx_local, "k_idx_local", (dims.B, ntok, dims.d_idx), torch.bfloat16, dev)
     _need(blocks, "blocks", (dims.B, dims.N, dims.H_kv, dims.topk + 1), torch.int32, dev)
+    h = _held(held, k_idx_local)
     ml = torch.empty(dims.B, dims.N, dims.H_kv, 2, dtype=torch.float32, device=dev)
     ws = _ws(ws, MSA_OP_LSE_IDX_LOCAL, dims, dev)
-    _check("msa_lse_idx_local", lib().msa_lse_idx_local(ctypes.byref(dims.c()), _p(q_idx), _p(k_idx_local), tok0, ntok,
-                                                        _p(blocks), _p(ml), _p(ws), ws.numel(), _stream(stream, dev)))
+    _check("msa_lse_idx_local",
+           lib().msa_lse_idx_local(ctypes.byref(dims.c()), _p(q_idx), _p(k_idx_local), ctypes.byref(h), _p(blocks),
+                                   _p(ml), _p(ws), ws.numel(), _stream(stream, dev)))
     return ml
 
 

@@ -320,13 +320,19 @@ static bool sp_range_ok(const msa_dims* d, int tok0, int ntok) {
            (ntok % d->block_k == 0 || tok0 + ntok == d->N);
 }
 
-msa_status msa_index_topk_local(const msa_dims* d, const void* q_idx, const void* k_idx_local, int tok0, int ntok,
-                                float* cand_scores, int32_t* cand_ids, void* ws, size_t ws_bytes,
-                                msa_stream_t stream_) {
+// one or two ranges of whole blocks, the second after the first
+static bool sp_held_ok(const msa_dims* d, const msa_key_ranges* h) {
+    if (!h || h->n < 1 || h->n > 2 || !sp_range_ok(d, h->tok0[0], h->ntok[0])) return false;
+    return h->n == 1 || (sp_range_ok(d, h->tok0[1], h->ntok[1]) && h->tok0[1] >= h->tok0[0] + h->ntok[0]);
+}
+
+msa_status msa_index_topk_local(const msa_dims* d, const void* q_idx, const void* k_idx_local,
+                                const msa_key_ranges* held, float* cand_scores, int32_t* cand_ids, void* ws,
+                                size_t ws_bytes, msa_stream_t stream_) {
     msa_status s = check_common(d);
     if (s != MSA_OK) return s;
     if (!q_idx || !k_idx_local || !cand_scores || !cand_ids || !aligned16(q_idx) || !aligned16(k_idx_local) ||
-        !aligned16(cand_scores) || !aligned16(cand_ids) || !sp_range_ok(d, tok0, ntok))
+        !aligned16(cand_scores) || !aligned16(cand_ids) || !sp_held_ok(d, held))
         return MSA_ERR_INVALID_ARG;
     s = ws_check(ws, ws_bytes, kStatusBytes);
     if (s != MSA_OK) return s;
@@ -334,7 +340,8 @@ msa_status msa_index_topk_local(const msa_dims* d, const void* q_idx, const void
     DevStatus* status = static_cast<DevStatus*>(ws);
     cudaError_t e = status_init(status, st);
     if (e != cudaSuccess) return MSA_ERR_CUDA;
-    IndexArgs a{d->B, d->N, d->H_kv, d->d_idx, d->block_k, d->topk, nullptr, status, tok0, ntok, cand_scores, cand_ids};
+    IndexArgs a{d->B, d->N, d->H_kv, d->d_idx, d->block_k, d->topk, nullptr, status, held->tok0[0], held->ntok[0],
+                cand_scores, cand_ids, held->n == 2 ? held->tok0[1] : 0, held->n == 2 ? held->ntok[1] : 0};
     return cuda_status(run_index_topk(a, q_idx, k_idx_local, st));
 }
 
@@ -349,12 +356,12 @@ msa_status msa_topk_merge(const msa_dims* d, int P, const float* cand_scores, co
                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
-msa_status msa_lse_idx_local(const msa_dims* d, const void* q_idx, const void* k_idx_local, int tok0, int ntok,
+msa_status msa_lse_idx_local(const msa_dims* d, const void* q_idx, const void* k_idx_local, const msa_key_ranges* held,
                              const int32_t* blocks, float* ml, void* ws, size_t ws_bytes, msa_stream_t stream_) {
     msa_status s = check_common(d);
     if (s != MSA_OK) return s;
     if (!q_idx || !k_idx_local || !blocks || !ml || !aligned16(q_idx) || !aligned16(k_idx_local) ||
-        !aligned16(blocks) || !aligned16(ml) || !sp_range_ok(d, tok0, ntok))
+        !aligned16(blocks) || !aligned16(ml) || !sp_held_ok(d, held))
         return MSA_ERR_INVALID_ARG;
     s = ws_check(ws, ws_bytes, ws_lse_local(d));
     if (s != MSA_OK) return s;
@@ -369,16 +376,21 @@ msa_status msa_lse_idx_local(const msa_dims* d, const void* q_idx, const void* k
     k.scale = eff_scale(d->scale, d->d); k.scale_idx = eff_scale(d->scale_idx, d->d_idx);
     csr_carve(&k.csr_idx, cv.take(csr_need(d)), d->B, d->N, d->H_kv, d->block_k, d->topk, 0);
     k.ml_part = reinterpret_cast<float2*>(cv.take(rows_kv(d) * (d->topk + 1) * sizeof(float2)));
-    int32_t* held = reinterpret_cast<int32_t*>(cv.take(rows_kv(d) * (d->topk + 1) * 4));
-    k.blocks = held;
+    int32_t* mine = reinterpret_cast<int32_t*>(cv.take(rows_kv(d) * (d->topk + 1) * 4));  // the held selected blocks
+    k.blocks = mine;
     k.status = status;
-    k.kv_tok0 = tok0;
-    k.kv_ntok = ntok;
+    k.kv_tok0 = held->tok0[0];
+    k.kv_ntok = held->ntok[0];
+    k.kv_tok0b = held->n == 2 ? held->tok0[1] : 0;
+    k.kv_ntokb = held->n == 2 ? held->ntok[1] : 0;
     k.ml_out = reinterpret_cast<float2*>(ml);
-    const int blk0 = tok0 / d->block_k, blk1 = (tok0 + ntok + d->block_k - 1) / d->block_k;
-    e = run_blocks_in_range((long long)rows_kv(d), d->topk + 1, blk0, blk1, blocks, held, st);
+    // first block of each range and the block past it (a range that ends at N may end inside a block)
+    const int bk = d->block_k;
+    const int blk0 = k.kv_tok0 / bk, blk1 = (k.kv_tok0 + k.kv_ntok + bk - 1) / bk;
+    const int blk2 = k.kv_tok0b / bk, blk3 = (k.kv_tok0b + k.kv_ntokb + bk - 1) / bk;
+    e = run_blocks_in_range((long long)rows_kv(d), d->topk + 1, blk0, blk1, blk2, blk3, blocks, mine, st);
     if (e == cudaSuccess)
-        e = run_csr_build(k.csr_idx, held, d->B, d->N, d->H_kv, d->block_k, d->topk, kIdxQpc, status, st);
+        e = run_csr_build(k.csr_idx, mine, d->B, d->N, d->H_kv, d->block_k, d->topk, kIdxQpc, status, st);
     if (e == cudaSuccess) e = run_lse_idx(k, q_idx, k_idx_local, num_sms(), st);
     return cuda_status(e);
 }

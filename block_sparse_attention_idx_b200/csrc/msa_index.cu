@@ -58,10 +58,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int i_hi = min(a.N - 1, (R0 + kRows - 1) / a.H_kv);
     const int bmax = i_hi / a.block_k;                      // largest local block among the rows
     const int ntok = bmax * a.block_k;                      // tokens of complete past blocks
-    // tiles of the held key range [tok0, tok0 + ntok_held) that hold complete past blocks
-    const int span = min(ntok, a.tok0 + a.ntok) - a.tok0;
-    const int nkt = span > 0 ? (span + kCols - 1) / kCols : 0;
-    const int blk_end = (a.tok0 + a.ntok) / a.block_k;      // first block past the held range
+    // tiles of the held key ranges that hold complete past blocks: those of [tok0, tok0 + ntok),
+    // then those of the second range [tok0b, tok0b + ntokb), whose tokens follow in k_idx
+    const int span_a = min(ntok, a.tok0 + a.ntok) - a.tok0;
+    const int nkt_a = span_a > 0 ? (span_a + kCols - 1) / kCols : 0;
+    const int span_b = a.ntokb > 0 ? min(ntok, a.tok0b + a.ntokb) - a.tok0b : 0;
+    const int nkt = nkt_a + (span_b > 0 ? (span_b + kCols - 1) / kCols : 0);
+    const int blk_end_a = (a.tok0 + a.ntok) / a.block_k;    // first block past each held range
+    const int blk_end_b = (a.tok0b + a.ntokb) / a.block_k;
 
     const int warp = warp_id(), lane = lane_id();
     if (threadIdx.x == 0) {
@@ -100,7 +104,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const uint32_t ph = (kt / kStages) & 1;
                 if (!mbar_wait(&s.k_empty[st], ph ^ 1, a.status, 0x101)) { s.abort = 1; break; }
                 mbar_arrive_expect_tx(&s.k_full[st], kCols * DIDX * 2);
-                tma_load_3d(s.k[st], &tm_k, &s.k_full[st], 0, kt * kCols, b);
+                const int row0 = kt < nkt_a ? kt * kCols : a.ntok + (kt - nkt_a) * kCols;  // token row in k_idx
+                tma_load_3d(s.k[st], &tm_k, &s.k_full[st], 0, row0, b);
             }
             // make sure no copy of ours is still landing when the CTA leaves
             for (int x = max(0, kt - kStages); x < kt; ++x)
@@ -174,10 +179,13 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             tc_fence_before();
             mbar_arrive(&s.acc_empty[acc]);
-            // one candidate per complete past block inside this tile
+            // one candidate per complete past block inside this tile (a tile of the first range that
+            // runs past its end holds blocks at or past blk_end_a, which the test below drops)
             const int chunks_per_block = a.block_k / 32;
+            const int tile_tok = kt < nkt_a ? a.tok0 + kt * kCols : a.tok0b + (kt - nkt_a) * kCols;
+            const int blk_end = kt < nkt_a ? blk_end_a : blk_end_b;
             for (int c0 = 0; c0 < 4; c0 += chunks_per_block) {
-                const int cb = (a.tok0 + kt * kCols + c0 * 32) / a.block_k;
+                const int cb = (tile_tok + c0 * 32) / a.block_k;
                 float v = cmax[c0];
                 for (int x = 1; x < chunks_per_block; ++x) v = fmaxf(v, cmax[c0 + x]);
                 if (cb < bi && cb < blk_end && v > topv[kKMax - 1]) {
@@ -249,7 +257,8 @@ cudaError_t run_index_topk(const IndexArgs& a, const void* q_idx, const void* k_
     const uint64_t rows = (uint64_t)a.B * a.N * a.H_kv;
     const int sw = a.d_idx == 64 ? 128 : 64;
     if (!make_tmap_2d(&tq, q_idx, a.d_idx, rows, (uint64_t)a.d_idx * 2, a.d_idx, kRows, sw)) return cudaErrorInvalidValue;
-    if (!make_tmap_3d(&tk, k_idx, a.d_idx, a.ntok, a.B, (uint64_t)a.d_idx * 2, (uint64_t)a.ntok * a.d_idx * 2,
+    const uint64_t held = (uint64_t)a.ntok + a.ntokb;
+    if (!make_tmap_3d(&tk, k_idx, a.d_idx, held, a.B, (uint64_t)a.d_idx * 2, held * a.d_idx * 2,
                       a.d_idx, kCols, 1, sw))
         return cudaErrorInvalidValue;
     return a.d_idx == 64 ? launch_index<64>(a, tq, tk, st) : launch_index<32>(a, tq, tk, st);

@@ -41,21 +41,24 @@ struct IndexArgs {
     int B, N, H_kv, d_idx, block_k, topk;
     int32_t* blocks;
     DevStatus* status;
-    // key range held in k_idx: tokens [tok0, tok0 + ntok) of every sequence, k_idx [B, ntok, d_idx]
-    // (0 and N for the whole sequence). With cand_ids set, the kernel writes each row's Top-k of the
-    // complete past blocks inside that range, unmerged (raw block maxima, -inf / -1 padded), instead
-    // of `blocks`.
+    // key range held in k_idx: tokens [tok0, tok0 + ntok) of every sequence, then (ntokb > 0) a
+    // second range [tok0b, tok0b + ntokb) after it; k_idx [B, ntok + ntokb, d_idx] stores the first
+    // range's tokens, then the second's (0 and N, no second range, for the whole sequence). With
+    // cand_ids set, the kernel writes each row's Top-k of the complete past blocks inside the held
+    // ranges, unmerged (raw block maxima, -inf / -1 padded), instead of `blocks`.
     int tok0, ntok;
     float* cand_scores;   // [B, N, H_kv, topk]
     int32_t* cand_ids;    // [B, N, H_kv, topk]
+    int tok0b, ntokb;
 };
 cudaError_t run_index_topk(const IndexArgs& a, const void* q_idx, const void* k_idx, cudaStream_t st);
 
 // ---------------------------------------------------------------- sequence-parallel indexer (msa_sp.cu)
 cudaError_t run_topk_merge(int B, int N, int H_kv, int block_k, int topk, int P, const float* cand_scores,
                            const int32_t* cand_ids, int32_t* blocks, cudaStream_t st);
-cudaError_t run_blocks_in_range(long long rows, int K1, int blk0, int blk1, const int32_t* blocks, int32_t* out,
-                                cudaStream_t st);
+// blocks kept where blk0 <= c < blk1 or blk2 <= c < blk3, else -1
+cudaError_t run_blocks_in_range(long long rows, int K1, int blk0, int blk1, int blk2, int blk3, const int32_t* blocks,
+                                int32_t* out, cudaStream_t st);
 cudaError_t run_lse_combine(int P, long long rows, const float2* ml, float* lse, cudaStream_t st);
 
 // ---------------------------------------------------------------- inverse selection lists (msa_csr.cu)
@@ -137,10 +140,11 @@ struct KlArgs {
     float* loss;        // [1]
     const int32_t* blocks;
     DevStatus* status;
-    // LSE_idx pass only: k_idx holds tokens [kv_tok0, kv_tok0 + kv_ntok) ([B, kv_ntok, d_idx]; 0 and N
+    // LSE_idx pass only: k_idx holds tokens [kv_tok0, kv_tok0 + kv_ntok), then those of a second
+    // range [kv_tok0b, kv_tok0b + kv_ntokb) if kv_ntokb > 0 ([B, kv_ntok + kv_ntokb, d_idx]; 0 and N
     // for the whole sequence); with ml_out set, each row's (max, exp-sum) is written there instead
     // of lse_idx
-    int kv_tok0, kv_ntok;
+    int kv_tok0, kv_ntok, kv_tok0b, kv_ntokb;
     float2* ml_out;     // [B, N, H_kv]
     // dense warm-up: every causal block is selected; the lists come from run_dense_lists, the
     // LSE_idx partial slot of an entry is its block (ml_part [B, N, H_kv, nb]), and dQ_idx / the

@@ -59,12 +59,16 @@ __global__ void __launch_bounds__(128) k_lse_idx(KlArgs a, const __nv_bfloat16* 
         __syncthreads();  // the previous item is done with kb / qb / s_i / red
         if (L != curL) {
             const int tok = c * a.block_k + tt;
-            const bool tvalid = tt < a.block_k && tok < a.N && tok >= a.kv_tok0 && tok < a.kv_tok0 + a.kv_ntok;
+            // the token's row in the held K_idx: first range, then the second one
+            int lt = -1;
+            if (tok >= a.kv_tok0 && tok < a.kv_tok0 + a.kv_ntok) lt = tok - a.kv_tok0;
+            else if (tok >= a.kv_tok0b && tok < a.kv_tok0b + a.kv_ntokb) lt = a.kv_ntok + (tok - a.kv_tok0b);
+            const bool tvalid = tt < a.block_k && tok < a.N && lt >= 0;
+            const size_t held = (size_t)a.kv_ntok + a.kv_ntokb;
 #pragma unroll
             for (int x = 0; x < DI / 8; ++x) {
                 uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if (tvalid)
-                    v = *reinterpret_cast<const uint4*>(k_idx + ((size_t)b * a.kv_ntok + (tok - a.kv_tok0)) * DI + x * 8);
+                if (tvalid) v = *reinterpret_cast<const uint4*>(k_idx + ((size_t)b * held + lt) * DI + x * 8);
                 *reinterpret_cast<uint4*>(&kb[tt * KBP + x * 8]) = v;
             }
             curL = L;

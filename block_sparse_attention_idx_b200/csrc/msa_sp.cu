@@ -1,5 +1,5 @@
-// Sequence-parallel indexer ("4.1.1 · 监督与联合训练", section 3): P ranks each hold a contiguous
-// range of every sequence's key blocks. Each takes the Top-k of its own complete past blocks
+// Sequence-parallel indexer ("4.1.1 · 监督与联合训练", section 3): P ranks each hold one or two
+// ranges of every sequence's key blocks. Each takes the Top-k of its own complete past blocks
 // (k_index_topk in key-range mode); only the (score, block id) pairs are exchanged, and the merge
 // below reproduces the single-device selection. LSE_idx over the selected tokens is rebuilt from
 // each rank's local (maximum a_p, exp-sum z_p) by eq (16): a = max a_p, z = sum exp(a_p - a) z_p;
@@ -65,12 +65,12 @@ __global__ void __launch_bounds__(256) k_topk_merge(int B, int N, int H_kv, int 
 
 // The selection restricted to the blocks [blk0, blk1) a rank holds (others -1): the LSE_idx pass
 // over it yields the rank's (a_p, z_p) per row.
-__global__ void k_blocks_in_range(long long n, int blk0, int blk1, const int32_t* __restrict__ blocks,
-                                  int32_t* __restrict__ out) {
+__global__ void k_blocks_in_range(long long n, int blk0, int blk1, int blk2, int blk3,
+                                  const int32_t* __restrict__ blocks, int32_t* __restrict__ out) {
     const long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (x >= n) return;
     const int c = blocks[x];
-    out[x] = (c >= blk0 && c < blk1) ? c : -1;
+    out[x] = ((c >= blk0 && c < blk1) || (c >= blk2 && c < blk3)) ? c : -1;
 }
 
 // eq (16) over the P ranks' pairs [P][rows]: LSE = a + log z.
@@ -98,10 +98,10 @@ cudaError_t run_topk_merge(int B, int N, int H_kv, int block_k, int topk, int P,
     return cudaGetLastError();
 }
 
-cudaError_t run_blocks_in_range(long long rows, int K1, int blk0, int blk1, const int32_t* blocks, int32_t* out,
-                                cudaStream_t st) {
+cudaError_t run_blocks_in_range(long long rows, int K1, int blk0, int blk1, int blk2, int blk3, const int32_t* blocks,
+                                int32_t* out, cudaStream_t st) {
     const long long n = rows * K1;
-    k_blocks_in_range<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(n, blk0, blk1, blocks, out);
+    k_blocks_in_range<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(n, blk0, blk1, blk2, blk3, blocks, out);
     return cudaGetLastError();
 }
 

@@ -132,12 +132,18 @@ MSA_API msa_status msa_sparse_attn_fwd(const msa_dims *dims, const void *q, cons
                                msa_stream_t stream);
 
 /*
- * Sequence-parallel index branch ("4.1.1 · 监督与联合训练", section 3, eq (16)): P ranks each hold a
- * contiguous range of every sequence's keys; only (score, block id) candidates and per-row
- * (max, exp-sum) pairs are exchanged, and the result equals the single-device msa_index_topk.
- * The key range of a rank is tokens [tok0, tok0 + ntok): tok0 a multiple of block_k, ntok a
- * multiple of block_k unless the range ends at N; k_idx_local holds those tokens, bf16
- * [B, ntok, d_idx]. The ranks' ranges tile [0, N) in rank order.
+ * Sequence-parallel index branch ("4.1.1 · 监督与联合训练", section 3, eq (16)): P ranks each hold
+ * part of every sequence's keys; only (score, block id) candidates and per-row (max, exp-sum) pairs
+ * are exchanged, and the result equals the single-device msa_index_topk.
+ * A rank holds one or two ranges of tokens (msa_key_ranges, host memory, read during the call):
+ * range x is tokens [tok0[x], tok0[x] + ntok[x]), tok0[x] a multiple of block_k, ntok[x] > 0 a
+ * multiple of block_k unless the range ends at N, and the second range starts at or after the end
+ * of the first. k_idx_local holds the first range's tokens, then the second's: bf16
+ * [B, ntok[0] + ntok[1], d_idx]. Across the ranks the ranges tile [0, N) without overlap; any
+ * assignment gives the same result. Under a causal mask the block at position c is in the past of
+ * (N - c) queries, so contiguous ranges load the first rank most; two ranges per rank, chunk p and
+ * chunk 2P-1-p of 2P equal chunks of blocks (zig-zag), give every rank about the same work.
+ * A null or malformed msa_key_ranges gives MSA_ERR_INVALID_ARG.
  *
  * msa_index_topk_local: for every (b, i, r), the Top-k of the complete past blocks c < b_i that this
  *   rank holds, by (M desc, block id asc), best first. cand_scores fp32 [B, N, H_kv, topk] are the
@@ -154,14 +160,20 @@ MSA_API msa_status msa_sparse_attn_fwd(const msa_dims *dims, const void *q, cons
  * msa_lse_combine: eq (16) over ml [P, B, N, H_kv, 2] gathered in rank order: lse_idx fp32
  *   [B, N, H_kv] = a + log(z), a = max_p a_p, z = sum_p exp(a_p - a) z_p.
  */
-MSA_API msa_status msa_index_topk_local(const msa_dims *dims, const void *q_idx, const void *k_idx_local, int tok0,
-                                        int ntok, float *cand_scores, int32_t *cand_ids, void *ws, size_t ws_bytes,
-                                        msa_stream_t stream);
+typedef struct msa_key_ranges {
+    int32_t n;        /* number of ranges: 1 or 2 */
+    int32_t tok0[2];  /* first token of each range */
+    int32_t ntok[2];  /* tokens in each range */
+} msa_key_ranges;
+
+MSA_API msa_status msa_index_topk_local(const msa_dims *dims, const void *q_idx, const void *k_idx_local,
+                                        const msa_key_ranges *held, float *cand_scores, int32_t *cand_ids, void *ws,
+                                        size_t ws_bytes, msa_stream_t stream);
 MSA_API msa_status msa_topk_merge(const msa_dims *dims, int P, const float *cand_scores, const int32_t *cand_ids,
                                   int32_t *blocks, msa_stream_t stream);
-MSA_API msa_status msa_lse_idx_local(const msa_dims *dims, const void *q_idx, const void *k_idx_local, int tok0,
-                                     int ntok, const int32_t *blocks, float *ml, void *ws, size_t ws_bytes,
-                                     msa_stream_t stream);
+MSA_API msa_status msa_lse_idx_local(const msa_dims *dims, const void *q_idx, const void *k_idx_local,
+                                     const msa_key_ranges *held, const int32_t *blocks, float *ml, void *ws,
+                                     size_t ws_bytes, msa_stream_t stream);
 MSA_API msa_status msa_lse_combine(const msa_dims *dims, int P, const float *ml, float *lse_idx, msa_stream_t stream);
 
 /*

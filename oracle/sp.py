@@ -1,5 +1,5 @@
 """Sequence-parallel indexer: plain float64 restatement of the exchange that lets P ranks, each
-holding a contiguous range of every sequence's key blocks, reproduce the single-device selection
+holding some ranges of every sequence's key blocks, reproduce the single-device selection
 and LSE_idx ("4.1.1 · 监督与联合训练", section 3: each rank takes its local top candidates and
 only the (score, index) pairs are exchanged and merged; the global log-sum-exp comes from each
 rank's local maximum a_p and exp-sum z_p by eq (16)).
@@ -15,10 +15,16 @@ import numpy as np
 from . import Dims, block_max_row, index_scores_row
 
 
-def local_topk(dims: Dims, q_idx, k_idx, blk0: int, blk1: int):
-    """For every (b, i, r): the Top-k of the complete past blocks c with blk0 <= c < blk1 by
-    (M desc, id asc). Returns scores [B, N, H_kv, k] (M with scale_idx, -inf padded) and ids
-    (int32, -1 padded)."""
+def held_blocks(held):
+    """The block ids of a rank's held ranges [(blk0, blk1), ...] (each half-open)."""
+    return sorted({c for b0, b1 in held for c in range(b0, b1)})
+
+
+def local_topk(dims: Dims, q_idx, k_idx, held):
+    """For every (b, i, r): the Top-k of the complete past blocks c < b_i that the rank holds (c in
+    one of its block ranges `held` = [(blk0, blk1), ...]) by (M desc, id asc). Returns scores
+    [B, N, H_kv, k] (M with scale_idx, -inf padded) and ids (int32, -1 padded)."""
+    mine = held_blocks(held)
     k = dims.topk
     scores = np.full((dims.B, dims.N, dims.H_kv, k), -np.inf)
     ids = np.full((dims.B, dims.N, dims.H_kv, k), -1, dtype=np.int32)
@@ -27,7 +33,7 @@ def local_topk(dims: Dims, q_idx, k_idx, blk0: int, blk1: int):
             bi = i // dims.block_k
             for r in range(dims.H_kv):
                 M = block_max_row(dims, index_scores_row(dims, q_idx, k_idx, b, i, r), i)
-                cand = sorted(range(blk0, min(blk1, bi)), key=lambda c: (-M[c], c))[:k]
+                cand = sorted((c for c in mine if c < bi), key=lambda c: (-M[c], c))[:k]
                 for p, c in enumerate(cand):
                     scores[b, i, r, p] = M[c]
                     ids[b, i, r, p] = c
@@ -51,15 +57,17 @@ def merge(dims: Dims, cand_scores, cand_ids):
     return blocks
 
 
-def local_lse(dims: Dims, q_idx, k_idx, blocks, blk0: int, blk1: int):
+def local_lse(dims: Dims, q_idx, k_idx, blocks, held):
     """Per (b, i, r): (a_p, z_p) = (max, sum of exp(s - a_p)) of the index scores over the causal
-    tokens of the selected blocks c with blk0 <= c < blk1; (-inf, 0) when there are none."""
+    tokens of the selected blocks the rank holds (block ranges `held`); (-inf, 0) when there are
+    none."""
+    mine = set(held_blocks(held))
     out = np.zeros((dims.B, dims.N, dims.H_kv, 2))
     for b in range(dims.B):
         for i in range(dims.N):
             for r in range(dims.H_kv):
                 s = index_scores_row(dims, q_idx, k_idx, b, i, r)
-                J = [j for c in blocks[b, i, r] if blk0 <= c < blk1
+                J = [j for c in blocks[b, i, r] if c in mine
                      for j in range(c * dims.block_k, min((c + 1) * dims.block_k, i + 1))]
                 if not J:
                     out[b, i, r] = (-np.inf, 0.0)

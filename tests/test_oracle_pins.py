@@ -589,11 +589,15 @@ def test_sp_eq16_hand_values():
     assert got == pytest.approx(math.log(np.exp(s1).sum() + np.exp(s2).sum()), abs=1e-14)
 
 
-@pytest.mark.parametrize("bounds", [[0, 4, 8], [0, 3, 6, 8], [0, 1, 2, 5, 8], [0, 8]])
-def test_sp_merge_and_lse_equal_single_device(bounds):
-    """Each rank's local Top-k of its block range, merged by (score desc, id asc), plus the local
+@pytest.mark.parametrize("held", [[[(0, 4)], [(4, 8)]], [[(0, 3)], [(3, 6)], [(6, 8)]],
+                                  [[(0, 1)], [(1, 2)], [(2, 5)], [(5, 8)]], [[(0, 8)]],
+                                  [[(0, 2), (6, 8)], [(2, 4), (4, 6)]], [[(0, 1), (7, 8)], [(1, 3), (5, 7)], [(3, 5)]]],
+                         ids=["halves", "thirds", "uneven", "one_rank", "zigzag_2", "zigzag_3_uneven"])
+def test_sp_merge_and_lse_equal_single_device(held):
+    """Each rank's local Top-k of its held blocks, merged by (score desc, id asc), plus the local
     block, is the single-device selection; eq (16) over the ranks' (a_p, z_p) is the single-device
-    LSE_idx (uneven ranges, a ragged last block, ranks without candidates for early rows)."""
+    LSE_idx (uneven ranges, two ranges per rank, a ragged last block, ranks without candidates for
+    early rows)."""
     from oracle import sp
     N, Bk, k, Hkv = 61, 8, 3, 2
     dims = oracle.Dims(B=2, N=N, H_q=2 * Hkv, H_kv=Hkv, d=8, d_idx=8, block_k=Bk, topk=k)
@@ -601,14 +605,15 @@ def test_sp_merge_and_lse_equal_single_device(bounds):
     blocks, _, lse = oracle.index_topk(dims, x["q_idx"], x["k_idx"], want_lse=True)
     blocks = blocks.reshape(2, N, Hkv, k + 1)
     cs, ci, ml = [], [], []
-    for p in range(len(bounds) - 1):
-        s_, i_ = sp.local_topk(dims, x["q_idx"], x["k_idx"], bounds[p], bounds[p + 1])
+    assert sp.held_blocks([r for h in held for r in h]) == list(range(8))  # the ranks' blocks tile [0, 8)
+    for h in held:
+        s_, i_ = sp.local_topk(dims, x["q_idx"], x["k_idx"], h)
         cs.append(s_)
         ci.append(i_)
     merged = sp.merge(dims, cs, ci)
     np.testing.assert_array_equal(merged, blocks)
-    for p in range(len(bounds) - 1):
-        ml.append(sp.local_lse(dims, x["q_idx"], x["k_idx"], blocks, bounds[p], bounds[p + 1]))
+    for h in held:
+        ml.append(sp.local_lse(dims, x["q_idx"], x["k_idx"], blocks, h))
     np.testing.assert_allclose(sp.combine_lse(ml), lse.reshape(2, N, Hkv), atol=1e-12)
 
 
