@@ -218,7 +218,8 @@ def streamed_steps(xs, host, out_host, dims, ws_i, ws_a, msa, n_steps: int) -> f
         with torch.cuda.stream(s_cmp):
             s_cmp.wait_event(ready)
             blocks = msa.msa_index_topk(dims, xs[j]["q_idx"], xs[j]["k_idx"], ws=ws_i)
-            out, _ = msa.msa_sparse_attn_fwd(dims, xs[j]["q"], xs[j]["k"], xs[j]["v"], blocks, ws=ws_a)
+            out, _ = msa.msa_sparse_attn_fwd(dims, xs[j]["q"], xs[j]["k"], xs[j]["v"], blocks, ws=ws_a,
+                                             out_dtype=torch.bfloat16)
             done[j] = torch.cuda.Event()
             done[j].record(s_cmp)
         with torch.cuda.stream(s_out):
@@ -282,7 +283,7 @@ def workload_config(w, world: int) -> dict:
             "parallelism": f"dp{world} (independent sequences)",
             "l2": "flushed (256 MiB read) before every timed step; inputs also larger than L2; the pipelined "
                   "e2e steps are not flushed (625 MB uploaded per step)",
-            "step": "msa_index_topk + msa_sparse_attn_fwd"}
+            "step": "msa_index_topk + msa_sparse_attn_fwd_bf16 (O stored as bf16, rounded from the fp32 result)"}
 
 
 def rnd(x, sig: int = 4):
@@ -370,6 +371,8 @@ def cpu_baseline(x, w, rows_n: int, blocks=None, out=None):
         differ = (gb != b).any(axis=-1)
         same = ~differ.any(axis=-1)
         err = np.abs(og[same] - oo[same])
+        # the output is bf16: the fp32 bound plus half a bf16 unit (at most 2^-8 |o|)
+        within = bool((err <= 1e-2 + 2.0 ** -8 * np.abs(oo[same])).all())
         par = {"sample": f"the cpu_baseline rows ({rows_n} query rows x {w.H_kv} groups)",
                "selection_pairs": int(gb.shape[0] * w.H_kv), "near_ties": int(near.sum()),
                "near_ties_selected_differently": int((differ & near).sum()),
@@ -377,7 +380,9 @@ def cpu_baseline(x, w, rows_n: int, blocks=None, out=None):
                "attn_rows_compared": int(same.sum()),
                "attn_max_abs_err": float(err.max()) if err.size else None,
                "attn_mean_abs_err": float(err.mean()) if err.size else None,
-               "tolerance": "selection bit-exact outside near-ties; attention max abs 1e-2, mean abs 1e-3"}
+               "attn_within_bound": within,
+               "tolerance": "selection bit-exact outside near-ties; attention (bf16 output) max abs "
+                            "1e-2 + 2^-8 |o| elementwise"}
     return res, par
 
 
@@ -392,15 +397,15 @@ def bench_prefill(args, world, rank, msa, pk):
 
     def step():
         blocks = msa.msa_index_topk(dims, x["q_idx"], x["k_idx"], ws=ws_i)
-        return blocks, msa.msa_sparse_attn_fwd(dims, x["q"], x["k"], x["v"], blocks, ws=ws_a)
+        return blocks, msa.msa_sparse_attn_fwd(dims, x["q"], x["k"], x["v"], blocks, ws=ws_a, out_dtype=torch.bfloat16)
 
     for _ in range(args.warmup):
         blocks, _ = step()
     torch.cuda.synchronize()
     sel_tok = selected_tokens(blocks, w.block_k)  # sum_{i,r} |J|
     G = w.H_q // w.H_kv
-    # merge: read every valid partial (fp16 o + fp32 lse) and the selection, write fp32 out + lse
-    merge_bytes = (valid_slots(blocks, w.block_k) * G * (2 * w.d + 4) + w.B * w.N * w.H_q * (4 * w.d + 4)
+    # merge: read every valid partial (fp16 o + fp32 lse) and the selection, write bf16 out + fp32 lse
+    merge_bytes = (valid_slots(blocks, w.block_k) * G * (2 * w.d + 4) + w.B * w.N * w.H_q * (2 * w.d + 4)
                    + blocks.numel() * 4)
     attn_flops = 4.0 * w.d * G * sel_tok
     index_flops = 2.0 * w.d_idx * w.H_kv * w.N * (w.N + 1) / 2
@@ -436,7 +441,7 @@ def bench_prefill(args, world, rank, msa, pk):
     roof["peak_source"] = f"{pk['source']} bf16 burst"
     # e2e through the public API with pinned host buffers (H2D inputs, D2H output inside the region)
     host = {k: x[k].cpu().pin_memory() for k in ("q", "k", "v", "q_idx", "k_idx")}
-    out_host = [torch.empty(x["q"].shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+    out_host = [torch.empty(x["q"].shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = out_host[0].numel() * out_host[0].element_size()
 

@@ -87,6 +87,7 @@ def lib() -> ctypes.CDLL:
         L.msa_workspace_size.argtypes = [ctypes.c_int, D, ctypes.POINTER(ctypes.c_size_t)]
         L.msa_index_topk.argtypes = [D, P, P, P, P, P, S, P]
         L.msa_sparse_attn_fwd.argtypes = [D, P, P, P, P, P, P, P, S, P]
+        L.msa_sparse_attn_fwd_bf16.argtypes = [D, P, P, P, P, P, P, P, S, P]
         L.msa_sparse_attn_decode.argtypes = [D, P, P, P, P, P, P, P, P, P, P, S, P]
         L.msa_sparse_attn_decode_fp8idx.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, S, P]
         L.msa_quantize_e4m3_rows.argtypes = [P, ctypes.c_int64, ctypes.c_int, P, P, P]
@@ -116,7 +117,8 @@ def lib() -> ctypes.CDLL:
         L.msa_status_string.argtypes = [ctypes.c_int]
         L.msa_status_string.restype = ctypes.c_char_p
         L.msa_version.restype = ctypes.c_char_p
-        for fn in ("msa_workspace_size", "msa_index_topk", "msa_sparse_attn_fwd", "msa_sparse_attn_decode",
+        for fn in ("msa_workspace_size", "msa_index_topk", "msa_sparse_attn_fwd", "msa_sparse_attn_fwd_bf16",
+                   "msa_sparse_attn_decode",
                    "msa_sparse_attn_decode_fp8idx", "msa_quantize_e4m3_rows", "msa_kl_fwd_grad",
                    "msa_sparse_attn_bwd", "msa_index_topk_local", "msa_topk_merge", "msa_lse_idx_local",
                    "msa_lse_combine", "msa_get_device_status", "msa_kl_dense_fwd_grad"):
@@ -202,18 +204,26 @@ def msa_index_topk(dims: MsaDims, q_idx, k_idx, want_lse: bool = False, ws=None,
     return (blocks, lse) if want_lse else blocks
 
 
-def msa_sparse_attn_fwd(dims: MsaDims, q, k, v, blocks, want_lse: bool = True, ws=None, stream=None):
-    """Sparse attention forward. Returns out fp32 [B,N,H_q,d] and LSE fp32 [B,N,H_q] (or None)."""
+def msa_sparse_attn_fwd(dims: MsaDims, q, k, v, blocks, want_lse: bool = True, ws=None, stream=None,
+                        out_dtype=torch.float32, out=None):
+    """Sparse attention forward. Returns out [B,N,H_q,d] (fp32, or with out_dtype=torch.bfloat16 the
+    same values rounded to bf16 by msa_sparse_attn_fwd_bf16) and LSE fp32 [B,N,H_q] (or None).
+    `out` may be given (contiguous, of out_dtype) to be written in place."""
     dev = q.device
     _need(q, "q", (dims.B, dims.N, dims.H_q, dims.d), torch.bfloat16, dev)
     _need(k, "k", (dims.B, dims.N, dims.H_kv, dims.d), torch.bfloat16, dev)
     _need(v, "v", (dims.B, dims.N, dims.H_kv, dims.d), torch.bfloat16, dev)
     _need(blocks, "blocks", (dims.B, dims.N, dims.H_kv, dims.topk + 1), torch.int32, dev)
-    out = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    if out_dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError(f"out_dtype must be torch.float32 or torch.bfloat16, not {out_dtype}")
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype, device=dev)
+    _need(out, "out", tuple(q.shape), out_dtype, dev)
     lse = torch.empty(dims.B, dims.N, dims.H_q, dtype=torch.float32, device=dev) if want_lse else None
     ws = _ws(ws, MSA_OP_ATTN_FWD, dims, dev)
-    _check("msa_sparse_attn_fwd", lib().msa_sparse_attn_fwd(ctypes.byref(dims.c()), _p(q), _p(k), _p(v), _p(blocks),
-                                                            _p(out), _p(lse), _p(ws), ws.numel(), _stream(stream, dev)))
+    fn = "msa_sparse_attn_fwd" if out_dtype == torch.float32 else "msa_sparse_attn_fwd_bf16"
+    _check(fn, getattr(lib(), fn)(ctypes.byref(dims.c()), _p(q), _p(k), _p(v), _p(blocks), _p(out), _p(lse), _p(ws),
+                                  ws.numel(), _stream(stream, dev)))
     return out, lse
 
 

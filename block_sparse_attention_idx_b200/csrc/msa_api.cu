@@ -222,8 +222,8 @@ msa_status msa_index_topk(const msa_dims* d, const void* q_idx, const void* k_id
     return cuda_status(e);
 }
 
-msa_status msa_sparse_attn_fwd(const msa_dims* d, const void* q, const void* k, const void* v, const int32_t* blocks,
-                               float* out, float* lse, void* ws, size_t ws_bytes, msa_stream_t stream_) {
+static msa_status attn_fwd(const msa_dims* d, const void* q, const void* k, const void* v, const int32_t* blocks,
+                           void* out, bool out_bf16, float* lse, void* ws, size_t ws_bytes, msa_stream_t stream_) {
     msa_status s = check_common(d);
     if (s != MSA_OK) return s;
     if (!attn_rows_fit(d)) return MSA_ERR_UNSUPPORTED;
@@ -241,11 +241,23 @@ msa_status msa_sparse_attn_fwd(const msa_dims* d, const void* q, const void* k, 
     a.topk = d->topk; a.scale = eff_scale(d->scale, d->d);
     attn_carve(&a, static_cast<uint8_t*>(ws) + kStatusBytes);
     a.blocks = blocks;
-    a.out = static_cast<float*>(out);
+    a.out = out_bf16 ? nullptr : static_cast<float*>(out);
+    a.out_bf16 = out_bf16 ? static_cast<__nv_bfloat16*>(out) : nullptr;
     a.lse = lse;
     a.status = status;
     e = run_attn(a, q, k, v, num_sms(), st);
     return cuda_status(e);
+}
+
+msa_status msa_sparse_attn_fwd(const msa_dims* d, const void* q, const void* k, const void* v, const int32_t* blocks,
+                               float* out, float* lse, void* ws, size_t ws_bytes, msa_stream_t stream) {
+    return attn_fwd(d, q, k, v, blocks, out, false, lse, ws, ws_bytes, stream);
+}
+
+msa_status msa_sparse_attn_fwd_bf16(const msa_dims* d, const void* q, const void* k, const void* v,
+                                    const int32_t* blocks, void* out, float* lse, void* ws, size_t ws_bytes,
+                                    msa_stream_t stream) {
+    return attn_fwd(d, q, k, v, blocks, out, true, lse, ws, ws_bytes, stream);
 }
 
 // The decode step with a bf16 K_idx cache (k_idx_scale null) or an e4m3 one (codes + scales).

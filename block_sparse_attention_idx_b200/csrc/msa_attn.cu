@@ -620,9 +620,21 @@ __global__ void __launch_bounds__(256) k_attn_merge(AttnArgs a) {
                 overflow |= !isfinite(acc[y]);
                 acc[y] *= zi;
             }
-            float4* o4 = reinterpret_cast<float4*>(a.out + (((size_t)b * a.N + i) * a.H_q + hq) * D + d0);
-            o4[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-            o4[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+            const size_t oo = (((size_t)b * a.N + i) * a.H_q + hq) * D + d0;
+            if (a.out_bf16) {
+                uint4 pk;
+                uint32_t* pw = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+                for (int y = 0; y < 4; ++y) {
+                    const __nv_bfloat162 h = __floats2bfloat162_rn(acc[2 * y], acc[2 * y + 1]);
+                    pw[y] = *reinterpret_cast<const uint32_t*>(&h);
+                }
+                *reinterpret_cast<uint4*>(a.out_bf16 + oo) = pk;
+            } else {
+                float4* o4 = reinterpret_cast<float4*>(a.out + oo);
+                o4[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                o4[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+            }
             if (a.lse && d0 == 0) a.lse[((size_t)b * a.N + i) * a.H_q + hq] = lmax + logf(z);
         }
     }

@@ -2,6 +2,7 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -99,9 +100,10 @@ struct AttnArgs {
     float* lse_part;     // [B, N, H_kv, topk+1, G]
     int32_t* sched;      // [1]           next item to hand out
     const int32_t* blocks;
-    float* out;          // [B, N, H_q, d]  fp32 (the fp32-accumulated result)
+    float* out;          // [B, N, H_q, d]  fp32 (the fp32-accumulated result), or null when out_bf16 is set
     float* lse;          // [B, N, H_q] or null
     DevStatus* status;
+    __nv_bfloat16* out_bf16;  // [B, N, H_q, d]  the same result rounded to bf16 (nearest even), or null
 };
 size_t attn_ws_bytes(int B, int N, int H_q, int H_kv, int d, int block_k, int topk);
 void attn_carve(AttnArgs* a, void* base);

@@ -130,6 +130,17 @@ MSA_API msa_status msa_index_topk(const msa_dims *dims, const void *q_idx, const
 MSA_API msa_status msa_sparse_attn_fwd(const msa_dims *dims, const void *q, const void *k, const void *v,
                                const int32_t *blocks, float *out, float *lse, void *ws, size_t ws_bytes,
                                msa_stream_t stream);
+/*
+ * The same computation with a bf16 output: out bf16 [B, N, H_q, d] holds the fp32 result above
+ * rounded to the nearest bf16 (ties to even), element for element the value msa_sparse_attn_fwd
+ * writes, rounded. Half the output bytes (for callers that copy O back to the host or keep it in
+ * bf16); the rounding adds at most half a bf16 unit in the last place (2^-8 |o| or less) to the
+ * fp32 result's error.
+ * Same workspace (MSA_OP_ATTN_FWD), status and errors as msa_sparse_attn_fwd.
+ */
+MSA_API msa_status msa_sparse_attn_fwd_bf16(const msa_dims *dims, const void *q, const void *k, const void *v,
+                                            const int32_t *blocks, void *out, float *lse, void *ws, size_t ws_bytes,
+                                            msa_stream_t stream);
 
 /*
  * Sequence-parallel index branch ("4.1.1 · 监督与联合训练", section 3, eq (16)): P ranks each hold

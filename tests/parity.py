@@ -49,6 +49,18 @@ def check_attention(out_gpu, out_ref, lse_gpu=None, lse_ref=None):
     return float(e.max()), float(e.mean())
 
 
+def check_attention_bf16(out_gpu, out_ref):
+    """A bf16-stored output: the fp32 bound plus the storage rounding, half a bf16 unit in the last
+    place (bf16 keeps 8 significant bits, so at most 2^-8 |o|)."""
+    g = np.asarray(out_gpu, dtype=np.float64)
+    r = np.asarray(out_ref, dtype=np.float64)
+    e = np.abs(g - r)
+    bound = ATT_MAX + 2.0 ** -8 * np.abs(r)
+    assert (e <= bound).all(), f"bf16 attention error {e.max():.3e} above its bound"
+    assert e.mean() <= ATT_MEAN + 2.0 ** -8 * np.abs(r).mean(), f"bf16 attention mean abs error {e.mean():.3e}"
+    return float(e.max())
+
+
 def check_grad(g_gpu, g_ref, name):
     g = np.asarray(g_gpu, dtype=np.float64)
     r = np.asarray(g_ref, dtype=np.float64)

@@ -72,9 +72,13 @@ def test_null_and_misaligned_pointers_are_rejected_on_the_host():
     # misaligned pointers (never dereferenced: rejected before any launch)
     assert L.msa_sparse_attn_fwd(ctypes.byref(c), P(0x1001), P(0x2000), P(0x3000), P(0x4000), P(0x5000), None,
                                  P(0x10000), 1 << 30, None) == msa.MSA_ERR_INVALID_ARG
+    assert L.msa_sparse_attn_fwd_bf16(ctypes.byref(c), P(0x1000), P(0x2000), P(0x3000), P(0x4000), P(0x5008),
+                                      None, P(0x10000), 1 << 30, None) == msa.MSA_ERR_INVALID_ARG
     # workspace too small / misaligned
     assert L.msa_sparse_attn_fwd(ctypes.byref(c), P(0x1000), P(0x2000), P(0x3000), P(0x4000), P(0x5000), None,
                                  P(0x10000), 16, None) == msa.MSA_ERR_WORKSPACE
+    assert L.msa_sparse_attn_fwd_bf16(ctypes.byref(c), P(0x1000), P(0x2000), P(0x3000), P(0x4000), P(0x5000),
+                                      None, P(0x10000), 16, None) == msa.MSA_ERR_WORKSPACE
     assert L.msa_sparse_attn_fwd(ctypes.byref(c), P(0x1000), P(0x2000), P(0x3000), P(0x4000), P(0x5000), None,
                                  P(0x10010), 1 << 30, None) == msa.MSA_ERR_WORKSPACE
     # KL: unsupported group size for the KL kernel family

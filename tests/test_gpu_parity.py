@@ -7,7 +7,7 @@ import torch
 import block_sparse_attention_idx_b200 as msa
 import oracle
 from msa_inputs import small_prefill, WORKLOADS, prefill_inputs
-from parity import compare_blocks, check_attention, check_grad, KL_REL, NEAR_TIE
+from parity import compare_blocks, check_attention, check_attention_bf16, check_grad, KL_REL, NEAR_TIE
 
 pytestmark = pytest.mark.gpu
 
@@ -72,6 +72,26 @@ def test_sparse_attention_matches_oracle(name):
     og = out.float().cpu().reshape(dm.B * dm.N, dm.H_q, dm.d).numpy()[rows]
     lg = lse.cpu().reshape(dm.B * dm.N, dm.H_q).numpy()[rows]
     check_attention(og, oo, lg, ol)
+
+
+@pytest.mark.parametrize("name", ["tiny_cfg", "main_ragged", "main_two_seqs", "small_bk64"])
+def test_sparse_attention_bf16_output_is_the_rounded_fp32_output(name):
+    """msa_sparse_attn_fwd_bf16 writes the fp32 entry point's values rounded to nearest-even bf16,
+    bit for bit, and stays within the fp32 bound plus half a bf16 unit of the oracle."""
+    dm, od, x = mk(name, seed=2)
+    ob, _, _ = oracle.index_topk(od, x["q_idx"], x["k_idx"])
+    ob = ob.reshape(dm.B, dm.N, dm.H_kv, dm.topk + 1)
+    g = to_dev(x)
+    blocks = torch.from_numpy(ob).to(DEV)
+    o32, l32 = msa.msa_sparse_attn_fwd(dm, g["q"], g["k"], g["v"], blocks)
+    o16, l16 = msa.msa_sparse_attn_fwd(dm, g["q"], g["k"], g["v"], blocks, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert o16.dtype == torch.bfloat16
+    assert torch.equal(o16, o32.to(torch.bfloat16))
+    assert torch.equal(l16, l32)
+    rows = sample_rows(dm.B, dm.N, 120, seed=5)
+    oo, _ = oracle.sparse_attn(od, x["q"], x["k"], x["v"], ob, rows=rows)
+    check_attention_bf16(o16.float().cpu().reshape(dm.B * dm.N, dm.H_q, dm.d).numpy()[rows], oo)
 
 
 def test_dense_limit_k_covers_all_blocks():
