@@ -129,17 +129,17 @@ def valid_slots(blocks: torch.Tensor, block_k: int) -> int:
 # ncu capture of the kernel; it holds only for the kernel source it was measured on (sha256 of the
 # file), and reads null once that file changes.
 MEASURED_TRAFFIC = {
-    # prefill_8k capture (dram read 206,501,632 B + write 1,970,068,224 B per launch over 60,309,504
+    # prefill_8k capture (dram read 206,667,520 B + write 1,967,239,936 B per launch over 60,309,504
     # selected tokens), scaled by the selected tokens of the timed launch
     "attn_kv_outer": {"file": "block_sparse_attention_idx_b200/csrc/msa_attn.cu",
-                      "sha256": "269122850540640827a73f8abc33c40ae5a5a5d3d25f6e037bf24701df279270",
-                      "bytes_per_unit": (206501632 + 1970068224) / 60309504, "unit": "selected token",
+                      "sha256": "11bf6bf43a5ec6c71421ad4d730aa2ad534fab2788f3cb4cb682f2627595f9c0",
+                      "bytes_per_unit": (206667520 + 1967239936) / 60309504, "unit": "selected token",
                       "capture": "profiles/attn_kv_outer_prefill_8k.md"},
-    # training capture at N=8192 (dram read 990,195,968 B + write 133,234,176 B per launch over
+    # training capture at N=8192 (dram read 993,972,992 B + write 132,998,656 B per launch over
     # 60,309,504 selected tokens), scaled by the selected tokens of the timed launch
     "kl_kv_outer": {"file": "block_sparse_attention_idx_b200/csrc/msa_kl.cu",
-                    "sha256": "cd1f5a11cf7d642f437922350ed4ec35ece93132b5aabbecb7fd3a8cd1695605",
-                    "bytes_per_unit": (990195968 + 133234176) / 60309504, "unit": "selected token",
+                    "sha256": "5bdbc48d446823c16a19b6fb37cd93766e699a6ebb9553cb0633fa63e61a978d",
+                    "bytes_per_unit": (993972992 + 132998656) / 60309504, "unit": "selected token",
                     "capture": "profiles/kl_kv_outer_train_8k.md"},
     # attention backward at N=8192 (dram read 6,612,550,485 B + write 3,289,236,480 B per launch over
     # 60,309,504 selected tokens; most of it is the read-modify-write of dQ by the per-item reductions)

@@ -202,7 +202,7 @@ msa_status msa_index_topk(const msa_dims* d, const void* q_idx, const void* k_id
     cudaError_t e = status_init(status, st);
     if (e != cudaSuccess) return MSA_ERR_CUDA;
     IndexArgs a{d->B, d->N, d->H_kv, d->d_idx, d->block_k, d->topk, blocks, status, 0, d->N, nullptr, nullptr};
-    e = run_index_topk(a, q_idx, k_idx, st);
+    e = run_index_topk(a, q_idx, k_idx, num_sms(), st);
     if (e != cudaSuccess || !lse_idx) return cuda_status(e);
     // LSE_idx over the selected token sets: per-(query, selected block) sum-exps, merged
     Carver cv{static_cast<uint8_t*>(ws) + kStatusBytes};
@@ -354,7 +354,7 @@ msa_status msa_index_topk_local(const msa_dims* d, const void* q_idx, const void
     if (e != cudaSuccess) return MSA_ERR_CUDA;
     IndexArgs a{d->B, d->N, d->H_kv, d->d_idx, d->block_k, d->topk, nullptr, status, held->tok0[0], held->ntok[0],
                 cand_scores, cand_ids, held->n == 2 ? held->tok0[1] : 0, held->n == 2 ? held->ntok[1] : 0};
-    return cuda_status(run_index_topk(a, q_idx, k_idx_local, st));
+    return cuda_status(run_index_topk(a, q_idx, k_idx_local, num_sms(), st));
 }
 
 msa_status msa_topk_merge(const msa_dims* d, int P, const float* cand_scores, const int32_t* cand_ids,

@@ -52,7 +52,7 @@ struct IndexArgs {
     int32_t* cand_ids;    // [B, N, H_kv, topk]
     int tok0b, ntokb;
 };
-cudaError_t run_index_topk(const IndexArgs& a, const void* q_idx, const void* k_idx, cudaStream_t st);
+cudaError_t run_index_topk(const IndexArgs& a, const void* q_idx, const void* k_idx, int num_sms, cudaStream_t st);
 
 // ---------------------------------------------------------------- sequence-parallel indexer (msa_sp.cu)
 cudaError_t run_topk_merge(int B, int N, int H_kv, int block_k, int topk, int P, const float* cand_scores,

@@ -59,6 +59,23 @@ def test_index_topk_matches_oracle(name):
     assert err.max() <= 1e-3, f"LSE_idx max abs error {err.max():.3e}"
 
 
+def test_index_topk_matches_oracle_on_a_grid_of_two_ctas_per_sm():
+    """Ten sequences of 1000 tokens: 320 row tiles, enough for the launch that puts two index CTAs on
+    every SM (the smaller cases above run one per SM)."""
+    B, N, H_q, H_kv, d, d_idx, bk, k = 10, 1000, 64, 4, 128, 64, 128, 16
+    x = small_prefill(N, H_q, H_kv, d, d_idx, bk, k, seed=4242, B=B)
+    dm = msa.MsaDims(B, N, H_q, H_kv, d, d_idx, bk, k)
+    od = oracle.Dims(B, N, H_q, H_kv, d, d_idx, bk, k)
+    g = to_dev(x)
+    blocks, lse_idx = msa.msa_index_topk(dm, g["q_idx"], g["k_idx"], want_lse=True)
+    torch.cuda.synchronize()
+    ob, om, ol = oracle.index_topk(od, x["q_idx"], x["k_idx"], want_lse=True)
+    bad, near = compare_blocks(blocks.cpu().numpy(), ob, om)
+    assert bad == 0, f"{bad} selection rows differ (near-ties excluded: {near})"
+    same = np.all(blocks.cpu().numpy().reshape(ob.shape) == ob, axis=-1)
+    assert np.abs(lse_idx.cpu().numpy().reshape(ol.shape) - ol)[same].max() <= 1e-3
+
+
 @pytest.mark.parametrize("name", list(SHAPES))
 def test_sparse_attention_matches_oracle(name):
     dm, od, x = mk(name, seed=1)
