@@ -139,3 +139,73 @@ def test_random_decode_matches_oracle(seed):
         for r in range(H_kv):
             if same[b, r]:
                 check_attention(og[b, r * G:(r + 1) * G], oo[b, r * G:(r + 1) * G])
+
+
+SP_CASES = list(range(8))
+
+
+@pytest.mark.parametrize("seed", SP_CASES)
+def test_random_sequence_parallel_matches_single_device(seed):
+    """P emulated ranks (2-8) on random shapes, zig-zag and contiguous key assignments: the merged
+    selection is the single-device selection bit for bit, LSE_idx the same value summed in
+    another order."""
+    from block_sparse_attention_idx_b200 import sp
+    B, N, H_q, H_kv, d, d_idx, bk, k = draw_case(100 + seed)
+    P = int(np.random.default_rng(60_000 + seed).integers(2, 9))
+    x = small_prefill(N, H_q, H_kv, d, d_idx, bk, k, seed=70_000 + seed, B=B, device=DEV)
+    dm = msa.MsaDims(B, N, H_q, H_kv, d, d_idx, bk, k)
+    ref_blocks, ref_lse = msa.msa_index_topk(dm, x["q_idx"], x["k_idx"], want_lse=True)
+    for ranges_of in (sp.zigzag_ranges, sp.contiguous_ranges):
+        helds = [ranges_of(N, bk, P, p) for p in range(P)]
+        cs, ci = [], []
+        for h in helds:
+            c = (msa.msa_index_topk_local(dm, x["q_idx"], sp.local_keys(x["k_idx"], h), h) if h
+                 else sp.no_candidates(dm, x["q_idx"].device))
+            cs.append(c[0])
+            ci.append(c[1])
+        blocks = msa.msa_topk_merge(dm, torch.stack(cs), torch.stack(ci))
+        ml = torch.stack([msa.msa_lse_idx_local(dm, x["q_idx"], sp.local_keys(x["k_idx"], h), h, blocks) if h
+                          else sp.no_lse_pairs(dm, x["q_idx"].device) for h in helds])
+        lse = msa.msa_lse_combine(dm, ml)
+        torch.cuda.synchronize()
+        assert torch.equal(blocks, ref_blocks), ranges_of.__name__
+        assert torch.allclose(lse, ref_lse, rtol=0, atol=2e-5 * max(1.0, float(ref_lse.abs().max())))
+
+
+DENSE_CASES = list(range(6))
+
+
+@pytest.mark.parametrize("seed", DENSE_CASES)
+def test_random_dense_warmup_matches_oracle(seed):
+    """The dense warm-up KL on random shapes its kernels support (G in {2, 16}, matching head
+    dims, every block size): loss, both index gradients and the teacher LSE against the oracle's KL
+    with every causal block selected."""
+    rng = np.random.default_rng(80_000 + seed)
+    d, d_idx = [(128, 64), (64, 32)][rng.integers(2)]
+    G = int(rng.choice([2, 16]))
+    H_kv = int(rng.choice([1, 2, 4]))
+    bk = int(rng.choice([32, 64, 128]))
+    B = int(rng.integers(1, 3))
+    N = int(rng.integers(2, 900))
+    H_q = G * H_kv
+    nb = -(-N // bk)
+    x = small_prefill(N, H_q, H_kv, d, d_idx, bk, 4, seed=90_000 + seed, B=B)
+    g = {kk: vv.to(DEV) for kk, vv in x.items()}
+    dm = msa.MsaDims(B, N, H_q, H_kv, d, d_idx, bk, 1)
+    od = oracle.Dims(B, N, H_q, H_kv, d, d_idx, bk, max(nb - 1, 1))
+    gs = float(B * N * H_kv)
+    loss, dq, dk, lse = msa.msa_kl_dense_fwd_grad(dm, g["q"], g["k"], g["q_idx"], g["k_idx"], grad_scale=gs,
+                                                  want_lse=True)
+    torch.cuda.synchronize()
+    ids = np.arange(nb, dtype=np.int32)[None, :].repeat(N, 0)
+    ids[ids > (np.arange(N) // bk)[:, None]] = -1
+    # one more slot than the oracle's k + 1 is never needed: k + 1 = max(nb, 2) >= nb
+    full = np.full((N, od.topk + 1), -1, dtype=np.int32)
+    full[:, :nb] = ids
+    blocks = np.broadcast_to(full[None, :, None, :], (B, N, H_kv, od.topk + 1)).copy()
+    ol, _, odq, odk = oracle.kl(od, x["q"], x["k"], x["q_idx"], x["k_idx"], blocks, grad_scale=gs)
+    _, olse = oracle.sparse_attn(od, x["q"], x["k"], x["v"], blocks)
+    assert abs(float(loss.item()) - ol) <= KL_REL * max(abs(ol), 1e-12), f"loss {loss.item()} vs {ol}"
+    check_grad(dq.cpu().numpy().reshape(odq.shape), odq, "dq_idx")
+    check_grad(dk.cpu().numpy(), odk, "dk_idx")
+    assert np.abs(lse.cpu().numpy().reshape(olse.shape) - olse).max() <= 2e-3
