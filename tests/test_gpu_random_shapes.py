@@ -209,3 +209,58 @@ def test_random_dense_warmup_matches_oracle(seed):
     check_grad(dq.cpu().numpy().reshape(odq.shape), odq, "dq_idx")
     check_grad(dk.cpu().numpy(), odk, "dk_idx")
     assert np.abs(lse.cpu().numpy().reshape(olse.shape) - olse).max() <= 2e-3
+
+
+FP8_CASES = list(range(6))
+
+
+@pytest.mark.parametrize("seed", FP8_CASES)
+def test_random_fp8_decode_matches_oracle(seed):
+    """The FP8-index decode step on random shapes: the quantiser's codes and scales bit-exact, then
+    selection (outside near-ties), cutoff margins and attention against the oracle's FP8 decode."""
+    rng = np.random.default_rng(95_000 + seed)
+    d, d_idx = [(128, 64), (64, 32), (128, 32), (64, 64)][rng.integers(4)]
+    bk = int(rng.choice([32, 64, 128]))
+    H_kv = int(rng.choice([1, 2, 4, 8]))
+    G = int(rng.choice([1, 2, 4, 8, 16]))
+    while H_kv * G > 64:
+        G //= 2
+    H_q = H_kv * G
+    B = int(rng.integers(1, 5))
+    L = int(rng.integers(200, 5000))
+    k = int(rng.integers(1, 17))
+    lens = rng.integers(1, L + 1, size=B).astype(np.int32)
+    lens[-1] = L
+    gen = torch.Generator().manual_seed(96_000 + seed)
+    mk = lambda *s: torch.randn(*s, generator=gen).to(torch.bfloat16)
+    x = dict(q=mk(B, H_q, d), q_idx=mk(B, H_kv, d_idx), k_cache=mk(B, L, H_kv, d), v_cache=mk(B, L, H_kv, d),
+             k_idx_cache=mk(B, L, d_idx), cache_len=torch.from_numpy(lens))
+    g = {kk: vv.to(DEV) for kk, vv in x.items()}
+    dm = msa.MsaDims(B, L, H_q, H_kv, d, d_idx, bk, k)
+    kcodes, kscale = msa.msa_quantize_e4m3_rows(g["k_idx_cache"])
+    out, blocks, margin = msa.msa_sparse_attn_decode_fp8idx(dm, g["cache_len"], g["q"], g["q_idx"], g["k_cache"],
+                                                            g["v_cache"], kcodes, kscale, want_margin=True)
+    torch.cuda.synchronize()
+    okc, oks = oracle.quantize_e4m3_rows(x["k_idx_cache"])
+    gc = kcodes.cpu().numpy().copy()
+    gc[gc == 0x80] = 0  # a negative value rounded to zero may keep its sign bit (either code is zero)
+    okc0 = okc.copy()
+    okc0[okc0 == 0x80] = 0
+    np.testing.assert_array_equal(gc, okc0)
+    np.testing.assert_array_equal(kscale.cpu().numpy(), oks)
+    od = oracle.Dims(B, L, H_q, H_kv, d, d_idx, bk, k)
+    ob, om, oo, _ = oracle.decode_fp8idx(od, x["cache_len"], x["q"], x["q_idx"], x["k_cache"], x["v_cache"], okc,
+                                         oks)
+    gb = blocks.cpu().numpy()
+    bad, near = compare_blocks(gb, ob, om)
+    assert bad == 0
+    gm = margin.cpu().numpy()
+    assert np.array_equal(np.isinf(gm), np.isinf(om))
+    fin = np.isfinite(om)
+    assert np.abs(gm[fin] - om[fin]).max(initial=0.0) <= 1e-4
+    same = np.all(gb == ob, axis=-1)
+    og = out.cpu().numpy()
+    for b in range(B):
+        for r in range(H_kv):
+            if same[b, r]:
+                check_attention(og[b, r * G:(r + 1) * G], oo[b, r * G:(r + 1) * G])
