@@ -6,7 +6,7 @@ import torch
 
 import block_sparse_attention_idx_b200 as msa
 import oracle
-from msa_inputs import small_prefill, WORKLOADS, prefill_inputs
+from msa_inputs import small_prefill
 from parity import compare_blocks, check_attention, check_attention_bf16, check_grad, KL_REL, NEAR_TIE
 
 pytestmark = pytest.mark.gpu
