@@ -13,6 +13,7 @@
 #include <cuda_fp8.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "msa_common.cuh"
 #include "msa_internal.h"
@@ -583,21 +584,24 @@ __global__ void __launch_bounds__(256) k_dec_topk(DecodeArgs a) {
 
 // Decode attention, persistent: one CTA per SM takes the (sequence, group, slot) items c, c + grid,
 // ... of the selection. Warp 8 streams each item's K and V block and the group's Q rows by TMA
-// (64-column boxes, 128B-swizzled) through a 3-stage ring; warps 0-7 compute the item: S = Q.K^T
+// (64-column boxes, 128B-swizzled) through a 3-stage ring; warps 0-7 compute the items: S = Q.K^T
 // for the G heads (mma.sync with Q by ldmatrix, 16-token units spread over the warps), the softmax
 // statistics (combined across warps in shared memory), P as bf16 in shared memory, then P.V split
-// by output columns. The slot's partial is normalised by the sum of the bf16-rounded P that the MMA
+// by output columns. With NG = 2 the eight warps form two groups of four that take alternate
+// items, so two items' dependent mma.sync chains are in flight at once (groups have their own P
+// tile, reduction rows and named barrier); NG = 1 keeps all eight on every item for G = 32, whose
+// two 16-row Q tiles per stage leave no room for a second P tile. The slot's partial is normalised by the sum of the bf16-rounded P that the MMA
 // multiplies, as in the prefill attention, with its LSE from the exact sum; k_dec_combine merges
 // the slots.
 constexpr int kAttnStages = 3;
 constexpr int kAttnWarps = 8;
 
-template <int D, int BK>
+template <int D, int BK, int NG, int MT>
 struct AttnSmem {
     alignas(1024) __nv_bfloat16 kv[kAttnStages][2][BK * D];  // [stage][K, V][D/64 halves of BK x 64]
-    __nv_bfloat16 qt[kAttnStages][2][16 * D];                // [stage][row tile][D/64 halves of 16 x 64]
-    __nv_bfloat16 p[16][BK + 8];                             // P rows (heads) of one 16-row tile
-    float red[3][kAttnWarps][16];                            // per-warp maxima, exact sums, rounded sums
+    __nv_bfloat16 qt[kAttnStages][MT][16 * D];               // [stage][row tile][D/64 halves of 16 x 64]
+    __nv_bfloat16 p[NG][16][BK + 8];                         // [group] P rows (heads) of one 16-row tile
+    float red[NG][3][kAttnWarps / NG][16];                   // [group] per-warp maxima, exact sums, rounded sums
     uint64_t full[kAttnStages], empty[kAttnStages];
 };
 
@@ -611,14 +615,15 @@ __device__ __forceinline__ void ldsm_x2_trans(uint32_t addr, uint32_t& r0, uint3
     asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
 }
 
-template <int D, int BK>
+template <int D, int BK, int NG, int MT>
 __global__ void __launch_bounds__((kAttnWarps + 1) * 32, 1)
     k_dec_attn_tma(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    const __grid_constant__ CUtensorMap tm_q, DecodeArgs a) {
-    using Sm = AttnSmem<D, BK>;
-    constexpr int NU = BK / 16;                              // 16-token units
-    constexpr int UPW = (NU + kAttnWarps - 1) / kAttnWarps;  // units per warp
-    constexpr int DW = D / kAttnWarps;                       // output columns per warp (8 or 16)
+    using Sm = AttnSmem<D, BK, NG, MT>;
+    constexpr int GW = kAttnWarps / NG;          // warps per group
+    constexpr int NU = BK / 16;                  // 16-token units
+    constexpr int UPW = (NU + GW - 1) / GW;      // units per warp
+    constexpr int DW = D / GW;                   // output columns per warp (8, 16 or 32)
     constexpr uint32_t kTileBytes = BK * D * 2;
     extern __shared__ uint8_t attn_raw[];
     Sm& s = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(attn_raw) + 1023) & ~uintptr_t(1023));
@@ -630,7 +635,7 @@ __global__ void __launch_bounds__((kAttnWarps + 1) * 32, 1)
     if (threadIdx.x == 0) {
         for (int x = 0; x < kAttnStages; ++x) {
             mbar_init(&s.full[x], 1);
-            mbar_init(&s.empty[x], kAttnWarps);  // each consumer warp releases the stage after its reads
+            mbar_init(&s.empty[x], GW);  // each warp of the consuming group releases the stage after its reads
         }
         fence_mbar_init();
     }
@@ -663,16 +668,21 @@ __global__ void __launch_bounds__((kAttnWarps + 1) * 32, 1)
         return;
     }
     const float sl2 = a.scale * 1.4426950408889634f;
-    int n = 0;
+    const int grp = warp / GW, lw = warp % GW;  // this warp's group and its rank in the group
+    const uint32_t bar = 1 + grp;               // the group's named barrier
+    int n_all = 0;                              // selected items seen so far (both groups)
     int c_next = blockIdx.x < n_items ? a.sel[blockIdx.x] : -1;
     for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
         const int c = c_next;
         if (it + (int)gridDim.x < n_items) c_next = a.sel[it + gridDim.x];  // in flight during this item
         float* lse_out = a.lse_part + (size_t)it * G;
         if (c < 0) {
-            for (int h = threadIdx.x; h < G; h += kAttnWarps * 32) lse_out[h] = -INFINITY;
+            if (grp == 0)
+                for (int h = lw * 32 + lane; h < G; h += GW * 32) lse_out[h] = -INFINITY;
             continue;
         }
+        const int n = n_all++;  // the item's place in the stage ring
+        if (n % NG != grp) continue;
         const int b = (it / K1) / a.H_kv;
         const int len = dec_len(a, b);
         const int st = n % kAttnStages;
@@ -680,7 +690,7 @@ __global__ void __launch_bounds__((kAttnWarps + 1) * 32, 1)
         float* o_out = a.o_part + (size_t)it * G * D;
         const bool ok = __all_sync(0xffffffffu, mbar_wait(&s.full[st], (n / kAttnStages) & 1, a.status, 0x923));
         // every warp learns whether any warp timed out
-        if (bar_red_or(1, kAttnWarps * 32, !ok)) break;
+        if (bar_red_or(bar, GW * 32, !ok)) break;
         for (int mt = 0; mt < n_mt; ++mt) {
             const int h0 = mt * 16 + g, h1 = h0 + 8;
             const uint32_t qbase = smem_u32(&s.qt[st][mt][0]);
@@ -689,7 +699,7 @@ __global__ void __launch_bounds__((kAttnWarps + 1) * 32, 1)
             float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
             for (int j = 0; j < UPW; ++j) {
-                const int u = warp + kAttnWarps * j;
+                const int u = lw + GW * j;
 #pragma unroll
                 for (int tl = 0; tl < 2; ++tl) sc[j][tl][0] = sc[j][tl][1] = sc[j][tl][2] = sc[j][tl][3] = 0.f;
                 if (u < NU) {
@@ -727,21 +737,21 @@ __global__ void __launch_bounds__((kAttnWarps + 1) * 32, 1)
                 mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
             }
             if (t4 == 0) {
-                s.red[0][warp][g] = mx0;
-                s.red[0][warp][g + 8] = mx1;
+                s.red[grp][0][lw][g] = mx0;
+                s.red[grp][0][lw][g + 8] = mx1;
             }
-            bar_sync_named(1, kAttnWarps * 32);
+            bar_sync_named(bar, GW * 32);
             float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-            for (int w = 0; w < kAttnWarps; ++w) {
-                m0 = fmaxf(m0, s.red[0][w][g]);
-                m1 = fmaxf(m1, s.red[0][w][g + 8]);
+            for (int w = 0; w < GW; ++w) {
+                m0 = fmaxf(m0, s.red[grp][0][w][g]);
+                m1 = fmaxf(m1, s.red[grp][0][w][g + 8]);
             }
             // P (bf16 into shared memory); l: exact sums, lr: sums of the rounded P
             float l0 = 0.f, l1 = 0.f, lr0 = 0.f, lr1 = 0.f;
 #pragma unroll
             for (int j = 0; j < UPW; ++j) {
-                const int u = warp + kAttnWarps * j;
+                const int u = lw + GW * j;
                 if (u >= NU) continue;
 #pragma unroll
                 for (int tl = 0; tl < 2; ++tl) {
@@ -755,8 +765,8 @@ __global__ void __launch_bounds__((kAttnWarps + 1) * 32, 1)
                     lr0 += __uint_as_float(w0 << 16) + __uint_as_float(w0 & 0xffff0000u);
                     lr1 += __uint_as_float(w1 << 16) + __uint_as_float(w1 & 0xffff0000u);
                     const int col = 16 * u + 8 * tl + 2 * t4;
-                    *reinterpret_cast<uint32_t*>(&s.p[g][col]) = w0;
-                    *reinterpret_cast<uint32_t*>(&s.p[g + 8][col]) = w1;
+                    *reinterpret_cast<uint32_t*>(&s.p[grp][g][col]) = w0;
+                    *reinterpret_cast<uint32_t*>(&s.p[grp][g + 8][col]) = w1;
                 }
             }
 #pragma unroll
@@ -767,12 +777,12 @@ __global__ void __launch_bounds__((kAttnWarps + 1) * 32, 1)
                 lr1 += __shfl_xor_sync(0xffffffffu, lr1, o);
             }
             if (t4 == 0) {
-                s.red[1][warp][g] = l0;
-                s.red[1][warp][g + 8] = l1;
-                s.red[2][warp][g] = lr0;
-                s.red[2][warp][g + 8] = lr1;
+                s.red[grp][1][lw][g] = l0;
+                s.red[grp][1][lw][g + 8] = l1;
+                s.red[grp][2][lw][g] = lr0;
+                s.red[grp][2][lw][g + 8] = lr1;
             }
-            bar_sync_named(1, kAttnWarps * 32);
+            bar_sync_named(bar, GW * 32);
             // O[:, this warp's DW columns] = P.V over all tokens, even and odd units in two
             // accumulator sets (two independent MMA chains)
             float ov[DW / 8][4], ow[DW / 8][4];
@@ -787,17 +797,20 @@ __global__ void __launch_bounds__((kAttnWarps + 1) * 32, 1)
                     const int prow = ((lane >> 3) & 1) * 8 + (lane & 7), pcol = 16 * u + 8 * (lane >> 4);
                     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                                  : "=r"(pa[0]), "=r"(pa[1]), "=r"(pa[2]), "=r"(pa[3])
-                                 : "r"(smem_u32(&s.p[prow][pcol])));
+                                 : "r"(smem_u32(&s.p[grp][prow][pcol])));
                 }
                 const int vrow = 16 * u + 8 * ((lane >> 3) & 1) + (lane & 7);
-                if constexpr (DW == 16) {
-                    uint32_t b00, b01, b10, b11;
-                    ldsm_x4_trans(vbase + tile_off<BK>(vrow, warp * DW + 8 * (lane >> 4)), b00, b01, b10, b11);
-                    mma_16816_bf16(acc[0], pa, b00, b01);
-                    mma_16816_bf16(acc[1], pa, b10, b11);
+                if constexpr (DW >= 16) {
+#pragma unroll
+                    for (int np = 0; np < DW / 16; ++np) {
+                        uint32_t b00, b01, b10, b11;
+                        ldsm_x4_trans(vbase + tile_off<BK>(vrow, lw * DW + 16 * np + 8 * (lane >> 4)), b00, b01, b10, b11);
+                        mma_16816_bf16(acc[2 * np], pa, b00, b01);
+                        mma_16816_bf16(acc[2 * np + 1], pa, b10, b11);
+                    }
                 } else {
                     uint32_t b00, b01;
-                    ldsm_x2_trans(vbase + tile_off<BK>(vrow, warp * DW), b00, b01);
+                    ldsm_x2_trans(vbase + tile_off<BK>(vrow, lw * DW), b00, b01);
                     mma_16816_bf16(acc[0], pa, b00, b01);
                 }
             }
@@ -812,27 +825,27 @@ __global__ void __launch_bounds__((kAttnWarps + 1) * 32, 1)
                 for (int e = 0; e < 4; ++e) ov[nd][e] += ow[nd][e];
             float L0 = 0.f, L1 = 0.f, Lr0 = 0.f, Lr1 = 0.f;
 #pragma unroll
-            for (int w = 0; w < kAttnWarps; ++w) {
-                L0 += s.red[1][w][g];
-                L1 += s.red[1][w][g + 8];
-                Lr0 += s.red[2][w][g];
-                Lr1 += s.red[2][w][g + 8];
+            for (int w = 0; w < GW; ++w) {
+                L0 += s.red[grp][1][w][g];
+                L1 += s.red[grp][1][w][g + 8];
+                Lr0 += s.red[grp][2][w][g];
+                Lr1 += s.red[grp][2][w][g + 8];
             }
             const float i0 = 1.f / Lr0, i1 = 1.f / Lr1;
 #pragma unroll
             for (int nd = 0; nd < DW / 8; ++nd) {
-                const int col = warp * DW + 8 * nd + 2 * t4;
+                const int col = lw * DW + 8 * nd + 2 * t4;
                 if (h0 < G) *reinterpret_cast<float2*>(o_out + (size_t)h0 * D + col) = make_float2(ov[nd][0] * i0, ov[nd][1] * i0);
                 if (h1 < G) *reinterpret_cast<float2*>(o_out + (size_t)h1 * D + col) = make_float2(ov[nd][2] * i1, ov[nd][3] * i1);
             }
-            if (warp == 0 && t4 == 0) {
+            if (lw == 0 && t4 == 0) {
                 if (h0 < G) lse_out[h0] = m0 * 0.6931471805599453f + logf(L0);
                 if (h1 < G) lse_out[h1] = m1 * 0.6931471805599453f + logf(L1);
             }
-            // the P tile and the reduction rows are rewritten only after the next row tile's (or
-            // item's) first barrier, which every warp reaches after its reads here
+            // the group's P tile and reduction rows are rewritten only after the next row tile's (or
+            // the group's next item's) first barrier, which every warp of the group reaches after its
+            // reads here
         }
-        ++n;
     }
     pdl_trigger();
 }
@@ -983,15 +996,20 @@ cudaError_t run_decode(const DecodeArgs& a, const void* q, const void* q_idx, co
         if (e != cudaSuccess) return e;
         return launch_pdl(kern, dim3(num_sms), dim3((kAttnWarps + 1) * 32), smem, st, tk, tv, tq, a);
     };
+    // two consumer groups when one 16-row Q tile holds the group's heads, else one (G = 32)
+    auto launch_nm = [&](auto d_c, auto bk_c) -> cudaError_t {
+        constexpr int D = decltype(d_c)::value, BK = decltype(bk_c)::value;
+        if (a.H_q / a.H_kv <= 16) return launch(k_dec_attn_tma<D, BK, 2, 1>, sizeof(AttnSmem<D, BK, 2, 1>));
+        return launch(k_dec_attn_tma<D, BK, 1, 2>, sizeof(AttnSmem<D, BK, 1, 2>));
+    };
+    using I64 = std::integral_constant<int, 64>;
+    using I128 = std::integral_constant<int, 128>;
+    using I32 = std::integral_constant<int, 32>;
     cudaError_t e;
     if (a.d == 128)
-        e = a.block_k == 128 ? launch(k_dec_attn_tma<128, 128>, sizeof(AttnSmem<128, 128>))
-            : a.block_k == 64 ? launch(k_dec_attn_tma<128, 64>, sizeof(AttnSmem<128, 64>))
-                              : launch(k_dec_attn_tma<128, 32>, sizeof(AttnSmem<128, 32>));
+        e = a.block_k == 128 ? launch_nm(I128{}, I128{}) : a.block_k == 64 ? launch_nm(I128{}, I64{}) : launch_nm(I128{}, I32{});
     else
-        e = a.block_k == 128 ? launch(k_dec_attn_tma<64, 128>, sizeof(AttnSmem<64, 128>))
-            : a.block_k == 64 ? launch(k_dec_attn_tma<64, 64>, sizeof(AttnSmem<64, 64>))
-                              : launch(k_dec_attn_tma<64, 32>, sizeof(AttnSmem<64, 32>));
+        e = a.block_k == 128 ? launch_nm(I64{}, I128{}) : a.block_k == 64 ? launch_nm(I64{}, I64{}) : launch_nm(I64{}, I32{});
     if (e != cudaSuccess) return e;
     const dim3 cgrid((a.B * a.H_q * 32 + 255) / 256);
     e = a.d == 128 ? launch_pdl(k_dec_combine<128>, cgrid, dim3(256), 0, st, a, static_cast<float*>(out))
