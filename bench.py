@@ -150,12 +150,12 @@ MEASURED_TRAFFIC = {
     # decode scans at 16 x 131,072 (read + write per launch over 16 x 130,944 scanned tokens), scaled
     # by the scanned tokens of the timed launch
     "dec_scan": {"file": "block_sparse_attention_idx_b200/csrc/msa_decode.cu",
-                 "sha256": "5420651959775c3eda231b8e78682d94e3e90e5128be9c7164f520c3120e3f31",
-                 "bytes_per_unit": (268226784 + 696704) / (16 * 130944), "unit": "scanned token",
+                 "sha256": "6536683ca241866d06dbf3a74a7c697920f32a8220c31477d321aeb30d8c10d5",
+                 "bytes_per_unit": (268228416 + 510176) / (16 * 130944), "unit": "scanned token",
                  "capture": "profiles/decode_16x256k.md"},
     "dec_scan_e4m3": {"file": "block_sparse_attention_idx_b200/csrc/msa_decode.cu",
-                      "sha256": "5420651959775c3eda231b8e78682d94e3e90e5128be9c7164f520c3120e3f31",
-                      "bytes_per_unit": (142527168 + 238272) / (16 * 130944), "unit": "scanned token",
+                      "sha256": "6536683ca241866d06dbf3a74a7c697920f32a8220c31477d321aeb30d8c10d5",
+                      "bytes_per_unit": (142535232 + 305984) / (16 * 130944), "unit": "scanned token",
                       "capture": "profiles/decode_16x256k.md"},
 }
 
