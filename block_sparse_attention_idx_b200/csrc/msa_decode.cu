@@ -671,10 +671,15 @@ __global__ void __launch_bounds__((kAttnWarps + 1) * 32, 1)
     const int grp = warp / GW, lw = warp % GW;  // this warp's group and its rank in the group
     const uint32_t bar = 1 + grp;               // the group's named barrier
     int n_all = 0;                              // selected items seen so far (both groups)
+    // the next item's block and its sequence's length are loaded while this item runs
     int c_next = blockIdx.x < n_items ? a.sel[blockIdx.x] : -1;
+    int len_next = blockIdx.x < n_items ? dec_len(a, (blockIdx.x / K1) / a.H_kv) : 1;
     for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
-        const int c = c_next;
-        if (it + (int)gridDim.x < n_items) c_next = a.sel[it + gridDim.x];  // in flight during this item
+        const int c = c_next, len = len_next;
+        if (it + (int)gridDim.x < n_items) {
+            c_next = a.sel[it + gridDim.x];
+            len_next = dec_len(a, ((it + (int)gridDim.x) / K1) / a.H_kv);
+        }
         float* lse_out = a.lse_part + (size_t)it * G;
         if (c < 0) {
             if (grp == 0)
@@ -683,8 +688,6 @@ __global__ void __launch_bounds__((kAttnWarps + 1) * 32, 1)
         }
         const int n = n_all++;  // the item's place in the stage ring
         if (n % NG != grp) continue;
-        const int b = (it / K1) / a.H_kv;
-        const int len = dec_len(a, b);
         const int st = n % kAttnStages;
         const uint32_t kbase = smem_u32(&s.kv[st][0][0]), vbase = smem_u32(&s.kv[st][1][0]);
         float* o_out = a.o_part + (size_t)it * G * D;
