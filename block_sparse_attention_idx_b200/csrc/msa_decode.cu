@@ -269,23 +269,26 @@ __global__ void __launch_bounds__(256) k_quant_e4m3_rows(const __nv_bfloat16* __
 // at this tile size a CTA must keep more tiles in flight than the bf16 scan to reach the same HBM
 // rate, and its per-tile compute (widening plus 32 MMAs) needs more warps to keep up.
 constexpr int kScan8Warps = 8;
-constexpr int kScan8Stages = 16;
+constexpr int kScan8Stages = 12;  // stages of two consecutive blocks each
 
 template <int DI, int BK>
 struct ScanSmem8 {
-    alignas(1024) uint8_t tile[kScan8Stages][BK * DI];
+    alignas(1024) uint8_t tile[kScan8Stages][2 * BK * DI];  // [stage][block 2k, block 2k+1]
     float scale[kScan8Warps][BK];
     uint64_t full[kScan8Stages], empty[kScan8Stages];
 };
 
 template <int DI, int BK>
 __global__ void __launch_bounds__((kScan8Warps + 1) * 32, 1)
-    k_dec_scan_e4m3(const __grid_constant__ CUtensorMap tm_codes, DecodeArgs a,
-                    const __nv_bfloat16* __restrict__ q_idx) {
+    k_dec_scan_e4m3(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_codes2,
+                    DecodeArgs a, const __nv_bfloat16* __restrict__ q_idx) {
     static_assert(DI % 32 == 0 && BK % 32 == 0, "chunk pairs and 32-row scale loads");
-    // item n uses stage n % stages and warp n % warps: the next item on a stage then belongs to the
-    // same warp, so no warp can wait on a stage's full barrier a phase early
-    static_assert(kScan8Stages % kScan8Warps == 0, "stages must be a multiple of the consumer warps");
+    // The CTA's blocks go in pairs: pair k (blocks 2k, 2k+1) uses stage k % stages, one 2*BK-token
+    // TMA box when both are consecutive blocks of one sequence (the common case: half the copies of
+    // one box per block), else one box per block. Block n goes to warp n % warps, so the two blocks
+    // of a stage's next use belong to the same two warps and no warp can wait on a stage's full
+    // barrier a phase early.
+    static_assert((2 * kScan8Stages) % kScan8Warps == 0, "a stage's uses must cycle through the same warps");
     using Sm = ScanSmem8<DI, BK>;
     extern __shared__ uint8_t scan8_raw[];
     Sm& s = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(scan8_raw) + 1023) & ~uintptr_t(1023));
@@ -294,7 +297,7 @@ __global__ void __launch_bounds__((kScan8Warps + 1) * 32, 1)
     if (threadIdx.x == 0) {
         for (int x = 0; x < kScan8Stages; ++x) {
             mbar_init(&s.full[x], 1);
-            mbar_init(&s.empty[x], 1);
+            mbar_init(&s.empty[x], 2);  // the warps of the stage's two blocks (a last lone block: one, never reused)
         }
         fence_mbar_init();
     }
@@ -303,16 +306,26 @@ __global__ void __launch_bounds__((kScan8Warps + 1) * 32, 1)
     const int count = scan_range(a, BK, cur);
     if (warp == kScan8Warps) {
         if (lane == 0) {
-            int n = 0;
-            for (; n < count; ++n, scan_advance(a, BK, cur, 1)) {
-                const int st = n % kScan8Stages;
-                if (n >= kScan8Stages && !mbar_wait(&s.empty[st], ((n / kScan8Stages) - 1) & 1, a.status, 0x911))
+            int k = 0;
+            for (int n = 0; n < count; n += 2, ++k) {
+                const int st = k % kScan8Stages;
+                if (k >= kScan8Stages && !mbar_wait(&s.empty[st], ((k / kScan8Stages) - 1) & 1, a.status, 0x911))
                     break;
-                mbar_arrive_expect_tx(&s.full[st], (uint32_t)(BK * DI));
-                tma_load_3d(s.tile[st], &tm_codes, &s.full[st], 0, cur.blk * BK, cur.b);
+                ScanCursor nxt = cur;
+                scan_advance(a, BK, nxt, 1);  // block n + 1
+                const bool two = n + 1 < count;
+                mbar_arrive_expect_tx(&s.full[st], (uint32_t)((two ? 2 : 1) * BK * DI));
+                if (two && nxt.b == cur.b && nxt.blk == cur.blk + 1) {
+                    tma_load_3d(s.tile[st], &tm_codes2, &s.full[st], 0, cur.blk * BK, cur.b);
+                } else {
+                    tma_load_3d(s.tile[st], &tm_codes, &s.full[st], 0, cur.blk * BK, cur.b);
+                    if (two) tma_load_3d(s.tile[st] + BK * DI, &tm_codes, &s.full[st], 0, nxt.blk * BK, nxt.b);
+                }
+                cur = nxt;
+                scan_advance(a, BK, cur, 1);  // block n + 2
             }
             // no copy of ours may still be landing when the CTA leaves
-            for (int m = max(0, n - kScan8Stages); m < n; ++m)
+            for (int m = max(0, k - kScan8Stages); m < k; ++m)
                 mbar_wait(&s.full[m % kScan8Stages], (m / kScan8Stages) & 1, a.status, 0x912);
         }
         pdl_trigger();
@@ -370,9 +383,9 @@ __global__ void __launch_bounds__((kScan8Warps + 1) * 32, 1)
             sq0 = __shfl_sync(0xffffffffu, sq, 8 * t4);      // lane of (group 2*t4, t4 = 0)
             sq1 = __shfl_sync(0xffffffffu, sq, 8 * t4 + 4);  // lane of (group 2*t4+1, t4 = 0)
         }
-        const int st = n % kScan8Stages;
-        if (!__all_sync(0xffffffffu, mbar_wait(&s.full[st], (n / kScan8Stages) & 1, a.status, 0x913))) break;
-        const uint32_t base = smem_u32(s.tile[st]);
+        const int pair = n >> 1, st = pair % kScan8Stages;
+        if (!__all_sync(0xffffffffu, mbar_wait(&s.full[st], (pair / kScan8Stages) & 1, a.status, 0x913))) break;
+        const uint32_t base = smem_u32(s.tile[st]) + (uint32_t)((n & 1) * BK * DI);  // this block's half
         float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
         for (int mt = 0; mt < BK / 16; ++mt) {
@@ -932,15 +945,17 @@ cudaError_t run_decode(const DecodeArgs& a, const void* q, const void* q_idx, co
     const auto* qi = static_cast<const __nv_bfloat16*>(q_idx);
     if (a.k_idx_scale) {
         ProfScope ps("dec_scan_e4m3", st);
-        CUtensorMap tm;
+        CUtensorMap tm, tm2;  // boxes of one block and of two consecutive blocks
         if (!make_tmap_3d_u8(&tm, k_idx_cache, (uint64_t)a.d_idx, (uint64_t)a.L, (uint64_t)a.B, (uint64_t)a.d_idx,
-                             (uint64_t)a.L * a.d_idx, (uint32_t)a.d_idx, (uint32_t)a.block_k, a.d_idx))
+                             (uint64_t)a.L * a.d_idx, (uint32_t)a.d_idx, (uint32_t)a.block_k, a.d_idx) ||
+            !make_tmap_3d_u8(&tm2, k_idx_cache, (uint64_t)a.d_idx, (uint64_t)a.L, (uint64_t)a.B, (uint64_t)a.d_idx,
+                             (uint64_t)a.L * a.d_idx, (uint32_t)a.d_idx, (uint32_t)(2 * a.block_k), a.d_idx))
             return cudaErrorInvalidValue;
         auto launch = [&](auto kern, size_t bytes) -> cudaError_t {
             const size_t smem = bytes + 1024;
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return e;
-            kern<<<num_sms, (kScan8Warps + 1) * 32, smem, st>>>(tm, a, qi);
+            kern<<<num_sms, (kScan8Warps + 1) * 32, smem, st>>>(tm, tm2, a, qi);
             return cudaGetLastError();
         };
         cudaError_t e;
