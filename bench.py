@@ -150,12 +150,12 @@ MEASURED_TRAFFIC = {
     # decode scans at 16 x 131,072 (read + write per launch over 16 x 130,944 scanned tokens), scaled
     # by the scanned tokens of the timed launch
     "dec_scan": {"file": "block_sparse_attention_idx_b200/csrc/msa_decode.cu",
-                 "sha256": "b71c0fcd226bf0b5ef37e38a6d58ee51d338711554b68412e0b9adf3ccb48cb6",
-                 "bytes_per_unit": (268231280 + 501760) / (16 * 130944), "unit": "scanned token",
+                 "sha256": "f603b9d207e2f59c5d3e090b6bded69c342452ba2fb824cc0959092b10450bfd",
+                 "bytes_per_unit": (268227744 + 606608) / (16 * 130944), "unit": "scanned token",
                  "capture": "profiles/decode_16x256k.md"},
     "dec_scan_e4m3": {"file": "block_sparse_attention_idx_b200/csrc/msa_decode.cu",
-                      "sha256": "b71c0fcd226bf0b5ef37e38a6d58ee51d338711554b68412e0b9adf3ccb48cb6",
-                      "bytes_per_unit": (142530048 + 289280) / (16 * 130944), "unit": "scanned token",
+                      "sha256": "f603b9d207e2f59c5d3e090b6bded69c342452ba2fb824cc0959092b10450bfd",
+                      "bytes_per_unit": (142531008 + 148864) / (16 * 130944), "unit": "scanned token",
                       "capture": "profiles/decode_16x256k.md"},
 }
 
