@@ -60,7 +60,8 @@ def test_quantize_three_dim_cache_layout():
 
 
 DECODE_SHAPES = [(3, 1000, 64, 4, 128, 64, 128, 16), (2, 700, 4, 2, 64, 32, 32, 4), (2, 901, 16, 2, 64, 64, 64, 8),
-                 (1, 300, 8, 8, 128, 32, 128, 1), (2, 1001, 8, 2, 64, 64, 128, 4)]
+                 (1, 300, 8, 8, 128, 32, 128, 1), (2, 1001, 8, 2, 64, 64, 128, 4), (2, 702, 8, 2, 64, 64, 32, 6),
+                 (2, 900, 8, 4, 64, 64, 64, 5)]
 
 
 def decode_case(shape, seed):
