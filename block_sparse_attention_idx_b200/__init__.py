@@ -109,6 +109,8 @@ def lib() -> ctypes.CDLL:
         L.msa_debug_set_wait_ns.restype = None
         L.msa_debug_wait_probe.argtypes = [P, S, P]
         L.msa_debug_wait_probe.restype = ctypes.c_int
+        L.msa_debug_exp2_fma.argtypes = [P, P, ctypes.c_int64, P]
+        L.msa_debug_exp2_fma.restype = ctypes.c_int
         L.msa_profile_enable.argtypes = [ctypes.c_int]
         L.msa_profile_enable.restype = None
         L.msa_profile_read.argtypes = [ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
@@ -467,6 +469,15 @@ def msa_debug_set_wait_ns(ns: int) -> None:
     lib().msa_debug_set_wait_ns(int(ns))
 
 
+def msa_debug_exp2_fma(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """2^x by the library's FMA-pipe exponential (fp32 device tensor in, same shape out)."""
+    if not (x.is_cuda and x.dtype == torch.float32 and x.is_contiguous()):
+        raise ValueError("msa_debug_exp2_fma: x must be a contiguous float32 CUDA tensor")
+    y = torch.empty_like(x)
+    _check("msa_debug_exp2_fma", lib().msa_debug_exp2_fma(_p(x), _p(y), x.numel(), _stream(stream, x.device)))
+    return y
+
+
 def msa_debug_wait_probe(ws: torch.Tensor, stream=None) -> None:
     """Test hook: enqueue the launch whose bounded wait can only run out (status MSA_ERR_TIMEOUT).
     ws: a uint8 CUDA tensor of at least 256 + 4096 bytes."""
@@ -480,5 +491,5 @@ __all__ = ["MsaDims", "MsaError", "msa_workspace_size", "msa_index_topk", "msa_s
            "msa_quantize_e4m3_rows", "msa_kl_fwd_grad", "msa_sparse_attn_bwd", "msa_index_topk_local",
            "msa_topk_merge", "msa_lse_idx_local", "msa_lse_combine", "msa_get_device_status", "msa_status_string",
            "msa_version", "msa_profile_enable", "msa_profile_read", "msa_decode_noalloc_status",
-           "msa_debug_set_wait_ns", "msa_debug_wait_probe", "msa_kl_dense_fwd_grad", "workspace", "lib",
+           "msa_debug_set_wait_ns", "msa_debug_wait_probe", "msa_debug_exp2_fma", "msa_kl_dense_fwd_grad", "workspace", "lib",
            "LIB_PATH"]

@@ -581,6 +581,11 @@ msa_status msa_debug_wait_probe(void* ws, size_t ws_bytes, msa_stream_t stream_)
     return cuda_status(e);
 }
 
+msa_status msa_debug_exp2_fma(const float* x, float* y, int64_t n, msa_stream_t stream_) {
+    if (n < 0 || (n > 0 && (!x || !y))) return MSA_ERR_INVALID_ARG;
+    return cuda_status(run_exp2_fma(x, y, n, num_sms(), reinterpret_cast<cudaStream_t>(stream_)));
+}
+
 msa_status msa_get_device_status(const void* ws, msa_stream_t stream_) {
     if (!ws) return MSA_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_);

@@ -451,6 +451,33 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
     return r;
 }
 
+// 2^x on the FMA pipe (no MUFU op), two values at once, for x <= 1/2. Cody-Waite reduction: adding
+// 1.5 * 2^23 rounds x to the nearest integer j and leaves j in the low mantissa bits of the sum;
+// f = x - j lies in [-1/2, 1/2] and is exact. 2^f is a degree-5 polynomial, minimax in relative
+// error on [-1/2, 1/2] (Remez exchange, coefficients from gen_exp2_poly.py: 2.4e-7 relative when
+// evaluated in fp32 by Horner's rule), and j is added to its exponent field. x is first raised to
+// -125, so that -inf and anything below give 2^-125 (negligible next to a sum that holds a 1)
+// instead of 0. A kernel bound by the MUFU pipe moves part of its exponentials here.
+__device__ __forceinline__ uint64_t exp2_fma_x2(uint64_t x2) {
+    constexpr uint32_t kC[6] = {0x3f800001u, 0x3f317214u, 0x3e75fc8cu, 0x3d635b72u, 0x3c1e8629u, 0x3aae0473u};
+    float a, b;
+    f2_unpack(x2, a, b);
+    const uint64_t x = f2_packf(fmaxf(a, -125.f), fmaxf(b, -125.f));
+    const uint64_t t = f2_add(x, f2_packf(12582912.f, 12582912.f));
+    const uint64_t j = f2_add(t, f2_packf(-12582912.f, -12582912.f));
+    const uint64_t f = f2_fma(j, f2_packf(-1.f, -1.f), x);
+    auto cc = [&](int i) { return f2_packf(__uint_as_float(kC[i]), __uint_as_float(kC[i])); };
+    uint64_t p = f2_fma(f, cc(5), cc(4));
+    p = f2_fma(p, f, cc(3));
+    p = f2_fma(p, f, cc(2));
+    p = f2_fma(p, f, cc(1));
+    p = f2_fma(p, f, cc(0));
+    float t0, t1, p0, p1;
+    f2_unpack(t, t0, t1);
+    f2_unpack(p, p0, p1);
+    return f2_pack(__float_as_uint(p0) + (__float_as_uint(t0) << 23), __float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -6,6 +6,8 @@
 // context stays usable. The probe below exercises that path on purpose without any fault: a
 // consumer waits on an mbarrier whose producer skips its arrival, while a real bulk copy is in
 // flight and TMEM is held. Nothing here traps, asserts or touches memory outside its buffers.
+#include <algorithm>
+
 #include "msa_common.cuh"
 #include "msa_internal.h"
 
@@ -62,6 +64,28 @@ cudaError_t run_set_wait(DevStatus* st, unsigned long long ns, cudaStream_t s) {
 }
 
 size_t wait_probe_bytes() { return kProbeBytes; }
+
+namespace {
+// y[i] = 2^x[i] by the FMA-pipe exponential the MUFU-bound loops use (pairs; a lone last value is
+// paired with 0).
+__global__ void k_exp2_fma(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+    for (int64_t i = 2 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x); i < n; i += 2 * (int64_t)gridDim.x * blockDim.x) {
+        const bool two = i + 1 < n;
+        float lo, hi;
+        f2_unpack(exp2_fma_x2(f2_packf(x[i], two ? x[i + 1] : 0.f)), lo, hi);
+        y[i] = lo;
+        if (two) y[i + 1] = hi;
+    }
+}
+}  // namespace
+
+cudaError_t run_exp2_fma(const float* x, float* y, int64_t n, int num_sms, cudaStream_t s) {
+    if (n <= 0) return cudaSuccess;
+    const int64_t threads = (n + 1) / 2;
+    const int grid = (int)std::min<int64_t>((threads + 255) / 256, (int64_t)num_sms * 8);
+    k_exp2_fma<<<grid, 256, 0, s>>>(x, y, n);
+    return cudaGetLastError();
+}
 
 cudaError_t run_wait_probe(const void* src, DevStatus* st, cudaStream_t s) {
     k_wait_probe<<<1, 96, 0, s>>>(static_cast<const uint8_t*>(src), st);

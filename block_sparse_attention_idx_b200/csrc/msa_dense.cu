@@ -66,6 +66,9 @@ __device__ __forceinline__ DenseTile dense_tile(const DenseLseArgs& a, int t) {
     return d;
 }
 
+// Column pairs of every 8 whose exponentials the teacher-LSE loop computes on the FMA pipe.
+constexpr int kPolyOf8 = 2;
+
 template <int D, int BK>
 __global__ void __launch_bounds__(kThreads, 1)
     k_dense_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -237,11 +240,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float mref = mn == -INFINITY ? 0.f : mn;
                 const uint64_t sl2x2 = f2_packf(sl2, sl2), moffx2 = f2_packf(-mref * sl2, -mref * sl2);
                 uint64_t acc[2] = {f2_packf(0.f, 0.f), f2_packf(0.f, 0.f)};
+                // the MUFU pipe bounds this loop: kPolyOf8 of every 8 column pairs take their
+                // exponentials on the FMA pipe instead
 #pragma unroll
                 for (int y = 0; y < BK; y += 2) {
-                    float x0, x1;
-                    f2_unpack(f2_fma(f2_pack(sv[y], sv[y + 1]), sl2x2, moffx2), x0, x1);
-                    acc[(y >> 1) & 1] = f2_add(acc[(y >> 1) & 1], f2_packf(fast_exp2(x0), fast_exp2(x1)));
+                    const uint64_t xx = f2_fma(f2_pack(sv[y], sv[y + 1]), sl2x2, moffx2);
+                    uint64_t ex;
+                    if (((y >> 1) & 7) < kPolyOf8) {
+                        ex = exp2_fma_x2(xx);
+                    } else {
+                        float x0, x1;
+                        f2_unpack(xx, x0, x1);
+                        ex = f2_packf(fast_exp2(x0), fast_exp2(x1));
+                    }
+                    acc[(y >> 1) & 1] = f2_add(acc[(y >> 1) & 1], ex);
                 }
                 float a0, a1, a2, a3;
                 f2_unpack(acc[0], a0, a1);

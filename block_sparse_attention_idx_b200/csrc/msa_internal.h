@@ -202,5 +202,7 @@ cudaError_t run_dense_lists(const Csr& cs, int B, int N, int H_kv, int block_k, 
 cudaError_t run_set_wait(DevStatus* st, unsigned long long ns, cudaStream_t s);
 size_t wait_probe_bytes();
 cudaError_t run_wait_probe(const void* src, DevStatus* st, cudaStream_t s);
+// y[i] = 2^x[i] through exp2_fma_x2 (the FMA-pipe exponential), for its accuracy test.
+cudaError_t run_exp2_fma(const float* x, float* y, int64_t n, int num_sms, cudaStream_t s);
 
 }  // namespace msa

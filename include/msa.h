@@ -370,6 +370,16 @@ MSA_API void msa_debug_set_wait_ns(unsigned long long ns);
 MSA_API msa_status msa_debug_wait_probe(void *ws, size_t ws_bytes, msa_stream_t stream);
 
 /*
+ * Test hook of the FMA-pipe exponential (no counterpart in the pages). The teacher-LSE loop of the
+ * dense warm-up is bound by the MUFU pipe, so it computes part of its exponentials as 2^x = 2^j 2^f
+ * (Cody-Waite reduction to f in [-1/2, 1/2], a degree-5 minimax polynomial for 2^f) on the FMA pipe.
+ * msa_debug_exp2_fma: y[i] = that 2^x[i] for i < n (device pointers to n fp32 values, enqueued on
+ *   `stream`). Relative error <= 3e-7 for -125 <= x <= 1/2; x below -125 (and -inf) gives 2^-125.
+ *   MSA_ERR_INVALID_ARG for n < 0 or a null pointer with n > 0.
+ */
+MSA_API msa_status msa_debug_exp2_fma(const float *x, float *y, int64_t n, msa_stream_t stream);
+
+/*
  * Kernel timing (off by default). While enabled, every entry point records a pair of CUDA events
  * on its stream around each kernel it launches. msa_profile_read synchronises on those events,
  * adds their durations per kernel name and clears the record: on return names[x] / total_ms[x] /
